@@ -1,0 +1,138 @@
+"""The pins catch plausible oracle mistakes: each case plants one in the oracle (CPU only)
+and checks that at least one pin then fails."""
+
+import numpy as np
+import pytest
+
+import oracle.svdquant as sq
+import oracle.nvfp4 as nv
+import oracle.prepared as pp
+from tests import test_oracle_svdquant as T1
+from tests import test_oracle_codes as T2
+
+
+def _golden_loader():
+    import json, os
+    root = os.path.join(os.path.dirname(__file__), "golden")
+    return lambda n: json.load(open(os.path.join(root, n)))
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except (AssertionError, ValueError):
+        return True
+    return False
+
+
+def _int_quantize_half_away(z, bits):
+    z64 = np.array(z, dtype=np.float64)
+    qm = sq.qmax_of(bits)
+    s = float(np.max(np.abs(z64))) / qm if z64.size else 0.0
+    if s == 0.0:
+        return np.zeros(z64.shape, np.int64), 0.0
+    t = z64 / s
+    return np.clip(np.sign(t) * np.floor(np.abs(t) + 0.5), -qm, qm).astype(np.int64), s
+
+
+def _int_quantize_wrong_qmax(z, bits):
+    z64 = np.array(z, dtype=np.float64)
+    qm = 2 ** (bits - 1)
+    s = float(np.max(np.abs(z64))) / qm
+    if s == 0.0:
+        return np.zeros(z64.shape, np.int64), 0.0
+    return np.clip(np.rint(z64 / s), -qm, qm).astype(np.int64), s
+
+
+def _smooth_multiply(x, w, s):
+    x64, w64, s64 = (np.array(a, dtype=np.float64) for a in (x, w, s))
+    return x64 * s64[None, :], w64 / s64[:, None]
+
+
+def _split_drop_sigma(weight, rank):
+    sq.check_rank(weight, rank)
+    w = np.array(weight, dtype=np.float64)
+    if rank == 0:
+        return np.zeros((w.shape[0], 0)), np.zeros((0, w.shape[1])), w.copy()
+    U, S, Vt = np.linalg.svd(w, full_matrices=False)
+    L, R = U[:, :rank], Vt[:rank]
+    return L, R, w - L @ R
+
+
+def _split_wrong_end(weight, rank):
+    sq.check_rank(weight, rank)
+    w = np.array(weight, dtype=np.float64)
+    if rank == 0:
+        return np.zeros((w.shape[0], 0)), np.zeros((0, w.shape[1])), w.copy()
+    U, S, Vt = np.linalg.svd(w, full_matrices=False)
+    L, R = U[:, -rank:] * S[-rank:], Vt[-rank:]
+    return L, R, w - L @ R
+
+
+def _linear_quantize_full_weight(x, weight, scale, rank, bits=4):
+    sq.check_smoothing(x, weight, scale)
+    xs, ws = sq.smooth_inputs(x, weight, scale)
+    L1, L2, R = sq.split_weight(ws, rank)
+    return (xs @ L1) @ L2 + sq.fake_quantize(xs, bits) @ sq.fake_quantize(ws, bits) - \
+        (xs @ L1) @ L2 * 0
+
+
+def _linear_quantized_low_rank(x, weight, scale, rank, bits=4):
+    sq.check_smoothing(x, weight, scale)
+    xs, ws = sq.smooth_inputs(x, weight, scale)
+    L1, L2, R = sq.split_weight(ws, rank)
+    qx = sq.fake_quantize(xs, bits)
+    return (qx @ L1) @ L2 + qx @ sq.fake_quantize(R, bits)
+
+
+def _e2m1_ties_away(v):
+    v = np.asarray(v, dtype=np.float64)
+    grid = nv._E2M1_GRID
+    a = np.abs(v)
+    idx = np.argmin(np.abs(a[..., None] - grid) - 1e-12 * np.arange(8), axis=-1)
+    idx = np.where(a >= 6, 7, idx).astype(np.uint8)
+    return (((v < 0) & (idx != 0)).astype(np.uint8) << 3) | idx
+
+
+def _pack_swapped(codes):
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[:, 1::2] & 0xF) | ((c[:, 0::2] & 0xF) << 4)
+
+
+def _sf_offset_transposed(r, c, rows, kblocks):
+    _, kbp = nv.sf_padded_shape(rows, kblocks)
+    r = np.asarray(r, dtype=np.int64); c = np.asarray(c, dtype=np.int64)
+    atom = (r // 128) * (kbp // 4) + (c // 4)
+    return atom * 512 + (r % 32) * 4 + ((r % 128) // 32) * 16 + (c % 4)
+
+
+def _int_product_transposed(a, w):
+    a = np.asarray(a, dtype=np.float64); w = np.asarray(w, dtype=np.float64)
+    return a @ w[::-1].T
+
+
+MUTATIONS = [
+    (sq, "int_quantize", _int_quantize_half_away, [T1.test_fake_quantize_hand_cases]),
+    (sq, "int_quantize", _int_quantize_wrong_qmax, [T1.test_fake_quantize_hand_cases]),
+    (sq, "smooth_inputs", _smooth_multiply, [T1.test_svdquant_linear_hand_case]),
+    (sq, "split_weight", _split_drop_sigma, [T1.test_split_weight_hand_case]),
+    (sq, "split_weight", _split_wrong_end, [T1.test_split_weight_hand_case]),
+    (sq, "svdquant_linear", _linear_quantize_full_weight, [T1.test_svdquant_linear_hand_case]),
+    (sq, "svdquant_linear", _linear_quantized_low_rank, [T1.test_svdquant_linear_hand_case]),
+    (nv, "e2m1_encode", _e2m1_ties_away, [T2.test_e2m1_rounding_ties]),
+    (nv, "pack_nibbles", _pack_swapped, [T2.test_pack_nibbles_order]),
+    (nv, "sf_offset", _sf_offset_transposed, [T2.test_sf_layout_points_and_bijection]),
+    (pp, "int_product", _int_product_transposed, [T1.test_integer_product_matches_brute_force]),
+]
+
+
+@pytest.mark.parametrize("mod,name,bad,pins", MUTATIONS,
+                         ids=[f"{m[1]}:{m[2].__name__}" for m in MUTATIONS])
+def test_planted_mistake_is_caught(monkeypatch, mod, name, bad, pins):
+    golden = _golden_loader()
+    monkeypatch.setattr(mod, name, bad)
+    caught = False
+    for pin in pins:
+        nargs = pin.__code__.co_argcount
+        caught |= _fails(pin, golden) if nargs == 1 else _fails(pin)
+    assert caught, f"no pin caught the planted mistake in {name}"
