@@ -1,0 +1,222 @@
+/*
+ * svdq.h - C ABI of the SVDQuant inference linear for NVIDIA B200 (sm_100a).
+ *
+ * The operator is the two-branch linear of "SVDQuant Smoothing, Low-rank and
+ * Residual Quantization" ("Formula and conventions", items 1-3):
+ *
+ *     Y[B,N] = (X_hat L1) L2 + Q(X_hat) Q(R),   X_hat = x / scale,
+ *
+ * with x[B,M] @ W[M,N] in that (not the nn.Linear) layout, L1[M,r] L2[r,N] the
+ * best rank-r approximation of the smoothed weight scale[:,None] * W, and R the
+ * residual. Q is either the per-tensor symmetric INT grid of that page
+ * (s = max|z| / (2^(bits-1) - 1), round half to even, 2 <= bits <= 8) or the
+ * NVFP4 format whose storage the "flashinfer.gemm.svdquant_linear" page lists
+ * (packed e2m1 residual, ue4m3 block scales in the 128x4 layout, fp32 global
+ * scales).
+ *
+ * Conventions shared by every call
+ *   - Device pointers are caller-allocated; the library allocates no device
+ *     memory. Scratch space is passed in as `workspace` (size from the matching
+ *     *_workspace_size query) and must not be shared by calls in flight.
+ *   - Every call is stream-ordered on `stream` and returns without a device
+ *     synchronisation, except svdq_prepare and svdq_check_status (documented).
+ *   - Inputs are never written. Matrices are row-major with a leading
+ *     dimension (in elements) >= the row length.
+ *   - Errors found on the host return a status and launch nothing. Errors found
+ *     on the device (a non-positive scale in svdq_prepare, a wait that ran out)
+ *     are recorded in a device status word read by svdq_check_status.
+ *   - Shape limits: M a positive multiple of 32; N a positive multiple of 16;
+ *     B >= 0 (B = 0 launches nothing); rank <= 256 (the down/up factors are
+ *     zero-padded to rank_pad = rank rounded up to 16, which changes nothing).
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* svdq_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_EINVAL = 1,        /* bad layout or scale ("_check_smoothing" raises ValueError) */
+  SVDQ_ERANK = 2,         /* rank outside [0, min(M,N)] ("_check_rank" raises ValueError) */
+  SVDQ_EUNSUPPORTED = 3,  /* valid per the pages, outside this library's limits */
+  SVDQ_ECUDA = 4,         /* a CUDA runtime/driver call failed */
+  SVDQ_ETIMEOUT = 5,      /* a bounded device wait ran out (kernel returned early) */
+  SVDQ_EWORKSPACE = 6     /* workspace missing or too small */
+} svdq_status;
+
+typedef enum svdq_dtype { SVDQ_F32 = 0, SVDQ_BF16 = 1 } svdq_dtype;
+
+typedef enum svdq_kind {
+  SVDQ_KIND_INT = 0,   /* per-tensor symmetric INT grid, bits in [2, 8] */
+  SVDQ_KIND_NVFP4 = 1  /* e2m1 codes, ue4m3 scale per 16 elements, fp32 global scale; bits = 4 */
+} svdq_kind;
+
+typedef struct svdq_fmt {
+  int32_t kind;  /* svdq_kind */
+  int32_t bits;
+} svdq_fmt;
+
+/*
+ * A prepared weight. The caller allocates every buffer (sizes from
+ * svdq_weight_buffer_sizes), fills the pointers, and svdq_prepare fills them.
+ * Layouts (all row-major, K = M is the reduction dim):
+ *   codes   INT:   int8  [N, M]      residual codes, K-major (row n holds column n of R)
+ *           NVFP4: uint8 [N, M/2]    e2m1 nibbles, element 2j in the low nibble of byte j
+ *   sf      NVFP4: uint8, 128x4 layout of the [N, M/16] ue4m3 block scales
+ *           (rows padded to 128, scale columns to 4); unused (may be NULL) for INT
+ *   w_scale fp32 device scalar: INT s_w = max|R| / qmax; NVFP4 global scale gs_w
+ *   ld      bf16  [rank_pad, M]      down factor transposed, smoothing folded in:
+ *           ld[j, m] = L1[m, j] / scale[m]  (the page's X_hat L1 = x ld^T)
+ *   ld32    fp32  [rank_pad, M]      same values as ld, for fp32 activations (may be NULL
+ *           if only bf16 activations are used)
+ *   lu      bf16  [N, 2*rank_pad]    up factor L2^T written twice along the row:
+ *           lu[n, j] = lu[n, rank_pad + j] = L2[j, n]
+ *   scale   fp32  [M]                the smoothing scale (referenced, not copied)
+ */
+typedef struct svdq_weight {
+  int64_t M, N;
+  int32_t rank, rank_pad;
+  svdq_fmt fmt;
+  void* codes;
+  void* sf;
+  float* w_scale;
+  void* ld;
+  void* ld32;
+  void* lu;
+  const float* scale;
+} svdq_weight;
+
+/* Byte sizes of the svdq_weight buffers, in order: codes, sf, w_scale, ld, ld32, lu. */
+svdq_status svdq_weight_buffer_sizes(int64_t M, int64_t N, int32_t rank, svdq_fmt fmt,
+                                     size_t sizes[6]);
+
+/* Scratch bytes svdq_prepare needs for this shape (randomized SVD with the given
+ * oversampling; <= 0 selects the default of 16). */
+svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq_fmt fmt,
+                                        int32_t oversample, size_t* bytes);
+
+/*
+ * svdq_prepare - one-time weight split ("split_weight" and "Formula and
+ * conventions" items 1-2; offline transforms of "flashinfer.gemm.svdquant_linear").
+ *
+ *   W      device, [M, N] (ldW >= N), bf16 or fp32
+ *   scale  device fp32 [M], must be finite and > 0 (checked on the device)
+ *   rank   0 <= rank <= min(M, N) (Python-int semantics are the binding's job)
+ *   seed   seeds the Gaussian test matrix of the randomized subspace iteration
+ *   oversample, power_iters  <= 0 select the defaults 16 and 2
+ *   out    caller-allocated buffers (see svdq_weight); M, N, rank, rank_pad,
+ *          fmt and scale are filled in by this call
+ *
+ * Computes ws = scale[:,None] * W, a rank-r truncated SVD of ws by randomized
+ * subspace iteration (Gaussian test matrix, power iterations with Householder
+ * re-orthonormalisation, one-sided Jacobi SVD of the small core), stores the
+ * factors in bf16 with 1/scale folded into ld, forms the residual
+ * R = ws - diag(scale) ld^T lu^T in fp32 against the stored (rounded) factors,
+ * and quantises R per tensor (INT) or per 16-element block (NVFP4).
+ *
+ * Synchronises `stream` before returning and returns SVDQ_EINVAL if scale held
+ * a non-positive or non-finite entry, SVDQ_ETIMEOUT if a device wait ran out.
+ */
+svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N, int64_t ldW,
+                         const float* scale, int32_t rank, svdq_fmt fmt, uint64_t seed,
+                         int32_t oversample, int32_t power_iters,
+                         void* workspace, size_t workspace_bytes, svdq_weight* out,
+                         svdq_stream_t stream);
+
+/*
+ * svdq_quantize_residual - the residual quantiser of svdq_prepare on its own
+ * ("fake_quantize" grid for INT; NVFP4 block scales for NVFP4).
+ *
+ *   R        device fp32 [M, N] (ldR >= N)
+ *   codes    INT int8 [N, M] / NVFP4 uint8 [N, M/2]   (K-major, as in svdq_weight)
+ *   sf       NVFP4 128x4 layout of [N, M/16] (NULL for INT)
+ *   w_scale  device fp32 scalar out: s_w (INT) or gs_w (NVFP4)
+ */
+svdq_status svdq_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
+                                   svdq_fmt fmt, void* codes, void* sf, float* w_scale,
+                                   void* workspace, size_t workspace_bytes,
+                                   svdq_stream_t stream);
+
+svdq_status svdq_quantize_residual_workspace_size(int64_t M, int64_t N, svdq_fmt fmt,
+                                                  size_t* bytes);
+
+/*
+ * svdq_quantize_act - one fused pass over the activation ("smooth_inputs" for
+ * X_hat = x / scale, the "fake_quantize" grid; step 1 and the down-projection
+ * GEMM of step 2 of "flashinfer.gemm.svdquant_linear").
+ *
+ *   x        device [B, M] (ldx >= M), bf16 or fp32
+ *   scale    device fp32 [M] (precondition: finite and > 0; not re-checked)
+ *   act_global_scale  NVFP4 only, nullable: a given gs_x; NULL computes
+ *            gs_x = 448*6 / max|X_hat| from the data. Ignored for INT.
+ *   ld       nullable: bf16 [rank_pad, M] (or fp32 for fp32 x) down factor;
+ *            NULL (or rank_pad = 0) skips the down-projection
+ *   codes    out INT int8 [B, M] / NVFP4 uint8 [B, M/2]
+ *   sf       out NVFP4 128x4 layout of [B, M/16]; NULL for INT
+ *   act_scale out device fp32 scalar: s_x (INT) or the gs_x used (NVFP4)
+ *   down     out bf16 [B, 2*rank_pad]: x ld^T split as hi | lo with
+ *            hi = bf16(v), lo = bf16(v - hi) of the fp32 dot product v
+ */
+svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
+                              int64_t ldx, const float* scale, svdq_fmt fmt,
+                              const float* act_global_scale, const void* ld, int32_t rank_pad,
+                              void* codes, void* sf, float* act_scale, void* down,
+                              void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
+svdq_status svdq_quantize_act_workspace_size(int64_t B, int64_t M, svdq_fmt fmt,
+                                             int32_t rank_pad, size_t* bytes);
+
+/*
+ * svdq_linear - the operator ("svdquant_linear" of both pages):
+ *   Y = x ld^T lu^T + alpha * (Q(X_hat) . Q(R)) [+ bias]
+ * with alpha = s_x * s_w (INT) or 1 / (gs_x * gs_w) (NVFP4). Runs the fused
+ * activation pass, then one tensor-core GEMM whose epilogue adds the low-rank
+ * up-projection and the bias.
+ *
+ *   w        prepared weight (svdq_prepare)
+ *   x        device [B, M] (ldx >= M), bf16 or fp32 (fp32 needs w->ld32)
+ *   bias     nullable device bf16 [N]
+ *   act_global_scale  NVFP4 only, nullable (see svdq_quantize_act)
+ *   y        device [B, N] (ldy >= N), bf16 or fp32
+ */
+svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype, int64_t B,
+                        int64_t ldx, const void* bias, const float* act_global_scale,
+                        void* y, svdq_dtype y_dtype, int64_t ldy,
+                        void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
+svdq_status svdq_linear_workspace_size(const svdq_weight* w, int64_t B, size_t* bytes);
+
+/*
+ * svdq_residual_product_i32 - the INT residual GEMM alone, exact int32:
+ *   acc[b, n] = sum_k act_codes[b, k] * w->codes[n, k]
+ * (the integer product inside Q(X_hat) Q(R)); acc is int32 [B, N] (ldacc >= N).
+ */
+svdq_status svdq_residual_product_i32(const svdq_weight* w, const int8_t* act_codes, int64_t B,
+                                      int32_t* acc, int64_t ldacc, svdq_stream_t stream);
+
+/* Synchronises `stream`, returns and clears the device status word
+ * (SVDQ_OK, SVDQ_EINVAL or SVDQ_ETIMEOUT), or SVDQ_ECUDA on a runtime error. */
+svdq_status svdq_check_status(svdq_stream_t stream);
+
+/* Failure-path self test: runs a bounded device wait on a flag that nothing sets,
+ * with a limit of `limit_us` microseconds, on a single block. Returns what
+ * svdq_check_status then reports (SVDQ_ETIMEOUT when the wait ran out). */
+svdq_status svdq_selftest_wait_timeout(int64_t limit_us, svdq_stream_t stream);
+
+const char* svdq_status_string(svdq_status s);
+
+/* Library version, e.g. "0.1.0". */
+const char* svdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */

@@ -1,0 +1,88 @@
+// internal.h - declarations shared by the library's translation units (not part
+// of the public C ABI in include/svdq.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "svdq.h"
+
+namespace svdq {
+
+// Device address of the library's status word (resolved once per device).
+unsigned* device_status_word();
+
+// Encode a 2-D tiled tensor map with 128-byte swizzle (or none). Returns false
+// if the driver rejects the arguments.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  int elem_bytes, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                  uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+inline int32_t rank_pad_of(int32_t rank) { return static_cast<int32_t>(round_up(rank, 16)); }
+
+int num_sms();
+
+// Bump-pointer carving of a caller workspace (256-byte aligned pieces).
+struct Carver {
+  char* base;
+  size_t cap;
+  size_t off = 0;
+  bool ok = true;
+  Carver(void* b, size_t c) : base(static_cast<char*>(b)), cap(c) {}
+  void* take(size_t bytes) {
+    off = static_cast<size_t>(round_up(static_cast<int64_t>(off), 256));
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    if (off > cap || base == nullptr) ok = false;
+    return p;
+  }
+};
+
+// ---------------------------------------------------------------- act pass
+struct ActPlan {
+  int64_t B, M;
+  int32_t rank_pad;
+  int tile_k;      // elements per 128-byte K tile (64 bf16 / 32 fp32)
+  int nrb;         // row blocks of 128
+  int nsteps;      // K tiles
+  int ksplit;      // CTAs along K
+  int nparts;      // partial maxima written (nrb * ksplit)
+};
+ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt);
+size_t act_scratch_bytes(const ActPlan& p);
+
+cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
+                       const float* scale, svdq_fmt fmt, const float* act_global_scale,
+                       const void* ld, void* codes, void* sf, float* act_scale, void* down,
+                       void* scratch, cudaStream_t stream, bool* bad_args);
+
+// ------------------------------------------------------------ residual GEMM
+cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
+                            const void* down2, int64_t B, const void* bias, void* y,
+                            svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                            bool* bad_args);
+
+cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
+                              const uint8_t* act_sf, const float* gs_x, const void* down2,
+                              int64_t B, const void* bias, void* y, svdq_dtype ydt,
+                              int64_t ldy, cudaStream_t stream, bool* bad_args);
+
+// -------------------------------------------------------------- quantisers
+size_t residual_scratch_bytes(int64_t M, int64_t N);
+cudaError_t launch_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
+                                     svdq_fmt fmt, void* codes, void* sf, float* w_scale,
+                                     void* scratch, cudaStream_t stream);
+
+// ------------------------------------------------------------------ prepare
+size_t prepare_scratch_bytes(int64_t M, int64_t N, int32_t rank, int32_t oversample);
+svdq_status run_prepare(const void* W, svdq_dtype wdt, int64_t M, int64_t N, int64_t ldW,
+                        const float* scale, int32_t rank, svdq_fmt fmt, uint64_t seed,
+                        int32_t oversample, int32_t power_iters, void* workspace,
+                        size_t ws_bytes, svdq_weight* out, cudaStream_t stream);
+
+
+}  // namespace svdq

@@ -1,0 +1,195 @@
+// quant.cu - quantisation of the residual weight R[M, N] (fp32).
+//
+// INT: the per-tensor grid of "SVDQuant Smoothing, Low-rank and Residual
+// Quantization" (Formula item 3): s_w = max|R| / qmax and
+// codes = clamp(round_half_even(R / s_w), -qmax, qmax), in fp32 with IEEE
+// division, written K-major as codes[N, M] (row n = column n of R).
+// NVFP4: 16-element blocks along M of each column of R, ue4m3 block scales in
+// the 128x4 layout and an fp32 global scale (the weight_fp4 / weight_sf /
+// alpha storage of "flashinfer.gemm.svdquant_linear"), same recipe as the
+// activation pass: gs = 448*6 / max|R|, sf = ue4m3(fl(amax_b / 6) * gs),
+// code = e2m1(R * fl(gs / sf)).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kMaxParts = 1024;
+
+__global__ void __launch_bounds__(256) absmax_partial_kernel(const float* __restrict__ R, int64_t M,
+                                                             int64_t N, int64_t ldR,
+                                                             float* __restrict__ parts) {
+  float m = 0.0f;
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / N, c = i - r * N;
+    m = fmaxf(m, fabsf(R[r * ldR + c]));
+  }
+  __shared__ float red[8];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int w = 1; w < 8; ++w) t = fmaxf(t, red[w]);
+    parts[blockIdx.x] = t;
+  }
+}
+
+__device__ float reduce_parts(const float* __restrict__ parts, int nparts) {
+  __shared__ float red[8];
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = fmaxf(m, parts[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) t = fmaxf(t, red[w]);
+    red[0] = t;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// 32 x 32 tiles: read R coalesced along N, write codes coalesced along M.
+__global__ void __launch_bounds__(256) quant_int_transpose_kernel(
+    const float* __restrict__ R, int64_t M, int64_t N, int64_t ldR, int qmax,
+    const float* __restrict__ parts, int nparts, int8_t* __restrict__ codes,
+    float* __restrict__ w_scale) {
+  const float m = reduce_parts(parts, nparts);
+  const float s = __fdiv_rn(m, static_cast<float>(qmax));
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *w_scale = s;
+  __shared__ int8_t tile[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * 32, n0 = static_cast<int64_t>(blockIdx.x) * 32;
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t r = m0 + i, c = n0 + tx;
+    int q = 0;
+    if (r < M && c < N && s > 0.0f) {
+      q = __float2int_rn(__fdiv_rn(R[r * ldR + c], s));
+      q = min(max(q, -qmax), qmax);
+    }
+    tile[i][tx] = static_cast<int8_t>(q);
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t n = n0 + i, mm = m0 + tx;
+    if (n < N && mm < M) codes[n * M + mm] = tile[tx][i];
+  }
+}
+
+__device__ __forceinline__ uint8_t f32_to_ue4m3_q(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return static_cast<uint8_t>(r & 0xFFu);
+}
+
+__device__ __forceinline__ float ue4m3_to_f32_q(uint8_t b) {
+  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+  return e == 0 ? static_cast<float>(m) * 0.001953125f
+                : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+__device__ __forceinline__ uint32_t f32x8_to_e2m1_q(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t mag = out & 0x77777777u;
+  const uint32_t nz = (mag + 0x77777777u) & 0x88888888u;
+  return out & (0x77777777u | nz);
+}
+
+// One thread per (column n, 16-row block kb) of R; consecutive threads take
+// consecutive n so every row read is coalesced.
+__global__ void __launch_bounds__(256) quant_nvfp4_kernel(
+    const float* __restrict__ R, int64_t M, int64_t N, int64_t ldR, const float* __restrict__ parts,
+    int nparts, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+    float* __restrict__ w_scale) {
+  const float m = reduce_parts(parts, nparts);
+  const float gs = m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *w_scale = gs;
+  const int64_t kb = M / 16;
+  const int64_t kbp = (kb + 3) / 4 * 4;
+  const int64_t np = (N + 127) / 128 * 128;
+  const int64_t total = np * kbp;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / np;
+    const int64_t n = i - b * np;
+    const int64_t off = ((n >> 7) * (kbp >> 2) + (b >> 2)) * 512 + (n & 31) * 16 +
+                        ((n & 127) >> 5) * 4 + (b & 3);
+    if (n >= N || b >= kb) {
+      sf[off] = 0;
+      continue;
+    }
+    float v[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      v[j] = R[(b * 16 + j) * ldR + n];
+      amax = fmaxf(amax, fabsf(v[j]));
+    }
+    const uint8_t sfb = f32_to_ue4m3_q(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
+    const float d = ue4m3_to_f32_q(sfb);
+    const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], enc);
+    *reinterpret_cast<uint2*>(codes + n * (M / 2) + b * 8) =
+        make_uint2(f32x8_to_e2m1_q(v), f32x8_to_e2m1_q(v + 8));
+    sf[off] = sfb;
+  }
+}
+
+int parts_for(int64_t M, int64_t N) {
+  return static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(kMaxParts, ceil_div(M * N, 256 * 16))));
+}
+
+}  // namespace
+
+size_t residual_scratch_bytes(int64_t M, int64_t N) {
+  return static_cast<size_t>(parts_for(M, N)) * sizeof(float) + 256;
+}
+
+cudaError_t launch_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
+                                     svdq_fmt fmt, void* codes, void* sf, float* w_scale,
+                                     void* scratch, cudaStream_t stream) {
+  const int nparts = parts_for(M, N);
+  float* parts = static_cast<float*>(scratch);
+  absmax_partial_kernel<<<nparts, 256, 0, stream>>>(R, M, N, ldR, parts);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (fmt.kind == SVDQ_KIND_INT) {
+    const int qmax = (1 << (fmt.bits - 1)) - 1;
+    dim3 grid(static_cast<unsigned>(ceil_div(N, 32)), static_cast<unsigned>(ceil_div(M, 32)));
+    quant_int_transpose_kernel<<<grid, 256, 0, stream>>>(R, M, N, ldR, qmax, parts, nparts,
+                                                          static_cast<int8_t*>(codes), w_scale);
+  } else {
+    const int64_t work = round_up(N, 128) * round_up(M / 16, 4);
+    const int blocks = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(work, 256), static_cast<int64_t>(num_sms()) * 8)));
+    quant_nvfp4_kernel<<<blocks, 256, 0, stream>>>(R, M, N, ldR, parts, nparts,
+                                                    static_cast<uint8_t*>(codes),
+                                                    static_cast<uint8_t*>(sf), w_scale);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

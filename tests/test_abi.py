@@ -1,0 +1,84 @@
+"""The C-ABI library builds, loads and exports every function include/svdq.h declares;
+its host-side argument checks work without a GPU (no kernel is launched here)."""
+
+import ctypes
+
+import pytest
+
+import rank_bit_residual_b200 as rb
+from rank_bit_residual_b200 import build as rbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rbuild.build()
+    return rb.load_library()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = rb.header_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/svdq.h but not exported"
+        assert n in rb._SIGS, f"{n} has no binding signature"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.svdq_version().decode().count(".") == 2
+    for s in range(7):
+        assert len(lib.svdq_status_string(s)) >= 2
+
+
+def _sizes(lib, M, N, r, fmt):
+    sizes = (ctypes.c_size_t * 6)()
+    st = lib.svdq_weight_buffer_sizes(M, N, r, rb.parse_fmt(fmt), sizes)
+    return st, list(sizes)
+
+
+def test_weight_buffer_sizes(lib):
+    st, s = _sizes(lib, 3072, 3072, 32, "int4")
+    assert st == rb.SVDQ_OK
+    assert s == [3072 * 3072, 0, 4, 32 * 3072 * 2, 32 * 3072 * 4, 3072 * 64 * 2]
+    st, s = _sizes(lib, 256, 3216, 20, "nvfp4")
+    assert st == rb.SVDQ_OK
+    assert s[0] == 3216 * 128 and s[1] == 3328 * 16   # rows padded to 128, 16 scale columns
+    assert s[3] == 32 * 256 * 2
+
+
+def test_host_checks_follow_the_page_contract(lib):
+    # "_check_rank": rank in [0, min(M, N)]
+    assert _sizes(lib, 64, 32, 33, "int4")[0] == rb.SVDQ_ERANK
+    assert _sizes(lib, 64, 32, -1, "int4")[0] == rb.SVDQ_ERANK
+    assert _sizes(lib, 64, 32, 32, "int4")[0] == rb.SVDQ_OK
+    assert _sizes(lib, 64, 32, 0, "int4")[0] == rb.SVDQ_OK
+    # "_check_smoothing": nonempty
+    assert _sizes(lib, 0, 32, 0, "int4")[0] == rb.SVDQ_EINVAL
+    # grid: 2 <= bits <= 8
+    assert _sizes(lib, 64, 32, 1, (0, 1))[0] == rb.SVDQ_EINVAL
+    assert _sizes(lib, 64, 32, 1, (0, 9))[0] == rb.SVDQ_EINVAL
+    assert _sizes(lib, 64, 32, 1, (1, 8))[0] == rb.SVDQ_EINVAL
+    # this library's limits
+    assert _sizes(lib, 48, 32, 1, "int4")[0] == rb.SVDQ_EUNSUPPORTED
+    assert _sizes(lib, 64, 40, 1, "int4")[0] == rb.SVDQ_EUNSUPPORTED
+    assert _sizes(lib, 512, 512, 257, "int4")[0] == rb.SVDQ_EUNSUPPORTED
+
+
+def test_workspace_queries(lib):
+    b = ctypes.c_size_t()
+    assert lib.svdq_quantize_act_workspace_size(4096, 3072, rb.parse_fmt("int4"), 32, ctypes.byref(b)) == 0
+    assert b.value > 0
+    assert lib.svdq_quantize_act_workspace_size(4096, 3072, rb.parse_fmt("int4"), 20, ctypes.byref(b)) \
+        == rb.SVDQ_EINVAL
+    assert lib.svdq_quantize_residual_workspace_size(3072, 3072, rb.parse_fmt("nvfp4"), ctypes.byref(b)) == 0
+    assert lib.svdq_prepare_workspace_size(3072, 3072, 32, rb.parse_fmt("int4"), 0, ctypes.byref(b)) == 0
+
+
+def test_python_binding_rejects_non_int_rank():
+    import torch
+    W = torch.zeros(64, 32)
+    s = torch.ones(64)
+    for r in (True, 1.0, "1"):
+        with pytest.raises(ValueError):
+            rb.svdq_prepare(W, s, r)
+    with pytest.raises(ValueError):      # CPU tensors are refused, never computed on the host
+        rb.svdq_prepare(W, s, 1)

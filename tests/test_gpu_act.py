@@ -1,0 +1,76 @@
+"""Activation pass on the GPU against the oracle: INT and NVFP4 codes bit-exact (up to
+flagged near-ties), the per-tensor scale bit-exact, and the fused down-projection."""
+
+import numpy as np
+import pytest
+import torch
+
+import rank_bit_residual_b200 as rb
+from oracle import codes as ocodes
+from oracle import nvfp4 as onv
+from synth import make_case, to_bf16
+from tests.gpu_util import assert_codes_match, device, to_dev, x_tensor, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 32), (17, 96), (128, 256), (300, 1024), (129, 3072)]
+
+
+@pytest.mark.parametrize("B,M", SHAPES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("bits", [4, 8, 2])
+def test_int_codes_and_scale(B, M, dtype, bits):
+    wl = make_case(B, M, 16, rank=0, seed=B + M + bits, dtype=dtype)
+    codes, sf, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), f"int{bits}")
+    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, bits)
+    assert np.float32(s.item()) == s_o, (s.item(), s_o)
+    assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype} int{bits}")
+    assert sf is None and down is None
+
+
+@pytest.mark.parametrize("B,M", SHAPES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("given_gs", [False, True])
+def test_nvfp4_codes_scales_and_layout(B, M, dtype, given_gs):
+    wl = make_case(B, M, 16, rank=0, seed=7 * B + M, dtype=dtype)
+    gs = np.float32(1234.5) if given_gs else None
+    gs_t = to_dev(np.array([gs], np.float32), torch.float32) if given_gs else None
+    codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "nvfp4",
+                                           act_global_scale=gs_t)
+    xs = ocodes.smooth_fp32(wl.x, wl.scale)
+    c_o, sf_o, g_o = onv.quantize(xs, gs=gs)
+    assert np.float32(g.item()) == np.float32(g_o)
+    got_sf = sf.cpu().numpy()
+    want_sf = onv.sf_swizzle(sf_o)
+    assert got_sf.shape == want_sf.shape
+    assert np.array_equal(got_sf, want_sf), f"{int((got_sf != want_sf).sum())} scale bytes differ"
+    got = onv.unpack_nibbles(codes.cpu().numpy())
+    assert np.array_equal(got, c_o), f"{int((got != c_o).sum())} nibbles differ"
+
+
+@pytest.mark.parametrize("B,M,rank", [(1, 64, 1), (17, 96, 16), (200, 512, 40), (129, 3072, 32),
+                                      (64, 256, 256)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_down_projection(B, M, rank, dtype):
+    wl = make_case(B, M, 16, rank=0, seed=3 * B + rank, dtype=dtype)
+    rp = (rank + 15) // 16 * 16
+    rng = np.random.default_rng(rank)
+    ld = np.zeros((rp, M), np.float32)
+    ld[:rank] = to_bf16(rng.standard_normal((rank, M)).astype(np.float32) * 0.1)
+    ld_t = to_dev(ld, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    codes, _, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "int4", ld=ld_t)
+    d = down.float().cpu().numpy().astype(np.float64)
+    got = d[:, :rp] + d[:, rp:]
+    want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
+    # bf16 x: exact products, fp32 sums; fp32 x: tf32 operands (10-bit mantissa)
+    tol = 2e-5 if dtype == "bf16" else 3e-3
+    assert rel_fro(got, want) <= tol, rel_fro(got, want)
+    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+    assert np.float32(s.item()) == s_o
+    assert_codes_match(codes.cpu().numpy(), q, near)
+
+
+def test_empty_batch_is_a_no_op():
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device=device())
+    codes, sf, s, down = rb.svdq_quantize_act(x, torch.ones(64, device=device()), "int4")
+    assert codes.shape == (0, 64)

@@ -1,0 +1,66 @@
+"""Residual GEMM + low-rank epilogue on the GPU against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import rank_bit_residual_b200 as rb
+from synth import make_case
+from tests.gpu_util import SyntheticWeight, assert_y_close, device, to_dev, x_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,M,N", [(1, 32, 16), (130, 160, 48), (257, 384, 272), (128, 1024, 512),
+                                   (300, 3072, 3072)])
+def test_int32_product_is_exact(B, M, N):
+    rng = np.random.default_rng(B + M + N)
+    w = SyntheticWeight(M, N, 0, "int8", seed=B)
+    a = rng.integers(-127, 128, (B, M)).astype(np.int8)
+    acc = rb.svdq_residual_product_i32(w.w, to_dev(a, torch.int8)).cpu().numpy()
+    want = a.astype(np.int64) @ w.codes.astype(np.int64).T
+    assert np.array_equal(acc.astype(np.int64), want), int((acc != want).sum())
+
+
+CASES = [
+    # B, M, N, rank, fmt, bias
+    (16, 256, 128, 16, "int4", False),
+    (1, 64, 16, 1, "int4", False),
+    (37, 96, 48, 0, "int4", True),
+    (130, 512, 272, 40, "int8", True),
+    (256, 1024, 512, 128, "int4", False),
+    (64, 512, 256, 256, "int2", True),
+    (300, 3072, 768, 32, "int4", True),
+]
+
+
+@pytest.mark.parametrize("B,M,N,rank,fmt,bias", CASES)
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_linear_int_matches_oracle(B, M, N, rank, fmt, bias, xdt):
+    wl = make_case(B, M, N, rank=rank, seed=B * 7 + N, dtype=xdt, bias=bias)
+    w = SyntheticWeight(M, N, rank, fmt, seed=N + rank, scale=wl.scale)
+    b = to_dev(wl.bias, torch.bfloat16) if bias else None
+    y32 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.float32)
+    y16 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.bfloat16)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    want = w.oracle_y(wl.x, wl.bias if bias else None)
+    assert_y_close(y32.cpu().numpy(), want, f"{B}x{M}x{N} r={rank} {fmt} {xdt}")
+    # bf16 output is the fp32 result rounded once (same arithmetic, last cast differs)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_linear_strided_output_and_input():
+    wl = make_case(40, 256, 64, rank=8, seed=11)
+    w = SyntheticWeight(256, 64, 8, "int4", seed=2, scale=wl.scale)
+    xbig = torch.zeros((40, 512), dtype=torch.bfloat16, device=device())
+    xbig[:, :256] = x_tensor(wl)
+    out = torch.full((40, 96), 7.0, dtype=torch.float32, device=device())
+    y = rb.svdq_linear(w.w, xbig[:, :256], out=out[:, :64], out_dtype=torch.float32)
+    assert torch.all(out[:, 64:] == 7.0)
+    assert_y_close(y.cpu().numpy(), w.oracle_y(wl.x))
+
+
+def test_linear_rejects_mismatched_input():
+    w = SyntheticWeight(64, 32, 4, "int4", seed=0)
+    with pytest.raises(ValueError):
+        rb.svdq_linear(w.w, torch.zeros((3, 96), dtype=torch.bfloat16, device=device()))
