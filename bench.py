@@ -1,0 +1,411 @@
+"""Benchmark of the SVDQuant inference linear on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the operator's hot path over one batch: the fused
+activation pass (smoothing, per-tensor max, codes, down-projection) and the
+residual tensor-core GEMM with the low-rank + bias epilogue, both through the
+C ABI. The weight split (svdq_prepare) is timed once, separately. Inputs are
+synthetic and seeded (synth/), resident in HBM when the timed region starts;
+L2 is flushed (a 256 MiB write) between timed steps, outside the events.
+
+value     whole-job TOPS (2BMN residual ops + 2Br(M+N) low-rank flops per step)
+e2e       the same metric through svdq_linear with pinned host x copied in and
+          Y copied out inside the timed region
+roofline  the GEMM kernel against the dense int8 tensor peak (measured bf16
+          GEMM peak x 2, the nominal int8:bf16 ratio)
+cpu_baseline / --impl reference   the float64 CPU oracle, timed on host cores
+
+Multi-GPU: replicas only (the operator is single-GPU); each rank runs the same
+workload on its own device, the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "svdq_linear TOPS and GB/s at 1 B200; % of roofline (HBM or int8/FP4 peak)"
+DEFAULT_WORKLOAD = "dit_attn_4096x3072x3072_int4"
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemm_int_dit_attn_4096x3072x3072_int4.md")
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_ops(B, M, N, rank):
+    return 2.0 * B * M * N + 2.0 * B * rank * (M + N)
+
+
+def alg_bytes(B, M, N, rank, fmt, bits, bias):
+    """Algorithmic bytes of one step: bf16 x, weight codes (+scales), bf16 factors,
+    fp32 scale, bias, bf16 Y."""
+    if fmt == "nvfp4":
+        wbytes = M * N * (0.5 + 1.0 / 16.0)
+    else:
+        wbytes = M * N * (0.5 if bits <= 4 else 1.0)
+    return (B * M * 2 + wbytes + 2 * rank * (M + N) + 4 * M + (2 * N if bias else 0)
+            + B * N * 2)
+
+
+def gemm_alg_ops(B, M, N, rank):
+    return 2.0 * B * M * N + 2.0 * B * rank * N
+
+
+def read_profile_traffic(gemm_src):
+    """traffic_bytes_per_launch from the committed ncu summary if it was taken on
+    this very kernel source (sha256 recorded beside it), else None."""
+    import hashlib
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    sha = hashlib.sha256(open(gemm_src, "rb").read()).hexdigest()
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("gemm_source_sha256") != sha:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1])); smax.append(float(parts[2])); power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def cpu_oracle_rate(wl, budget_s=12.0, rows=None):
+    """Time the float64 oracle (prepared-operand linear) on the host cores over a
+    bounded sample; returns (TOPS, seconds, cores, sample description)."""
+    import numpy as np
+    from oracle import codes as ocodes
+    from oracle import prepared as oprep
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    B, M, N, r = wl.B, wl.M, wl.N, wl.rank
+    rows = rows or min(B, 512)
+    ld = (rng.standard_normal((M, r)) * 0.01).astype(np.float64)
+    L2 = (rng.standard_normal((r, N)) * 0.01).astype(np.float64)
+    cw = rng.integers(-7, 8, (N, M)).astype(np.int8)
+    x = wl.x[:rows]
+    t0 = time.perf_counter()
+    ops = 0.0
+    reps = 0
+    while True:
+        q, s_x, _ = ocodes.act_codes_int_fp32(x, wl.scale, wl.bits)
+        oprep.linear_int(x, ld, L2, q, s_x, cw, 0.01)
+        ops += workload_ops(rows, M, N, r)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sample = (f"{reps} pass(es) of the oracle's prepared-operand linear (fp32-mode codes + float64 "
+              f"integer product + low-rank) over {rows} of {B} rows of {wl.name}")
+    return ops / dt / 1e12, dt, cores, sample
+
+
+# ------------------------------------------------------------- reference
+def run_reference(args, wl_name):
+    """Reference arm: the CPU oracle, timed on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from synth import make_workload
+    wl = make_workload(wl_name)
+    per_step = max(0.5, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        cpu_oracle_rate(wl, budget_s=0.0, rows=64)
+    vals, secs = [], 0.0
+    cores, sample = 1, ""
+    for _ in range(args.steps):
+        v, dt, cores, sample = cpu_oracle_rate(wl, budget_s=per_step, rows=256)
+        vals.append(v)
+        secs += dt
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * secs / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl_name, "B": wl.B, "M": wl.M, "N": wl.N, "rank": wl.rank,
+                   "fmt": f"{wl.fmt}{wl.bits}" if wl.fmt == "int" else wl.fmt},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import rank_bit_residual_b200 as rb
+    from synth import make_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    wl = make_workload(args.workload)
+    B, M, N, r = wl.B, wl.M, wl.N, wl.rank
+    fmt = f"int{wl.bits}" if wl.fmt == "int" else "nvfp4"
+    xdt = torch.bfloat16 if wl.x_dtype == "bf16" else torch.float32
+    x = torch.from_numpy(wl.x).to(xdt).to(dev)
+    W = torch.from_numpy(wl.W).to(xdt).to(dev)
+    scale = torch.from_numpy(wl.scale).to(dev)
+    bias = torch.from_numpy(wl.bias).to(torch.bfloat16).to(dev) if wl.bias is not None else None
+
+    # one-time split (timed separately)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    w = rb.svdq_prepare(W, scale, r, fmt, seed=0)
+    torch.cuda.synchronize()
+    prepare_ms = 1000.0 * (time.perf_counter() - t0)
+    del W
+
+    # buffers of the two stages (allocated once, outside the timed region)
+    codes, sf, act_scale, down = rb.svdq_quantize_act(x, scale, fmt, ld=w.ld if r else None)
+    y = torch.empty((B, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def act_stage():
+        rb.svdq_quantize_act_into(x, scale, fmt, w.ld if r else None, codes, sf, act_scale, down)
+
+    def gemm_stage():
+        rb.svdq_residual_linear(w, codes, sf, act_scale, down, bias=bias, out=y)
+
+    for _ in range(args.warmup):
+        act_stage()
+        gemm_stage()
+    torch.cuda.synchronize()
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+
+    sampler = ClockSampler(local)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        act_stage()
+        ev[i][1].record(stream)
+        gemm_stage()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    act_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ops_step = workload_ops(B, M, N, r)
+    value = world * K * ops_step / (total_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / K
+    gemm_avg_ms = sum(gemm_ms) / K
+    act_avg_ms = sum(act_ms) / K
+
+    # parity on sampled rows of the timed output (oracle from the prepared buffers)
+    parity = None
+    if rank == 0:
+        from oracle import codes as ocodes
+        from oracle import prepared as oprep
+        rows = np.random.default_rng(1).choice(B, size=min(B, 48), replace=False)
+        ld = w.ld.float().cpu().numpy()[: w.rank_pad].T
+        L2 = w.lu.float().cpu().numpy()[:, : w.rank_pad].T
+        if wl.fmt == "int":
+            q, s_x, _ = ocodes.act_codes_int_fp32(wl.x, wl.scale, wl.bits)
+            cw = w.codes.view(torch.int8).cpu().numpy().reshape(N, M)
+            want = oprep.linear_int(wl.x[rows], ld, L2, q[rows], s_x, cw, float(w.w_scale[0].item()),
+                                    wl.bias)
+            got = y[torch.from_numpy(rows).to(dev)].float().cpu().numpy()
+            rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
+            parity = {"rows_sampled": int(len(rows)), "rel_fro": rel,
+                      "max_rel": float(np.max(np.abs(got - want)) / np.max(np.abs(want)))}
+
+    # end to end through svdq_linear with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((B, N), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+    ws = rb.LinearWorkspace()
+    Ke = max(3, min(50, K))
+    for _ in range(3):
+        xd.copy_(x_host, non_blocking=True)
+        rb.svdq_linear(w, xd, bias=bias, out=y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        xd.copy_(x_host, non_blocking=True)
+        rb.svdq_linear(w, xd, bias=bias, out=y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * Ke * ops_step / (float(e2e_ms.item()) * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    int8_peak = 2.0 * peaks["bf16_tflops"]
+    g_ops = gemm_alg_ops(B, M, N, r)
+    achieved = g_ops / (gemm_avg_ms * 1e-3) / 1e12
+    traffic = read_profile_traffic(os.path.join(ROOT, "rank_bit_residual_b200", "csrc", "gemm.cu"))
+    bytes_step = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
+    t_rf = max(bytes_step / (peaks["hbm_gbs"] * 1e9),
+               (2.0 * B * M * N) / (int8_peak * 1e12) + (2.0 * B * r * (M + N)) / (peaks["bf16_tflops"] * 1e12))
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "M": M, "N": N, "rank": r, "fmt": fmt,
+                   "x": wl.x_dtype, "y": "bf16", "bias": wl.bias is not None,
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": f"replicas{world}"},
+        "gbs": bytes_step / (ms_per_step * 1e-3) / 1e9,
+        "step_roofline": {"t_roofline_us": t_rf * 1e6, "frac": t_rf / (ms_per_step * 1e-3),
+                          "alg_bytes": bytes_step, "ops": ops_step},
+        "stages_ms": {"act": act_avg_ms, "gemm": gemm_avg_ms},
+        "roofline": {"bound": "tensor", "kernel": "gemm_int_kernel (int8 residual + bf16 up-projection)",
+                     "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / int8_peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 GEMM burst x 2 (nominal int8:bf16)"},
+        "prepare_ms": prepare_ms,
+        "parity": parity,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(y.numel() * y.element_size()), "steps": Ke,
+                "call": "svdq_linear (pinned host x -> device, Y -> pinned host)"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        v, dt, cores, sample = cpu_oracle_rate(wl)
+        out["cpu_baseline"] = {"value": v, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                               "sample": sample, "seconds": dt}
+    elif rank == 0:
+        out["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -110,7 +110,7 @@ svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq
  *   scale  device fp32 [M], must be finite and > 0 (checked on the device)
  *   rank   0 <= rank <= min(M, N) (Python-int semantics are the binding's job)
  *   seed   seeds the Gaussian test matrix of the randomized subspace iteration
- *   oversample, power_iters  <= 0 select the defaults 16 and 2
+ *   oversample, power_iters  <= 0 select the defaults 16 and 4
  *   out    caller-allocated buffers (see svdq_weight); M, N, rank, rank_pad,
  *          fmt and scale are filled in by this call
  *
@@ -192,6 +192,24 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
                         void* workspace, size_t workspace_bytes, svdq_stream_t stream);
 
 svdq_status svdq_linear_workspace_size(const svdq_weight* w, int64_t B, size_t* bytes);
+
+/*
+ * svdq_residual_linear - the GEMM stage of svdq_linear on its own, from
+ * activation codes made by svdq_quantize_act (step 3 of the three-step chain of
+ * "flashinfer.gemm.svdquant_linear": residual GEMM with the low-rank
+ * up-projection and bias in its epilogue):
+ *   Y = alpha * (codes . w->codes^T) + down_hi.lu^T + down_lo.lu^T [+ bias]
+ *
+ *   act_codes INT int8 [B, M] / NVFP4 uint8 [B, M/2] (from svdq_quantize_act)
+ *   act_sf    NVFP4 128x4 scale layout of [B, M/16]; NULL for INT
+ *   act_scale device fp32 scalar from svdq_quantize_act (s_x or gs_x)
+ *   down      bf16 [B, 2 * w->rank_pad] from svdq_quantize_act; NULL iff rank == 0
+ *   bias      nullable bf16 [N];  y [B, N] (ldy >= N) bf16 or fp32
+ */
+svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, const void* act_sf,
+                                 const float* act_scale, const void* down, int64_t B,
+                                 const void* bias, void* y, svdq_dtype y_dtype, int64_t ldy,
+                                 svdq_stream_t stream);
 
 /*
  * svdq_residual_product_i32 - the INT residual GEMM alone, exact int32:

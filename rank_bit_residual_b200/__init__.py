@@ -60,6 +60,8 @@ _SIGS = {
                             c_vp, c_i32, c_i64, c_vp, c_sz, c_vp]),
     "svdq_linear_workspace_size": (c_i32, [ctypes.POINTER(SvdqWeight), c_i64, ctypes.POINTER(c_sz)]),
     "svdq_residual_product_i32": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i64, c_vp, c_i64, c_vp]),
+    "svdq_residual_linear": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
+                                     c_vp, c_i32, c_i64, c_vp]),
     "svdq_check_status": (c_i32, [c_vp]),
     "svdq_selftest_wait_timeout": (c_i32, [c_i64, c_vp]),
 }
@@ -274,20 +276,7 @@ def svdq_quantize_residual(R: torch.Tensor, fmt="int4"):
     return codes, sf, w_scale
 
 
-def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Optional[torch.Tensor] = None,
-                      act_global_scale: Optional[torch.Tensor] = None):
-    """Fused activation pass: returns (codes, sf or None, act_scale, down or None).
-
-    ld is the [rank_pad, M] down factor (bf16 for bf16 x, fp32 for fp32 x); down is
-    bf16 [B, 2 * rank_pad] (hi | lo).
-    """
-    lib = load_library()
-    _require_cuda(x, scale)
-    f = parse_fmt(fmt)
-    x = _rows_ready(x)
-    B, M = x.shape
-    rp = ld.shape[0] if ld is not None else 0
-    dev = x.device
+def _act_buffers(B, M, f, rp, dev):
     if f.kind == KIND_INT:
         codes = torch.empty((B, M), dtype=torch.int8, device=dev)
         sf = None
@@ -297,14 +286,49 @@ def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Opti
                          dtype=torch.uint8, device=dev)
     act_scale = torch.zeros(1, dtype=torch.float32, device=dev)
     down = torch.empty((B, 2 * rp), dtype=torch.bfloat16, device=dev) if rp else None
-    wsz = c_sz()
-    _check(lib.svdq_quantize_act_workspace_size(B, M, f, rp, ctypes.byref(wsz)), "workspace")
-    ws = torch.empty(max(wsz.value, 1), dtype=torch.uint8, device=dev)
-    _check(lib.svdq_quantize_act(_ptr(x), _dt(x), B, M, x.stride(0), _ptr(scale.contiguous()), f,
-                                 _ptr(act_global_scale), _ptr(ld), rp, _ptr(codes), _ptr(sf),
-                                 _ptr(act_scale), _ptr(down), _ptr(ws), wsz.value, _stream()),
-           "svdq_quantize_act")
     return codes, sf, act_scale, down
+
+
+_act_ws = {}
+
+
+def svdq_quantize_act_into(x: torch.Tensor, scale: torch.Tensor, fmt, ld: Optional[torch.Tensor],
+                           codes: torch.Tensor, sf: Optional[torch.Tensor], act_scale: torch.Tensor,
+                           down: Optional[torch.Tensor], act_global_scale: Optional[torch.Tensor] = None):
+    """svdq_quantize_act writing into caller buffers (shapes as returned by svdq_quantize_act)."""
+    lib = load_library()
+    f = parse_fmt(fmt)
+    x = _rows_ready(x)
+    B, M = x.shape
+    rp = ld.shape[0] if ld is not None else 0
+    key = (x.device, B, M, f.kind, rp)
+    ws = _act_ws.get(key)
+    if ws is None:
+        wsz = c_sz()
+        _check(lib.svdq_quantize_act_workspace_size(B, M, f, rp, ctypes.byref(wsz)), "workspace")
+        ws = torch.empty(max(wsz.value, 1), dtype=torch.uint8, device=x.device)
+        _act_ws[key] = ws
+    _check(lib.svdq_quantize_act(_ptr(x), _dt(x), B, M, x.stride(0), _ptr(scale), f,
+                                 _ptr(act_global_scale), _ptr(ld), rp, _ptr(codes), _ptr(sf),
+                                 _ptr(act_scale), _ptr(down), _ptr(ws), ws.numel(), _stream()),
+           "svdq_quantize_act")
+
+
+def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Optional[torch.Tensor] = None,
+                      act_global_scale: Optional[torch.Tensor] = None):
+    """Fused activation pass: returns (codes, sf or None, act_scale, down or None).
+
+    ld is the [rank_pad, M] down factor (bf16 for bf16 x, fp32 for fp32 x); down is
+    bf16 [B, 2 * rank_pad] (hi | lo).
+    """
+    _require_cuda(x, scale)
+    f = parse_fmt(fmt)
+    x = _rows_ready(x)
+    B, M = x.shape
+    rp = ld.shape[0] if ld is not None else 0
+    bufs = _act_buffers(B, M, f, rp, x.device)
+    svdq_quantize_act_into(x, scale.contiguous(), f, ld, *bufs, act_global_scale=act_global_scale)
+    return bufs
 
 
 class LinearWorkspace:
@@ -353,6 +377,23 @@ def svdq_linear(w: PreparedWeight, x: torch.Tensor, bias: Optional[torch.Tensor]
     return y
 
 
+def svdq_residual_linear(w: PreparedWeight, act_codes: torch.Tensor, act_sf: Optional[torch.Tensor],
+                         act_scale: torch.Tensor, down: Optional[torch.Tensor],
+                         bias: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
+                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """GEMM stage alone: Y from the outputs of svdq_quantize_act (current stream)."""
+    lib = load_library()
+    _require_cuda(act_codes, act_scale)
+    B = act_codes.shape[0]
+    y = out if out is not None else torch.empty((B, w.N), dtype=out_dtype, device=act_codes.device)
+    if bias is not None:
+        bias = bias.to(torch.bfloat16).contiguous()
+    _check(lib.svdq_residual_linear(ctypes.byref(w.desc), _ptr(act_codes), _ptr(act_sf), _ptr(act_scale),
+                                    _ptr(down), B, _ptr(bias), _ptr(y), _dt(y), y.stride(0), _stream()),
+           "svdq_residual_linear")
+    return y
+
+
 def svdq_residual_product_i32(w: PreparedWeight, act_codes: torch.Tensor) -> torch.Tensor:
     """Exact int32 product act_codes[B, M] . codes[N, M]^T of the INT residual branch."""
     lib = load_library()
@@ -376,8 +417,8 @@ def svdq_selftest_wait_timeout(limit_us: int = 1000) -> int:
 
 
 __all__ = [
-    "svdq_prepare", "svdq_quantize_act", "svdq_quantize_residual", "svdq_linear",
-    "svdq_residual_product_i32", "svdq_check_status", "svdq_selftest_wait_timeout",
+    "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_residual", "svdq_linear",
+    "svdq_residual_product_i32", "svdq_residual_linear", "svdq_check_status", "svdq_selftest_wait_timeout",
     "PreparedWeight", "LinearWorkspace", "allocate_weight", "weight_from_buffers",
     "weight_buffer_sizes", "load_library", "header_functions", "parse_fmt",
 ]

@@ -355,6 +355,33 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
   return from_cuda(e);
 }
 
+svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, const void* act_sf,
+                                 const float* act_scale, const void* down, int64_t B,
+                                 const void* bias, void* y, svdq_dtype y_dtype, int64_t ldy,
+                                 svdq_stream_t stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (B < 0 || (y_dtype != SVDQ_BF16 && y_dtype != SVDQ_F32)) return SVDQ_EINVAL;
+  if (B == 0) return SVDQ_OK;
+  if (!act_codes || !act_scale || !y || ldy < w->N) return SVDQ_EINVAL;
+  if (w->fmt.kind == SVDQ_KIND_NVFP4 && !act_sf) return SVDQ_EINVAL;
+  if (w->rank > 0 && !down) return SVDQ_EINVAL;
+  if (!aligned16(act_codes) || (down && !aligned16(down)) || (bias && !aligned16(bias)))
+    return SVDQ_EUNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bool bad = false;
+  cudaError_t e;
+  if (w->fmt.kind == SVDQ_KIND_INT)
+    e = launch_gemm_int(w, static_cast<const int8_t*>(act_codes), act_scale,
+                        w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, st, &bad);
+  else
+    e = launch_gemm_nvfp4(w, static_cast<const uint8_t*>(act_codes),
+                          static_cast<const uint8_t*>(act_sf), act_scale,
+                          w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, st, &bad);
+  if (bad) return SVDQ_EUNSUPPORTED;
+  return from_cuda(e);
+}
+
 svdq_status svdq_residual_product_i32(const svdq_weight* w, const int8_t* act_codes, int64_t B,
                                       int32_t* acc, int64_t ldacc, svdq_stream_t stream) {
   svdq_status s = check_weight(w);

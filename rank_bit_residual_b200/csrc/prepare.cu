@@ -34,7 +34,7 @@ namespace svdq {
 namespace {
 
 constexpr int kDefaultOversample = 16;
-constexpr int kDefaultPowerIters = 2;
+constexpr int kDefaultPowerIters = 4;
 constexpr int kQrThreads = 512;
 constexpr int kMaxL = 288;
 
