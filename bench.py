@@ -268,13 +268,17 @@ def main():
     del W
 
     # buffers of the two stages (allocated once, outside the timed region)
-    codes, sf, act_scale, down = rb.svdq_quantize_act(x, scale, fmt, ld=w.ld if r else None)
+    codes, sf, act_scale, down = rb.svdq_quantize_act(
+        x, scale, fmt, ld=w.ld if r else None, w_global_scale=w.w_scale if wl.fmt == "nvfp4" else None)
     y = torch.empty((B, N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    wgs = w.w_scale if wl.fmt == "nvfp4" else None
+
     def act_stage():
-        rb.svdq_quantize_act_into(x, scale, fmt, w.ld if r else None, codes, sf, act_scale, down)
+        rb.svdq_quantize_act_into(x, scale, fmt, w.ld if r else None, codes, sf, act_scale, down,
+                                  w_global_scale=wgs)
 
     def gemm_stage():
         rb.svdq_residual_linear(w, codes, sf, act_scale, down, bias=bias, out=y)

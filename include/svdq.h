@@ -156,6 +156,11 @@ svdq_status svdq_quantize_residual_workspace_size(int64_t M, int64_t N, svdq_fmt
  *   scale    device fp32 [M] (precondition: finite and > 0; not re-checked)
  *   act_global_scale  NVFP4 only, nullable: a given gs_x; NULL computes
  *            gs_x = 448*6 / max|X_hat| from the data. Ignored for INT.
+ *   w_global_scale    NVFP4 only, nullable: the weight's gs_w (w->w_scale). The
+ *            NVFP4 GEMM accumulates both branches in one fp32 accumulator in units
+ *            of 1 / (gs_x gs_w), so for NVFP4 `down` is written already multiplied
+ *            by gs_x (and by gs_w when given); svdq_residual_linear expects the
+ *            gs_x gs_w form. Ignored for INT.
  *   ld       nullable: bf16 [rank_pad, M] (or fp32 for fp32 x) down factor;
  *            NULL (or rank_pad = 0) skips the down-projection
  *   codes    out INT int8 [B, M] / NVFP4 uint8 [B, M/2]
@@ -166,7 +171,8 @@ svdq_status svdq_quantize_residual_workspace_size(int64_t M, int64_t N, svdq_fmt
  */
 svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
                               int64_t ldx, const float* scale, svdq_fmt fmt,
-                              const float* act_global_scale, const void* ld, int32_t rank_pad,
+                              const float* act_global_scale, const float* w_global_scale,
+                              const void* ld, int32_t rank_pad,
                               void* codes, void* sf, float* act_scale, void* down,
                               void* workspace, size_t workspace_bytes, svdq_stream_t stream);
 
@@ -203,7 +209,8 @@ svdq_status svdq_linear_workspace_size(const svdq_weight* w, int64_t B, size_t* 
  *   act_codes INT int8 [B, M] / NVFP4 uint8 [B, M/2] (from svdq_quantize_act)
  *   act_sf    NVFP4 128x4 scale layout of [B, M/16]; NULL for INT
  *   act_scale device fp32 scalar from svdq_quantize_act (s_x or gs_x)
- *   down      bf16 [B, 2 * w->rank_pad] from svdq_quantize_act; NULL iff rank == 0
+ *   down      bf16 [B, 2 * w->rank_pad] from svdq_quantize_act (NVFP4: called with
+ *             w_global_scale = w->w_scale); NULL iff rank == 0
  *   bias      nullable bf16 [N];  y [B, N] (ldy >= N) bf16 or fp32
  */
 svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, const void* act_sf,

@@ -53,7 +53,7 @@ _SIGS = {
     "svdq_quantize_residual": (c_i32, [c_vp, c_i64, c_i64, c_i64, SvdqFmt, c_vp, c_vp, c_vp,
                                        c_vp, c_sz, c_vp]),
     "svdq_quantize_residual_workspace_size": (c_i32, [c_i64, c_i64, SvdqFmt, ctypes.POINTER(c_sz)]),
-    "svdq_quantize_act": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, SvdqFmt, c_vp, c_vp,
+    "svdq_quantize_act": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, SvdqFmt, c_vp, c_vp, c_vp,
                                   c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "svdq_quantize_act_workspace_size": (c_i32, [c_i64, c_i64, SvdqFmt, c_i32, ctypes.POINTER(c_sz)]),
     "svdq_linear": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i32, c_i64, c_i64, c_vp, c_vp,
@@ -294,7 +294,8 @@ _act_ws = {}
 
 def svdq_quantize_act_into(x: torch.Tensor, scale: torch.Tensor, fmt, ld: Optional[torch.Tensor],
                            codes: torch.Tensor, sf: Optional[torch.Tensor], act_scale: torch.Tensor,
-                           down: Optional[torch.Tensor], act_global_scale: Optional[torch.Tensor] = None):
+                           down: Optional[torch.Tensor], act_global_scale: Optional[torch.Tensor] = None,
+                           w_global_scale: Optional[torch.Tensor] = None):
     """svdq_quantize_act writing into caller buffers (shapes as returned by svdq_quantize_act)."""
     lib = load_library()
     f = parse_fmt(fmt)
@@ -309,17 +310,20 @@ def svdq_quantize_act_into(x: torch.Tensor, scale: torch.Tensor, fmt, ld: Option
         ws = torch.empty(max(wsz.value, 1), dtype=torch.uint8, device=x.device)
         _act_ws[key] = ws
     _check(lib.svdq_quantize_act(_ptr(x), _dt(x), B, M, x.stride(0), _ptr(scale), f,
-                                 _ptr(act_global_scale), _ptr(ld), rp, _ptr(codes), _ptr(sf),
+                                 _ptr(act_global_scale), _ptr(w_global_scale), _ptr(ld), rp,
+                                 _ptr(codes), _ptr(sf),
                                  _ptr(act_scale), _ptr(down), _ptr(ws), ws.numel(), _stream()),
            "svdq_quantize_act")
 
 
 def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Optional[torch.Tensor] = None,
-                      act_global_scale: Optional[torch.Tensor] = None):
+                      act_global_scale: Optional[torch.Tensor] = None,
+                      w_global_scale: Optional[torch.Tensor] = None):
     """Fused activation pass: returns (codes, sf or None, act_scale, down or None).
 
     ld is the [rank_pad, M] down factor (bf16 for bf16 x, fp32 for fp32 x); down is
-    bf16 [B, 2 * rank_pad] (hi | lo).
+    bf16 [B, 2 * rank_pad] (hi | lo). For NVFP4, down is multiplied by gs_x (and by
+    w_global_scale when given), the units the NVFP4 GEMM accumulates in.
     """
     _require_cuda(x, scale)
     f = parse_fmt(fmt)
@@ -327,7 +331,8 @@ def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Opti
     B, M = x.shape
     rp = ld.shape[0] if ld is not None else 0
     bufs = _act_buffers(B, M, f, rp, x.device)
-    svdq_quantize_act_into(x, scale.contiguous(), f, ld, *bufs, act_global_scale=act_global_scale)
+    svdq_quantize_act_into(x, scale.contiguous(), f, ld, *bufs, act_global_scale=act_global_scale,
+                           w_global_scale=w_global_scale)
     return bufs
 
 

@@ -279,9 +279,10 @@ __device__ __forceinline__ void load8_scale(const float* __restrict__ p, float (
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Sum the K-split partial down tiles and store bf16 hi | lo.
+// Sum the K-split partial down tiles, multiply by `mult` and store bf16 hi | lo.
 __device__ __forceinline__ void finalize_down(const float* __restrict__ ws_down, int ksplit,
-                                              int B, int rank_pad, __nv_bfloat16* down) {
+                                              int B, int rank_pad, __nv_bfloat16* down,
+                                              float mult) {
   const int64_t total = static_cast<int64_t>(B) * rank_pad;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -289,6 +290,7 @@ __device__ __forceinline__ void finalize_down(const float* __restrict__ ws_down,
     const int j = static_cast<int>(i - row * rank_pad);
     float v = 0.0f;
     for (int sp = 0; sp < ksplit; ++sp) v += ws_down[(static_cast<int64_t>(sp) * B + row) * rank_pad + j];
+    v = __fmul_rn(v, mult);
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
     down[row * 2 * rank_pad + j] = hi;
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(256)
     }
     *reinterpret_cast<uint2*>(codes + row * M + k0) = make_uint2(packed[0], packed[1]);
   }
-  if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down);
+  if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down, 1.0f);
 }
 
 // ------------------------------------------------------------------ NVFP4
@@ -372,7 +374,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(256)
     act_quant_nvfp4_kernel(const TIn* __restrict__ x, int64_t ldx, const float* __restrict__ scale,
                            int B, int M, const float* __restrict__ ws_max, int nparts,
-                           const float* __restrict__ gs_given, const float* __restrict__ ws_down,
+                           const float* __restrict__ gs_given, const float* __restrict__ gs_w,
+                           const float* __restrict__ ws_down,
                            int ksplit, int rank_pad, uint8_t* __restrict__ codes,
                            uint8_t* __restrict__ sf, __nv_bfloat16* __restrict__ down,
                            float* __restrict__ act_scale) {
@@ -426,7 +429,10 @@ __global__ void __launch_bounds__(256)
         make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
     sf[off] = sfb;
   }
-  if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down);
+  // down in the units of the NVFP4 GEMM accumulator: x ld^T gs_x gs_w (gs_w when given)
+  if (rank_pad > 0 && down != nullptr)
+    finalize_down(ws_down, ksplit, B, rank_pad, down,
+                  gs_w != nullptr ? __fmul_rn(gs, __ldg(gs_w)) : gs);
 }
 
 }  // namespace
@@ -456,8 +462,9 @@ size_t act_scratch_bytes(const ActPlan& p) {
 
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
-                       const void* ld, void* codes, void* sf, float* act_scale, void* down,
-                       void* scratch, cudaStream_t stream, bool* bad_args) {
+                       const float* w_global_scale, const void* ld, void* codes, void* sf,
+                       float* act_scale, void* down, void* scratch, cudaStream_t stream,
+                       bool* bad_args) {
   *bad_args = false;
   if (p.B == 0) return cudaSuccess;
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
@@ -532,12 +539,12 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
     if (xdt == SVDQ_BF16)
       act_quant_nvfp4_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(x), ldx, scale, static_cast<int>(p.B),
-          static_cast<int>(p.M), ws_max, p.nparts, act_global_scale, ws_down, p.ksplit, rp,
-          static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
+          static_cast<int>(p.M), ws_max, p.nparts, act_global_scale, w_global_scale, ws_down,
+          p.ksplit, rp, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
     else
       act_quant_nvfp4_kernel<float><<<blocks, threads, 0, stream>>>(
           static_cast<const float*>(x), ldx, scale, static_cast<int>(p.B), static_cast<int>(p.M),
-          ws_max, p.nparts, act_global_scale, ws_down, p.ksplit, rp,
+          ws_max, p.nparts, act_global_scale, w_global_scale, ws_down, p.ksplit, rp,
           static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
   }
   return cudaGetLastError();

@@ -286,7 +286,8 @@ svdq_status svdq_quantize_act_workspace_size(int64_t B, int64_t M, svdq_fmt fmt,
 
 svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
                               int64_t ldx, const float* scale, svdq_fmt fmt,
-                              const float* act_global_scale, const void* ld, int32_t rank_pad,
+                              const float* act_global_scale, const float* w_global_scale,
+                              const void* ld, int32_t rank_pad,
                               void* codes, void* sf, float* act_scale, void* down,
                               void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
   svdq_status s = check_act_input(x, x_dtype, B, M, ldx);
@@ -302,9 +303,10 @@ svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int6
   if (!workspace || workspace_bytes < act_scratch_bytes(p)) return SVDQ_EWORKSPACE;
   bool bad = false;
   const cudaError_t e =
-      launch_act(p, x, x_dtype, ldx, scale, fmt, act_global_scale, rank_pad > 0 ? ld : nullptr,
-                 codes, sf, act_scale, down, workspace, reinterpret_cast<cudaStream_t>(stream),
-                 &bad);
+      launch_act(p, x, x_dtype, ldx, scale, fmt, act_global_scale,
+                 fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr,
+                 rank_pad > 0 ? ld : nullptr, codes, sf, act_scale, down, workspace,
+                 reinterpret_cast<cudaStream_t>(stream), &bad);
   if (bad) return SVDQ_EUNSUPPORTED;
   return from_cuda(e);
 }
@@ -339,6 +341,7 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
   const ActPlan p = plan_act(B, w->M, w->rank_pad, x_dtype);
   bool bad = false;
   cudaError_t e = launch_act(p, x, x_dtype, ldx, w->scale, w->fmt, act_global_scale,
+                             w->fmt.kind == SVDQ_KIND_NVFP4 ? w->w_scale : nullptr,
                              w->rank > 0 ? ld : nullptr, c.codes, c.sf, c.act_scale,
                              w->rank > 0 ? c.down : nullptr, c.act_scratch, st, &bad);
   if (bad) return SVDQ_EUNSUPPORTED;

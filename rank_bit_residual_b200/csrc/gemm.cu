@@ -1,20 +1,28 @@
-// gemm.cu - the residual GEMM with the low-rank epilogue (INT grid).
+// gemm.cu - the residual GEMM with the low-rank epilogue.
 //
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula item 3:
 //   Y = (X_hat L1) L2 + Q(X_hat) Q(R)
-// evaluated from prepared operands as
-//   Y[b, n] = s_x s_w * sum_k cx[b, k] cw[n, k] + sum_j down[b, j] lu[n, j] (+ bias[n])
-// where the integer product runs on tcgen05 kind::i8 (int8 x int8 -> exact int32
-// in TMEM) and the up-projection down . lu^T is a second, small kind::f16 MMA
-// into its own fp32 TMEM accumulator, so the low-rank branch costs no pass
-// over Y. `down` holds hi | lo bf16 halves of the fp32 down-projection and `lu`
-// holds the up factor twice, so one K = 2 r MMA chain sums hi.lu + lo.lu.
+// evaluated from prepared operands ("flashinfer.gemm.svdquant_linear", step 3:
+// residual GEMM with the low-rank up-projection and bias in the epilogue).
+//
+// INT grid:   Y[b, n] = s_x s_w sum_k cx[b, k] cw[n, k] + sum_j down[b, j] lu[n, j] (+ bias)
+//   the integer product runs on tcgen05 kind::i8 (exact int32 in TMEM columns
+//   [0, 256)) and the up-projection on kind::f16 into its own fp32 accumulator
+//   (columns [256, 512)).
+// NVFP4:      Y[b, n] = (1 / (gs_x gs_w)) (sum_blocks (a sfa)(w sfw) + sum_j down'[b, j] lu[n, j])
+//   with down' = down gs_x gs_w written by the activation pass (the alpha fold
+//   of the NVFP4 operator's l1_scaled, applied to the down side because gs_x
+//   is per call), so both branches share one fp32 accumulator (columns
+//   [0, 256)) and the block scales take columns [256, 304): kind::mxf4nvf4
+//   with scale_vec::4X, the scales copied from shared memory by tcgen05.cp.
+// `down` holds hi | lo bf16 halves of the fp32 down-projection and `lu` holds
+// the up factor twice, so one K = 2 r MMA chain sums hi.lu + lo.lu.
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles, 6 warps:
-//   warp 0     TMA producer (4-stage ring of 48 KB: A 128x128 B, B 256x128 B)
+//   warp 0     TMA / bulk-copy producer (4-stage ring)
 //   warp 1     TMEM allocation and the single MMA-issuing thread
-//   warps 2-5  epilogue: TMEM -> registers -> dequantise + up + bias -> global
-// The low-rank K steps go through the same ring as the integer K steps.
+//   warps 2-5  epilogue: TMEM -> registers -> dequantise (+ up) + bias -> global
+// The low-rank K steps go through the same ring as the residual K steps.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -32,24 +40,47 @@ constexpr int kBN = 256;
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * 128;
 constexpr int kBBytes = kBN * 128;
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kSfaBytes = 4 * 512;       // 4 scale atoms (128 rows x 4 blocks each)
+constexpr int kSfbBytes = 2 * 4 * 512;   // two 128-row tiles of B
 constexpr int kGemmThreads = 192;
-constexpr uint32_t kTmemCols = 512;  // [0,256) int32 residual acc, [256,512) fp32 low-rank acc
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = 256;        // NVFP4: scale factors of A, 4 columns per MMA
+constexpr uint32_t kSfbCol = 272;        // NVFP4: scale factors of B, 8 columns per MMA
 
+enum Kind { kKindInt = 0, kKindNvfp4 = 1 };
 enum OutKind { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
+
+template <int kKind>
+struct Cfg {
+  static constexpr int kStageBytes =
+      kABytes + kBBytes + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
+};
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // a -> low half
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int kOut>
+struct GemmArgs {
+  int B, N, M, lr_steps;
+  const float* s_x;               // INT: s_x, NVFP4: gs_x
+  const float* s_w;               // INT: s_w, NVFP4: gs_w
+  const __nv_bfloat16* bias;
+  void* y;
+  int64_t ldy;
+  int vec_ok;
+  const uint8_t* sfa;             // NVFP4 activation scales (128x4 layout)
+  const uint8_t* sfb;             // NVFP4 weight scales (128x4 layout)
+  int katoms;                     // NVFP4: 64-element scale atoms per row tile = ceil(M / 64)
+  unsigned* status;
+};
+
+template <int kKind, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_int_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                    const __grid_constant__ CUtensorMap tm_da, const __grid_constant__ CUtensorMap tm_lu,
-                    int B, int N, int M, int lr_steps, const float* __restrict__ s_x,
-                    const float* __restrict__ s_w, const __nv_bfloat16* __restrict__ bias,
-                    void* __restrict__ y, int64_t ldy, int vec_ok, unsigned* status) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ CUtensorMap tm_da, const __grid_constant__ CUtensorMap tm_lu,
+                const GemmArgs args) {
+  constexpr int kStageBytes = Cfg<kKind>::kStageBytes;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
@@ -61,13 +92,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  const int B = args.B, N = args.N, M = args.M, lr_steps = args.lr_steps;
+  unsigned* status = args.status;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tiles_m = (B + kBM - 1) / kBM;
   const int tiles_n = (N + kBN - 1) / kBN;
   const int total = tiles_m * tiles_n;
-  const int ksteps = (M + 127) / 128;
+  // K elements per 128-byte stage row: 128 int8 or 256 e2m1
+  constexpr int kStageK = kKind == kKindNvfp4 ? 256 : 128;
+  const int ksteps = (M + kStageK - 1) / kStageK;
   const int steps_per_tile = lr_steps + ksteps;
+  const int n_rows_p = ((N + 127) / 128) * 128;  // rows of the weight scale layout
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -109,14 +145,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = mbar_wait(&empty_bar[s], ph ^ 1, status, &abort_sh);
           if (!ok) break;
           uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
           if (j < lr_steps) {
+            mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
             tma_load_2d(st, &tm_da, &full_bar[s], 64 * j, m0);
             tma_load_2d(st + kABytes, &tm_lu, &full_bar[s], 64 * j, n0);
           } else {
             const int k = j - lr_steps;
-            tma_load_2d(st, &tm_a, &full_bar[s], 128 * k, m0);
-            tma_load_2d(st + kABytes, &tm_b, &full_bar[s], 128 * k, n0);
+            if constexpr (kKind == kKindNvfp4) {
+              // scale atoms of this stage: one per 64 K elements that exist
+              const int a0 = 4 * k;
+              const int na = min(4, args.katoms - a0);
+              const int nrt = (n0 + 128 < n_rows_p) ? 2 : 1;
+              mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes + na * 512 * (1 + nrt));
+              tma_load_2d(st, &tm_a, &full_bar[s], 128 * k, m0);
+              tma_load_2d(st + kABytes, &tm_b, &full_bar[s], 128 * k, n0);
+              uint8_t* sfa_s = st + kABytes + kBBytes;
+              uint8_t* sfb_s = sfa_s + kSfaBytes;
+              bulk_load(sfa_s, args.sfa + (static_cast<int64_t>(m0 / 128) * args.katoms + a0) * 512,
+                        na * 512, &full_bar[s]);
+              for (int rt = 0; rt < nrt; ++rt)
+                bulk_load(sfb_s + rt * 2048,
+                          args.sfb + (static_cast<int64_t>(n0 / 128 + rt) * args.katoms + a0) * 512,
+                          na * 512, &full_bar[s]);
+            } else {
+              mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
+              tma_load_2d(st, &tm_a, &full_bar[s], 128 * k, m0);
+              tma_load_2d(st + kABytes, &tm_b, &full_bar[s], 128 * k, n0);
+            }
           }
         }
       }
@@ -130,12 +185,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint32_t id_i8 = idesc_i8(kBM, kBN);
       const uint32_t id_bf = idesc_bf16(kBM, kBN);
+      const uint32_t id_f4 = idesc_nvf4(kBM, kBN);
+      // INT: low-rank into its own fp32 accumulator; NVFP4: everything into one
+      const uint32_t lr_acc = kKind == kKindNvfp4 ? tmem : tmem + 256;
       uint32_t it = 0, lt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
         ok = mbar_wait(&tmem_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
         if (!ok) break;
         tc_fence_after();
+        const int n0 = (t / tiles_m) * kBN;
         for (int j = 0; j < steps_per_tile; ++j, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -147,14 +206,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (j < lr_steps) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_f16(tmem + 256, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk),
-                      id_bf, (j > 0 || kk > 0) ? 1u : 0u);
+              mma_f16(lr_acc, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_bf,
+                      (j > 0 || kk > 0) ? 1u : 0u);
           } else {
             const int k = j - lr_steps;
+            if constexpr (kKind == kKindNvfp4) {
+              const int na = min(4, args.katoms - 4 * k);
+              const int nrt = (n0 + 128 < n_rows_p) ? 2 : 1;
+              const uint32_t sfa_s = b0 + kBBytes;
+              const uint32_t sfb_s = sfa_s + kSfaBytes;
+              // scale atoms -> TMEM; tcgen05.cp and tcgen05.mma issued by one
+              // thread execute in order, so the columns can be reused per stage
+              for (int kk = 0; kk < na; ++kk) {
+                tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * kk, smem_desc_plain(sfa_s + 512 * kk));
+                for (int rt = 0; rt < nrt; ++rt)
+                  tmem_cp_32x128b_warpx4(tmem + kSfbCol + 8 * kk + 4 * rt,
+                                         smem_desc_plain(sfb_s + 2048 * rt + 512 * kk));
+              }
+              for (int kk = 0; kk < na; ++kk)
+                mma_nvf4(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
+                         (lr_steps > 0 || k > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk,
+                         tmem + kSfbCol + 8 * kk);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_i8(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_i8,
-                     (k > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_i8,
+                       (k > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(&empty_bar[s]);
         }
@@ -169,7 +247,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r_in = q * 32 + lane;
-    const float alpha = kOut == kOutI32 ? 0.0f : __ldg(s_x) * __ldg(s_w);
+    float alpha = 0.0f;
+    if (kOut != kOutI32) {
+      if (kKind == kKindNvfp4)
+        alpha = __fdiv_rn(1.0f, __fmul_rn(__ldg(args.s_x), __ldg(args.s_w)));
+      else
+        alpha = __ldg(args.s_x) * __ldg(args.s_w);
+    }
+    const bool sep_lr = kKind == kKindInt && kOut != kOutI32 && lr_steps > 0;
     uint32_t lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       if (!mbar_wait(&tmem_full_bar, lt & 1, status, &abort_sh)) break;
@@ -182,13 +267,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();  // the TMEM loads below are warp-collective
         uint32_t acc[32], up[32];
         tmem_ld_32x32b_x32(lane_addr + c0, acc);
-        if (kOut != kOutI32 && lr_steps) tmem_ld_32x32b_x32(lane_addr + 256 + c0, up);
+        if (sep_lr) tmem_ld_32x32b_x32(lane_addr + 256 + c0, up);
         tmem_ld_wait();
         const int n = n0 + c0;
         if (row >= B || n >= N) continue;
-        const bool full = vec_ok && (n + 32 <= N);
+        const bool full = args.vec_ok && (n + 32 <= N);
         if (kOut == kOutI32) {
-          int32_t* dst = static_cast<int32_t*>(y) + static_cast<int64_t>(row) * ldy + n;
+          int32_t* dst = static_cast<int32_t*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
           if (full) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
@@ -203,12 +288,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          v[j] = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
-          if (lr_steps) v[j] += __uint_as_float(up[j]);
+          if (kKind == kKindNvfp4) {
+            v[j] = alpha * __uint_as_float(acc[j]);
+          } else {
+            v[j] = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
+            if (sep_lr) v[j] += __uint_as_float(up[j]);
+          }
         }
-        if (bias != nullptr) {
+        if (args.bias != nullptr) {
           if (n + 32 <= N) {
-            const uint4* bp = reinterpret_cast<const uint4*>(bias + n);
+            const uint4* bp = reinterpret_cast<const uint4*>(args.bias + n);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const uint4 bb = __ldg(bp + g);
@@ -222,11 +311,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (n + j < N) v[j] += __bfloat162float(bias[n + j]);
+              if (n + j < N) v[j] += __bfloat162float(args.bias[n + j]);
           }
         }
         if (kOut == kOutF32) {
-          float* dst = static_cast<float*>(y) + static_cast<int64_t>(row) * ldy + n;
+          float* dst = static_cast<float*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
           if (full) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
@@ -237,7 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (n + j < N) dst[j] = v[j];
           }
         } else {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(y) + static_cast<int64_t>(row) * ldy + n;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
           if (full) {
 #pragma unroll
             for (int j = 0; j < 32; j += 8)
@@ -265,20 +354,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-}  // namespace
+template <int kKind, int kOut>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& da,
+                       const CUtensorMap& lu, const GemmArgs& args, int grid, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kStages) * Cfg<kKind>::kStageBytes + 1024;
+  cudaError_t err = cudaFuncSetAttribute(gemm_kernel<kKind, kOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  gemm_kernel<kKind, kOut><<<grid, kGemmThreads, smem, st>>>(a, b, da, lu, args);
+  return cudaGetLastError();
+}
 
-cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
-                            const void* down2, int64_t B, const void* bias, void* y,
-                            svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
-                            bool* bad_args) {
+// Shared host part: tensor maps, launch geometry, argument block.
+template <int kKind>
+cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8_t* act_sf,
+                        const float* s_x, const void* down2, int64_t B, const void* bias, void* y,
+                        svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                        bool* bad_args) {
   *bad_args = false;
   if (B == 0) return cudaSuccess;
   const int64_t M = w->M, N = w->N;
   const int rp = w->rank_pad;
   const bool has_lr = !raw_i32 && rp > 0 && down2 != nullptr;
+  // codes rows are 128 bytes per K step: M int8 or M/2 packed e2m1 bytes
+  const int64_t row_bytes = kKind == kKindNvfp4 ? M / 2 : M;
   CUtensorMap tm_a, tm_b, tm_da, tm_lu;
-  bool ok = make_tmap_2d(&tm_a, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, B, M, 128, kBM, true) &&
-            make_tmap_2d(&tm_b, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, N, M, 128, kBN, true);
+  bool ok =
+      make_tmap_2d(&tm_a, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, B, row_bytes, 128, kBM, true) &&
+      make_tmap_2d(&tm_b, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, N, row_bytes, 128, kBN, true);
   if (ok && has_lr) {
     ok = make_tmap_2d(&tm_da, down2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, B, 2 * rp, 64, kBM, true) &&
          make_tmap_2d(&tm_lu, w->lu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, N, 2 * rp, 64, kBN, true);
@@ -290,32 +394,57 @@ cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const
     *bad_args = true;
     return cudaSuccess;
   }
-  const int lr_steps = has_lr ? static_cast<int>(ceil_div(2 * rp, 64)) : 0;
+  GemmArgs args{};
+  args.B = static_cast<int>(B);
+  args.N = static_cast<int>(N);
+  args.M = static_cast<int>(M);
+  args.lr_steps = has_lr ? static_cast<int>(ceil_div(2 * rp, 64)) : 0;
+  args.s_x = s_x;
+  args.s_w = w->w_scale;
+  args.bias = static_cast<const __nv_bfloat16*>(raw_i32 ? nullptr : bias);
+  args.y = y;
+  args.ldy = ldy;
   const int elem = raw_i32 ? 4 : (ydt == SVDQ_F32 ? 4 : 2);
-  const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15) == 0 && (ldy * elem) % 16 == 0) ? 1 : 0;
+  args.vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15) == 0 && (ldy * elem) % 16 == 0) ? 1 : 0;
+  args.sfa = act_sf;
+  args.sfb = static_cast<const uint8_t*>(w->sf);
+  args.katoms = static_cast<int>(ceil_div(M, 64));
+  args.status = device_status_word();
   const int64_t tiles = ceil_div(B, kBM) * ceil_div(N, kBN);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
-  const size_t smem = static_cast<size_t>(kStages) * kStageBytes + 1024;
-  unsigned* status = device_status_word();
-  const float* sw = w->w_scale;
-  const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(raw_i32 ? nullptr : bias);
-  cudaError_t err;
-#define SVDQ_LAUNCH_GEMM(K)                                                                        \
-  err = cudaFuncSetAttribute(gemm_int_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
-                             static_cast<int>(smem));                                               \
-  if (err != cudaSuccess) return err;                                                               \
-  gemm_int_kernel<K><<<grid, kGemmThreads, smem, stream>>>(                                         \
-      tm_a, tm_b, tm_da, tm_lu, static_cast<int>(B), static_cast<int>(N), static_cast<int>(M),      \
-      lr_steps, s_x, sw, bb, y, ldy, vec_ok, status);
   if (raw_i32) {
-    SVDQ_LAUNCH_GEMM(kOutI32)
-  } else if (ydt == SVDQ_F32) {
-    SVDQ_LAUNCH_GEMM(kOutF32)
-  } else {
-    SVDQ_LAUNCH_GEMM(kOutBF16)
+    if constexpr (kKind == kKindInt) {
+      return launch_one<kKind, kOutI32>(tm_a, tm_b, tm_da, tm_lu, args, grid, stream);
+    } else {
+      *bad_args = true;
+      return cudaSuccess;
+    }
   }
-#undef SVDQ_LAUNCH_GEMM
-  return cudaGetLastError();
+  if (ydt == SVDQ_F32) return launch_one<kKind, kOutF32>(tm_a, tm_b, tm_da, tm_lu, args, grid, stream);
+  return launch_one<kKind, kOutBF16>(tm_a, tm_b, tm_da, tm_lu, args, grid, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
+                            const void* down2, int64_t B, const void* bias, void* y,
+                            svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                            bool* bad_args) {
+  return launch_gemm<kKindInt>(w, act_codes, nullptr, s_x, down2, B, bias, y, ydt, ldy, raw_i32,
+                               stream, bad_args);
+}
+
+cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
+                              const uint8_t* act_sf, const float* gs_x, const void* down2,
+                              int64_t B, const void* bias, void* y, svdq_dtype ydt,
+                              int64_t ldy, cudaStream_t stream, bool* bad_args) {
+  if (!act_sf || !w->sf || (reinterpret_cast<uintptr_t>(act_sf) & 15) ||
+      (reinterpret_cast<uintptr_t>(w->sf) & 15)) {
+    *bad_args = true;
+    return cudaSuccess;
+  }
+  return launch_gemm<kKindNvfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false,
+                                 stream, bad_args);
 }
 
 }  // namespace svdq

@@ -57,8 +57,9 @@ size_t act_scratch_bytes(const ActPlan& p);
 
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
-                       const void* ld, void* codes, void* sf, float* act_scale, void* down,
-                       void* scratch, cudaStream_t stream, bool* bad_args);
+                       const float* w_global_scale, const void* ld, void* codes, void* sf,
+                       float* act_scale, void* down, void* scratch, cudaStream_t stream,
+                       bool* bad_args);
 
 // ------------------------------------------------------------ residual GEMM
 cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,

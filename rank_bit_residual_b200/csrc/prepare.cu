@@ -772,11 +772,4 @@ svdq_status run_prepare(const void* W, svdq_dtype wdt, int64_t M, int64_t N, int
   return SVDQ_OK;
 }
 
-cudaError_t launch_gemm_nvfp4(const svdq_weight*, const uint8_t*, const uint8_t*, const float*,
-                              const void*, int64_t, const void*, void*, svdq_dtype, int64_t,
-                              cudaStream_t, bool* bad_args) {
-  *bad_args = true;
-  return cudaSuccess;
-}
-
 }  // namespace svdq

@@ -98,6 +98,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (no tensor map); both addresses 16-byte aligned,
+// size a multiple of 16; completes `bytes` on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------------------------------------------- tcgen05
 // TMEM addresses: bits [31:16] lane, [15:0] column.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -165,6 +175,24 @@ __device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t a, uint64_t b, uin
       : "memory");
 }
 
+// Block-scaled e2m1 x e2m1 -> fp32 with one ue4m3 scale per 16 elements (K = 64
+// per instruction); sfa / sfb are the TMEM addresses of the scale factors.
+__device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 32-row x 16-byte shared-memory tile into 4 TMEM columns of all four
+// 32-lane groups (row i of the tile lands in lanes i, 32+i, 64+i, 96+i).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 // Load 32 consecutive 32-bit columns of this warp's 32 TMEM lanes (one lane per thread).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -198,6 +226,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of an unswizzled run of 16-byte rows, 8-row groups 128 bytes apart
+// (the source of tcgen05.cp for scale factors).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
 // Instruction descriptors (dense, both operands K-major).
 //   bits [4,6) accumulator format (1 = f32, 2 = s32); [7,10) A format; [10,13) B
 //   format; [17,23) N >> 3; [24,29) M >> 4.
@@ -211,6 +249,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 }
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
   return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Block-scaled instruction descriptor: A and B e2m1 ([7,10) and [10,13) = 1),
+// ue4m3 scales (bit 23 = 0), scale-factor ids 0, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -64,3 +64,30 @@ def test_linear_rejects_mismatched_input():
     w = SyntheticWeight(64, 32, 4, "int4", seed=0)
     with pytest.raises(ValueError):
         rb.svdq_linear(w.w, torch.zeros((3, 96), dtype=torch.bfloat16, device=device()))
+
+
+NVFP4_CASES = [
+    (16, 256, 128, 16, False),
+    (1, 64, 16, 1, False),
+    (37, 96, 48, 0, True),
+    (130, 512, 272, 40, True),
+    (256, 1024, 512, 128, False),
+    (300, 3072, 768, 32, True),
+]
+
+
+@pytest.mark.parametrize("B,M,N,rank,bias", NVFP4_CASES)
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+@pytest.mark.parametrize("given_gs", [False, True])
+def test_linear_nvfp4_matches_oracle(B, M, N, rank, bias, xdt, given_gs):
+    wl = make_case(B, M, N, rank=rank, seed=B * 5 + N, dtype=xdt, bias=bias)
+    w = SyntheticWeight(M, N, rank, "nvfp4", seed=N + rank, scale=wl.scale)
+    b = to_dev(wl.bias, torch.bfloat16) if bias else None
+    gs = np.float32(321.0) if given_gs else None
+    gs_t = to_dev(np.array([gs], np.float32), torch.float32) if given_gs else None
+    y32 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.float32, act_global_scale=gs_t)
+    y16 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.bfloat16, act_global_scale=gs_t)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    want = w.oracle_y(wl.x, wl.bias if bias else None, gs_x=gs)
+    assert_y_close(y32.cpu().numpy(), want, f"nvfp4 {B}x{M}x{N} r={rank} {xdt}")
+    assert torch.equal(y16, y32.to(torch.bfloat16))

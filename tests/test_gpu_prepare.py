@@ -122,3 +122,24 @@ def test_prepare_is_deterministic_for_a_seed():
     a = rb.svdq_prepare(W, s, 16, "int4", seed=3)
     b = rb.svdq_prepare(W, s, 16, "int4", seed=3)
     assert torch.equal(a.codes, b.codes) and torch.equal(a.ld, b.ld) and torch.equal(a.lu, b.lu)
+
+
+@pytest.mark.parametrize("M,N,rank,bias", [(256, 128, 16, False), (1024, 768, 32, True)])
+def test_prepare_then_linear_nvfp4(M, N, rank, bias):
+    wl = make_case(64, M, N, rank=rank, seed=M + 3, bias=bias)
+    w = rb.svdq_prepare(to_dev(wl.W, torch.bfloat16), to_dev(wl.scale, torch.float32), rank, "nvfp4")
+    b = to_dev(wl.bias, torch.bfloat16) if bias else None
+    y = rb.svdq_linear(w, x_tensor(wl), bias=b, out_dtype=torch.float32).cpu().numpy()
+    ld, lu = _host(w)
+    rp = w.rank_pad
+    cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
+    sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 16)
+    gs_w = float(w.w_scale[0].item())
+    xs = ocodes.smooth_fp32(wl.x, wl.scale)
+    ca, sa, gx = onv.quantize(xs)
+    want = oprep.linear_nvfp4(wl.x, ld.T, lu[:, :rp].T, ca, sa, gx, cw, sfw, gs_w,
+                              wl.bias if bias else None)
+    assert_y_close(y, want, "prepare+nvfp4")
+    # the residual codes are the oracle's NVFP4 codes of the GPU residual's own recipe
+    ws, R = _residual(wl, w)
+    assert np.linalg.norm(R) <= 1.01 * osq.tail_norm(ws, rank)
