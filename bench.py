@@ -335,10 +335,18 @@ def main():
             cw = w.codes.view(torch.int8).cpu().numpy().reshape(N, M)
             want = oprep.linear_int(wl.x[rows], ld, L2, q[rows], s_x, cw, float(w.w_scale[0].item()),
                                     wl.bias)
-            got = y[torch.from_numpy(rows).to(dev)].float().cpu().numpy()
-            rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
-            parity = {"rows_sampled": int(len(rows)), "rel_fro": rel,
-                      "max_rel": float(np.max(np.abs(got - want)) / np.max(np.abs(want)))}
+        else:
+            from oracle import nvfp4 as onv
+            xs = ocodes.smooth_fp32(wl.x, wl.scale)
+            ca, sa, gx = onv.quantize(xs)
+            cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
+            sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 16)
+            want = oprep.linear_nvfp4(wl.x[rows], ld, L2, ca[rows], sa[rows], gx, cw, sfw,
+                                      float(w.w_scale[0].item()), wl.bias)
+        got = y[torch.from_numpy(rows).to(dev)].float().cpu().numpy()
+        rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
+        parity = {"rows_sampled": int(len(rows)), "rel_fro": rel, "y": "bf16 (rounding included)",
+                  "max_rel": float(np.max(np.abs(got - want)) / np.max(np.abs(want)))}
 
     # end to end through svdq_linear with host buffers
     x_host = x.cpu().pin_memory()
@@ -366,18 +374,21 @@ def main():
     e2e_value = world * Ke * ops_step / (float(e2e_ms.item()) * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    int8_peak = 2.0 * peaks["bf16_tflops"]
+    # a contraction takes the peak of its own dtype: measured bf16 x nominal ratio
+    ratio = 4.0 if wl.fmt == "nvfp4" else 2.0
+    lowp_peak = ratio * peaks["bf16_tflops"]
     g_ops = gemm_alg_ops(B, M, N, r)
     achieved = g_ops / (gemm_avg_ms * 1e-3) / 1e12
     traffic = read_profile_traffic(os.path.join(ROOT, "rank_bit_residual_b200", "csrc", "gemm.cu"))
     bytes_step = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
     t_rf = max(bytes_step / (peaks["hbm_gbs"] * 1e9),
-               (2.0 * B * M * N) / (int8_peak * 1e12) + (2.0 * B * r * (M + N)) / (peaks["bf16_tflops"] * 1e12))
+               (2.0 * B * M * N) / (lowp_peak * 1e12) + (2.0 * B * r * (M + N)) / (peaks["bf16_tflops"] * 1e12))
 
     out = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1" if wl.fmt == "nvfp4" else "int8",
+        "data": "synthetic",
         "config": {"workload": args.workload, "B": B, "M": M, "N": N, "rank": r, "fmt": fmt,
                    "x": wl.x_dtype, "y": "bf16", "bias": wl.bias is not None,
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
@@ -386,10 +397,14 @@ def main():
         "step_roofline": {"t_roofline_us": t_rf * 1e6, "frac": t_rf / (ms_per_step * 1e-3),
                           "alg_bytes": bytes_step, "ops": ops_step},
         "stages_ms": {"act": act_avg_ms, "gemm": gemm_avg_ms},
-        "roofline": {"bound": "tensor", "kernel": "gemm_int_kernel (int8 residual + bf16 up-projection)",
-                     "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
-                     "frac": achieved / int8_peak, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 GEMM burst x 2 (nominal int8:bf16)"},
+        "roofline": {"bound": "tensor",
+                     "kernel": ("gemm_kernel<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
+                                if wl.fmt == "nvfp4" else
+                                "gemm_kernel<INT> (int8 residual + bf16 up-projection)"),
+                     "achieved": achieved, "peak": lowp_peak, "unit": "TFLOP/s",
+                     "frac": achieved / lowp_peak, "traffic": traffic,
+                     "peak_source": (f"{peak_src} bf16 GEMM burst x {ratio:g} "
+                                     f"(nominal {'fp4' if ratio == 4 else 'int8'}:bf16)")},
         "prepare_ms": prepare_ms,
         "parity": parity,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x.numel() * x.element_size()),

@@ -3,17 +3,22 @@
 The page-1 grid ("Formula and conventions", item 3) is
 s = max|z| / qmax, q = clamp(round_half_even(z / s), -qmax, qmax), with
 X_hat = x / scale (item 1). Exact mode (oracle.svdquant) evaluates this in
-float64; a GPU evaluates it in fp32. For bit-exact code comparison the oracle
-repeats the fp32 evaluation, each step one IEEE fp32 operation:
+float64; a GPU evaluates it in fp32, where a division per element costs an
+order of magnitude more than a multiply. The fp32 reading used here replaces
+each per-element division by a multiply with a correctly rounded reciprocal
+taken once per column (smoothing) or once per tensor (the grid step); every
+step is one IEEE fp32 operation:
 
-  xs = fl32(x / scale)          IEEE division, x already fp32 (bf16 upcast is exact)
-  m  = max |xs|                 exact in any order
-  s  = fl32(m / qmax)
-  q  = rint_even(fl32(xs / s)), clamped to [-qmax, qmax]
+  r_k = fl(1 / scale_k)          once per input channel
+  xs  = fl(x * r_k)              x already fp32 (the bf16 upcast is exact)
+  m   = max |xs|                 exact in any order
+  s   = fl(m / qmax);  u = fl(1 / s)
+  q   = rint_even(fl(xs * u)), clamped to [-qmax, qmax]
 
-Elements whose exact quotient lies within one fp32 ulp of a rounding
-boundary (k + 1/2) are flagged: a different but still correctly rounded fp32
-evaluation could decide them either way, and the comparison reports them.
+Each quotient is then within ~2 ulp of the exact one, so a code can differ from
+the float64 definition only when the exact quotient lies within 2 fp32 ulps of
+a rounding boundary (k + 1/2); those elements are flagged, and comparisons
+report them.
 """
 
 from __future__ import annotations
@@ -23,24 +28,26 @@ import numpy as np
 from .svdquant import qmax_of
 
 
-def _near_half(xs32: np.ndarray, s32: np.float32) -> np.ndarray:
-    t = xs32.astype(np.float64) / np.float64(s32)
+def _near_half(t: np.ndarray) -> np.ndarray:
+    """Quotients within 2 fp32 ulps of a half-integer."""
+    t = np.asarray(t, dtype=np.float64)
     frac = t - np.floor(t)
     ulp = np.spacing(np.abs(t).astype(np.float32)).astype(np.float64)
-    return np.abs(frac - 0.5) <= ulp
+    return np.abs(frac - 0.5) <= 2.0 * ulp
 
 
 def smooth_fp32(x, scale) -> np.ndarray:
-    """X_hat = fl32(x / scale) with IEEE fp32 division, per input channel."""
+    """X_hat = fl(x * fl(1 / scale)) per input channel."""
     x32 = np.asarray(x, dtype=np.float32)
-    s32 = np.asarray(scale, dtype=np.float32)
-    return (x32 / s32[None, :]).astype(np.float32)
+    r32 = (np.float32(1.0) / np.asarray(scale, dtype=np.float32)).astype(np.float32)
+    return (x32 * r32[None, :]).astype(np.float32)
 
 
-def int_codes_fp32(z32: np.ndarray, bits: int):
+def int_codes_fp32(z32: np.ndarray, bits: int, exact_quotient=None):
     """Per-tensor symmetric INT codes of an fp32 tensor: (codes int8, s fp32, near_tie).
 
-    An all-zero tensor has s = 0 and zero codes.
+    An all-zero tensor has s = 0 and zero codes. `exact_quotient(s)` may supply
+    the float64 quotient the near-tie flags are taken on (default z / s).
     """
     z32 = np.asarray(z32, dtype=np.float32)
     qm = np.float32(qmax_of(bits))
@@ -49,14 +56,22 @@ def int_codes_fp32(z32: np.ndarray, bits: int):
     if s == 0:
         return (np.zeros(z32.shape, dtype=np.int8), np.float32(0.0),
                 np.zeros(z32.shape, dtype=bool))
-    t = (z32 / s).astype(np.float32)
+    u = np.float32(np.float32(1.0) / s)
+    t = (z32 * u).astype(np.float32)
     q = np.clip(np.rint(t), -qm, qm).astype(np.int8)
-    return q, s, _near_half(z32, s)
+    tq = exact_quotient(s) if exact_quotient is not None else z32.astype(np.float64) / np.float64(s)
+    return q, s, _near_half(tq)
 
 
 def act_codes_int_fp32(x, scale, bits: int):
-    """Activation branch: INT codes of X_hat = x / scale (per tensor)."""
-    return int_codes_fp32(smooth_fp32(x, scale), bits)
+    """Activation branch: INT codes of X_hat = x / scale (per tensor).
+
+    Near-tie flags are taken on the exact quotient x / (scale * s).
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    sc64 = np.asarray(scale, dtype=np.float64)
+    return int_codes_fp32(smooth_fp32(x, scale), bits,
+                          exact_quotient=lambda s: x64 / (sc64[None, :] * np.float64(s)))
 
 
 def residual_codes_int_fp32(R32, bits: int):

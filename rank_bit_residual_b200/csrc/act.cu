@@ -19,6 +19,10 @@
 //                     the partial maxima to the per-tensor scale and writes the
 //                     codes; it also sums the partial down tiles and writes them
 //                     as bf16 hi | lo for the GEMM's low-rank MMA.
+// fp32 evaluation order (the one the oracle's fp32 code mode repeats): the
+// per-element divisions of the definition are multiplies by correctly rounded
+// reciprocals, r_k = fl(1 / scale_k) once per column and u = fl(1 / s) once
+// per tensor: X_hat = fl(x r_k), code = rint(fl(X_hat u)).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -75,7 +79,7 @@ __device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* _
         const int k = kbase + 8 * c + 2 * w + h;
         if (k < M) {
           const uint32_t bits = h ? (mx[w] & 0xFFFF0000u) : (mx[w] << 16);
-          run = fmaxf(run, __fdiv_rn(__uint_as_float(bits), __ldg(scale + k)));
+          run = fmaxf(run, __fmul_rn(__uint_as_float(bits), __frcp_rn(__ldg(scale + k))));
         }
       }
     }
@@ -83,7 +87,7 @@ __device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* _
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int k = kbase + 4 * c + w;
-      if (k < M) run = fmaxf(run, __fdiv_rn(__uint_as_float(mx[w]), __ldg(scale + k)));
+      if (k < M) run = fmaxf(run, __fmul_rn(__uint_as_float(mx[w]), __frcp_rn(__ldg(scale + k))));
     }
   }
   return run;
@@ -284,8 +288,9 @@ __device__ __forceinline__ void finalize_down(const float* __restrict__ ws_down,
                                               int B, int rank_pad, __nv_bfloat16* down,
                                               float mult) {
   const int64_t total = static_cast<int64_t>(B) * rank_pad;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
+  const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+  for (int64_t i = bid * blockDim.x + threadIdx.x; i < total; i += nblk * blockDim.x) {
     const int64_t row = i / rank_pad;
     const int j = static_cast<int>(i - row * rank_pad);
     float v = 0.0f;
@@ -298,38 +303,45 @@ __device__ __forceinline__ void finalize_down(const float* __restrict__ ws_down,
   }
 }
 
+// 2-D grid: blockIdx.x picks 32 chunks of 8 columns (one per lane), blockIdx.y a
+// band of rows; warp ty takes rows ty, ty + 8, ... of the band. A warp reads one
+// 512-byte run of a row per step; the reciprocals are taken once per thread.
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     act_quant_int_kernel(const TIn* __restrict__ x, int64_t ldx, const float* __restrict__ scale,
-                         int B, int M, int qmax, const float* __restrict__ ws_max, int nparts,
+                         int B, int M, int qmax, int rows_per_block,
+                         const float* __restrict__ ws_max, int nparts,
                          const float* __restrict__ ws_down, int ksplit, int rank_pad,
                          int8_t* __restrict__ codes, __nv_bfloat16* __restrict__ down,
                          float* __restrict__ act_scale) {
   __shared__ float red[8];
   const float m = block_max_of_parts(ws_max, nparts, red);
   const float s = __fdiv_rn(m, static_cast<float>(qmax));
-  if (blockIdx.x == 0 && threadIdx.x == 0) *act_scale = s;
-  const int64_t cpr = M / 8;
-  const int64_t total = static_cast<int64_t>(B) * cpr;
-  for (int64_t ci = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; ci < total;
-       ci += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = ci / cpr;
-    const int k0 = static_cast<int>(ci - row * cpr) * 8;
-    float xv[8], sc[8];
-    load8<TIn>(x + row * ldx + k0, xv);
-    load8_scale(scale + k0, sc);
-    uint32_t packed[2] = {0u, 0u};
+  const float u = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *act_scale = s;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int cc = blockIdx.x * 32 + tx;
+  if (cc < M / 8) {
+    const int k0 = cc * 8;
+    float r[8];
+    load8_scale(scale + k0, r);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      int q = 0;
-      if (s > 0.0f) {
-        const float xs = __fdiv_rn(xv[j], sc[j]);
-        q = __float2int_rn(__fdiv_rn(xs, s));
+    for (int j = 0; j < 8; ++j) r[j] = __frcp_rn(r[j]);
+    const int row0 = blockIdx.y * rows_per_block;
+    const int row1 = min(B, row0 + rows_per_block);
+    for (int row = row0 + ty; row < row1; row += 8) {
+      float xv[8];
+      load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv);
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        int q = __float2int_rn(__fmul_rn(__fmul_rn(xv[j], r[j]), u));
         q = min(max(q, -qmax), qmax);
+        packed[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
       }
-      packed[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
+      *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * M + k0) =
+          make_uint2(packed[0], packed[1]);
     }
-    *reinterpret_cast<uint2*>(codes + row * M + k0) = make_uint2(packed[0], packed[1]);
   }
   if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down, 1.0f);
 }
@@ -370,12 +382,13 @@ __device__ __forceinline__ int64_t sf_swizzle_offset(int64_t row, int64_t col, i
          (col & 3);
 }
 
+// 2-D grid like the INT kernel, one thread per 16-element block of a row.
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     act_quant_nvfp4_kernel(const TIn* __restrict__ x, int64_t ldx, const float* __restrict__ scale,
-                           int B, int M, const float* __restrict__ ws_max, int nparts,
-                           const float* __restrict__ gs_given, const float* __restrict__ gs_w,
-                           const float* __restrict__ ws_down,
+                           int B, int M, int rows_per_block, const float* __restrict__ ws_max,
+                           int nparts, const float* __restrict__ gs_given,
+                           const float* __restrict__ gs_w, const float* __restrict__ ws_down,
                            int ksplit, int rank_pad, uint8_t* __restrict__ codes,
                            uint8_t* __restrict__ sf, __nv_bfloat16* __restrict__ down,
                            float* __restrict__ act_scale) {
@@ -386,48 +399,61 @@ __global__ void __launch_bounds__(256)
     gs = __ldg(gs_given);
   else
     gs = m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *act_scale = gs;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *act_scale = gs;
   const int kb = M / 16;
   const int64_t kbp = (kb + 3) / 4 * 4;
-  const int64_t rows_p = (static_cast<int64_t>(B) + 127) / 128 * 128;
-  const int64_t total = rows_p * kbp;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / kbp;
-    const int b = static_cast<int>(i - row * kbp);
-    const int64_t off = sf_swizzle_offset(row, b, kbp);
-    if (row >= B || b >= kb) {
-      sf[off] = 0;
-      continue;
-    }
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int b = blockIdx.x * 32 + tx;
+  if (b < kb) {
     const int k0 = b * 16;
-    float xs[16];
+    float r[16];
     {
-      float xv[8], sc[8];
-      load8<TIn>(x + row * ldx + k0, xv);
-      load8_scale(scale + k0, sc);
+      float t[8];
+      load8_scale(scale + k0, t);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) xs[j] = __fdiv_rn(xv[j], sc[j]);
-      load8<TIn>(x + row * ldx + k0 + 8, xv);
-      load8_scale(scale + k0 + 8, sc);
+      for (int j = 0; j < 8; ++j) r[j] = __frcp_rn(t[j]);
+      load8_scale(scale + k0 + 8, t);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) xs[8 + j] = __fdiv_rn(xv[j], sc[j]);
+      for (int j = 0; j < 8; ++j) r[8 + j] = __frcp_rn(t[j]);
     }
-    float amax = 0.0f;
+    const int row0 = blockIdx.y * rows_per_block;
+    const int row1 = min(B, row0 + rows_per_block);
+    for (int row = row0 + ty; row < row1; row += 8) {
+      float xs[16];
+      {
+        float xv[8];
+        load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs[j]));
-    const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
-    const float d = ue4m3_to_f32(sfb);
-    const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
-    float lo[8], hi[8];
+        for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(xv[j], r[j]);
+        load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0 + 8, xv);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      lo[j] = __fmul_rn(xs[j], enc);
-      hi[j] = __fmul_rn(xs[8 + j], enc);
+        for (int j = 0; j < 8; ++j) xs[8 + j] = __fmul_rn(xv[j], r[8 + j]);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs[j]));
+      const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
+      const float d = ue4m3_to_f32(sfb);
+      const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
+      float lo[8], hi[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        lo[j] = __fmul_rn(xs[j], enc);
+        hi[j] = __fmul_rn(xs[8 + j], enc);
+      }
+      *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * (M / 2) + b * 8) =
+          make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
+      sf[sf_swizzle_offset(row, b, kbp)] = sfb;
     }
-    *reinterpret_cast<uint2*>(codes + row * (M / 2) + b * 8) =
-        make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
-    sf[off] = sfb;
+  }
+  // zero the scale padding (rows up to a multiple of 128, columns up to 4)
+  const int64_t rows_p = (static_cast<int64_t>(B) + 127) / 128 * 128;
+  const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
+  const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+  for (int64_t i = bid * blockDim.x + threadIdx.x; i < rows_p * kbp; i += nblk * blockDim.x) {
+    const int64_t row = i / kbp;
+    const int64_t c = i - row * kbp;
+    if (row >= B || c >= kb) sf[sf_swizzle_offset(row, c, kbp)] = 0;
   }
   // down in the units of the NVFP4 GEMM accumulator: x ld^T gs_x gs_w (gs_w when given)
   if (rank_pad > 0 && down != nullptr)
@@ -512,39 +538,42 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
+  // quantise: 32 column chunks per block along x, a band of rows along y, sized
+  // for about eight blocks per SM
+  const int chunk = fmt.kind == SVDQ_KIND_INT ? 8 : 16;
+  const int gx = static_cast<int>(ceil_div(p.M / chunk, 32));
+  const int64_t want_blocks = static_cast<int64_t>(num_sms()) * 8;
+  int64_t rows_per_block = round_up(std::max<int64_t>(1, ceil_div(p.B * gx, want_blocks)), 8);
+  rows_per_block = std::max<int64_t>(rows_per_block, 8);
+  const int gy = static_cast<int>(ceil_div(p.B, rows_per_block));
+  dim3 qgrid(gx, gy);
   const int threads = 256;
-  int64_t work;
-  if (fmt.kind == SVDQ_KIND_INT)
-    work = p.B * (p.M / 8);
-  else
-    work = round_up(p.B, 128) * round_up(p.M / 16, 4);
-  work = std::max<int64_t>(work, has_ld ? p.B * p.rank_pad : 0);
-  const int blocks = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>(ceil_div(work, threads), static_cast<int64_t>(num_sms()) * 8)));
   __nv_bfloat16* down_bf = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
   const int rp = has_ld ? p.rank_pad : 0;
+  const int rpb = static_cast<int>(rows_per_block);
   if (fmt.kind == SVDQ_KIND_INT) {
     const int qmax = (1 << (fmt.bits - 1)) - 1;
     if (xdt == SVDQ_BF16)
-      act_quant_int_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
+      act_quant_int_kernel<__nv_bfloat16><<<qgrid, threads, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(x), ldx, scale, static_cast<int>(p.B),
-          static_cast<int>(p.M), qmax, ws_max, p.nparts, ws_down, p.ksplit, rp,
+          static_cast<int>(p.M), qmax, rpb, ws_max, p.nparts, ws_down, p.ksplit, rp,
           static_cast<int8_t*>(codes), down_bf, act_scale);
     else
-      act_quant_int_kernel<float><<<blocks, threads, 0, stream>>>(
+      act_quant_int_kernel<float><<<qgrid, threads, 0, stream>>>(
           static_cast<const float*>(x), ldx, scale, static_cast<int>(p.B), static_cast<int>(p.M),
-          qmax, ws_max, p.nparts, ws_down, p.ksplit, rp, static_cast<int8_t*>(codes), down_bf,
-          act_scale);
+          qmax, rpb, ws_max, p.nparts, ws_down, p.ksplit, rp, static_cast<int8_t*>(codes),
+          down_bf, act_scale);
   } else {
     if (xdt == SVDQ_BF16)
-      act_quant_nvfp4_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
+      act_quant_nvfp4_kernel<__nv_bfloat16><<<qgrid, threads, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(x), ldx, scale, static_cast<int>(p.B),
-          static_cast<int>(p.M), ws_max, p.nparts, act_global_scale, w_global_scale, ws_down,
-          p.ksplit, rp, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
+          static_cast<int>(p.M), rpb, ws_max, p.nparts, act_global_scale, w_global_scale,
+          ws_down, p.ksplit, rp, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf,
+          act_scale);
     else
-      act_quant_nvfp4_kernel<float><<<blocks, threads, 0, stream>>>(
+      act_quant_nvfp4_kernel<float><<<qgrid, threads, 0, stream>>>(
           static_cast<const float*>(x), ldx, scale, static_cast<int>(p.B), static_cast<int>(p.M),
-          ws_max, p.nparts, act_global_scale, w_global_scale, ws_down, p.ksplit, rp,
+          rpb, ws_max, p.nparts, act_global_scale, w_global_scale, ws_down, p.ksplit, rp,
           static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
   }
   return cudaGetLastError();

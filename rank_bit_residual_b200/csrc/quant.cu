@@ -2,8 +2,9 @@
 //
 // INT: the per-tensor grid of "SVDQuant Smoothing, Low-rank and Residual
 // Quantization" (Formula item 3): s_w = max|R| / qmax and
-// codes = clamp(round_half_even(R / s_w), -qmax, qmax), in fp32 with IEEE
-// division, written K-major as codes[N, M] (row n = column n of R).
+// codes = clamp(round_half_even(R / s_w), -qmax, qmax), in fp32 with the
+// division taken as a multiply by u = fl(1 / s_w), written K-major as
+// codes[N, M] (row n = column n of R).
 // NVFP4: 16-element blocks along M of each column of R, ue4m3 block scales in
 // the 128x4 layout and an fp32 global scale (the weight_fp4 / weight_sf /
 // alpha storage of "flashinfer.gemm.svdquant_linear"), same recipe as the
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(256) quant_int_transpose_kernel(
     float* __restrict__ w_scale) {
   const float m = reduce_parts(parts, nparts);
   const float s = __fdiv_rn(m, static_cast<float>(qmax));
+  const float u = s > 0.0f ? __frcp_rn(s) : 0.0f;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *w_scale = s;
   __shared__ int8_t tile[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(256) quant_int_transpose_kernel(
     const int64_t r = m0 + i, c = n0 + tx;
     int q = 0;
     if (r < M && c < N && s > 0.0f) {
-      q = __float2int_rn(__fdiv_rn(R[r * ldR + c], s));
+      q = __float2int_rn(__fmul_rn(R[r * ldR + c], u));
       q = min(max(q, -qmax), qmax);
     }
     tile[i][tx] = static_cast<int8_t>(q);
