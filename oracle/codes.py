@@ -15,10 +15,10 @@ step is one IEEE fp32 operation:
   s   = fl(m / qmax);  u = fl(1 / s)
   q   = rint_even(fl(xs * u)), clamped to [-qmax, qmax]
 
-Each quotient is then within ~2 ulp of the exact one, so a code can differ from
-the float64 definition only when the exact quotient lies within 2 fp32 ulps of
-a rounding boundary (k + 1/2); those elements are flagged, and comparisons
-report them.
+Each quotient then carries four roundings of at most half an ulp, so it lies
+within 4 fp32 ulps of the exact one, and a code can differ from the float64
+definition only when the exact quotient lies within 4 ulps of a rounding
+boundary (k + 1/2); those elements are flagged, and comparisons report them.
 """
 
 from __future__ import annotations
@@ -29,11 +29,11 @@ from .svdquant import qmax_of
 
 
 def _near_half(t: np.ndarray) -> np.ndarray:
-    """Quotients within 2 fp32 ulps of a half-integer."""
+    """Quotients within 4 fp32 ulps of a half-integer."""
     t = np.asarray(t, dtype=np.float64)
     frac = t - np.floor(t)
     ulp = np.spacing(np.abs(t).astype(np.float32)).astype(np.float64)
-    return np.abs(frac - 0.5) <= 2.0 * ulp
+    return np.abs(frac - 0.5) <= 4.0 * ulp
 
 
 def smooth_fp32(x, scale) -> np.ndarray:

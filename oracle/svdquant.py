@@ -137,6 +137,12 @@ def svdquant_linear(x, weight, scale, rank: int, bits: int = 4) -> np.ndarray:
 
 
 def tail_norm(weight, rank: int) -> float:
-    """Frobenius norm of the optimal rank-r residual (Eckart-Young), from the SVD."""
-    s = np.linalg.svd(_f64(weight), compute_uv=False)
-    return float(np.sqrt(np.sum(s[rank:] ** 2)))
+    """Frobenius norm of the optimal rank-r residual (Eckart-Young).
+
+    The squared singular values are the eigenvalues of the smaller Gram matrix,
+    so the tail is sqrt(sum of all but the r largest of them).
+    """
+    w = _f64(weight)
+    g = w.T @ w if w.shape[0] >= w.shape[1] else w @ w.T
+    lam = np.clip(np.sort(np.linalg.eigvalsh(g))[::-1], 0.0, None)
+    return float(np.sqrt(np.sum(lam[rank:])))

@@ -39,6 +39,8 @@ constexpr int kActThreads = 128;
 constexpr int kActStages = 4;
 constexpr int kRowsPerBlock = 128;
 constexpr int kTileBytes = kRowsPerBlock * 128;  // one 128 x 128-byte x tile
+constexpr int kRowsPerThread = 8;     // INT quantise: rows in flight per thread
+constexpr int kRowsPerThreadF4 = 4;   // NVFP4 quantise: rows in flight per thread
 
 __host__ __device__ constexpr uint32_t pow2_cols(int n) {
   return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : 256u;
@@ -327,20 +329,29 @@ __global__ void __launch_bounds__(256)
     load8_scale(scale + k0, r);
 #pragma unroll
     for (int j = 0; j < 8; ++j) r[j] = __frcp_rn(r[j]);
-    const int row0 = blockIdx.y * rows_per_block;
-    const int row1 = min(B, row0 + rows_per_block);
-    for (int row = row0 + ty; row < row1; row += 8) {
-      float xv[8];
-      load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv);
-      uint32_t packed[2] = {0u, 0u};
+    const int row0 = blockIdx.y * rows_per_block + ty;
+    // rows row0, row0 + 8, ... : all loads of a group are in flight before the math
+    for (int g = 0; g < rows_per_block; g += 8 * kRowsPerThread) {
+      float xv[kRowsPerThread][8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        int q = __float2int_rn(__fmul_rn(__fmul_rn(xv[j], r[j]), u));
-        q = min(max(q, -qmax), qmax);
-        packed[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int row = row0 + g + 8 * i;
+        if (row < B) load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv[i]);
       }
-      *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * M + k0) =
-          make_uint2(packed[0], packed[1]);
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int row = row0 + g + 8 * i;
+        if (row >= B) continue;
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          int q = __float2int_rn(__fmul_rn(__fmul_rn(xv[i][j], r[j]), u));
+          q = min(max(q, -qmax), qmax);
+          packed[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
+        }
+        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * M + k0) =
+            make_uint2(packed[0], packed[1]);
+      }
     }
   }
   if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down, 1.0f);
@@ -416,34 +427,40 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int j = 0; j < 8; ++j) r[8 + j] = __frcp_rn(t[j]);
     }
-    const int row0 = blockIdx.y * rows_per_block;
-    const int row1 = min(B, row0 + rows_per_block);
-    for (int row = row0 + ty; row < row1; row += 8) {
-      float xs[16];
-      {
-        float xv[8];
-        load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv);
+    const int row0 = blockIdx.y * rows_per_block + ty;
+    for (int g = 0; g < rows_per_block; g += 8 * kRowsPerThreadF4) {
+      float xv[kRowsPerThreadF4][16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(xv[j], r[j]);
-        load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0 + 8, xv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xs[8 + j] = __fmul_rn(xv[j], r[8 + j]);
+      for (int i = 0; i < kRowsPerThreadF4; ++i) {
+        const int row = row0 + g + 8 * i;
+        if (row < B) {
+          load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, *reinterpret_cast<float(*)[8]>(&xv[i][0]));
+          load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0 + 8, *reinterpret_cast<float(*)[8]>(&xv[i][8]));
+        }
       }
-      float amax = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs[j]));
-      const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
-      const float d = ue4m3_to_f32(sfb);
-      const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
-      float lo[8], hi[8];
+      for (int i = 0; i < kRowsPerThreadF4; ++i) {
+        const int row = row0 + g + 8 * i;
+        if (row >= B) continue;
+        float xs[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        lo[j] = __fmul_rn(xs[j], enc);
-        hi[j] = __fmul_rn(xs[8 + j], enc);
+        for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xv[i][j], r[j]);
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs[j]));
+        const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
+        const float d = ue4m3_to_f32(sfb);
+        const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
+        float lo[8], hi[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          lo[j] = __fmul_rn(xs[j], enc);
+          hi[j] = __fmul_rn(xs[8 + j], enc);
+        }
+        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * (M / 2) + b * 8) =
+            make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
+        sf[sf_swizzle_offset(row, b, kbp)] = sfb;
       }
-      *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * (M / 2) + b * 8) =
-          make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
-      sf[sf_swizzle_offset(row, b, kbp)] = sfb;
     }
   }
   // zero the scale padding (rows up to a multiple of 128, columns up to 4)
@@ -471,8 +488,9 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt) {
   p.tile_k = xdt == SVDQ_BF16 ? 64 : 32;
   p.nrb = static_cast<int>(ceil_div(B, kRowsPerBlock));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
+  // one wave: two CTAs per SM (shared memory allows two), split K to fill it
   const int target = 2 * num_sms();
-  int ks = static_cast<int>(ceil_div(target, std::max(p.nrb, 1)));
+  int ks = target / std::max(p.nrb, 1);
   ks = std::max(1, std::min(ks, p.nsteps));
   p.ksplit = ks;
   p.nparts = p.nrb * p.ksplit;
@@ -543,8 +561,9 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   const int chunk = fmt.kind == SVDQ_KIND_INT ? 8 : 16;
   const int gx = static_cast<int>(ceil_div(p.M / chunk, 32));
   const int64_t want_blocks = static_cast<int64_t>(num_sms()) * 8;
-  int64_t rows_per_block = round_up(std::max<int64_t>(1, ceil_div(p.B * gx, want_blocks)), 8);
-  rows_per_block = std::max<int64_t>(rows_per_block, 8);
+  const int64_t rows_step = 8 * (fmt.kind == SVDQ_KIND_INT ? kRowsPerThread : kRowsPerThreadF4);
+  int64_t rows_per_block =
+      round_up(std::max<int64_t>(1, ceil_div(p.B * gx, want_blocks)), rows_step);
   const int gy = static_cast<int>(ceil_div(p.B, rows_per_block));
   dim3 qgrid(gx, gy);
   const int threads = 256;

@@ -235,3 +235,11 @@ def test_integer_product_matches_brute_force():
     K = 12288
     big = prepared.int_product(np.full((1, K), 127), np.full((1, K), -127))
     assert big[0, 0] == -127 * 127 * K
+
+
+def test_tail_norm_matches_split_residual():
+    rng = _rng(12)
+    for shape, r in (((50, 30), 5), ((30, 50), 0), ((40, 40), 40)):
+        W = rng.standard_normal(shape)
+        res = sq.split_weight(W, r)[2]
+        assert abs(sq.tail_norm(W, r) - np.linalg.norm(res)) <= 1e-9 * np.linalg.norm(W)
