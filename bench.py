@@ -410,7 +410,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()), "steps": Ke,
                 "call": "svdq_linear (pinned host x -> device, Y -> pinned host)"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 2 * K,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:

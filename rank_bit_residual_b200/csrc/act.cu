@@ -1,28 +1,27 @@
-// act.cu - the activation pass of the SVDQuant linear.
+// act.cu - the activation pass of the SVDQuant linear, one cooperative kernel.
 //
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula items 1
 // and 3: X_hat = x / scale is quantised per tensor (INT grid, or NVFP4 blocks
 // for the variant of "flashinfer.gemm.svdquant_linear" step 1), and the
-// low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) in the same
-// pass over x.
+// low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) from the same
+// read of x.
 //
-// Two kernels:
-//   act_stats_kernel  reads x once through TMA (128-byte swizzled tiles). Per
-//                     tile it issues the down-projection MMA (tcgen05, bf16 or
-//                     tf32 in, fp32 in TMEM) and takes column maxima of |x|
-//                     from the same shared-memory tile. Since fl(a / s) is
-//                     monotone in a, max_b fl(|x_bk| / s_k) = fl(max_b |x_bk| / s_k):
-//                     one IEEE division per column instead of per element.
-//                     Grid = row blocks of 128 x K splits; each CTA writes a
-//                     partial max and a partial down tile (fp32).
-//   act_quant_*       re-reads x (L2-resident after the first kernel), reduces
-//                     the partial maxima to the per-tensor scale and writes the
-//                     codes; it also sums the partial down tiles and writes them
-//                     as bf16 hi | lo for the GEMM's low-rank MMA.
+// Work unit = 128 rows x a range of 128-byte K tiles. Phase 1 streams the
+// unit's x tiles in by TMA (128-byte swizzle), runs the down-projection on
+// tcgen05 (bf16, or tf32 for fp32 x, accumulated in TMEM) and takes column
+// maxima of |x| from the same shared-memory tiles; it writes a partial down
+// tile and a partial maximum. Since fl(a r) is monotone in a, the tensor
+// maximum of |X_hat| is max_k fl(colmax_k r_k). A bounded grid barrier then
+// makes the per-tensor scale known everywhere, and phase 2 writes the codes:
+// from the tiles still held in shared memory when the unit fits there (x is
+// then read from HBM exactly once), else by re-reading the unit from global
+// memory. Phase 2 also sums the partial down tiles into bf16 hi | lo.
+//
 // fp32 evaluation order (the one the oracle's fp32 code mode repeats): the
 // per-element divisions of the definition are multiplies by correctly rounded
 // reciprocals, r_k = fl(1 / scale_k) once per column and u = fl(1 / s) once
-// per tensor: X_hat = fl(x r_k), code = rint(fl(X_hat u)).
+// per tensor: X_hat = fl(x r_k), INT code = rint(fl(x c_k)) with the per-column
+// constant c_k = fl(r_k u).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,329 +34,36 @@ namespace svdq {
 
 namespace {
 
-constexpr int kActThreads = 128;
-constexpr int kActStages = 4;
-constexpr int kRowsPerBlock = 128;
-constexpr int kTileBytes = kRowsPerBlock * 128;  // one 128 x 128-byte x tile
-constexpr int kRowsPerThread = 8;     // INT quantise: rows in flight per thread
-constexpr int kRowsPerThreadF4 = 4;   // NVFP4 quantise: rows in flight per thread
+constexpr int kThreads = 512;
+constexpr int kRows = 128;                  // rows per unit (MMA M)
+constexpr int kTileBytes = kRows * 128;     // one 128 x 128-byte x tile
+constexpr int kRing = 4;                    // ring depth for ld tiles (and x tiles when not held)
+constexpr int kMaxHold = 12;                // x tiles a unit may keep in shared memory
+constexpr int kSmemBudget = 224 * 1024;
 
 __host__ __device__ constexpr uint32_t pow2_cols(int n) {
   return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : 256u;
 }
 
-// Column maxima of |x| over the 128-row tile for this thread's 16-byte chunk
-// (rows rg, rg+16, ..., rg+112), then fold fl(colmax / scale) into `run`.
-template <typename TIn>
-__device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* __restrict__ scale,
-                                             int kbase, int M, float run) {
-  const int tid = threadIdx.x;
-  const int c = tid & 7;     // logical 16-byte chunk of the 128-byte row
-  const int rg = tid >> 3;   // row group 0..15
-  const int p = c ^ (rg & 7);  // physical chunk position under the 128-byte swizzle
-  uint32_t mx0 = 0, mx1 = 0, mx2 = 0, mx3 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = rg + 16 * i;
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 128 + p * 16);
-    if constexpr (sizeof(TIn) == 2) {
-      mx0 = __vmaxu2(mx0, v.x & 0x7FFF7FFFu);
-      mx1 = __vmaxu2(mx1, v.y & 0x7FFF7FFFu);
-      mx2 = __vmaxu2(mx2, v.z & 0x7FFF7FFFu);
-      mx3 = __vmaxu2(mx3, v.w & 0x7FFF7FFFu);
-    } else {
-      mx0 = max(mx0, v.x & 0x7FFFFFFFu);
-      mx1 = max(mx1, v.y & 0x7FFFFFFFu);
-      mx2 = max(mx2, v.z & 0x7FFFFFFFu);
-      mx3 = max(mx3, v.w & 0x7FFFFFFFu);
-    }
-  }
-  const uint32_t mx[4] = {mx0, mx1, mx2, mx3};
-  if constexpr (sizeof(TIn) == 2) {
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int k = kbase + 8 * c + 2 * w + h;
-        if (k < M) {
-          const uint32_t bits = h ? (mx[w] & 0xFFFF0000u) : (mx[w] << 16);
-          run = fmaxf(run, __fmul_rn(__uint_as_float(bits), __frcp_rn(__ldg(scale + k))));
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int k = kbase + 4 * c + w;
-      if (k < M) run = fmaxf(run, __fmul_rn(__uint_as_float(mx[w]), __frcp_rn(__ldg(scale + k))));
-    }
-  }
-  return run;
-}
+struct ActArgs {
+  int B, M;
+  int64_t ldx;
+  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, hold, xbuf, fmt_kind, qmax;
+  const void* x;
+  const float* scale;
+  const float* gs_given;
+  const float* gs_w;
+  float* ws_down;   // [ksplit][B][rank_pad]
+  float* ws_max;    // [gridDim.x]
+  unsigned* sync;   // [0] barrier counter, [1] abort flag (zeroed before launch)
+  void* codes;
+  uint8_t* sf;
+  __nv_bfloat16* down;
+  float* act_scale;
+  unsigned* status;
+};
 
-template <typename TIn>
-__global__ void __launch_bounds__(kActThreads, 1)
-    act_stats_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_ld,
-                     const float* __restrict__ scale, int B, int M, int nsteps, int ksplit,
-                     int rank_pad, int has_ld, float* __restrict__ ws_down,
-                     float* __restrict__ ws_max, unsigned* status) {
-  constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kActStages];
-  __shared__ __align__(8) uint64_t mma_bar[kActStages];
-  __shared__ __align__(8) uint64_t final_bar;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
-  __shared__ float red_sh[kActThreads / 32];
-
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const int ld_bytes = rank_pad * 128;
-  const int stage_bytes = kTileBytes + (has_ld ? ld_bytes : 0);
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const int m0 = blockIdx.x * kRowsPerBlock;
-  const int sp = blockIdx.y;
-  const int k_lo = static_cast<int>((static_cast<int64_t>(nsteps) * sp) / ksplit);
-  const int k_hi = static_cast<int>((static_cast<int64_t>(nsteps) * (sp + 1)) / ksplit);
-  const int n = k_hi - k_lo;
-  const uint32_t tcols = pow2_cols(rank_pad);
-
-  if (tid == 0) {
-    for (int s = 0; s < kActStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&mma_bar[s], 1);
-    }
-    mbar_init(&final_bar, 1);
-    fence_mbar_init();
-    abort_sh = 0;
-    tma_prefetch_desc(&tm_x);
-    if (has_ld) tma_prefetch_desc(&tm_ld);
-  }
-  if (has_ld && warp == 0) {
-    tmem_alloc(&tmem_base_sh, tcols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = has_ld ? tmem_base_sh : 0u;
-
-  auto issue = [&](int i) {
-    const int s = i % kActStages;
-    uint8_t* st = smem + s * stage_bytes;
-    mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-    const int kc = (k_lo + i) * kTileK;
-    tma_load_2d(st, &tm_x, &full_bar[s], kc, m0);
-    if (has_ld) tma_load_2d(st + kTileBytes, &tm_ld, &full_bar[s], kc, 0);
-  };
-
-  if (tid == 0) {
-    for (int i = 0; i < min(n, kActStages); ++i) issue(i);
-  }
-
-  const uint32_t idesc = sizeof(TIn) == 2 ? idesc_bf16(128, rank_pad) : idesc_tf32(128, rank_pad);
-  float run = 0.0f;
-  int issued = min(n, kActStages);
-  int consumed = 0;
-  bool ok_all = true;
-  // Every thread runs every iteration (and its __syncthreads) even after a
-  // failed wait: a failure only turns the work of the remaining steps off.
-  for (int i = 0; i < n; ++i) {
-    const int s = i % kActStages;
-    const uint32_t ph = (i / kActStages) & 1;
-    ok_all = ok_all && mbar_wait(&full_bar[s], ph, status, &abort_sh);
-    if (ok_all) consumed = i + 1;
-    uint8_t* st = smem + s * stage_bytes;
-    if (ok_all && has_ld && tid == 0) {
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(st);
-      const uint32_t b0 = smem_u32(st + kTileBytes);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc_sw128(a0 + 32 * kk);
-        const uint64_t bd = smem_desc_sw128(b0 + 32 * kk);
-        if (sizeof(TIn) == 2)
-          mma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        else
-          mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(&mma_bar[s]);
-    }
-    if (ok_all) run = tile_absmax<TIn>(st, scale, (k_lo + i) * kTileK, M, run);
-    __syncthreads();
-    if (tid == 0 && ok_all && issued < n && !abort_sh) {
-      bool ok = true;
-      if (has_ld) ok = mbar_wait(&mma_bar[s], ph, status, &abort_sh);
-      if (ok) {
-        issue(issued);
-        ++issued;
-      }
-    }
-  }
-
-  // After a failed wait, let the loads already issued land before the shared
-  // memory they target is released (bounded like every other wait).
-  if (tid == 0) {
-    for (int i = consumed; i < issued; ++i)
-      mbar_wait(&full_bar[i % kActStages], (i / kActStages) & 1, status, nullptr);
-  }
-
-  // Partial down tile: TMEM lane = row, one fp32 column per factor column.
-  if (has_ld) {
-    if (tid == 0) mma_commit(&final_bar);
-    const bool ok = mbar_wait(&final_bar, 0, status, nullptr) && ok_all;
-    tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
-    float* dst = ws_down + (static_cast<int64_t>(sp) * B + row) * rank_pad;
-    for (int c0 = 0; c0 < rank_pad; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-      tmem_ld_wait();
-      if (ok && row < B) {
-        const int cnt = min(32, rank_pad - c0);
-        for (int j = 0; j < cnt; j += 4) {
-          *reinterpret_cast<float4*>(dst + c0 + j) =
-              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        }
-      }
-    }
-  }
-
-  // Partial per-tensor maximum of |X_hat|.
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-  if (lane == 0) red_sh[warp] = run;
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {
-    float m = red_sh[0];
-    for (int w = 1; w < kActThreads / 32; ++w) m = fmaxf(m, red_sh[w]);
-    ws_max[static_cast<int64_t>(sp) * gridDim.x + blockIdx.x] = m;
-  }
-  if (has_ld && warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, tcols);
-  }
-}
-
-__device__ __forceinline__ float block_max_of_parts(const float* __restrict__ parts, int nparts,
-                                                    float* red) {
-  float m = 0.0f;
-  for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = fmaxf(m, parts[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = red[0];
-    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) t = fmaxf(t, red[w]);
-    red[0] = t;
-  }
-  __syncthreads();
-  return red[0];
-}
-
-template <typename TIn>
-__device__ __forceinline__ void load8(const TIn* __restrict__ p, float (&v)[8]) {
-  if constexpr (sizeof(TIn) == 2) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = __uint_as_float(w[j] << 16);
-      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  } else {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
-}
-
-__device__ __forceinline__ void load8_scale(const float* __restrict__ p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-// Sum the K-split partial down tiles, multiply by `mult` and store bf16 hi | lo.
-__device__ __forceinline__ void finalize_down(const float* __restrict__ ws_down, int ksplit,
-                                              int B, int rank_pad, __nv_bfloat16* down,
-                                              float mult) {
-  const int64_t total = static_cast<int64_t>(B) * rank_pad;
-  const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
-  const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
-  for (int64_t i = bid * blockDim.x + threadIdx.x; i < total; i += nblk * blockDim.x) {
-    const int64_t row = i / rank_pad;
-    const int j = static_cast<int>(i - row * rank_pad);
-    float v = 0.0f;
-    for (int sp = 0; sp < ksplit; ++sp) v += ws_down[(static_cast<int64_t>(sp) * B + row) * rank_pad + j];
-    v = __fmul_rn(v, mult);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-    down[row * 2 * rank_pad + j] = hi;
-    down[row * 2 * rank_pad + rank_pad + j] = lo;
-  }
-}
-
-// 2-D grid: blockIdx.x picks 32 chunks of 8 columns (one per lane), blockIdx.y a
-// band of rows; warp ty takes rows ty, ty + 8, ... of the band. A warp reads one
-// 512-byte run of a row per step; the reciprocals are taken once per thread.
-template <typename TIn>
-__global__ void __launch_bounds__(256)
-    act_quant_int_kernel(const TIn* __restrict__ x, int64_t ldx, const float* __restrict__ scale,
-                         int B, int M, int qmax, int rows_per_block,
-                         const float* __restrict__ ws_max, int nparts,
-                         const float* __restrict__ ws_down, int ksplit, int rank_pad,
-                         int8_t* __restrict__ codes, __nv_bfloat16* __restrict__ down,
-                         float* __restrict__ act_scale) {
-  __shared__ float red[8];
-  const float m = block_max_of_parts(ws_max, nparts, red);
-  const float s = __fdiv_rn(m, static_cast<float>(qmax));
-  const float u = s > 0.0f ? __frcp_rn(s) : 0.0f;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *act_scale = s;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int cc = blockIdx.x * 32 + tx;
-  if (cc < M / 8) {
-    const int k0 = cc * 8;
-    float r[8];
-    load8_scale(scale + k0, r);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) r[j] = __frcp_rn(r[j]);
-    const int row0 = blockIdx.y * rows_per_block + ty;
-    // rows row0, row0 + 8, ... : all loads of a group are in flight before the math
-    for (int g = 0; g < rows_per_block; g += 8 * kRowsPerThread) {
-      float xv[kRowsPerThread][8];
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        const int row = row0 + g + 8 * i;
-        if (row < B) load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, xv[i]);
-      }
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        const int row = row0 + g + 8 * i;
-        if (row >= B) continue;
-        uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          int q = __float2int_rn(__fmul_rn(__fmul_rn(xv[i][j], r[j]), u));
-          q = min(max(q, -qmax), qmax);
-          packed[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
-        }
-        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * M + k0) =
-            make_uint2(packed[0], packed[1]);
-      }
-    }
-  }
-  if (rank_pad > 0 && down != nullptr) finalize_down(ws_down, ksplit, B, rank_pad, down, 1.0f);
-}
-
-// ------------------------------------------------------------------ NVFP4
+// ------------------------------------------------------------- small helpers
 __device__ __forceinline__ uint8_t f32_to_ue4m3(float v) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
@@ -371,8 +77,9 @@ __device__ __forceinline__ float ue4m3_to_f32(uint8_t b) {
                 : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// Eight floats -> eight e2m1 nibbles, element j in nibble j (low nibble first).
-__device__ __forceinline__ uint32_t f32x8_to_e2m1(const float (&v)[8]) {
+// Eight floats -> eight e2m1 nibbles, element j in nibble j (low nibble first);
+// a code whose magnitude is zero is stored as +0.
+__device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
   uint32_t out;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -382,7 +89,6 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float (&v)[8]) {
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(out)
       : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  // a code whose magnitude is zero is stored as +0
   const uint32_t mag = out & 0x77777777u;
   const uint32_t nz = (mag + 0x77777777u) & 0x88888888u;
   return out & (0x77777777u | nz);
@@ -393,112 +99,467 @@ __device__ __forceinline__ int64_t sf_swizzle_offset(int64_t row, int64_t col, i
          (col & 3);
 }
 
-// 2-D grid like the INT kernel, one thread per 16-element block of a row.
+// 16 bytes of x as floats: 8 bf16 or 4 fp32
 template <typename TIn>
-__global__ void __launch_bounds__(256)
-    act_quant_nvfp4_kernel(const TIn* __restrict__ x, int64_t ldx, const float* __restrict__ scale,
-                           int B, int M, int rows_per_block, const float* __restrict__ ws_max,
-                           int nparts, const float* __restrict__ gs_given,
-                           const float* __restrict__ gs_w, const float* __restrict__ ws_down,
-                           int ksplit, int rank_pad, uint8_t* __restrict__ codes,
-                           uint8_t* __restrict__ sf, __nv_bfloat16* __restrict__ down,
-                           float* __restrict__ act_scale) {
-  __shared__ float red[8];
-  const float m = block_max_of_parts(ws_max, nparts, red);
-  float gs;
-  if (gs_given != nullptr)
-    gs = __ldg(gs_given);
+__device__ __forceinline__ void unpack16(const uint4 u, float* v) {
+  if constexpr (sizeof(TIn) == 2) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
+  }
+}
+
+// Column maxima of |x| over a 128 x 128-byte swizzled tile. Thread t owns the
+// logical 16-byte chunk c = t % 8 of rows t/8 and t/8 + 64; it folds
+// fl(colmax r_k) of its chunk's columns into `run` (rcp: reciprocals of the
+// tile's columns, 0 past M).
+template <typename TIn>
+__device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* rcp, float run) {
+  const int tid = threadIdx.x;
+  const int c = tid & 7;
+  const int rg = tid >> 3;
+  const int p = c ^ (rg & 7);  // rows rg + 64 i share rg & 7
+  uint32_t mx[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < kRows / (kThreads / 8); ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + (rg + (kThreads / 8) * i) * 128 + p * 16);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if constexpr (sizeof(TIn) == 2)
+        mx[q] = __vmaxu2(mx[q], w[q] & 0x7FFF7FFFu);
+      else
+        mx[q] = max(mx[q], w[q] & 0x7FFFFFFFu);
+    }
+  }
+  if constexpr (sizeof(TIn) == 2) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q] << 16), rcp[8 * c + 2 * q]));
+      run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q] & 0xFFFF0000u), rcp[8 * c + 2 * q + 1]));
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q]), rcp[4 * c + q]));
+  }
+  return run;
+}
+
+// -------------------------------------------------------------- the kernel
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 1)
+    act_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_ld,
+                     const ActArgs a) {
+  constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));   // elements per 128-byte row
+  constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn)); // elements per 16 bytes
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t xfull[kMaxHold];
+  __shared__ __align__(8) uint64_t ldfull[kRing];
+  __shared__ __align__(8) uint64_t mmadone[kRing];
+  __shared__ __align__(8) uint64_t final_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float red[kThreads / 32];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ld_bytes = a.rank_pad * 128;
+  uint8_t* xbuf = smem;                                               // a.xbuf tiles
+  uint8_t* ldbuf = smem + static_cast<size_t>(a.xbuf) * kTileBytes;   // kRing ld tiles
+  float* rcp = reinterpret_cast<float*>(ldbuf + (a.has_ld ? kRing * ld_bytes : 0));
+  const uint32_t tcols = pow2_cols(a.rank_pad);
+  unsigned* status = a.status;
+
+  if (tid == 0) {
+    for (int s = 0; s < kMaxHold; ++s) mbar_init(&xfull[s], 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&ldfull[s], 1);
+      mbar_init(&mmadone[s], 1);
+    }
+    mbar_init(&final_bar, 1);
+    fence_mbar_init();
+    abort_sh = 0;
+    tma_prefetch_desc(&tm_x);
+    if (a.has_ld) tma_prefetch_desc(&tm_ld);
+  }
+  if (a.has_ld && warp == 0) {
+    tmem_alloc(&tmem_base_sh, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = a.has_ld ? tmem_base_sh : 0u;
+  const uint32_t idesc = sizeof(TIn) == 2 ? idesc_bf16(128, a.rank_pad) : idesc_tf32(128, a.rank_pad);
+
+  // barrier uses so far (phase parities carry across units)
+  uint32_t xuse[kMaxHold] = {};
+  uint32_t lduse = 0;
+  uint32_t final_use = 0;
+  float run = 0.0f;
+  bool ok = true;
+
+  // ================================================================ phase 1
+  for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
+    const int rb = unit % a.nrb, sp = unit / a.nrb;
+    const int m0 = rb * kRows;
+    const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
+    const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
+    const int n = k_hi - k_lo;
+    for (int j = tid; j < n * kTileK; j += kThreads) {
+      const int col = k_lo * kTileK + j;
+      rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
+    }
+    __syncthreads();
+    const uint32_t ld0 = lduse;
+    auto issue_x = [&](int i) {
+      const int b = i % a.xbuf;
+      mbar_arrive_expect_tx(&xfull[b], kTileBytes);
+      tma_load_2d(xbuf + static_cast<size_t>(b) * kTileBytes, &tm_x, &xfull[b], (k_lo + i) * kTileK, m0);
+    };
+    auto issue_ld = [&](int i) {
+      const uint32_t q = (ld0 + i) % kRing;
+      mbar_arrive_expect_tx(&ldfull[q], ld_bytes);
+      tma_load_2d(ldbuf + static_cast<size_t>(q) * ld_bytes, &tm_ld, &ldfull[q], (k_lo + i) * kTileK, 0);
+    };
+    if (tid == 0 && ok) {
+      for (int i = 0; i < min(n, a.xbuf); ++i) issue_x(i);
+      if (a.has_ld)
+        for (int i = 0; i < min(n, kRing); ++i) issue_ld(i);
+    }
+    // Step i reads x buffer i % xbuf and ld slot (ld0 + i) % kRing. At step i,
+    // thread 0 refills the buffers step i - 1 used (its MMA was issued a step
+    // ago, so the wait for it is normally already satisfied).
+    for (int i = 0; i < n; ++i) {
+      const int b = i % a.xbuf;
+      const uint32_t q = (ld0 + i) % kRing;
+      ok = ok && mbar_wait(&xfull[b], xuse[b] & 1, status, &abort_sh);
+      ++xuse[b];
+      if (a.has_ld && tid == 0) {
+        ok = ok && mbar_wait(&ldfull[q], ((ld0 + i) / kRing) & 1, status, &abort_sh);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(xbuf + static_cast<size_t>(b) * kTileBytes);
+          const uint32_t b0 = smem_u32(ldbuf + static_cast<size_t>(q) * ld_bytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a0 + 32 * kk);
+            const uint64_t bd = smem_desc_sw128(b0 + 32 * kk);
+            if (sizeof(TIn) == 2)
+              mma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&mmadone[q]);
+        }
+      }
+      if (ok) run = tile_absmax<TIn>(xbuf + static_cast<size_t>(b) * kTileBytes, rcp + i * kTileK, run);
+      __syncthreads();
+      if (tid == 0 && ok && i >= 1) {
+        const int jl = i - 1 + kRing;     // ld step that takes over slot of step i - 1
+        const int jx = i - 1 + a.xbuf;    // x step that takes over buffer of step i - 1
+        const bool need_ld = a.has_ld && jl < n;
+        const bool need_x = !a.hold && jx < n;
+        if (a.has_ld && (need_ld || need_x))
+          ok = mbar_wait(&mmadone[(ld0 + i - 1) % kRing], ((ld0 + i - 1) / kRing) & 1, status,
+                         &abort_sh);
+        if (ok && need_ld) issue_ld(jl);
+        if (ok && need_x) issue_x(jx);
+      }
+    }
+    if (a.has_ld) lduse += n;
+    if (a.has_ld) {
+      if (tid == 0) mma_commit(&final_bar);
+      const bool fin = mbar_wait(&final_bar, final_use & 1, status, nullptr);
+      ++final_use;
+      tc_fence_after();
+      // TMEM lane = row; warps 0-3 cover the 128 lanes (one lane quarter each)
+      if (warp < 4) {
+        const int row = m0 + warp * 32 + lane;
+        float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * a.rank_pad;
+        for (int c0 = 0; c0 < a.rank_pad; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          if (fin && ok && row < a.B) {
+            const int cnt = min(32, a.rank_pad - c0);
+            for (int j = 0; j < cnt; j += 4)
+              *reinterpret_cast<float4*>(dst + c0 + j) =
+                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                              __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
+  }
+  // a failed wait: let loads already issued land before the block moves on
+  if (tid == 0 && !ok) {
+    for (int s = 0; s < min(a.xbuf, kMaxHold); ++s)
+      mbar_wait(&xfull[s], xuse[s] & 1, status, nullptr, 1000000ull);
+  }
+  // per-CTA maximum -> ws_max[blockIdx.x]
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
+  if (lane == 0) red[warp] = run;
+  __syncthreads();
+  if (tid == 0) {
+    float m = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    a.ws_max[blockIdx.x] = m;
+  }
+
+  // ======================================================== grid barrier
+  GridSync gs{a.sync, a.sync + 1, status, 0};
+  ok = grid_sync(gs, &abort_sh) && ok;
+
+  // ================================================================ phase 2
+  if (ok) {
+    float m = 0.0f;
+    for (int i = tid; i < static_cast<int>(gridDim.x); i += kThreads) m = fmaxf(m, a.ws_max[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __syncthreads();
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
+    float s = 0.0f, u = 0.0f, gs_x = 1.0f;
+    if (nv) {
+      gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
+    } else {
+      s = __fdiv_rn(m, static_cast<float>(a.qmax));
+      u = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    }
+    if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv ? gs_x : s;
+    const int kb = a.M / 16;
+    const int64_t kbp = (kb + 3) / 4 * 4;
+
+    for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
+      const int rb = unit % a.nrb, sp = unit / a.nrb;
+      const int m0 = rb * kRows;
+      const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
+      const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
+      const int n = k_hi - k_lo;
+      if (!a.hold) {
+        __syncthreads();
+        for (int j = tid; j < n * kTileK; j += kThreads) {
+          const int col = k_lo * kTileK + j;
+          rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
+        }
+        __syncthreads();
+      }
+      const int rows = min(kRows, a.B - m0);
+      // the unit's 16-byte chunk (row r, logical chunk c) of tile t
+      auto chunk = [&](int t, int r, int c) -> uint4 {
+        if (a.hold)
+          return *reinterpret_cast<const uint4*>(xbuf + static_cast<size_t>(t) * kTileBytes + r * 128 +
+                                                 ((c ^ (r & 7)) * 16));
+        return __ldg(reinterpret_cast<const uint4*>(static_cast<const TIn*>(a.x) +
+                                                    static_cast<int64_t>(m0 + r) * a.ldx +
+                                                    (k_lo + t) * kTileK + c * kPerChunk));
+      };
+      if (!nv) {
+        // thread -> chunk c of rows r0, r0 + 64 of every tile; c_k = fl(r_k u) per column
+        const int c = tid & 7, r0 = tid >> 3;
+        for (int t = 0; t < n; ++t) {
+          const int col = (k_lo + t) * kTileK + c * kPerChunk;
+          if (col >= a.M) continue;
+          float ck[kPerChunk];
+#pragma unroll
+          for (int j = 0; j < kPerChunk; ++j) ck[j] = __fmul_rn(rcp[t * kTileK + c * kPerChunk + j], u);
+          uint4 raw[kRows / (kThreads / 8)];
+#pragma unroll
+          for (int i = 0; i < kRows / (kThreads / 8); ++i) {
+            const int r = r0 + (kThreads / 8) * i;
+            if (r < rows) raw[i] = chunk(t, r, c);
+          }
+#pragma unroll
+          for (int i = 0; i < kRows / (kThreads / 8); ++i) {
+            const int r = r0 + (kThreads / 8) * i;
+            if (r >= rows) continue;
+            float v[kPerChunk];
+            unpack16<TIn>(raw[i], v);
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < kPerChunk; ++j) {
+              int qv = __float2int_rn(__fmul_rn(v[j], ck[j]));
+              qv = min(max(qv, -a.qmax), a.qmax);
+              packed[j >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (j & 3));
+            }
+            int8_t* dst = static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r) * a.M + col;
+            if constexpr (kPerChunk == 8)
+              *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+            else
+              *reinterpret_cast<uint32_t*>(dst) = packed[0];
+          }
+        }
+      } else {
+        // thread -> 16-element block b of row r of every tile
+        constexpr int kBlk = kTileK / 16;                 // blocks per tile row
+        constexpr int kChunksPerBlk = 16 / kPerChunk;
+        constexpr int kRowsPerPass = kThreads / kBlk;     // rows covered per pass
+        const int bk = tid % kBlk, r0 = tid / kBlk;
+        for (int t = 0; t < n; ++t) {
+          const int col = (k_lo + t) * kTileK + bk * 16;
+          if (col >= a.M) continue;
+          for (int r = r0; r < rows; r += kRowsPerPass) {
+            float xs[16];
+#pragma unroll
+            for (int h = 0; h < kChunksPerBlk; ++h) {
+              unpack16<TIn>(chunk(t, r, bk * kChunksPerBlk + h), xs + h * kPerChunk);
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              xs[j] = __fmul_rn(xs[j], rcp[t * kTileK + bk * 16 + j]);
+              amax = fmaxf(amax, fabsf(xs[j]));
+            }
+            const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+            const float d = ue4m3_to_f32(sfb);
+            const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
+            const int row = m0 + r;
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(row) * (a.M / 2) +
+                                      col / 2) = make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
+            a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+          }
+        }
+      }
+      // down: this unit's share of the row block's rows, all K splits summed
+      if (a.has_ld && a.down != nullptr) {
+        const int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
+        const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
+        const int cnt = (r_hi - r_lo) * a.rank_pad;
+        for (int i = tid; i < cnt; i += kThreads) {
+          const int rr = r_lo + i / a.rank_pad, j = i % a.rank_pad;
+          const int row = m0 + rr;
+          if (row >= a.B) continue;
+          float acc = 0.0f;
+          for (int z = 0; z < a.ksplit; ++z)
+            acc += a.ws_down[(static_cast<int64_t>(z) * a.B + row) * a.rank_pad + j];
+          acc = __fmul_rn(acc, mult);
+          const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
+          a.down[static_cast<int64_t>(row) * 2 * a.rank_pad + j] = hi;
+          a.down[static_cast<int64_t>(row) * 2 * a.rank_pad + a.rank_pad + j] = lo;
+        }
+      }
+    }
+    // NVFP4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
+    if (nv) {
+      const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
+      const int64_t pad_cols = kbp - kb;
+      const int64_t n_pad = (rows_p - a.B) * kbp + static_cast<int64_t>(a.B) * pad_cols;
+      for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + tid; i < n_pad;
+           i += static_cast<int64_t>(gridDim.x) * kThreads) {
+        int64_t row, c;
+        if (i < static_cast<int64_t>(a.B) * pad_cols) {
+          row = i / pad_cols;
+          c = kb + (i - row * pad_cols);
+        } else {
+          const int64_t j = i - static_cast<int64_t>(a.B) * pad_cols;
+          row = a.B + j / kbp;
+          c = j - (j / kbp) * kbp;
+        }
+        a.sf[sf_swizzle_offset(row, c, kbp)] = 0;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (a.has_ld && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
+size_t smem_for(const ActPlan& p, int xbuf) {
+  const int ld_bytes = p.rank_pad * 128;
+  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+  return static_cast<size_t>(xbuf) * kTileBytes + (p.rank_pad > 0 ? kRing * ld_bytes : 0) +
+         static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
+}
+
+// Resident CTAs per SM for a given dynamic shared memory size (at most two:
+// each may hold TMEM for its down accumulator).
+int resident_per_sm(size_t smem, bool bf16) {
+  int n = 0;
+  cudaError_t e;
+  // the occupancy query honours the kernel's opt-in shared memory limit
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+      optin > 4096) {
+    const int lim = optin - 2048;
+    if (bf16)
+      cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    else
+      cudaFuncSetAttribute(act_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  }
+  if (bf16)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_fused_kernel<__nv_bfloat16>, kThreads,
+                                                      smem);
   else
-    gs = m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *act_scale = gs;
-  const int kb = M / 16;
-  const int64_t kbp = (kb + 3) / 4 * 4;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int b = blockIdx.x * 32 + tx;
-  if (b < kb) {
-    const int k0 = b * 16;
-    float r[16];
-    {
-      float t[8];
-      load8_scale(scale + k0, t);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) r[j] = __frcp_rn(t[j]);
-      load8_scale(scale + k0 + 8, t);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) r[8 + j] = __frcp_rn(t[j]);
-    }
-    const int row0 = blockIdx.y * rows_per_block + ty;
-    for (int g = 0; g < rows_per_block; g += 8 * kRowsPerThreadF4) {
-      float xv[kRowsPerThreadF4][16];
-#pragma unroll
-      for (int i = 0; i < kRowsPerThreadF4; ++i) {
-        const int row = row0 + g + 8 * i;
-        if (row < B) {
-          load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0, *reinterpret_cast<float(*)[8]>(&xv[i][0]));
-          load8<TIn>(x + static_cast<int64_t>(row) * ldx + k0 + 8, *reinterpret_cast<float(*)[8]>(&xv[i][8]));
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kRowsPerThreadF4; ++i) {
-        const int row = row0 + g + 8 * i;
-        if (row >= B) continue;
-        float xs[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xv[i][j], r[j]);
-        float amax = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs[j]));
-        const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
-        const float d = ue4m3_to_f32(sfb);
-        const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
-        float lo[8], hi[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          lo[j] = __fmul_rn(xs[j], enc);
-          hi[j] = __fmul_rn(xs[8 + j], enc);
-        }
-        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(row) * (M / 2) + b * 8) =
-            make_uint2(f32x8_to_e2m1(lo), f32x8_to_e2m1(hi));
-        sf[sf_swizzle_offset(row, b, kbp)] = sfb;
-      }
-    }
-  }
-  // zero the scale padding (rows up to a multiple of 128, columns up to 4)
-  const int64_t rows_p = (static_cast<int64_t>(B) + 127) / 128 * 128;
-  const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
-  const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
-  for (int64_t i = bid * blockDim.x + threadIdx.x; i < rows_p * kbp; i += nblk * blockDim.x) {
-    const int64_t row = i / kbp;
-    const int64_t c = i - row * kbp;
-    if (row >= B || c >= kb) sf[sf_swizzle_offset(row, c, kbp)] = 0;
-  }
-  // down in the units of the NVFP4 GEMM accumulator: x ld^T gs_x gs_w (gs_w when given)
-  if (rank_pad > 0 && down != nullptr)
-    finalize_down(ws_down, ksplit, B, rank_pad, down,
-                  gs_w != nullptr ? __fmul_rn(gs, __ldg(gs_w)) : gs);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_fused_kernel<float>, kThreads, smem);
+  if (e != cudaSuccess || n <= 0) n = smem > 110 * 1024 ? 1 : 2;
+  return std::max(1, std::min(n, 2));
 }
 
 }  // namespace
+
+void finish_act_plan(ActPlan& p) {
+  p.nunits = p.nrb * p.ksplit;
+  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+  // hold the unit's x tiles when they fit and every unit gets a CTA of its own
+  p.hold = 0;
+  p.xbuf = kRing;
+  if (steps_max <= kMaxHold) {
+    const size_t sm = smem_for(p, steps_max);
+    if (sm <= static_cast<size_t>(kSmemBudget) && p.nunits <= num_sms() * resident_per_sm(sm, p.bf16)) {
+      p.hold = 1;
+      p.xbuf = steps_max;
+    }
+  }
+  p.smem = smem_for(p, p.xbuf);
+  p.grid = std::min(p.nunits, num_sms() * resident_per_sm(p.smem, p.bf16));
+  p.nparts = p.grid;
+}
 
 ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt) {
   ActPlan p{};
   p.B = B;
   p.M = M;
   p.rank_pad = rank_pad;
-  p.tile_k = xdt == SVDQ_BF16 ? 64 : 32;
-  p.nrb = static_cast<int>(ceil_div(B, kRowsPerBlock));
+  p.bf16 = xdt == SVDQ_BF16;
+  p.tile_k = p.bf16 ? 64 : 32;
+  p.nrb = static_cast<int>(ceil_div(B, kRows));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
-  // one wave: two CTAs per SM (shared memory allows two), split K to fill it
-  const int target = 2 * num_sms();
-  int ks = target / std::max(p.nrb, 1);
-  ks = std::max(1, std::min(ks, p.nsteps));
+  // one unit per SM; split K further when that lets each unit's tiles stay in
+  // shared memory (then two units share an SM)
+  const int sms = num_sms();
+  int ks = std::max(1, std::min(p.nsteps, sms / std::max(p.nrb, 1)));
+  while (ks < p.nsteps && ceil_div(p.nsteps, ks) > kMaxHold && p.nrb * (ks + 1) <= 2 * sms) ++ks;
   p.ksplit = ks;
-  p.nparts = p.nrb * p.ksplit;
+  finish_act_plan(p);
   return p;
 }
 
 size_t act_scratch_bytes(const ActPlan& p) {
-  size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(p.nparts) * 4, 256));
+  size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));
+  b += 256;  // grid barrier words
   if (p.rank_pad > 0)
     b += static_cast<size_t>(round_up(static_cast<int64_t>(p.ksplit) * p.B * p.rank_pad * 4, 256));
   return b + 256;
@@ -513,7 +574,8 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   if (p.B == 0) return cudaSuccess;
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
   Carver cv(scratch, ~size_t(0));
-  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(p.nparts) * 4));
+  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));
+  unsigned* sync = static_cast<unsigned*>(cv.take(256));
   float* ws_down =
       has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4))
              : nullptr;
@@ -521,7 +583,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   const CUtensorMapDataType cdt =
       xdt == SVDQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUtensorMap tm_x, tm_ld;
-  if (!make_tmap_2d(&tm_x, x, cdt, esz, p.M, p.B, ldx, p.tile_k, kRowsPerBlock, true)) {
+  if (!make_tmap_2d(&tm_x, x, cdt, esz, p.M, p.B, ldx, p.tile_k, kRows, true)) {
     *bad_args = true;
     return cudaSuccess;
   }
@@ -533,69 +595,53 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   } else {
     tm_ld = tm_x;
   }
-  unsigned* status = device_status_word();
-  const int stage_bytes = kTileBytes + (has_ld ? p.rank_pad * 128 : 0);
-  const size_t smem = static_cast<size_t>(kActStages) * stage_bytes + 1024;
-  dim3 grid(p.nrb, p.ksplit);
-  cudaError_t err;
+  cudaError_t err = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), stream);
+  if (err != cudaSuccess) return err;
+  ActArgs a{};
+  a.B = static_cast<int>(p.B);
+  a.M = static_cast<int>(p.M);
+  a.ldx = ldx;
+  a.nsteps = p.nsteps;
+  a.ksplit = p.ksplit;
+  a.nrb = p.nrb;
+  a.nunits = p.nunits;
+  a.rank_pad = has_ld ? p.rank_pad : 0;
+  a.has_ld = has_ld ? 1 : 0;
+  a.hold = p.hold;
+  a.xbuf = p.xbuf;
+  a.fmt_kind = fmt.kind;
+  a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
+  a.x = x;
+  a.scale = scale;
+  a.gs_given = fmt.kind == SVDQ_KIND_NVFP4 ? act_global_scale : nullptr;
+  a.gs_w = fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr;
+  a.ws_down = ws_down;
+  a.ws_max = ws_max;
+  a.sync = sync;
+  a.codes = codes;
+  a.sf = static_cast<uint8_t*>(sf);
+  a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
+  a.act_scale = act_scale;
+  a.status = device_status_word();
+  // without the down factor the launch needs no ld ring (plan keeps its grid)
+  ActPlan q = p;
+  if (!has_ld) q.rank_pad = 0;
+  const size_t smem = smem_for(q, p.xbuf);
+  void* args[] = {&tm_x, &tm_ld, &a};
   if (xdt == SVDQ_BF16) {
-    err = cudaFuncSetAttribute(act_stats_kernel<__nv_bfloat16>,
+    err = cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    act_stats_kernel<__nv_bfloat16><<<grid, kActThreads, smem, stream>>>(
-        tm_x, tm_ld, scale, static_cast<int>(p.B), static_cast<int>(p.M), p.nsteps, p.ksplit,
-        p.rank_pad, has_ld ? 1 : 0, ws_down, ws_max, status);
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_fused_kernel<__nv_bfloat16>),
+                                      dim3(p.grid), dim3(kThreads), args, smem, stream);
   } else {
-    err = cudaFuncSetAttribute(act_stats_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(act_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    act_stats_kernel<float><<<grid, kActThreads, smem, stream>>>(
-        tm_x, tm_ld, scale, static_cast<int>(p.B), static_cast<int>(p.M), p.nsteps, p.ksplit,
-        p.rank_pad, has_ld ? 1 : 0, ws_down, ws_max, status);
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_fused_kernel<float>), dim3(p.grid),
+                                      dim3(kThreads), args, smem, stream);
   }
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-
-  // quantise: 32 column chunks per block along x, a band of rows along y, sized
-  // for about eight blocks per SM
-  const int chunk = fmt.kind == SVDQ_KIND_INT ? 8 : 16;
-  const int gx = static_cast<int>(ceil_div(p.M / chunk, 32));
-  const int64_t want_blocks = static_cast<int64_t>(num_sms()) * 8;
-  const int64_t rows_step = 8 * (fmt.kind == SVDQ_KIND_INT ? kRowsPerThread : kRowsPerThreadF4);
-  int64_t rows_per_block =
-      round_up(std::max<int64_t>(1, ceil_div(p.B * gx, want_blocks)), rows_step);
-  const int gy = static_cast<int>(ceil_div(p.B, rows_per_block));
-  dim3 qgrid(gx, gy);
-  const int threads = 256;
-  __nv_bfloat16* down_bf = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
-  const int rp = has_ld ? p.rank_pad : 0;
-  const int rpb = static_cast<int>(rows_per_block);
-  if (fmt.kind == SVDQ_KIND_INT) {
-    const int qmax = (1 << (fmt.bits - 1)) - 1;
-    if (xdt == SVDQ_BF16)
-      act_quant_int_kernel<__nv_bfloat16><<<qgrid, threads, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(x), ldx, scale, static_cast<int>(p.B),
-          static_cast<int>(p.M), qmax, rpb, ws_max, p.nparts, ws_down, p.ksplit, rp,
-          static_cast<int8_t*>(codes), down_bf, act_scale);
-    else
-      act_quant_int_kernel<float><<<qgrid, threads, 0, stream>>>(
-          static_cast<const float*>(x), ldx, scale, static_cast<int>(p.B), static_cast<int>(p.M),
-          qmax, rpb, ws_max, p.nparts, ws_down, p.ksplit, rp, static_cast<int8_t*>(codes),
-          down_bf, act_scale);
-  } else {
-    if (xdt == SVDQ_BF16)
-      act_quant_nvfp4_kernel<__nv_bfloat16><<<qgrid, threads, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(x), ldx, scale, static_cast<int>(p.B),
-          static_cast<int>(p.M), rpb, ws_max, p.nparts, act_global_scale, w_global_scale,
-          ws_down, p.ksplit, rp, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf,
-          act_scale);
-    else
-      act_quant_nvfp4_kernel<float><<<qgrid, threads, 0, stream>>>(
-          static_cast<const float*>(x), ldx, scale, static_cast<int>(p.B), static_cast<int>(p.M),
-          rpb, ws_max, p.nparts, act_global_scale, w_global_scale, ws_down, p.ksplit, rp,
-          static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), down_bf, act_scale);
-  }
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace svdq

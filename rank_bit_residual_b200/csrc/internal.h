@@ -46,13 +46,21 @@ struct Carver {
 struct ActPlan {
   int64_t B, M;
   int32_t rank_pad;
+  bool bf16;       // x is bf16 (else fp32)
   int tile_k;      // elements per 128-byte K tile (64 bf16 / 32 fp32)
   int nrb;         // row blocks of 128
   int nsteps;      // K tiles
-  int ksplit;      // CTAs along K
-  int nparts;      // partial maxima written (nrb * ksplit)
+  int ksplit;      // K ranges per row block
+  int nunits;      // nrb * ksplit work units
+  int hold;        // 1: each unit keeps its x tiles in shared memory for phase 2
+  int xbuf;        // x tile buffers per CTA
+  int grid;        // CTAs of the cooperative launch (all resident)
+  int nparts;      // partial maxima written (one per CTA)
+  size_t smem;     // dynamic shared memory per CTA
 };
 ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt);
+// Recompute the derived fields after changing ksplit.
+void finish_act_plan(ActPlan& p);
 size_t act_scratch_bytes(const ActPlan& p);
 
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,

@@ -175,46 +175,6 @@ __global__ void __launch_bounds__(256) sum_parts_kernel(const float* __restrict_
   }
 }
 
-// --------------------------------------------------------- grid barrier
-// All CTAs of a cooperative launch arrive on a monotone counter; the wait is
-// bounded and any CTA that gives up raises a global abort seen by the others.
-struct GridSync {
-  unsigned* counter;
-  unsigned* abort_flag;
-  unsigned* status;
-  unsigned epoch;
-};
-
-__device__ bool grid_sync(GridSync& gs, volatile int* abort_sh) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    ++gs.epoch;
-    __threadfence();
-    atomicAdd(gs.counter, 1u);
-    const unsigned target = gs.epoch * gridDim.x;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-      unsigned v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gs.counter) : "memory");
-      if (v >= target) break;
-      if (*reinterpret_cast<volatile unsigned*>(gs.abort_flag)) {
-        *abort_sh = 1;
-        break;
-      }
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        record_status(gs.status, kStatusTimeout);
-        atomicExch(gs.abort_flag, 1u);
-        *abort_sh = 1;
-        break;
-      }
-      __nanosleep(64);
-    }
-    __threadfence();
-  }
-  __syncthreads();
-  return *abort_sh == 0;
-}
-
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
