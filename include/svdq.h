@@ -180,6 +180,32 @@ svdq_status svdq_quantize_act_workspace_size(int64_t B, int64_t M, svdq_fmt fmt,
                                              int32_t rank_pad, size_t* bytes);
 
 /*
+ * svdq_quantize_act_noalloc - svdq_quantize_act with no workspace argument. The
+ * pages have no counterpart; it is here for callers that cannot allocate device
+ * memory: code running inside a host runtime that owns all device memory and
+ * offers no allocator on its request path (a static memory plan of an inference
+ * server, the plugin interface of another engine). Neither the caller nor the
+ * library calls cudaMalloc; the caller still passes inputs and outputs, with the
+ * layouts of svdq_quantize_act.
+ *
+ * Scratch lives in one fixed 8 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits. The first
+ * call on a device looks up the array's address on that device; make that
+ * call before any stream capture. All calls share the array and it keeps the
+ * last call's contents: every scratch word a call reads is written by that call
+ * first, so nothing needs clearing, but calls that overlap on the GPU (other
+ * streams or other host threads) race on it. Shapes whose scratch does not fit
+ * in 8 MiB even with the K split reduced - B * rank_pad of 2^21 or more
+ * - return SVDQ_EWORKSPACE and launch nothing.
+ */
+svdq_status svdq_quantize_act_noalloc(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
+                                      int64_t ldx, const float* scale, svdq_fmt fmt,
+                                      const float* act_global_scale,
+                                      const float* w_global_scale, const void* ld,
+                                      int32_t rank_pad, void* codes, void* sf, float* act_scale,
+                                      void* down, svdq_stream_t stream);
+
+/*
  * svdq_linear - the operator ("svdquant_linear" of both pages):
  *   Y = x ld^T lu^T + alpha * (Q(X_hat) . Q(R)) [+ bias]
  * with alpha = s_x * s_w (INT) or 1 / (gs_x * gs_w) (NVFP4). Runs the fused

@@ -62,6 +62,8 @@ _SIGS = {
     "svdq_residual_product_i32": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i64, c_vp, c_i64, c_vp]),
     "svdq_residual_linear": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
                                      c_vp, c_i32, c_i64, c_vp]),
+    "svdq_quantize_act_noalloc": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, SvdqFmt, c_vp, c_vp,
+                                          c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "svdq_check_status": (c_i32, [c_vp]),
     "svdq_selftest_wait_timeout": (c_i32, [c_i64, c_vp]),
 }
@@ -336,6 +338,33 @@ def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Opti
     return bufs
 
 
+def svdq_quantize_act_noalloc(x: torch.Tensor, scale: torch.Tensor, fmt="int4",
+                              ld: Optional[torch.Tensor] = None,
+                              act_global_scale: Optional[torch.Tensor] = None,
+                              w_global_scale: Optional[torch.Tensor] = None):
+    """The activation pass through svdq_quantize_act_noalloc.
+
+    For callers whose runtime gives them no way to allocate device memory on the
+    request path: the library passes no workspace and allocates nothing, using a
+    fixed scratch array of its own (8 MiB per GPU, shared by all calls, so calls
+    that overlap on the GPU must not be issued). Only the outputs are allocated
+    here, on the caller's side. Returns (codes, sf or None, act_scale, down or None)
+    like svdq_quantize_act.
+    """
+    lib = load_library()
+    _require_cuda(x, scale)
+    f = parse_fmt(fmt)
+    x = _rows_ready(x)
+    B, M = x.shape
+    rp = ld.shape[0] if ld is not None else 0
+    codes, sf, act_scale, down = _act_buffers(B, M, f, rp, x.device)
+    _check(lib.svdq_quantize_act_noalloc(_ptr(x), _dt(x), B, M, x.stride(0), _ptr(scale.contiguous()), f,
+                                         _ptr(act_global_scale), _ptr(w_global_scale), _ptr(ld), rp,
+                                         _ptr(codes), _ptr(sf), _ptr(act_scale), _ptr(down), _stream()),
+           "svdq_quantize_act_noalloc")
+    return codes, sf, act_scale, down
+
+
 class LinearWorkspace:
     """Reusable scratch for svdq_linear (one per stream in flight)."""
 
@@ -422,7 +451,8 @@ def svdq_selftest_wait_timeout(limit_us: int = 1000) -> int:
 
 
 __all__ = [
-    "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_residual", "svdq_linear",
+    "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_act_noalloc",
+    "svdq_quantize_residual", "svdq_linear",
     "svdq_residual_product_i32", "svdq_residual_linear", "svdq_check_status", "svdq_selftest_wait_timeout",
     "PreparedWeight", "LinearWorkspace", "allocate_weight", "weight_from_buffers",
     "weight_buffer_sizes", "load_library", "header_functions", "parse_fmt",

@@ -1,0 +1,94 @@
+// noalloc.cu - svdq_quantize_act_noalloc: the activation pass with its scratch
+// in a fixed device array that lives inside this library, for callers that
+// cannot hand the library a workspace.
+//
+// Who needs it: code that runs inside a host runtime which owns every byte of
+// device memory and exposes no allocator on the request path (static memory
+// plans of inference servers, plugin interfaces of other engines, tightly
+// budgeted real-time loops), so neither the caller nor this library may call
+// cudaMalloc there. The caller still provides the inputs and outputs.
+//
+// The array is a file-scope __device__ variable, so every GPU that loads the
+// library holds kNoallocScratchBytes of it until the process exits. Its device
+// address is looked up once per device (cudaGetSymbolAddress, with that device
+// current) on the first call made on that device; make that first call before
+// any stream capture. All calls share the one array and it keeps the previous
+// call's contents: the kernels overwrite every scratch word they read, so
+// nothing needs clearing, but calls whose kernels overlap on the GPU (two
+// streams, or two host threads) race on it.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+
+namespace svdq {
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDev = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDev] = {};
+
+// Device address of the array on the current device (nullptr on failure).
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" svdq_status svdq_quantize_act_noalloc(
+    const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx, const float* scale,
+    svdq_fmt fmt, const float* act_global_scale, const float* w_global_scale, const void* ld,
+    int32_t rank_pad, void* codes, void* sf, float* act_scale, void* down,
+    svdq_stream_t stream) {
+  if (B < 0 || M <= 0 || (x_dtype != SVDQ_BF16 && x_dtype != SVDQ_F32)) return SVDQ_EINVAL;
+  const bool int_fmt = fmt.kind == SVDQ_KIND_INT && fmt.bits >= 2 && fmt.bits <= 8;
+  const bool f4_fmt = fmt.kind == SVDQ_KIND_NVFP4 && fmt.bits == 4;
+  if (!int_fmt && !f4_fmt) return SVDQ_EINVAL;
+  if (!scale || rank_pad < 0 || rank_pad % 16 || rank_pad > 256) return SVDQ_EINVAL;
+  if (B == 0) return SVDQ_OK;
+  if (!x || ldx < M || !codes || !act_scale || (f4_fmt && !sf)) return SVDQ_EINVAL;
+  if (ld && rank_pad > 0 && !down) return SVDQ_EINVAL;
+  const int esz = x_dtype == SVDQ_BF16 ? 2 : 4;
+  if (M % 32 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) || (ldx * esz) % 16 ||
+      (reinterpret_cast<uintptr_t>(scale) & 15) || B > (int64_t(1) << 30))
+    return SVDQ_EUNSUPPORTED;
+
+  // Same launch plan as svdq_quantize_act, with fewer K splits if that is what
+  // it takes to fit the fixed array; beyond that the shape is refused.
+  const int32_t rp = (ld != nullptr) ? rank_pad : 0;
+  ActPlan p = plan_act(B, M, rp, x_dtype);
+  while (act_scratch_bytes(p) > kNoallocScratchBytes && p.ksplit > 1) {
+    p.ksplit = std::max(1, p.ksplit / 2);
+    finish_act_plan(p);
+  }
+  if (act_scratch_bytes(p) > kNoallocScratchBytes) return SVDQ_EWORKSPACE;
+
+  void* scratch = noalloc_scratch();
+  if (!scratch) return SVDQ_ECUDA;
+  bool bad = false;
+  const cudaError_t e =
+      launch_act(p, x, x_dtype, ldx, scale, fmt, act_global_scale,
+                 f4_fmt ? w_global_scale : nullptr, rp > 0 ? ld : nullptr, codes, sf, act_scale,
+                 down, scratch, reinterpret_cast<cudaStream_t>(stream), &bad);
+  if (bad) return SVDQ_EUNSUPPORTED;
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;
+}
