@@ -34,10 +34,15 @@ namespace svdq {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kWorkWarps = 16;
+constexpr int kWork = 32 * kWorkWarps;      // threads for column maxima, codes and down
+constexpr int kThreads = kWork + 64;        // + a TMA warp and an MMA warp
+constexpr int kTmaWarp = kWorkWarps;
+constexpr int kMmaWarp = kWorkWarps + 1;
 constexpr int kRows = 128;                  // rows per unit (MMA M)
 constexpr int kTileBytes = kRows * 128;     // one 128 x 128-byte x tile
-constexpr int kRing = 4;                    // ring depth for ld tiles (and x tiles when not held)
+constexpr int kXRing = 4;                   // x tile buffers when the tiles are not held
+constexpr int kLdRing = 6;                  // ld tile slots
 constexpr int kMaxHold = 12;                // x tiles a unit may keep in shared memory
 constexpr int kSmemBudget = 224 * 1024;
 
@@ -53,6 +58,7 @@ struct ActArgs {
   const float* scale;
   const float* gs_given;
   const float* gs_w;
+  const void* ld;   // [rank_pad][M], x's dtype
   float* ws_down;   // [ksplit][B][rank_pad]
   float* ws_max;    // [gridDim.x]
   unsigned* sync;   // [0] barrier counter, [1] abort flag (zeroed before launch)
@@ -117,7 +123,8 @@ __device__ __forceinline__ void unpack16(const uint4 u, float* v) {
   }
 }
 
-// Column maxima of |x| over a 128 x 128-byte swizzled tile. Thread t owns the
+// Column maxima of |x| over a 128 x 128-byte swizzled tile (work threads only,
+// t < kWork). Thread t owns the
 // logical 16-byte chunk c = t % 8 of rows t/8 and t/8 + 64; it folds
 // fl(colmax r_k) of its chunk's columns into `run` (rcp: reciprocals of the
 // tile's columns, 0 past M).
@@ -129,8 +136,8 @@ __device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* r
   const int p = c ^ (rg & 7);  // rows rg + 64 i share rg & 7
   uint32_t mx[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int i = 0; i < kRows / (kThreads / 8); ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + (rg + (kThreads / 8) * i) * 128 + p * 16);
+  for (int i = 0; i < kRows / (kWork / 8); ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + (rg + (kWork / 8) * i) * 128 + p * 16);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -154,44 +161,163 @@ __device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* r
 }
 
 // -------------------------------------------------------------- the kernel
+// Barrier among the work warps only (the TMA and MMA warps run their own loops).
+__device__ __forceinline__ void work_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kWork) : "memory");
+}
+
+// Grid-wide barrier of the work warps of every CTA (see grid_sync; the block
+// barriers are the work warps' own). counter and abort_flag are zeroed before
+// the launch.
+__device__ __forceinline__ bool grid_sync_work(unsigned* counter, unsigned* abort_flag, unsigned* status,
+                                               volatile int* abort_sh) {
+  work_sync();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+    const unsigned target = gridDim.x;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+      if (v >= target) break;
+      if (*reinterpret_cast<volatile unsigned*>(abort_flag)) {
+        *abort_sh = 1;
+        break;
+      }
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_status(status, kStatusTimeout);
+        atomicExch(abort_flag, 1u);
+        *abort_sh = 1;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  work_sync();
+  return *abort_sh == 0;
+}
+
+// Eight consecutive elements of x (16 bytes of bf16, or 32 of fp32) from a held
+// swizzled tile row or from global memory; cl: column within the unit, a
+// multiple of 8.
+template <typename TIn>
+__device__ __forceinline__ void load8(const uint8_t* xbuf, bool hold, const void* x, int64_t ldx,
+                                      int64_t row, int64_t col0, int r, int cl, uint4 (&u)[2]) {
+  constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));
+  constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn));
+  constexpr int kChunks = 8 / kPerChunk;   // 1 (bf16) or 2 (fp32)
+  if (hold) {
+    const int t = cl / kTileK, c = (cl % kTileK) / kPerChunk;
+    const uint8_t* base = xbuf + static_cast<size_t>(t) * kTileBytes + r * 128;
+#pragma unroll
+    for (int h = 0; h < kChunks; ++h) u[h] = *reinterpret_cast<const uint4*>(base + (((c + h) ^ (r & 7)) << 4));
+  } else {
+    const uint4* g = reinterpret_cast<const uint4*>(static_cast<const TIn*>(x) + row * ldx + col0 + cl);
+#pragma unroll
+    for (int h = 0; h < kChunks; ++h) u[h] = __ldg(g + h);
+  }
+}
+
+template <typename TIn>
+__device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
+  if constexpr (sizeof(TIn) == 2) {
+    unpack16<TIn>(u[0], v);
+  } else {
+    unpack16<TIn>(u[0], v);
+    unpack16<TIn>(u[1], v + 4);
+  }
+}
+
+// INT codes of 8 elements: rint(fl(x c_k)), packed as 8 bytes. Adding
+// 1.5 * 2^23 rounds an fp32 value below 2^22 in magnitude to the nearest
+// integer, ties to even, and leaves that integer in the low bits of the sum,
+// so the low byte of the sum is the two's-complement code. The clamp to
+// [-qmax, qmax] of the definition is omitted: with s = fl(m / qmax) and
+// c_k = fl(fl(1 / scale_k) fl(1 / s)), every |fl(x c_k)| is at most
+// qmax (1 + 6 * 2^-24) < qmax + 1/2, so no code can leave the range.
+__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8]) {
+  uint32_t f[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) f[j] = __float_as_uint(__fadd_rn(__fmul_rn(v[j], ck[j]), 12582912.0f));
+  const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(f[4], f[5], 0x0040), __byte_perm(f[6], f[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most n of this thread's copy groups are still in flight.
+__device__ __forceinline__ void cp_async_wait(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+  }
+}
+
+// Warp roles: warps 0-15 ("work") take the column maxima in phase 1 and write
+// the codes and the down factor in phase 2; warp 16 loads the x tiles by TMA
+// (lane 0); warp 17 copies the ld tiles with cp.async (all lanes: a path apart
+// from the TMA queue, so the small ld tiles never wait behind the x tiles) and
+// issues the down-projection MMAs (lane 0). No block-wide barrier separates the
+// K steps: the work warps follow the x tiles as they land, and the MMA chain
+// runs on its own. The MMA warp issues one throwaway MMA first: the first
+// tcgen05.mma a kernel issues takes microseconds longer than the ones after
+// it, and this way that start-up overlaps the first loads.
 template <typename TIn>
 __global__ void __launch_bounds__(kThreads, 1)
-    act_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_ld,
-                     const ActArgs a) {
+    act_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const ActArgs a) {
   constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));   // elements per 128-byte row
   constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn)); // elements per 16 bytes
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t xfull[kMaxHold];
-  __shared__ __align__(8) uint64_t ldfull[kRing];
-  __shared__ __align__(8) uint64_t mmadone[kRing];
-  __shared__ __align__(8) uint64_t final_bar;
+  __shared__ __align__(8) uint64_t xempty[kMaxHold];
+  __shared__ __align__(8) uint64_t ld_free;
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ __align__(8) uint64_t tmem_free;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[kWorkWarps];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp >= kWorkWarps;   // the TMA or the MMA warp
   const int ld_bytes = a.rank_pad * 128;
   uint8_t* xbuf = smem;                                               // a.xbuf tiles
-  uint8_t* ldbuf = smem + static_cast<size_t>(a.xbuf) * kTileBytes;   // kRing ld tiles
-  float* rcp = reinterpret_cast<float*>(ldbuf + (a.has_ld ? kRing * ld_bytes : 0));
+  uint8_t* ldbuf = smem + static_cast<size_t>(a.xbuf) * kTileBytes;   // kLdRing ld tiles
+  float* rcp = reinterpret_cast<float*>(ldbuf + (a.has_ld ? kLdRing * ld_bytes : 0));
   const uint32_t tcols = pow2_cols(a.rank_pad);
   unsigned* status = a.status;
 
-  if (tid == 0) {
-    for (int s = 0; s < kMaxHold; ++s) mbar_init(&xfull[s], 1);
-    for (int s = 0; s < kRing; ++s) {
-      mbar_init(&ldfull[s], 1);
-      mbar_init(&mmadone[s], 1);
+  auto unit_range = [&](int unit, int& m0, int& k_lo, int& n) {
+    const int rb = unit % a.nrb, sp = unit / a.nrb;
+    m0 = rb * kRows;
+    k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
+    n = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit) - k_lo;
+  };
+
+  if (tid == kWork) {
+    for (int s = 0; s < kMaxHold; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], kWorkWarps + (a.has_ld ? 1 : 0));
     }
-    mbar_init(&final_bar, 1);
+    mbar_init(&ld_free, 1);
+    mbar_init(&mma_done, 1);
+    mbar_init(&tmem_free, 4);
     fence_mbar_init();
     abort_sh = 0;
     tma_prefetch_desc(&tm_x);
-    if (a.has_ld) tma_prefetch_desc(&tm_ld);
   }
-  if (a.has_ld && warp == 0) {
+  if (warp == kMmaWarp && a.has_ld) {
     tmem_alloc(&tmem_base_sh, tcols);
     tmem_relinquish();
   }
@@ -199,98 +325,153 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = a.has_ld ? tmem_base_sh : 0u;
-  const uint32_t idesc = sizeof(TIn) == 2 ? idesc_bf16(128, a.rank_pad) : idesc_tf32(128, a.rank_pad);
-
-  // barrier uses so far (phase parities carry across units)
-  uint32_t xuse[kMaxHold] = {};
-  uint32_t lduse = 0;
-  uint32_t final_use = 0;
   float run = 0.0f;
   bool ok = true;
 
   // ================================================================ phase 1
-  for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
-    const int rb = unit % a.nrb, sp = unit / a.nrb;
-    const int m0 = rb * kRows;
-    const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
-    const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
-    const int n = k_hi - k_lo;
-    for (int j = tid; j < n * kTileK; j += kThreads) {
-      const int col = k_lo * kTileK + j;
-      rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
+  // x steps flow through the buffers as one ring over all of this CTA's units:
+  // step G + i uses buffer (G + i) % xbuf in its use (G + i) / xbuf (counters
+  // in registers: an indexed array would live in local memory)
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      uint32_t G = 0;   // x steps of the previous units
+      bool pok = true;
+      for (int unit = blockIdx.x; unit < a.nunits && pok; unit += gridDim.x) {
+        int m0, k_lo, n;
+        unit_range(unit, m0, k_lo, n);
+        for (int i = 0; i < n && pok; ++i) {
+          const uint32_t gs = G + i;
+          const uint32_t b = gs % a.xbuf, use = gs / a.xbuf;
+          if (use > 0)  // the previous tile in this buffer is fully read
+            pok = mbar_wait(&xempty[b], (use - 1) & 1, status, &abort_sh);
+          if (!pok) break;
+          mbar_arrive_expect_tx(&xfull[b], kTileBytes);
+          tma_load_2d(xbuf + static_cast<size_t>(b) * kTileBytes, &tm_x, &xfull[b], (k_lo + i) * kTileK, m0);
+        }
+        G += n;
+      }
+      if (!pok) {
+        abort_sh = 1;
+        // let loads already issued land before the block moves on (the loads
+        // of the last xbuf steps of the ring, at most)
+        for (uint32_t gs = G > static_cast<uint32_t>(a.xbuf) ? G - a.xbuf : 0u; gs < G; ++gs)
+          mbar_wait(&xfull[gs % a.xbuf], (gs / a.xbuf) & 1, status, nullptr, 1000000ull);
+      }
     }
-    __syncthreads();
-    const uint32_t ld0 = lduse;
-    auto issue_x = [&](int i) {
-      const int b = i % a.xbuf;
-      mbar_arrive_expect_tx(&xfull[b], kTileBytes);
-      tma_load_2d(xbuf + static_cast<size_t>(b) * kTileBytes, &tm_x, &xfull[b], (k_lo + i) * kTileK, m0);
-    };
-    auto issue_ld = [&](int i) {
-      const uint32_t q = (ld0 + i) % kRing;
-      mbar_arrive_expect_tx(&ldfull[q], ld_bytes);
-      tma_load_2d(ldbuf + static_cast<size_t>(q) * ld_bytes, &tm_ld, &ldfull[q], (k_lo + i) * kTileK, 0);
-    };
-    if (tid == 0 && ok) {
-      for (int i = 0; i < min(n, a.xbuf); ++i) issue_x(i);
-      if (a.has_ld)
-        for (int i = 0; i < min(n, kRing); ++i) issue_ld(i);
-    }
-    // Step i reads x buffer i % xbuf and ld slot (ld0 + i) % kRing. At step i,
-    // thread 0 refills the buffers step i - 1 used (its MMA was issued a step
-    // ago, so the wait for it is normally already satisfied).
-    for (int i = 0; i < n; ++i) {
-      const int b = i % a.xbuf;
-      const uint32_t q = (ld0 + i) % kRing;
-      ok = ok && mbar_wait(&xfull[b], xuse[b] & 1, status, &abort_sh);
-      ++xuse[b];
-      if (a.has_ld && tid == 0) {
-        ok = ok && mbar_wait(&ldfull[q], ((ld0 + i) / kRing) & 1, status, &abort_sh);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(xbuf + static_cast<size_t>(b) * kTileBytes);
-          const uint32_t b0 = smem_u32(ldbuf + static_cast<size_t>(q) * ld_bytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a0 + 32 * kk);
-            const uint64_t bd = smem_desc_sw128(b0 + 32 * kk);
-            if (sizeof(TIn) == 2)
-              mma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-            else
-              mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+  } else if (warp == kMmaWarp) {
+    if (a.has_ld) {
+      uint32_t G = 0;        // x steps of the previous units
+      uint32_t nbatch = 0;   // ld batches whose MMAs were committed to ld_free
+      bool pok = true;
+      // ld tiles of K tiles k_lo + j0 .. + cnt - 1 into slots 0 .. cnt - 1, one
+      // copy group per lane; ld is [rank_pad, M] row-major, columns past M are
+      // filled with zeros. The slots are free once the previous batch's MMAs
+      // are done.
+      auto copy_batch = [&](int k_lo, int j0, int cnt) {
+        if (nbatch > 0) pok = mbar_wait_warp(&ld_free, (nbatch - 1) & 1, status, &abort_sh) && pok;
+        const TIn* ld = static_cast<const TIn*>(a.ld);
+        for (int t = 0; t < cnt; ++t) {
+          uint8_t* dst = ldbuf + static_cast<size_t>(t) * ld_bytes;
+          for (int c = lane; c < a.rank_pad * 8; c += 32) {
+            const int r = c >> 3, cc = c & 7;
+            const int col = (k_lo + j0 + t) * kTileK + cc * kPerChunk;
+            const bool in = col < a.M;
+            cp_async16(smem_u32(dst + r * 128 + ((cc ^ (r & 7)) << 4)),
+                       in ? static_cast<const void*>(ld + static_cast<int64_t>(r) * a.M + col) : a.ld,
+                       in ? 16u : 0u);
           }
-          mma_commit(&mmadone[q]);
+        }
+        cp_async_commit();
+      };
+      const uint32_t idesc = sizeof(TIn) == 2 ? idesc_bf16(128, a.rank_pad) : idesc_tf32(128, a.rank_pad);
+      if (lane == 0) {
+        // throwaway MMA (its result is overwritten by the first real one)
+        const uint64_t ad = smem_desc_sw128(smem_u32(xbuf)), bd = smem_desc_sw128(smem_u32(ldbuf));
+        if (sizeof(TIn) == 2)
+          mma_f16(tmem, ad, bd, idesc, 0u);
+        else
+          mma_tf32(tmem, ad, bd, idesc, 0u);
+      }
+      __syncwarp();
+      uint32_t ucount = 0;
+      for (int unit = blockIdx.x; unit < a.nunits && pok; unit += gridDim.x, ++ucount) {
+        int m0, k_lo, n;
+        unit_range(unit, m0, k_lo, n);
+        for (int j0 = 0; j0 < n && pok; j0 += kLdRing) {
+          const int cnt = min(kLdRing, n - j0);
+          copy_batch(k_lo, j0, cnt);
+          if (lane == 0 && ucount > 0 && j0 == 0)  // the work warps have read the previous unit's accumulator
+            pok = pok && mbar_wait(&tmem_free, (ucount - 1) & 1, status, &abort_sh);
+          cp_async_wait(0);  // this lane's copies have landed
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            for (int t = 0; t < cnt && pok; ++t) {
+              const int i = j0 + t;
+              const uint32_t b = (G + i) % a.xbuf;
+              pok = mbar_wait(&xfull[b], ((G + i) / a.xbuf) & 1, status, &abort_sh);
+              if (!pok) break;
+              tc_fence_after();
+              const uint32_t a0 = smem_u32(xbuf + static_cast<size_t>(b) * kTileBytes);
+              const uint32_t b0 = smem_u32(ldbuf + static_cast<size_t>(t) * ld_bytes);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc_sw128(a0 + 32 * kk);
+                const uint64_t bd = smem_desc_sw128(b0 + 32 * kk);
+                if (sizeof(TIn) == 2)
+                  mma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                else
+                  mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+              }
+              if (!a.hold) mma_commit(&xempty[b]);
+            }
+            if (pok) mma_commit(&ld_free);
+          }
+          ++nbatch;
+          pok = __shfl_sync(0xffffffffu, pok ? 1 : 0, 0) != 0;
+        }
+        if (lane == 0 && pok) mma_commit(&mma_done);
+        G += n;
+      }
+      cp_async_wait(0);
+      if (lane == 0 && !pok) abort_sh = 1;
+    }
+  } else {
+    uint32_t G = 0;   // x steps of the previous units (the same ring as the producer's)
+    uint32_t ucount = 0;
+    for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x, ++ucount) {
+      int m0, k_lo, n;
+      unit_range(unit, m0, k_lo, n);
+      work_sync();  // the previous unit's reciprocals are no longer read
+      for (int j = tid; j < n * kTileK; j += kWork) {
+        const int col = k_lo * kTileK + j;
+        rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
+      }
+      work_sync();
+      for (int i = 0; i < n; ++i) {
+        const uint32_t b = (G + i) % a.xbuf;
+        ok = mbar_wait_warp(&xfull[b], ((G + i) / a.xbuf) & 1, status, &abort_sh) && ok;
+        if (ok) run = tile_absmax<TIn>(xbuf + static_cast<size_t>(b) * kTileBytes, rcp + i * kTileK, run);
+        if (!a.hold) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xempty[b]);
         }
       }
-      if (ok) run = tile_absmax<TIn>(xbuf + static_cast<size_t>(b) * kTileBytes, rcp + i * kTileK, run);
-      __syncthreads();
-      if (tid == 0 && ok && i >= 1) {
-        const int jl = i - 1 + kRing;     // ld step that takes over slot of step i - 1
-        const int jx = i - 1 + a.xbuf;    // x step that takes over buffer of step i - 1
-        const bool need_ld = a.has_ld && jl < n;
-        const bool need_x = !a.hold && jx < n;
-        if (a.has_ld && (need_ld || need_x))
-          ok = mbar_wait(&mmadone[(ld0 + i - 1) % kRing], ((ld0 + i - 1) / kRing) & 1, status,
-                         &abort_sh);
-        if (ok && need_ld) issue_ld(jl);
-        if (ok && need_x) issue_x(jx);
-      }
-    }
-    if (a.has_ld) lduse += n;
-    if (a.has_ld) {
-      if (tid == 0) mma_commit(&final_bar);
-      const bool fin = mbar_wait(&final_bar, final_use & 1, status, nullptr);
-      ++final_use;
-      tc_fence_after();
-      // TMEM lane = row; warps 0-3 cover the 128 lanes (one lane quarter each)
-      if (warp < 4) {
+      if (a.has_ld && !a.hold && warp < 4) {
+        // ring mode: drain the unit's accumulator before the next unit's MMAs
+        // (held tiles: one unit per CTA, drained after the codes in phase 2)
+        // TMEM lane = row; warps 0-3 cover the 128 lanes (one lane quarter each)
+        const bool fin = mbar_wait_warp(&mma_done, ucount & 1, status, &abort_sh) && ok;
+        tc_fence_after();
         const int row = m0 + warp * 32 + lane;
+        const int sp = unit / a.nrb;
         float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * a.rank_pad;
         for (int c0 = 0; c0 < a.rank_pad; c0 += 32) {
           uint32_t v[32];
+          __syncwarp();
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-          tmem_ld_wait();
-          if (fin && ok && row < a.B) {
+          tmem_ld_wait_regs(v);
+          if (fin && row < a.B) {
             const int cnt = min(32, a.rank_pad - c0);
             for (int j = 0; j < cnt; j += 4)
               *reinterpret_cast<float4*>(dst + c0 + j) =
@@ -298,42 +479,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                               __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tmem_free);
+        ok = ok && fin;
       }
-      tc_fence_before();
-      __syncthreads();
+      G += n;
     }
-  }
-  // a failed wait: let loads already issued land before the block moves on
-  if (tid == 0 && !ok) {
-    for (int s = 0; s < min(a.xbuf, kMaxHold); ++s)
-      mbar_wait(&xfull[s], xuse[s] & 1, status, nullptr, 1000000ull);
-  }
-  // per-CTA maximum -> ws_max[blockIdx.x]
+    // per-CTA maximum -> ws_max[blockIdx.x]
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-  if (lane == 0) red[warp] = run;
-  __syncthreads();
-  if (tid == 0) {
-    float m = red[0];
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-    a.ws_max[blockIdx.x] = m;
+    for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
+    if (lane == 0) red[warp] = run;
+    work_sync();
+    if (tid == 0) {
+      float m = red[0];
+      for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
+      a.ws_max[blockIdx.x] = m;
+    }
   }
 
   // ======================================================== grid barrier
-  GridSync gs{a.sync, a.sync + 1, status, 0};
-  ok = grid_sync(gs, &abort_sh) && ok;
+  // (work warps only: the MMA warp's chain may still be running, it is
+  // collected after the codes)
+  if (!producer) ok = grid_sync_work(a.sync, a.sync + 1, status, &abort_sh) && ok;
 
   // ================================================================ phase 2
-  if (ok) {
+  if (ok && !producer) {
     float m = 0.0f;
-    for (int i = tid; i < static_cast<int>(gridDim.x); i += kThreads) m = fmaxf(m, a.ws_max[i]);
+    for (int i = tid; i < static_cast<int>(gridDim.x); i += kWork) m = fmaxf(m, a.ws_max[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __syncthreads();
+    work_sync();
     if (lane == 0) red[warp] = m;
-    __syncthreads();
+    work_sync();
     m = red[0];
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
     const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
     float s = 0.0f, u = 0.0f, gs_x = 1.0f;
     if (nv) {
@@ -347,103 +527,130 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t kbp = (kb + 3) / 4 * 4;
 
     for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
-      const int rb = unit % a.nrb, sp = unit / a.nrb;
-      const int m0 = rb * kRows;
-      const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
-      const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
-      const int n = k_hi - k_lo;
+      int m0, k_lo, n;
+      unit_range(unit, m0, k_lo, n);
+      const int sp = unit / a.nrb;
+      const int64_t col0 = static_cast<int64_t>(k_lo) * kTileK;
       if (!a.hold) {
-        __syncthreads();
-        for (int j = tid; j < n * kTileK; j += kThreads) {
+        work_sync();
+        for (int j = tid; j < n * kTileK; j += kWork) {
           const int col = k_lo * kTileK + j;
           rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
         }
-        __syncthreads();
+        work_sync();
       }
       const int rows = min(kRows, a.B - m0);
-      // the unit's 16-byte chunk (row r, logical chunk c) of tile t
-      auto chunk = [&](int t, int r, int c) -> uint4 {
-        if (a.hold)
-          return *reinterpret_cast<const uint4*>(xbuf + static_cast<size_t>(t) * kTileBytes + r * 128 +
-                                                 ((c ^ (r & 7)) * 16));
-        return __ldg(reinterpret_cast<const uint4*>(static_cast<const TIn*>(a.x) +
-                                                    static_cast<int64_t>(m0 + r) * a.ldx +
-                                                    (k_lo + t) * kTileK + c * kPerChunk));
-      };
+      const int ncols = min(n * kTileK, a.M - k_lo * kTileK);   // a multiple of 32
       if (!nv) {
-        // thread -> chunk c of rows r0, r0 + 64 of every tile; c_k = fl(r_k u) per column
-        const int c = tid & 7, r0 = tid >> 3;
-        for (int t = 0; t < n; ++t) {
-          const int col = (k_lo + t) * kTileK + c * kPerChunk;
-          if (col >= a.M) continue;
-          float ck[kPerChunk];
+        // a warp writes 256 consecutive codes of a row (8 per lane, one 256-byte
+        // store), two rows (r, r + 16) at a time
+        for (int c256 = 0; c256 < ncols; c256 += 256) {
+          const int cl = c256 + 8 * lane;
+          const bool live = cl < ncols;
+          float ck[8];
 #pragma unroll
-          for (int j = 0; j < kPerChunk; ++j) ck[j] = __fmul_rn(rcp[t * kTileK + c * kPerChunk + j], u);
-          uint4 raw[kRows / (kThreads / 8)];
-#pragma unroll
-          for (int i = 0; i < kRows / (kThreads / 8); ++i) {
-            const int r = r0 + (kThreads / 8) * i;
-            if (r < rows) raw[i] = chunk(t, r, c);
-          }
-#pragma unroll
-          for (int i = 0; i < kRows / (kThreads / 8); ++i) {
-            const int r = r0 + (kThreads / 8) * i;
-            if (r >= rows) continue;
-            float v[kPerChunk];
-            unpack16<TIn>(raw[i], v);
-            uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-            for (int j = 0; j < kPerChunk; ++j) {
-              int qv = __float2int_rn(__fmul_rn(v[j], ck[j]));
-              qv = min(max(qv, -a.qmax), a.qmax);
-              packed[j >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (j & 3));
+          for (int j = 0; j < 8; ++j) ck[j] = live ? __fmul_rn(rcp[cl + j], u) : 0.0f;
+          for (int r = warp; r < rows; r += 2 * kWorkWarps) {
+            const int r2 = r + kWorkWarps;
+            const bool two = r2 < rows;
+            uint4 ua[2], ub[2];
+            if (live) {
+              load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r, col0, r, cl, ua);
+              if (two) load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r2, col0, r2, cl, ub);
             }
-            int8_t* dst = static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r) * a.M + col;
-            if constexpr (kPerChunk == 8)
-              *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-            else
-              *reinterpret_cast<uint32_t*>(dst) = packed[0];
+            if (live) {
+              float v[8];
+              unpack8<TIn>(ua, v);
+              *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r) * a.M +
+                                        col0 + cl) = int_codes8(v, ck);
+              if (two) {
+                unpack8<TIn>(ub, v);
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) +
+                                          static_cast<int64_t>(m0 + r2) * a.M + col0 + cl) = int_codes8(v, ck);
+              }
+            }
           }
         }
       } else {
-        // thread -> 16-element block b of row r of every tile
-        constexpr int kBlk = kTileK / 16;                 // blocks per tile row
-        constexpr int kChunksPerBlk = 16 / kPerChunk;
-        constexpr int kRowsPerPass = kThreads / kBlk;     // rows covered per pass
-        const int bk = tid % kBlk, r0 = tid / kBlk;
-        for (int t = 0; t < n; ++t) {
-          const int col = (k_lo + t) * kTileK + bk * 16;
-          if (col >= a.M) continue;
-          for (int r = r0; r < rows; r += kRowsPerPass) {
-            float xs[16];
+        // half a warp = 256 consecutive elements of one row (one 16-element block per lane)
+        const int nch = (ncols + 255) / 256;
+        const int items = nch * rows;
+        for (int base = 2 * warp; base < items; base += 2 * kWorkWarps) {
+          const int it = base + (lane >> 4);
+          if (it >= items) continue;
+          const int cc = it / rows, r = it - cc * rows;
+          const int cl = cc * 256 + 16 * (lane & 15);
+          if (cl >= ncols) continue;
+          float xs[16];
 #pragma unroll
-            for (int h = 0; h < kChunksPerBlk; ++h) {
-              unpack16<TIn>(chunk(t, r, bk * kChunksPerBlk + h), xs + h * kPerChunk);
-            }
-            float amax = 0.0f;
+          for (int h = 0; h < 2; ++h) {
+            uint4 uu[2];
+            float v8[8];
+            load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r, col0, r, cl + 8 * h, uu);
+            unpack8<TIn>(uu, v8);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              xs[j] = __fmul_rn(xs[j], rcp[t * kTileK + bk * 16 + j]);
-              amax = fmaxf(amax, fabsf(xs[j]));
-            }
-            const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
-            const float d = ue4m3_to_f32(sfb);
-            const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
-            const int row = m0 + r;
-            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(row) * (a.M / 2) +
-                                      col / 2) = make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
-            a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+            for (int j = 0; j < 8; ++j) xs[8 * h + j] = v8[j];
           }
+          float amax = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            xs[j] = __fmul_rn(xs[j], rcp[cl + j]);
+            amax = fmaxf(amax, fabsf(xs[j]));
+          }
+          const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+          const float d = ue4m3_to_f32(sfb);
+          const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
+          const int64_t row = m0 + r;
+          const int64_t col = col0 + cl;
+          *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
+              make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
+          a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
         }
       }
-      // down: this unit's share of the row block's rows, all K splits summed
+      // down = the K-split partials summed in split order, as bf16 hi | lo
       if (a.has_ld && a.down != nullptr) {
-        const int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
+        int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
+        if (a.hold) {
+          // drain this unit's accumulator into its partial, then the last of
+          // the row block's K splits to arrive sums the whole row block
+          if (warp < 4) {
+            const bool fin = mbar_wait_warp(&mma_done, 0, status, &abort_sh);
+            tc_fence_after();
+            const int row = m0 + warp * 32 + lane;
+            float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * a.rank_pad;
+            for (int c0 = 0; c0 < a.rank_pad; c0 += 32) {
+              uint32_t v[32];
+              __syncwarp();
+              tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+              tmem_ld_wait_regs(v);
+              if (fin && row < a.B) {
+                const int cnt = min(32, a.rank_pad - c0);
+                for (int j = 0; j < cnt; j += 4)
+                  *reinterpret_cast<float4*>(dst + c0 + j) =
+                      make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                  __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+              }
+            }
+            tc_fence_before();
+            if (!fin) abort_sh = 1;
+          }
+          __threadfence();
+          work_sync();
+          if (tid == 0) {
+            const unsigned prev = atomicAdd(a.sync + 2 + (unit % a.nrb), 1u);
+            red[0] = prev == static_cast<unsigned>(a.ksplit - 1) ? 1.0f : 0.0f;
+          }
+          work_sync();
+          const bool last = red[0] != 0.0f && abort_sh == 0;
+          __threadfence();
+          r_lo = 0;
+          r_hi = last ? kRows : 0;
+        }
         const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
         const int cnt = (r_hi - r_lo) * a.rank_pad;
-        for (int i = tid; i < cnt; i += kThreads) {
+        for (int i = tid; i < cnt; i += kWork) {
           const int rr = r_lo + i / a.rank_pad, j = i % a.rank_pad;
           const int row = m0 + rr;
           if (row >= a.B) continue;
@@ -463,8 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
       const int64_t pad_cols = kbp - kb;
       const int64_t n_pad = (rows_p - a.B) * kbp + static_cast<int64_t>(a.B) * pad_cols;
-      for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + tid; i < n_pad;
-           i += static_cast<int64_t>(gridDim.x) * kThreads) {
+      for (int64_t i = static_cast<int64_t>(blockIdx.x) * kWork + tid; i < n_pad;
+           i += static_cast<int64_t>(gridDim.x) * kWork) {
         int64_t row, c;
         if (i < static_cast<int64_t>(a.B) * pad_cols) {
           row = i / pad_cols;
@@ -480,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (a.has_ld && warp == 0) {
+  if (a.has_ld && warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, tcols);
   }
@@ -489,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t smem_for(const ActPlan& p, int xbuf) {
   const int ld_bytes = p.rank_pad * 128;
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
-  return static_cast<size_t>(xbuf) * kTileBytes + (p.rank_pad > 0 ? kRing * ld_bytes : 0) +
+  return static_cast<size_t>(xbuf) * kTileBytes + (p.rank_pad > 0 ? kLdRing * ld_bytes : 0) +
          static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
 }
 
@@ -525,7 +732,7 @@ void finish_act_plan(ActPlan& p) {
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   // hold the unit's x tiles when they fit and every unit gets a CTA of its own
   p.hold = 0;
-  p.xbuf = kRing;
+  p.xbuf = kXRing;
   if (steps_max <= kMaxHold) {
     const size_t sm = smem_for(p, steps_max);
     if (sm <= static_cast<size_t>(kSmemBudget) && p.nunits <= num_sms() * resident_per_sm(sm, p.bf16)) {
@@ -557,9 +764,15 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt) {
   return p;
 }
 
+// Barrier words: [0] grid barrier counter, [1] abort flag, [2 + rb] K-split
+// arrivals of row block rb (all zeroed before each launch).
+size_t act_sync_bytes(const ActPlan& p) {
+  return static_cast<size_t>(round_up((2 + static_cast<int64_t>(p.nrb)) * 4, 256));
+}
+
 size_t act_scratch_bytes(const ActPlan& p) {
   size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));
-  b += 256;  // grid barrier words
+  b += act_sync_bytes(p);
   if (p.rank_pad > 0)
     b += static_cast<size_t>(round_up(static_cast<int64_t>(p.ksplit) * p.B * p.rank_pad * 4, 256));
   return b + 256;
@@ -575,27 +788,20 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
   Carver cv(scratch, ~size_t(0));
   float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));
-  unsigned* sync = static_cast<unsigned*>(cv.take(256));
+  unsigned* sync = static_cast<unsigned*>(cv.take(act_sync_bytes(p)));
   float* ws_down =
       has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4))
              : nullptr;
   const int esz = xdt == SVDQ_BF16 ? 2 : 4;
   const CUtensorMapDataType cdt =
       xdt == SVDQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  CUtensorMap tm_x, tm_ld;
-  if (!make_tmap_2d(&tm_x, x, cdt, esz, p.M, p.B, ldx, p.tile_k, kRows, true)) {
+  CUtensorMap tm_x;
+  if (!make_tmap_2d(&tm_x, x, cdt, esz, p.M, p.B, ldx, p.tile_k, kRows, true) ||
+      (has_ld && (reinterpret_cast<uintptr_t>(ld) & 15) != 0)) {
     *bad_args = true;
     return cudaSuccess;
   }
-  if (has_ld) {
-    if (!make_tmap_2d(&tm_ld, ld, cdt, esz, p.M, p.rank_pad, p.M, p.tile_k, p.rank_pad, true)) {
-      *bad_args = true;
-      return cudaSuccess;
-    }
-  } else {
-    tm_ld = tm_x;
-  }
-  cudaError_t err = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), stream);
+  cudaError_t err = cudaMemsetAsync(sync, 0, (2 + static_cast<size_t>(p.nrb)) * sizeof(unsigned), stream);
   if (err != cudaSuccess) return err;
   ActArgs a{};
   a.B = static_cast<int>(p.B);
@@ -615,6 +821,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.scale = scale;
   a.gs_given = fmt.kind == SVDQ_KIND_NVFP4 ? act_global_scale : nullptr;
   a.gs_w = fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr;
+  a.ld = has_ld ? ld : nullptr;
   a.ws_down = ws_down;
   a.ws_max = ws_max;
   a.sync = sync;
@@ -627,7 +834,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   ActPlan q = p;
   if (!has_ld) q.rank_pad = 0;
   const size_t smem = smem_for(q, p.xbuf);
-  void* args[] = {&tm_x, &tm_ld, &a};
+  void* args[] = {&tm_x, &a};
   if (xdt == SVDQ_BF16) {
     err = cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -28,6 +28,7 @@
 
 #include <algorithm>
 
+#include "gemm_common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -47,32 +48,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfaCol = 256;        // NVFP4: scale factors of A, 4 columns per MMA
 constexpr uint32_t kSfbCol = 272;        // NVFP4: scale factors of B, 8 columns per MMA
 
-enum Kind { kKindInt = 0, kKindNvfp4 = 1 };
-enum OutKind { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
-
 template <int kKind>
 struct Cfg {
   static constexpr int kStageBytes =
       kABytes + kBBytes + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
-};
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // a -> low half
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-struct GemmArgs {
-  int B, N, M, lr_steps;
-  const float* s_x;               // INT: s_x, NVFP4: gs_x
-  const float* s_w;               // INT: s_w, NVFP4: gs_w
-  const __nv_bfloat16* bias;
-  void* y;
-  int64_t ldy;
-  int vec_ok;
-  const uint8_t* sfa;             // NVFP4 activation scales (128x4 layout)
-  const uint8_t* sfb;             // NVFP4 weight scales (128x4 layout)
-  int katoms;                     // NVFP4: 64-element scale atoms per row tile = ceil(M / 64)
-  unsigned* status;
 };
 
 template <int kKind, int kOut>
@@ -188,6 +167,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t id_f4 = idesc_nvf4(kBM, kBN);
       // INT: low-rank into its own fp32 accumulator; NVFP4: everything into one
       const uint32_t lr_acc = kKind == kKindNvfp4 ? tmem : tmem + 256;
+      {
+        // throwaway MMA: the first tcgen05.mma of a kernel takes microseconds
+        // longer than the rest; issued now, that start-up overlaps the first
+        // loads (the first real MMA of the tile overwrites the accumulator)
+        const uint64_t d0 = smem_desc_sw128(smem_u32(smem));
+        if constexpr (kKind == kKindNvfp4)
+          mma_nvf4(tmem, d0, d0, id_f4, 0u, tmem + kSfaCol, tmem + kSfbCol);
+        else
+          mma_i8(tmem, d0, d0, id_i8, 0u);
+      }
       uint32_t it = 0, lt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
@@ -247,99 +236,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r_in = q * 32 + lane;
-    float alpha = 0.0f;
-    if (kOut != kOutI32) {
-      if (kKind == kKindNvfp4)
-        alpha = __fdiv_rn(1.0f, __fmul_rn(__ldg(args.s_x), __ldg(args.s_w)));
-      else
-        alpha = __ldg(args.s_x) * __ldg(args.s_w);
-    }
+    const float alpha = epilogue_alpha<kKind, kOut>(args);
     const bool sep_lr = kKind == kKindInt && kOut != kOutI32 && lr_steps > 0;
     uint32_t lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
-      if (!mbar_wait(&tmem_full_bar, lt & 1, status, &abort_sh)) break;
+      if (!mbar_wait_warp(&tmem_full_bar, lt & 1, status, &abort_sh)) break;
       tc_fence_after();
       const int m0 = (t % tiles_m) * kBM;
       const int n0 = (t / tiles_m) * kBN;
-      const int row = m0 + r_in;
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
-        __syncwarp();  // the TMEM loads below are warp-collective
-        uint32_t acc[32], up[32];
-        tmem_ld_32x32b_x32(lane_addr + c0, acc);
-        if (sep_lr) tmem_ld_32x32b_x32(lane_addr + 256 + c0, up);
-        tmem_ld_wait();
-        const int n = n0 + c0;
-        if (row >= B || n >= N) continue;
-        const bool full = args.vec_ok && (n + 32 <= N);
-        if (kOut == kOutI32) {
-          int32_t* dst = static_cast<int32_t*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
-          if (full) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<uint4*>(dst + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n + j < N) dst[j] = static_cast<int32_t>(acc[j]);
-          }
-          continue;
-        }
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (kKind == kKindNvfp4) {
-            v[j] = alpha * __uint_as_float(acc[j]);
-          } else {
-            v[j] = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
-            if (sep_lr) v[j] += __uint_as_float(up[j]);
-          }
-        }
-        if (args.bias != nullptr) {
-          if (n + 32 <= N) {
-            const uint4* bp = reinterpret_cast<const uint4*>(args.bias + n);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint4 bb = __ldg(bp + g);
-              const uint32_t w4[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                v[8 * g + 2 * h] += __uint_as_float(w4[h] << 16);
-                v[8 * g + 2 * h + 1] += __uint_as_float(w4[h] & 0xFFFF0000u);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n + j < N) v[j] += __bfloat162float(args.bias[n + j]);
-          }
-        }
-        if (kOut == kOutF32) {
-          float* dst = static_cast<float*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
-          if (full) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n + j < N) dst[j] = v[j];
-          }
-        } else {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.y) + static_cast<int64_t>(row) * args.ldy + n;
-          if (full) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 8)
-              *reinterpret_cast<uint4*>(dst + j) =
-                  make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]),
-                             pack_bf16x2(v[j + 4], v[j + 5]), pack_bf16x2(v[j + 6], v[j + 7]));
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n + j < N) dst[j] = __float2bfloat16_rn(v[j]);
-          }
-        }
-      }
+      epilogue_slab<kKind, kOut>(args, lane_addr, m0 + r_in, n0, alpha, sep_lr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tmem_empty_bar);
@@ -410,6 +316,15 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
   args.sfb = static_cast<const uint8_t*>(w->sf);
   args.katoms = static_cast<int>(ceil_div(M, 64));
   args.status = device_status_word();
+  // more than one 128-row block: CTA pairs (256 x 256 tiles)
+  if (B > kBM) {
+    cudaError_t err = cudaSuccess;
+    const int out = raw_i32 ? kOutI32 : (ydt == SVDQ_F32 ? kOutF32 : kOutBF16);
+    if (launch_gemm_pair(kKind, out, args, act_codes, has_lr ? down2 : nullptr, w, stream, &err))
+      return err;
+    *bad_args = true;
+    return cudaSuccess;
+  }
   const int64_t tiles = ceil_div(B, kBM) * ceil_div(N, kBN);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   if (raw_i32) {

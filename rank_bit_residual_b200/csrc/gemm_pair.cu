@@ -1,0 +1,387 @@
+// gemm_pair.cu - the residual GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same operator as gemm.cu ("SVDQuant Smoothing, Low-rank and Residual
+// Quantization", Formula item 3; step 3 of "flashinfer.gemm.svdquant_linear"):
+// Y = alpha * Q(X_hat) Q(R) + down . lu^T [+ bias], INT (kind::i8) or NVFP4
+// (kind::mxf4nvf4 with ue4m3 scales per 16 elements).
+//
+// A cluster of two CTAs computes one 256 x 256 output tile: CTA r holds rows
+// [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128) of the B
+// tile in its shared memory, and its TMEM receives its 128 rows of the
+// accumulator for all 256 columns. One thread of the even CTA issues every MMA
+// for the pair. Each CTA loads its own halves by TMA and signals the even CTA's
+// barrier; the MMA commits signal the barriers of both CTAs; each CTA's
+// epilogue drains its own TMEM and reports back to the even CTA. Per SM this
+// halves the B-operand traffic of the one-CTA kernel and, for NVFP4, the scale
+// copies per multiply-accumulate.
+//
+// Warps: 0 TMA producer, 1 MMA (even CTA), 2-9 epilogue (two warps per TMEM
+// lane quarter, each for 128 of the 256 columns). The epilogue runs in two
+// passes so that the global stores overlap the next tile's MMAs:
+//   pass 1  alpha * acc (+ up) + bias, rounded to the output type, written back
+//           into TMEM columns the next tile's residual MMAs do not touch; then
+//           the accumulator columns are released (acc_empty);
+//   pass 2  those columns -> Y; then (INT) the low-rank columns are released
+//           (lr_empty).
+// Each tile runs its residual K steps first and its low-rank K steps last, so
+// the next tile's MMAs need the low-rank columns only at the end of its chain.
+// TMEM columns (512):
+//   INT    [0, 256) int32 residual | [256, 512) fp32 up-projection, which
+//          pass 1 overwrites in place with the combined result
+//   NVFP4  [0, 256) fp32 (both branches) | [256, 304) block scales |
+//          [384, 512) bf16 result of pass 1 (fp32 output: one direct pass)
+// NVFP4: each CTA's TMEM holds the scales of its 128 A rows (4 columns per
+// K = 64 step) and of all 256 B rows (8 columns), copied from its own shared
+// memory by the pair-wide tcgen05.cp the even CTA issues.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "gemm_common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kEpiWarps = 8;
+constexpr int kPairThreads = 64 + 32 * kEpiWarps;
+constexpr int kHalf = 128;                        // rows of A and of B per CTA
+constexpr int kTileN = 256;
+constexpr int kABytes = kHalf * 128;
+constexpr int kBBytes = kHalf * 128;
+constexpr int kSfaBytes = 4 * 512;                // this CTA's A rows, 4 atoms
+constexpr int kSfbBytes = 2 * 4 * 512;            // both B row tiles, 4 atoms each
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = 256;
+constexpr uint32_t kSfbCol = 272;
+constexpr uint32_t kNvOutCol = 384;               // NVFP4 bf16 pass-1 result
+
+template <int kKind>
+struct PairCfg {
+  static constexpr int kStages = kKind == kKindNvfp4 ? 5 : 6;
+  static constexpr int kStageBytes = kABytes + kBBytes + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
+};
+
+// Whether the epilogue's stores overlap the next tile's MMAs.
+template <int kKind, int kOut>
+struct TwoPass {
+  static constexpr bool value = kOut == kOutBF16 || (kKind == kKindInt && kOut == kOutF32);
+};
+
+template <int kKind, int kOut>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_da, const __grid_constant__ CUtensorMap tm_lu,
+                     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                     const GemmArgs args) {
+  constexpr int kStages = PairCfg<kKind>::kStages;
+  constexpr int kStageBytes = PairCfg<kKind>::kStageBytes;
+  constexpr bool kTwoPass = TwoPass<kKind, kOut>::value;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tmem_full_bar;
+  __shared__ __align__(8) uint64_t acc_empty_bar;
+  __shared__ __align__(8) uint64_t lr_empty_bar;
+  __shared__ __align__(8) uint64_t exit_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int B = args.B, N = args.N, M = args.M, lr_steps = args.lr_steps;
+  unsigned* status = args.status;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int tiles_m = (B + 2 * kHalf - 1) / (2 * kHalf);
+  const int tiles_n = (N + kTileN - 1) / kTileN;
+  const int total = tiles_m * tiles_n;
+  constexpr int kStageK = kKind == kKindNvfp4 ? 256 : 128;
+  const int ksteps = (M + kStageK - 1) / kStageK;
+  const int steps_per_tile = ksteps + lr_steps;   // residual steps first
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&tmem_full_bar, 1);
+    mbar_init(&acc_empty_bar, 2 * kEpiWarps);   // the epilogue warps of both CTAs
+    mbar_init(&lr_empty_bar, 2 * kEpiWarps);
+    mbar_init(&exit_bar, 1);                    // the peer's arrival at teardown
+    fence_mbar_init();
+    abort_sh = 0;
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    if (lr_steps) {
+      tma_prefetch_desc(&tm_da);
+      tma_prefetch_desc(&tm_lu);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs: barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const int m0 = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf;
+        const int nt = (t / tiles_m) * kTileN;
+        const int n0 = nt + static_cast<int>(rank) * kHalf;
+        for (int j = 0; j < steps_per_tile && ok; ++j, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          ok = mbar_wait(&empty_bar[s], ph ^ 1, status, &abort_sh);
+          if (!ok) break;
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
+          if (j >= ksteps) {
+            const int l = j - ksteps;
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
+            tma_load_2d_pair(st, &tm_da, fb, 64 * l, m0);
+            tma_load_2d_pair(st + kABytes, &tm_lu, fb, 64 * l, n0);
+          } else if constexpr (kKind == kKindNvfp4) {
+            if (rank == 0)
+              mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
+            tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
+            tma_load_2d_pair(st + kABytes, &tm_b, fb, 128 * j, n0);
+            // scale atoms: rows of 256 bytes, two rows per 512-byte atom
+            uint8_t* sfa_s = st + kABytes + kBBytes;
+            uint8_t* sfb_s = sfa_s + kSfaBytes;
+            const int a0 = 4 * j;
+            tma_load_2d_pair(sfa_s, &tm_sfa, fb, 0, 2 * ((m0 / 128) * args.katoms + a0));
+            for (int rt = 0; rt < 2; ++rt)
+              tma_load_2d_pair(sfb_s + rt * 2048, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
+          } else {
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
+            tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
+            tma_load_2d_pair(st + kABytes, &tm_b, fb, 128 * j, n0);
+          }
+        }
+      }
+      // wait for the MMA's release of the last stages, so no commit arrival
+      // is still on its way to this CTA's barriers when it exits
+      if (ok) {
+        const uint32_t first = it > static_cast<uint32_t>(kStages) ? it - kStages : 0u;
+        for (uint32_t i = first; i < it; ++i)
+          mbar_wait(&empty_bar[i % kStages], (i / kStages) & 1, status, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA (even CTA only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t id_i8 = idesc_i8(2 * kHalf, kTileN);
+      const uint32_t id_bf = idesc_bf16(2 * kHalf, kTileN);
+      const uint32_t id_f4 = idesc_nvf4(2 * kHalf, kTileN);
+      const uint32_t lr_acc = kKind == kKindNvfp4 ? tmem : tmem + 256;
+      {
+        // throwaway MMA: the first tcgen05.mma of a kernel takes microseconds
+        // longer than the rest; issued now, that start-up overlaps the first
+        // loads (the first real MMA of the tile overwrites the accumulator)
+        const uint64_t d0 = smem_desc_sw128(smem_u32(smem));
+        if constexpr (kKind == kKindNvfp4)
+          mma_nvf4_pair(tmem, d0, d0, id_f4, 0u, tmem + kSfaCol, tmem + kSfbCol);
+        else
+          mma_i8_pair(tmem, d0, d0, id_i8, 0u);
+      }
+      uint32_t it = 0, lt = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+        ok = mbar_wait(&acc_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
+        if (!ok) break;
+        tc_fence_after();
+        for (int j = 0; j < steps_per_tile; ++j, ++it) {
+          if (kKind == kKindInt && j == ksteps) {
+            // the low-rank columns: the previous tile's stores are done
+            ok = mbar_wait(&lr_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          ok = mbar_wait(&full_bar[s], ph, status, &abort_sh);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+          if (j >= ksteps) {
+            const int l = j - ksteps;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_pair(lr_acc, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_bf,
+                           (kKind == kKindNvfp4 || l > 0 || kk > 0) ? 1u : 0u);
+          } else if constexpr (kKind == kKindNvfp4) {
+            const int na = min(4, args.katoms - 4 * j);
+            const uint32_t sfa_s = b0 + kBBytes;
+            const uint32_t sfb_s = sfa_s + kSfaBytes;
+            for (int kk = 0; kk < na; ++kk) {
+              tmem_cp_32x128b_warpx4_pair(tmem + kSfaCol + 4 * kk, smem_desc_plain(sfa_s + 512 * kk));
+              for (int rt = 0; rt < 2; ++rt)
+                tmem_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * kk + 4 * rt,
+                                            smem_desc_plain(sfb_s + 2048 * rt + 512 * kk));
+            }
+            for (int kk = 0; kk < na; ++kk)
+              mma_nvf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
+                            (j > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_i8_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_i8,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty_bar[s], 0x3);
+        }
+        if (!ok) break;
+        if (kKind == kKindInt && lr_steps == 0) {
+          // keep the low-rank barrier's phases in step with the tiles
+          ok = mbar_wait(&lr_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
+          if (!ok) break;
+        }
+        mma_commit_pair(&tmem_full_bar, 0x3);
+      }
+      // both epilogues have released the last tile: no arrival from the odd
+      // CTA is still on its way when this CTA leaves
+      if (ok && lt > 0) {
+        mbar_wait(&acc_empty_bar, (lt - 1) & 1, status, &abort_sh);
+        if (kKind == kKindInt) mbar_wait(&lr_empty_bar, (lt - 1) & 1, status, &abort_sh);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;                         // TMEM lane quarter
+    const int h = (warp - 2) >> 2;                  // column half of the tile
+    const int r_in = q * 32 + lane;
+    const float alpha = epilogue_alpha<kKind, kOut>(args);
+    const bool sep_lr = kKind == kKindInt && kOut != kOutI32 && lr_steps > 0;
+    const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty_bar), 0);
+    const uint32_t lr_empty_even = mapa_shared(smem_u32(&lr_empty_bar), 0);
+    auto release = [&](uint32_t even_addr, uint64_t* local) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(local);
+        else
+          mbar_arrive_remote(even_addr);
+      }
+    };
+    uint32_t lt = 0;
+    for (int t = pair; t < total; t += npairs, ++lt) {
+      if (!mbar_wait_warp(&tmem_full_bar, lt & 1, status, &abort_sh)) break;
+      tc_fence_after();
+      const int row = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf + r_in;
+      const int nt = (t / tiles_m) * kTileN;
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (kTwoPass) {
+        // the result of column chunk c goes to dst(c): INT in place over its
+        // own low-rank columns, NVFP4 (bf16) to the free columns from 384
+        auto dst = [](int c) -> uint32_t {
+          return kKind == kKindInt ? 256u + 32u * c : kNvOutCol + 16u * c;
+        };
+        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+          const int n = nt + 32 * c;
+          if (n < N)
+            epilogue_combine<kKind, kOut>(args, lane_addr, n, 32u * c, 256u + 32u * c, dst(c), alpha, sep_lr);
+        }
+        tmem_st_wait();
+        release(acc_empty_even, &acc_empty_bar);
+        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+          const int n = nt + 32 * c;
+          if (n < N) epilogue_store<kOut>(args, lane_addr, row, n, dst(c));
+        }
+        if (kKind == kKindInt) release(lr_empty_even, &lr_empty_bar);
+      } else {
+        for (int c = 4 * h; c < 4 * h + 4; ++c)
+          epilogue_chunk_direct<kKind, kOut>(args, lane_addr, row, nt + 32 * c, 32u * c, alpha, sep_lr);
+        release(acc_empty_even, &acc_empty_bar);
+        if (kKind == kKindInt) release(lr_empty_even, &lr_empty_bar);
+      }
+    }
+  }
+
+  // teardown: each CTA tells the other it is done and waits (bounded) to hear
+  // the same, so neither releases TMEM or shared memory the other still uses
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_remote(mapa_shared(smem_u32(&exit_bar), rank ^ 1u));
+    mbar_wait(&exit_bar, 0, status, nullptr);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+template <int kKind, int kOut>
+cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int grid, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(PairCfg<kKind>::kStages) * PairCfg<kKind>::kStageBytes + 1024;
+  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<kKind, kOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  gemm_pair_kernel<kKind, kOut><<<grid, kPairThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                    maps[4], maps[5], args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Builds the pair kernel's tensor maps and launches it; returns false (and
+// launches nothing) if a map cannot be encoded.
+bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
+                      const void* down2, const svdq_weight* w, cudaStream_t stream,
+                      cudaError_t* err) {
+  *err = cudaSuccess;
+  const int64_t M = args.M, N = args.N, B = args.B;
+  const int rp = w->rank_pad;
+  const int64_t row_bytes = kind == kKindNvfp4 ? M / 2 : M;
+  CUtensorMap maps[6];
+  bool ok =
+      make_tmap_2d(&maps[0], act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, B, row_bytes, 128, kHalf, true) &&
+      make_tmap_2d(&maps[1], w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, N, row_bytes, 128, kHalf, true);
+  if (ok && args.lr_steps) {
+    ok = make_tmap_2d(&maps[2], down2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, B, 2 * rp, 64, kHalf, true) &&
+         make_tmap_2d(&maps[3], w->lu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, N, 2 * rp, 64, kHalf, true);
+  } else {
+    maps[2] = maps[0];
+    maps[3] = maps[1];
+  }
+  if (ok && kind == kKindNvfp4) {
+    const int64_t rows_a = ceil_div(B, 128) * args.katoms * 2;
+    const int64_t rows_b = ceil_div(N, 128) * args.katoms * 2;
+    ok = make_tmap_2d(&maps[4], args.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_a, 256, 256, 8, false) &&
+         make_tmap_2d(&maps[5], args.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_b, 256, 256, 8, false);
+  } else {
+    maps[4] = maps[0];
+    maps[5] = maps[1];
+  }
+  if (!ok) return false;
+  const int64_t tiles = ceil_div(B, 2 * kHalf) * ceil_div(N, kTileN);
+  const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, num_sms() / 2));
+  if (kind == kKindInt) {
+    if (out == kOutI32) *err = launch_pair_one<kKindInt, kOutI32>(maps, args, grid, stream);
+    else if (out == kOutF32) *err = launch_pair_one<kKindInt, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindInt, kOutBF16>(maps, args, grid, stream);
+  } else {
+    if (out == kOutF32) *err = launch_pair_one<kKindNvfp4, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindNvfp4, kOutBF16>(maps, args, grid, stream);
+  }
+  return true;
+}
+
+}  // namespace svdq
