@@ -6,8 +6,11 @@ A step is one pass of the operator's hot path over one batch: the fused
 activation pass (smoothing, per-tensor max, codes, down-projection) and the
 residual tensor-core GEMM with the low-rank + bias epilogue, both through the
 C ABI. The weight split (svdq_prepare) is timed once, separately. Inputs are
-synthetic and seeded (synth/), resident in HBM when the timed region starts;
-L2 is flushed (a 256 MiB write) between timed steps, outside the events.
+synthetic and seeded (synth/), resident in HBM when the timed region starts.
+The run keeps R buffer sets (x, prepared weight, codes, down, Y) spanning at
+least three L2 sizes and step i uses set i % R, so no step finds its inputs in
+L2; the K steps run back to back (one CUDA graph per step when capture works)
+between one pair of CUDA events.
 
 value     whole-job TOPS (2BMN residual ops + 2Br(M+N) low-rank flops per step)
 e2e       the same metric through svdq_linear with pinned host x copied in and
@@ -37,7 +40,7 @@ if ROOT not in sys.path:
 
 METRIC = "svdq_linear TOPS and GB/s at 1 B200; % of roofline (HBM or int8/FP4 peak)"
 DEFAULT_WORKLOAD = "dit_attn_4096x3072x3072_int4"
-L2_FLUSH_BYTES = 256 << 20
+L2_ROTATE_BYTES = 3 * (126 << 20)   # the buffer sets of a run span three L2 sizes at least
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemm_int_dit_attn_4096x3072x3072_int4.md")
@@ -265,53 +268,90 @@ def main():
     w = rb.svdq_prepare(W, scale, r, fmt, seed=0)
     torch.cuda.synchronize()
     prepare_ms = 1000.0 * (time.perf_counter() - t0)
-    del W
+    wgs_of = (lambda wt: wt.w_scale) if wl.fmt == "nvfp4" else (lambda wt: None)
 
-    # buffers of the two stages (allocated once, outside the timed region)
-    codes, sf, act_scale, down = rb.svdq_quantize_act(
-        x, scale, fmt, ld=w.ld if r else None, w_global_scale=w.w_scale if wl.fmt == "nvfp4" else None)
-    y = torch.empty((B, N), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # R buffer sets (x, weight, codes, down, Y) whose union is several times
+    # the L2 size: step i runs on set i % R, so no step finds its inputs in L2
+    bytes_set = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None) + B * M  # + act codes
+    R = int(min(64, max(2, -(-L2_ROTATE_BYTES // bytes_set))))
+    sets = []
+    for k in range(R):
+        wk = w if k == 0 else rb.svdq_prepare(W, scale, r, fmt, seed=0)
+        xk = x if k == 0 else x.clone()
+        c, sfk, asc, dn = rb.svdq_quantize_act(xk, scale, fmt, ld=wk.ld if r else None,
+                                               w_global_scale=wgs_of(wk))
+        yk = torch.empty((B, N), dtype=torch.bfloat16, device=dev)
+        sets.append((wk, xk, c, sfk, asc, dn, yk))
+    del W
+    y = sets[0][6]
     stream = torch.cuda.current_stream()
 
-    wgs = w.w_scale if wl.fmt == "nvfp4" else None
+    def act_stage(k):
+        wk, xk, c, sfk, asc, dn, yk = sets[k]
+        rb.svdq_quantize_act_into(xk, scale, fmt, wk.ld if r else None, c, sfk, asc, dn,
+                                  w_global_scale=wgs_of(wk))
 
-    def act_stage():
-        rb.svdq_quantize_act_into(x, scale, fmt, w.ld if r else None, codes, sf, act_scale, down,
-                                  w_global_scale=wgs)
+    def gemm_stage(k):
+        wk, xk, c, sfk, asc, dn, yk = sets[k]
+        rb.svdq_residual_linear(wk, c, sfk, asc, dn, bias=bias, out=yk)
 
-    def gemm_stage():
-        rb.svdq_residual_linear(w, codes, sf, act_scale, down, bias=bias, out=y)
+    def step(k):
+        act_stage(k)
+        gemm_stage(k)
 
-    for _ in range(args.warmup):
-        act_stage()
-        gemm_stage()
+    for i in range(max(args.warmup, R)):
+        step(i % R)
     torch.cuda.synchronize()
     assert rb.svdq_check_status() == rb.SVDQ_OK
 
+    # one CUDA graph per buffer set holds a whole step (the activation pass and
+    # the GEMM with their launches); plain stream launches if capture fails
+    graphs = None
+    try:
+        gs = []
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            for k in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    step(k)
+                gs.append(g)
+        stream.wait_stream(cap)
+        for k in range(R):
+            gs[k].replay()
+        torch.cuda.synchronize()
+        assert rb.svdq_check_status() == rb.SVDQ_OK
+        graphs = gs
+    except Exception as e:  # noqa: BLE001 - any capture failure falls back to launches
+        print(f"bench: CUDA graph capture unavailable ({type(e).__name__}: {e}); stream launches",
+              file=sys.stderr)
+        torch.cuda.synchronize()
+
+    def run_step(k):
+        if graphs is not None:
+            graphs[k].replay()
+        else:
+            step(k)
+
     sampler = ClockSampler(local)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.2)
+    e_start.record(stream)
     for i in range(K):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        act_stage()
-        ev[i][1].record(stream)
-        gemm_stage()
-        ev[i][2].record(stream)
+        run_step(i % R)
+    e_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    act_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
+    total_ms = e_start.elapsed_time(e_end)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -319,8 +359,36 @@ def main():
     ops_step = workload_ops(B, M, N, r)
     value = world * K * ops_step / (total_ms * 1e-3) / 1e12
     ms_per_step = total_ms / K
-    gemm_avg_ms = sum(gemm_ms) / K
-    act_avg_ms = sum(act_ms) / K
+
+    # the GEMM kernel alone, K launches back to back on the rotating sets: its
+    # average launch duration for the roofline line
+    Kg = max(20, min(K, 400))
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    g0.record(stream)
+    for i in range(Kg):
+        gemm_stage(i % R)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    gemm_avg_ms = g0.elapsed_time(g1) / Kg
+
+    # per-stage breakdown (diagnostic: an event between the stages drains the
+    # stream, so these include a few microseconds each)
+    Ks = max(10, min(K, 100))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ks)]
+    for i in range(Ks):
+        ev[i][0].record(stream)
+        act_stage(i % R)
+        ev[i][1].record(stream)
+        gemm_stage(i % R)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    act_avg_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / Ks
+    gemm_ev_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / Ks
+    # the step the parity check reads: set 0 once more
+    step(0)
+    torch.cuda.synchronize()
 
     # parity on sampled rows of the timed output (oracle from the prepared buffers)
     parity = None
@@ -391,12 +459,15 @@ def main():
         "data": "synthetic",
         "config": {"workload": args.workload, "B": B, "M": M, "N": N, "rank": r, "fmt": fmt,
                    "x": wl.x_dtype, "y": "bf16", "bias": wl.bias is not None,
-                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "l2": f"inputs larger than L2: {R} rotating buffer sets of {bytes_set / 1e6:.0f} MB",
+                   "launch": "CUDA graph per step" if graphs is not None else "stream launches",
                    "parallelism": f"replicas{world}"},
         "gbs": bytes_step / (ms_per_step * 1e-3) / 1e9,
         "step_roofline": {"t_roofline_us": t_rf * 1e6, "frac": t_rf / (ms_per_step * 1e-3),
                           "alg_bytes": bytes_step, "ops": ops_step},
-        "stages_ms": {"act": act_avg_ms, "gemm": gemm_avg_ms},
+        "stages_ms": {"act": act_avg_ms, "gemm": gemm_ev_ms, "gemm_back_to_back": gemm_avg_ms,
+                      "note": "act/gemm: events around each stage (each includes the drain an event "
+                              "adds); gemm_back_to_back: Kg launches between one event pair"},
         "roofline": {"bound": "tensor",
                      "kernel": ("gemm_kernel<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
                                 if wl.fmt == "nvfp4" else

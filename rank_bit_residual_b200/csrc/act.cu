@@ -636,17 +636,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             if (!fin) abort_sh = 1;
           }
+          // the row block's K splits meet here (all CTAs are resident: bounded
+          // wait on the arrival count), then each sums its own share of rows
           __threadfence();
           work_sync();
           if (tid == 0) {
-            const unsigned prev = atomicAdd(a.sync + 2 + (unit % a.nrb), 1u);
-            red[0] = prev == static_cast<unsigned>(a.ksplit - 1) ? 1.0f : 0.0f;
+            unsigned* cnt = a.sync + 2 + (unit % a.nrb);
+            atomicAdd(cnt, 1u);
+            const unsigned long long t0 = globaltimer_ns();
+            while (true) {
+              unsigned v;
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+              if (v >= static_cast<unsigned>(a.ksplit)) break;
+              if (*reinterpret_cast<volatile unsigned*>(a.sync + 1)) {
+                abort_sh = 1;
+                break;
+              }
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_status(status, kStatusTimeout);
+                atomicExch(a.sync + 1, 1u);
+                abort_sh = 1;
+                break;
+              }
+              __nanosleep(64);
+            }
+            __threadfence();
           }
           work_sync();
-          const bool last = red[0] != 0.0f && abort_sh == 0;
-          __threadfence();
-          r_lo = 0;
-          r_hi = last ? kRows : 0;
+          if (abort_sh) r_hi = r_lo;
         }
         const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
         const int cnt = (r_hi - r_lo) * a.rank_pad;
