@@ -43,7 +43,6 @@ DEFAULT_WORKLOAD = "dit_attn_4096x3072x3072_int4"
 L2_ROTATE_BYTES = 3 * (126 << 20)   # the buffer sets of a run span three L2 sizes at least
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemm_int_dit_attn_4096x3072x3072_int4.md")
 
 
 # ---------------------------------------------------------------- helpers
@@ -75,21 +74,24 @@ def gemm_alg_ops(B, M, N, rank):
     return 2.0 * B * M * N + 2.0 * B * rank * N
 
 
-def read_profile_traffic(gemm_src):
-    """traffic_bytes_per_launch from the committed ncu summary if it was taken on
-    this very kernel source (sha256 recorded beside it), else None."""
+def read_profile_traffic(workload, sources):
+    """DRAM traffic per launch of the GEMM kernel from the committed ncu summary of
+    this workload, if it was taken on these very kernel sources (a sha256 of the
+    sources is recorded beside it), else None."""
     import hashlib
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(os.path.join(ROOT, "profiles", f"gemm_pair_{workload}.md")).read()
     except OSError:
         return None
-    sha = hashlib.sha256(open(gemm_src, "rb").read()).hexdigest()
+    h = hashlib.sha256()
+    for src in sources:
+        h.update(open(src, "rb").read())
     vals = {}
     for line in text.splitlines():
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("gemm_source_sha256") != sha:
+            vals[k.strip()] = v.strip().split()[0].strip("`") if v.strip() else ""
+    if vals.get("kernel_source_sha256") != h.hexdigest():
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -447,7 +449,10 @@ def main():
     lowp_peak = ratio * peaks["bf16_tflops"]
     g_ops = gemm_alg_ops(B, M, N, r)
     achieved = g_ops / (gemm_avg_ms * 1e-3) / 1e12
-    traffic = read_profile_traffic(os.path.join(ROOT, "rank_bit_residual_b200", "csrc", "gemm.cu"))
+    csrc = os.path.join(ROOT, "rank_bit_residual_b200", "csrc")
+    traffic = read_profile_traffic(args.workload, [os.path.join(csrc, f) for f in
+                                                   ("gemm_pair.cu", "gemm_common.cuh", "ptx.cuh")]) \
+        if B > 128 else None
     bytes_step = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
     t_rf = max(bytes_step / (peaks["hbm_gbs"] * 1e9),
                (2.0 * B * M * N) / (lowp_peak * 1e12) + (2.0 * B * r * (M + N)) / (peaks["bf16_tflops"] * 1e12))
@@ -469,9 +474,11 @@ def main():
                       "note": "act/gemm: events around each stage (each includes the drain an event "
                               "adds); gemm_back_to_back: Kg launches between one event pair"},
         "roofline": {"bound": "tensor",
-                     "kernel": ("gemm_kernel<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
-                                if wl.fmt == "nvfp4" else
-                                "gemm_kernel<INT> (int8 residual + bf16 up-projection)"),
+                     "kernel": (("gemm_pair_kernel" if B > 128 else "gemm_kernel") +
+                                ("<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
+                                 if wl.fmt == "nvfp4" else "<INT> (int8 residual + bf16 up-projection)")),
+                     "duration_us": gemm_avg_ms * 1e3,
+                     "timing": "Kg launches back to back on rotating sets between one CUDA event pair",
                      "achieved": achieved, "peak": lowp_peak, "unit": "TFLOP/s",
                      "frac": achieved / lowp_peak, "traffic": traffic,
                      "peak_source": (f"{peak_src} bf16 GEMM burst x {ratio:g} "
