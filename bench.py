@@ -70,6 +70,17 @@ def alg_bytes(B, M, N, rank, fmt, bits, bias):
             + B * N * 2)
 
 
+def gemm_alg_bytes(B, M, N, rank, fmt, bits, bias):
+    """Algorithmic bytes of one GEMM launch: weight codes (+ scales), the bf16 up
+    factor, the activation codes (+ scales) and the bf16 down tile it reads, bias,
+    and the bf16 Y it writes."""
+    if fmt == "nvfp4":
+        wbytes, abytes = M * N * (0.5 + 1.0 / 16.0), B * M * (0.5 + 1.0 / 16.0)
+    else:
+        wbytes, abytes = M * N * (0.5 if bits <= 4 else 1.0), B * M
+    return wbytes + 2 * rank * N + abytes + 2 * B * rank + (2 * N if bias else 0) + 2 * B * N
+
+
 def gemm_alg_ops(B, M, N, rank):
     return 2.0 * B * M * N + 2.0 * B * rank * N
 
@@ -110,6 +121,7 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.t = None
+        self.clocks = None
 
     def start(self):
         try:
@@ -233,6 +245,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sets", type=int, default=0,
+                    help="rotating buffer sets (default: enough to span three L2 sizes)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -275,7 +289,7 @@ def main():
     # R buffer sets (x, weight, codes, down, Y) whose union is several times
     # the L2 size: step i runs on set i % R, so no step finds its inputs in L2
     bytes_set = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None) + B * M  # + act codes
-    R = int(min(64, max(2, -(-L2_ROTATE_BYTES // bytes_set))))
+    R = int(min(64, max(2, -(-L2_ROTATE_BYTES // bytes_set)))) if args.sets <= 0 else args.sets
     sets = []
     for k in range(R):
         wk = w if k == 0 else rb.svdq_prepare(W, scale, r, fmt, seed=0)
@@ -283,23 +297,28 @@ def main():
         c, sfk, asc, dn = rb.svdq_quantize_act(xk, scale, fmt, ld=wk.ld if r else None,
                                                w_global_scale=wgs_of(wk))
         yk = torch.empty((B, N), dtype=torch.bfloat16, device=dev)
-        sets.append((wk, xk, c, sfk, asc, dn, yk))
+        sets.append((wk, xk, c, sfk, asc, dn, yk, rb.LinearWorkspace()))
     del W
     y = sets[0][6]
     stream = torch.cuda.current_stream()
 
     def act_stage(k):
-        wk, xk, c, sfk, asc, dn, yk = sets[k]
+        wk, xk, c, sfk, asc, dn, yk, _ = sets[k]
         rb.svdq_quantize_act_into(xk, scale, fmt, wk.ld if r else None, c, sfk, asc, dn,
                                   w_global_scale=wgs_of(wk))
 
     def gemm_stage(k):
-        wk, xk, c, sfk, asc, dn, yk = sets[k]
+        wk, xk, c, sfk, asc, dn, yk, _ = sets[k]
         rb.svdq_residual_linear(wk, c, sfk, asc, dn, bias=bias, out=yk)
 
-    def step(k):
-        act_stage(k)
-        gemm_stage(k)
+    def step(k, rows=None):
+        # the operator through its C-ABI call: activation pass, then the GEMM
+        # (for B <= 128 a dependent launch whose weight loads overlap the first)
+        wk, xk, c, sfk, asc, dn, yk, wsk = sets[k]
+        if rows is None:
+            rb.svdq_linear(wk, xk, bias=bias, out=yk, workspace=wsk)
+        else:
+            rb.svdq_linear(wk, xk[:rows], bias=bias, out=yk[:rows], workspace=wsk)
 
     for i in range(max(args.warmup, R)):
         step(i % R)
@@ -308,52 +327,66 @@ def main():
 
     # one CUDA graph per buffer set holds a whole step (the activation pass and
     # the GEMM with their launches); plain stream launches if capture fails
-    graphs = None
-    try:
-        gs = []
+    def capture_seq(fn, n):
+        """One CUDA graph holding n consecutive calls fn(i), i = 0 .. n-1 (set i % R)."""
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
         with torch.cuda.stream(cap):
-            for k in range(R):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=cap):
-                    step(k)
-                gs.append(g)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(n):
+                    fn(i)
         stream.wait_stream(cap)
-        for k in range(R):
-            gs[k].replay()
+        g.replay()
         torch.cuda.synchronize()
         assert rb.svdq_check_status() == rb.SVDQ_OK
-        graphs = gs
-    except Exception as e:  # noqa: BLE001 - any capture failure falls back to launches
-        print(f"bench: CUDA graph capture unavailable ({type(e).__name__}: {e}); stream launches",
-              file=sys.stderr)
+        return g
+
+    graph_mode = {"ok": True}
+
+    def time_calls(fn, K, sampler=None):
+        """Device time (ms) of K calls fn(i) back to back, set i % R. The calls are
+        captured in CUDA graphs of L calls (L a multiple of R), replayed between one
+        pair of CUDA events, so the host's launch cost is not inside the interval."""
+        L = R * max(1, 64 // R)
+        graphs_ = None
+        if graph_mode["ok"]:
+            try:
+                graphs_ = (capture_seq(fn, min(L, K)), capture_seq(fn, K % L) if K > L and K % L else None)
+            except Exception as e:  # noqa: BLE001 - any capture failure falls back to launches
+                print(f"bench: CUDA graph capture unavailable ({type(e).__name__}: {e}); stream launches",
+                      file=sys.stderr)
+                graph_mode["ok"] = False
+                torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
         torch.cuda.synchronize()
-
-    def run_step(k):
-        if graphs is not None:
-            graphs[k].replay()
+        if sampler is not None:
+            sampler.start()
+            time.sleep(0.2)
+        e0.record(stream)
+        if graphs_ is not None:
+            for _ in range(K // L if K >= L else 1):
+                graphs_[0].replay()
+            if graphs_[1] is not None:
+                graphs_[1].replay()
         else:
-            step(k)
+            for i in range(K):
+                fn(i % R)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.clocks = sampler.stop()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
 
-    sampler = ClockSampler(local)
     K = args.steps
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.2)
-    e_start.record(stream)
-    for i in range(K):
-        run_step(i % R)
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    if world > 1:
-        dist.barrier()
-    total_ms = e_start.elapsed_time(e_end)
+    sampler = ClockSampler(local)
+    total_ms = time_calls(lambda i: step(i % R), K, sampler)
+    clocks = sampler.clocks
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -362,32 +395,29 @@ def main():
     value = world * K * ops_step / (total_ms * 1e-3) / 1e12
     ms_per_step = total_ms / K
 
-    # the GEMM kernel alone, K launches back to back on the rotating sets: its
-    # average launch duration for the roofline line
-    Kg = max(20, min(K, 400))
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    g0.record(stream)
-    for i in range(Kg):
-        gemm_stage(i % R)
-    g1.record(stream)
-    torch.cuda.synchronize()
-    gemm_avg_ms = g0.elapsed_time(g1) / Kg
+    # decode shapes: the shorter batches of the sweep (the first rows of the same
+    # x, same weights and rotation), each timed the same way
+    sweep = None
+    if args.workload.startswith("decode_") and B == 128:
+        sweep = []
+        peaks0, _ = load_peaks()
+        for rows in (1, 16):
+            for i in range(max(args.warmup, R)):
+                step(i % R, rows)
+            torch.cuda.synchronize()
+            us = time_calls(lambda i, rows=rows: step(i % R, rows), K) / K * 1e3
+            byt = alg_bytes(rows, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
+            t_mem = byt / (peaks0["hbm_gbs"] * 1e9)
+            sweep.append({"B": rows, "us_per_step": us, "gbs": byt / (us * 1e-6) / 1e9,
+                          "tops": workload_ops(rows, M, N, r) / (us * 1e-6) / 1e12,
+                          "hbm_roofline_frac": t_mem / (us * 1e-6), "alg_bytes": byt})
+        assert rb.svdq_check_status() == rb.SVDQ_OK
 
-    # per-stage breakdown (diagnostic: an event between the stages drains the
-    # stream, so these include a few microseconds each)
-    Ks = max(10, min(K, 100))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ks)]
-    for i in range(Ks):
-        ev[i][0].record(stream)
-        act_stage(i % R)
-        ev[i][1].record(stream)
-        gemm_stage(i % R)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    act_avg_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / Ks
-    gemm_ev_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / Ks
+    # each stage alone, Ks launches back to back on the rotating sets: the GEMM's
+    # average launch duration is the roofline line's
+    Kg = max(20, min(K, 400))
+    gemm_avg_ms = time_calls(lambda i: gemm_stage(i % R), Kg) / Kg
+    act_avg_ms = time_calls(lambda i: act_stage(i % R), Kg) / Kg
     # the step the parity check reads: set 0 once more
     step(0)
     torch.cuda.synchronize()
@@ -454,6 +484,30 @@ def main():
                                                    ("gemm_pair.cu", "gemm_common.cuh", "ptx.cuh")]) \
         if B > 128 else None
     bytes_step = alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
+    if B <= 128:
+        # short batch: the GEMM streams the weights; its roofline is HBM
+        gb = gemm_alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
+        roof = {"bound": "hbm",
+                "kernel": "skinny_kernel<" + ("NVFP4" if wl.fmt == "nvfp4" else
+                                              ("INT4 packed" if wl.bits <= 4 else "INT8")) +
+                          "> (split-K clusters, residual + bf16 up-projection)",
+                "duration_us": gemm_avg_ms * 1e3,
+                "timing": "Kg launches back to back on rotating sets (CUDA graphs) between one CUDA event pair",
+                "achieved": gb / (gemm_avg_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gb / (gemm_avg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "alg_bytes_per_launch": gb,
+                "peak_source": f"{peak_src} HBM copy bandwidth"}
+    else:
+        roof = {"bound": "tensor",
+                "kernel": "gemm_pair_kernel" + ("<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
+                                                if wl.fmt == "nvfp4" else
+                                                "<INT> (int8 residual + bf16 up-projection)"),
+                "duration_us": gemm_avg_ms * 1e3,
+                "timing": "Kg launches back to back on rotating sets (CUDA graphs) between one CUDA event pair",
+                "achieved": achieved, "peak": lowp_peak, "unit": "TFLOP/s",
+                "frac": achieved / lowp_peak, "traffic": traffic,
+                "peak_source": (f"{peak_src} bf16 GEMM burst x {ratio:g} "
+                                f"(nominal {'fp4' if ratio == 4 else 'int8'}:bf16)")}
     t_rf = max(bytes_step / (peaks["hbm_gbs"] * 1e9),
                (2.0 * B * M * N) / (lowp_peak * 1e12) + (2.0 * B * r * (M + N)) / (peaks["bf16_tflops"] * 1e12))
 
@@ -465,30 +519,23 @@ def main():
         "config": {"workload": args.workload, "B": B, "M": M, "N": N, "rank": r, "fmt": fmt,
                    "x": wl.x_dtype, "y": "bf16", "bias": wl.bias is not None,
                    "l2": f"inputs larger than L2: {R} rotating buffer sets of {bytes_set / 1e6:.0f} MB",
-                   "launch": "CUDA graph per step" if graphs is not None else "stream launches",
+                   "launch": ("CUDA graphs of many steps" if graph_mode["ok"] else "stream launches"),
                    "parallelism": f"replicas{world}"},
         "gbs": bytes_step / (ms_per_step * 1e-3) / 1e9,
         "step_roofline": {"t_roofline_us": t_rf * 1e6, "frac": t_rf / (ms_per_step * 1e-3),
                           "alg_bytes": bytes_step, "ops": ops_step},
-        "stages_ms": {"act": act_avg_ms, "gemm": gemm_ev_ms, "gemm_back_to_back": gemm_avg_ms,
-                      "note": "act/gemm: events around each stage (each includes the drain an event "
-                              "adds); gemm_back_to_back: Kg launches between one event pair"},
-        "roofline": {"bound": "tensor",
-                     "kernel": (("gemm_pair_kernel" if B > 128 else "gemm_kernel") +
-                                ("<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
-                                 if wl.fmt == "nvfp4" else "<INT> (int8 residual + bf16 up-projection)")),
-                     "duration_us": gemm_avg_ms * 1e3,
-                     "timing": "Kg launches back to back on rotating sets between one CUDA event pair",
-                     "achieved": achieved, "peak": lowp_peak, "unit": "TFLOP/s",
-                     "frac": achieved / lowp_peak, "traffic": traffic,
-                     "peak_source": (f"{peak_src} bf16 GEMM burst x {ratio:g} "
-                                     f"(nominal {'fp4' if ratio == 4 else 'int8'}:bf16)")},
+        "stages_ms": {"act": act_avg_ms, "gemm": gemm_avg_ms,
+                      "note": "each stage alone, launched back to back on the rotating sets (CUDA "
+                              "graphs of many launches between one event pair); in a step the GEMM "
+                              "of a short batch overlaps the activation pass (dependent launch)"},
+        "roofline": roof,
         "prepare_ms": prepare_ms,
         "parity": parity,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()), "steps": Ke,
                 "call": "svdq_linear (pinned host x -> device, Y -> pinned host)"},
         "gpu_launches": 2 * K,
+        "sweep": sweep,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:

@@ -79,6 +79,11 @@ typedef struct svdq_fmt {
  *   lu      bf16  [N, 2*rank_pad]    up factor L2^T written twice along the row:
  *           lu[n, j] = lu[n, rank_pad + j] = L2[j, n]
  *   scale   fp32  [M]                the smoothing scale (referenced, not copied)
+ *   codes4  INT with bits <= 4: uint8 [N, M/2], the same codes two per byte
+ *           (element 2j in the low nibble of byte j, two's complement). Nullable:
+ *           the short-batch GEMM (B <= 128) streams this half-size copy from HBM
+ *           when it is there and the int8 codes otherwise; svdq_prepare fills it
+ *           when non-NULL. NULL for NVFP4 and for bits > 4.
  */
 typedef struct svdq_weight {
   int64_t M, N;
@@ -91,11 +96,24 @@ typedef struct svdq_weight {
   void* ld32;
   void* lu;
   const float* scale;
+  void* codes4;
 } svdq_weight;
 
-/* Byte sizes of the svdq_weight buffers, in order: codes, sf, w_scale, ld, ld32, lu. */
+/* Byte sizes of the svdq_weight buffers, in order: codes, sf, w_scale, ld, ld32, lu,
+ * codes4 (0 where a buffer is unused by the format). */
 svdq_status svdq_weight_buffer_sizes(int64_t M, int64_t N, int32_t rank, svdq_fmt fmt,
-                                     size_t sizes[6]);
+                                     size_t sizes[7]);
+
+/*
+ * svdq_pack_int4 - the packed copy of INT codes with bits <= 4 (svdq_weight.codes4):
+ *   packed[n, j] = (codes[n, 2j] & 15) | ((codes[n, 2j + 1] & 15) << 4)
+ *   codes   device int8 [N, M] (values in [-8, 7]), M a positive multiple of 32
+ *   packed  device uint8 [N, M/2]
+ * Stream-ordered, no synchronisation. Layout and packing only: the codes are
+ * those of the "fake_quantize" grid, two per byte.
+ */
+svdq_status svdq_pack_int4(const int8_t* codes, int64_t N, int64_t M, uint8_t* packed,
+                           svdq_stream_t stream);
 
 /* Scratch bytes svdq_prepare needs for this shape (randomized SVD with the given
  * oversampling; <= 0 selects the default of 16). */
@@ -112,7 +130,8 @@ svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq
  *   seed   seeds the Gaussian test matrix of the randomized subspace iteration
  *   oversample, power_iters  <= 0 select the defaults 16 and 4
  *   out    caller-allocated buffers (see svdq_weight); M, N, rank, rank_pad,
- *          fmt and scale are filled in by this call
+ *          fmt and scale are filled in by this call; codes4 (INT, bits <= 4),
+ *          when non-NULL, receives the packed copy of the codes
  *
  * Computes ws = scale[:,None] * W, a rank-r truncated SVD of ws by randomized
  * subspace iteration (Gaussian test matrix, power iterations with Householder

@@ -40,7 +40,7 @@ class SvdqFmt(ctypes.Structure):
 class SvdqWeight(ctypes.Structure):
     _fields_ = [("M", c_i64), ("N", c_i64), ("rank", c_i32), ("rank_pad", c_i32),
                 ("fmt", SvdqFmt), ("codes", c_vp), ("sf", c_vp), ("w_scale", c_vp),
-                ("ld", c_vp), ("ld32", c_vp), ("lu", c_vp), ("scale", c_vp)]
+                ("ld", c_vp), ("ld32", c_vp), ("lu", c_vp), ("scale", c_vp), ("codes4", c_vp)]
 
 
 _SIGS = {
@@ -64,6 +64,7 @@ _SIGS = {
                                      c_vp, c_i32, c_i64, c_vp]),
     "svdq_quantize_act_noalloc": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, SvdqFmt, c_vp, c_vp,
                                           c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "svdq_pack_int4": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_vp]),
     "svdq_check_status": (c_i32, [c_vp]),
     "svdq_selftest_wait_timeout": (c_i32, [c_i64, c_vp]),
 }
@@ -172,6 +173,7 @@ class PreparedWeight:
     ld32: torch.Tensor
     lu: torch.Tensor
     scale: torch.Tensor
+    codes4: Optional[torch.Tensor] = None
 
     @property
     def M(self):
@@ -196,7 +198,7 @@ class PreparedWeight:
 
 def weight_buffer_sizes(M: int, N: int, rank: int, fmt):
     lib = load_library()
-    sizes = (c_sz * 6)()
+    sizes = (c_sz * 7)()
     _check(lib.svdq_weight_buffer_sizes(M, N, rank, parse_fmt(fmt), sizes), "svdq_weight_buffer_sizes")
     return list(sizes)
 
@@ -213,22 +215,37 @@ def allocate_weight(M: int, N: int, rank: int, fmt, scale: torch.Tensor) -> Prep
     ld = torch.zeros((max(rp, 1), M), dtype=torch.bfloat16, device=dev)
     ld32 = torch.zeros((max(rp, 1), M), dtype=torch.float32, device=dev)
     lu = torch.zeros((N, max(2 * rp, 1)), dtype=torch.bfloat16, device=dev)
+    codes4 = torch.empty(sizes[6], dtype=torch.uint8, device=dev) if sizes[6] else None
     d = SvdqWeight(M=M, N=N, rank=rank, rank_pad=rp, fmt=f,
                    codes=codes.data_ptr(), sf=sf.data_ptr() if sf is not None else None,
                    w_scale=w_scale.data_ptr(), ld=ld.data_ptr(), ld32=ld32.data_ptr(),
-                   lu=lu.data_ptr(), scale=scale.data_ptr())
-    return PreparedWeight(d, codes, sf, w_scale, ld, ld32, lu, scale)
+                   lu=lu.data_ptr(), scale=scale.data_ptr(),
+                   codes4=codes4.data_ptr() if codes4 is not None else None)
+    return PreparedWeight(d, codes, sf, w_scale, ld, ld32, lu, scale, codes4)
 
 
-def weight_from_buffers(M, N, rank, fmt, codes, sf, w_scale, ld, ld32, lu, scale) -> PreparedWeight:
+def weight_from_buffers(M, N, rank, fmt, codes, sf, w_scale, ld, ld32, lu, scale,
+                        codes4=None) -> PreparedWeight:
     """Wrap caller-made device buffers (layouts of svdq_weight in include/svdq.h)."""
     f = parse_fmt(fmt)
     rp = (rank + 15) // 16 * 16
     d = SvdqWeight(M=M, N=N, rank=rank, rank_pad=rp, fmt=f, codes=codes.data_ptr(),
                    sf=sf.data_ptr() if sf is not None else None, w_scale=w_scale.data_ptr(),
                    ld=ld.data_ptr(), ld32=ld32.data_ptr() if ld32 is not None else None,
-                   lu=lu.data_ptr(), scale=scale.data_ptr())
-    return PreparedWeight(d, codes, sf, w_scale, ld, ld32, lu, scale)
+                   lu=lu.data_ptr(), scale=scale.data_ptr(),
+                   codes4=codes4.data_ptr() if codes4 is not None else None)
+    return PreparedWeight(d, codes, sf, w_scale, ld, ld32, lu, scale, codes4)
+
+
+def svdq_pack_int4(codes: torch.Tensor) -> torch.Tensor:
+    """INT codes int8 [N, M] -> the packed copy uint8 [N, M // 2] (svdq_weight.codes4)."""
+    lib = load_library()
+    _require_cuda(codes)
+    N, M = codes.shape
+    c = codes.contiguous()
+    out = torch.empty((N, M // 2), dtype=torch.uint8, device=codes.device)
+    _check(lib.svdq_pack_int4(_ptr(c), N, M, _ptr(out), _stream()), "svdq_pack_int4")
+    return out
 
 
 def svdq_prepare(W: torch.Tensor, scale: torch.Tensor, rank: int, fmt="int4", seed: int = 0,
@@ -452,7 +469,7 @@ def svdq_selftest_wait_timeout(limit_us: int = 1000) -> int:
 
 __all__ = [
     "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_act_noalloc",
-    "svdq_quantize_residual", "svdq_linear",
+    "svdq_quantize_residual", "svdq_linear", "svdq_pack_int4",
     "svdq_residual_product_i32", "svdq_residual_linear", "svdq_check_status", "svdq_selftest_wait_timeout",
     "PreparedWeight", "LinearWorkspace", "allocate_weight", "weight_from_buffers",
     "weight_buffer_sizes", "load_library", "header_functions", "parse_fmt",

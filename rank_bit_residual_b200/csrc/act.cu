@@ -27,6 +27,7 @@
 
 #include <algorithm>
 
+#include "encode.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -68,60 +69,6 @@ struct ActArgs {
   float* act_scale;
   unsigned* status;
 };
-
-// ------------------------------------------------------------- small helpers
-__device__ __forceinline__ uint8_t f32_to_ue4m3(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return static_cast<uint8_t>(r & 0xFFu);
-}
-
-// Exact value of a non-negative e4m3 byte (bias 7; exponent 0 is subnormal).
-__device__ __forceinline__ float ue4m3_to_f32(uint8_t b) {
-  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
-  return e == 0 ? static_cast<float>(m) * 0.001953125f  // m * 2^-9
-                : __uint_as_float(((e + 120u) << 23) | (m << 20));
-}
-
-// Eight floats -> eight e2m1 nibbles, element j in nibble j (low nibble first);
-// a code whose magnitude is zero is stored as +0.
-__device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  const uint32_t mag = out & 0x77777777u;
-  const uint32_t nz = (mag + 0x77777777u) & 0x88888888u;
-  return out & (0x77777777u | nz);
-}
-
-__device__ __forceinline__ int64_t sf_swizzle_offset(int64_t row, int64_t col, int64_t kbp) {
-  return ((row >> 7) * (kbp >> 2) + (col >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 +
-         (col & 3);
-}
-
-// 16 bytes of x as floats: 8 bf16 or 4 fp32
-template <typename TIn>
-__device__ __forceinline__ void unpack16(const uint4 u, float* v) {
-  if constexpr (sizeof(TIn) == 2) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = __uint_as_float(w[j] << 16);
-      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  } else {
-    v[0] = __uint_as_float(u.x);
-    v[1] = __uint_as_float(u.y);
-    v[2] = __uint_as_float(u.z);
-    v[3] = __uint_as_float(u.w);
-  }
-}
 
 // Column maxima of |x| over a 128 x 128-byte swizzled tile (work threads only,
 // t < kWork). Thread t owns the
@@ -228,22 +175,6 @@ __device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
     unpack16<TIn>(u[0], v);
     unpack16<TIn>(u[1], v + 4);
   }
-}
-
-// INT codes of 8 elements: rint(fl(x c_k)), packed as 8 bytes. Adding
-// 1.5 * 2^23 rounds an fp32 value below 2^22 in magnitude to the nearest
-// integer, ties to even, and leaves that integer in the low bits of the sum,
-// so the low byte of the sum is the two's-complement code. The clamp to
-// [-qmax, qmax] of the definition is omitted: with s = fl(m / qmax) and
-// c_k = fl(fl(1 / scale_k) fl(1 / s)), every |fl(x c_k)| is at most
-// qmax (1 + 6 * 2^-24) < qmax + 1/2, so no code can leave the range.
-__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8]) {
-  uint32_t f[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) f[j] = __float_as_uint(__fadd_rn(__fmul_rn(v[j], ck[j]), 12582912.0f));
-  const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(f[4], f[5], 0x0040), __byte_perm(f[6], f[7], 0x0040), 0x5410);
-  return make_uint2(lo, hi);
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -745,6 +676,10 @@ int resident_per_sm(size_t smem, bool bf16) {
 }  // namespace
 
 void finish_act_plan(ActPlan& p) {
+  if (p.small) {
+    finish_act_plan_small(p);
+    return;
+  }
   p.nunits = p.nrb * p.ksplit;
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   // hold the unit's x tiles when they fit and every unit gets a CTA of its own
@@ -762,12 +697,24 @@ void finish_act_plan(ActPlan& p) {
   p.nparts = p.grid;
 }
 
-ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt) {
+ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool allow_small) {
   ActPlan p{};
   p.B = B;
   p.M = M;
   p.rank_pad = rank_pad;
   p.bf16 = xdt == SVDQ_BF16;
+  if (allow_small && B <= kActSmallMaxB) {
+    // short batch: one column chunk per SM
+    p.small = 1;
+    p.ksplit = num_sms();
+    finish_act_plan_small(p);
+    if (p.smem <= kActSmallSmemMax) return p;
+    p = ActPlan{};
+    p.B = B;
+    p.M = M;
+    p.rank_pad = rank_pad;
+    p.bf16 = xdt == SVDQ_BF16;
+  }
   p.tile_k = p.bf16 ? 64 : 32;
   p.nrb = static_cast<int>(ceil_div(B, kRows));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
@@ -788,6 +735,10 @@ size_t act_sync_bytes(const ActPlan& p) {
 }
 
 size_t act_scratch_bytes(const ActPlan& p) {
+  if (p.small)
+    return static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * 4, 256)) + 256 +
+           (p.rank_pad > 0 ? static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * p.B * p.rank_pad * 4, 256)) : 0) +
+           256;
   size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));
   b += act_sync_bytes(p);
   if (p.rank_pad > 0)
@@ -802,6 +753,9 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
                        bool* bad_args) {
   *bad_args = false;
   if (p.B == 0) return cudaSuccess;
+  if (p.small)
+    return launch_act_small(p, x, xdt, ldx, scale, fmt, act_global_scale, w_global_scale, ld, codes, sf,
+                            act_scale, down, scratch, stream, bad_args);
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
   Carver cv(scratch, ~size_t(0));
   float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));

@@ -1,0 +1,410 @@
+// act_small.cu - the activation pass for short batches (B <= 128 rows).
+//
+// Same result as the large-batch kernel in act.cu ("SVDQuant Smoothing,
+// Low-rank and Residual Quantization", Formula items 1 and 3; steps 1-2 of
+// "flashinfer.gemm.svdquant_linear"): X_hat = x / scale quantised per tensor
+// (INT) or per 16-element block (NVFP4), and the down-projection x ld^T as
+// bf16 hi | lo. At decode sizes the whole of x is a few hundred KB, so the work
+// is latency-bound: this kernel spreads the columns of x over one CTA per SM,
+// keeps each CTA's column chunk in shared memory across one grid barrier, and
+// uses no TMEM (the down-projection is a handful of warp-level MMAs per CTA).
+//
+//   phase 1  chunk of x -> shared memory; column maxima of |x| times
+//            r_k = fl(1 / scale_k) -> one partial maximum per CTA; partial
+//            down-projection of the chunk -> ws_down[g][b][j]
+//   barrier  (bounded; the counter is zeroed before the launch)
+//   phase 2  per-tensor scale from the partial maxima; codes of the chunk
+//            from the shared copy; each CTA sums its share of the (b, j)
+//            down outputs over the partials in a fixed order
+//
+// fp32 evaluation order of the codes is the one act.cu documents (and the
+// oracle's fp32 code mode repeats): r_k = fl(1 / scale_k), u = fl(1 / s),
+// INT code = rint(fl(x fl(r_k u))); NVFP4 X_hat = fl(x r_k),
+// sf = ue4m3(fl(fl(amax_b / 6) gs)), code = e2m1(fl(X_hat fl(gs / sf))).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "encode.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kZParts = 8;   // threads that share one down output's sum in phase 2
+
+struct SmallArgs {
+  int B, M, wc, G, rank_pad, fmt_kind, qmax, has_ld;
+  int64_t ldx;
+  const void* x;
+  const float* scale;
+  const float* gs_given;
+  const float* gs_w;
+  const void* ld;     // [rank_pad][M], x's dtype
+  float* ws_max;      // [G]
+  float* ws_down;     // [G][B][rank_pad]
+  unsigned* sync;     // [0] barrier counter, [1] abort flag (zeroed before the launch)
+  void* codes;
+  uint8_t* sf;
+  __nv_bfloat16* down;
+  float* act_scale;
+  unsigned* status;
+};
+
+// Row pitch (bytes) of a shared-memory chunk of `wc` elements: 16 bytes of
+// padding make the 8 rows read by one MMA fragment load hit distinct banks.
+__host__ __device__ constexpr int chunk_pitch(int wc, int esz) { return wc * esz + 16; }
+
+// D[16x8] += A[16x16] B[16x8], bf16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D[16x8] += A[16x8] B[8x8], tf32 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(uint32_t f) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__uint_as_float(f)));
+  return r;
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs a) {
+  constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ float red[kWarps];
+  __shared__ int abort_sh;
+
+  pdl_trigger();   // a GEMM launched after this kernel may start its weight loads now
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.x;
+  const int c0 = g * a.wc;
+  const int ncols = min(a.wc, a.M - c0);     // a multiple of 32
+  const int B = a.B;
+  const int bp16 = (B + 15) & ~15;
+  const int pitch = chunk_pitch(a.wc, kEsz);
+  uint8_t* xs = smem;                                               // bp16 rows
+  uint8_t* lds = xs + static_cast<size_t>(bp16) * pitch;            // rank_pad rows
+  float* rcp = reinterpret_cast<float*>(lds + static_cast<size_t>(a.has_ld ? a.rank_pad : 0) * pitch);
+  uint32_t* cm = reinterpret_cast<uint32_t*>(rcp + a.wc);           // kThreads column-max slots
+  if (tid == 0) abort_sh = 0;
+
+  // ------------------------------------------------------------ loads
+  const int vpr = ncols * kEsz / 16;   // 16-byte vectors per chunk row
+  for (int i = tid; i < B * vpr; i += kThreads) {
+    const int r = i / vpr, v = i - r * vpr;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+        static_cast<const uint8_t*>(a.x) + (static_cast<int64_t>(r) * a.ldx + c0) * kEsz) + v);
+    *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = u;
+  }
+  if (a.has_ld) {
+    for (int i = tid; i < (bp16 - B) * vpr; i += kThreads) {   // zero rows up to a multiple of 16
+      const int r = B + i / vpr, v = i % vpr;
+      *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int i = tid; i < a.rank_pad * vpr; i += kThreads) {
+      const int r = i / vpr, v = i - r * vpr;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+          static_cast<const uint8_t*>(a.ld) + (static_cast<int64_t>(r) * a.M + c0) * kEsz) + v);
+      *reinterpret_cast<uint4*>(lds + r * pitch + v * 16) = u;
+    }
+  }
+  for (int k = tid; k < ncols; k += kThreads) rcp[k] = __frcp_rn(__ldg(a.scale + c0 + k));
+  __syncthreads();
+
+  // ------------------------------------------------- column maxima of |x|
+  // thread -> (column, row slice); |x| compared as integers (monotone for
+  // non-negative floats), then fl(colmax r_k)
+  {
+    auto abs_bits = [&](int r, int col) -> uint32_t {
+      if constexpr (kEsz == 2)
+        return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(xs + r * pitch + col * 2) & 0x7FFFu) << 16;
+      else
+        return *reinterpret_cast<const uint32_t*>(xs + r * pitch + col * 4) & 0x7FFFFFFFu;
+    };
+    float run = 0.0f;
+    if (ncols <= kThreads) {
+      const int nsl = kThreads / ncols;
+      uint32_t m = 0u;
+      if (tid < ncols * nsl) {
+        const int col = tid % ncols, sl = tid / ncols;
+        for (int r = sl; r < B; r += nsl) m = max(m, abs_bits(r, col));
+      }
+      cm[tid] = m;
+      __syncthreads();
+      if (tid < ncols) {
+        uint32_t mm = 0u;
+        for (int sl = 0; sl < nsl; ++sl) mm = max(mm, cm[sl * ncols + tid]);
+        run = __fmul_rn(__uint_as_float(mm), rcp[tid]);
+      }
+    } else {
+      for (int col = tid; col < ncols; col += kThreads) {
+        uint32_t m = 0u;
+        for (int r = 0; r < B; ++r) m = max(m, abs_bits(r, col));
+        run = fmaxf(run, __fmul_rn(__uint_as_float(m), rcp[col]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
+    if (lane == 0) red[warp] = run;
+    __syncthreads();
+    if (tid == 0) {
+      float t = red[0];
+      for (int w = 1; w < kWarps; ++w) t = fmaxf(t, red[w]);
+      a.ws_max[g] = t;
+    }
+  }
+
+  // ------------------------------------------- partial down-projection
+  // 16 x 8 output tiles (rows b, factor columns j) spread over the warps; the
+  // chunk's columns are the K of each tile's MMA chain
+  if (a.has_ld) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const int mt = bp16 / 16, nt = a.rank_pad / 8;
+    for (int t = warp; t < mt * nt; t += kWarps) {
+      const int b0 = (t / nt) * 16, j0 = (t % nt) * 8;
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const uint8_t* xa = xs + (b0 + gid) * pitch;
+      const uint8_t* xb = xa + 8 * pitch;
+      const uint8_t* lb = lds + (j0 + gid) * pitch;
+      if constexpr (kEsz == 2) {
+        for (int k = 0; k < ncols; k += 16) {
+          const int o0 = (k + 2 * tig) * 2, o1 = o0 + 16;
+          const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(xa + o0), *reinterpret_cast<const uint32_t*>(xb + o0),
+                                  *reinterpret_cast<const uint32_t*>(xa + o1), *reinterpret_cast<const uint32_t*>(xb + o1)};
+          const uint32_t bf[2] = {*reinterpret_cast<const uint32_t*>(lb + o0), *reinterpret_cast<const uint32_t*>(lb + o1)};
+          mma_bf16_16816(d, af, bf);
+        }
+      } else {
+        for (int k = 0; k < ncols; k += 8) {
+          const int o0 = (k + tig) * 4, o1 = o0 + 16;
+          const uint32_t af[4] = {to_tf32(*reinterpret_cast<const uint32_t*>(xa + o0)),
+                                  to_tf32(*reinterpret_cast<const uint32_t*>(xb + o0)),
+                                  to_tf32(*reinterpret_cast<const uint32_t*>(xa + o1)),
+                                  to_tf32(*reinterpret_cast<const uint32_t*>(xb + o1))};
+          const uint32_t bf[2] = {to_tf32(*reinterpret_cast<const uint32_t*>(lb + o0)),
+                                  to_tf32(*reinterpret_cast<const uint32_t*>(lb + o1))};
+          mma_tf32_1688(d, af, bf);
+        }
+      }
+      const int r0 = b0 + gid, r1 = r0 + 8, j = j0 + 2 * tig;
+      float* base = a.ws_down + static_cast<int64_t>(g) * B * a.rank_pad;
+      if (r0 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r0) * a.rank_pad + j) = make_float2(d[0], d[1]);
+      if (r1 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r1) * a.rank_pad + j) = make_float2(d[2], d[3]);
+    }
+  }
+
+  // ================================================================ barrier
+  GridSync gsync{a.sync, a.sync + 1, a.status, 0u};
+  if (!grid_sync(gsync, &abort_sh)) return;
+
+  // ================================================================ phase 2
+  float m = 0.0f;
+  for (int i = tid; i < a.G; i += kThreads) m = fmaxf(m, __ldcg(a.ws_max + i));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = red[0];
+  for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w]);
+  const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
+  float u = 0.0f, gs_x = 1.0f;
+  if (nv) {
+    gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
+    if (g == 0 && tid == 0) *a.act_scale = gs_x;
+  } else {
+    const float s = __fdiv_rn(m, static_cast<float>(a.qmax));
+    u = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    if (g == 0 && tid == 0) *a.act_scale = s;
+  }
+
+  constexpr int kPer16 = 16 / kEsz;   // elements per 16 bytes
+  if (!nv) {
+    // 8 codes per item: one 8-byte store
+    const int per_row = ncols / 8;
+    for (int i = tid; i < B * per_row; i += kThreads) {
+      const int r = i / per_row, c8 = (i - r * per_row) * 8;
+      float v[8], ck[8];
+#pragma unroll
+      for (int h = 0; h < 8 / kPer16; ++h)
+        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c8 + h * kPer16) * kEsz), v + h * kPer16);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ck[j] = __fmul_rn(rcp[c8 + j], u);
+      *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(r) * a.M + c0 + c8) =
+          int_codes8(v, ck);
+    }
+  } else {
+    // one 16-element block per item: a scale byte and 8 code bytes
+    const int per_row = ncols / 16;
+    const int64_t kbp = (a.M / 16 + 3) / 4 * 4;
+    for (int i = tid; i < B * per_row; i += kThreads) {
+      const int r = i / per_row, c16 = (i - r * per_row) * 16;
+      float v[16];
+#pragma unroll
+      for (int h = 0; h < 16 / kPer16; ++h)
+        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c16 + h * kPer16) * kEsz), v + h * kPer16);
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[j] = __fmul_rn(v[j], rcp[c16 + j]);
+        amax = fmaxf(amax, fabsf(v[j]));
+      }
+      const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+      const float dsf = ue4m3_to_f32(sfb);
+      const float enc = dsf > 0.0f ? __fdiv_rn(gs_x, dsf) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], enc);
+      const int64_t col = c0 + c16;
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(r) * (a.M / 2) + col / 2) =
+          make_uint2(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8));
+      a.sf[sf_swizzle_offset(r, col / 16, kbp)] = sfb;
+    }
+    // zero the scale padding: rows B..127 of every scale column, and the
+    // columns past M / 16 (up to a multiple of 4) of rows < B
+    const int64_t kb = a.M / 16;
+    const int64_t pad_cols = kbp - kb;
+    const int64_t n_pad = (128 - B) * kbp + static_cast<int64_t>(B) * pad_cols;
+    for (int64_t i = static_cast<int64_t>(g) * kThreads + tid; i < n_pad; i += static_cast<int64_t>(a.G) * kThreads) {
+      int64_t row, c;
+      if (i < static_cast<int64_t>(B) * pad_cols) {
+        row = i / pad_cols;
+        c = kb + (i - row * pad_cols);
+      } else {
+        const int64_t j = i - static_cast<int64_t>(B) * pad_cols;
+        row = B + j / kbp;
+        c = j - (j / kbp) * kbp;
+      }
+      a.sf[sf_swizzle_offset(row, c, kbp)] = 0;
+    }
+  }
+
+  // down: this CTA's share of the B * rank_pad outputs; kZParts threads split
+  // the G partials of one output (partial z to thread z % kZParts) and their
+  // sums are added in thread order: a fixed summation order
+  if (a.has_ld) {
+    const int total = B * a.rank_pad;
+    const int lo = static_cast<int>((static_cast<int64_t>(total) * g) / a.G);
+    const int hi = static_cast<int>((static_cast<int64_t>(total) * (g + 1)) / a.G);
+    const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
+    const int zp = tid % kZParts;
+    const int64_t stride = static_cast<int64_t>(B) * a.rank_pad;
+    for (int base = lo; base < hi; base += kThreads / kZParts) {
+      const int idx = base + tid / kZParts;
+      float acc = 0.0f;
+      if (idx < hi)
+        for (int z = zp; z < a.G; z += kZParts) acc += __ldcg(a.ws_down + z * stride + idx);
+      // fixed-order combine of the kZParts partial sums (lanes zp = 0..7 of a group)
+#pragma unroll
+      for (int o = 1; o < kZParts; o <<= 1) {
+        const float other = __shfl_down_sync(0xffffffffu, acc, o);
+        if ((zp & (2 * o - 1)) == 0) acc += other;
+      }
+      if (zp == 0 && idx < hi) {
+        acc = __fmul_rn(acc, mult);
+        const int b = idx / a.rank_pad, j = idx - b * a.rank_pad;
+        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
+        const __nv_bfloat16 l = __float2bfloat16_rn(acc - __bfloat162float(h));
+        a.down[static_cast<int64_t>(b) * 2 * a.rank_pad + j] = h;
+        a.down[static_cast<int64_t>(b) * 2 * a.rank_pad + a.rank_pad + j] = l;
+      }
+    }
+  }
+}
+
+size_t small_smem(const ActPlan& p, bool has_ld) {
+  const int esz = p.bf16 ? 2 : 4;
+  const int bp16 = static_cast<int>(round_up(p.B, 16));
+  return static_cast<size_t>(bp16 + (has_ld ? p.rank_pad : 0)) * chunk_pitch(p.wc, esz) +
+         static_cast<size_t>(p.wc) * 4 + kThreads * 4 + 64;
+}
+
+}  // namespace
+
+void finish_act_plan_small(ActPlan& p) {
+  p.wc = static_cast<int>(round_up(ceil_div(p.M, std::max(p.ksplit, 1)), 32));
+  p.grid = static_cast<int>(ceil_div(p.M, p.wc));
+  p.ksplit = p.grid;
+  p.nunits = p.grid;
+  p.nparts = p.grid;
+  p.hold = 1;
+  p.xbuf = 0;
+  p.smem = small_smem(p, p.rank_pad > 0);
+}
+
+cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
+                             const float* scale, svdq_fmt fmt, const float* act_global_scale,
+                             const float* w_global_scale, const void* ld, void* codes, void* sf,
+                             float* act_scale, void* down, void* scratch, cudaStream_t stream,
+                             bool* bad_args) {
+  *bad_args = false;
+  const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
+  const int esz = xdt == SVDQ_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (ldx * esz) % 16 ||
+      (has_ld && (reinterpret_cast<uintptr_t>(ld) & 15))) {
+    *bad_args = true;
+    return cudaSuccess;
+  }
+  Carver cv(scratch, ~size_t(0));
+  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * 4));
+  unsigned* sync = static_cast<unsigned*>(cv.take(256));
+  float* ws_down = has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * p.B * p.rank_pad * 4))
+                          : nullptr;
+  cudaError_t err = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), stream);
+  if (err != cudaSuccess) return err;
+  SmallArgs a{};
+  a.B = static_cast<int>(p.B);
+  a.M = static_cast<int>(p.M);
+  a.wc = p.wc;
+  a.G = p.grid;
+  a.rank_pad = has_ld ? p.rank_pad : 0;
+  a.fmt_kind = fmt.kind;
+  a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
+  a.has_ld = has_ld ? 1 : 0;
+  a.ldx = ldx;
+  a.x = x;
+  a.scale = scale;
+  a.gs_given = fmt.kind == SVDQ_KIND_NVFP4 ? act_global_scale : nullptr;
+  a.gs_w = fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr;
+  a.ld = has_ld ? ld : nullptr;
+  a.ws_max = ws_max;
+  a.ws_down = ws_down;
+  a.sync = sync;
+  a.codes = codes;
+  a.sf = static_cast<uint8_t*>(sf);
+  a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
+  a.act_scale = act_scale;
+  a.status = device_status_word();
+  const size_t smem = small_smem(p, has_ld);
+  void* args[] = {&a};
+  if (xdt == SVDQ_BF16) {
+    err = cudaFuncSetAttribute(act_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<__nv_bfloat16>), dim3(p.grid),
+                                       dim3(kThreads), args, smem, stream);
+  }
+  err = cudaFuncSetAttribute(act_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<float>), dim3(p.grid),
+                                     dim3(kThreads), args, smem, stream);
+}
+
+}  // namespace svdq

@@ -144,7 +144,9 @@ svdq_status check_weight(const svdq_weight* w) {
   if (!w->codes || !w->w_scale || !w->scale) return SVDQ_EINVAL;
   if (w->fmt.kind == SVDQ_KIND_NVFP4 && !w->sf) return SVDQ_EINVAL;
   if (w->rank > 0 && (!w->ld || !w->lu)) return SVDQ_EINVAL;
+  if (w->codes4 && (w->fmt.kind != SVDQ_KIND_INT || w->fmt.bits > 4)) return SVDQ_EINVAL;
   if (!aligned16(w->codes) || !aligned16(w->scale) || (w->ld && !aligned16(w->ld)) ||
+      (w->codes4 && !aligned16(w->codes4)) ||
       (w->lu && !aligned16(w->lu)) || (w->ld32 && !aligned16(w->ld32)))
     return SVDQ_EUNSUPPORTED;
   return SVDQ_OK;
@@ -210,7 +212,7 @@ const char* svdq_status_string(svdq_status s) {
 }
 
 svdq_status svdq_weight_buffer_sizes(int64_t M, int64_t N, int32_t rank, svdq_fmt fmt,
-                                     size_t sizes[6]) {
+                                     size_t sizes[7]) {
   if (!sizes) return SVDQ_EINVAL;
   const svdq_status s = check_shape(M, N, rank, fmt);
   if (s != SVDQ_OK) return s;
@@ -221,7 +223,15 @@ svdq_status svdq_weight_buffer_sizes(int64_t M, int64_t N, int32_t rank, svdq_fm
   sizes[3] = static_cast<size_t>(rp * M * 2);
   sizes[4] = static_cast<size_t>(rp * M * 4);
   sizes[5] = static_cast<size_t>(N * 2 * rp * 2);
+  sizes[6] = fmt.kind == SVDQ_KIND_INT && fmt.bits <= 4 ? static_cast<size_t>(N * M / 2) : 0;
   return SVDQ_OK;
+}
+
+svdq_status svdq_pack_int4(const int8_t* codes, int64_t N, int64_t M, uint8_t* packed,
+                           svdq_stream_t stream) {
+  if (N <= 0 || M <= 0 || !codes || !packed) return SVDQ_EINVAL;
+  if (M % 32 != 0 || !aligned16(codes) || !aligned16(packed)) return SVDQ_EUNSUPPORTED;
+  return from_cuda(launch_pack_int4(codes, N, M, packed, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq_fmt fmt,
@@ -348,11 +358,11 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
   if (e != cudaSuccess) return SVDQ_ECUDA;
   if (w->fmt.kind == SVDQ_KIND_INT) {
     e = launch_gemm_int(w, static_cast<const int8_t*>(c.codes), c.act_scale,
-                        w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, false, st, &bad);
+                        w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, false, true, st, &bad);
   } else {
     e = launch_gemm_nvfp4(w, static_cast<const uint8_t*>(c.codes),
                           static_cast<const uint8_t*>(c.sf), c.act_scale,
-                          w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, st, &bad);
+                          w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, true, st, &bad);
   }
   if (bad) return SVDQ_EUNSUPPORTED;
   return from_cuda(e);
@@ -376,11 +386,11 @@ svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, co
   cudaError_t e;
   if (w->fmt.kind == SVDQ_KIND_INT)
     e = launch_gemm_int(w, static_cast<const int8_t*>(act_codes), act_scale,
-                        w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, st, &bad);
+                        w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, false, st, &bad);
   else
     e = launch_gemm_nvfp4(w, static_cast<const uint8_t*>(act_codes),
                           static_cast<const uint8_t*>(act_sf), act_scale,
-                          w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, st, &bad);
+                          w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, st, &bad);
   if (bad) return SVDQ_EUNSUPPORTED;
   return from_cuda(e);
 }
@@ -396,7 +406,7 @@ svdq_status svdq_residual_product_i32(const svdq_weight* w, const int8_t* act_co
   if (!aligned16(act_codes)) return SVDQ_EUNSUPPORTED;
   bool bad = false;
   const cudaError_t e = launch_gemm_int(w, act_codes, nullptr, nullptr, B, nullptr, acc, SVDQ_F32,
-                                        ldacc, true, reinterpret_cast<cudaStream_t>(stream), &bad);
+                                        ldacc, true, false, reinterpret_cast<cudaStream_t>(stream), &bad);
   if (bad) return SVDQ_EUNSUPPORTED;
   return from_cuda(e);
 }

@@ -276,7 +276,7 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
 template <int kKind>
 cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8_t* act_sf,
                         const float* s_x, const void* down2, int64_t B, const void* bias, void* y,
-                        svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                        svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
                         bool* bad_args) {
   *bad_args = false;
   if (B == 0) return cudaSuccess;
@@ -325,6 +325,15 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
     *bad_args = true;
     return cudaSuccess;
   }
+  {
+    // short batch: split-K clusters over all SMs (gemm_skinny.cu)
+    cudaError_t err = cudaSuccess;
+    const int out = raw_i32 ? kOutI32 : (ydt == SVDQ_F32 ? kOutF32 : kOutBF16);
+    if (launch_gemm_skinny(kKind, out, args, act_codes, act_sf, has_lr ? down2 : nullptr, w, pdl, stream, &err))
+      return err;
+    *bad_args = true;
+    return cudaSuccess;
+  }
   const int64_t tiles = ceil_div(B, kBM) * ceil_div(N, kBN);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   if (raw_i32) {
@@ -343,22 +352,22 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
 
 cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
                             const void* down2, int64_t B, const void* bias, void* y,
-                            svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                            svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
                             bool* bad_args) {
-  return launch_gemm<kKindInt>(w, act_codes, nullptr, s_x, down2, B, bias, y, ydt, ldy, raw_i32,
+  return launch_gemm<kKindInt>(w, act_codes, nullptr, s_x, down2, B, bias, y, ydt, ldy, raw_i32, pdl,
                                stream, bad_args);
 }
 
 cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
                               const uint8_t* act_sf, const float* gs_x, const void* down2,
                               int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                              int64_t ldy, cudaStream_t stream, bool* bad_args) {
+                              int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args) {
   if (!act_sf || !w->sf || (reinterpret_cast<uintptr_t>(act_sf) & 15) ||
       (reinterpret_cast<uintptr_t>(w->sf) & 15)) {
     *bad_args = true;
     return cudaSuccess;
   }
-  return launch_gemm<kKindNvfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false,
+  return launch_gemm<kKindNvfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false, pdl,
                                  stream, bad_args);
 }
 

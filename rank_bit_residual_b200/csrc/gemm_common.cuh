@@ -194,6 +194,13 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& args, uint32_t la
   }
 }
 
+// Host: the short-batch kernel (gemm_skinny.cu, B <= 128); false if a tensor map
+// cannot be encoded. pdl: launch with programmatic serialization (only right
+// after this library's activation pass, which writes nothing the weight loads read).
+bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_codes, const uint8_t* act_sf,
+                        const void* down2, const svdq_weight* w, bool pdl, cudaStream_t stream,
+                        cudaError_t* err);
+
 // Host: the CTA-pair kernel (gemm_pair.cu); false if a tensor map cannot be encoded.
 bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
                       const void* down2, const svdq_weight* w, cudaStream_t stream,

@@ -1,0 +1,621 @@
+// gemm_skinny.cu - the residual GEMM with the low-rank epilogue for short
+// batches (B <= 128 rows), where the weight stream from HBM is the cost.
+//
+// "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula item 3:
+//   Y = (X_hat L1) L2 + Q(X_hat) Q(R)
+// from prepared operands (step 3 of "flashinfer.gemm.svdquant_linear": the
+// residual GEMM with the low-rank up-projection and bias in its epilogue).
+//
+// Orientation: the weight rows are the MMA's M side (128 per tile) and the
+// batch is its N side (Bp = B rounded up to 16), so a batch of one wastes no
+// tensor-core rows:  D[n, b] = sum_k W[n, k] X[b, k].
+// Each 128-row weight tile is one cluster of S CTAs that split K; every CTA
+// sees only 1/S of the tile's weights, so all SMs stream weights at once.
+// The partial tiles are combined through distributed shared memory: each CTA
+// stores its partial of the output columns owned by CTA p straight into p's
+// shared memory, and p sums the S partials in rank order (a fixed order) and
+// writes Y.
+//
+// Weights are loaded before griddepcontrol.wait: launched with programmatic
+// serialization right after the activation pass, the weight stream overlaps
+// that kernel; only the activation-side loads and the epilogue wait for it.
+//
+// Formats:
+//   INT, int8 codes     A tiles come by TMA (128-byte swizzle)       kind::i8
+//   INT, packed 4-bit   64-byte packed rows by TMA, widened to int8 in shared
+//                       memory by the epilogue warps                 kind::i8
+//   NVFP4               e2m1 tiles by TMA, ue4m3 scales by bulk copy
+//                       then tcgen05.cp to TMEM                      kind::mxf4nvf4
+// Low-rank branch: lu (weight side) x down hi|lo (batch side), kind::f16, in
+// 64-wide K boxes spread over the cluster's CTAs; INT keeps it in its own fp32
+// accumulator, NVFP4 adds it to the residual accumulator (down is pre-scaled
+// by gs_x gs_w).
+//
+// Warps: 0 weight loads, 1 activation loads, 2 TMEM + MMA issue,
+//        3-6 widening of packed codes, then the epilogue (TMEM lane quarter w % 4).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "gemm_common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kTileN = 128;
+constexpr int kThreads = 224;
+constexpr int kWarpW = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi0 = 3;
+constexpr int kMaxRing = 8;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kLrCol = 128;                      // INT: low-rank fp32 accumulator
+constexpr uint32_t kSfaCol = 128, kSfbCol = 144;      // NVFP4: scale factors (4 columns per MMA)
+constexpr int kATile = 16384;                         // 128 rows x 128 bytes
+constexpr int kPSlot = 8192;                          // 128 rows x 64 packed bytes
+constexpr int kSfBytes = 2048;                        // 4 scale atoms of 512 bytes
+constexpr size_t kSmemBudget = 200 * 1024;
+constexpr size_t kMinSmem = 120 * 1024;
+
+enum SkinnyFmt { kFmtInt8 = 0, kFmtInt4 = 1, kFmtNvfp4 = 2 };
+
+struct SkinnyArgs {
+  int B, Bp, N, M, S, kst, lr_boxes, sh;
+  int da, db, dp, a_slot, b_slot;
+  int katoms;
+  const float* s_x;
+  const float* s_w;
+  const __nv_bfloat16* bias;
+  void* y;
+  int64_t ldy;
+  int vec_ok;
+  const uint8_t* sfw;   // NVFP4 weight scales, 128x4 layout
+  const uint8_t* sfx;   // NVFP4 activation scales, 128x4 layout
+  unsigned* status;
+};
+
+// 16 packed bytes (32 two's-complement nibbles, element 2j in the low nibble
+// of byte j) -> 32 int8 codes in element order.
+__device__ __forceinline__ void widen_int4(const uint4 v, uint32_t (&o)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo = w[i] & 0x0F0F0F0Fu;          // elements 8i + 0, 2, 4, 6
+    uint32_t hi = (w[i] >> 4) & 0x0F0F0F0Fu;   // elements 8i + 1, 3, 5, 7
+    lo |= (lo & 0x08080808u) * 0x1Eu;          // sign-extend each nibble to its byte
+    hi |= (hi & 0x08080808u) * 0x1Eu;
+    o[2 * i] = __byte_perm(lo, hi, 0x5140);
+    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+}
+
+// Dequantisation factor of the residual accumulator (s_x s_w for INT,
+// 1 / (gs_x gs_w) for NVFP4; unused for the raw int32 product).
+template <int kFmt, int kOut>
+__device__ __forceinline__ float skinny_alpha(const SkinnyArgs& a) {
+  if (kOut == kOutI32) return 0.0f;
+  if (kFmt == kFmtNvfp4) return __fdiv_rn(1.0f, __fmul_rn(__ldg(a.s_x), __ldg(a.s_w)));
+  return __ldg(a.s_x) * __ldg(a.s_w);
+}
+
+template <int kFmt, int kOut>
+__global__ void __launch_bounds__(kThreads, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                  const __grid_constant__ CUtensorMap tm_lu, const __grid_constant__ CUtensorMap tm_dn,
+                  const SkinnyArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_a[kMaxRing];
+  __shared__ __align__(8) uint64_t empty_a[kMaxRing];
+  __shared__ __align__(8) uint64_t full_b[kMaxRing];
+  __shared__ __align__(8) uint64_t empty_b[kMaxRing];
+  __shared__ __align__(8) uint64_t full_p[kMaxRing];
+  __shared__ __align__(8) uint64_t empty_p[kMaxRing];
+  __shared__ __align__(8) uint64_t tmem_full;
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* ring_a = smem;
+  uint8_t* ring_b = ring_a + static_cast<size_t>(a.da) * a.a_slot;
+  uint8_t* ring_p = ring_b + static_cast<size_t>(a.db) * a.b_slot;
+  uint32_t* recv = reinterpret_cast<uint32_t*>(smem);   // reuses the rings once every MMA is done
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int n0 = blockIdx.y * kTileN;
+  const int k_lo = (a.kst * rank) / S, k_hi = (a.kst * (rank + 1)) / S;
+  const int nres = k_hi - k_lo;
+  const int nlr = a.lr_boxes > rank ? (a.lr_boxes - rank + S - 1) / S : 0;  // boxes rank, rank + S, ...
+  const int nsteps = nlr + nres;
+  unsigned* status = a.status;
+  constexpr uint32_t kFullACount = kFmt == kFmtInt4 ? 4u : 1u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMaxRing; ++s) {
+      mbar_init(&full_a[s], kFullACount);
+      mbar_init(&empty_a[s], 1);
+      mbar_init(&full_b[s], 1);
+      mbar_init(&empty_b[s], 1);
+      mbar_init(&full_p[s], 1);
+      mbar_init(&empty_p[s], 4);
+    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&mma_done, 1);
+    fence_mbar_init();
+    abort_sh = 0;
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+    if (a.lr_boxes) {
+      tma_prefetch_desc(&tm_lu);
+      tma_prefetch_desc(&tm_dn);
+    }
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == kWarpW) {
+    // ---------------------------------------------------- weight producer
+    if (lane == 0) {
+      bool ok = true;
+      int ia = 0, ip = 0;   // A-ring loads (lu boxes, direct weight tiles) and packed loads issued
+      // low-rank step i (< nlr): the lu box rank + i S into A slot i % da
+      auto load_lu = [&](int i) {
+        const int s = i % a.da;
+        if (i >= a.da) ok = ok && mbar_wait(&empty_a[s], ((i / a.da) - 1) & 1, status, &abort_sh);
+        if (!ok) return;
+        mbar_arrive_expect_tx(&full_a[s], kATile);
+        for (uint32_t c = 1; c < kFullACount; ++c) mbar_arrive(&full_a[s]);
+        tma_load_2d(ring_a + static_cast<size_t>(s) * a.a_slot, &tm_lu, &full_a[s], 64 * (rank + i * S), n0);
+        ++ia;
+      };
+      if constexpr (kFmt == kFmtInt4) {
+        // packed residual step r into P slot r % dp; the first dp go out before
+        // anything can block
+        auto load_p = [&](int r) {
+          const int s = r % a.dp;
+          if (r >= a.dp) ok = ok && mbar_wait(&empty_p[s], ((r / a.dp) - 1) & 1, status, &abort_sh);
+          if (!ok) return;
+          mbar_arrive_expect_tx(&full_p[s], kPSlot);
+          tma_load_2d(ring_p + static_cast<size_t>(s) * kPSlot, &tm_w, &full_p[s], 64 * (k_lo + r), n0);
+          ++ip;
+        };
+        int r = 0;
+        for (; r < min(a.dp, nres) && ok; ++r) load_p(r);
+        for (int i = 0; i < nlr && ok; ++i) load_lu(i);
+        for (; r < nres && ok; ++r) load_p(r);
+      } else {
+        for (int i = 0; i < nsteps && ok; ++i) {
+          if (i < nlr) {
+            load_lu(i);
+            continue;
+          }
+          const int s = i % a.da, k = k_lo + (i - nlr);
+          if (i >= a.da) ok = ok && mbar_wait(&empty_a[s], ((i / a.da) - 1) & 1, status, &abort_sh);
+          if (!ok) break;
+          uint8_t* dst = ring_a + static_cast<size_t>(s) * a.a_slot;
+          if constexpr (kFmt == kFmtNvfp4) {
+            const int na = min(4, a.katoms - 4 * k);
+            mbar_arrive_expect_tx(&full_a[s], kATile + na * 512);
+            tma_load_2d(dst, &tm_w, &full_a[s], 128 * k, n0);
+            bulk_load(dst + kATile, a.sfw + (static_cast<int64_t>(n0 / 128) * a.katoms + 4 * k) * 512, na * 512,
+                      &full_a[s]);
+          } else {
+            mbar_arrive_expect_tx(&full_a[s], kATile);
+            tma_load_2d(dst, &tm_w, &full_a[s], 128 * k, n0);
+          }
+          ++ia;
+        }
+      }
+      if (!ok) {
+        // the MMAs will not consume what is in flight: let it land before the
+        // block can exit (on the normal path every load was consumed)
+        abort_sh = 1;
+        if (kFmt != kFmtInt4)
+          for (int q = max(0, ia - a.da); q < ia; ++q)
+            mbar_wait(&full_a[q % a.da], (q / a.da) & 1, status, nullptr, 1000000ull);
+        for (int q = max(0, ip - a.dp); q < ip; ++q)
+          mbar_wait(&full_p[q % a.dp], (q / a.dp) & 1, status, nullptr, 1000000ull);
+      }
+    }
+  } else if (warp == kWarpX) {
+    // ------------------------------------------------ activation producer
+    if (lane == 0) {
+      pdl_wait();   // codes, scales and down come from the activation pass
+      bool ok = true;
+      int ib = 0;   // loads issued
+      const int xbytes = a.Bp * 128;
+      for (int i = 0; i < nsteps && ok; ++i, ++ib) {
+        const int s = i % a.db;
+        if (i >= a.db) ok = mbar_wait(&empty_b[s], ((i / a.db) - 1) & 1, status, &abort_sh);
+        if (!ok) break;
+        uint8_t* dst = ring_b + static_cast<size_t>(s) * a.b_slot;
+        if (i < nlr) {
+          mbar_arrive_expect_tx(&full_b[s], xbytes);
+          tma_load_2d(dst, &tm_dn, &full_b[s], 64 * (rank + i * S), 0);
+        } else {
+          const int k = k_lo + (i - nlr);
+          if constexpr (kFmt == kFmtNvfp4) {
+            const int na = min(4, a.katoms - 4 * k);
+            mbar_arrive_expect_tx(&full_b[s], xbytes + na * 512);
+            tma_load_2d(dst, &tm_x, &full_b[s], 128 * k, 0);
+            bulk_load(dst + xbytes, a.sfx + static_cast<int64_t>(4 * k) * 512, na * 512, &full_b[s]);
+          } else {
+            mbar_arrive_expect_tx(&full_b[s], xbytes);
+            tma_load_2d(dst, &tm_x, &full_b[s], 128 * k, 0);
+          }
+        }
+      }
+      if (!ok) {
+        abort_sh = 1;
+        for (int q = max(0, ib - a.db); q < ib; ++q)
+          mbar_wait(&full_b[q % a.db], (q / a.db) & 1, status, nullptr, 1000000ull);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_i8 = idesc_i8(kTileN, a.Bp);
+      const uint32_t id_bf = idesc_bf16(kTileN, a.Bp);
+      const uint32_t id_f4 = idesc_nvf4(kTileN, a.Bp);
+      const uint32_t lr_acc = kFmt == kFmtNvfp4 ? tmem : tmem + kLrCol;
+      {
+        // throwaway MMA: the first tcgen05.mma of a kernel completes microseconds
+        // after the rest; issued now it overlaps the first loads (the first real
+        // MMA overwrites its accumulator)
+        const uint64_t d0 = smem_desc_sw128(smem_u32(smem));
+        if constexpr (kFmt == kFmtNvfp4)
+          mma_nvf4(tmem, d0, d0, id_f4, 0u, tmem + kSfaCol, tmem + kSfbCol);
+        else
+          mma_i8(tmem, d0, d0, id_i8, 0u);
+      }
+      bool ok = true;
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int sa = i % a.da, sb = i % a.db;
+        ok = mbar_wait(&full_a[sa], (i / a.da) & 1, status, &abort_sh) &&
+             mbar_wait(&full_b[sb], (i / a.db) & 1, status, &abort_sh);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(ring_a + static_cast<size_t>(sa) * a.a_slot);
+        const uint32_t b0 = smem_u32(ring_b + static_cast<size_t>(sb) * a.b_slot);
+        if (i < nlr) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(lr_acc, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_bf,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+        } else {
+          const int r = i - nlr;
+          if constexpr (kFmt == kFmtNvfp4) {
+            const int k = k_lo + r;
+            const int na = min(4, a.katoms - 4 * k);
+            const uint32_t sfa_s = a0 + kATile;
+            const uint32_t sfb_s = b0 + a.Bp * 128;
+            // tcgen05.cp and tcgen05.mma from one thread execute in order, so
+            // the scale columns can be refilled every step
+            for (int kk = 0; kk < na; ++kk) {
+              tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * kk, smem_desc_plain(sfa_s + 512 * kk));
+              tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4 * kk, smem_desc_plain(sfb_s + 512 * kk));
+            }
+            for (int kk = 0; kk < na; ++kk)
+              mma_nvf4(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
+                       (i > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 4 * kk);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_i8(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_i8,
+                     (r > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&empty_a[sa]);
+        mma_commit(&empty_b[sb]);
+      }
+      if (ok) mma_commit(&tmem_full);
+      if (!ok) abort_sh = 1;
+      // every MMA issued so far has completed before TMEM can be released
+      mma_commit(&mma_done);
+      mbar_wait(&mma_done, 0, status, nullptr);
+    }
+  } else {
+    // ------------------------------------------- widening of packed codes
+    if constexpr (kFmt == kFmtInt4) {
+      const int t = (warp - kWarpEpi0) * 32 + lane;   // 0..127
+      bool ok = true;
+      for (int r = 0; r < nres && ok; ++r) {
+        const int ps = r % a.dp, i = nlr + r, as = i % a.da;
+        ok = mbar_wait_warp(&full_p[ps], (r / a.dp) & 1, status, &abort_sh);
+        if (ok && i >= a.da) ok = mbar_wait_warp(&empty_a[as], ((i / a.da) - 1) & 1, status, &abort_sh);
+        if (!ok) break;
+        const uint8_t* src = ring_p + static_cast<size_t>(ps) * kPSlot;
+        uint8_t* dst = ring_a + static_cast<size_t>(as) * a.a_slot;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int idx = t + 128 * it;            // 16-byte piece of the packed tile
+          const int row = idx >> 2, q = idx & 3;   // row, quarter of its 64 bytes
+          const uint4 v = *reinterpret_cast<const uint4*>(src + row * 64 + q * 16);
+          uint32_t o[8];
+          widen_int4(v, o);
+          uint8_t* drow = dst + row * 128;
+          *reinterpret_cast<uint4*>(drow + (((2 * q) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(drow + (((2 * q + 1) ^ (row & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full_a[as]);
+          mbar_arrive(&empty_p[ps]);
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ epilogue
+  const bool epi = warp >= kWarpEpi0;
+  float alpha = 0.0f;
+  bool fin = false;
+  if (epi) {
+    fin = mbar_wait_warp(&tmem_full, 0, status, &abort_sh);
+    tc_fence_after();
+    pdl_wait();   // the activation scale comes from the activation pass
+    alpha = skinny_alpha<kFmt, kOut>(a);
+  }
+  // every CTA of the cluster is past its MMAs: the rings are free for the partials
+  __syncwarp();
+  cluster_sync();
+  if (epi && fin) {
+    const int q = warp & 3;
+    const int nloc = q * 32 + lane;                 // weight row within the tile
+    const int p = nloc / a.sh, nl = nloc - p * a.sh;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t base = mapa_shared(smem_u32(recv), static_cast<uint32_t>(p));
+    const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
+    for (int c0 = 0; c0 < a.B; c0 += 16) {
+      uint32_t acc[16], up[16];
+      __syncwarp();
+      tmem_ld_32x32b_x16(lane_addr + c0, acc);
+      if (lr_here) tmem_ld_32x32b_x16(lane_addr + kLrCol + c0, up);
+      tmem_ld_wait_regs(acc);
+      if (lr_here) tmem_ld_wait_regs(up);
+      const int cnt = min(16, a.B - c0);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j >= cnt) break;
+        uint32_t v = acc[j];
+        if (kFmt != kFmtNvfp4 && kOut != kOutI32) {
+          float f = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
+          if (lr_here) f += __uint_as_float(up[j]);
+          v = __float_as_uint(f);
+        }
+        const int b = c0 + j;
+        st_cluster_u32(base + static_cast<uint32_t>(((rank * a.Bp + b) * a.sh + nl) * 4), v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+
+  // ------------------------------------- sum of the partials, bias, store
+  {
+    const int cnt = min(a.sh, kTileN - rank * a.sh);      // weight rows this CTA owns
+    const int nq = cnt / 4;
+    const int nbase = n0 + rank * a.sh;
+    pdl_wait();   // returns at once: the epilogue warps waited before the barriers
+    const float alpha_f4 = kFmt == kFmtNvfp4 ? skinny_alpha<kFmt, kOut>(a) : 1.0f;
+    for (int it = threadIdx.x; it < a.B * nq; it += kThreads) {
+      const int b = it / nq, nl = (it - b * nq) * 4;
+      const int n = nbase + nl;
+      if (n >= a.N || abort_sh) continue;
+      if constexpr (kOut == kOutI32) {
+        int4 s = make_int4(0, 0, 0, 0);
+        for (int c = 0; c < S; ++c) {
+          const int4 v = *reinterpret_cast<const int4*>(recv + (c * a.Bp + b) * a.sh + nl);
+          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        int32_t* dst = static_cast<int32_t*>(a.y) + static_cast<int64_t>(b) * a.ldy + n;
+        if (a.vec_ok) {
+          *reinterpret_cast<int4*>(dst) = s;
+        } else {
+          dst[0] = s.x; dst[1] = s.y; dst[2] = s.z; dst[3] = s.w;
+        }
+      } else {
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < S; ++c) {
+          const float4 v = *reinterpret_cast<const float4*>(recv + (c * a.Bp + b) * a.sh + nl);
+          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        float o[4] = {s.x, s.y, s.z, s.w};
+        if (kFmt == kFmtNvfp4) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) o[j] *= alpha_f4;
+        }
+        if (a.bias != nullptr) {
+          const uint2 bb = *reinterpret_cast<const uint2*>(a.bias + n);
+          o[0] += __uint_as_float(bb.x << 16);
+          o[1] += __uint_as_float(bb.x & 0xFFFF0000u);
+          o[2] += __uint_as_float(bb.y << 16);
+          o[3] += __uint_as_float(bb.y & 0xFFFF0000u);
+        }
+        if constexpr (kOut == kOutF32) {
+          float* dst = static_cast<float*>(a.y) + static_cast<int64_t>(b) * a.ldy + n;
+          if (a.vec_ok) {
+            *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+          } else {
+            dst[0] = o[0]; dst[1] = o[1]; dst[2] = o[2]; dst[3] = o[3];
+          }
+        } else {
+          uint16_t* dst = static_cast<uint16_t*>(a.y) + static_cast<int64_t>(b) * a.ldy + n;
+          const uint32_t p0 = pack_bf16x2(o[0], o[1]), p1 = pack_bf16x2(o[2], o[3]);
+          if (a.vec_ok) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(p0, p1);
+          } else {
+            dst[0] = static_cast<uint16_t>(p0 & 0xFFFFu); dst[1] = static_cast<uint16_t>(p0 >> 16);
+            dst[2] = static_cast<uint16_t>(p1 & 0xFFFFu); dst[3] = static_cast<uint16_t>(p1 >> 16);
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+struct SkinnyPlan {
+  int S, sh, da, db, dp, a_slot, b_slot;
+  size_t smem;
+};
+
+SkinnyPlan plan_skinny(int kFmt, int Bp, int64_t N, int kst, int lr_boxes) {
+  SkinnyPlan p{};
+  const int64_t tiles = ceil_div(N, kTileN);
+  const int sms = num_sms();
+  int S = 1;
+  for (int s = std::min(8, kst); s >= 1; --s)
+    if (tiles * s <= sms) {
+      S = s;
+      break;
+    }
+  p.S = S;
+  p.sh = static_cast<int>(round_up(ceil_div(kTileN, S), 4));
+  p.a_slot = kATile + (kFmt == kFmtNvfp4 ? kSfBytes : 0);
+  p.b_slot = Bp * 128 + (kFmt == kFmtNvfp4 ? kSfBytes : 0);
+  const int nres_max = static_cast<int>(ceil_div(kst, S));
+  const int nsteps_max = nres_max + static_cast<int>(ceil_div(lr_boxes, S));
+  p.dp = kFmt == kFmtInt4 ? std::min(nres_max, kMaxRing) : 0;
+  p.da = std::min(nsteps_max, kFmt == kFmtInt4 ? 4 : 6);
+  p.db = std::min(nsteps_max, 4);
+  auto total = [&]() {
+    return static_cast<size_t>(p.da) * p.a_slot + static_cast<size_t>(p.db) * p.b_slot +
+           static_cast<size_t>(p.dp) * kPSlot;
+  };
+  while (total() > kSmemBudget) {
+    if (p.dp > 4) --p.dp;
+    else if (p.db > 2) --p.db;
+    else if (p.da > 2) --p.da;
+    else if (p.dp > 2) --p.dp;
+    else break;
+  }
+  const size_t recv = static_cast<size_t>(S) * Bp * p.sh * 4;
+  // more than half an SM's shared memory: one CTA of this kernel per SM, so
+  // the TMEM allocation never waits on another cluster's CTA
+  p.smem = std::max({total(), recv, kMinSmem}) + 1024;
+  return p;
+}
+
+template <int kFmt, int kOut>
+cudaError_t launch_one(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& lu, const CUtensorMap& dn,
+                       const SkinnyArgs& args, int tiles, size_t smem, bool pdl, cudaStream_t st) {
+  auto kern = skinny_kernel<kFmt, kOut>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(args.S), static_cast<unsigned>(tiles));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(args.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, w, x, lu, dn, args);
+}
+
+}  // namespace
+
+// Host side: tensor maps and launch. kind: 0 INT, 1 NVFP4; out: GemmOut.
+bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_codes, const uint8_t* act_sf,
+                        const void* down2, const svdq_weight* w, bool pdl, cudaStream_t stream,
+                        cudaError_t* err) {
+  *err = cudaSuccess;
+  const int64_t M = w->M, N = w->N, B = g.B;
+  if (B <= 0 || B > 128) return false;
+  const int Bp = static_cast<int>(std::max<int64_t>(16, round_up(B, 16)));
+  const bool packed = kind == kKindInt && w->fmt.bits <= 4 && w->codes4 != nullptr;
+  const int fmt = kind == kKindNvfp4 ? kFmtNvfp4 : (packed ? kFmtInt4 : kFmtInt8);
+  const int kst = static_cast<int>(kind == kKindNvfp4 ? ceil_div(M, 256) : ceil_div(M, 128));
+  const int rp = w->rank_pad;
+  const bool has_lr = out != kOutI32 && rp > 0 && down2 != nullptr;
+  const int lr_boxes = has_lr ? static_cast<int>(ceil_div(2 * rp, 64)) : 0;
+  const SkinnyPlan p = plan_skinny(fmt, Bp, N, kst, lr_boxes);
+
+  CUtensorMap tm_w, tm_x, tm_lu, tm_dn;
+  bool ok;
+  if (fmt == kFmtInt4)
+    ok = make_tmap_2d(&tm_w, w->codes4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M / 2, N, M / 2, 64, kTileN, false);
+  else if (fmt == kFmtNvfp4)
+    ok = make_tmap_2d(&tm_w, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M / 2, N, M / 2, 128, kTileN, true);
+  else
+    ok = make_tmap_2d(&tm_w, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, N, M, 128, kTileN, true);
+  const int64_t xrow = kind == kKindNvfp4 ? M / 2 : M;
+  ok = ok && make_tmap_2d(&tm_x, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xrow, B, xrow, 128, Bp, true);
+  if (ok && has_lr) {
+    ok = make_tmap_2d(&tm_lu, w->lu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, N, 2 * rp, 64, kTileN, true) &&
+         make_tmap_2d(&tm_dn, down2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, B, 2 * rp, 64, Bp, true);
+  } else {
+    tm_lu = tm_w;
+    tm_dn = tm_x;
+  }
+  if (!ok) return false;
+
+  SkinnyArgs a{};
+  a.B = static_cast<int>(B);
+  a.Bp = Bp;
+  a.N = static_cast<int>(N);
+  a.M = static_cast<int>(M);
+  a.S = p.S;
+  a.kst = kst;
+  a.lr_boxes = lr_boxes;
+  a.sh = p.sh;
+  a.da = p.da;
+  a.db = p.db;
+  a.dp = p.dp;
+  a.a_slot = p.a_slot;
+  a.b_slot = p.b_slot;
+  a.katoms = static_cast<int>(ceil_div(M, 64));
+  a.s_x = g.s_x;
+  a.s_w = g.s_w;
+  a.bias = g.bias;
+  a.y = g.y;
+  a.ldy = g.ldy;
+  a.vec_ok = g.vec_ok;
+  a.sfw = static_cast<const uint8_t*>(w->sf);
+  a.sfx = act_sf;
+  a.status = g.status;
+  const int tiles = static_cast<int>(ceil_div(N, kTileN));
+#define SVDQ_SKINNY(F, O) *err = launch_one<F, O>(tm_w, tm_x, tm_lu, tm_dn, a, tiles, p.smem, pdl, stream)
+  if (out == kOutI32) {
+    if (fmt == kFmtInt4) SVDQ_SKINNY(kFmtInt4, kOutI32);
+    else if (fmt == kFmtInt8) SVDQ_SKINNY(kFmtInt8, kOutI32);
+    else return false;
+  } else if (out == kOutF32) {
+    if (fmt == kFmtInt4) SVDQ_SKINNY(kFmtInt4, kOutF32);
+    else if (fmt == kFmtInt8) SVDQ_SKINNY(kFmtInt8, kOutF32);
+    else SVDQ_SKINNY(kFmtNvfp4, kOutF32);
+  } else {
+    if (fmt == kFmtInt4) SVDQ_SKINNY(kFmtInt4, kOutBF16);
+    else if (fmt == kFmtInt8) SVDQ_SKINNY(kFmtInt8, kOutBF16);
+    else SVDQ_SKINNY(kFmtNvfp4, kOutBF16);
+  }
+#undef SVDQ_SKINNY
+  return true;
+}
+
+}  // namespace svdq

@@ -57,10 +57,18 @@ struct ActPlan {
   int grid;        // CTAs of the cooperative launch (all resident)
   int nparts;      // partial maxima written (one per CTA)
   size_t smem;     // dynamic shared memory per CTA
+  int small;       // 1: the short-batch kernel (act_small.cu): one column chunk per CTA
+  int wc;          // short-batch kernel: columns per chunk (a multiple of 32)
 };
-ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt);
-// Recompute the derived fields after changing ksplit.
+// Batches up to this many rows take the short-batch kernel.
+constexpr int64_t kActSmallMaxB = 128;
+// Dynamic shared memory the short-batch kernel may use (else the large-batch plan).
+constexpr size_t kActSmallSmemMax = 200 * 1024;
+ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool allow_small = true);
+// Recompute the derived fields after changing ksplit (for the short-batch
+// kernel, ksplit is the number of column chunks).
 void finish_act_plan(ActPlan& p);
+void finish_act_plan_small(ActPlan& p);
 size_t act_scratch_bytes(const ActPlan& p);
 
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
@@ -68,23 +76,31 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
                        const float* w_global_scale, const void* ld, void* codes, void* sf,
                        float* act_scale, void* down, void* scratch, cudaStream_t stream,
                        bool* bad_args);
+cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
+                             const float* scale, svdq_fmt fmt, const float* act_global_scale,
+                             const float* w_global_scale, const void* ld, void* codes, void* sf,
+                             float* act_scale, void* down, void* scratch, cudaStream_t stream,
+                             bool* bad_args);
 
 // ------------------------------------------------------------ residual GEMM
 cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
                             const void* down2, int64_t B, const void* bias, void* y,
-                            svdq_dtype ydt, int64_t ldy, bool raw_i32, cudaStream_t stream,
+                            svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
                             bool* bad_args);
 
 cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
                               const uint8_t* act_sf, const float* gs_x, const void* down2,
                               int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                              int64_t ldy, cudaStream_t stream, bool* bad_args);
+                              int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args);
 
 // -------------------------------------------------------------- quantisers
 size_t residual_scratch_bytes(int64_t M, int64_t N);
 cudaError_t launch_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
                                      svdq_fmt fmt, void* codes, void* sf, float* w_scale,
                                      void* scratch, cudaStream_t stream);
+// INT codes int8 [N, M] -> two per byte [N, M / 2] (element 2j in the low nibble).
+cudaError_t launch_pack_int4(const int8_t* codes, int64_t N, int64_t M, uint8_t* packed,
+                             cudaStream_t stream);
 
 // ------------------------------------------------------------------ prepare
 size_t prepare_scratch_bytes(int64_t M, int64_t N, int32_t rank, int32_t oversample);

@@ -79,6 +79,9 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
   while (act_scratch_bytes(p) > kNoallocScratchBytes && p.ksplit > 1) {
     p.ksplit = std::max(1, p.ksplit / 2);
     finish_act_plan(p);
+    // fewer, wider column chunks of the short-batch kernel may outgrow its
+    // shared memory: continue with the large-batch plan then
+    if (p.small && p.smem > kActSmallSmemMax) p = plan_act(B, M, rp, x_dtype, false);
   }
   if (act_scratch_bytes(p) > kNoallocScratchBytes) return SVDQ_EWORKSPACE;
 

@@ -721,6 +721,10 @@ svdq_status run_prepare(const void* W, svdq_dtype wdt, int64_t M, int64_t N, int
   if (launch_quantize_residual(c.ws, M, N, N, fmt, out->codes, out->sf, out->w_scale, c.qscratch,
                                st) != cudaSuccess)
     return SVDQ_ECUDA;
+  if (out->codes4 && fmt.kind == SVDQ_KIND_INT && fmt.bits <= 4 &&
+      launch_pack_int4(static_cast<const int8_t*>(out->codes), N, M, static_cast<uint8_t*>(out->codes4),
+                       st) != cudaSuccess)
+    return SVDQ_ECUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SVDQ_ECUDA;
   unsigned v = 0;
   if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ECUDA;

@@ -462,4 +462,20 @@ __device__ __forceinline__ uint32_t elect_one() {
   return pred;
 }
 
+// ------------------------------------------------ clusters and dependent launch
+// Store one 32-bit word into the shared memory of a CTA of this cluster
+// (`cluster_addr` from mapa_shared).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their memory is visible (returns at once when there are none).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let a grid launched after this one with programmatic serialization start.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace svdq

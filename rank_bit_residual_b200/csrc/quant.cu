@@ -15,6 +15,7 @@
 
 #include <algorithm>
 
+#include "encode.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -91,33 +92,6 @@ __global__ void __launch_bounds__(256) quant_int_transpose_kernel(
   }
 }
 
-__device__ __forceinline__ uint8_t f32_to_ue4m3_q(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return static_cast<uint8_t>(r & 0xFFu);
-}
-
-__device__ __forceinline__ float ue4m3_to_f32_q(uint8_t b) {
-  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
-  return e == 0 ? static_cast<float>(m) * 0.001953125f
-                : __uint_as_float(((e + 120u) << 23) | (m << 20));
-}
-
-__device__ __forceinline__ uint32_t f32x8_to_e2m1_q(const float* v) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  const uint32_t mag = out & 0x77777777u;
-  const uint32_t nz = (mag + 0x77777777u) & 0x88888888u;
-  return out & (0x77777777u | nz);
-}
-
 // One thread per (column n, 16-row block kb) of R; consecutive threads take
 // consecutive n so every row read is coalesced.
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
@@ -148,14 +122,34 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
       v[j] = R[(b * 16 + j) * ldR + n];
       amax = fmaxf(amax, fabsf(v[j]));
     }
-    const uint8_t sfb = f32_to_ue4m3_q(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
-    const float d = ue4m3_to_f32_q(sfb);
+    const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
+    const float d = ue4m3_to_f32(sfb);
     const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], enc);
     *reinterpret_cast<uint2*>(codes + n * (M / 2) + b * 8) =
-        make_uint2(f32x8_to_e2m1_q(v), f32x8_to_e2m1_q(v + 8));
+        make_uint2(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8));
     sf[off] = sfb;
+  }
+}
+
+// 32 codes (32 bytes) -> 16 packed bytes per thread; element 2j in the low nibble.
+__global__ void __launch_bounds__(256) pack_int4_kernel(const int8_t* __restrict__ codes, int64_t n16,
+                                                        uint8_t* __restrict__ packed) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * i);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * i + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // bytes e0..e7 of two words -> nibbles: even elements low, odd elements high
+      const uint32_t lo = __byte_perm(w[2 * j], w[2 * j + 1], 0x6420) & 0x0F0F0F0Fu;
+      const uint32_t hi = __byte_perm(w[2 * j], w[2 * j + 1], 0x7531) & 0x0F0F0F0Fu;
+      o[j] = lo | (hi << 4);
+    }
+    reinterpret_cast<uint4*>(packed)[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -191,6 +185,15 @@ cudaError_t launch_quantize_residual(const float* R, int64_t M, int64_t N, int64
                                                     static_cast<uint8_t*>(codes),
                                                     static_cast<uint8_t*>(sf), w_scale);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4(const int8_t* codes, int64_t N, int64_t M, uint8_t* packed,
+                             cudaStream_t stream) {
+  const int64_t n16 = N * M / 32;   // 16-byte outputs (M is a multiple of 32)
+  const int blocks = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(ceil_div(n16, 256), static_cast<int64_t>(num_sms()) * 8)));
+  pack_int4_kernel<<<blocks, 256, 0, stream>>>(codes, n16, packed);
   return cudaGetLastError();
 }
 

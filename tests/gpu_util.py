@@ -63,7 +63,7 @@ def assert_codes_match(got: np.ndarray, want: np.ndarray, near: np.ndarray, what
 class SyntheticWeight:
     """A prepared weight with random codes and factors (host copies kept for the oracle)."""
 
-    def __init__(self, M, N, rank, fmt="int4", seed=0, scale=None, s_w=0.013):
+    def __init__(self, M, N, rank, fmt="int4", seed=0, scale=None, s_w=0.013, packed=False):
         rng = np.random.default_rng(seed)
         f = rb.parse_fmt(fmt)
         self.fmt, self.M, self.N, self.rank = f, M, N, rank
@@ -87,16 +87,20 @@ class SyntheticWeight:
             codes_buf = to_dev(self.codes.view(np.uint8).reshape(-1), torch.uint8)
             self.s_w = np.float32(s_w)
             sf_buf = None
+            # the half-size copy the short-batch GEMM streams (nibble packing done here)
+            codes4 = to_dev(onv.pack_nibbles(self.codes.view(np.uint8) & 0xF).reshape(-1),
+                            torch.uint8) if packed else None
         else:
             self.codes = rng.integers(0, 16, (N, M)).astype(np.uint8)
             self.sf = rng.integers(0x20, 0x48, (N, M // 16)).astype(np.uint8)  # ~2^-3 .. 2^2
             codes_buf = to_dev(onv.pack_nibbles(self.codes).reshape(-1), torch.uint8)
             sf_buf = to_dev(onv.sf_swizzle(self.sf), torch.uint8)
             self.s_w = np.float32(2688.0 / 3.0)
+            codes4 = None
         self.w = rb.weight_from_buffers(
             M, N, rank, f, codes_buf, sf_buf, to_dev(np.array([self.s_w], np.float32), torch.float32),
             to_dev(ld, torch.bfloat16), to_dev(ld, torch.float32), to_dev(lu, torch.bfloat16),
-            to_dev(self.scale, torch.float32))
+            to_dev(self.scale, torch.float32), codes4=codes4)
 
     def oracle_y(self, x: np.ndarray, bias=None, gs_x=None) -> np.ndarray:
         ldT = self.ld[: self.rp].T if self.rp else np.zeros((self.M, 0))

@@ -30,7 +30,7 @@ def test_version_and_status_strings(lib):
 
 
 def _sizes(lib, M, N, r, fmt):
-    sizes = (ctypes.c_size_t * 6)()
+    sizes = (ctypes.c_size_t * 7)()
     st = lib.svdq_weight_buffer_sizes(M, N, r, rb.parse_fmt(fmt), sizes)
     return st, list(sizes)
 
@@ -38,11 +38,13 @@ def _sizes(lib, M, N, r, fmt):
 def test_weight_buffer_sizes(lib):
     st, s = _sizes(lib, 3072, 3072, 32, "int4")
     assert st == rb.SVDQ_OK
-    assert s == [3072 * 3072, 0, 4, 32 * 3072 * 2, 32 * 3072 * 4, 3072 * 64 * 2]
+    assert s == [3072 * 3072, 0, 4, 32 * 3072 * 2, 32 * 3072 * 4, 3072 * 64 * 2, 3072 * 3072 // 2]
+    assert _sizes(lib, 3072, 3072, 32, "int8")[1][6] == 0      # no packed copy above 4 bits
     st, s = _sizes(lib, 256, 3216, 20, "nvfp4")
     assert st == rb.SVDQ_OK
     assert s[0] == 3216 * 128 and s[1] == 3328 * 16   # rows padded to 128, 16 scale columns
     assert s[3] == 32 * 256 * 2
+    assert s[6] == 0
 
 
 def test_host_checks_follow_the_page_contract(lib):
