@@ -735,8 +735,8 @@ size_t act_sync_bytes(const ActPlan& p) {
 }
 
 size_t act_scratch_bytes(const ActPlan& p) {
-  if (p.small)
-    return static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * 4, 256)) + 256 +
+  if (p.small)   // barrier word, then the partial down tiles (act_small.cu)
+    return 256 +
            (p.rank_pad > 0 ? static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * p.B * p.rank_pad * 4, 256)) : 0) +
            256;
   size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));

@@ -12,8 +12,9 @@
 //   phase 1  chunk of x -> shared memory; column maxima of |x| times
 //            r_k = fl(1 / scale_k) -> one partial maximum per CTA; partial
 //            down-projection of the chunk -> ws_down[g][b][j]
-//   barrier  (bounded; the counter is zeroed before the launch)
-//   phase 2  per-tensor scale from the partial maxima; codes of the chunk
+//   barrier  bounded; its 64-bit word (zeroed before the launch) counts the
+//            arrivals and carries the largest partial maximum
+//   phase 2  per-tensor scale from that maximum; codes of the chunk
 //            from the shared copy; each CTA sums its share of the (b, j)
 //            down outputs over the partials in a fixed order
 //
@@ -37,6 +38,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kZParts = 8;   // threads that share one down output's sum in phase 2
+constexpr int kZBatch = 20;  // partials one thread loads at once (covers 160 CTAs in one batch)
 
 struct SmallArgs {
   int B, M, wc, G, rank_pad, fmt_kind, qmax, has_ld;
@@ -46,9 +48,8 @@ struct SmallArgs {
   const float* gs_given;
   const float* gs_w;
   const void* ld;     // [rank_pad][M], x's dtype
-  float* ws_max;      // [G]
   float* ws_down;     // [G][B][rank_pad]
-  unsigned* sync;     // [0] barrier counter, [1] abort flag (zeroed before the launch)
+  unsigned long long* sync;   // barrier word (arrivals | max) and abort flag, zeroed before the launch
   void* codes;
   uint8_t* sf;
   __nv_bfloat16* down;
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float red[kWarps];
+  __shared__ float cta_max_sh;
   __shared__ int abort_sh;
 
   pdl_trigger();   // a GEMM launched after this kernel may start its weight loads now
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
     if (tid == 0) {
       float t = red[0];
       for (int w = 1; w < kWarps; ++w) t = fmaxf(t, red[w]);
-      a.ws_max[g] = t;
+      cta_max_sh = t;
     }
   }
 
@@ -177,53 +179,87 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
   // chunk's columns are the K of each tile's MMA chain
   if (a.has_ld) {
     const int gid = lane >> 2, tig = lane & 3;
-    const int mt = bp16 / 16, nt = a.rank_pad / 8;
-    for (int t = warp; t < mt * nt; t += kWarps) {
-      const int b0 = (t / nt) * 16, j0 = (t % nt) * 8;
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      const uint8_t* xa = xs + (b0 + gid) * pitch;
-      const uint8_t* xb = xa + 8 * pitch;
-      const uint8_t* lb = lds + (j0 + gid) * pitch;
-      if constexpr (kEsz == 2) {
-        for (int k = 0; k < ncols; k += 16) {
-          const int o0 = (k + 2 * tig) * 2, o1 = o0 + 16;
-          const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(xa + o0), *reinterpret_cast<const uint32_t*>(xb + o0),
-                                  *reinterpret_cast<const uint32_t*>(xa + o1), *reinterpret_cast<const uint32_t*>(xb + o1)};
-          const uint32_t bf[2] = {*reinterpret_cast<const uint32_t*>(lb + o0), *reinterpret_cast<const uint32_t*>(lb + o1)};
-          mma_bf16_16816(d, af, bf);
-        }
-      } else {
-        for (int k = 0; k < ncols; k += 8) {
-          const int o0 = (k + tig) * 4, o1 = o0 + 16;
-          const uint32_t af[4] = {to_tf32(*reinterpret_cast<const uint32_t*>(xa + o0)),
-                                  to_tf32(*reinterpret_cast<const uint32_t*>(xb + o0)),
-                                  to_tf32(*reinterpret_cast<const uint32_t*>(xa + o1)),
-                                  to_tf32(*reinterpret_cast<const uint32_t*>(xb + o1))};
-          const uint32_t bf[2] = {to_tf32(*reinterpret_cast<const uint32_t*>(lb + o0)),
-                                  to_tf32(*reinterpret_cast<const uint32_t*>(lb + o1))};
-          mma_tf32_1688(d, af, bf);
+    const int mt = bp16 / 16, nt = a.rank_pad / 8, ntile = mt * nt;
+    // up to four tiles per warp at a time: their MMAs are independent, so they
+    // issue back to back instead of waiting on one accumulator
+    for (int t0 = warp; t0 < ntile; t0 += 4 * kWarps) {
+      float d[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) d[q][0] = d[q][1] = d[q][2] = d[q][3] = 0.0f;
+      constexpr int kStep = kEsz == 2 ? 16 : 8;
+      for (int k = 0; k < ncols; k += kStep) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = t0 + q * kWarps;
+          if (t >= ntile) break;
+          const int b0 = (t / nt) * 16, j0 = (t % nt) * 8;
+          const uint8_t* xa = xs + (b0 + gid) * pitch;
+          const uint8_t* xb = xa + 8 * pitch;
+          const uint8_t* lb = lds + (j0 + gid) * pitch;
+          if constexpr (kEsz == 2) {
+            const int o0 = (k + 2 * tig) * 2, o1 = o0 + 16;
+            const uint32_t af[4] = {*reinterpret_cast<const uint32_t*>(xa + o0), *reinterpret_cast<const uint32_t*>(xb + o0),
+                                    *reinterpret_cast<const uint32_t*>(xa + o1), *reinterpret_cast<const uint32_t*>(xb + o1)};
+            const uint32_t bf[2] = {*reinterpret_cast<const uint32_t*>(lb + o0), *reinterpret_cast<const uint32_t*>(lb + o1)};
+            mma_bf16_16816(d[q], af, bf);
+          } else {
+            const int o0 = (k + tig) * 4, o1 = o0 + 16;
+            const uint32_t af[4] = {to_tf32(*reinterpret_cast<const uint32_t*>(xa + o0)),
+                                    to_tf32(*reinterpret_cast<const uint32_t*>(xb + o0)),
+                                    to_tf32(*reinterpret_cast<const uint32_t*>(xa + o1)),
+                                    to_tf32(*reinterpret_cast<const uint32_t*>(xb + o1))};
+            const uint32_t bf[2] = {to_tf32(*reinterpret_cast<const uint32_t*>(lb + o0)),
+                                    to_tf32(*reinterpret_cast<const uint32_t*>(lb + o1))};
+            mma_tf32_1688(d[q], af, bf);
+          }
         }
       }
-      const int r0 = b0 + gid, r1 = r0 + 8, j = j0 + 2 * tig;
       float* base = a.ws_down + static_cast<int64_t>(g) * B * a.rank_pad;
-      if (r0 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r0) * a.rank_pad + j) = make_float2(d[0], d[1]);
-      if (r1 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r1) * a.rank_pad + j) = make_float2(d[2], d[3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = t0 + q * kWarps;
+        if (t >= ntile) break;
+        const int r0 = (t / nt) * 16 + gid, r1 = r0 + 8, j = (t % nt) * 8 + 2 * tig;
+        if (r0 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r0) * a.rank_pad + j) = make_float2(d[q][0], d[q][1]);
+        if (r1 < B) *reinterpret_cast<float2*>(base + static_cast<int64_t>(r1) * a.rank_pad + j) = make_float2(d[q][2], d[q][3]);
+      }
     }
   }
 
   // ================================================================ barrier
-  GridSync gsync{a.sync, a.sync + 1, a.status, 0u};
-  if (!grid_sync(gsync, &abort_sh)) return;
+  // One 64-bit word: arrivals in the low half, the largest partial maximum
+  // (non-negative floats order like their bit patterns) in the high half. Each
+  // CTA raises the maximum, then adds its arrival with release semantics; once
+  // the count reaches G an acquire load of the word also yields the final max.
+  __syncthreads();   // this CTA's partial down tile is written
+  if (tid == 0) {
+    unsigned* words = reinterpret_cast<unsigned*>(a.sync);
+    atomicMax(words + 1, __float_as_uint(cta_max_sh));
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(words) : "memory");
+    const unsigned long long t0 = globaltimer_ns();
+    unsigned long long v = 0;
+    while (true) {
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.sync) : "memory");
+      if (static_cast<unsigned>(v & 0xFFFFFFFFull) >= static_cast<unsigned>(a.G)) break;
+      if (*reinterpret_cast<volatile unsigned*>(words + 2)) {
+        abort_sh = 1;
+        break;
+      }
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_status(a.status, kStatusTimeout);
+        atomicExch(words + 2, 1u);
+        abort_sh = 1;
+        break;
+      }
+    }
+    red[0] = __uint_as_float(static_cast<unsigned>(v >> 32));
+  }
+  __syncthreads();
+  if (abort_sh) return;
 
   // ================================================================ phase 2
-  float m = 0.0f;
-  for (int i = tid; i < a.G; i += kThreads) m = fmaxf(m, __ldcg(a.ws_max + i));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  m = red[0];
-  for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w]);
+  const float m = red[0];
   const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
   float u = 0.0f, gs_x = 1.0f;
   if (nv) {
@@ -308,8 +344,20 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
     for (int base = lo; base < hi; base += kThreads / kZParts) {
       const int idx = base + tid / kZParts;
       float acc = 0.0f;
-      if (idx < hi)
-        for (int z = zp; z < a.G; z += kZParts) acc += __ldcg(a.ws_down + z * stride + idx);
+      if (idx < hi) {
+        // all of this thread's partials are loaded before any is added, so the
+        // loads overlap instead of paying the L2 latency one after another
+        for (int z0 = zp; z0 < a.G; z0 += kZParts * kZBatch) {
+          float v[kZBatch];
+#pragma unroll
+          for (int u = 0; u < kZBatch; ++u) {
+            const int z = z0 + u * kZParts;
+            v[u] = z < a.G ? __ldcg(a.ws_down + z * stride + idx) : 0.0f;
+          }
+#pragma unroll
+          for (int u = 0; u < kZBatch; ++u) acc += v[u];
+        }
+      }
       // fixed-order combine of the kZParts partial sums (lanes zp = 0..7 of a group)
 #pragma unroll
       for (int o = 1; o < kZParts; o <<= 1) {
@@ -362,11 +410,10 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
     return cudaSuccess;
   }
   Carver cv(scratch, ~size_t(0));
-  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * 4));
-  unsigned* sync = static_cast<unsigned*>(cv.take(256));
+  auto* sync = static_cast<unsigned long long*>(cv.take(256));
   float* ws_down = has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * p.B * p.rank_pad * 4))
                           : nullptr;
-  cudaError_t err = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), stream);
+  cudaError_t err = cudaMemsetAsync(sync, 0, 16, stream);
   if (err != cudaSuccess) return err;
   SmallArgs a{};
   a.B = static_cast<int>(p.B);
@@ -383,7 +430,6 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
   a.gs_given = fmt.kind == SVDQ_KIND_NVFP4 ? act_global_scale : nullptr;
   a.gs_w = fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr;
   a.ld = has_ld ? ld : nullptr;
-  a.ws_max = ws_max;
   a.ws_down = ws_down;
   a.sync = sync;
   a.codes = codes;
@@ -397,11 +443,20 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
     err = cudaFuncSetAttribute(act_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
+    // the largest shared-memory configuration, the one the GEMM launched after
+    // this kernel needs: with equal configurations its CTAs can share SMs with
+    // these and start early (a different split makes an SM drain first)
+    err = cudaFuncSetAttribute(act_small_kernel<__nv_bfloat16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (err != cudaSuccess) return err;
     return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<__nv_bfloat16>), dim3(p.grid),
                                        dim3(kThreads), args, smem, stream);
   }
   err = cudaFuncSetAttribute(act_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(act_small_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (err != cudaSuccess) return err;
   return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<float>), dim3(p.grid),
                                      dim3(kThreads), args, smem, stream);

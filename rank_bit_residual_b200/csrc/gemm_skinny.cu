@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t empty_p[kMaxRing];
   __shared__ __align__(8) uint64_t tmem_full;
   __shared__ __align__(8) uint64_t mma_done;
+  __shared__ __align__(8) uint64_t recv_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring_a = smem;
   uint8_t* ring_b = ring_a + static_cast<size_t>(a.da) * a.a_slot;
   uint8_t* ring_p = ring_b + static_cast<size_t>(a.db) * a.b_slot;
-  uint32_t* recv = reinterpret_cast<uint32_t*>(smem);   // reuses the rings once every MMA is done
+  uint32_t* recv_base = reinterpret_cast<uint32_t*>(smem);   // partials: reuse the rings once every MMA is done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -146,7 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&tmem_full, 1);
     mbar_init(&mma_done, 1);
+    mbar_init(&recv_bar, 1);
     fence_mbar_init();
+    // the shares the other S - 1 CTAs will copy here
+    mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>((S - 1) * a.B * a.sh * 4));
     abort_sh = 0;
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
@@ -359,50 +363,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ------------------------------------------------------------ epilogue
+  // Partials of the whole tile are staged per owner in this CTA's shared memory
+  // (stg[p][b][nl], p the CTA that owns weight rows [p sh, p sh + sh)), then
+  // one bulk copy per owner moves each share into recv[rank] of that owner,
+  // completing on the owner's recv_bar; the owner sums recv[c] (stg[rank] for
+  // its own) in rank order. Both buffers reuse the operand rings, whose last
+  // reads are the MMAs: staging waits for this CTA's accumulator, the copies
+  // for the cluster barrier that follows every CTA's staging.
   const bool epi = warp >= kWarpEpi0;
+  const int slot_words = a.B * a.sh;
+  uint32_t* stg = recv_base;
+  uint32_t* recv = recv_base + static_cast<size_t>(S) * slot_words;
   float alpha = 0.0f;
-  bool fin = false;
   if (epi) {
-    fin = mbar_wait_warp(&tmem_full, 0, status, &abort_sh);
+    const bool fin = mbar_wait_warp(&tmem_full, 0, status, &abort_sh);
     tc_fence_after();
     pdl_wait();   // the activation scale comes from the activation pass
     alpha = skinny_alpha<kFmt, kOut>(a);
-  }
-  // every CTA of the cluster is past its MMAs: the rings are free for the partials
-  __syncwarp();
-  cluster_sync();
-  if (epi && fin) {
-    const int q = warp & 3;
-    const int nloc = q * 32 + lane;                 // weight row within the tile
-    const int p = nloc / a.sh, nl = nloc - p * a.sh;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t base = mapa_shared(smem_u32(recv), static_cast<uint32_t>(p));
-    const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
-    for (int c0 = 0; c0 < a.B; c0 += 16) {
-      uint32_t acc[16], up[16];
-      __syncwarp();
-      tmem_ld_32x32b_x16(lane_addr + c0, acc);
-      if (lr_here) tmem_ld_32x32b_x16(lane_addr + kLrCol + c0, up);
-      tmem_ld_wait_regs(acc);
-      if (lr_here) tmem_ld_wait_regs(up);
-      const int cnt = min(16, a.B - c0);
+    if (fin) {
+      const int q = warp & 3;
+      const int nloc = q * 32 + lane;                 // weight row within the tile
+      const int p = nloc / a.sh, nl = nloc - p * a.sh;
+      uint32_t* dst = stg + static_cast<size_t>(p) * slot_words + nl;
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
+      for (int c0 = 0; c0 < a.B; c0 += 16) {
+        uint32_t acc[16], up[16];
+        __syncwarp();
+        tmem_ld_32x32b_x16(lane_addr + c0, acc);
+        if (lr_here) tmem_ld_32x32b_x16(lane_addr + kLrCol + c0, up);
+        tmem_ld_wait_regs(acc);
+        if (lr_here) tmem_ld_wait_regs(up);
+        const int cnt = min(16, a.B - c0);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j >= cnt) break;
-        uint32_t v = acc[j];
-        if (kFmt != kFmtNvfp4 && kOut != kOutI32) {
-          float f = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
-          if (lr_here) f += __uint_as_float(up[j]);
-          v = __float_as_uint(f);
+        for (int j = 0; j < 16; ++j) {
+          if (j >= cnt) break;
+          uint32_t v = acc[j];
+          if (kFmt != kFmtNvfp4 && kOut != kOutI32) {
+            float f = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
+            if (lr_here) f += __uint_as_float(up[j]);
+            v = __float_as_uint(f);
+          }
+          dst[(c0 + j) * a.sh] = v;
         }
-        const int b = c0 + j;
-        st_cluster_u32(base + static_cast<uint32_t>(((rank * a.Bp + b) * a.sh + nl) * 4), v);
       }
     }
+    fence_proxy_async_smem();   // the staged partials are read by the bulk copies
   }
   tc_fence_before();
   __syncwarp();
   cluster_sync();
+  if (threadIdx.x == kWarpEpi0 * 32) {
+    const uint32_t bytes = static_cast<uint32_t>(slot_words) * 4u;
+    for (int p = 0; p < S; ++p) {
+      if (p == rank) continue;
+      bulk_copy_to_cluster(mapa_shared(smem_u32(recv + static_cast<size_t>(rank) * slot_words), p),
+                           smem_u32(stg + static_cast<size_t>(p) * slot_words), bytes,
+                           mapa_shared(smem_u32(&recv_bar), p));
+    }
+  }
+  const bool got = mbar_wait(&recv_bar, 0, status, &abort_sh);
 
   // ------------------------------------- sum of the partials, bias, store
   {
@@ -414,11 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = threadIdx.x; it < a.B * nq; it += kThreads) {
       const int b = it / nq, nl = (it - b * nq) * 4;
       const int n = nbase + nl;
-      if (n >= a.N || abort_sh) continue;
+      if (n >= a.N || !got) continue;
       if constexpr (kOut == kOutI32) {
         int4 s = make_int4(0, 0, 0, 0);
         for (int c = 0; c < S; ++c) {
-          const int4 v = *reinterpret_cast<const int4*>(recv + (c * a.Bp + b) * a.sh + nl);
+          const uint32_t* src = (c == rank ? stg + static_cast<size_t>(c) * slot_words : recv + static_cast<size_t>(c) * slot_words);
+          const int4 v = *reinterpret_cast<const int4*>(src + b * a.sh + nl);
           s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
         }
         int32_t* dst = static_cast<int32_t*>(a.y) + static_cast<int64_t>(b) * a.ldy + n;
@@ -430,7 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int c = 0; c < S; ++c) {
-          const float4 v = *reinterpret_cast<const float4*>(recv + (c * a.Bp + b) * a.sh + nl);
+          const uint32_t* src = (c == rank ? stg + static_cast<size_t>(c) * slot_words : recv + static_cast<size_t>(c) * slot_words);
+          const float4 v = *reinterpret_cast<const float4*>(src + b * a.sh + nl);
           s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
         }
         float o[4] = {s.x, s.y, s.z, s.w};
@@ -466,7 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  __syncthreads();
+  // every owner has received its shares (so every copy out of this CTA's
+  // shared memory is done) before any CTA of the cluster exits
+  __syncwarp();
+  cluster_sync();
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -508,7 +533,7 @@ SkinnyPlan plan_skinny(int kFmt, int Bp, int64_t N, int kst, int lr_boxes) {
     else if (p.dp > 2) --p.dp;
     else break;
   }
-  const size_t recv = static_cast<size_t>(S) * Bp * p.sh * 4;
+  const size_t recv = 2 * static_cast<size_t>(S) * Bp * p.sh * 4;   // staged and received partials
   // more than half an SM's shared memory: one CTA of this kernel per SM, so
   // the TMEM allocation never waits on another cluster's CTA
   p.smem = std::max({total(), recv, kMinSmem}) + 1024;
@@ -520,6 +545,10 @@ cudaError_t launch_one(const CUtensorMap& w, const CUtensorMap& x, const CUtenso
                        const SkinnyArgs& args, int tiles, size_t smem, bool pdl, cudaStream_t st) {
   auto kern = skinny_kernel<kFmt, kOut>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  // same (largest) shared-memory configuration as the activation pass, so CTAs
+  // of the two kernels can share an SM under a dependent launch
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(args.S), static_cast<unsigned>(tiles));
