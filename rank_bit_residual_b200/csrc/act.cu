@@ -6,16 +6,18 @@
 // low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) from the same
 // read of x.
 //
-// Work unit = 128 rows x a range of 128-byte K tiles. Phase 1 streams the
-// unit's x tiles in by TMA (128-byte swizzle), runs the down-projection on
-// tcgen05 (bf16, or tf32 for fp32 x, accumulated in TMEM) and takes column
-// maxima of |x| from the same shared-memory tiles; it writes a partial down
-// tile and a partial maximum. Since fl(a r) is monotone in a, the tensor
-// maximum of |X_hat| is max_k fl(colmax_k r_k). A bounded grid barrier then
-// makes the per-tensor scale known everywhere, and phase 2 writes the codes:
-// from the tiles still held in shared memory when the unit fits there (x is
-// then read from HBM exactly once), else by re-reading the unit from global
-// memory. Phase 2 also sums the partial down tiles into bf16 hi | lo.
+// Work unit = 128 rows x a range of 128-byte K tiles. The kernel runs twice,
+// and the boundary between the two launches is the grid-wide barrier the
+// per-tensor scale needs (an in-kernel barrier would need its counter zeroed
+// before every launch, a graph node that costs more than the barrier itself).
+// Phase 1 streams the unit's x tiles in by TMA (128-byte swizzle), runs the
+// down-projection on tcgen05 (bf16, or tf32 for fp32 x, accumulated in TMEM)
+// and takes column maxima of |x| from the same shared-memory tiles; it writes
+// a partial down tile and a partial maximum. Since fl(a r) is monotone in a,
+// the tensor maximum of |X_hat| is max_k fl(colmax_k r_k). Phase 2 takes the
+// per-tensor scale from the partial maxima, writes the codes from a second
+// read of x (from L2 when x fits there) and sums the partial down tiles into
+// bf16 hi | lo.
 //
 // fp32 evaluation order (the one the oracle's fp32 code mode repeats): the
 // per-element divisions of the definition are multiplies by correctly rounded
@@ -54,15 +56,16 @@ __host__ __device__ constexpr uint32_t pow2_cols(int n) {
 struct ActArgs {
   int B, M;
   int64_t ldx;
-  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, hold, xbuf, fmt_kind, qmax;
+  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, xbuf, fmt_kind, qmax;
+  int phase;        // 1: tiles, column maxima, partial down tiles; 2: codes and the down tile
+  int nparts;       // partial maxima written by phase 1
   const void* x;
   const float* scale;
   const float* gs_given;
   const float* gs_w;
   const void* ld;   // [rank_pad][M], x's dtype
   float* ws_down;   // [ksplit][B][rank_pad]
-  float* ws_max;    // [gridDim.x]
-  unsigned* sync;   // [0] barrier counter, [1] abort flag (zeroed before launch)
+  float* ws_max;    // [nparts]
   void* codes;
   uint8_t* sf;
   __nv_bfloat16* down;
@@ -113,58 +116,17 @@ __device__ __forceinline__ void work_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kWork) : "memory");
 }
 
-// Grid-wide barrier of the work warps of every CTA (see grid_sync; the block
-// barriers are the work warps' own). counter and abort_flag are zeroed before
-// the launch.
-__device__ __forceinline__ bool grid_sync_work(unsigned* counter, unsigned* abort_flag, unsigned* status,
-                                               volatile int* abort_sh) {
-  work_sync();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(counter, 1u);
-    const unsigned target = gridDim.x;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-      unsigned v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-      if (v >= target) break;
-      if (*reinterpret_cast<volatile unsigned*>(abort_flag)) {
-        *abort_sh = 1;
-        break;
-      }
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        record_status(status, kStatusTimeout);
-        atomicExch(abort_flag, 1u);
-        *abort_sh = 1;
-        break;
-      }
-      __nanosleep(64);
-    }
-    __threadfence();
-  }
-  work_sync();
-  return *abort_sh == 0;
-}
-
 // Eight consecutive elements of x (16 bytes of bf16, or 32 of fp32) from a held
 // swizzled tile row or from global memory; cl: column within the unit, a
 // multiple of 8.
 template <typename TIn>
-__device__ __forceinline__ void load8(const uint8_t* xbuf, bool hold, const void* x, int64_t ldx,
-                                      int64_t row, int64_t col0, int r, int cl, uint4 (&u)[2]) {
-  constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));
+__device__ __forceinline__ void load8(const void* x, int64_t ldx, int64_t row, int64_t col0, int cl,
+                                      uint4 (&u)[2]) {
   constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn));
   constexpr int kChunks = 8 / kPerChunk;   // 1 (bf16) or 2 (fp32)
-  if (hold) {
-    const int t = cl / kTileK, c = (cl % kTileK) / kPerChunk;
-    const uint8_t* base = xbuf + static_cast<size_t>(t) * kTileBytes + r * 128;
+  const uint4* g = reinterpret_cast<const uint4*>(static_cast<const TIn*>(x) + row * ldx + col0 + cl);
 #pragma unroll
-    for (int h = 0; h < kChunks; ++h) u[h] = *reinterpret_cast<const uint4*>(base + (((c + h) ^ (r & 7)) << 4));
-  } else {
-    const uint4* g = reinterpret_cast<const uint4*>(static_cast<const TIn*>(x) + row * ldx + col0 + cl);
-#pragma unroll
-    for (int h = 0; h < kChunks; ++h) u[h] = __ldg(g + h);
-  }
+  for (int h = 0; h < kChunks; ++h) u[h] = __ldg(g + h);
 }
 
 template <typename TIn>
@@ -225,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ld_bytes = a.rank_pad * 128;
   uint8_t* xbuf = smem;                                               // a.xbuf tiles
   uint8_t* ldbuf = smem + static_cast<size_t>(a.xbuf) * kTileBytes;   // kLdRing ld tiles
-  float* rcp = reinterpret_cast<float*>(ldbuf + (a.has_ld ? kLdRing * ld_bytes : 0));
+  const bool mma_phase = a.phase == 1 && a.has_ld;   // the down-projection runs in phase 1
+  float* rcp = reinterpret_cast<float*>(ldbuf + (mma_phase ? kLdRing * ld_bytes : 0));
   const uint32_t tcols = pow2_cols(a.rank_pad);
   unsigned* status = a.status;
 
@@ -248,18 +211,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_sh = 0;
     tma_prefetch_desc(&tm_x);
   }
-  if (warp == kMmaWarp && a.has_ld) {
+  if (warp == kMmaWarp && mma_phase) {
     tmem_alloc(&tmem_base_sh, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = a.has_ld ? tmem_base_sh : 0u;
+  const uint32_t tmem = mma_phase ? tmem_base_sh : 0u;
   float run = 0.0f;
   bool ok = true;
 
   // ================================================================ phase 1
+  if (a.phase == 1) {
   // x steps flow through the buffers as one ring over all of this CTA's units:
   // step G + i uses buffer (G + i) % xbuf in its use (G + i) / xbuf (counters
   // in registers: an indexed array would live in local memory)
@@ -290,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    if (a.has_ld) {
+    if (mma_phase) {
       uint32_t G = 0;        // x steps of the previous units
       uint32_t nbatch = 0;   // ld batches whose MMAs were committed to ld_free
       bool pok = true;
@@ -354,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else
                   mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
               }
-              if (!a.hold) mma_commit(&xempty[b]);
+              mma_commit(&xempty[b]);
             }
             if (pok) mma_commit(&ld_free);
           }
@@ -383,15 +347,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b = (G + i) % a.xbuf;
         ok = mbar_wait_warp(&xfull[b], ((G + i) / a.xbuf) & 1, status, &abort_sh) && ok;
         if (ok) run = tile_absmax<TIn>(xbuf + static_cast<size_t>(b) * kTileBytes, rcp + i * kTileK, run);
-        if (!a.hold) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&xempty[b]);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xempty[b]);
       }
-      if (a.has_ld && !a.hold && warp < 4) {
-        // ring mode: drain the unit's accumulator before the next unit's MMAs
-        // (held tiles: one unit per CTA, drained after the codes in phase 2)
-        // TMEM lane = row; warps 0-3 cover the 128 lanes (one lane quarter each)
+      if (mma_phase && warp < 4) {
+        // drain the unit's accumulator into its partial before the next
+        // unit's MMAs; TMEM lane = row, warps 0-3 cover the 128 lanes
         const bool fin = mbar_wait_warp(&mma_done, ucount & 1, status, &abort_sh) && ok;
         tc_fence_after();
         const int row = m0 + warp * 32 + lane;
@@ -425,19 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       float m = red[0];
       for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
-      a.ws_max[blockIdx.x] = m;
+      a.ws_max[blockIdx.x] = ok ? m : 0.0f;
     }
   }
-
-  // ======================================================== grid barrier
-  // (work warps only: the MMA warp's chain may still be running, it is
-  // collected after the codes)
-  if (!producer) ok = grid_sync_work(a.sync, a.sync + 1, status, &abort_sh) && ok;
+  }   // phase 1
 
   // ================================================================ phase 2
-  if (ok && !producer) {
+  if (a.phase == 2 && !producer) {
     float m = 0.0f;
-    for (int i = tid; i < static_cast<int>(gridDim.x); i += kWork) m = fmaxf(m, a.ws_max[i]);
+    for (int i = tid; i < a.nparts; i += kWork) m = fmaxf(m, __ldcg(a.ws_max + i));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     work_sync();
@@ -462,14 +419,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit_range(unit, m0, k_lo, n);
       const int sp = unit / a.nrb;
       const int64_t col0 = static_cast<int64_t>(k_lo) * kTileK;
-      if (!a.hold) {
-        work_sync();
-        for (int j = tid; j < n * kTileK; j += kWork) {
-          const int col = k_lo * kTileK + j;
-          rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
-        }
-        work_sync();
+      work_sync();
+      for (int j = tid; j < n * kTileK; j += kWork) {
+        const int col = k_lo * kTileK + j;
+        rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
       }
+      work_sync();
       const int rows = min(kRows, a.B - m0);
       const int ncols = min(n * kTileK, a.M - k_lo * kTileK);   // a multiple of 32
       if (!nv) {
@@ -486,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool two = r2 < rows;
             uint4 ua[2], ub[2];
             if (live) {
-              load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r, col0, r, cl, ua);
-              if (two) load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r2, col0, r2, cl, ub);
+              load8<TIn>(a.x, a.ldx, m0 + r, col0, cl, ua);
+              if (two) load8<TIn>(a.x, a.ldx, m0 + r2, col0, cl, ub);
             }
             if (live) {
               float v[8];
@@ -517,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int h = 0; h < 2; ++h) {
             uint4 uu[2];
             float v8[8];
-            load8<TIn>(xbuf, a.hold, a.x, a.ldx, m0 + r, col0, r, cl + 8 * h, uu);
+            load8<TIn>(a.x, a.ldx, m0 + r, col0, cl + 8 * h, uu);
             unpack8<TIn>(uu, v8);
 #pragma unroll
             for (int j = 0; j < 8; ++j) xs[8 * h + j] = v8[j];
@@ -542,60 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // down = the K-split partials summed in split order, as bf16 hi | lo
       if (a.has_ld && a.down != nullptr) {
-        int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
-        if (a.hold) {
-          // drain this unit's accumulator into its partial, then the last of
-          // the row block's K splits to arrive sums the whole row block
-          if (warp < 4) {
-            const bool fin = mbar_wait_warp(&mma_done, 0, status, &abort_sh);
-            tc_fence_after();
-            const int row = m0 + warp * 32 + lane;
-            float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * a.rank_pad;
-            for (int c0 = 0; c0 < a.rank_pad; c0 += 32) {
-              uint32_t v[32];
-              __syncwarp();
-              tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-              tmem_ld_wait_regs(v);
-              if (fin && row < a.B) {
-                const int cnt = min(32, a.rank_pad - c0);
-                for (int j = 0; j < cnt; j += 4)
-                  *reinterpret_cast<float4*>(dst + c0 + j) =
-                      make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                  __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-              }
-            }
-            tc_fence_before();
-            if (!fin) abort_sh = 1;
-          }
-          // the row block's K splits meet here (all CTAs are resident: bounded
-          // wait on the arrival count), then each sums its own share of rows
-          __threadfence();
-          work_sync();
-          if (tid == 0) {
-            unsigned* cnt = a.sync + 2 + (unit % a.nrb);
-            atomicAdd(cnt, 1u);
-            const unsigned long long t0 = globaltimer_ns();
-            while (true) {
-              unsigned v;
-              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-              if (v >= static_cast<unsigned>(a.ksplit)) break;
-              if (*reinterpret_cast<volatile unsigned*>(a.sync + 1)) {
-                abort_sh = 1;
-                break;
-              }
-              if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                record_status(status, kStatusTimeout);
-                atomicExch(a.sync + 1, 1u);
-                abort_sh = 1;
-                break;
-              }
-              __nanosleep(64);
-            }
-            __threadfence();
-          }
-          work_sync();
-          if (abort_sh) r_hi = r_lo;
-        }
+        const int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
         const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
         const int cnt = (r_hi - r_lo) * a.rank_pad;
         for (int i = tid; i < cnt; i += kWork) {
@@ -604,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row >= a.B) continue;
           float acc = 0.0f;
           for (int z = 0; z < a.ksplit; ++z)
-            acc += a.ws_down[(static_cast<int64_t>(z) * a.B + row) * a.rank_pad + j];
+            acc += __ldcg(a.ws_down + (static_cast<int64_t>(z) * a.B + row) * a.rank_pad + j);
           acc = __fmul_rn(acc, mult);
           const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
           const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
@@ -635,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (a.has_ld && warp == kMmaWarp) {
+  if (mma_phase && warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, tcols);
   }
@@ -682,16 +584,10 @@ void finish_act_plan(ActPlan& p) {
   }
   p.nunits = p.nrb * p.ksplit;
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
-  // hold the unit's x tiles when they fit and every unit gets a CTA of its own
-  p.hold = 0;
+  // all of a unit's x tiles in flight at once when they fit (a deep TMA queue),
+  // else a ring of kXRing tiles
   p.xbuf = kXRing;
-  if (steps_max <= kMaxHold) {
-    const size_t sm = smem_for(p, steps_max);
-    if (sm <= static_cast<size_t>(kSmemBudget) && p.nunits <= num_sms() * resident_per_sm(sm, p.bf16)) {
-      p.hold = 1;
-      p.xbuf = steps_max;
-    }
-  }
+  if (steps_max <= kMaxHold && smem_for(p, steps_max) <= static_cast<size_t>(kSmemBudget)) p.xbuf = steps_max;
   p.smem = smem_for(p, p.xbuf);
   p.grid = std::min(p.nunits, num_sms() * resident_per_sm(p.smem, p.bf16));
   p.nparts = p.grid;
@@ -728,19 +624,12 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool al
   return p;
 }
 
-// Barrier words: [0] grid barrier counter, [1] abort flag, [2 + rb] K-split
-// arrivals of row block rb (all zeroed before each launch).
-size_t act_sync_bytes(const ActPlan& p) {
-  return static_cast<size_t>(round_up((2 + static_cast<int64_t>(p.nrb)) * 4, 256));
-}
-
 size_t act_scratch_bytes(const ActPlan& p) {
-  if (p.small)   // barrier word, then the partial down tiles (act_small.cu)
-    return 256 +
+  if (p.small)   // partial maxima, then the partial down tiles (act_small.cu)
+    return static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * 4, 256)) +
            (p.rank_pad > 0 ? static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * p.B * p.rank_pad * 4, 256)) : 0) +
            256;
   size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));
-  b += act_sync_bytes(p);
   if (p.rank_pad > 0)
     b += static_cast<size_t>(round_up(static_cast<int64_t>(p.ksplit) * p.B * p.rank_pad * 4, 256));
   return b + 256;
@@ -759,7 +648,6 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
   Carver cv(scratch, ~size_t(0));
   float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));
-  unsigned* sync = static_cast<unsigned*>(cv.take(act_sync_bytes(p)));
   float* ws_down =
       has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4))
              : nullptr;
@@ -772,8 +660,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
     *bad_args = true;
     return cudaSuccess;
   }
-  cudaError_t err = cudaMemsetAsync(sync, 0, (2 + static_cast<size_t>(p.nrb)) * sizeof(unsigned), stream);
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
   ActArgs a{};
   a.B = static_cast<int>(p.B);
   a.M = static_cast<int>(p.M);
@@ -784,8 +671,8 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.nunits = p.nunits;
   a.rank_pad = has_ld ? p.rank_pad : 0;
   a.has_ld = has_ld ? 1 : 0;
-  a.hold = p.hold;
   a.xbuf = p.xbuf;
+  a.nparts = p.grid;
   a.fmt_kind = fmt.kind;
   a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
   a.x = x;
@@ -795,7 +682,6 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.ld = has_ld ? ld : nullptr;
   a.ws_down = ws_down;
   a.ws_max = ws_max;
-  a.sync = sync;
   a.codes = codes;
   a.sf = static_cast<uint8_t*>(sf);
   a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
@@ -804,22 +690,32 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   // without the down factor the launch needs no ld ring (plan keeps its grid)
   ActPlan q = p;
   if (!has_ld) q.rank_pad = 0;
-  const size_t smem = smem_for(q, p.xbuf);
-  void* args[] = {&tm_x, &a};
+  const size_t smem1 = smem_for(q, p.xbuf);
+  // phase 2 keeps only the unit's reciprocals in shared memory
+  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+  const size_t smem2 = static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
+  ActArgs a2 = a;
+  a.phase = 1;
+  a2.phase = 2;
+  a2.xbuf = 0;
   if (xdt == SVDQ_BF16) {
-    err = cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    err = cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(std::max(smem1, smem2)));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_fused_kernel<__nv_bfloat16>),
-                                      dim3(p.grid), dim3(kThreads), args, smem, stream);
+    act_fused_kernel<__nv_bfloat16><<<p.grid, kThreads, smem1, stream>>>(tm_x, a);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    act_fused_kernel<__nv_bfloat16><<<p.nunits, kThreads, smem2, stream>>>(tm_x, a2);
   } else {
     err = cudaFuncSetAttribute(act_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+                               static_cast<int>(std::max(smem1, smem2)));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_fused_kernel<float>), dim3(p.grid),
-                                      dim3(kThreads), args, smem, stream);
+    act_fused_kernel<float><<<p.grid, kThreads, smem1, stream>>>(tm_x, a);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    act_fused_kernel<float><<<p.nunits, kThreads, smem2, stream>>>(tm_x, a2);
   }
-  return err;
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

@@ -5,18 +5,20 @@
 // "flashinfer.gemm.svdquant_linear"): X_hat = x / scale quantised per tensor
 // (INT) or per 16-element block (NVFP4), and the down-projection x ld^T as
 // bf16 hi | lo. At decode sizes the whole of x is a few hundred KB, so the work
-// is latency-bound: this kernel spreads the columns of x over one CTA per SM,
-// keeps each CTA's column chunk in shared memory across one grid barrier, and
-// uses no TMEM (the down-projection is a handful of warp-level MMAs per CTA).
+// is latency-bound: the columns of x are spread over one CTA per SM, and the
+// pass is two plain kernels whose boundary replaces a grid barrier (a barrier
+// word would need zeroing before every launch, a graph node that costs more
+// than the kernels). No TMEM: the down-projection is a handful of warp-level
+// MMAs per CTA.
 //
-//   phase 1  chunk of x -> shared memory; column maxima of |x| times
-//            r_k = fl(1 / scale_k) -> one partial maximum per CTA; partial
-//            down-projection of the chunk -> ws_down[g][b][j]
-//   barrier  bounded; its 64-bit word (zeroed before the launch) counts the
-//            arrivals and carries the largest partial maximum
-//   phase 2  per-tensor scale from that maximum; codes of the chunk
-//            from the shared copy; each CTA sums its share of the (b, j)
-//            down outputs over the partials in a fixed order
+//   stats kernel  chunk of x and of ld -> shared memory; column maxima of |x|
+//                 times r_k = fl(1 / scale_k) -> one partial maximum per CTA;
+//                 partial down-projection of the chunk -> ws_down[g][b][j]
+//   codes kernel  launched as a dependent of the stats kernel: loads its chunk
+//                 of x while that kernel runs, then takes the per-tensor scale
+//                 from the partial maxima, writes the codes of the chunk, and
+//                 sums its share of the (b, j) down outputs over the partials
+//                 in a fixed order
 //
 // fp32 evaluation order of the codes is the one act.cu documents (and the
 // oracle's fp32 code mode repeats): r_k = fl(1 / scale_k), u = fl(1 / s),
@@ -48,8 +50,8 @@ struct SmallArgs {
   const float* gs_given;
   const float* gs_w;
   const void* ld;     // [rank_pad][M], x's dtype
-  float* ws_down;     // [G][B][rank_pad]
-  unsigned long long* sync;   // barrier word (arrivals | max) and abort flag, zeroed before the launch
+  float* ws_max;      // [G] partial maxima
+  float* ws_down;     // [G][B][rank_pad] partial down tiles
   void* codes;
   uint8_t* sf;
   __nv_bfloat16* down;
@@ -86,14 +88,12 @@ __device__ __forceinline__ uint32_t to_tf32(uint32_t f) {
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const SmallArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float red[kWarps];
-  __shared__ float cta_max_sh;
-  __shared__ int abort_sh;
 
-  pdl_trigger();   // a GEMM launched after this kernel may start its weight loads now
+  pdl_trigger();   // the codes kernel launched after this one may start loading x now
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.x;
@@ -106,7 +106,6 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
   uint8_t* lds = xs + static_cast<size_t>(bp16) * pitch;            // rank_pad rows
   float* rcp = reinterpret_cast<float*>(lds + static_cast<size_t>(a.has_ld ? a.rank_pad : 0) * pitch);
   uint32_t* cm = reinterpret_cast<uint32_t*>(rcp + a.wc);           // kThreads column-max slots
-  if (tid == 0) abort_sh = 0;
 
   // ------------------------------------------------------------ loads
   const int vpr = ncols * kEsz / 16;   // 16-byte vectors per chunk row
@@ -170,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
     if (tid == 0) {
       float t = red[0];
       for (int w = 1; w < kWarps; ++w) t = fmaxf(t, red[w]);
-      cta_max_sh = t;
+      a.ws_max[g] = t;
     }
   }
 
@@ -226,40 +225,44 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_kernel(const SmallArgs 
     }
   }
 
-  // ================================================================ barrier
-  // One 64-bit word: arrivals in the low half, the largest partial maximum
-  // (non-negative floats order like their bit patterns) in the high half. Each
-  // CTA raises the maximum, then adds its arrival with release semantics; once
-  // the count reaches G an acquire load of the word also yields the final max.
-  __syncthreads();   // this CTA's partial down tile is written
-  if (tid == 0) {
-    unsigned* words = reinterpret_cast<unsigned*>(a.sync);
-    atomicMax(words + 1, __float_as_uint(cta_max_sh));
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(words) : "memory");
-    const unsigned long long t0 = globaltimer_ns();
-    unsigned long long v = 0;
-    while (true) {
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.sync) : "memory");
-      if (static_cast<unsigned>(v & 0xFFFFFFFFull) >= static_cast<unsigned>(a.G)) break;
-      if (*reinterpret_cast<volatile unsigned*>(words + 2)) {
-        abort_sh = 1;
-        break;
-      }
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        record_status(a.status, kStatusTimeout);
-        atomicExch(words + 2, 1u);
-        abort_sh = 1;
-        break;
-      }
-    }
-    red[0] = __uint_as_float(static_cast<unsigned>(v >> 32));
-  }
-  __syncthreads();
-  if (abort_sh) return;
+}
 
-  // ================================================================ phase 2
-  const float m = red[0];
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const SmallArgs a) {
+  constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ float red[kWarps];
+
+  pdl_trigger();   // a GEMM launched after this kernel may start its weight loads now
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.x;
+  const int c0 = g * a.wc;
+  const int ncols = min(a.wc, a.M - c0);     // a multiple of 32
+  const int B = a.B;
+  const int pitch = chunk_pitch(a.wc, kEsz);
+  uint8_t* xs = smem;
+  float* rcp = reinterpret_cast<float*>(xs + static_cast<size_t>((B + 15) & ~15) * pitch);
+
+  // x and the scale do not come from the stats kernel: loaded while it runs
+  const int vpr = ncols * kEsz / 16;
+  for (int i = tid; i < B * vpr; i += kThreads) {
+    const int r = i / vpr, v = i - r * vpr;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+        static_cast<const uint8_t*>(a.x) + (static_cast<int64_t>(r) * a.ldx + c0) * kEsz) + v);
+    *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = u;
+  }
+  for (int k = tid; k < ncols; k += kThreads) rcp[k] = __frcp_rn(__ldg(a.scale + c0 + k));
+  pdl_wait();   // the partial maxima and down tiles of every CTA of the stats kernel
+  float m = 0.0f;
+  for (int i = tid; i < a.G; i += kThreads) m = fmaxf(m, __ldcg(a.ws_max + i));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = red[0];
+  for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w]);
+
   const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
   float u = 0.0f, gs_x = 1.0f;
   if (nv) {
@@ -383,6 +386,37 @@ size_t small_smem(const ActPlan& p, bool has_ld) {
          static_cast<size_t>(p.wc) * 4 + kThreads * 4 + 64;
 }
 
+// The stats kernel, then the codes kernel as a dependent launch (it may start
+// while the stats kernel runs and waits for it with griddepcontrol.wait). Both
+// take the largest shared-memory configuration, the one the GEMM launched after
+// them needs, so CTAs of the three kernels can share SMs.
+template <typename K1, typename K2>
+cudaError_t launch_pair_of_kernels(K1 k1, K2 k2, const SmallArgs& a, int grid, size_t smem1, size_t smem2,
+                                   cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem1));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k2, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
+  k1<<<grid, kThreads, smem1, stream>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem2;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k2, a);
+}
+
 }  // namespace
 
 void finish_act_plan_small(ActPlan& p) {
@@ -391,7 +425,6 @@ void finish_act_plan_small(ActPlan& p) {
   p.ksplit = p.grid;
   p.nunits = p.grid;
   p.nparts = p.grid;
-  p.hold = 1;
   p.xbuf = 0;
   p.smem = small_smem(p, p.rank_pad > 0);
 }
@@ -410,11 +443,9 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
     return cudaSuccess;
   }
   Carver cv(scratch, ~size_t(0));
-  auto* sync = static_cast<unsigned long long*>(cv.take(256));
+  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * 4));
   float* ws_down = has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.grid) * p.B * p.rank_pad * 4))
                           : nullptr;
-  cudaError_t err = cudaMemsetAsync(sync, 0, 16, stream);
-  if (err != cudaSuccess) return err;
   SmallArgs a{};
   a.B = static_cast<int>(p.B);
   a.M = static_cast<int>(p.M);
@@ -430,36 +461,20 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
   a.gs_given = fmt.kind == SVDQ_KIND_NVFP4 ? act_global_scale : nullptr;
   a.gs_w = fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr;
   a.ld = has_ld ? ld : nullptr;
+  a.ws_max = ws_max;
   a.ws_down = ws_down;
-  a.sync = sync;
   a.codes = codes;
   a.sf = static_cast<uint8_t*>(sf);
   a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
   a.act_scale = act_scale;
   a.status = device_status_word();
-  const size_t smem = small_smem(p, has_ld);
-  void* args[] = {&a};
-  if (xdt == SVDQ_BF16) {
-    err = cudaFuncSetAttribute(act_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    // the largest shared-memory configuration, the one the GEMM launched after
-    // this kernel needs: with equal configurations its CTAs can share SMs with
-    // these and start early (a different split makes an SM drain first)
-    err = cudaFuncSetAttribute(act_small_kernel<__nv_bfloat16>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
-    if (err != cudaSuccess) return err;
-    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<__nv_bfloat16>), dim3(p.grid),
-                                       dim3(kThreads), args, smem, stream);
-  }
-  err = cudaFuncSetAttribute(act_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(act_small_kernel<float>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-  if (err != cudaSuccess) return err;
-  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(act_small_kernel<float>), dim3(p.grid),
-                                     dim3(kThreads), args, smem, stream);
+  const size_t smem1 = small_smem(p, has_ld);
+  const size_t smem2 = small_smem(p, false);
+  if (xdt == SVDQ_BF16)
+    return launch_pair_of_kernels(act_small_stats_kernel<__nv_bfloat16>, act_small_codes_kernel<__nv_bfloat16>, a,
+                                  p.grid, smem1, smem2, stream);
+  return launch_pair_of_kernels(act_small_stats_kernel<float>, act_small_codes_kernel<float>, a, p.grid, smem1,
+                                smem2, stream);
 }
 
 }  // namespace svdq

@@ -63,7 +63,7 @@ enum SkinnyFmt { kFmtInt8 = 0, kFmtInt4 = 1, kFmtNvfp4 = 2 };
 
 struct SkinnyArgs {
   int B, Bp, N, M, S, kst, lr_boxes, sh;
-  int da, db, dp, a_slot, b_slot;
+  int dr, dp, a_slot, b_slot;   // ring depth (both operands), packed-weight ring depth
   int katoms;
   const float* s_x;
   const float* s_w;
@@ -106,10 +106,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_lu, const __grid_constant__ CUtensorMap tm_dn,
                   const SkinnyArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_a[kMaxRing];
-  __shared__ __align__(8) uint64_t empty_a[kMaxRing];
-  __shared__ __align__(8) uint64_t full_b[kMaxRing];
-  __shared__ __align__(8) uint64_t empty_b[kMaxRing];
+  // one ring for both operands: full[s] completes when the weight side (TMA, or
+  // the four widening warps) and the activation side have both landed; one
+  // MMA commit per step frees both halves of the slot (empty[s])
+  __shared__ __align__(8) uint64_t full[kMaxRing];
+  __shared__ __align__(8) uint64_t empty[kMaxRing];
   __shared__ __align__(8) uint64_t full_p[kMaxRing];
   __shared__ __align__(8) uint64_t empty_p[kMaxRing];
   __shared__ __align__(8) uint64_t tmem_full;
@@ -121,8 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring_a = smem;
-  uint8_t* ring_b = ring_a + static_cast<size_t>(a.da) * a.a_slot;
-  uint8_t* ring_p = ring_b + static_cast<size_t>(a.db) * a.b_slot;
+  uint8_t* ring_b = ring_a + static_cast<size_t>(a.dr) * a.a_slot;
+  uint8_t* ring_p = ring_b + static_cast<size_t>(a.dr) * a.b_slot;
   uint32_t* recv_base = reinterpret_cast<uint32_t*>(smem);   // partials: reuse the rings once every MMA is done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,10 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxRing; ++s) {
-      mbar_init(&full_a[s], kFullACount);
-      mbar_init(&empty_a[s], 1);
-      mbar_init(&full_b[s], 1);
-      mbar_init(&empty_b[s], 1);
+      mbar_init(&full[s], kFullACount + 1);
+      mbar_init(&empty[s], 1);
       mbar_init(&full_p[s], 1);
       mbar_init(&empty_p[s], 4);
     }
@@ -175,12 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ia = 0, ip = 0;   // A-ring loads (lu boxes, direct weight tiles) and packed loads issued
       // low-rank step i (< nlr): the lu box rank + i S into A slot i % da
       auto load_lu = [&](int i) {
-        const int s = i % a.da;
-        if (i >= a.da) ok = ok && mbar_wait(&empty_a[s], ((i / a.da) - 1) & 1, status, &abort_sh);
+        const int s = i % a.dr;
+        if (i >= a.dr) ok = ok && mbar_wait(&empty[s], ((i / a.dr) - 1) & 1, status, &abort_sh);
         if (!ok) return;
-        mbar_arrive_expect_tx(&full_a[s], kATile);
-        for (uint32_t c = 1; c < kFullACount; ++c) mbar_arrive(&full_a[s]);
-        tma_load_2d(ring_a + static_cast<size_t>(s) * a.a_slot, &tm_lu, &full_a[s], 64 * (rank + i * S), n0);
+        mbar_arrive_expect_tx(&full[s], kATile);
+        for (uint32_t c = 1; c < kFullACount; ++c) mbar_arrive(&full[s]);
+        tma_load_2d(ring_a + static_cast<size_t>(s) * a.a_slot, &tm_lu, &full[s], 64 * (rank + i * S), n0);
         ++ia;
       };
       if constexpr (kFmt == kFmtInt4) {
@@ -204,19 +203,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_lu(i);
             continue;
           }
-          const int s = i % a.da, k = k_lo + (i - nlr);
-          if (i >= a.da) ok = ok && mbar_wait(&empty_a[s], ((i / a.da) - 1) & 1, status, &abort_sh);
+          const int s = i % a.dr, k = k_lo + (i - nlr);
+          if (i >= a.dr) ok = ok && mbar_wait(&empty[s], ((i / a.dr) - 1) & 1, status, &abort_sh);
           if (!ok) break;
           uint8_t* dst = ring_a + static_cast<size_t>(s) * a.a_slot;
           if constexpr (kFmt == kFmtNvfp4) {
             const int na = min(4, a.katoms - 4 * k);
-            mbar_arrive_expect_tx(&full_a[s], kATile + na * 512);
-            tma_load_2d(dst, &tm_w, &full_a[s], 128 * k, n0);
+            mbar_arrive_expect_tx(&full[s], kATile + na * 512);
+            tma_load_2d(dst, &tm_w, &full[s], 128 * k, n0);
             bulk_load(dst + kATile, a.sfw + (static_cast<int64_t>(n0 / 128) * a.katoms + 4 * k) * 512, na * 512,
-                      &full_a[s]);
+                      &full[s]);
           } else {
-            mbar_arrive_expect_tx(&full_a[s], kATile);
-            tma_load_2d(dst, &tm_w, &full_a[s], 128 * k, n0);
+            mbar_arrive_expect_tx(&full[s], kATile);
+            tma_load_2d(dst, &tm_w, &full[s], 128 * k, n0);
           }
           ++ia;
         }
@@ -226,8 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // block can exit (on the normal path every load was consumed)
         abort_sh = 1;
         if (kFmt != kFmtInt4)
-          for (int q = max(0, ia - a.da); q < ia; ++q)
-            mbar_wait(&full_a[q % a.da], (q / a.da) & 1, status, nullptr, 1000000ull);
+          for (int q = max(0, ia - a.dr); q < ia; ++q)
+            mbar_wait(&full[q % a.dr], (q / a.dr) & 1, status, nullptr, 1000000ull);
         for (int q = max(0, ip - a.dp); q < ip; ++q)
           mbar_wait(&full_p[q % a.dp], (q / a.dp) & 1, status, nullptr, 1000000ull);
       }
@@ -240,30 +239,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ib = 0;   // loads issued
       const int xbytes = a.Bp * 128;
       for (int i = 0; i < nsteps && ok; ++i, ++ib) {
-        const int s = i % a.db;
-        if (i >= a.db) ok = mbar_wait(&empty_b[s], ((i / a.db) - 1) & 1, status, &abort_sh);
+        const int s = i % a.dr;
+        if (i >= a.dr) ok = mbar_wait(&empty[s], ((i / a.dr) - 1) & 1, status, &abort_sh);
         if (!ok) break;
         uint8_t* dst = ring_b + static_cast<size_t>(s) * a.b_slot;
         if (i < nlr) {
-          mbar_arrive_expect_tx(&full_b[s], xbytes);
-          tma_load_2d(dst, &tm_dn, &full_b[s], 64 * (rank + i * S), 0);
+          mbar_arrive_expect_tx(&full[s], xbytes);
+          tma_load_2d(dst, &tm_dn, &full[s], 64 * (rank + i * S), 0);
         } else {
           const int k = k_lo + (i - nlr);
           if constexpr (kFmt == kFmtNvfp4) {
             const int na = min(4, a.katoms - 4 * k);
-            mbar_arrive_expect_tx(&full_b[s], xbytes + na * 512);
-            tma_load_2d(dst, &tm_x, &full_b[s], 128 * k, 0);
-            bulk_load(dst + xbytes, a.sfx + static_cast<int64_t>(4 * k) * 512, na * 512, &full_b[s]);
+            mbar_arrive_expect_tx(&full[s], xbytes + na * 512);
+            tma_load_2d(dst, &tm_x, &full[s], 128 * k, 0);
+            bulk_load(dst + xbytes, a.sfx + static_cast<int64_t>(4 * k) * 512, na * 512, &full[s]);
           } else {
-            mbar_arrive_expect_tx(&full_b[s], xbytes);
-            tma_load_2d(dst, &tm_x, &full_b[s], 128 * k, 0);
+            mbar_arrive_expect_tx(&full[s], xbytes);
+            tma_load_2d(dst, &tm_x, &full[s], 128 * k, 0);
           }
         }
       }
       if (!ok) {
         abort_sh = 1;
-        for (int q = max(0, ib - a.db); q < ib; ++q)
-          mbar_wait(&full_b[q % a.db], (q / a.db) & 1, status, nullptr, 1000000ull);
+        for (int q = max(0, ib - a.dr); q < ib; ++q)
+          mbar_wait(&full[q % a.dr], (q / a.dr) & 1, status, nullptr, 1000000ull);
       }
     }
   } else if (warp == kWarpMma) {
@@ -285,9 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bool ok = true;
       for (int i = 0; i < nsteps && ok; ++i) {
-        const int sa = i % a.da, sb = i % a.db;
-        ok = mbar_wait(&full_a[sa], (i / a.da) & 1, status, &abort_sh) &&
-             mbar_wait(&full_b[sb], (i / a.db) & 1, status, &abort_sh);
+        const int sa = i % a.dr, sb = sa;
+        ok = mbar_wait(&full[sa], (i / a.dr) & 1, status, &abort_sh);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(ring_a + static_cast<size_t>(sa) * a.a_slot);
@@ -320,8 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      (r > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&empty_a[sa]);
-        mma_commit(&empty_b[sb]);
+        mma_commit(&empty[sa]);
       }
       if (ok) mma_commit(&tmem_full);
       if (!ok) abort_sh = 1;
@@ -335,9 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = (warp - kWarpEpi0) * 32 + lane;   // 0..127
       bool ok = true;
       for (int r = 0; r < nres && ok; ++r) {
-        const int ps = r % a.dp, i = nlr + r, as = i % a.da;
+        const int ps = r % a.dp, i = nlr + r, as = i % a.dr;
         ok = mbar_wait_warp(&full_p[ps], (r / a.dp) & 1, status, &abort_sh);
-        if (ok && i >= a.da) ok = mbar_wait_warp(&empty_a[as], ((i / a.da) - 1) & 1, status, &abort_sh);
+        if (ok && i >= a.dr) ok = mbar_wait_warp(&empty[as], ((i / a.dr) - 1) & 1, status, &abort_sh);
         if (!ok) break;
         const uint8_t* src = ring_p + static_cast<size_t>(ps) * kPSlot;
         uint8_t* dst = ring_a + static_cast<size_t>(as) * a.a_slot;
@@ -355,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&full_a[as]);
+          mbar_arrive(&full[as]);
           mbar_arrive(&empty_p[ps]);
         }
       }
@@ -387,16 +384,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t* dst = stg + static_cast<size_t>(p) * slot_words + nl;
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
       const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
-      for (int c0 = 0; c0 < a.B; c0 += 16) {
-        uint32_t acc[16], up[16];
+      for (int c0 = 0; c0 < a.B; c0 += 32) {
+        uint32_t acc[32], up[32];
         __syncwarp();
-        tmem_ld_32x32b_x16(lane_addr + c0, acc);
-        if (lr_here) tmem_ld_32x32b_x16(lane_addr + kLrCol + c0, up);
+        if (c0 + 16 < a.Bp) {   // 32 columns are allocated to the accumulator
+          tmem_ld_32x32b_x32(lane_addr + c0, acc);
+          if (lr_here) tmem_ld_32x32b_x32(lane_addr + kLrCol + c0, up);
+        } else {
+          tmem_ld_32x32b_x16(lane_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(acc));
+          if (lr_here) tmem_ld_32x32b_x16(lane_addr + kLrCol + c0, *reinterpret_cast<uint32_t(*)[16]>(up));
+        }
         tmem_ld_wait_regs(acc);
         if (lr_here) tmem_ld_wait_regs(up);
-        const int cnt = min(16, a.B - c0);
+        const int cnt = min(32, a.B - c0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 32; ++j) {
           if (j >= cnt) break;
           uint32_t v = acc[j];
           if (kFmt != kFmtNvfp4 && kOut != kOutI32) {
@@ -499,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct SkinnyPlan {
-  int S, sh, da, db, dp, a_slot, b_slot;
+  int S, sh, dr, dp, a_slot, b_slot;
   size_t smem;
 };
 
@@ -520,16 +522,13 @@ SkinnyPlan plan_skinny(int kFmt, int Bp, int64_t N, int kst, int lr_boxes) {
   const int nres_max = static_cast<int>(ceil_div(kst, S));
   const int nsteps_max = nres_max + static_cast<int>(ceil_div(lr_boxes, S));
   p.dp = kFmt == kFmtInt4 ? std::min(nres_max, kMaxRing) : 0;
-  p.da = std::min(nsteps_max, kFmt == kFmtInt4 ? 4 : 6);
-  p.db = std::min(nsteps_max, 4);
+  p.dr = std::min(nsteps_max, kMaxRing);
   auto total = [&]() {
-    return static_cast<size_t>(p.da) * p.a_slot + static_cast<size_t>(p.db) * p.b_slot +
-           static_cast<size_t>(p.dp) * kPSlot;
+    return static_cast<size_t>(p.dr) * (p.a_slot + p.b_slot) + static_cast<size_t>(p.dp) * kPSlot;
   };
   while (total() > kSmemBudget) {
     if (p.dp > 4) --p.dp;
-    else if (p.db > 2) --p.db;
-    else if (p.da > 2) --p.da;
+    else if (p.dr > 2) --p.dr;
     else if (p.dp > 2) --p.dp;
     else break;
   }
@@ -613,8 +612,7 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   a.kst = kst;
   a.lr_boxes = lr_boxes;
   a.sh = p.sh;
-  a.da = p.da;
-  a.db = p.db;
+  a.dr = p.dr;
   a.dp = p.dp;
   a.a_slot = p.a_slot;
   a.b_slot = p.b_slot;

@@ -52,7 +52,6 @@ struct ActPlan {
   int nsteps;      // K tiles
   int ksplit;      // K ranges per row block
   int nunits;      // nrb * ksplit work units
-  int hold;        // 1: each unit keeps its x tiles in shared memory for phase 2
   int xbuf;        // x tile buffers per CTA
   int grid;        // CTAs of the cooperative launch (all resident)
   int nparts;      // partial maxima written (one per CTA)

@@ -74,3 +74,53 @@ def test_empty_batch_is_a_no_op():
     x = torch.zeros((0, 64), dtype=torch.bfloat16, device=device())
     codes, sf, s, down = rb.svdq_quantize_act(x, torch.ones(64, device=device()), "int4")
     assert codes.shape == (0, 64)
+
+
+# long batches (B >= 1024) take the row-slab kernels: ragged last slab, M not a
+# multiple of the chunk width, both input types
+LONG = [(1024, 256), (1100, 96), (2048, 3072)]
+
+
+@pytest.mark.parametrize("B,M", LONG)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_long_batch_int_codes_and_scale(B, M, dtype, bits):
+    wl = make_case(B, M, 16, rank=0, seed=B + M + bits, dtype=dtype)
+    codes, sf, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), f"int{bits}")
+    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, bits)
+    assert np.float32(s.item()) == s_o, (s.item(), s_o)
+    assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype} int{bits}")
+
+
+@pytest.mark.parametrize("B,M", LONG)
+@pytest.mark.parametrize("given_gs", [False, True])
+def test_long_batch_nvfp4_codes_scales_and_layout(B, M, given_gs):
+    wl = make_case(B, M, 16, rank=0, seed=3 * B + M)
+    gs = np.float32(777.25) if given_gs else None
+    gs_t = to_dev(np.array([gs], np.float32), torch.float32) if given_gs else None
+    codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "nvfp4",
+                                           act_global_scale=gs_t)
+    c_o, sf_o, g_o = onv.quantize(ocodes.smooth_fp32(wl.x, wl.scale), gs=gs)
+    assert np.float32(g.item()) == np.float32(g_o)
+    assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
+    assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
+
+
+@pytest.mark.parametrize("B,M,rank", [(1024, 512, 32), (1100, 96, 256), (2048, 3072, 40)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_long_batch_down_projection(B, M, rank, dtype):
+    wl = make_case(B, M, 16, rank=0, seed=5 * B + rank, dtype=dtype)
+    rp = (rank + 15) // 16 * 16
+    rng = np.random.default_rng(rank + 1)
+    ld = np.zeros((rp, M), np.float32)
+    ld[:rank] = to_bf16(rng.standard_normal((rank, M)).astype(np.float32) * 0.1)
+    ld_t = to_dev(ld, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    codes, _, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "int4", ld=ld_t)
+    d = down.float().cpu().numpy().astype(np.float64)
+    got = d[:, :rp] + d[:, rp:]
+    want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
+    tol = 2e-5 if dtype == "bf16" else 3e-3
+    assert rel_fro(got, want) <= tol, rel_fro(got, want)
+    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+    assert np.float32(s.item()) == s_o
+    assert_codes_match(codes.cpu().numpy(), q, near)
