@@ -1,4 +1,5 @@
-// act.cu - the activation pass of the SVDQuant linear, one cooperative kernel.
+// act.cu - the activation pass of the SVDQuant linear for batches of more
+// than 128 rows: a stats kernel and a codes kernel.
 //
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula items 1
 // and 3: X_hat = x / scale is quantised per tensor (INT grid, or NVFP4 blocks
@@ -6,18 +7,22 @@
 // low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) from the same
 // read of x.
 //
-// Work unit = 128 rows x a range of 128-byte K tiles. The kernel runs twice,
-// and the boundary between the two launches is the grid-wide barrier the
-// per-tensor scale needs (an in-kernel barrier would need its counter zeroed
-// before every launch, a graph node that costs more than the barrier itself).
-// Phase 1 streams the unit's x tiles in by TMA (128-byte swizzle), runs the
-// down-projection on tcgen05 (bf16, or tf32 for fp32 x, accumulated in TMEM)
-// and takes column maxima of |x| from the same shared-memory tiles; it writes
-// a partial down tile and a partial maximum. Since fl(a r) is monotone in a,
-// the tensor maximum of |X_hat| is max_k fl(colmax_k r_k). Phase 2 takes the
-// per-tensor scale from the partial maxima, writes the codes from a second
-// read of x (from L2 when x fits there) and sums the partial down tiles into
-// bf16 hi | lo.
+// Work unit = 128 rows x a range of columns; the per-tensor scale needs every
+// unit's maximum before any code is written, and the boundary between the
+// two kernels is that grid-wide barrier (an in-kernel barrier would need its
+// counter zeroed before every launch, a graph node that costs more than the
+// barrier itself).
+//   stats kernel  streams the unit's rows with coalesced 16-byte loads (whole
+//                 row segments: DRAM pages are read front to back), takes the
+//                 column maxima of |x| from registers, and runs the unit's
+//                 down-projection x ld^T with warp-level MMAs from padded
+//                 shared-memory tiles; it writes one partial maximum per CTA
+//                 and one partial down tile per unit. Since fl(a r) is monotone
+//                 in a, the tensor maximum of |X_hat| is max_k fl(colmax_k r_k).
+//   codes kernel  takes the per-tensor scale from the partial maxima, writes
+//                 the codes from a second read of x (from L2 when x fits
+//                 there) and sums each row block's partial down tiles in split
+//                 order into bf16 hi | lo.
 //
 // fp32 evaluation order (the one the oracle's fp32 code mode repeats): the
 // per-element divisions of the definition are multiplies by correctly rounded
@@ -38,27 +43,21 @@ namespace svdq {
 namespace {
 
 constexpr int kWorkWarps = 16;
-constexpr int kWork = 32 * kWorkWarps;      // threads for column maxima, codes and down
-constexpr int kThreads = kWork + 64;        // + a TMA warp and an MMA warp
-constexpr int kTmaWarp = kWorkWarps;
-constexpr int kMmaWarp = kWorkWarps + 1;
-constexpr int kRows = 128;                  // rows per unit (MMA M)
-constexpr int kTileBytes = kRows * 128;     // one 128 x 128-byte x tile
-constexpr int kXRing = 4;                   // x tile buffers when the tiles are not held
-constexpr int kLdRing = 6;                  // ld tile slots
-constexpr int kMaxHold = 12;                // x tiles a unit may keep in shared memory
-constexpr int kSmemBudget = 224 * 1024;
-
-__host__ __device__ constexpr uint32_t pow2_cols(int n) {
-  return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : 256u;
-}
+constexpr int kWork = 32 * kWorkWarps;      // threads of both kernels
+constexpr int kRows = 128;                  // rows per unit
+constexpr int kTileBytes = 128;             // bytes of a row per column tile (64 bf16 / 32 fp32)
+constexpr int kSub = 256;                   // bytes of a row per stats sub-chunk (two tiles)
+constexpr int kPitch = kSub + 16;           // padded shared row: 8 ldmatrix rows hit distinct banks
+constexpr int kMaxStages = 6;
+constexpr int kScaleBytes = 512;            // a stage's scale values (at most 128 columns)
+constexpr size_t kStatsSmemBudget = 220 * 1024;
 
 struct ActArgs {
   int B, M;
   int64_t ldx;
-  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, xbuf, fmt_kind, qmax;
-  int phase;        // 1: tiles, column maxima, partial down tiles; 2: codes and the down tile
-  int nparts;       // partial maxima written by phase 1
+  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
+  int nparts;       // partial maxima written by the stats kernel
+  int stages;       // stats kernel: shared-memory stages
   const void* x;
   const float* scale;
   const float* gs_given;
@@ -70,55 +69,11 @@ struct ActArgs {
   uint8_t* sf;
   __nv_bfloat16* down;
   float* act_scale;
-  unsigned* status;
 };
 
-// Column maxima of |x| over a 128 x 128-byte swizzled tile (work threads only,
-// t < kWork). Thread t owns the
-// logical 16-byte chunk c = t % 8 of rows t/8 and t/8 + 64; it folds
-// fl(colmax r_k) of its chunk's columns into `run` (rcp: reciprocals of the
-// tile's columns, 0 past M).
-template <typename TIn>
-__device__ __forceinline__ float tile_absmax(const uint8_t* tile, const float* rcp, float run) {
-  const int tid = threadIdx.x;
-  const int c = tid & 7;
-  const int rg = tid >> 3;
-  const int p = c ^ (rg & 7);  // rows rg + 64 i share rg & 7
-  uint32_t mx[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int i = 0; i < kRows / (kWork / 8); ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + (rg + (kWork / 8) * i) * 128 + p * 16);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if constexpr (sizeof(TIn) == 2)
-        mx[q] = __vmaxu2(mx[q], w[q] & 0x7FFF7FFFu);
-      else
-        mx[q] = max(mx[q], w[q] & 0x7FFFFFFFu);
-    }
-  }
-  if constexpr (sizeof(TIn) == 2) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q] << 16), rcp[8 * c + 2 * q]));
-      run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q] & 0xFFFF0000u), rcp[8 * c + 2 * q + 1]));
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) run = fmaxf(run, __fmul_rn(__uint_as_float(mx[q]), rcp[4 * c + q]));
-  }
-  return run;
-}
 
-// -------------------------------------------------------------- the kernel
-// Barrier among the work warps only (the TMA and MMA warps run their own loops).
-__device__ __forceinline__ void work_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kWork) : "memory");
-}
-
-// Eight consecutive elements of x (16 bytes of bf16, or 32 of fp32) from a held
-// swizzled tile row or from global memory; cl: column within the unit, a
-// multiple of 8.
+// Eight consecutive elements of x (16 bytes of bf16, or 32 of fp32) from
+// global memory; cl: column within the unit, a multiple of 8.
 template <typename TIn>
 __device__ __forceinline__ void load8(const void* x, int64_t ldx, int64_t row, int64_t col0, int cl,
                                       uint4 (&u)[2]) {
@@ -139,267 +94,267 @@ __device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(uint32_t f) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__uint_as_float(f)));
+  return r;
+}
+
+// Copy 16 bytes global -> shared, bypassing L1; src_bytes = 0 fills zeros and
+// reads nothing (src must still be a valid address).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const float* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Waits until at most n of this thread's copy groups are still in flight.
-__device__ __forceinline__ void cp_async_wait(int n) {
-  switch (n) {
-    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+template <int kN>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kN) : "memory");
+}
+// Wait until at most stages - 2 groups are pending (stages in [2, kMaxStages]).
+__device__ __forceinline__ void cp_async_wait_ring(int stages) {
+  switch (stages) {
+    case 2: cp_async_wait<0>(); break;
+    case 3: cp_async_wait<1>(); break;
+    case 4: cp_async_wait<2>(); break;
+    case 5: cp_async_wait<3>(); break;
+    default: cp_async_wait<4>(); break;
   }
 }
 
-// Warp roles: warps 0-15 ("work") take the column maxima in phase 1 and write
-// the codes and the down factor in phase 2; warp 16 loads the x tiles by TMA
-// (lane 0); warp 17 copies the ld tiles with cp.async (all lanes: a path apart
-// from the TMA queue, so the small ld tiles never wait behind the x tiles) and
-// issues the down-projection MMAs (lane 0). No block-wide barrier separates the
-// K steps: the work warps follow the x tiles as they land, and the MMA chain
-// runs on its own. The MMA warp issues one throwaway MMA first: the first
-// tcgen05.mma a kernel issues takes microseconds longer than the ones after
-// it, and this way that start-up overlaps the first loads.
+// Running maximum of |x| over one 32-bit word of a row: two bf16 lanes (the
+// packed 16-bit magnitudes, one SIMD max) or one fp32 (its magnitude bits);
+// for non-negative values both orders agree with the float order.
 template <typename TIn>
-__global__ void __launch_bounds__(kThreads, 1)
-    act_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const ActArgs a) {
-  constexpr int kTileK = 128 / static_cast<int>(sizeof(TIn));   // elements per 128-byte row
-  constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn)); // elements per 16 bytes
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t xfull[kMaxHold];
-  __shared__ __align__(8) uint64_t xempty[kMaxHold];
-  __shared__ __align__(8) uint64_t ld_free;
-  __shared__ __align__(8) uint64_t mma_done;
-  __shared__ __align__(8) uint64_t tmem_free;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
+__device__ __forceinline__ uint32_t abs_max_word(uint32_t m, uint32_t w) {
+  if constexpr (sizeof(TIn) == 2)
+    return __vmaxu2(m, w & 0x7FFF7FFFu);
+  else
+    return max(m, w & 0x7FFFFFFFu);
+}
+template <typename TIn>
+__device__ __forceinline__ uint32_t max_word(uint32_t m, uint32_t w) {
+  if constexpr (sizeof(TIn) == 2)
+    return __vmaxu2(m, w);
+  else
+    return max(m, w);
+}
+
+// ------------------------------------------------------------ stats kernel
+// A unit is streamed in sub-chunks of kSub bytes per row through a ring of
+// `stages` shared-memory stages filled by cp.async (stages - 1 sub-chunks in
+// flight while one is consumed); a stage holds the x rows, the ld rows and the
+// sub-chunk's scale values. Copies: thread t moves the 16-byte piece t % 16 of
+// rows t / 16 + 32 i (i < 4), so a warp moves two whole 256-byte row segments
+// per instruction. Column maxima: warp w scans 32-bit words 4 w .. 4 w + 3 of
+// rows l / 4 + 8 i (lane l, i < 16; conflict-free with the padded pitch), the
+// eight row slices meet by shuffles, and each column's fl(colmax r_k) is taken
+// once. Down projection: warp w owns m-tile w % 8 of the 128 x rank_pad tile
+// and n-tiles w / 8 + 2 q (q < kP), so one A fragment serves all of its MMAs;
+// the fp32 accumulators live across the unit's sub-chunks.
+template <typename TIn, int kP>
+__global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
+  constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  constexpr int kSubCols = kSub / kEsz;             // 128 bf16 or 64 fp32 columns
+  constexpr int kPer16 = 16 / kEsz;                 // elements per 16-byte piece
+  constexpr int kKStep = kEsz == 2 ? 16 : 8;        // K of one warp MMA
+  constexpr int kTileK = kTileBytes / kEsz;         // columns per K tile
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kWorkWarps];
 
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp >= kWorkWarps;   // the TMA or the MMA warp
-  const int ld_bytes = a.rank_pad * 128;
-  uint8_t* xbuf = smem;                                               // a.xbuf tiles
-  uint8_t* ldbuf = smem + static_cast<size_t>(a.xbuf) * kTileBytes;   // kLdRing ld tiles
-  const bool mma_phase = a.phase == 1 && a.has_ld;   // the down-projection runs in phase 1
-  float* rcp = reinterpret_cast<float*>(ldbuf + (mma_phase ? kLdRing * ld_bytes : 0));
-  const uint32_t tcols = pow2_cols(a.rank_pad);
-  unsigned* status = a.status;
+  const int rp = a.rank_pad;                        // 0 without the down factor
+  const int stages = a.stages;
+  const int stage_bytes = (kRows + rp) * kPitch + kScaleBytes;
+  const int piece = tid & 15, rg = tid >> 4;
+  const int wi = warp * 4 + (lane & 3), rs = lane >> 2;   // column-max word and row slice
+  const int gid = lane >> 2, tig = lane & 3;
+  const int mt = warp & 7, nt0 = warp >> 3, nnt = rp / 8;
+  const TIn* x = static_cast<const TIn*>(a.x);
+  const TIn* ld = static_cast<const TIn*>(a.ld);
+  float run = 0.0f;
 
+  for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
+    const int rb = unit % a.nrb, sp = unit / a.nrb;
+    const int m0 = rb * kRows;
+    const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
+    const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
+    const int c_lo = k_lo * kTileK;
+    const int c_hi = min(a.M, k_hi * kTileK);
+    const int nsub = (c_hi - c_lo + kSubCols - 1) / kSubCols;
+    float acc[kP][4];
+#pragma unroll
+    for (int q = 0; q < kP; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
+
+    // sub-chunk c -> stage c % stages (one commit group per call, empty past the end)
+    auto issue = [&](int c) {
+      if (c < nsub) {
+        uint8_t* xs = smem + (c % stages) * stage_bytes;
+        const int col = c_lo + c * kSubCols + piece * kPer16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = m0 + rg + 32 * i;
+          const bool ok = col < c_hi && row < a.B;
+          cp_async16(xs + (rg + 32 * i) * kPitch + piece * 16,
+                     ok ? static_cast<const void*>(x + static_cast<int64_t>(row) * a.ldx + col) : a.x, ok ? 16 : 0);
+        }
+        uint8_t* ls = xs + kRows * kPitch;
+        for (int idx = tid; idx < rp * 16; idx += kWork) {
+          const int j = idx >> 4, cc = c_lo + c * kSubCols + (idx & 15) * kPer16;
+          const bool ok = cc < c_hi;
+          cp_async16(ls + j * kPitch + (idx & 15) * 16,
+                     ok ? static_cast<const void*>(ld + static_cast<int64_t>(j) * a.M + cc) : a.ld, ok ? 16 : 0);
+        }
+        if (tid < kSubCols) {   // the sub-chunk's scale values (any 4-byte alignment)
+          const int cc = c_lo + c * kSubCols + tid;
+          const bool ok = cc < c_hi;
+          cp_async4(ls + rp * kPitch + 4 * tid, ok ? a.scale + cc : a.scale, ok ? 4 : 0);
+        }
+      }
+      cp_async_commit();
+    };
+    for (int c = 0; c < stages - 1; ++c) issue(c);
+    for (int c = 0; c < nsub; ++c) {
+      cp_async_wait_ring(stages);   // this thread's copies of sub-chunk c have landed
+      __syncthreads();              // everyone's have; stage (c - 1) % stages is free
+      issue(c + stages - 1);
+      const uint8_t* xs = smem + (c % stages) * stage_bytes;
+      const uint8_t* ls = xs + kRows * kPitch;
+      {
+        // max_k fl(colmax_k r_k): fl(a r) is monotone in a, so the column maximum
+        // of |x| is scaled once per column
+        uint32_t m = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          m = abs_max_word<TIn>(m, *reinterpret_cast<const uint32_t*>(xs + (rs + 8 * i) * kPitch + 4 * wi));
+        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        // every lane of the word's group holds its maximum; row slice 0 (and 1
+        // for the second bf16 lane) scales it
+        const float* sc = reinterpret_cast<const float*>(ls + rp * kPitch);
+        if constexpr (kEsz == 2) {
+          if (rs < 2) {
+            const int e = 2 * wi + rs;
+            if (c_lo + c * kSubCols + e < c_hi) {
+              const float v = __uint_as_float(rs == 0 ? m << 16 : m & 0xFFFF0000u);
+              run = fmaxf(run, __fmul_rn(v, __frcp_rn(sc[e])));
+            }
+          }
+        } else {
+          if (rs == 0 && c_lo + c * kSubCols + wi < c_hi)
+            run = fmaxf(run, __fmul_rn(__uint_as_float(m), __frcp_rn(sc[wi])));
+        }
+      }
+      if (rp) {
+#pragma unroll 2
+        for (int k = 0; k < kSubCols; k += kKStep) {
+          const int kb = k * kEsz;
+          uint32_t af[4];
+          ldmatrix_x4(af, smem_u32(xs + (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + kb +
+                                   ((lane >> 4) & 1) * 16));
+          if constexpr (kEsz == 4) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) af[e] = to_tf32(af[e]);
+          }
+#pragma unroll
+          for (int q = 0; q < kP; ++q) {
+            const int nt = nt0 + 2 * q;
+            if (nt < nnt) {
+              uint32_t bf[2];
+              ldmatrix_x2(bf, smem_u32(ls + (nt * 8 + (lane & 7)) * kPitch + kb + ((lane >> 3) & 1) * 16));
+              if constexpr (kEsz == 2) {
+                mma_bf16_16816(acc[q], af, bf);
+              } else {
+                bf[0] = to_tf32(bf[0]);
+                bf[1] = to_tf32(bf[1]);
+                mma_tf32_1688(acc[q], af, bf);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();   // the next unit's first copies reuse the stages
+    // the unit's partial down tile
+    if (rp) {
+      const int row = m0 + mt * 16 + gid;
+#pragma unroll
+      for (int q = 0; q < kP; ++q) {
+        const int nt = nt0 + 2 * q;
+        if (nt < nnt) {
+          float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp + nt * 8 + 2 * tig;
+          if (row < a.B) *reinterpret_cast<float2*>(dst) = make_float2(acc[q][0], acc[q][1]);
+          if (row + 8 < a.B)
+            *reinterpret_cast<float2*>(dst + 8 * static_cast<int64_t>(rp)) = make_float2(acc[q][2], acc[q][3]);
+        }
+      }
+    }
+  }
+  // per-CTA maximum -> ws_max[blockIdx.x]
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
+  if (lane == 0) red[warp] = run;
+  __syncthreads();
+  if (tid == 0) {
+    float mx = red[0];
+    for (int w = 1; w < kWorkWarps; ++w) mx = fmaxf(mx, red[w]);
+    a.ws_max[blockIdx.x] = mx;
+  }
+}
+
+// ------------------------------------------------------------ codes kernel
+template <typename TIn>
+__global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
+  constexpr int kTileK = kTileBytes / static_cast<int>(sizeof(TIn));
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float red[kWorkWarps];
+  float* rcp = reinterpret_cast<float*>(smem);   // the unit's reciprocals
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto unit_range = [&](int unit, int& m0, int& k_lo, int& n) {
     const int rb = unit % a.nrb, sp = unit / a.nrb;
     m0 = rb * kRows;
     k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
     n = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit) - k_lo;
   };
-
-  if (tid == kWork) {
-    for (int s = 0; s < kMaxHold; ++s) {
-      mbar_init(&xfull[s], 1);
-      mbar_init(&xempty[s], kWorkWarps + (a.has_ld ? 1 : 0));
-    }
-    mbar_init(&ld_free, 1);
-    mbar_init(&mma_done, 1);
-    mbar_init(&tmem_free, 4);
-    fence_mbar_init();
-    abort_sh = 0;
-    tma_prefetch_desc(&tm_x);
-  }
-  if (warp == kMmaWarp && mma_phase) {
-    tmem_alloc(&tmem_base_sh, tcols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = mma_phase ? tmem_base_sh : 0u;
-  float run = 0.0f;
-  bool ok = true;
-
-  // ================================================================ phase 1
-  if (a.phase == 1) {
-  // x steps flow through the buffers as one ring over all of this CTA's units:
-  // step G + i uses buffer (G + i) % xbuf in its use (G + i) / xbuf (counters
-  // in registers: an indexed array would live in local memory)
-  if (warp == kTmaWarp) {
-    if (lane == 0) {
-      uint32_t G = 0;   // x steps of the previous units
-      bool pok = true;
-      for (int unit = blockIdx.x; unit < a.nunits && pok; unit += gridDim.x) {
-        int m0, k_lo, n;
-        unit_range(unit, m0, k_lo, n);
-        for (int i = 0; i < n && pok; ++i) {
-          const uint32_t gs = G + i;
-          const uint32_t b = gs % a.xbuf, use = gs / a.xbuf;
-          if (use > 0)  // the previous tile in this buffer is fully read
-            pok = mbar_wait(&xempty[b], (use - 1) & 1, status, &abort_sh);
-          if (!pok) break;
-          mbar_arrive_expect_tx(&xfull[b], kTileBytes);
-          tma_load_2d(xbuf + static_cast<size_t>(b) * kTileBytes, &tm_x, &xfull[b], (k_lo + i) * kTileK, m0);
-        }
-        G += n;
-      }
-      if (!pok) {
-        abort_sh = 1;
-        // let loads already issued land before the block moves on (the loads
-        // of the last xbuf steps of the ring, at most)
-        for (uint32_t gs = G > static_cast<uint32_t>(a.xbuf) ? G - a.xbuf : 0u; gs < G; ++gs)
-          mbar_wait(&xfull[gs % a.xbuf], (gs / a.xbuf) & 1, status, nullptr, 1000000ull);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    if (mma_phase) {
-      uint32_t G = 0;        // x steps of the previous units
-      uint32_t nbatch = 0;   // ld batches whose MMAs were committed to ld_free
-      bool pok = true;
-      // ld tiles of K tiles k_lo + j0 .. + cnt - 1 into slots 0 .. cnt - 1, one
-      // copy group per lane; ld is [rank_pad, M] row-major, columns past M are
-      // filled with zeros. The slots are free once the previous batch's MMAs
-      // are done.
-      auto copy_batch = [&](int k_lo, int j0, int cnt) {
-        if (nbatch > 0) pok = mbar_wait_warp(&ld_free, (nbatch - 1) & 1, status, &abort_sh) && pok;
-        const TIn* ld = static_cast<const TIn*>(a.ld);
-        for (int t = 0; t < cnt; ++t) {
-          uint8_t* dst = ldbuf + static_cast<size_t>(t) * ld_bytes;
-          for (int c = lane; c < a.rank_pad * 8; c += 32) {
-            const int r = c >> 3, cc = c & 7;
-            const int col = (k_lo + j0 + t) * kTileK + cc * kPerChunk;
-            const bool in = col < a.M;
-            cp_async16(smem_u32(dst + r * 128 + ((cc ^ (r & 7)) << 4)),
-                       in ? static_cast<const void*>(ld + static_cast<int64_t>(r) * a.M + col) : a.ld,
-                       in ? 16u : 0u);
-          }
-        }
-        cp_async_commit();
-      };
-      const uint32_t idesc = sizeof(TIn) == 2 ? idesc_bf16(128, a.rank_pad) : idesc_tf32(128, a.rank_pad);
-      if (lane == 0) {
-        // throwaway MMA (its result is overwritten by the first real one)
-        const uint64_t ad = smem_desc_sw128(smem_u32(xbuf)), bd = smem_desc_sw128(smem_u32(ldbuf));
-        if (sizeof(TIn) == 2)
-          mma_f16(tmem, ad, bd, idesc, 0u);
-        else
-          mma_tf32(tmem, ad, bd, idesc, 0u);
-      }
-      __syncwarp();
-      uint32_t ucount = 0;
-      for (int unit = blockIdx.x; unit < a.nunits && pok; unit += gridDim.x, ++ucount) {
-        int m0, k_lo, n;
-        unit_range(unit, m0, k_lo, n);
-        for (int j0 = 0; j0 < n && pok; j0 += kLdRing) {
-          const int cnt = min(kLdRing, n - j0);
-          copy_batch(k_lo, j0, cnt);
-          if (lane == 0 && ucount > 0 && j0 == 0)  // the work warps have read the previous unit's accumulator
-            pok = pok && mbar_wait(&tmem_free, (ucount - 1) & 1, status, &abort_sh);
-          cp_async_wait(0);  // this lane's copies have landed
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            for (int t = 0; t < cnt && pok; ++t) {
-              const int i = j0 + t;
-              const uint32_t b = (G + i) % a.xbuf;
-              pok = mbar_wait(&xfull[b], ((G + i) / a.xbuf) & 1, status, &abort_sh);
-              if (!pok) break;
-              tc_fence_after();
-              const uint32_t a0 = smem_u32(xbuf + static_cast<size_t>(b) * kTileBytes);
-              const uint32_t b0 = smem_u32(ldbuf + static_cast<size_t>(t) * ld_bytes);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = smem_desc_sw128(a0 + 32 * kk);
-                const uint64_t bd = smem_desc_sw128(b0 + 32 * kk);
-                if (sizeof(TIn) == 2)
-                  mma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-                else
-                  mma_tf32(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-              }
-              mma_commit(&xempty[b]);
-            }
-            if (pok) mma_commit(&ld_free);
-          }
-          ++nbatch;
-          pok = __shfl_sync(0xffffffffu, pok ? 1 : 0, 0) != 0;
-        }
-        if (lane == 0 && pok) mma_commit(&mma_done);
-        G += n;
-      }
-      cp_async_wait(0);
-      if (lane == 0 && !pok) abort_sh = 1;
-    }
-  } else {
-    uint32_t G = 0;   // x steps of the previous units (the same ring as the producer's)
-    uint32_t ucount = 0;
-    for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x, ++ucount) {
-      int m0, k_lo, n;
-      unit_range(unit, m0, k_lo, n);
-      work_sync();  // the previous unit's reciprocals are no longer read
-      for (int j = tid; j < n * kTileK; j += kWork) {
-        const int col = k_lo * kTileK + j;
-        rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
-      }
-      work_sync();
-      for (int i = 0; i < n; ++i) {
-        const uint32_t b = (G + i) % a.xbuf;
-        ok = mbar_wait_warp(&xfull[b], ((G + i) / a.xbuf) & 1, status, &abort_sh) && ok;
-        if (ok) run = tile_absmax<TIn>(xbuf + static_cast<size_t>(b) * kTileBytes, rcp + i * kTileK, run);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xempty[b]);
-      }
-      if (mma_phase && warp < 4) {
-        // drain the unit's accumulator into its partial before the next
-        // unit's MMAs; TMEM lane = row, warps 0-3 cover the 128 lanes
-        const bool fin = mbar_wait_warp(&mma_done, ucount & 1, status, &abort_sh) && ok;
-        tc_fence_after();
-        const int row = m0 + warp * 32 + lane;
-        const int sp = unit / a.nrb;
-        float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * a.rank_pad;
-        for (int c0 = 0; c0 < a.rank_pad; c0 += 32) {
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-          tmem_ld_wait_regs(v);
-          if (fin && row < a.B) {
-            const int cnt = min(32, a.rank_pad - c0);
-            for (int j = 0; j < cnt; j += 4)
-              *reinterpret_cast<float4*>(dst + c0 + j) =
-                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                              __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tmem_free);
-        ok = ok && fin;
-      }
-      G += n;
-    }
-    // per-CTA maximum -> ws_max[blockIdx.x]
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-    if (lane == 0) red[warp] = run;
-    work_sync();
-    if (tid == 0) {
-      float m = red[0];
-      for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
-      a.ws_max[blockIdx.x] = ok ? m : 0.0f;
-    }
-  }
-  }   // phase 1
-
-  // ================================================================ phase 2
-  if (a.phase == 2 && !producer) {
+  {
     float m = 0.0f;
     for (int i = tid; i < a.nparts; i += kWork) m = fmaxf(m, __ldcg(a.ws_max + i));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    work_sync();
+    __syncthreads();
     if (lane == 0) red[warp] = m;
-    work_sync();
+    __syncthreads();
     m = red[0];
     for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
     const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
@@ -419,80 +374,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit_range(unit, m0, k_lo, n);
       const int sp = unit / a.nrb;
       const int64_t col0 = static_cast<int64_t>(k_lo) * kTileK;
-      work_sync();
+      __syncthreads();
       for (int j = tid; j < n * kTileK; j += kWork) {
         const int col = k_lo * kTileK + j;
         rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
       }
-      work_sync();
+      __syncthreads();
       const int rows = min(kRows, a.B - m0);
       const int ncols = min(n * kTileK, a.M - k_lo * kTileK);   // a multiple of 32
       if (!nv) {
         // a warp writes 256 consecutive codes of a row (8 per lane, one 256-byte
-        // store), two rows (r, r + 16) at a time
+        // store) for kR rows, whose loads are all issued first
+        constexpr int kR = sizeof(TIn) == 2 ? 8 : 4;
         for (int c256 = 0; c256 < ncols; c256 += 256) {
           const int cl = c256 + 8 * lane;
-          const bool live = cl < ncols;
+          if (cl >= ncols) continue;
           float ck[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ck[j] = live ? __fmul_rn(rcp[cl + j], u) : 0.0f;
-          for (int r = warp; r < rows; r += 2 * kWorkWarps) {
-            const int r2 = r + kWorkWarps;
-            const bool two = r2 < rows;
-            uint4 ua[2], ub[2];
-            if (live) {
-              load8<TIn>(a.x, a.ldx, m0 + r, col0, cl, ua);
-              if (two) load8<TIn>(a.x, a.ldx, m0 + r2, col0, cl, ub);
-            }
-            if (live) {
-              float v[8];
-              unpack8<TIn>(ua, v);
-              *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r) * a.M +
-                                        col0 + cl) = int_codes8(v, ck);
-              if (two) {
-                unpack8<TIn>(ub, v);
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) +
-                                          static_cast<int64_t>(m0 + r2) * a.M + col0 + cl) = int_codes8(v, ck);
+          for (int j = 0; j < 8; ++j) ck[j] = __fmul_rn(rcp[cl + j], u);
+          for (int r0 = warp * kR; r0 < rows; r0 += kWorkWarps * kR) {
+            uint4 uv[kR][2];
+#pragma unroll
+            for (int i = 0; i < kR; ++i)
+              if (r0 + i < rows) load8<TIn>(a.x, a.ldx, m0 + r0 + i, col0, cl, uv[i]);
+#pragma unroll
+            for (int i = 0; i < kR; ++i) {
+              if (r0 + i < rows) {
+                float v[8];
+                unpack8<TIn>(uv[i], v);
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r0 + i) * a.M +
+                                          col0 + cl) = int_codes8(v, ck);
               }
             }
           }
         }
       } else {
-        // half a warp = 256 consecutive elements of one row (one 16-element block per lane)
+        // half a warp = 256 consecutive elements of one row (one 16-element block
+        // per lane), kR rows per half warp with all loads issued first
+        constexpr int kR = sizeof(TIn) == 2 ? 4 : 2;
+        constexpr int kHalves = 2 * kWorkWarps;
+        const int hw = 2 * warp + (lane >> 4);
         const int nch = (ncols + 255) / 256;
-        const int items = nch * rows;
-        for (int base = 2 * warp; base < items; base += 2 * kWorkWarps) {
-          const int it = base + (lane >> 4);
-          if (it >= items) continue;
-          const int cc = it / rows, r = it - cc * rows;
+        for (int cc = 0; cc < nch; ++cc) {
           const int cl = cc * 256 + 16 * (lane & 15);
           if (cl >= ncols) continue;
-          float xs[16];
+          for (int r0 = hw; r0 < rows; r0 += kR * kHalves) {
+            uint4 uv[kR][2][2];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint4 uu[2];
-            float v8[8];
-            load8<TIn>(a.x, a.ldx, m0 + r, col0, cl + 8 * h, uu);
-            unpack8<TIn>(uu, v8);
+            for (int i = 0; i < kR; ++i)
+              if (r0 + kHalves * i < rows) {
+                load8<TIn>(a.x, a.ldx, m0 + r0 + kHalves * i, col0, cl, uv[i][0]);
+                load8<TIn>(a.x, a.ldx, m0 + r0 + kHalves * i, col0, cl + 8, uv[i][1]);
+              }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) xs[8 * h + j] = v8[j];
+            for (int i = 0; i < kR; ++i) {
+              const int r = r0 + kHalves * i;
+              if (r >= rows) continue;
+              float xs[16];
+              unpack8<TIn>(uv[i][0], *reinterpret_cast<float(*)[8]>(xs));
+              unpack8<TIn>(uv[i][1], *reinterpret_cast<float(*)[8]>(xs + 8));
+              float amax = 0.0f;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                xs[j] = __fmul_rn(xs[j], rcp[cl + j]);
+                amax = fmaxf(amax, fabsf(xs[j]));
+              }
+              const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+              const float d = ue4m3_to_f32(sfb);
+              const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
+              const int64_t row = m0 + r;
+              const int64_t col = col0 + cl;
+              *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
+                  make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
+              a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+            }
           }
-          float amax = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            xs[j] = __fmul_rn(xs[j], rcp[cl + j]);
-            amax = fmaxf(amax, fabsf(xs[j]));
-          }
-          const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
-          const float d = ue4m3_to_f32(sfb);
-          const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
-          const int64_t row = m0 + r;
-          const int64_t col = col0 + cl;
-          *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
-              make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
-          a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
         }
       }
       // down = the K-split partials summed in split order, as bf16 hi | lo
@@ -535,44 +493,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-
-  __syncthreads();
-  if (mma_phase && warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, tcols);
-  }
 }
 
-size_t smem_for(const ActPlan& p, int xbuf) {
-  const int ld_bytes = p.rank_pad * 128;
-  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
-  return static_cast<size_t>(xbuf) * kTileBytes + (p.rank_pad > 0 ? kLdRing * ld_bytes : 0) +
-         static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
+// x rows, ld rows and the scale values (kSub bytes of x hold at most 128 columns)
+size_t stage_bytes(int rank_pad) { return static_cast<size_t>(kRows + rank_pad) * kPitch + kScaleBytes; }
+
+template <typename TIn>
+cudaError_t launch_stats(const ActArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  cudaError_t err;
+  if (a.rank_pad <= 64) {
+    err = cudaFuncSetAttribute(act_stats_kernel<TIn, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    act_stats_kernel<TIn, 4><<<grid, kWork, smem, stream>>>(a);
+  } else {
+    err = cudaFuncSetAttribute(act_stats_kernel<TIn, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    act_stats_kernel<TIn, 16><<<grid, kWork, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
 }
 
-// Resident CTAs per SM for a given dynamic shared memory size (at most two:
-// each may hold TMEM for its down accumulator).
-int resident_per_sm(size_t smem, bool bf16) {
-  int n = 0;
-  cudaError_t e;
-  // the occupancy query honours the kernel's opt-in shared memory limit
-  int dev = 0, optin = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess &&
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
-      optin > 4096) {
-    const int lim = optin - 2048;
-    if (bf16)
-      cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    else
-      cudaFuncSetAttribute(act_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-  }
-  if (bf16)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_fused_kernel<__nv_bfloat16>, kThreads,
-                                                      smem);
-  else
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_fused_kernel<float>, kThreads, smem);
-  if (e != cudaSuccess || n <= 0) n = smem > 110 * 1024 ? 1 : 2;
-  return std::max(1, std::min(n, 2));
+template <typename TIn>
+cudaError_t launch_codes(const ActArgs& a, size_t smem, cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(act_codes_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  act_codes_kernel<TIn><<<a.nunits, kWork, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -583,13 +532,15 @@ void finish_act_plan(ActPlan& p) {
     return;
   }
   p.nunits = p.nrb * p.ksplit;
+  // stages: as many as fit, no more than the longest unit's sub-chunks + 1
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
-  // all of a unit's x tiles in flight at once when they fit (a deep TMA queue),
-  // else a ring of kXRing tiles
-  p.xbuf = kXRing;
-  if (steps_max <= kMaxHold && smem_for(p, steps_max) <= static_cast<size_t>(kSmemBudget)) p.xbuf = steps_max;
-  p.smem = smem_for(p, p.xbuf);
-  p.grid = std::min(p.nunits, num_sms() * resident_per_sm(p.smem, p.bf16));
+  const int sub_max = (steps_max * kTileBytes + kSub - 1) / kSub;
+  const size_t sb = stage_bytes(p.rank_pad);
+  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, kStatsSmemBudget / sb));
+  p.stages = std::max(2, std::min(p.stages, sub_max + 1));
+  p.smem = sb * p.stages;
+  // one CTA per SM (512 threads, most of the shared memory)
+  p.grid = std::min(p.nunits, num_sms());
   p.nparts = p.grid;
 }
 
@@ -614,12 +565,9 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool al
   p.tile_k = p.bf16 ? 64 : 32;
   p.nrb = static_cast<int>(ceil_div(B, kRows));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
-  // one unit per SM; split K further when that lets each unit's tiles stay in
-  // shared memory (then two units share an SM)
+  // at most one unit per SM: split K until the units cover the SMs
   const int sms = num_sms();
-  int ks = std::max(1, std::min(p.nsteps, sms / std::max(p.nrb, 1)));
-  while (ks < p.nsteps && ceil_div(p.nsteps, ks) > kMaxHold && p.nrb * (ks + 1) <= 2 * sms) ++ks;
-  p.ksplit = ks;
+  p.ksplit = std::max(1, std::min(p.nsteps, sms / std::max(p.nrb, 1)));
   finish_act_plan(p);
   return p;
 }
@@ -646,21 +594,18 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
     return launch_act_small(p, x, xdt, ldx, scale, fmt, act_global_scale, w_global_scale, ld, codes, sf,
                             act_scale, down, scratch, stream, bad_args);
   const bool has_ld = ld != nullptr && p.rank_pad > 0 && down != nullptr;
+  const int esz = xdt == SVDQ_BF16 ? 2 : 4;
+  // 16-byte copies of x and ld rows
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (ldx * esz) % 16 != 0 || (p.M * esz) % 16 != 0 ||
+      (has_ld && (reinterpret_cast<uintptr_t>(ld) & 15) != 0)) {
+    *bad_args = true;
+    return cudaSuccess;
+  }
   Carver cv(scratch, ~size_t(0));
   float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));
   float* ws_down =
       has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4))
              : nullptr;
-  const int esz = xdt == SVDQ_BF16 ? 2 : 4;
-  const CUtensorMapDataType cdt =
-      xdt == SVDQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  CUtensorMap tm_x;
-  if (!make_tmap_2d(&tm_x, x, cdt, esz, p.M, p.B, ldx, p.tile_k, kRows, true) ||
-      (has_ld && (reinterpret_cast<uintptr_t>(ld) & 15) != 0)) {
-    *bad_args = true;
-    return cudaSuccess;
-  }
-  cudaError_t err;
   ActArgs a{};
   a.B = static_cast<int>(p.B);
   a.M = static_cast<int>(p.M);
@@ -671,7 +616,6 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.nunits = p.nunits;
   a.rank_pad = has_ld ? p.rank_pad : 0;
   a.has_ld = has_ld ? 1 : 0;
-  a.xbuf = p.xbuf;
   a.nparts = p.grid;
   a.fmt_kind = fmt.kind;
   a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
@@ -686,36 +630,20 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.sf = static_cast<uint8_t*>(sf);
   a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
   a.act_scale = act_scale;
-  a.status = device_status_word();
-  // without the down factor the launch needs no ld ring (plan keeps its grid)
+  // without the down factor the stages hold x alone (fewer bytes per stage)
   ActPlan q = p;
-  if (!has_ld) q.rank_pad = 0;
-  const size_t smem1 = smem_for(q, p.xbuf);
-  // phase 2 keeps only the unit's reciprocals in shared memory
+  if (!has_ld) {
+    q.rank_pad = 0;
+    finish_act_plan(q);
+  }
+  a.stages = q.stages;
+  // the codes kernel keeps only the unit's reciprocals in shared memory
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   const size_t smem2 = static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
-  ActArgs a2 = a;
-  a.phase = 1;
-  a2.phase = 2;
-  a2.xbuf = 0;
-  if (xdt == SVDQ_BF16) {
-    err = cudaFuncSetAttribute(act_fused_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(std::max(smem1, smem2)));
-    if (err != cudaSuccess) return err;
-    act_fused_kernel<__nv_bfloat16><<<p.grid, kThreads, smem1, stream>>>(tm_x, a);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    act_fused_kernel<__nv_bfloat16><<<p.nunits, kThreads, smem2, stream>>>(tm_x, a2);
-  } else {
-    err = cudaFuncSetAttribute(act_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(std::max(smem1, smem2)));
-    if (err != cudaSuccess) return err;
-    act_fused_kernel<float><<<p.grid, kThreads, smem1, stream>>>(tm_x, a);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    act_fused_kernel<float><<<p.nunits, kThreads, smem2, stream>>>(tm_x, a2);
-  }
-  return cudaGetLastError();
+  cudaError_t err = xdt == SVDQ_BF16 ? launch_stats<__nv_bfloat16>(a, p.grid, q.smem, stream)
+                                     : launch_stats<float>(a, p.grid, q.smem, stream);
+  if (err != cudaSuccess) return err;
+  return xdt == SVDQ_BF16 ? launch_codes<__nv_bfloat16>(a, smem2, stream) : launch_codes<float>(a, smem2, stream);
 }
 
 }  // namespace svdq

@@ -425,7 +425,7 @@ void finish_act_plan_small(ActPlan& p) {
   p.ksplit = p.grid;
   p.nunits = p.grid;
   p.nparts = p.grid;
-  p.xbuf = 0;
+  p.stages = 0;
   p.smem = small_smem(p, p.rank_pad > 0);
 }
 

@@ -1,6 +1,6 @@
-// gemm_common.cuh - pieces shared by the residual GEMM kernels (one CTA per
-// tile in gemm.cu, a CTA pair per tile in gemm_pair.cu): the argument block
-// and the epilogue that turns one 128-row slab of TMEM accumulators into Y.
+// gemm_common.cuh - pieces shared by the residual GEMM kernels (gemm_pair.cu,
+// gemm_skinny.cu): the argument block and the epilogue that turns 128-row slabs
+// of TMEM accumulators into Y.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -135,15 +135,6 @@ __device__ __forceinline__ void epilogue_chunk_direct(const GemmArgs& args, uint
     for (int j = 0; j < 16; ++j) p[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
     store_row32<kOutBF16>(args, row, n, p);
   }
-}
-
-// One warp's 32 rows of a 128 x 256 accumulator slab -> Y.
-template <int kKind, int kOut>
-__device__ __forceinline__ void epilogue_slab(const GemmArgs& args, uint32_t lane_addr, int row,
-                                              int n0, float alpha, bool sep_lr) {
-  for (int c0 = 0; c0 < 256; c0 += 32)
-    epilogue_chunk_direct<kKind, kOut>(args, lane_addr, row, n0 + c0, static_cast<uint32_t>(c0), alpha,
-                                       sep_lr);
 }
 
 // Two-pass epilogue (overlaps the global stores with the next tile's MMAs).

@@ -52,8 +52,8 @@ struct ActPlan {
   int nsteps;      // K tiles
   int ksplit;      // K ranges per row block
   int nunits;      // nrb * ksplit work units
-  int xbuf;        // x tile buffers per CTA
-  int grid;        // CTAs of the cooperative launch (all resident)
+  int stages;      // large-batch stats kernel: sub-chunk stages in shared memory
+  int grid;        // CTAs of the stats (large batch) or first (short batch) kernel
   int nparts;      // partial maxima written (one per CTA)
   size_t smem;     // dynamic shared memory per CTA
   int small;       // 1: the short-batch kernel (act_small.cu): one column chunk per CTA
