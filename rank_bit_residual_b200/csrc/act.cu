@@ -47,9 +47,19 @@ constexpr int kWork = 32 * kWorkWarps;      // threads of both kernels
 constexpr int kRows = 128;                  // rows per unit
 constexpr int kTileBytes = 128;             // bytes of a row per column tile (64 bf16 / 32 fp32)
 constexpr int kSub = 256;                   // bytes of a row per stats sub-chunk (two tiles)
-constexpr int kPitch = kSub + 16;           // padded shared row: 8 ldmatrix rows hit distinct banks
 constexpr int kMaxStages = 6;
 constexpr int kScaleBytes = 512;            // a stage's scale values (at most 128 columns)
+
+// Bytes of one stats-kernel stage: x and ld as two 128-byte K blocks each, then
+// the scale values; a multiple of 1024 so every block keeps the swizzle atom.
+__host__ __device__ constexpr int stats_stage_bytes(int rank_pad) {
+  return (2 * kRows * kTileBytes + 2 * rank_pad * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
+}
+
+// TMEM columns for a rank_pad-column fp32 accumulator (a power of two >= 32).
+__host__ __device__ constexpr uint32_t tmem_cols_for(int rank_pad) {
+  return rank_pad <= 32 ? 32u : rank_pad <= 64 ? 64u : rank_pad <= 128 ? 128u : 256u;
+}
 constexpr size_t kStatsSmemBudget = 220 * 1024;
 
 struct ActArgs {
@@ -69,6 +79,7 @@ struct ActArgs {
   uint8_t* sf;
   __nv_bfloat16* down;
   float* act_scale;
+  unsigned* status;   // bounded waits record a timeout here
 };
 
 
@@ -92,38 +103,6 @@ __device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
     unpack16<TIn>(u[0], v);
     unpack16<TIn>(u[1], v + 4);
   }
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t to_tf32(uint32_t f) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__uint_as_float(f)));
-  return r;
 }
 
 // Copy 16 bytes global -> shared, bypassing L1; src_bytes = 0 fills zeros and
@@ -173,37 +152,67 @@ __device__ __forceinline__ uint32_t max_word(uint32_t m, uint32_t w) {
 // ------------------------------------------------------------ stats kernel
 // A unit is streamed in sub-chunks of kSub bytes per row through a ring of
 // `stages` shared-memory stages filled by cp.async (stages - 1 sub-chunks in
-// flight while one is consumed); a stage holds the x rows, the ld rows and the
-// sub-chunk's scale values. Copies: thread t moves the 16-byte piece t % 16 of
-// rows t / 16 + 32 i (i < 4), so a warp moves two whole 256-byte row segments
-// per instruction. Column maxima: warp w scans 32-bit words 4 w .. 4 w + 3 of
-// rows l / 4 + 8 i (lane l, i < 16; conflict-free with the padded pitch), the
-// eight row slices meet by shuffles, and each column's fl(colmax r_k) is taken
-// once. Down projection: warp w owns m-tile w % 8 of the 128 x rank_pad tile
-// and n-tiles w / 8 + 2 q (q < kP), so one A fragment serves all of its MMAs;
-// the fp32 accumulators live across the unit's sub-chunks.
-template <typename TIn, int kP>
+// flight while one is consumed). A stage holds the x rows and the ld rows as
+// two 128-byte-wide K blocks each, in the 128-byte-swizzled K-major layout the
+// tensor core reads (16-byte chunk c of row r at chunk c ^ (r & 7) of the
+// row's 128 bytes), then the sub-chunk's scale values.
+//   copies        thread t moves the 16-byte piece t % 16 of rows t / 16 + 32 i
+//                 (i < 4): a warp moves two whole 256-byte row segments;
+//   column maxima warp w scans 32-bit words 4 w .. 4 w + 3 of rows l / 4 + 8 i
+//                 (lane l, i < 16; conflict-free under the swizzle), the eight
+//                 row slices meet by shuffles, and each column's fl(colmax r_k)
+//                 is taken once;
+//   down tile     one thread issues the sub-chunk's tcgen05 MMAs (M = 128 rows,
+//                 N = rank_pad, kind::f16 for bf16 x, kind::tf32 for fp32 x)
+//                 into a TMEM accumulator that lives across the unit; their
+//                 commit frees the stage for the copies of a later sub-chunk;
+//                 at the unit's end warps 0-3 drain it (TMEM lane = row).
+template <typename TIn>
 __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
   constexpr int kSubCols = kSub / kEsz;             // 128 bf16 or 64 fp32 columns
   constexpr int kPer16 = 16 / kEsz;                 // elements per 16-byte piece
-  constexpr int kKStep = kEsz == 2 ? 16 : 8;        // K of one warp MMA
   constexpr int kTileK = kTileBytes / kEsz;         // columns per K tile
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ float red[kWorkWarps];
+  __shared__ __align__(8) uint64_t mma_bar[kMaxStages];
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
 
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rp = a.rank_pad;                        // 0 without the down factor
   const int stages = a.stages;
-  const int stage_bytes = (kRows + rp) * kPitch + kScaleBytes;
+  const int stage_bytes = stats_stage_bytes(rp);
+  const int ld_off = 2 * kRows * kTileBytes;        // the ld blocks follow the x blocks
+  const int sc_off = ld_off + 2 * rp * kTileBytes;  // then the scale values
   const int piece = tid & 15, rg = tid >> 4;
   const int wi = warp * 4 + (lane & 3), rs = lane >> 2;   // column-max word and row slice
-  const int gid = lane >> 2, tig = lane & 3;
-  const int mt = warp & 7, nt0 = warp >> 3, nnt = rp / 8;
   const TIn* x = static_cast<const TIn*>(a.x);
   const TIn* ld = static_cast<const TIn*>(a.ld);
+  const uint32_t idesc = kEsz == 2 ? idesc_bf16(kRows, rp > 0 ? rp : 16) : idesc_tf32(kRows, rp > 0 ? rp : 16);
   float run = 0.0f;
 
+  if (tid == 0) {
+    for (int s = 0; s < kMaxStages; ++s) mbar_init(&mma_bar[s], 1);
+    fence_mbar_init();
+    abort_sh = 0;
+  }
+  if (rp > 0 && warp == 0) {
+    tmem_alloc(&tmem_sh, tmem_cols_for(rp));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+
+  // 16-byte chunk c (0..15) of row r of a two-block region with `rows` rows
+  auto swz = [](int r, int c, int rows) -> int {
+    return (c >> 3) * rows * kTileBytes + r * kTileBytes + (((c & 7) ^ (r & 7)) << 4);
+  };
+  uint32_t g = 0;   // sub-chunks begun so far: stage g % stages, barrier phase (g / stages) & 1
   for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
     const int rb = unit % a.nrb, sp = unit / a.nrb;
     const int m0 = rb * kRows;
@@ -212,57 +221,72 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
     const int c_lo = k_lo * kTileK;
     const int c_hi = min(a.M, k_hi * kTileK);
     const int nsub = (c_hi - c_lo + kSubCols - 1) / kSubCols;
-    float acc[kP][4];
-#pragma unroll
-    for (int q = 0; q < kP; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
 
-    // sub-chunk c -> stage c % stages (one commit group per call, empty past the end)
+    // sub-chunk c -> its stage (one commit group per call, empty past the end)
     auto issue = [&](int c) {
       if (c < nsub) {
-        uint8_t* xs = smem + (c % stages) * stage_bytes;
+        uint8_t* st = smem + ((g + c) % stages) * stage_bytes;
         const int col = c_lo + c * kSubCols + piece * kPer16;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int row = m0 + rg + 32 * i;
-          const bool ok = col < c_hi && row < a.B;
-          cp_async16(xs + (rg + 32 * i) * kPitch + piece * 16,
-                     ok ? static_cast<const void*>(x + static_cast<int64_t>(row) * a.ldx + col) : a.x, ok ? 16 : 0);
+          const int r = rg + 32 * i, row = m0 + r;
+          const bool in = col < c_hi && row < a.B;
+          cp_async16(st + swz(r, piece, kRows),
+                     in ? static_cast<const void*>(x + static_cast<int64_t>(row) * a.ldx + col) : a.x, in ? 16 : 0);
         }
-        uint8_t* ls = xs + kRows * kPitch;
         for (int idx = tid; idx < rp * 16; idx += kWork) {
-          const int j = idx >> 4, cc = c_lo + c * kSubCols + (idx & 15) * kPer16;
-          const bool ok = cc < c_hi;
-          cp_async16(ls + j * kPitch + (idx & 15) * 16,
-                     ok ? static_cast<const void*>(ld + static_cast<int64_t>(j) * a.M + cc) : a.ld, ok ? 16 : 0);
+          const int j = idx >> 4, cc = idx & 15, colj = c_lo + c * kSubCols + cc * kPer16;
+          const bool in = colj < c_hi;
+          cp_async16(st + ld_off + swz(j, cc, rp),
+                     in ? static_cast<const void*>(ld + static_cast<int64_t>(j) * a.M + colj) : a.ld, in ? 16 : 0);
         }
         if (tid < kSubCols) {   // the sub-chunk's scale values (any 4-byte alignment)
           const int cc = c_lo + c * kSubCols + tid;
-          const bool ok = cc < c_hi;
-          cp_async4(ls + rp * kPitch + 4 * tid, ok ? a.scale + cc : a.scale, ok ? 4 : 0);
+          const bool in = cc < c_hi;
+          cp_async4(st + sc_off + 4 * tid, in ? a.scale + cc : a.scale, in ? 4 : 0);
         }
       }
       cp_async_commit();
     };
     for (int c = 0; c < stages - 1; ++c) issue(c);
     for (int c = 0; c < nsub; ++c) {
+      const uint32_t gc = g + c;
+      const uint8_t* st = smem + (gc % stages) * stage_bytes;
       cp_async_wait_ring(stages);   // this thread's copies of sub-chunk c have landed
-      __syncthreads();              // everyone's have; stage (c - 1) % stages is free
+      fence_proxy_async_smem();     // ... and are visible to the tensor core
+      __syncthreads();              // everyone's have; every thread is done with sub-chunk c - 1
+      if (abort_sh) break;          // a bounded wait gave up (uniform after the barrier)
+      if (rp > 0 && tid == 0) {
+        tc_fence_after();
+        const uint32_t xa = smem_u32(st), la = xa + ld_off;
+#pragma unroll
+        for (int kk = 0; kk < kSub / 32; ++kk) {   // 32 bytes of K per MMA
+          const uint32_t off = (kk >> 2) * kRows * kTileBytes + (kk & 3) * 32;
+          const uint32_t offl = (kk >> 2) * rp * kTileBytes + (kk & 3) * 32;
+          if constexpr (kEsz == 2)
+            mma_f16(tmem, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_tf32(tmem, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&mma_bar[gc % stages]);
+      }
+      // refill the stage of sub-chunk c - 1 once its MMAs are done (each warp
+      // waits for itself, then copies its share)
+      if (rp > 0 && c > 0) mbar_wait_warp(&mma_bar[(gc - 1) % stages], ((gc - 1) / stages) & 1, a.status, &abort_sh);
       issue(c + stages - 1);
-      const uint8_t* xs = smem + (c % stages) * stage_bytes;
-      const uint8_t* ls = xs + kRows * kPitch;
       {
         // max_k fl(colmax_k r_k): fl(a r) is monotone in a, so the column maximum
         // of |x| is scaled once per column
         uint32_t m = 0u;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          m = abs_max_word<TIn>(m, *reinterpret_cast<const uint32_t*>(xs + (rs + 8 * i) * kPitch + 4 * wi));
+          m = abs_max_word<TIn>(m, *reinterpret_cast<const uint32_t*>(st + swz(rs + 8 * i, wi >> 2, kRows) + 4 * (wi & 3)));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 4));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 8));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 16));
         // every lane of the word's group holds its maximum; row slice 0 (and 1
         // for the second bf16 lane) scales it
-        const float* sc = reinterpret_cast<const float*>(ls + rp * kPitch);
+        const float* sc = reinterpret_cast<const float*>(st + sc_off);
         if constexpr (kEsz == 2) {
           if (rs < 2) {
             const int e = 2 * wi + rs;
@@ -276,51 +300,35 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
             run = fmaxf(run, __fmul_rn(__uint_as_float(m), __frcp_rn(sc[wi])));
         }
       }
-      if (rp) {
-#pragma unroll 2
-        for (int k = 0; k < kSubCols; k += kKStep) {
-          const int kb = k * kEsz;
-          uint32_t af[4];
-          ldmatrix_x4(af, smem_u32(xs + (mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + kb +
-                                   ((lane >> 4) & 1) * 16));
-          if constexpr (kEsz == 4) {
+    }
+    // the unit's partial down tile: wait for its last MMAs, then TMEM -> ws_down
+    if (rp > 0 && !abort_sh) {
+      if (warp < 4) {
+        const uint32_t gl = g + nsub - 1;
+        const bool ok = mbar_wait_warp(&mma_bar[gl % stages], (gl / stages) & 1, a.status, &abort_sh);
+        tc_fence_after();
+        const int row = m0 + warp * 32 + lane;
+        float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp;
+        for (int c0 = 0; c0 < rp; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+          tmem_ld_wait_regs(v);
+          if (ok && row < a.B) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) af[e] = to_tf32(af[e]);
-          }
-#pragma unroll
-          for (int q = 0; q < kP; ++q) {
-            const int nt = nt0 + 2 * q;
-            if (nt < nnt) {
-              uint32_t bf[2];
-              ldmatrix_x2(bf, smem_u32(ls + (nt * 8 + (lane & 7)) * kPitch + kb + ((lane >> 3) & 1) * 16));
-              if constexpr (kEsz == 2) {
-                mma_bf16_16816(acc[q], af, bf);
-              } else {
-                bf[0] = to_tf32(bf[0]);
-                bf[1] = to_tf32(bf[1]);
-                mma_tf32_1688(acc[q], af, bf);
-              }
-            }
+            for (int j = 0; j < 16; j += 4)
+              *reinterpret_cast<float4*>(dst + c0 + j) =
+                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                              __uint_as_float(v[j + 3]));
           }
         }
+        tc_fence_before();
       }
     }
-    __syncthreads();   // the next unit's first copies reuse the stages
-    // the unit's partial down tile
-    if (rp) {
-      const int row = m0 + mt * 16 + gid;
-#pragma unroll
-      for (int q = 0; q < kP; ++q) {
-        const int nt = nt0 + 2 * q;
-        if (nt < nnt) {
-          float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp + nt * 8 + 2 * tig;
-          if (row < a.B) *reinterpret_cast<float2*>(dst) = make_float2(acc[q][0], acc[q][1]);
-          if (row + 8 < a.B)
-            *reinterpret_cast<float2*>(dst + 8 * static_cast<int64_t>(rp)) = make_float2(acc[q][2], acc[q][3]);
-        }
-      }
-    }
+    g += nsub;
+    __syncthreads();   // the drain is done before the next unit's first MMA; stages are free
+    if (abort_sh) break;
   }
+  cp_async_wait<0>();   // no copy is still on its way when the CTA ends
   // per-CTA maximum -> ws_max[blockIdx.x]
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
@@ -330,6 +338,10 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
     float mx = red[0];
     for (int w = 1; w < kWorkWarps; ++w) mx = fmaxf(mx, red[w]);
     a.ws_max[blockIdx.x] = mx;
+  }
+  if (rp > 0 && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols_for(rp));
   }
 }
 
@@ -495,23 +507,12 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
   }
 }
 
-// x rows, ld rows and the scale values (kSub bytes of x hold at most 128 columns)
-size_t stage_bytes(int rank_pad) { return static_cast<size_t>(kRows + rank_pad) * kPitch + kScaleBytes; }
-
 template <typename TIn>
 cudaError_t launch_stats(const ActArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  cudaError_t err;
-  if (a.rank_pad <= 64) {
-    err = cudaFuncSetAttribute(act_stats_kernel<TIn, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    act_stats_kernel<TIn, 4><<<grid, kWork, smem, stream>>>(a);
-  } else {
-    err = cudaFuncSetAttribute(act_stats_kernel<TIn, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    act_stats_kernel<TIn, 16><<<grid, kWork, smem, stream>>>(a);
-  }
+  cudaError_t err = cudaFuncSetAttribute(act_stats_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  act_stats_kernel<TIn><<<grid, kWork, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -535,10 +536,10 @@ void finish_act_plan(ActPlan& p) {
   // stages: as many as fit, no more than the longest unit's sub-chunks + 1
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   const int sub_max = (steps_max * kTileBytes + kSub - 1) / kSub;
-  const size_t sb = stage_bytes(p.rank_pad);
-  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, kStatsSmemBudget / sb));
+  const size_t sb = static_cast<size_t>(stats_stage_bytes(p.rank_pad));
+  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kStatsSmemBudget - 1024) / sb));
   p.stages = std::max(2, std::min(p.stages, sub_max + 1));
-  p.smem = sb * p.stages;
+  p.smem = sb * p.stages + 1024;   // + alignment of the first stage to 1024 bytes
   // one CTA per SM (512 threads, most of the shared memory)
   p.grid = std::min(p.nunits, num_sms());
   p.nparts = p.grid;
@@ -630,6 +631,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.sf = static_cast<uint8_t*>(sf);
   a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
   a.act_scale = act_scale;
+  a.status = device_status_word();
   // without the down factor the stages hold x alone (fewer bytes per stage)
   ActPlan q = p;
   if (!has_ld) {
