@@ -534,7 +534,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()), "steps": Ke,
                 "call": "svdq_linear (pinned host x -> device, Y -> pinned host)"},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 3 * K,   # per step: activation stats, activation codes, residual GEMM
         "sweep": sweep,
         "clocks": clocks,
     }
