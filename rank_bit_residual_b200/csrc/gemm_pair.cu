@@ -61,8 +61,10 @@ constexpr uint32_t kNvOutCol = 384;               // NVFP4 bf16 pass-1 result
 
 template <int kKind>
 struct PairCfg {
-  static constexpr int kStages = kKind == kKindNvfp4 ? 5 : 6;
-  static constexpr int kStageBytes = kABytes + kBBytes + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
+  // INT: two 128-byte K blocks per stage (8 MMAs per barrier wait and commit)
+  static constexpr int kKb = kKind == kKindNvfp4 ? 1 : 2;
+  static constexpr int kStages = kKind == kKindNvfp4 ? 5 : 3;
+  static constexpr int kStageBytes = kKb * (kABytes + kBBytes) + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
 };
 
 // Whether the epilogue's stores overlap the next tile's MMAs.
@@ -102,7 +104,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int tiles_m = (B + 2 * kHalf - 1) / (2 * kHalf);
   const int tiles_n = (N + kTileN - 1) / kTileN;
   const int total = tiles_m * tiles_n;
-  constexpr int kStageK = kKind == kKindNvfp4 ? 256 : 128;
+  constexpr int kKb = PairCfg<kKind>::kKb;
+  constexpr int kStageK = kKind == kKindNvfp4 ? 256 : 128 * kKb;   // K elements per stage
   const int ksteps = (M + kStageK - 1) / kStageK;
   const int steps_per_tile = ksteps + lr_steps;   // residual steps first
 
@@ -167,9 +170,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int rt = 0; rt < 2; ++rt)
               tma_load_2d_pair(sfb_s + rt * 2048, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
           } else {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
-            tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
-            tma_load_2d_pair(st + kABytes, &tm_b, fb, 128 * j, n0);
+            // A blocks then B blocks, 128 bytes of K each
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kKb * (kABytes + kBBytes));
+            for (int kb = 0; kb < kKb; ++kb) {
+              tma_load_2d_pair(st + kb * kABytes, &tm_a, fb, kStageK * j + 128 * kb, m0);
+              tma_load_2d_pair(st + kKb * kABytes + kb * kBBytes, &tm_b, fb, kStageK * j + 128 * kb, n0);
+            }
           }
         }
       }
@@ -238,9 +244,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               mma_nvf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
                             (j > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
           } else {
+            const uint32_t bb = a0 + kKb * kABytes;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_i8_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_i8,
+            for (int kk = 0; kk < 4 * kKb; ++kk)
+              mma_i8_pair(tmem, smem_desc_sw128(a0 + (kk >> 2) * kABytes + 32 * (kk & 3)),
+                          smem_desc_sw128(bb + (kk >> 2) * kBBytes + 32 * (kk & 3)), id_i8,
                           (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty_bar[s], 0x3);
@@ -286,7 +294,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int row = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf + r_in;
       const int nt = (t / tiles_m) * kTileN;
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (kTwoPass) {
+      if constexpr (kTwoPass && kKind == kKindInt) {
+        // the warp's four accumulator chunks go to registers first, so the
+        // accumulator is handed back to the next tile's MMAs before any
+        // arithmetic; each chunk's result then goes in place over its own
+        // low-rank columns
+        uint32_t accs[4][32];
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(lane_addr + 32u * (4 * h + i), accs[i]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_ld_wait_regs(accs[i]);
+        release(acc_empty_even, &acc_empty_bar);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = 4 * h + i;
+          const int n = nt + 32 * c;
+          if (n < N) epilogue_combine_regs<kOut>(args, lane_addr, n, accs[i], 256u + 32u * c, alpha, sep_lr);
+        }
+        tmem_st_wait();
+        for (int c = 4 * h; c < 4 * h + 4; ++c) {
+          const int n = nt + 32 * c;
+          if (n < N) epilogue_store<kOut>(args, lane_addr, row, n, 256u + 32u * c);
+        }
+        release(lr_empty_even, &lr_empty_bar);
+      } else if constexpr (kTwoPass) {
         // the result of column chunk c goes to dst(c): INT in place over its
         // own low-rank columns, NVFP4 (bf16) to the free columns from 384
         auto dst = [](int c) -> uint32_t {
