@@ -138,19 +138,19 @@ __device__ __forceinline__ void epilogue_chunk_direct(const GemmArgs& args, uint
 }
 
 // Two-pass epilogue (overlaps the global stores with the next tile's MMAs).
-// Pass 1, one warp and 32 columns: alpha * acc (+ up) + bias is written back
-// into TMEM at dst_col (bf16 pairs in 16 columns, or fp32 in 32), so the
-// accumulator columns can be handed back to the MMA before any store to Y.
+// Pass 1 from accumulator values already in registers (the accumulator columns
+// are free again): the INT up-projection columns at lr_col are read, and the
+// result goes to dst_col (bf16 pairs in 16 columns, or fp32 in 32).
 template <int kKind, int kOut>
-__device__ __forceinline__ void epilogue_combine(const GemmArgs& args, uint32_t lane_addr, int n,
-                                                 uint32_t acc_col, uint32_t lr_col, uint32_t dst_col,
-                                                 float alpha, bool sep_lr) {
+__device__ __forceinline__ void epilogue_combine_regs(const GemmArgs& args, uint32_t lane_addr, int n,
+                                                      const uint32_t (&acc)[32], uint32_t lr_col,
+                                                      uint32_t dst_col, float alpha, bool sep_lr) {
   __syncwarp();
-  uint32_t acc[32], up[32];
-  tmem_ld_32x32b_x32(lane_addr + acc_col, acc);
-  if (sep_lr) tmem_ld_32x32b_x32(lane_addr + lr_col, up);
-  tmem_ld_wait_regs(acc);
-  if (sep_lr) tmem_ld_wait_regs(up);
+  uint32_t up[32];
+  if (sep_lr) {
+    tmem_ld_32x32b_x32(lane_addr + lr_col, up);
+    tmem_ld_wait_regs(up);
+  }
   float v[32];
   dequant32<kKind>(acc, up, alpha, sep_lr, v);
   add_bias32(args, n, v);
@@ -164,34 +164,6 @@ __device__ __forceinline__ void epilogue_combine(const GemmArgs& args, uint32_t 
 #pragma unroll
     for (int j = 0; j < 32; ++j) p[j] = __float_as_uint(v[j]);
     tmem_st_32x32b_x32(lane_addr + dst_col, p);
-  }
-}
-
-// Pass 1 of the INT epilogue from accumulator values already in registers: the
-// up-projection columns at lr_col are read and overwritten in place by the result.
-template <int kOut>
-__device__ __forceinline__ void epilogue_combine_regs(const GemmArgs& args, uint32_t lane_addr, int n,
-                                                      const uint32_t (&acc)[32], uint32_t lr_col, float alpha,
-                                                      bool sep_lr) {
-  __syncwarp();
-  uint32_t up[32];
-  if (sep_lr) {
-    tmem_ld_32x32b_x32(lane_addr + lr_col, up);
-    tmem_ld_wait_regs(up);
-  }
-  float v[32];
-  dequant32<kKindInt>(acc, up, alpha, sep_lr, v);
-  add_bias32(args, n, v);
-  if (kOut == kOutBF16) {
-    uint32_t p[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) p[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-    tmem_st_32x32b_x16(lane_addr + lr_col, p);
-  } else {
-    uint32_t p[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) p[j] = __float_as_uint(v[j]);
-    tmem_st_32x32b_x32(lane_addr + lr_col, p);
   }
 }
 

@@ -294,11 +294,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int row = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf + r_in;
       const int nt = (t / tiles_m) * kTileN;
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (kTwoPass && kKind == kKindInt) {
+      if constexpr (kTwoPass) {
         // the warp's four accumulator chunks go to registers first, so the
         // accumulator is handed back to the next tile's MMAs before any
-        // arithmetic; each chunk's result then goes in place over its own
-        // low-rank columns
+        // arithmetic; the result of chunk c then goes to dst(c): INT in place
+        // over its own low-rank columns, NVFP4 (bf16) to the free columns
+        // from 384
+        auto dst = [](int c) -> uint32_t {
+          return kKind == kKindInt ? 256u + 32u * c : kNvOutCol + 16u * c;
+        };
         uint32_t accs[4][32];
         __syncwarp();
 #pragma unroll
@@ -310,27 +314,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int c = 4 * h + i;
           const int n = nt + 32 * c;
-          if (n < N) epilogue_combine_regs<kOut>(args, lane_addr, n, accs[i], 256u + 32u * c, alpha, sep_lr);
-        }
-        tmem_st_wait();
-        for (int c = 4 * h; c < 4 * h + 4; ++c) {
-          const int n = nt + 32 * c;
-          if (n < N) epilogue_store<kOut>(args, lane_addr, row, n, 256u + 32u * c);
-        }
-        release(lr_empty_even, &lr_empty_bar);
-      } else if constexpr (kTwoPass) {
-        // the result of column chunk c goes to dst(c): INT in place over its
-        // own low-rank columns, NVFP4 (bf16) to the free columns from 384
-        auto dst = [](int c) -> uint32_t {
-          return kKind == kKindInt ? 256u + 32u * c : kNvOutCol + 16u * c;
-        };
-        for (int c = 4 * h; c < 4 * h + 4; ++c) {
-          const int n = nt + 32 * c;
           if (n < N)
-            epilogue_combine<kKind, kOut>(args, lane_addr, n, 32u * c, 256u + 32u * c, dst(c), alpha, sep_lr);
+            epilogue_combine_regs<kKind, kOut>(args, lane_addr, n, accs[i], 256u + 32u * c, dst(c), alpha, sep_lr);
         }
         tmem_st_wait();
-        release(acc_empty_even, &acc_empty_bar);
         for (int c = 4 * h; c < 4 * h + 4; ++c) {
           const int n = nt + 32 * c;
           if (n < N) epilogue_store<kOut>(args, lane_addr, row, n, dst(c));
