@@ -124,3 +124,24 @@ def test_long_batch_down_projection(B, M, rank, dtype):
     q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
     assert np.float32(s.item()) == s_o
     assert_codes_match(codes.cpu().numpy(), q, near)
+
+
+# long units (many stats-kernel sub-chunks per unit, ring refills) and short
+# ones, both input types; two calls in a row on the same workspace
+@pytest.mark.parametrize("B,M,dtype", [(2048, 16384, "bf16"), (2048, 3072, "f32"), (2048, 3072, "bf16")])
+def test_large_batch_units_long_and_short(B, M, dtype):
+    wl = make_case(B, M, 16, rank=0, seed=B + M, dtype=dtype)
+    rank = 32
+    rng = np.random.default_rng(9)
+    ld = to_bf16(rng.standard_normal((rank, M)).astype(np.float32) * 0.1)
+    ld_t = to_dev(ld, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    for _ in range(2):
+        codes, _, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "int4", ld=ld_t)
+        q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+        assert np.float32(s.item()) == s_o
+        assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype}")
+        d = down.float().cpu().numpy().astype(np.float64)
+        got = d[:, :rank] + d[:, rank:]
+        want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
+        tol = 2e-5 if dtype == "bf16" else 3e-3
+        assert rel_fro(got, want) <= tol, rel_fro(got, want)

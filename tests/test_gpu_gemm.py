@@ -91,3 +91,20 @@ def test_linear_nvfp4_matches_oracle(B, M, N, rank, bias, xdt, given_gs):
     want = w.oracle_y(wl.x, wl.bias if bias else None, gs_x=gs)
     assert_y_close(y32.cpu().numpy(), want, f"nvfp4 {B}x{M}x{N} r={rank} {xdt}")
     assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_linear_workspace_reused_across_shapes():
+    """One workspace for calls of different batch sizes (the large- and the
+    short-batch paths): each call equals a call on a fresh workspace, bit for
+    bit, and the oracle within tolerance."""
+    M, N, rank = 512, 256, 32
+    w = SyntheticWeight(M, N, rank, "int4", seed=5)
+    shared = rb.LinearWorkspace()
+    for i, B in enumerate((300, 1024, 64, 300, 2048, 300)):
+        wl = make_case(B, M, N, rank=0, seed=100 + i)
+        x = x_tensor(wl)
+        y_shared = rb.svdq_linear(w.w, x, out_dtype=torch.float32, workspace=shared)
+        y_fresh = rb.svdq_linear(w.w, x, out_dtype=torch.float32, workspace=rb.LinearWorkspace())
+        assert rb.svdq_check_status() == rb.SVDQ_OK
+        assert torch.equal(y_shared, y_fresh), f"call {i} (B={B})"
+        assert_y_close(y_shared.cpu().numpy(), w.oracle_y(wl.x), f"call {i} B={B}")
