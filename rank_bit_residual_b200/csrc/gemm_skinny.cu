@@ -381,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q = warp & 3;
       const int nloc = q * 32 + lane;                 // weight row within the tile
       const int p = nloc / a.sh, nl = nloc - p * a.sh;
-      uint32_t* dst = stg + static_cast<size_t>(p) * slot_words + nl;
+      // shared-window stores (the pointer's origin is not visible to the compiler)
+      const uint32_t dst_s = smem_u32(stg + static_cast<size_t>(p) * slot_words + nl);
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
       const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
       for (int c0 = 0; c0 < a.B; c0 += 32) {
@@ -406,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lr_here) f += __uint_as_float(up[j]);
             v = __float_as_uint(f);
           }
-          dst[(c0 + j) * a.sh] = v;
+          st_shared_u32(dst_s + static_cast<uint32_t>((c0 + j) * a.sh) * 4u, v);
         }
       }
     }
@@ -441,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int4 s = make_int4(0, 0, 0, 0);
         for (int c = 0; c < S; ++c) {
           const uint32_t* src = (c == rank ? stg + static_cast<size_t>(c) * slot_words : recv + static_cast<size_t>(c) * slot_words);
-          const int4 v = *reinterpret_cast<const int4*>(src + b * a.sh + nl);
-          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+          const uint4 v = ld_shared_v4(smem_u32(src + b * a.sh + nl));
+          s.x += static_cast<int>(v.x); s.y += static_cast<int>(v.y); s.z += static_cast<int>(v.z); s.w += static_cast<int>(v.w);
         }
         int32_t* dst = static_cast<int32_t*>(a.y) + static_cast<int64_t>(b) * a.ldy + n;
         if (a.vec_ok) {
@@ -454,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int c = 0; c < S; ++c) {
           const uint32_t* src = (c == rank ? stg + static_cast<size_t>(c) * slot_words : recv + static_cast<size_t>(c) * slot_words);
-          const float4 v = *reinterpret_cast<const float4*>(src + b * a.sh + nl);
-          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+          const uint4 v = ld_shared_v4(smem_u32(src + b * a.sh + nl));
+          s.x += __uint_as_float(v.x); s.y += __uint_as_float(v.y); s.z += __uint_as_float(v.z); s.w += __uint_as_float(v.w);
         }
         float o[4] = {s.x, s.y, s.z, s.w};
         if (kFmt == kFmtNvfp4) {
