@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
         uint32_t m = 0u;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          m = abs_max_word<TIn>(m, *reinterpret_cast<const uint32_t*>(st + swz(rs + 8 * i, wi >> 2, kRows) + 4 * (wi & 3)));
+          m = abs_max_word<TIn>(m, ld_shared_u32(smem_u32(st + swz(rs + 8 * i, wi >> 2, kRows) + 4 * (wi & 3))));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 4));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 8));
         m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 16));

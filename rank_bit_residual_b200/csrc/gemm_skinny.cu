@@ -342,12 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < 4; ++it) {
           const int idx = t + 128 * it;            // 16-byte piece of the packed tile
           const int row = idx >> 2, q = idx & 3;   // row, quarter of its 64 bytes
-          const uint4 v = *reinterpret_cast<const uint4*>(src + row * 64 + q * 16);
+          const uint4 v = ld_shared_v4(smem_u32(src + row * 64 + q * 16));
           uint32_t o[8];
           widen_int4(v, o);
           uint8_t* drow = dst + row * 128;
-          *reinterpret_cast<uint4*>(drow + (((2 * q) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(drow + (((2 * q + 1) ^ (row & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          st_shared_v4(smem_u32(drow + (((2 * q) ^ (row & 7)) << 4)), make_uint4(o[0], o[1], o[2], o[3]));
+          st_shared_v4(smem_u32(drow + (((2 * q + 1) ^ (row & 7)) << 4)), make_uint4(o[4], o[5], o[6], o[7]));
         }
         fence_proxy_async_smem();
         __syncwarp();
