@@ -68,6 +68,7 @@ struct ActArgs {
   int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
   int nparts;       // partial maxima written by the stats kernel
   int stages;       // stats kernel: shared-memory stages
+  int nacc;         // stats kernel: MMA issuers, each with its own TMEM accumulator
   const void* x;
   const float* scale;
   const float* gs_given;
@@ -194,13 +195,15 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   const uint32_t idesc = kEsz == 2 ? idesc_bf16(kRows, rp > 0 ? rp : 16) : idesc_tf32(kRows, rp > 0 ? rp : 16);
   float run = 0.0f;
 
+  const int nacc = a.nacc;
+  const uint32_t acc_cols = tmem_cols_for(rp);
   if (tid == 0) {
-    for (int s = 0; s < kMaxStages; ++s) mbar_init(&mma_bar[s], 1);
+    for (int s = 0; s < kMaxStages; ++s) mbar_init(&mma_bar[s], nacc);
     fence_mbar_init();
     abort_sh = 0;
   }
   if (rp > 0 && warp == 0) {
-    tmem_alloc(&tmem_sh, tmem_cols_for(rp));
+    tmem_alloc(&tmem_sh, acc_cols * nacc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -256,17 +259,20 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
       fence_proxy_async_smem();     // ... and are visible to the tensor core
       __syncthreads();              // everyone's have; every thread is done with sub-chunk c - 1
       if (abort_sh) break;          // a bounded wait gave up (uniform after the barrier)
-      if (rp > 0 && tid == 0) {
+      if (rp > 0 && lane == 0 && warp < nacc) {
+        // lane 0 of warps 0 .. nacc - 1 (one per SM sub-partition) each issue a
+        // share of the sub-chunk's MMAs into an accumulator of their own
         tc_fence_after();
         const uint32_t xa = smem_u32(st), la = xa + ld_off;
-#pragma unroll
-        for (int kk = 0; kk < kSub / 32; ++kk) {   // 32 bytes of K per MMA
+        const uint32_t acc = tmem + acc_cols * warp;
+        const int kk0 = warp * (kSub / 32) / nacc, kk1 = (warp + 1) * (kSub / 32) / nacc;
+        for (int kk = kk0; kk < kk1; ++kk) {   // 32 bytes of K per MMA
           const uint32_t off = (kk >> 2) * kRows * kTileBytes + (kk & 3) * 32;
           const uint32_t offl = (kk >> 2) * rp * kTileBytes + (kk & 3) * 32;
           if constexpr (kEsz == 2)
-            mma_f16(tmem, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(acc, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > kk0) ? 1u : 0u);
           else
-            mma_tf32(tmem, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+            mma_tf32(acc, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > kk0) ? 1u : 0u);
         }
         mma_commit(&mma_bar[gc % stages]);
       }
@@ -310,15 +316,19 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
         const int row = m0 + warp * 32 + lane;
         float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp;
         for (int c0 = 0; c0 < rp; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-          tmem_ld_wait_regs(v);
+          // the accumulators summed in issuer order
+          float sum[16];
+          for (int q = 0; q < nacc; ++q) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc_cols * q + c0, v);
+            tmem_ld_wait_regs(v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) sum[j] = q == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+          }
           if (ok && row < a.B) {
 #pragma unroll
             for (int j = 0; j < 16; j += 4)
-              *reinterpret_cast<float4*>(dst + c0 + j) =
-                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                              __uint_as_float(v[j + 3]));
+              *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
           }
         }
         tc_fence_before();
@@ -341,7 +351,7 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   }
   if (rp > 0 && warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols_for(rp));
+    tmem_dealloc(tmem, acc_cols * nacc);
   }
 }
 
@@ -639,6 +649,8 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
     finish_act_plan(q);
   }
   a.stages = q.stages;
+  // as many MMA issuers (up to 4) as TMEM holds accumulators of rank_pad columns
+  a.nacc = a.rank_pad > 0 ? static_cast<int>(std::min<uint32_t>(4u, 512u / tmem_cols_for(a.rank_pad))) : 1;
   // the codes kernel keeps only the unit's reciprocals in shared memory
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   const size_t smem2 = static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
