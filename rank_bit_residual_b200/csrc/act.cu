@@ -106,21 +106,6 @@ __device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
   }
 }
 
-// Copy 16 bytes global -> shared, bypassing L1; src_bytes = 0 fills zeros and
-// reads nothing (src must still be a valid address).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const float* src, int src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int kN>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(kN) : "memory");
-}
 // Wait until at most stages - 2 groups are pending (stages in [2, kMaxStages]).
 __device__ __forceinline__ void cp_async_wait_ring(int stages) {
   switch (stages) {

@@ -501,6 +501,227 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ GEMV
+// Batches of at most kGemvMaxB rows with INT weights. The tensor-core path
+// above issues one MMA per 32 bytes of K per 128 weight rows whatever the
+// batch, and for one or two rows that issue rate, not HBM, sets its time; here
+// the int32 dot products run on the integer units (dp4a) instead. (dp4a runs
+// at a fraction of the FP32 rate on this part: measured per decode step, one
+// row 13.1 us here against 15.4 us on the tensor cores, two rows 14.5 us, four
+// 17.5 us, eight 24.1 us.) Each CTA
+// owns rows_per_cta consecutive weight rows: it copies them (and their lu rows)
+// into shared memory before griddepcontrol.wait, so the whole weight stream
+// overlaps the activation pass; after the wait it copies the activation codes
+// and down hi | lo, and each warp forms the B dot products of its rows (lanes
+// split K), then Y = alpha acc + down . lu + bias.
+constexpr int kGemvMaxB = 2;   // past two rows the dp4a rate makes the tensor-core path faster
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr size_t kGemvSmemMax = 200 * 1024;
+
+struct GemvArgs {
+  int B, N, M, rp, rows_per_cta, row_bytes;
+  const uint8_t* w;             // packed [N, M/2] or int8 [N, M]
+  const int8_t* act;            // [B, M]
+  const __nv_bfloat16* down2;   // [B, 2 rp]
+  const __nv_bfloat16* lu;      // [N, 2 rp]
+  const float* s_x;
+  const float* s_w;
+  const __nv_bfloat16* bias;
+  void* y;
+  int64_t ldy;
+};
+
+__host__ __device__ constexpr size_t gemv_smem(int rows, int row_bytes, int B, int M, int rp) {
+  return static_cast<size_t>(rows) * row_bytes + static_cast<size_t>(rows) * 4 * rp +
+         static_cast<size_t>(B) * M + static_cast<size_t>(B) * 4 * rp + 64;
+}
+
+template <bool kPacked, int kOut>
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs g) {
+  extern __shared__ __align__(16) uint8_t gsm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * g.rows_per_cta;
+  const int rows = min(g.rows_per_cta, g.N - n0);
+  const int lrw = 2 * g.rp * 2;   // bytes of a lu / down2 row
+  uint8_t* ws = gsm;                                                  // [rows_per_cta][row_bytes]
+  uint8_t* lus = ws + static_cast<size_t>(g.rows_per_cta) * g.row_bytes;       // [rows_per_cta][4 rp]
+  uint8_t* acts = lus + static_cast<size_t>(g.rows_per_cta) * lrw;              // [B][M]
+  uint8_t* dns = acts + static_cast<size_t>(g.B) * g.M;                         // [B][4 rp]
+  // weight side, independent of the activation pass
+  {
+    const int per_row = g.row_bytes / 16, total = rows * per_row;
+    for (int i = tid; i < total; i += kGemvThreads) {
+      const int r = i / per_row, c = i - r * per_row;
+      cp_async16(ws + static_cast<size_t>(r) * g.row_bytes + 16 * c,
+                 g.w + static_cast<int64_t>(n0 + r) * g.row_bytes + 16 * c, 16);
+    }
+    const int lper = lrw / 16, ltot = (kOut == kOutI32 ? 0 : rows * lper);
+    for (int i = tid; i < ltot; i += kGemvThreads) {
+      const int r = i / lper, c = i - r * lper;
+      cp_async16(lus + r * lrw + 16 * c, reinterpret_cast<const uint8_t*>(g.lu) + static_cast<int64_t>(n0 + r) * lrw + 16 * c,
+                 16);
+    }
+    cp_async_commit();
+  }
+  pdl_wait();   // codes, down and s_x come from the activation pass
+  {
+    const int per_row = g.M / 16, total = g.B * per_row;
+    for (int i = tid; i < total; i += kGemvThreads)
+      cp_async16(acts + 16 * i, reinterpret_cast<const uint8_t*>(g.act) + 16 * i, 16);
+    const int dtot = (kOut == kOutI32 ? 0 : g.B * lrw / 16);
+    for (int i = tid; i < dtot; i += kGemvThreads)
+      cp_async16(dns + 16 * i, reinterpret_cast<const uint8_t*>(g.down2) + 16 * i, 16);
+    cp_async_commit();
+  }
+  const float alpha = kOut == kOutI32 ? 0.0f : __ldg(g.s_x) * __ldg(g.s_w);
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // one 16-byte weight chunk per lane and step (32 packed codes, K = 32, or 16
+  // int8 codes) for kRB rows at once, so each activation chunk read from shared
+  // memory serves kRB rows
+  constexpr int kK = kPacked ? 32 : 16;
+  constexpr int kRB = 4;
+  const int nchunks = g.row_bytes / 16;
+  for (int r0 = warp * kRB; r0 < rows; r0 += kGemvWarps * kRB) {
+    int acc[kRB][kGemvMaxB];
+#pragma unroll
+    for (int i = 0; i < kRB; ++i)
+#pragma unroll
+      for (int b = 0; b < kGemvMaxB; ++b) acc[i][b] = 0;
+    for (int j = lane; j < nchunks; j += 32) {
+      uint32_t w8[kRB][kK / 4];
+#pragma unroll
+      for (int i = 0; i < kRB; ++i) {
+        const int r = min(r0 + i, rows - 1);   // rows past the end repeat the last (not stored)
+        const uint4 wv = ld_shared_v4(smem_u32(ws + static_cast<size_t>(r) * g.row_bytes + 16 * j));
+        if constexpr (kPacked) {
+          widen_int4(wv, *reinterpret_cast<uint32_t(*)[8]>(w8[i]));
+        } else {
+          w8[i][0] = wv.x; w8[i][1] = wv.y; w8[i][2] = wv.z; w8[i][3] = wv.w;
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kGemvMaxB; ++b) {
+        if (b >= g.B) break;
+        const uint32_t abase = smem_u32(acts + static_cast<size_t>(b) * g.M + kK * j);
+#pragma unroll
+        for (int h = 0; h < kK / 16; ++h) {
+          const uint4 av = ld_shared_v4(abase + 16 * h);
+#pragma unroll
+          for (int i = 0; i < kRB; ++i) {
+            acc[i][b] = __dp4a(static_cast<int>(w8[i][4 * h + 0]), static_cast<int>(av.x), acc[i][b]);
+            acc[i][b] = __dp4a(static_cast<int>(w8[i][4 * h + 1]), static_cast<int>(av.y), acc[i][b]);
+            acc[i][b] = __dp4a(static_cast<int>(w8[i][4 * h + 2]), static_cast<int>(av.z), acc[i][b]);
+            acc[i][b] = __dp4a(static_cast<int>(w8[i][4 * h + 3]), static_cast<int>(av.w), acc[i][b]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRB; ++i) {
+      const int r = r0 + i;
+      if (r >= rows) break;
+      // every lane ends up with every batch row's sum; lane b keeps row b's
+      int mine = 0;
+#pragma unroll
+      for (int b = 0; b < kGemvMaxB; ++b) {
+        if (b >= g.B) break;
+        int v = acc[i][b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == b) mine = v;
+      }
+      const int n = n0 + r;
+      if (lane < g.B) {
+        const int b = lane;
+        if constexpr (kOut == kOutI32) {
+          static_cast<int32_t*>(g.y)[static_cast<int64_t>(b) * g.ldy + n] = mine;
+        } else {
+          // the up-projection: down hi | lo against lu (both halves of lu hold L2)
+          float up = 0.0f;
+          const __nv_bfloat16* dr = reinterpret_cast<const __nv_bfloat16*>(dns + b * lrw);
+          const __nv_bfloat16* lr = reinterpret_cast<const __nv_bfloat16*>(lus + r * lrw);
+          for (int q = 0; q < 2 * g.rp; ++q) up = fmaf(__bfloat162float(dr[q]), __bfloat162float(lr[q]), up);
+          float v = alpha * static_cast<float>(mine) + up;
+          if (g.bias != nullptr) v += __bfloat162float(g.bias[n]);
+          if constexpr (kOut == kOutF32)
+            static_cast<float*>(g.y)[static_cast<int64_t>(b) * g.ldy + n] = v;
+          else
+            static_cast<__nv_bfloat16*>(g.y)[static_cast<int64_t>(b) * g.ldy + n] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+  }
+}
+
+template <bool kPacked, int kOut>
+cudaError_t launch_gemv_one(const GemvArgs& g, int grid, size_t smem, bool pdl, cudaStream_t st) {
+  auto kern = gemv_kernel<kPacked, kOut>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, g);
+}
+
+// The GEMV path when it applies (INT weights, B <= kGemvMaxB, everything in
+// shared memory); false (nothing launched) otherwise.
+bool launch_gemv(int out, const GemmArgs& ga, const void* act_codes, const void* down2, const svdq_weight* w,
+                 bool pdl, cudaStream_t stream, cudaError_t* err) {
+  const int64_t M = w->M, N = w->N, B = ga.B;
+  if (B < 1 || B > kGemvMaxB) return false;
+  const bool packed = w->fmt.bits <= 4 && w->codes4 != nullptr;
+  const int row_bytes = static_cast<int>(packed ? M / 2 : M);
+  const int rp = (out != kOutI32 && down2 != nullptr) ? w->rank_pad : 0;
+  const int rows = static_cast<int>(round_up(ceil_div(N, num_sms()), kGemvWarps));
+  const size_t smem = gemv_smem(rows, row_bytes, static_cast<int>(B), static_cast<int>(M), rp);
+  if (smem > kGemvSmemMax) return false;
+  for (const void* q : {static_cast<const void*>(packed ? w->codes4 : w->codes), act_codes, down2,
+                        static_cast<const void*>(w->lu)})
+    if (q != nullptr && (reinterpret_cast<uintptr_t>(q) & 15) != 0) return false;
+  GemvArgs g{};
+  g.B = static_cast<int>(B);
+  g.N = static_cast<int>(N);
+  g.M = static_cast<int>(M);
+  g.rp = rp;
+  g.rows_per_cta = rows;
+  g.row_bytes = row_bytes;
+  g.w = static_cast<const uint8_t*>(packed ? w->codes4 : w->codes);
+  g.act = static_cast<const int8_t*>(act_codes);
+  g.down2 = static_cast<const __nv_bfloat16*>(down2);
+  g.lu = static_cast<const __nv_bfloat16*>(w->lu);
+  g.s_x = ga.s_x;
+  g.s_w = ga.s_w;
+  g.bias = ga.bias;
+  g.y = ga.y;
+  g.ldy = ga.ldy;
+  const int grid = static_cast<int>(ceil_div(N, rows));
+#define SVDQ_GEMV(P, O) *err = launch_gemv_one<P, O>(g, grid, smem, pdl, stream)
+  if (packed) {
+    if (out == kOutI32) SVDQ_GEMV(true, kOutI32);
+    else if (out == kOutF32) SVDQ_GEMV(true, kOutF32);
+    else SVDQ_GEMV(true, kOutBF16);
+  } else {
+    if (out == kOutI32) SVDQ_GEMV(false, kOutI32);
+    else if (out == kOutF32) SVDQ_GEMV(false, kOutF32);
+    else SVDQ_GEMV(false, kOutBF16);
+  }
+#undef SVDQ_GEMV
+  return true;
+}
+
 struct SkinnyPlan {
   int S, sh, dr, dp, a_slot, b_slot;
   size_t smem;
@@ -576,6 +797,7 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   *err = cudaSuccess;
   const int64_t M = w->M, N = w->N, B = g.B;
   if (B <= 0 || B > 128) return false;
+  if (kind == kKindInt && launch_gemv(out, g, act_codes, down2, w, pdl, stream, err)) return true;
   const int Bp = static_cast<int>(std::max<int64_t>(16, round_up(B, 16)));
   const bool packed = kind == kKindInt && w->fmt.bits <= 4 && w->codes4 != nullptr;
   const int fmt = kind == kKindNvfp4 ? kFmtNvfp4 : (packed ? kFmtInt4 : kFmtInt8);
