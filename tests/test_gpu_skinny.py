@@ -27,7 +27,7 @@ def test_pack_int4_matches_nibble_packing(N, M):
 # (B, M, N): cluster sizes 1..8 (K steps and tile count decide it), ragged N
 # tiles, B from 1 to 128
 SHAPES = [(1, 32, 16), (1, 4096, 4096), (16, 1024, 16), (77, 768, 272), (128, 4096, 3072),
-          (128, 512, 12288), (33, 2048, 1040), (128, 128, 128), (5, 896, 144)]
+          (128, 512, 12288), (33, 2048, 1040), (128, 128, 128), (5, 896, 144), (2, 512, 272)]
 
 
 @pytest.mark.parametrize("B,M,N", SHAPES)
