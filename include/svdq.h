@@ -271,6 +271,28 @@ svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, co
 svdq_status svdq_residual_product_i32(const svdq_weight* w, const int8_t* act_codes, int64_t B,
                                       int32_t* acc, int64_t ldacc, svdq_stream_t stream);
 
+/*
+ * svdq_smooth_scale - the per-channel smoothing scale, upstream of svdq_prepare.
+ * "SVDQuant Smoothing, Low-rank and Residual Quantization" (Formula item 1) takes
+ * the scale as given; the "SVDQuant parameter configuration guide" (msModelSlim),
+ * step 3 "choose and tune the parameters", tunes its migration strength
+ * (iter_smooth.alpha). Read as
+ *   scale[j] = max_b |x[b, j]|^alpha / max_n |W[j, n]|^(1 - alpha)
+ * over calibration activations x, where a factor whose maximum is zero is 1.
+ *
+ *   x        device [B, M] (ldx >= M), bf16 or fp32 (B = 0: the x factor is 1)
+ *   W        device [M, N] (ldw >= N), bf16 or fp32
+ *   alpha    migration strength in [0, 1]
+ *   scale    out device fp32 [M]
+ *   workspace  at least 8 * M bytes (two maxima arrays), overwritten
+ * Host errors: SVDQ_EINVAL for null pointers, alpha outside [0, 1], M or N < 1,
+ * B < 0, ldx < M or ldw < N; SVDQ_EWORKSPACE for a short workspace. The fp32 pow
+ * is not correctly rounded: scale is within a few ulps of the exact value.
+ */
+svdq_status svdq_smooth_scale(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx,
+                              const void* W, svdq_dtype w_dtype, int64_t N, int64_t ldw, float alpha,
+                              float* scale, void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
 /* Synchronises `stream`, returns and clears the device status word
  * (SVDQ_OK, SVDQ_EINVAL or SVDQ_ETIMEOUT), or SVDQ_ECUDA on a runtime error. */
 svdq_status svdq_check_status(svdq_stream_t stream);

@@ -11,9 +11,17 @@ relative Frobenius distance of Y to x @ W (float64), and the singular values are
 of W and of the smoothed weight diag(scale) W, whose leading directions are what a
 rank-r branch can keep out of the quantiser.
 
-    python -m rank_bit_residual_b200.ablation [--workload NAME] [--rows B] [--ranks 0,1,2,...]
+The smoothing scale's migration strength (the "SVDQuant parameter configuration
+guide", step 3 "choose and tune the parameters": iter_smooth.alpha) is chosen the
+same way: select_alpha computes the scale of each candidate strength on the GPU
+(svdq_smooth_scale) from calibration activations, runs the two-branch linear at the
+given rank, and keeps the strength with the smallest output error.
 
-prints one JSON object (errors per variant and rank, singular values, timings).
+    python -m rank_bit_residual_b200.ablation [--workload NAME] [--rows B] [--ranks 0,1,2,...]
+                                              [--alphas 0.25,0.5,0.75,0.9]
+
+prints one JSON object (errors per variant and rank, singular values, timings, and
+the error per migration strength).
 """
 
 from __future__ import annotations
@@ -28,7 +36,7 @@ from typing import Dict, Optional, Sequence
 import numpy as np
 import torch
 
-from . import svdq_linear, svdq_prepare
+from . import svdq_linear, svdq_prepare, svdq_smooth_scale
 
 
 def rel_fro(y: torch.Tensor, ref: torch.Tensor) -> float:
@@ -78,12 +86,37 @@ def ablation(x: torch.Tensor, W: torch.Tensor, scale: torch.Tensor, ranks: Seque
     return out
 
 
+def select_alpha(x_calib: torch.Tensor, W: torch.Tensor, rank: int, fmt: str = "int4",
+                 alphas: Sequence[float] = (0.25, 0.5, 0.75, 0.9), x_eval: Optional[torch.Tensor] = None,
+                 seed: int = 0) -> Dict:
+    """The migration strength with the smallest two-branch output error.
+
+    The scale of each strength comes from the calibration activations x_calib; the
+    error is measured on x_eval (default: x_calib). Returns the error per strength,
+    the chosen strength and its scale.
+    """
+    xe = x_calib if x_eval is None else x_eval
+    ref = xe.double() @ W.double()
+    table = {}
+    best = None
+    for a in alphas:
+        scale = svdq_smooth_scale(x_calib, W, float(a))
+        w = svdq_prepare(W, scale, rank, fmt, seed=seed)
+        err = rel_fro(svdq_linear(w, xe, out_dtype=torch.float32), ref)
+        table[float(a)] = err
+        if best is None or err < best[1]:
+            best = (float(a), err, scale)
+    return {"errors": table, "alpha": best[0], "error": best[1], "scale": best[2]}
+
+
 def main(argv: Optional[Sequence[str]] = None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--workload", default="dit_attn_4096x3072x3072_int4")
     ap.add_argument("--rows", type=int, default=None, help="keep only the first rows of x")
     ap.add_argument("--ranks", default="0,1,2,3,4,5,6,16,32")
     ap.add_argument("--fmt", default=None, help="override the workload's format (int4, int8, nvfp4)")
+    ap.add_argument("--alphas", default="0.25,0.5,0.75,0.9",
+                    help="migration strengths to compare at the largest rank (empty: skip)")
     args = ap.parse_args(argv)
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     from synth import make_workload
@@ -94,8 +127,12 @@ def main(argv: Optional[Sequence[str]] = None) -> int:
     W = torch.from_numpy(wl.W).to(dev).to(torch.bfloat16 if wl.w_dtype == "bf16" else torch.float32)
     scale = torch.from_numpy(wl.scale).to(dev)
     fmt = args.fmt or (wl.fmt if wl.fmt == "nvfp4" else f"int{wl.bits}")
-    res = ablation(x, W, scale, [int(r) for r in args.ranks.split(",")], fmt=fmt)
+    ranks = [int(r) for r in args.ranks.split(",")]
+    res = ablation(x, W, scale, ranks, fmt=fmt)
     res["workload"] = args.workload
+    if args.alphas:
+        sel = select_alpha(x, W, max(ranks), fmt, [float(a) for a in args.alphas.split(",")])
+        res["alpha_selection"] = {"rank": max(ranks), "errors": sel["errors"], "alpha": sel["alpha"]}
     print(json.dumps(res))
     return 0
 

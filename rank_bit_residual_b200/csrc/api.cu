@@ -411,6 +411,19 @@ svdq_status svdq_residual_product_i32(const svdq_weight* w, const int8_t* act_co
   return from_cuda(e);
 }
 
+svdq_status svdq_smooth_scale(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx,
+                              const void* W, svdq_dtype w_dtype, int64_t N, int64_t ldw, float alpha,
+                              float* scale, void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
+  if (!W || !scale || M < 1 || N < 1 || B < 0 || ldw < N || !(alpha >= 0.0f && alpha <= 1.0f))
+    return SVDQ_EINVAL;
+  if (B > 0 && (!x || ldx < M)) return SVDQ_EINVAL;
+  if ((x_dtype != SVDQ_BF16 && x_dtype != SVDQ_F32) || (w_dtype != SVDQ_BF16 && w_dtype != SVDQ_F32))
+    return SVDQ_EINVAL;
+  if (!workspace || workspace_bytes < static_cast<size_t>(8 * M)) return SVDQ_EWORKSPACE;
+  return from_cuda(launch_smooth_scale(x, x_dtype, B, M, ldx, W, w_dtype, N, ldw, alpha, scale, workspace,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 svdq_status svdq_check_status(svdq_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SVDQ_ECUDA;

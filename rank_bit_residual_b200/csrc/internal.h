@@ -70,6 +70,11 @@ void finish_act_plan(ActPlan& p);
 void finish_act_plan_small(ActPlan& p);
 size_t act_scratch_bytes(const ActPlan& p);
 
+// svdq_smooth_scale (smooth.cu): workspace of 2 * M uint32.
+cudaError_t launch_smooth_scale(const void* x, svdq_dtype xdt, int64_t B, int64_t M, int64_t ldx, const void* w,
+                                svdq_dtype wdt, int64_t N, int64_t ldw, float alpha, float* scale, void* workspace,
+                                cudaStream_t st);
+
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
                        const float* w_global_scale, const void* ld, void* codes, void* sf,
