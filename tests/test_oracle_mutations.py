@@ -136,3 +136,28 @@ def test_planted_mistake_is_caught(monkeypatch, mod, name, bad, pins):
         nargs = pin.__code__.co_argcount
         caught |= _fails(pin, golden) if nargs == 1 else _fails(pin)
     assert caught, f"no pin caught the planted mistake in {name}"
+
+
+# ------------------------------------------------------------------ MXFP4
+import oracle.mxfp4 as mx
+from tests import test_oracle_mxfp4 as T5
+
+
+@pytest.mark.parametrize("emax", [1, 3])
+def test_mxfp4_wrong_element_exponent_is_caught(monkeypatch, emax):
+    monkeypatch.setattr(mx, "E2M1_EMAX", emax)
+    assert _fails(T5.test_worked_blocks) or _fails(T5.test_block_exponent, 6.0, 0)
+
+
+def test_mxfp4_ceil_exponent_is_caught(monkeypatch):
+    def ceil_exp(amax):
+        a = np.asarray(amax, dtype=np.float64)
+        x = np.ceil(np.log2(np.where(a > 0, a, 1.0))).astype(np.int64) - mx.E2M1_EMAX
+        return np.where(a > 0, np.clip(x, -127, 127), -127)
+    monkeypatch.setattr(mx, "block_exponent", ceil_exp)
+    assert _fails(T5.test_worked_blocks)
+
+
+def test_mxfp4_block_of_16_is_caught(monkeypatch):
+    monkeypatch.setattr(mx, "BLOCK", 16)
+    assert _fails(T5.test_worked_blocks) or _fails(T5.test_error_bound_and_product)
