@@ -55,7 +55,11 @@ typedef enum svdq_dtype { SVDQ_F32 = 0, SVDQ_BF16 = 1 } svdq_dtype;
 
 typedef enum svdq_kind {
   SVDQ_KIND_INT = 0,   /* per-tensor symmetric INT grid, bits in [2, 8] */
-  SVDQ_KIND_NVFP4 = 1  /* e2m1 codes, ue4m3 scale per 16 elements, fp32 global scale; bits = 4 */
+  SVDQ_KIND_NVFP4 = 1, /* e2m1 codes, ue4m3 scale per 16 elements, fp32 global scale; bits = 4 */
+  SVDQ_KIND_MXFP4 = 2  /* e2m1 codes, E8M0 (power-of-two) scale per 32 elements, no global
+                          scale; bits = 4. Storage as NVFP4 (packed nibbles, scales in the
+                          128x4 layout over [rows, M/32]); the fp32 "global scale" outputs
+                          (w_scale, act_scale) hold 1 */
 } svdq_kind;
 
 typedef struct svdq_fmt {

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import nvfp4
+from . import mxfp4, nvfp4
 
 
 def low_rank(x, ld, lu) -> np.ndarray:
@@ -56,6 +56,15 @@ def linear_nvfp4(x, ld, lu, a_codes, a_sf, gs_x, w_codes_nk, w_sf, gs_w, bias=No
     """Y = x Ld Lu + (1 / (gs_x gs_w)) sum_blocks (a sfa)(w sfw) [+ bias]."""
     y = low_rank(x, ld, lu) + nvfp4_product(a_codes, a_sf, w_codes_nk, w_sf) / (
         float(gs_x) * float(gs_w))
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
+
+
+def linear_mxfp4(x, ld, lu, a_codes, a_sf, w_codes_nk, w_sf, bias=None):
+    """Y = x Ld Lu + sum_blocks (a 2^Xa)(w 2^Xw) [+ bias]: the MXFP4 variant of
+    the same operator (E8M0 block scales per 32 elements, no global scale)."""
+    y = low_rank(x, ld, lu) + mxfp4.product(a_codes, a_sf, w_codes_nk, w_sf)
     if bias is not None:
         y = y + np.asarray(bias, dtype=np.float64)[None, :]
     return y

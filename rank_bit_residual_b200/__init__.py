@@ -28,7 +28,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "svdq.h")
 
 SVDQ_OK, SVDQ_EINVAL, SVDQ_ERANK, SVDQ_EUNSUPPORTED, SVDQ_ECUDA, SVDQ_ETIMEOUT, SVDQ_EWORKSPACE = range(7)
 SVDQ_F32, SVDQ_BF16 = 0, 1
-KIND_INT, KIND_NVFP4 = 0, 1
+KIND_INT, KIND_NVFP4, KIND_MXFP4 = 0, 1, 2
 
 c_i32, c_i64, c_u64, c_sz, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -114,7 +114,7 @@ def _check(status: int, what: str):
 
 
 def parse_fmt(fmt) -> SvdqFmt:
-    """'int4' / 'int8' / ... / 'nvfp4', or (kind, bits)."""
+    """'int4' / 'int8' / ... / 'nvfp4' / 'mxfp4', or (kind, bits)."""
     if isinstance(fmt, SvdqFmt):
         return fmt
     if isinstance(fmt, tuple):
@@ -124,6 +124,8 @@ def parse_fmt(fmt) -> SvdqFmt:
         return SvdqFmt(KIND_INT, int(m.group(1)))
     if str(fmt) == "nvfp4":
         return SvdqFmt(KIND_NVFP4, 4)
+    if str(fmt) == "mxfp4":
+        return SvdqFmt(KIND_MXFP4, 4)
     raise ValueError(f"unknown format {fmt!r}")
 
 
@@ -212,7 +214,7 @@ def allocate_weight(M: int, N: int, rank: int, fmt, scale: torch.Tensor) -> Prep
     dev = scale.device
     rp = (rank + 15) // 16 * 16
     codes = torch.empty(sizes[0], dtype=torch.uint8, device=dev)
-    sf = torch.zeros(max(sizes[1], 1), dtype=torch.uint8, device=dev) if f.kind == KIND_NVFP4 else None
+    sf = torch.zeros(max(sizes[1], 1), dtype=torch.uint8, device=dev) if f.kind != KIND_INT else None
     w_scale = torch.zeros(4, dtype=torch.float32, device=dev)
     ld = torch.zeros((max(rp, 1), M), dtype=torch.bfloat16, device=dev)
     ld32 = torch.zeros((max(rp, 1), M), dtype=torch.float32, device=dev)
@@ -282,7 +284,7 @@ def svdq_quantize_residual(R: torch.Tensor, fmt="int4"):
     M, N = R.shape
     sizes = weight_buffer_sizes(M, N, 0, f)
     codes = torch.empty(sizes[0], dtype=torch.uint8, device=R.device)
-    sf = torch.empty(max(sizes[1], 1), dtype=torch.uint8, device=R.device) if f.kind == KIND_NVFP4 else None
+    sf = torch.empty(max(sizes[1], 1), dtype=torch.uint8, device=R.device) if f.kind != KIND_INT else None
     w_scale = torch.zeros(1, dtype=torch.float32, device=R.device)
     wsz = c_sz()
     _check(lib.svdq_quantize_residual_workspace_size(M, N, f, ctypes.byref(wsz)), "workspace")
@@ -303,7 +305,8 @@ def _act_buffers(B, M, f, rp, dev):
         sf = None
     else:
         codes = torch.empty((B, M // 2), dtype=torch.uint8, device=dev)
-        sf = torch.empty(max(((B + 127) // 128 * 128) * ((M // 16 + 3) // 4 * 4), 1),
+        block = 32 if f.kind == KIND_MXFP4 else 16
+        sf = torch.empty(max(((B + 127) // 128 * 128) * ((M // block + 3) // 4 * 4), 1),
                          dtype=torch.uint8, device=dev)
     act_scale = torch.zeros(1, dtype=torch.float32, device=dev)
     down = torch.empty((B, 2 * rp), dtype=torch.bfloat16, device=dev) if rp else None
@@ -344,7 +347,8 @@ def svdq_quantize_act(x: torch.Tensor, scale: torch.Tensor, fmt="int4", ld: Opti
 
     ld is the [rank_pad, M] down factor (bf16 for bf16 x, fp32 for fp32 x); down is
     bf16 [B, 2 * rank_pad] (hi | lo). For NVFP4, down is multiplied by gs_x (and by
-    w_global_scale when given), the units the NVFP4 GEMM accumulates in.
+    w_global_scale when given), the units the NVFP4 GEMM accumulates in. MXFP4 has
+    no global scales: act_scale is 1 and down is unscaled.
     """
     _require_cuda(x, scale)
     f = parse_fmt(fmt)

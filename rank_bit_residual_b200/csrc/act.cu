@@ -3,7 +3,9 @@
 //
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula items 1
 // and 3: X_hat = x / scale is quantised per tensor (INT grid, or NVFP4 blocks
-// for the variant of "flashinfer.gemm.svdquant_linear" step 1), and the
+// for the variant of "flashinfer.gemm.svdquant_linear" step 1, or MXFP4 blocks
+// of 32 with power-of-two scales for the "mxfp4" per-block format of the
+// SVDQuant parameter configuration guide), and the
 // low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) from the same
 // read of x.
 //
@@ -365,15 +367,16 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
     m = red[0];
     for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
     const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
-    float s = 0.0f, u = 0.0f, gs_x = 1.0f;
+    const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
+    float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
     if (nv) {
       gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
-    } else {
+    } else if (!mx) {
       s = __fdiv_rn(m, static_cast<float>(a.qmax));
       u = s > 0.0f ? __frcp_rn(s) : 0.0f;
     }
-    if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv ? gs_x : s;
-    const int kb = a.M / 16;
+    if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv || mx ? gs_x : s;
+    const int kb = a.M / (mx ? 32 : 16);   // fp4 scale blocks per row
     const int64_t kbp = (kb + 3) / 4 * 4;
 
     for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
       __syncthreads();
       const int rows = min(kRows, a.B - m0);
       const int ncols = min(n * kTileK, a.M - k_lo * kTileK);   // a multiple of 32
-      if (!nv) {
+      if (!nv && !mx) {
         // a warp writes 256 consecutive codes of a row (8 per lane, one 256-byte
         // store) for kR rows, whose loads are all issued first
         constexpr int kR = sizeof(TIn) == 2 ? 8 : 4;
@@ -416,8 +419,9 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
           }
         }
       } else {
-        // half a warp = 256 consecutive elements of one row (one 16-element block
-        // per lane), kR rows per half warp with all loads issued first
+        // half a warp = 256 consecutive elements of one row (16 elements per
+        // lane: one NVFP4 block, half an MXFP4 block whose other half is the
+        // neighbouring lane's), kR rows per half warp with all loads issued first
         constexpr int kR = sizeof(TIn) == 2 ? 4 : 2;
         constexpr int kHalves = 2 * kWorkWarps;
         const int hw = 2 * warp + (lane >> 4);
@@ -446,16 +450,31 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
                 xs[j] = __fmul_rn(xs[j], rcp[cl + j]);
                 amax = fmaxf(amax, fabsf(xs[j]));
               }
-              const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
-              const float d = ue4m3_to_f32(sfb);
-              const float enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
               const int64_t row = m0 + r;
               const int64_t col = col0 + cl;
+              uint8_t sfb;
+              float enc;
+              if (mx) {
+                // lanes 2i and 2i + 1 hold one 32-element block; both take the
+                // same exits above (ncols is a multiple of 32), so the pair is
+                // converged here
+                amax = fmaxf(amax, __shfl_xor_sync(3u << (lane & 30), amax, 1));
+                const int X = mx_block_exponent(amax);
+                sfb = static_cast<uint8_t>(X + 127);
+                enc = mx_inv_scale(X);
+              } else {
+                sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+                const float d = ue4m3_to_f32(sfb);
+                enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
               *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
                   make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
-              a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+              if (!mx)
+                a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+              else if ((lane & 1) == 0)
+                a.sf[sf_swizzle_offset(row, col / 32, kbp)] = sfb;
             }
           }
         }
@@ -480,8 +499,8 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
         }
       }
     }
-    // NVFP4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
-    if (nv) {
+    // fp4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
+    if (nv || mx) {
       const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
       const int64_t pad_cols = kbp - kb;
       const int64_t n_pad = (rows_p - a.B) * kbp + static_cast<int64_t>(a.B) * pad_cols;

@@ -3,7 +3,8 @@
 // Same result as the large-batch kernel in act.cu ("SVDQuant Smoothing,
 // Low-rank and Residual Quantization", Formula items 1 and 3; steps 1-2 of
 // "flashinfer.gemm.svdquant_linear"): X_hat = x / scale quantised per tensor
-// (INT) or per 16-element block (NVFP4), and the down-projection x ld^T as
+// (INT), per 16-element block (NVFP4) or per 32-element block with a
+// power-of-two scale (MXFP4), and the down-projection x ld^T as
 // bf16 hi | lo. At decode sizes the whole of x is a few hundred KB, so the work
 // is latency-bound: the columns of x are spread over one CTA per SM, and the
 // pass is two plain kernels whose boundary replaces a grid barrier (a barrier
@@ -264,9 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
   for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w]);
 
   const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
-  float u = 0.0f, gs_x = 1.0f;
-  if (nv) {
-    gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
+  const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
+  float u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
+  if (nv || mx) {
+    if (nv) gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
     if (g == 0 && tid == 0) *a.act_scale = gs_x;
   } else {
     const float s = __fdiv_rn(m, static_cast<float>(a.qmax));
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
   }
 
   constexpr int kPer16 = 16 / kEsz;   // elements per 16 bytes
-  if (!nv) {
+  if (!nv && !mx) {
     // 8 codes per item: one 8-byte store
     const int per_row = ncols / 8;
     for (int i = tid; i < B * per_row; i += kThreads) {
@@ -288,6 +290,31 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
       for (int j = 0; j < 8; ++j) ck[j] = __fmul_rn(rcp[c8 + j], u);
       *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(r) * a.M + c0 + c8) =
           int_codes8(v, ck);
+    }
+  } else if (mx) {
+    // one 32-element block per item: a scale byte and 16 code bytes
+    const int per_row = ncols / 32;
+    const int64_t kbp = (a.M / 32 + 3) / 4 * 4;
+    for (int i = tid; i < B * per_row; i += kThreads) {
+      const int r = i / per_row, c32 = (i - r * per_row) * 32;
+      float v[32];
+#pragma unroll
+      for (int h = 0; h < 32 / kPer16; ++h)
+        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c32 + h * kPer16) * kEsz), v + h * kPer16);
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        v[j] = __fmul_rn(v[j], rcp[c32 + j]);
+        amax = fmaxf(amax, fabsf(v[j]));
+      }
+      const int X = mx_block_exponent(amax);
+      const float enc = mx_inv_scale(X);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], enc);
+      const int64_t col = c0 + c32;
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(r) * (a.M / 2) + col / 2) =
+          make_uint4(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8), f32x8_to_e2m1(v + 16), f32x8_to_e2m1(v + 24));
+      a.sf[sf_swizzle_offset(r, col / 32, kbp)] = static_cast<uint8_t>(X + 127);
     }
   } else {
     // one 16-element block per item: a scale byte and 8 code bytes
@@ -315,9 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
           make_uint2(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8));
       a.sf[sf_swizzle_offset(r, col / 16, kbp)] = sfb;
     }
+  }
+  if (nv || mx) {
     // zero the scale padding: rows B..127 of every scale column, and the
-    // columns past M / 16 (up to a multiple of 4) of rows < B
-    const int64_t kb = a.M / 16;
+    // columns past M / block (up to a multiple of 4) of rows < B
+    const int64_t kb = a.M / (mx ? 32 : 16);
+    const int64_t kbp = (kb + 3) / 4 * 4;
     const int64_t pad_cols = kbp - kb;
     const int64_t n_pad = (128 - B) * kbp + static_cast<int64_t>(B) * pad_cols;
     for (int64_t i = static_cast<int64_t>(g) * kThreads + tid; i < n_pad; i += static_cast<int64_t>(a.G) * kThreads) {

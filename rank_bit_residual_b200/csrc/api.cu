@@ -104,7 +104,7 @@ __global__ void wait_selftest_kernel(long long limit_ns, unsigned* status) {
 
 svdq_status check_fmt(svdq_fmt fmt) {
   if (fmt.kind == SVDQ_KIND_INT) return (fmt.bits >= 2 && fmt.bits <= 8) ? SVDQ_OK : SVDQ_EINVAL;
-  if (fmt.kind == SVDQ_KIND_NVFP4) return fmt.bits == 4 ? SVDQ_OK : SVDQ_EINVAL;
+  if (fmt.kind == SVDQ_KIND_NVFP4 || fmt.kind == SVDQ_KIND_MXFP4) return fmt.bits == 4 ? SVDQ_OK : SVDQ_EINVAL;
   return SVDQ_EINVAL;
 }
 
@@ -131,9 +131,12 @@ size_t act_codes_bytes(int64_t B, int64_t M, svdq_fmt fmt) {
   return fmt.kind == SVDQ_KIND_INT ? static_cast<size_t>(B * M) : static_cast<size_t>(B * M / 2);
 }
 
-size_t act_sf_bytes(int64_t B, int64_t M, svdq_fmt fmt) {
-  if (fmt.kind != SVDQ_KIND_NVFP4) return 0;
-  return static_cast<size_t>(round_up(B, 128) * round_up(M / 16, 4));
+// Block-scale bytes of a [rows, M] fp4 operand: the 128x4 layout over
+// [rows, M / block], block 16 (NVFP4) or 32 (MXFP4); 0 for INT.
+size_t fp4_sf_bytes(int64_t rows, int64_t M, svdq_fmt fmt) {
+  if (fmt.kind == SVDQ_KIND_INT) return 0;
+  const int64_t block = fmt.kind == SVDQ_KIND_MXFP4 ? 32 : 16;
+  return static_cast<size_t>(round_up(rows, 128) * round_up(M / block, 4));
 }
 
 svdq_status check_weight(const svdq_weight* w) {
@@ -142,7 +145,7 @@ svdq_status check_weight(const svdq_weight* w) {
   if (s != SVDQ_OK) return s;
   if (w->rank_pad != rank_pad_of(w->rank)) return SVDQ_EINVAL;
   if (!w->codes || !w->w_scale || !w->scale) return SVDQ_EINVAL;
-  if (w->fmt.kind == SVDQ_KIND_NVFP4 && !w->sf) return SVDQ_EINVAL;
+  if (w->fmt.kind != SVDQ_KIND_INT && !w->sf) return SVDQ_EINVAL;
   if (w->rank > 0 && (!w->ld || !w->lu)) return SVDQ_EINVAL;
   if (w->codes4 && (w->fmt.kind != SVDQ_KIND_INT || w->fmt.bits > 4)) return SVDQ_EINVAL;
   if (!aligned16(w->codes) || !aligned16(w->scale) || (w->ld && !aligned16(w->ld)) ||
@@ -179,7 +182,7 @@ LinearCarve carve_linear(const svdq_weight* w, int64_t B, void* ws, size_t ws_by
   Carver cv(ws, ws_bytes);
   LinearCarve c{};
   c.codes = cv.take(act_codes_bytes(B, w->M, w->fmt));
-  c.sf = cv.take(act_sf_bytes(B, w->M, w->fmt));
+  c.sf = cv.take(fp4_sf_bytes(B, w->M, w->fmt));
   c.act_scale = static_cast<float*>(cv.take(16));
   c.down = cv.take(static_cast<size_t>(B) * 2 * w->rank_pad * 2);
   c.act_scratch = cv.take(act_scratch_bytes(p));
@@ -218,7 +221,7 @@ svdq_status svdq_weight_buffer_sizes(int64_t M, int64_t N, int32_t rank, svdq_fm
   if (s != SVDQ_OK) return s;
   const int64_t rp = rank_pad_of(rank);
   sizes[0] = fmt.kind == SVDQ_KIND_INT ? static_cast<size_t>(N * M) : static_cast<size_t>(N * M / 2);
-  sizes[1] = fmt.kind == SVDQ_KIND_NVFP4 ? static_cast<size_t>(round_up(N, 128) * round_up(M / 16, 4)) : 0;
+  sizes[1] = fp4_sf_bytes(N, M, fmt);
   sizes[2] = sizeof(float);
   sizes[3] = static_cast<size_t>(rp * M * 2);
   sizes[4] = static_cast<size_t>(rp * M * 4);
@@ -252,7 +255,7 @@ svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N
   if (!W || !scale || !out || ldW < N || (w_dtype != SVDQ_BF16 && w_dtype != SVDQ_F32))
     return SVDQ_EINVAL;
   if (!aligned16(scale)) return SVDQ_EUNSUPPORTED;
-  if (!out->codes || !out->w_scale || (fmt.kind == SVDQ_KIND_NVFP4 && !out->sf) ||
+  if (!out->codes || !out->w_scale || (fmt.kind != SVDQ_KIND_INT && !out->sf) ||
       (rank > 0 && (!out->ld || !out->lu)))
     return SVDQ_EINVAL;
   if (!workspace || workspace_bytes < prepare_scratch_bytes(M, N, rank, oversample))
@@ -276,7 +279,7 @@ svdq_status svdq_quantize_residual(const float* R, int64_t M, int64_t N, int64_t
                                    svdq_stream_t stream) {
   const svdq_status s = check_shape(M, N, 0, fmt);
   if (s != SVDQ_OK) return s;
-  if (!R || ldR < N || !codes || !w_scale || (fmt.kind == SVDQ_KIND_NVFP4 && !sf))
+  if (!R || ldR < N || !codes || !w_scale || (fmt.kind != SVDQ_KIND_INT && !sf))
     return SVDQ_EINVAL;
   if (!workspace || workspace_bytes < residual_scratch_bytes(M, N)) return SVDQ_EWORKSPACE;
   return from_cuda(launch_quantize_residual(R, M, N, ldR, fmt, codes, sf, w_scale, workspace,
@@ -307,7 +310,7 @@ svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int6
   if (M % 32 != 0) return SVDQ_EUNSUPPORTED;
   if (!aligned16(scale)) return SVDQ_EUNSUPPORTED;
   if (B == 0) return SVDQ_OK;
-  if (!codes || !act_scale || (fmt.kind == SVDQ_KIND_NVFP4 && !sf)) return SVDQ_EINVAL;
+  if (!codes || !act_scale || (fmt.kind != SVDQ_KIND_INT && !sf)) return SVDQ_EINVAL;
   if (ld && rank_pad > 0 && (!down || !aligned16(ld))) return SVDQ_EINVAL;
   const ActPlan p = plan_act(B, M, rank_pad, x_dtype);
   if (!workspace || workspace_bytes < act_scratch_bytes(p)) return SVDQ_EWORKSPACE;
@@ -360,7 +363,7 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
     e = launch_gemm_int(w, static_cast<const int8_t*>(c.codes), c.act_scale,
                         w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, false, true, st, &bad);
   } else {
-    e = launch_gemm_nvfp4(w, static_cast<const uint8_t*>(c.codes),
+    e = launch_gemm_fp4(w, static_cast<const uint8_t*>(c.codes),
                           static_cast<const uint8_t*>(c.sf), c.act_scale,
                           w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, true, st, &bad);
   }
@@ -377,7 +380,7 @@ svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, co
   if (B < 0 || (y_dtype != SVDQ_BF16 && y_dtype != SVDQ_F32)) return SVDQ_EINVAL;
   if (B == 0) return SVDQ_OK;
   if (!act_codes || !act_scale || !y || ldy < w->N) return SVDQ_EINVAL;
-  if (w->fmt.kind == SVDQ_KIND_NVFP4 && !act_sf) return SVDQ_EINVAL;
+  if (w->fmt.kind != SVDQ_KIND_INT && !act_sf) return SVDQ_EINVAL;
   if (w->rank > 0 && !down) return SVDQ_EINVAL;
   if (!aligned16(act_codes) || (down && !aligned16(down)) || (bias && !aligned16(bias)))
     return SVDQ_EUNSUPPORTED;
@@ -388,7 +391,7 @@ svdq_status svdq_residual_linear(const svdq_weight* w, const void* act_codes, co
     e = launch_gemm_int(w, static_cast<const int8_t*>(act_codes), act_scale,
                         w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, false, st, &bad);
   else
-    e = launch_gemm_nvfp4(w, static_cast<const uint8_t*>(act_codes),
+    e = launch_gemm_fp4(w, static_cast<const uint8_t*>(act_codes),
                           static_cast<const uint8_t*>(act_sf), act_scale,
                           w->rank > 0 ? down : nullptr, B, bias, y, y_dtype, ldy, false, st, &bad);
   if (bad) return SVDQ_EUNSUPPORTED;

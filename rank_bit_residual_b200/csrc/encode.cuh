@@ -5,7 +5,9 @@
 // Formats ("flashinfer.gemm.svdquant_linear", Parameters: packed e2m1 residual,
 // ue4m3 scales in the 128x4 layout): e2m1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6},
 // ue4m3 = e4m3 (bias 7, max 448) restricted to >= 0; the INT grid of "SVDQuant
-// Smoothing, Low-rank and Residual Quantization" (Formula item 3).
+// Smoothing, Low-rank and Residual Quantization" (Formula item 3); MXFP4 block
+// exponents (the "mxfp4" per-block format of the SVDQuant parameter
+// configuration guide).
 #pragma once
 
 #include <cstdint>
@@ -41,6 +43,20 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(const float* v) {
   const uint32_t mag = out & 0x77777777u;
   const uint32_t nz = (mag + 0x77777777u) & 0x88888888u;
   return out & (0x77777777u | nz);
+}
+
+// MXFP4 block exponent (OCP microscaling, the "mxfp4" per-block MinMax format):
+// X = floor(log2(amax)) - 2 (2 = the exponent of e2m1's largest value 6),
+// clamped to [-127, 127]; a zero (or subnormal) amax gives -127. The E8M0 scale
+// byte is X + 127 and the block's values are encoded as e2m1(v * 2^-X).
+__device__ __forceinline__ int mx_block_exponent(float amax) {
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);   // amax >= 0
+  return e == 0 ? -127 : max(-127, e - 129);
+}
+
+// 2^-X as an fp32 (exact: -X lies in [-125, 127]).
+__device__ __forceinline__ float mx_inv_scale(int X) {
+  return __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
 }
 
 // Byte offset of scale (row, col) in the 128x4 layout: 128-row x 4-column atoms

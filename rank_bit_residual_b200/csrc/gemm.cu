@@ -58,7 +58,7 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
   args.vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15) == 0 && (ldy * elem) % 16 == 0) ? 1 : 0;
   args.sfa = act_sf;
   args.sfb = static_cast<const uint8_t*>(w->sf);
-  args.katoms = static_cast<int>(ceil_div(M, 64));
+  args.katoms = static_cast<int>(kKind == kKindMxfp4 ? ceil_div(M, 128) : ceil_div(M, 64));
   args.status = device_status_word();
   const int out = raw_i32 ? kOutI32 : (ydt == SVDQ_F32 ? kOutF32 : kOutBF16);
   cudaError_t err = cudaSuccess;
@@ -80,15 +80,18 @@ cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const
                                stream, bad_args);
 }
 
-cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
-                              const uint8_t* act_sf, const float* gs_x, const void* down2,
-                              int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                              int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args) {
+cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,
+                            const uint8_t* act_sf, const float* gs_x, const void* down2,
+                            int64_t B, const void* bias, void* y, svdq_dtype ydt,
+                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args) {
   if (!act_sf || !w->sf || (reinterpret_cast<uintptr_t>(act_sf) & 15) ||
       (reinterpret_cast<uintptr_t>(w->sf) & 15)) {
     *bad_args = true;
     return cudaSuccess;
   }
+  if (w->fmt.kind == SVDQ_KIND_MXFP4)
+    return launch_gemm<kKindMxfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false, pdl,
+                                   stream, bad_args);
   return launch_gemm<kKindNvfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false, pdl,
                                  stream, bad_args);
 }

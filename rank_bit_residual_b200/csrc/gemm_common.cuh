@@ -10,20 +10,22 @@
 
 namespace svdq {
 
-enum GemmKind { kKindInt = 0, kKindNvfp4 = 1 };
+// INT: kind::i8; NVFP4: e2m1 with ue4m3 scales per 16 elements and fp32 global
+// scales; MXFP4: e2m1 with E8M0 scales per 32 elements, global scales 1.
+enum GemmKind { kKindInt = 0, kKindNvfp4 = 1, kKindMxfp4 = 2 };
 enum GemmOut { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
 
 struct GemmArgs {
   int B, N, M, lr_steps;
-  const float* s_x;               // INT: s_x, NVFP4: gs_x
-  const float* s_w;               // INT: s_w, NVFP4: gs_w
+  const float* s_x;               // INT: s_x, fp4: gs_x (1 for MXFP4)
+  const float* s_w;               // INT: s_w, fp4: gs_w (1 for MXFP4)
   const __nv_bfloat16* bias;
   void* y;
   int64_t ldy;
   int vec_ok;
-  const uint8_t* sfa;             // NVFP4 activation scales (128x4 layout)
-  const uint8_t* sfb;             // NVFP4 weight scales (128x4 layout)
-  int katoms;                     // NVFP4: 64-element scale atoms per row tile = ceil(M / 64)
+  const uint8_t* sfa;             // fp4 activation scales (128x4 layout)
+  const uint8_t* sfb;             // fp4 weight scales (128x4 layout)
+  int katoms;                     // fp4: 4-scale atoms per row tile, ceil(M / 64) NVFP4, ceil(M / 128) MXFP4
   unsigned* status;
 };
 
@@ -36,7 +38,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 template <int kKind, int kOut>
 __device__ __forceinline__ float epilogue_alpha(const GemmArgs& args) {
   if (kOut == kOutI32) return 0.0f;
-  if (kKind == kKindNvfp4) return __fdiv_rn(1.0f, __fmul_rn(__ldg(args.s_x), __ldg(args.s_w)));
+  if (kKind != kKindInt) return __fdiv_rn(1.0f, __fmul_rn(__ldg(args.s_x), __ldg(args.s_w)));
   return __ldg(args.s_x) * __ldg(args.s_w);
 }
 
@@ -68,7 +70,7 @@ __device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], const uint3
                                           float alpha, bool sep_lr, float (&v)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    if (kKind == kKindNvfp4) {
+    if (kKind != kKindInt) {
       v[j] = alpha * __uint_as_float(acc[j]);
     } else {
       v[j] = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));

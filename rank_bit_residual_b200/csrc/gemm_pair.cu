@@ -2,8 +2,9 @@
 //
 // Same operator as gemm.cu ("SVDQuant Smoothing, Low-rank and Residual
 // Quantization", Formula item 3; step 3 of "flashinfer.gemm.svdquant_linear"):
-// Y = alpha * Q(X_hat) Q(R) + down . lu^T [+ bias], INT (kind::i8) or NVFP4
-// (kind::mxf4nvf4 with ue4m3 scales per 16 elements).
+// Y = alpha * Q(X_hat) Q(R) + down . lu^T [+ bias], INT (kind::i8), NVFP4
+// (kind::mxf4nvf4 with ue4m3 scales per 16 elements) or MXFP4 (kind::mxf4 with
+// E8M0 scales per 32 elements).
 //
 // A cluster of two CTAs computes one 256 x 256 output tile: CTA r holds rows
 // [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128) of the B
@@ -28,11 +29,15 @@
 // TMEM columns (512):
 //   INT    [0, 256) int32 residual | [256, 512) fp32 up-projection, which
 //          pass 1 overwrites in place with the combined result
-//   NVFP4  [0, 256) fp32 (both branches) | [256, 304) block scales |
+//   fp4    [0, 256) fp32 (both branches) | [256, 304) block scales |
 //          [384, 512) bf16 result of pass 1 (fp32 output: one direct pass)
-// NVFP4: each CTA's TMEM holds the scales of its 128 A rows (4 columns per
-// K = 64 step) and of all 256 B rows (8 columns), copied from its own shared
-// memory by the pair-wide tcgen05.cp the even CTA issues.
+// fp4: each CTA's TMEM holds the scales of its 128 A rows (4 columns per
+// 128 x 4 scale atom) and of all 256 B rows (8 columns), copied from its own
+// shared memory by the pair-wide tcgen05.cp the even CTA issues. An atom holds
+// four scales per row: one K = 64 MMA's worth for NVFP4 (16-element blocks),
+// two MMAs' for MXFP4 (32-element blocks; the MMA's scale-factor id picks the
+// byte pair), so a 256-element stage copies 4 atoms per row tile for NVFP4 and
+// 2 for MXFP4.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -52,19 +57,22 @@ constexpr int kHalf = 128;                        // rows of A and of B per CTA
 constexpr int kTileN = 256;
 constexpr int kABytes = kHalf * 128;
 constexpr int kBBytes = kHalf * 128;
-constexpr int kSfaBytes = 4 * 512;                // this CTA's A rows, 4 atoms
-constexpr int kSfbBytes = 2 * 4 * 512;            // both B row tiles, 4 atoms each
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfaCol = 256;
 constexpr uint32_t kSfbCol = 272;
-constexpr uint32_t kNvOutCol = 384;               // NVFP4 bf16 pass-1 result
+constexpr uint32_t kNvOutCol = 384;               // fp4 bf16 pass-1 result
 
 template <int kKind>
 struct PairCfg {
+  static constexpr bool kF4 = kKind != kKindInt;
   // INT: two 128-byte K blocks per stage (8 MMAs per barrier wait and commit)
-  static constexpr int kKb = kKind == kKindNvfp4 ? 1 : 2;
-  static constexpr int kStages = kKind == kKindNvfp4 ? 5 : 3;
-  static constexpr int kStageBytes = kKb * (kABytes + kBBytes) + (kKind == kKindNvfp4 ? kSfaBytes + kSfbBytes : 0);
+  static constexpr int kKb = kF4 ? 1 : 2;
+  // scale atoms per 128-row tile and stage (256 elements of K)
+  static constexpr int kSfAtoms = kKind == kKindNvfp4 ? 4 : (kKind == kKindMxfp4 ? 2 : 0);
+  static constexpr int kSfaBytes = kSfAtoms * 512;       // this CTA's A rows
+  static constexpr int kSfbBytes = 2 * kSfAtoms * 512;   // both B row tiles
+  static constexpr int kStages = kKind == kKindNvfp4 ? 5 : (kKind == kKindMxfp4 ? 6 : 3);
+  static constexpr int kStageBytes = kKb * (kABytes + kBBytes) + kSfaBytes + kSfbBytes;
 };
 
 // Whether the epilogue's stores overlap the next tile's MMAs.
@@ -81,6 +89,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                      const GemmArgs args) {
   constexpr int kStages = PairCfg<kKind>::kStages;
   constexpr int kStageBytes = PairCfg<kKind>::kStageBytes;
+  constexpr bool kF4 = PairCfg<kKind>::kF4;
+  constexpr int kSfAtoms = PairCfg<kKind>::kSfAtoms;
+  constexpr int kSfaBytes = PairCfg<kKind>::kSfaBytes;
+  constexpr int kSfbBytes = PairCfg<kKind>::kSfbBytes;
   constexpr bool kTwoPass = TwoPass<kKind, kOut>::value;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -105,7 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int tiles_n = (N + kTileN - 1) / kTileN;
   const int total = tiles_m * tiles_n;
   constexpr int kKb = PairCfg<kKind>::kKb;
-  constexpr int kStageK = kKind == kKindNvfp4 ? 256 : 128 * kKb;   // K elements per stage
+  constexpr int kStageK = kF4 ? 256 : 128 * kKb;   // K elements per stage
   const int ksteps = (M + kStageK - 1) / kStageK;
   const int steps_per_tile = ksteps + lr_steps;   // residual steps first
 
@@ -157,7 +169,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
             tma_load_2d_pair(st, &tm_da, fb, 64 * l, m0);
             tma_load_2d_pair(st + kABytes, &tm_lu, fb, 64 * l, n0);
-          } else if constexpr (kKind == kKindNvfp4) {
+          } else if constexpr (kF4) {
             if (rank == 0)
               mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
             tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
@@ -165,10 +177,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             // scale atoms: rows of 256 bytes, two rows per 512-byte atom
             uint8_t* sfa_s = st + kABytes + kBBytes;
             uint8_t* sfb_s = sfa_s + kSfaBytes;
-            const int a0 = 4 * j;
+            const int a0 = kSfAtoms * j;
             tma_load_2d_pair(sfa_s, &tm_sfa, fb, 0, 2 * ((m0 / 128) * args.katoms + a0));
             for (int rt = 0; rt < 2; ++rt)
-              tma_load_2d_pair(sfb_s + rt * 2048, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
+              tma_load_2d_pair(sfb_s + rt * kSfaBytes, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
           } else {
             // A blocks then B blocks, 128 bytes of K each
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kKb * (kABytes + kBBytes));
@@ -193,7 +205,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint32_t id_i8 = idesc_i8(2 * kHalf, kTileN);
       const uint32_t id_bf = idesc_bf16(2 * kHalf, kTileN);
       const uint32_t id_f4 = idesc_nvf4(2 * kHalf, kTileN);
-      const uint32_t lr_acc = kKind == kKindNvfp4 ? tmem : tmem + 256;
+      const uint32_t id_mx0 = idesc_mxf4(2 * kHalf, kTileN, 0), id_mx1 = idesc_mxf4(2 * kHalf, kTileN, 2);
+      const int kmma = (M + 63) / 64;   // fp4 K = 64 MMAs of the residual
+      const uint32_t lr_acc = kF4 ? tmem : tmem + 256;
       {
         // throwaway MMA: the first tcgen05.mma of a kernel takes microseconds
         // longer than the rest; issued now, that start-up overlaps the first
@@ -201,6 +215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint64_t d0 = smem_desc_sw128(smem_u32(smem));
         if constexpr (kKind == kKindNvfp4)
           mma_nvf4_pair(tmem, d0, d0, id_f4, 0u, tmem + kSfaCol, tmem + kSfbCol);
+        else if constexpr (kKind == kKindMxfp4)
+          mma_mxf4_pair(tmem, d0, d0, id_mx0, 0u, tmem + kSfaCol, tmem + kSfbCol);
         else
           mma_i8_pair(tmem, d0, d0, id_i8, 0u);
       }
@@ -229,20 +245,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_f16_pair(lr_acc, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_bf,
-                           (kKind == kKindNvfp4 || l > 0 || kk > 0) ? 1u : 0u);
-          } else if constexpr (kKind == kKindNvfp4) {
-            const int na = min(4, args.katoms - 4 * j);
+                           (kF4 || l > 0 || kk > 0) ? 1u : 0u);
+          } else if constexpr (kF4) {
+            const int na = min(kSfAtoms, args.katoms - kSfAtoms * j);
             const uint32_t sfa_s = b0 + kBBytes;
             const uint32_t sfb_s = sfa_s + kSfaBytes;
             for (int kk = 0; kk < na; ++kk) {
               tmem_cp_32x128b_warpx4_pair(tmem + kSfaCol + 4 * kk, smem_desc_plain(sfa_s + 512 * kk));
               for (int rt = 0; rt < 2; ++rt)
                 tmem_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * kk + 4 * rt,
-                                            smem_desc_plain(sfb_s + 2048 * rt + 512 * kk));
+                                            smem_desc_plain(sfb_s + kSfaBytes * rt + 512 * kk));
             }
-            for (int kk = 0; kk < na; ++kk)
-              mma_nvf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
-                            (j > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
+            if constexpr (kKind == kKindNvfp4) {
+              for (int kk = 0; kk < na; ++kk)
+                mma_nvf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
+                              (j > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
+            } else {
+              // MMA kk: atom kk / 2, scale bytes 2 (kk % 2) and up of each row's four
+              const int nm = min(4, kmma - 4 * j);
+              for (int kk = 0; kk < nm; ++kk)
+                mma_mxf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), ((kk & 1) ? id_mx1 : id_mx0),
+                              (j > 0 || kk > 0) ? 1u : 0u, sf_taddr(tmem + kSfaCol + 4 * (kk >> 1), kk),
+                              sf_taddr(tmem + kSfbCol + 8 * (kk >> 1), kk));
+            }
           } else {
             const uint32_t bb = a0 + kKb * kABytes;
 #pragma unroll
@@ -298,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // the warp's four accumulator chunks go to registers first, so the
         // accumulator is handed back to the next tile's MMAs before any
         // arithmetic; the result of chunk c then goes to dst(c): INT in place
-        // over its own low-rank columns, NVFP4 (bf16) to the free columns
+        // over its own low-rank columns, fp4 (bf16) to the free columns
         // from 384
         auto dst = [](int c) -> uint32_t {
           return kKind == kKindInt ? 256u + 32u * c : kNvOutCol + 16u * c;
@@ -368,7 +393,7 @@ bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_c
   *err = cudaSuccess;
   const int64_t M = args.M, N = args.N, B = args.B;
   const int rp = w->rank_pad;
-  const int64_t row_bytes = kind == kKindNvfp4 ? M / 2 : M;
+  const int64_t row_bytes = kind != kKindInt ? M / 2 : M;
   CUtensorMap maps[6];
   bool ok =
       make_tmap_2d(&maps[0], act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, B, row_bytes, 128, kHalf, true) &&
@@ -380,11 +405,13 @@ bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_c
     maps[2] = maps[0];
     maps[3] = maps[1];
   }
-  if (ok && kind == kKindNvfp4) {
+  if (ok && kind != kKindInt) {
+    // one box = the scale atoms of one stage (two 256-byte rows per atom)
+    const int box = kind == kKindMxfp4 ? 2 * PairCfg<kKindMxfp4>::kSfAtoms : 2 * PairCfg<kKindNvfp4>::kSfAtoms;
     const int64_t rows_a = ceil_div(B, 128) * args.katoms * 2;
     const int64_t rows_b = ceil_div(N, 128) * args.katoms * 2;
-    ok = make_tmap_2d(&maps[4], args.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_a, 256, 256, 8, false) &&
-         make_tmap_2d(&maps[5], args.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_b, 256, 256, 8, false);
+    ok = make_tmap_2d(&maps[4], args.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_a, 256, 256, box, false) &&
+         make_tmap_2d(&maps[5], args.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, rows_b, 256, 256, box, false);
   } else {
     maps[4] = maps[0];
     maps[5] = maps[1];
@@ -396,6 +423,9 @@ bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_c
     if (out == kOutI32) *err = launch_pair_one<kKindInt, kOutI32>(maps, args, grid, stream);
     else if (out == kOutF32) *err = launch_pair_one<kKindInt, kOutF32>(maps, args, grid, stream);
     else *err = launch_pair_one<kKindInt, kOutBF16>(maps, args, grid, stream);
+  } else if (kind == kKindMxfp4) {
+    if (out == kOutF32) *err = launch_pair_one<kKindMxfp4, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindMxfp4, kOutBF16>(maps, args, grid, stream);
   } else {
     if (out == kOutF32) *err = launch_pair_one<kKindNvfp4, kOutF32>(maps, args, grid, stream);
     else *err = launch_pair_one<kKindNvfp4, kOutBF16>(maps, args, grid, stream);

@@ -26,10 +26,11 @@
 //                       memory by the epilogue warps                 kind::i8
 //   NVFP4               e2m1 tiles by TMA, ue4m3 scales by bulk copy
 //                       then tcgen05.cp to TMEM                      kind::mxf4nvf4
+//   MXFP4               the same with E8M0 scales per 32 elements    kind::mxf4
 // Low-rank branch: lu (weight side) x down hi|lo (batch side), kind::f16, in
 // 64-wide K boxes spread over the cluster's CTAs; INT keeps it in its own fp32
-// accumulator, NVFP4 adds it to the residual accumulator (down is pre-scaled
-// by gs_x gs_w).
+// accumulator, fp4 adds it to the residual accumulator (down is pre-scaled
+// by gs_x gs_w, which MXFP4 does not have: 1).
 //
 // Warps: 0 weight loads, 1 activation loads, 2 TMEM + MMA issue,
 //        3-6 widening of packed codes, then the epilogue (TMEM lane quarter w % 4).
@@ -52,14 +53,19 @@ constexpr int kWarpW = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi0 = 3;
 constexpr int kMaxRing = 8;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kLrCol = 128;                      // INT: low-rank fp32 accumulator
-constexpr uint32_t kSfaCol = 128, kSfbCol = 144;      // NVFP4: scale factors (4 columns per MMA)
+constexpr uint32_t kSfaCol = 128, kSfbCol = 144;      // fp4: scale factors (4 columns per 128x4 atom)
 constexpr int kATile = 16384;                         // 128 rows x 128 bytes
 constexpr int kPSlot = 8192;                          // 128 rows x 64 packed bytes
-constexpr int kSfBytes = 2048;                        // 4 scale atoms of 512 bytes
+constexpr int kSfBytes = 2048;                        // up to 4 scale atoms of 512 bytes
 constexpr size_t kSmemBudget = 200 * 1024;
 constexpr size_t kMinSmem = 120 * 1024;
 
-enum SkinnyFmt { kFmtInt8 = 0, kFmtInt4 = 1, kFmtNvfp4 = 2 };
+enum SkinnyFmt { kFmtInt8 = 0, kFmtInt4 = 1, kFmtNvfp4 = 2, kFmtMxfp4 = 3 };
+
+constexpr bool fmt_is_f4(int f) { return f == kFmtNvfp4 || f == kFmtMxfp4; }
+// 128x4 scale atoms per 128-row tile and 256-element K step: four scales per
+// row cover 64 elements of NVFP4 (16-element blocks), 128 of MXFP4
+constexpr int sf_atoms_per_step(int f) { return f == kFmtNvfp4 ? 4 : (f == kFmtMxfp4 ? 2 : 0); }
 
 struct SkinnyArgs {
   int B, Bp, N, M, S, kst, lr_boxes, sh;
@@ -71,8 +77,8 @@ struct SkinnyArgs {
   void* y;
   int64_t ldy;
   int vec_ok;
-  const uint8_t* sfw;   // NVFP4 weight scales, 128x4 layout
-  const uint8_t* sfx;   // NVFP4 activation scales, 128x4 layout
+  const uint8_t* sfw;   // fp4 weight scales, 128x4 layout
+  const uint8_t* sfx;   // fp4 activation scales, 128x4 layout
   unsigned* status;
 };
 
@@ -92,11 +98,11 @@ __device__ __forceinline__ void widen_int4(const uint4 v, uint32_t (&o)[8]) {
 }
 
 // Dequantisation factor of the residual accumulator (s_x s_w for INT,
-// 1 / (gs_x gs_w) for NVFP4; unused for the raw int32 product).
+// 1 / (gs_x gs_w) for fp4, 1 for MXFP4; unused for the raw int32 product).
 template <int kFmt, int kOut>
 __device__ __forceinline__ float skinny_alpha(const SkinnyArgs& a) {
   if (kOut == kOutI32) return 0.0f;
-  if (kFmt == kFmtNvfp4) return __fdiv_rn(1.0f, __fmul_rn(__ldg(a.s_x), __ldg(a.s_w)));
+  if (fmt_is_f4(kFmt)) return __fdiv_rn(1.0f, __fmul_rn(__ldg(a.s_x), __ldg(a.s_w)));
   return __ldg(a.s_x) * __ldg(a.s_w);
 }
 
@@ -207,11 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i >= a.dr) ok = ok && mbar_wait(&empty[s], ((i / a.dr) - 1) & 1, status, &abort_sh);
           if (!ok) break;
           uint8_t* dst = ring_a + static_cast<size_t>(s) * a.a_slot;
-          if constexpr (kFmt == kFmtNvfp4) {
-            const int na = min(4, a.katoms - 4 * k);
+          if constexpr (fmt_is_f4(kFmt)) {
+            constexpr int kAt = sf_atoms_per_step(kFmt);
+            const int na = min(kAt, a.katoms - kAt * k);
             mbar_arrive_expect_tx(&full[s], kATile + na * 512);
             tma_load_2d(dst, &tm_w, &full[s], 128 * k, n0);
-            bulk_load(dst + kATile, a.sfw + (static_cast<int64_t>(n0 / 128) * a.katoms + 4 * k) * 512, na * 512,
+            bulk_load(dst + kATile, a.sfw + (static_cast<int64_t>(n0 / 128) * a.katoms + kAt * k) * 512, na * 512,
                       &full[s]);
           } else {
             mbar_arrive_expect_tx(&full[s], kATile);
@@ -248,11 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, &tm_dn, &full[s], 64 * (rank + i * S), 0);
         } else {
           const int k = k_lo + (i - nlr);
-          if constexpr (kFmt == kFmtNvfp4) {
-            const int na = min(4, a.katoms - 4 * k);
+          if constexpr (fmt_is_f4(kFmt)) {
+            constexpr int kAt = sf_atoms_per_step(kFmt);
+            const int na = min(kAt, a.katoms - kAt * k);
             mbar_arrive_expect_tx(&full[s], xbytes + na * 512);
             tma_load_2d(dst, &tm_x, &full[s], 128 * k, 0);
-            bulk_load(dst + xbytes, a.sfx + static_cast<int64_t>(4 * k) * 512, na * 512, &full[s]);
+            bulk_load(dst + xbytes, a.sfx + static_cast<int64_t>(kAt * k) * 512, na * 512, &full[s]);
           } else {
             mbar_arrive_expect_tx(&full[s], xbytes);
             tma_load_2d(dst, &tm_x, &full[s], 128 * k, 0);
@@ -271,7 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_i8 = idesc_i8(kTileN, a.Bp);
       const uint32_t id_bf = idesc_bf16(kTileN, a.Bp);
       const uint32_t id_f4 = idesc_nvf4(kTileN, a.Bp);
-      const uint32_t lr_acc = kFmt == kFmtNvfp4 ? tmem : tmem + kLrCol;
+      const uint32_t id_mx0 = idesc_mxf4(kTileN, a.Bp, 0), id_mx1 = idesc_mxf4(kTileN, a.Bp, 2);
+      const int kmma = (a.M + 63) / 64;   // fp4 K = 64 MMAs of the residual
+      const uint32_t lr_acc = fmt_is_f4(kFmt) ? tmem : tmem + kLrCol;
       {
         // throwaway MMA: the first tcgen05.mma of a kernel completes microseconds
         // after the rest; issued now it overlaps the first loads (the first real
@@ -279,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t d0 = smem_desc_sw128(smem_u32(smem));
         if constexpr (kFmt == kFmtNvfp4)
           mma_nvf4(tmem, d0, d0, id_f4, 0u, tmem + kSfaCol, tmem + kSfbCol);
+        else if constexpr (kFmt == kFmtMxfp4)
+          mma_mxf4(tmem, d0, d0, id_mx0, 0u, tmem + kSfaCol, tmem + kSfbCol);
         else
           mma_i8(tmem, d0, d0, id_i8, 0u);
       }
@@ -297,9 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (i > 0 || kk > 0) ? 1u : 0u);
         } else {
           const int r = i - nlr;
-          if constexpr (kFmt == kFmtNvfp4) {
+          if constexpr (fmt_is_f4(kFmt)) {
+            constexpr int kAt = sf_atoms_per_step(kFmt);
             const int k = k_lo + r;
-            const int na = min(4, a.katoms - 4 * k);
+            const int na = min(kAt, a.katoms - kAt * k);
             const uint32_t sfa_s = a0 + kATile;
             const uint32_t sfb_s = b0 + a.Bp * 128;
             // tcgen05.cp and tcgen05.mma from one thread execute in order, so
@@ -308,9 +321,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * kk, smem_desc_plain(sfa_s + 512 * kk));
               tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4 * kk, smem_desc_plain(sfb_s + 512 * kk));
             }
-            for (int kk = 0; kk < na; ++kk)
-              mma_nvf4(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
-                       (i > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 4 * kk);
+            if constexpr (kFmt == kFmtNvfp4) {
+              for (int kk = 0; kk < na; ++kk)
+                mma_nvf4(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
+                         (i > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 4 * kk);
+            } else {
+              // MMA kk: atom kk / 2, scale bytes 2 (kk % 2) and up of each row's four
+              const int nm = min(4, kmma - 4 * k);
+              for (int kk = 0; kk < nm; ++kk)
+                mma_mxf4(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), ((kk & 1) ? id_mx1 : id_mx0),
+                         (i > 0 || kk > 0) ? 1u : 0u, sf_taddr(tmem + kSfaCol + 4 * (kk >> 1), kk),
+                         sf_taddr(tmem + kSfbCol + 4 * (kk >> 1), kk));
+            }
           } else {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -384,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // shared-window stores (the pointer's origin is not visible to the compiler)
       const uint32_t dst_s = smem_u32(stg + static_cast<size_t>(p) * slot_words + nl);
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      const bool lr_here = kFmt != kFmtNvfp4 && kOut != kOutI32 && nlr > 0;
+      const bool lr_here = !fmt_is_f4(kFmt) && kOut != kOutI32 && nlr > 0;
       for (int c0 = 0; c0 < a.B; c0 += 32) {
         uint32_t acc[32], up[32];
         __syncwarp();
@@ -402,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) {
           if (j >= cnt) break;
           uint32_t v = acc[j];
-          if (kFmt != kFmtNvfp4 && kOut != kOutI32) {
+          if (!fmt_is_f4(kFmt) && kOut != kOutI32) {
             float f = alpha * static_cast<float>(static_cast<int32_t>(acc[j]));
             if (lr_here) f += __uint_as_float(up[j]);
             v = __float_as_uint(f);
@@ -433,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nq = cnt / 4;
     const int nbase = n0 + rank * a.sh;
     pdl_wait();   // returns at once: the epilogue warps waited before the barriers
-    const float alpha_f4 = kFmt == kFmtNvfp4 ? skinny_alpha<kFmt, kOut>(a) : 1.0f;
+    const float alpha_f4 = fmt_is_f4(kFmt) ? skinny_alpha<kFmt, kOut>(a) : 1.0f;
     for (int it = threadIdx.x; it < a.B * nq; it += kThreads) {
       const int b = it / nq, nl = (it - b * nq) * 4;
       const int n = nbase + nl;
@@ -459,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s.x += __uint_as_float(v.x); s.y += __uint_as_float(v.y); s.z += __uint_as_float(v.z); s.w += __uint_as_float(v.w);
         }
         float o[4] = {s.x, s.y, s.z, s.w};
-        if (kFmt == kFmtNvfp4) {
+        if (fmt_is_f4(kFmt)) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) o[j] *= alpha_f4;
         }
@@ -739,8 +761,8 @@ SkinnyPlan plan_skinny(int kFmt, int Bp, int64_t N, int kst, int lr_boxes) {
     }
   p.S = S;
   p.sh = static_cast<int>(round_up(ceil_div(kTileN, S), 4));
-  p.a_slot = kATile + (kFmt == kFmtNvfp4 ? kSfBytes : 0);
-  p.b_slot = Bp * 128 + (kFmt == kFmtNvfp4 ? kSfBytes : 0);
+  p.a_slot = kATile + sf_atoms_per_step(kFmt) * 512;
+  p.b_slot = Bp * 128 + sf_atoms_per_step(kFmt) * 512;
   const int nres_max = static_cast<int>(ceil_div(kst, S));
   const int nsteps_max = nres_max + static_cast<int>(ceil_div(lr_boxes, S));
   p.dp = kFmt == kFmtInt4 ? std::min(nres_max, kMaxRing) : 0;
@@ -790,7 +812,7 @@ cudaError_t launch_one(const CUtensorMap& w, const CUtensorMap& x, const CUtenso
 
 }  // namespace
 
-// Host side: tensor maps and launch. kind: 0 INT, 1 NVFP4; out: GemmOut.
+// Host side: tensor maps and launch. kind: GemmKind; out: GemmOut.
 bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_codes, const uint8_t* act_sf,
                         const void* down2, const svdq_weight* w, bool pdl, cudaStream_t stream,
                         cudaError_t* err) {
@@ -800,8 +822,8 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   if (kind == kKindInt && launch_gemv(out, g, act_codes, down2, w, pdl, stream, err)) return true;
   const int Bp = static_cast<int>(std::max<int64_t>(16, round_up(B, 16)));
   const bool packed = kind == kKindInt && w->fmt.bits <= 4 && w->codes4 != nullptr;
-  const int fmt = kind == kKindNvfp4 ? kFmtNvfp4 : (packed ? kFmtInt4 : kFmtInt8);
-  const int kst = static_cast<int>(kind == kKindNvfp4 ? ceil_div(M, 256) : ceil_div(M, 128));
+  const int fmt = kind == kKindNvfp4 ? kFmtNvfp4 : kind == kKindMxfp4 ? kFmtMxfp4 : (packed ? kFmtInt4 : kFmtInt8);
+  const int kst = static_cast<int>(kind != kKindInt ? ceil_div(M, 256) : ceil_div(M, 128));
   const int rp = w->rank_pad;
   const bool has_lr = out != kOutI32 && rp > 0 && down2 != nullptr;
   const int lr_boxes = has_lr ? static_cast<int>(ceil_div(2 * rp, 64)) : 0;
@@ -811,11 +833,11 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   bool ok;
   if (fmt == kFmtInt4)
     ok = make_tmap_2d(&tm_w, w->codes4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M / 2, N, M / 2, 64, kTileN, false);
-  else if (fmt == kFmtNvfp4)
+  else if (fmt_is_f4(fmt))
     ok = make_tmap_2d(&tm_w, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M / 2, N, M / 2, 128, kTileN, true);
   else
     ok = make_tmap_2d(&tm_w, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, N, M, 128, kTileN, true);
-  const int64_t xrow = kind == kKindNvfp4 ? M / 2 : M;
+  const int64_t xrow = kind != kKindInt ? M / 2 : M;
   ok = ok && make_tmap_2d(&tm_x, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xrow, B, xrow, 128, Bp, true);
   if (ok && has_lr) {
     ok = make_tmap_2d(&tm_lu, w->lu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * rp, N, 2 * rp, 64, kTileN, true) &&
@@ -839,7 +861,7 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   a.dp = p.dp;
   a.a_slot = p.a_slot;
   a.b_slot = p.b_slot;
-  a.katoms = static_cast<int>(ceil_div(M, 64));
+  a.katoms = g.katoms;
   a.s_x = g.s_x;
   a.s_w = g.s_w;
   a.bias = g.bias;
@@ -858,10 +880,12 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
   } else if (out == kOutF32) {
     if (fmt == kFmtInt4) SVDQ_SKINNY(kFmtInt4, kOutF32);
     else if (fmt == kFmtInt8) SVDQ_SKINNY(kFmtInt8, kOutF32);
+    else if (fmt == kFmtMxfp4) SVDQ_SKINNY(kFmtMxfp4, kOutF32);
     else SVDQ_SKINNY(kFmtNvfp4, kOutF32);
   } else {
     if (fmt == kFmtInt4) SVDQ_SKINNY(kFmtInt4, kOutBF16);
     else if (fmt == kFmtInt8) SVDQ_SKINNY(kFmtInt8, kOutBF16);
+    else if (fmt == kFmtMxfp4) SVDQ_SKINNY(kFmtMxfp4, kOutBF16);
     else SVDQ_SKINNY(kFmtNvfp4, kOutBF16);
   }
 #undef SVDQ_SKINNY

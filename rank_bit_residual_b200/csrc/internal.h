@@ -92,10 +92,11 @@ cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const
                             svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
                             bool* bad_args);
 
-cudaError_t launch_gemm_nvfp4(const svdq_weight* w, const uint8_t* act_codes,
-                              const uint8_t* act_sf, const float* gs_x, const void* down2,
-                              int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                              int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args);
+// NVFP4 or MXFP4, after w->fmt.kind
+cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,
+                            const uint8_t* act_sf, const float* gs_x, const void* down2,
+                            int64_t B, const void* bias, void* y, svdq_dtype ydt,
+                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args);
 
 // -------------------------------------------------------------- quantisers
 size_t residual_scratch_bytes(int64_t M, int64_t N);

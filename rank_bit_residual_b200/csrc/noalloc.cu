@@ -61,7 +61,7 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
     svdq_stream_t stream) {
   if (B < 0 || M <= 0 || (x_dtype != SVDQ_BF16 && x_dtype != SVDQ_F32)) return SVDQ_EINVAL;
   const bool int_fmt = fmt.kind == SVDQ_KIND_INT && fmt.bits >= 2 && fmt.bits <= 8;
-  const bool f4_fmt = fmt.kind == SVDQ_KIND_NVFP4 && fmt.bits == 4;
+  const bool f4_fmt = (fmt.kind == SVDQ_KIND_NVFP4 || fmt.kind == SVDQ_KIND_MXFP4) && fmt.bits == 4;
   if (!int_fmt && !f4_fmt) return SVDQ_EINVAL;
   if (!scale || rank_pad < 0 || rank_pad % 16 || rank_pad > 256) return SVDQ_EINVAL;
   if (B == 0) return SVDQ_OK;
@@ -90,7 +90,7 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
   bool bad = false;
   const cudaError_t e =
       launch_act(p, x, x_dtype, ldx, scale, fmt, act_global_scale,
-                 f4_fmt ? w_global_scale : nullptr, rp > 0 ? ld : nullptr, codes, sf, act_scale,
+                 fmt.kind == SVDQ_KIND_NVFP4 ? w_global_scale : nullptr, rp > 0 ? ld : nullptr, codes, sf, act_scale,
                  down, scratch, reinterpret_cast<cudaStream_t>(stream), &bad);
   if (bad) return SVDQ_EUNSUPPORTED;
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ECUDA;

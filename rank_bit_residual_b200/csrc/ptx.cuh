@@ -200,6 +200,19 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t a, uint64_t b, uin
       : "memory");
 }
 
+// Block-scaled e2m1 x e2m1 -> fp32 with one E8M0 (power-of-two) scale per 32
+// elements: K = 64 per instruction, two scale bytes per row, taken at byte
+// offset sf_id (0 or 2) of the row's 32-bit word in the scale columns (the
+// ids are in the instruction descriptor, idesc_mxf4).
+__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
 // Copy a 32-row x 16-byte shared-memory tile into 4 TMEM columns of all four
 // 32-lane groups (row i of the tile lands in lanes i, 32+i, 64+i, 96+i).
 __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
@@ -354,6 +367,20 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with E8M0 scales (bit 23 = 1) and scale-factor ids sf_id for A
+// ([29,31)) and B ([4,6)): the byte offset of the MMA's two scales within each
+// row's four.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+  return idesc_nvf4(M, N) | (1u << 23) | (sf_id << 4) | (sf_id << 29);
+}
+
+// TMEM address of the scales of the kk-th K = 64 MXFP4 MMA of a 128x4 atom at
+// column `col`: the byte offset 2 (kk % 2) rides in the address's top two
+// bits, as in the descriptor's scale-factor ids.
+__device__ __forceinline__ uint32_t sf_taddr(uint32_t col, int kk) {
+  return col | (static_cast<uint32_t>(2 * (kk & 1)) << 30);
+}
+
 // --------------------------------------------------- CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -440,6 +467,15 @@ __device__ __forceinline__ void mma_nvf4_pair(uint32_t d, uint64_t a, uint64_t b
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t acc, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
       : "memory");
 }

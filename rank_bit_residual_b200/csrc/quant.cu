@@ -10,6 +10,9 @@
 // alpha storage of "flashinfer.gemm.svdquant_linear"), same recipe as the
 // activation pass: gs = 448*6 / max|R|, sf = ue4m3(fl(amax_b / 6) * gs),
 // code = e2m1(R * fl(gs / sf)).
+// MXFP4 (the "mxfp4" per-block format of the SVDQuant parameter configuration
+// guide): 32-element blocks along M, E8M0 scales 2^X with X = floor(log2 amax) - 2,
+// codes e2m1(R * 2^-X), no global scale.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -133,6 +136,42 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   }
 }
 
+// MXFP4: one thread per (column n, 32-row block b) of R; e2m1 codes of R * 2^-X
+// with X from the block's amax (encode.cuh), E8M0 byte X + 127; w_scale = 1.
+__global__ void __launch_bounds__(256) quant_mxfp4_kernel(const float* __restrict__ R, int64_t M, int64_t N,
+                                                          int64_t ldR, uint8_t* __restrict__ codes,
+                                                          uint8_t* __restrict__ sf, float* __restrict__ w_scale) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *w_scale = 1.0f;
+  const int64_t kb = M / 32;
+  const int64_t kbp = (kb + 3) / 4 * 4;
+  const int64_t np = (N + 127) / 128 * 128;
+  const int64_t total = np * kbp;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / np;
+    const int64_t n = i - b * np;
+    const int64_t off = sf_swizzle_offset(n, b, kbp);
+    if (n >= N || b >= kb) {
+      sf[off] = 0;
+      continue;
+    }
+    float v[32];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      v[j] = R[(b * 32 + j) * ldR + n];
+      amax = fmaxf(amax, fabsf(v[j]));
+    }
+    const int X = mx_block_exponent(amax);
+    const float inv = mx_inv_scale(X);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], inv);
+    *reinterpret_cast<uint4*>(codes + n * (M / 2) + b * 16) =
+        make_uint4(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8), f32x8_to_e2m1(v + 16), f32x8_to_e2m1(v + 24));
+    sf[off] = static_cast<uint8_t>(X + 127);
+  }
+}
+
 // 32 codes (32 bytes) -> 16 packed bytes per thread; element 2j in the low nibble.
 __global__ void __launch_bounds__(256) pack_int4_kernel(const int8_t* __restrict__ codes, int64_t n16,
                                                         uint8_t* __restrict__ packed) {
@@ -177,6 +216,12 @@ cudaError_t launch_quantize_residual(const float* R, int64_t M, int64_t N, int64
     dim3 grid(static_cast<unsigned>(ceil_div(N, 32)), static_cast<unsigned>(ceil_div(M, 32)));
     quant_int_transpose_kernel<<<grid, 256, 0, stream>>>(R, M, N, ldR, qmax, parts, nparts,
                                                           static_cast<int8_t*>(codes), w_scale);
+  } else if (fmt.kind == SVDQ_KIND_MXFP4) {
+    const int64_t work = round_up(N, 128) * round_up(M / 32, 4);
+    const int blocks = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(work, 256), static_cast<int64_t>(num_sms()) * 8)));
+    quant_mxfp4_kernel<<<blocks, 256, 0, stream>>>(R, M, N, ldR, static_cast<uint8_t*>(codes),
+                                                    static_cast<uint8_t*>(sf), w_scale);
   } else {
     const int64_t work = round_up(N, 128) * round_up(M / 16, 4);
     const int blocks = static_cast<int>(std::max<int64_t>(

@@ -11,6 +11,7 @@ import torch
 
 import rank_bit_residual_b200 as rb
 from oracle import codes as ocodes
+from oracle import mxfp4 as omx
 from oracle import nvfp4 as onv
 from oracle import prepared as oprep
 from synth import to_bf16
@@ -90,6 +91,13 @@ class SyntheticWeight:
             # the half-size copy the short-batch GEMM streams (nibble packing done here)
             codes4 = to_dev(onv.pack_nibbles(self.codes.view(np.uint8) & 0xF).reshape(-1),
                             torch.uint8) if packed else None
+        elif f.kind == rb.KIND_MXFP4:
+            self.codes = rng.integers(0, 16, (N, M)).astype(np.uint8)
+            self.sf = rng.integers(121, 127, (N, M // 32)).astype(np.uint8)    # 2^-6 .. 2^-1
+            codes_buf = to_dev(onv.pack_nibbles(self.codes).reshape(-1), torch.uint8)
+            sf_buf = to_dev(onv.sf_swizzle(self.sf), torch.uint8)
+            self.s_w = np.float32(1.0)
+            codes4 = None
         else:
             self.codes = rng.integers(0, 16, (N, M)).astype(np.uint8)
             self.sf = rng.integers(0x20, 0x48, (N, M // 16)).astype(np.uint8)  # ~2^-3 .. 2^2
@@ -109,5 +117,8 @@ class SyntheticWeight:
             q, s_x, _ = ocodes.act_codes_int_fp32(x, self.scale, self.fmt.bits)
             return oprep.linear_int(x, ldT, L2, q, s_x, self.codes, self.s_w, bias)
         xs = ocodes.smooth_fp32(x, self.scale)
+        if self.fmt.kind == rb.KIND_MXFP4:
+            ca, sa = omx.quantize(xs)
+            return oprep.linear_mxfp4(x, ldT, L2, ca, sa, self.codes, self.sf, bias)
         ca, sa, gx = onv.quantize(xs, gs=gs_x)
         return oprep.linear_nvfp4(x, ldT, L2, ca, sa, gx, self.codes, self.sf, self.s_w, bias)

@@ -45,6 +45,12 @@ def test_weight_buffer_sizes(lib):
     assert s[0] == 3216 * 128 and s[1] == 3328 * 16   # rows padded to 128, 16 scale columns
     assert s[3] == 32 * 256 * 2
     assert s[6] == 0
+    st, s = _sizes(lib, 288, 3216, 20, "mxfp4")
+    assert st == rb.SVDQ_OK
+    assert s[0] == 3216 * 144 and s[1] == 3328 * 12   # 9 scale columns padded to 12
+    assert s[6] == 0
+    assert _sizes(lib, 64, 32, 1, (2, 8))[0] == rb.SVDQ_EINVAL   # MXFP4 has 4 bits only
+    assert _sizes(lib, 64, 32, 1, (3, 4))[0] == rb.SVDQ_EINVAL   # no fourth kind
 
 
 def test_host_checks_follow_the_page_contract(lib):

@@ -7,6 +7,7 @@ import torch
 
 import rank_bit_residual_b200 as rb
 from oracle import codes as ocodes
+from oracle import mxfp4 as omx
 from oracle import nvfp4 as onv
 from synth import make_case, to_bf16
 from tests.gpu_util import assert_codes_match, device, to_dev, x_tensor, rel_fro
@@ -145,3 +146,35 @@ def test_large_batch_units_long_and_short(B, M, dtype):
         want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
         tol = 2e-5 if dtype == "bf16" else 3e-3
         assert rel_fro(got, want) <= tol, rel_fro(got, want)
+
+
+# MXFP4: codes and E8M0 scales bit-exact (a power-of-two scale leaves no
+# rounding but the smoothing's own), act_scale 1, both batch paths
+@pytest.mark.parametrize("B,M", SHAPES + LONG)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_mxfp4_codes_scales_and_layout(B, M, dtype):
+    wl = make_case(B, M, 16, rank=0, seed=11 * B + M, dtype=dtype)
+    codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "mxfp4")
+    c_o, sf_o = omx.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
+    assert g.item() == 1.0
+    got_sf = sf.cpu().numpy()
+    want_sf = onv.sf_swizzle(sf_o)
+    assert got_sf.shape == want_sf.shape
+    assert np.array_equal(got_sf, want_sf), f"{int((got_sf != want_sf).sum())} scale bytes differ"
+    got = onv.unpack_nibbles(codes.cpu().numpy())
+    assert np.array_equal(got, c_o), f"{int((got != c_o).sum())} nibbles differ"
+
+
+@pytest.mark.parametrize("B,M,rank", [(17, 96, 16), (1100, 96, 256), (2048, 3072, 40)])
+def test_mxfp4_down_projection_is_unscaled(B, M, rank):
+    wl = make_case(B, M, 16, rank=0, seed=B + rank)
+    rp = (rank + 15) // 16 * 16
+    rng = np.random.default_rng(rank + 2)
+    ld = np.zeros((rp, M), np.float32)
+    ld[:rank] = to_bf16(rng.standard_normal((rank, M)).astype(np.float32) * 0.1)
+    _, _, g, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "mxfp4",
+                                         ld=to_dev(ld, torch.bfloat16))
+    d = down.float().cpu().numpy().astype(np.float64)
+    want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
+    assert g.item() == 1.0
+    assert rel_fro(d[:, :rp] + d[:, rp:], want) <= 2e-5

@@ -93,6 +93,20 @@ def test_linear_nvfp4_matches_oracle(B, M, N, rank, bias, xdt, given_gs):
     assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("B,M,N,rank,bias", NVFP4_CASES + [(2048, 1152, 640, 32, True)])
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_linear_mxfp4_matches_oracle(B, M, N, rank, bias, xdt):
+    wl = make_case(B, M, N, rank=rank, seed=B * 7 + N, dtype=xdt, bias=bias)
+    w = SyntheticWeight(M, N, rank, "mxfp4", seed=N + 2 * rank, scale=wl.scale)
+    b = to_dev(wl.bias, torch.bfloat16) if bias else None
+    y32 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.float32)
+    y16 = rb.svdq_linear(w.w, x_tensor(wl), bias=b, out_dtype=torch.bfloat16)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    want = w.oracle_y(wl.x, wl.bias if bias else None)
+    assert_y_close(y32.cpu().numpy(), want, f"mxfp4 {B}x{M}x{N} r={rank} {xdt}")
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
 def test_linear_workspace_reused_across_shapes():
     """One workspace for calls of different batch sizes (the large- and the
     short-batch paths): each call equals a call on a fresh workspace, bit for

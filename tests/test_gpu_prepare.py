@@ -12,6 +12,7 @@ import torch
 
 import rank_bit_residual_b200 as rb
 from oracle import codes as ocodes
+from oracle import mxfp4 as omx
 from oracle import nvfp4 as onv
 from oracle import prepared as oprep
 from oracle import svdquant as osq
@@ -73,7 +74,7 @@ def test_prepare_rank_zero_quantises_smoothed_weight_exactly(fmt):
 
 
 @pytest.mark.parametrize("M,N", [(32, 16), (256, 272), (1024, 3072)])
-@pytest.mark.parametrize("fmt", ["int4", "int8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "int8", "nvfp4", "mxfp4"])
 def test_quantize_residual_bit_exact(M, N, fmt):
     rng = np.random.default_rng(M + N)
     R = (rng.standard_t(4, (M, N)) * 0.02).astype(np.float32)
@@ -81,6 +82,11 @@ def test_quantize_residual_bit_exact(M, N, fmt):
     if fmt == "nvfp4":
         c_o, sf_o, g_o = onv.quantize(np.ascontiguousarray(R.T))
         assert np.float32(g.item()) == np.float32(g_o)
+        assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
+        assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
+    elif fmt == "mxfp4":
+        c_o, sf_o = omx.quantize(np.ascontiguousarray(R.T))
+        assert g.item() == 1.0
         assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
         assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
     else:
@@ -143,3 +149,19 @@ def test_prepare_then_linear_nvfp4(M, N, rank, bias):
     # the residual codes are the oracle's NVFP4 codes of the GPU residual's own recipe
     ws, R = _residual(wl, w)
     assert np.linalg.norm(R) <= 1.01 * osq.tail_norm(ws, rank)
+
+
+@pytest.mark.parametrize("M,N,rank,B", [(256, 128, 16, 64), (1024, 768, 32, 300)])
+def test_prepare_then_linear_mxfp4(M, N, rank, B):
+    wl = make_case(B, M, N, rank=rank, seed=M + 5, bias=True)
+    w = rb.svdq_prepare(to_dev(wl.W, torch.bfloat16), to_dev(wl.scale, torch.float32), rank, "mxfp4")
+    assert w.w_scale[0].item() == 1.0
+    y = rb.svdq_linear(w, x_tensor(wl), bias=to_dev(wl.bias, torch.bfloat16), out_dtype=torch.float32)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    ld, lu = _host(w)
+    rp = w.rank_pad
+    cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
+    sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 32)
+    ca, sa = omx.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
+    want = oprep.linear_mxfp4(wl.x, ld.T, lu[:, :rp].T, ca, sa, cw, sfw, wl.bias)
+    assert_y_close(y.cpu().numpy(), want, "prepare+mxfp4")

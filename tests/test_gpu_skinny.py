@@ -43,7 +43,7 @@ def test_short_batch_int32_product_is_exact(B, M, N, packed):
 
 @pytest.mark.parametrize("B,M,N", SHAPES)
 @pytest.mark.parametrize("fmt,packed", [("int4", True), ("int4", False), ("int8", False),
-                                        ("nvfp4", False)])
+                                        ("nvfp4", False), ("mxfp4", False)])
 def test_short_batch_linear_matches_oracle(B, M, N, fmt, packed):
     rank = 32 if M >= 64 and N >= 64 else 8
     wl = make_case(B, M, N, rank=rank, seed=B + 2 * N + M, bias=True)
@@ -54,7 +54,7 @@ def test_short_batch_linear_matches_oracle(B, M, N, fmt, packed):
     assert_y_close(y.cpu().numpy(), w.oracle_y(wl.x, wl.bias), f"{fmt} packed={packed} {B}x{M}x{N}")
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4"])
 def test_chained_launch_equals_separate_calls(fmt):
     """svdq_linear launches the GEMM as a dependent launch of the activation pass
     (its weight loads overlap that kernel); the result must equal the two stages

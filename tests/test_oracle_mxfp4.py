@@ -73,3 +73,29 @@ def test_error_bound_and_product():
     w = rng.standard_normal((8, 128))
     wc, ws = mx.quantize(w)
     assert np.allclose(mx.product(codes, sf, wc, ws), d @ mx.dequantize(wc, ws).T, rtol=0, atol=1e-12)
+
+
+def test_linear_on_representable_operands_is_the_plain_product():
+    """Operands already on the MXFP4 grid quantise to themselves, so the two-branch
+    linear is x Ld Lu + x W^T + bias, summed here element by element."""
+    from oracle import prepared as oprep
+    rng = np.random.default_rng(3)
+    grid = nv.e2m1_decode(np.arange(16))
+
+    def on_grid(rows, K):
+        v = rng.choice(grid, (rows, K))
+        v[:, ::32] = 6.0
+        return v * np.repeat(2.0 ** rng.integers(-6, 4, (rows, K // 32)), 32, axis=1)
+
+    B, M, N, r = 2, 64, 3, 2
+    x, W = on_grid(B, M), on_grid(N, M)
+    ld, lu = rng.standard_normal((M, r)), rng.standard_normal((r, N))
+    bias = rng.standard_normal(N)
+    ca, sa = mx.quantize(x)
+    cw, sw = mx.quantize(W)
+    y = oprep.linear_mxfp4(x, ld, lu, ca, sa, cw, sw, bias)
+    for b in range(B):
+        for n in range(N):
+            res = sum(x[b, k] * W[n, k] for k in range(M))
+            low = sum(sum(x[b, k] * ld[k, j] for k in range(M)) * lu[j, n] for j in range(r))
+            assert abs(y[b, n] - (res + low + bias[n])) <= 1e-12 * (1 + abs(res) + abs(low))
