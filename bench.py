@@ -62,8 +62,8 @@ def workload_ops(B, M, N, rank):
 def alg_bytes(B, M, N, rank, fmt, bits, bias):
     """Algorithmic bytes of one step: bf16 x, weight codes (+scales), bf16 factors,
     fp32 scale, bias, bf16 Y."""
-    if fmt == "nvfp4":
-        wbytes = M * N * (0.5 + 1.0 / 16.0)
+    if fmt in ("nvfp4", "mxfp4"):
+        wbytes = M * N * (0.5 + (1.0 / 16.0 if fmt == "nvfp4" else 1.0 / 32.0))
     else:
         wbytes = M * N * (0.5 if bits <= 4 else 1.0)
     return (B * M * 2 + wbytes + 2 * rank * (M + N) + 4 * M + (2 * N if bias else 0)
@@ -74,8 +74,9 @@ def gemm_alg_bytes(B, M, N, rank, fmt, bits, bias):
     """Algorithmic bytes of one GEMM launch: weight codes (+ scales), the bf16 up
     factor, the activation codes (+ scales) and the bf16 down tile it reads, bias,
     and the bf16 Y it writes."""
-    if fmt == "nvfp4":
-        wbytes, abytes = M * N * (0.5 + 1.0 / 16.0), B * M * (0.5 + 1.0 / 16.0)
+    if fmt in ("nvfp4", "mxfp4"):
+        per = 0.5 + (1.0 / 16.0 if fmt == "nvfp4" else 1.0 / 32.0)
+        wbytes, abytes = M * N * per, B * M * per
     else:
         wbytes, abytes = M * N * (0.5 if bits <= 4 else 1.0), B * M
     return wbytes + 2 * rank * N + abytes + 2 * B * rank + (2 * N if bias else 0) + 2 * B * N
@@ -271,7 +272,7 @@ def main():
 
     wl = make_workload(args.workload)
     B, M, N, r = wl.B, wl.M, wl.N, wl.rank
-    fmt = f"int{wl.bits}" if wl.fmt == "int" else "nvfp4"
+    fmt = f"int{wl.bits}" if wl.fmt == "int" else wl.fmt
     xdt = torch.bfloat16 if wl.x_dtype == "bf16" else torch.float32
     x = torch.from_numpy(wl.x).to(xdt).to(dev)
     W = torch.from_numpy(wl.W).to(xdt).to(dev)
@@ -435,6 +436,13 @@ def main():
             cw = w.codes.view(torch.int8).cpu().numpy().reshape(N, M)
             want = oprep.linear_int(wl.x[rows], ld, L2, q[rows], s_x, cw, float(w.w_scale[0].item()),
                                     wl.bias)
+        elif wl.fmt == "mxfp4":
+            from oracle import mxfp4 as omx
+            from oracle import nvfp4 as onv
+            ca, sa = omx.quantize(ocodes.smooth_fp32(wl.x[rows], wl.scale))
+            cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
+            sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 32)
+            want = oprep.linear_mxfp4(wl.x[rows], ld, L2, ca, sa, cw, sfw, wl.bias)
         else:
             from oracle import nvfp4 as onv
             xs = ocodes.smooth_fp32(wl.x, wl.scale)
@@ -475,7 +483,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     # a contraction takes the peak of its own dtype: measured bf16 x nominal ratio
-    ratio = 4.0 if wl.fmt == "nvfp4" else 2.0
+    ratio = 4.0 if wl.fmt != "int" else 2.0
     lowp_peak = ratio * peaks["bf16_tflops"]
     g_ops = gemm_alg_ops(B, M, N, r)
     achieved = g_ops / (gemm_avg_ms * 1e-3) / 1e12
@@ -488,7 +496,7 @@ def main():
         # short batch: the GEMM streams the weights; its roofline is HBM
         gb = gemm_alg_bytes(B, M, N, r, wl.fmt, wl.bits, wl.bias is not None)
         roof = {"bound": "hbm",
-                "kernel": "skinny_kernel<" + ("NVFP4" if wl.fmt == "nvfp4" else
+                "kernel": "skinny_kernel<" + (wl.fmt.upper() if wl.fmt != "int" else
                                               ("INT4 packed" if wl.bits <= 4 else "INT8")) +
                           "> (split-K clusters, residual + bf16 up-projection)",
                 "duration_us": gemm_avg_ms * 1e3,
@@ -499,8 +507,8 @@ def main():
                 "peak_source": f"{peak_src} HBM copy bandwidth"}
     else:
         roof = {"bound": "tensor",
-                "kernel": "gemm_pair_kernel" + ("<NVFP4> (e2m1 block-scaled residual + bf16 up-projection)"
-                                                if wl.fmt == "nvfp4" else
+                "kernel": "gemm_pair_kernel" + (f"<{wl.fmt.upper()}> (e2m1 block-scaled residual + bf16 "
+                                                "up-projection)" if wl.fmt != "int" else
                                                 "<INT> (int8 residual + bf16 up-projection)"),
                 "duration_us": gemm_avg_ms * 1e3,
                 "timing": "Kg launches back to back on rotating sets (CUDA graphs) between one CUDA event pair",
@@ -514,7 +522,7 @@ def main():
     out = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1" if wl.fmt == "nvfp4" else "int8",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1" if wl.fmt != "int" else "int8",
         "data": "synthetic",
         "config": {"workload": args.workload, "B": B, "M": M, "N": N, "rank": r, "fmt": fmt,
                    "x": wl.x_dtype, "y": "bf16", "bias": wl.bias is not None,

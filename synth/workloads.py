@@ -52,8 +52,8 @@ class Workload:
     w_dtype: str
     scale: np.ndarray             # float32 [M], > 0
     rank: int
-    fmt: str                      # "int" or "nvfp4"
-    bits: int                     # 2..8 for "int", 4 for "nvfp4"
+    fmt: str                      # "int", "nvfp4" or "mxfp4"
+    bits: int                     # 2..8 for "int", 4 for the fp4 formats
     bias: Optional[np.ndarray] = None   # float32 [N], bf16-representable
     seed: int = 0
     notes: dict = field(default_factory=dict)
@@ -156,6 +156,17 @@ _SPECS = {
                  outlier_frac=0.005, outlier_factor=20.0, w_std=0.02,
                  spikes=tuple(np.linspace(8.0, 0.5, 16)), alpha=0.5),
         rank=32, fmt="nvfp4", bits=4),
+    # the same two shapes with MXFP4 blocks (E8M0 scales per 32 elements)
+    "dit_mlp_4096x3072x12288_mxfp4": dict(
+        gen=dict(B=4096, M=3072, N=12288, seed=2, x_dist="student_t", dtype="bf16",
+                 outlier_frac=0.01, outlier_factor=30.0, w_std=0.02,
+                 spikes=tuple(np.linspace(5.0, 1.0, 8)), alpha=0.5, bias_std=0.01),
+        rank=32, fmt="mxfp4", bits=4),
+    "decode_128x4096x4096_mxfp4": dict(
+        gen=dict(B=128, M=4096, N=4096, seed=3, x_dist="normal", dtype="bf16",
+                 outlier_frac=0.005, outlier_factor=20.0, w_std=0.02,
+                 spikes=tuple(np.linspace(8.0, 0.5, 16)), alpha=0.5),
+        rank=32, fmt="mxfp4", bits=4),
     # large compute-bound sweep
     "large_8192x12288x3072_int4_r32": dict(
         gen=dict(B=8192, M=12288, N=3072, seed=4, x_dist="student_t", dtype="bf16",
