@@ -414,6 +414,51 @@ def main():
                           "hbm_roofline_frac": t_mem / (us * 1e-6), "alg_bytes": byt})
         assert rb.svdq_check_status() == rb.SVDQ_OK
 
+    # consecutive linears (square shapes): layer k of a chain of R runs on set k's
+    # weights and reads layer k-1's Y, so the weights stream from HBM while the
+    # activations stay in L2, as in a network; timed plain and with each layer's
+    # activation pass a programmatic dependent of the previous layer's GEMM
+    chain = None
+    if M == N:
+        def chain_graph(pdl, rows):
+            def run():
+                prev = x[:rows]
+                for k in range(R):
+                    wk, _, _, _, _, _, yk, wsk = sets[k]
+                    rb.svdq_linear(wk, prev, bias=bias, out=yk[:rows], workspace=wsk, pdl=pdl and k > 0)
+                    prev = yk[:rows]
+            run()
+            torch.cuda.synchronize()
+            cap = torch.cuda.Stream()
+            cap.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                run()
+            stream.wait_stream(cap)
+            return g
+
+        def time_chain(pdl, rows, reps):
+            g = chain_graph(pdl, rows)
+            g.replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) * 1e3 / (reps * R)
+
+        chain = {"layers_per_chain": R, "note": "us per linear, chains of R layers of this shape "
+                                               "captured in one CUDA graph; layer 0 plain in both"}
+        for rows in ((1, B) if args.workload.startswith("decode_") else (B,)):
+            reps = max(3, min(50, (200 * 1000) // max(1, R * int(ms_per_step * 1e3 + 1))))
+            plain = time_chain(False, rows, reps)
+            pdl = time_chain(True, rows, reps)
+            chain[f"B={rows}"] = {"plain_us": plain, "pdl_us": pdl, "saved_us": plain - pdl}
+        assert rb.svdq_check_status() == rb.SVDQ_OK
+
     # each stage alone, Ks launches back to back on the rotating sets: the GEMM's
     # average launch duration is the roofline line's
     Kg = max(20, min(K, 400))
@@ -544,6 +589,7 @@ def main():
                 "call": "svdq_linear (pinned host x -> device, Y -> pinned host)"},
         "gpu_launches": 3 * K,   # per step: activation stats, activation codes, residual GEMM
         "sweep": sweep,
+        "chain": chain,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:

@@ -248,6 +248,33 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
 
 svdq_status svdq_linear_workspace_size(const svdq_weight* w, int64_t B, size_t* bytes);
 
+/* Flags of svdq_linear_ex. */
+#define SVDQ_LINEAR_PDL 1u
+
+/*
+ * svdq_linear_ex - svdq_linear with launch options; flags = 0 is svdq_linear.
+ *
+ * SVDQ_LINEAR_PDL ("flashinfer.gemm.svdquant_linear", its enable_pdl option,
+ * here across consecutive linears): the activation pass's first kernel is
+ * launched as a programmatic dependent of the kernel queued just before it on
+ * `stream` - typically the GEMM of the previous linear, whose Y is this call's
+ * x. It starts on the SMs that kernel frees (or leaves idle), does its
+ * weight-side setup (w->scale, w->ld: shared-memory staging, barriers, tensor
+ * memory), and reads x only after griddepcontrol.wait, when that kernel has
+ * finished and its writes are visible; everything after it, and every write
+ * of this call, comes after that wait. Precondition: w's buffers (scale, ld,
+ * codes, sf, lu, w_scale) and the bias are not written by work still in flight
+ * on the stream (e.g. an svdq_prepare queued just before: synchronise, or
+ * record an event, before the first chained call). The workspace may be the
+ * one the previous call used. Any flag bit other than SVDQ_LINEAR_PDL returns
+ * SVDQ_EINVAL. The result equals svdq_linear's, bit for bit.
+ */
+svdq_status svdq_linear_ex(const svdq_weight* w, const void* x, svdq_dtype x_dtype, int64_t B,
+                           int64_t ldx, const void* bias, const float* act_global_scale,
+                           void* y, svdq_dtype y_dtype, int64_t ldy,
+                           void* workspace, size_t workspace_bytes, uint32_t flags,
+                           svdq_stream_t stream);
+
 /*
  * svdq_residual_linear - the GEMM stage of svdq_linear on its own, from
  * activation codes made by svdq_quantize_act (step 3 of the three-step chain of

@@ -29,6 +29,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "svdq.h")
 SVDQ_OK, SVDQ_EINVAL, SVDQ_ERANK, SVDQ_EUNSUPPORTED, SVDQ_ECUDA, SVDQ_ETIMEOUT, SVDQ_EWORKSPACE = range(7)
 SVDQ_F32, SVDQ_BF16 = 0, 1
 KIND_INT, KIND_NVFP4, KIND_MXFP4 = 0, 1, 2
+SVDQ_LINEAR_PDL = 1
 
 c_i32, c_i64, c_u64, c_sz, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -60,6 +61,8 @@ _SIGS = {
     "svdq_quantize_act_workspace_size": (c_i32, [c_i64, c_i64, SvdqFmt, c_i32, ctypes.POINTER(c_sz)]),
     "svdq_linear": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i32, c_i64, c_i64, c_vp, c_vp,
                             c_vp, c_i32, c_i64, c_vp, c_sz, c_vp]),
+    "svdq_linear_ex": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i32, c_i64, c_i64, c_vp, c_vp,
+                               c_vp, c_i32, c_i64, c_vp, c_sz, ctypes.c_uint32, c_vp]),
     "svdq_linear_workspace_size": (c_i32, [ctypes.POINTER(SvdqWeight), c_i64, ctypes.POINTER(c_sz)]),
     "svdq_residual_product_i32": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_i64, c_vp, c_i64, c_vp]),
     "svdq_residual_linear": (c_i32, [ctypes.POINTER(SvdqWeight), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
@@ -412,8 +415,15 @@ def linear_workspace_size(w: PreparedWeight, B: int) -> int:
 
 def svdq_linear(w: PreparedWeight, x: torch.Tensor, bias: Optional[torch.Tensor] = None,
                 out_dtype=torch.bfloat16, act_global_scale: Optional[torch.Tensor] = None,
-                out: Optional[torch.Tensor] = None, workspace: Optional[LinearWorkspace] = None):
-    """Y[B, N] = x ld^T lu^T + alpha Q(X_hat) Q(R) (+ bias) on the current stream."""
+                out: Optional[torch.Tensor] = None, workspace: Optional[LinearWorkspace] = None,
+                pdl: bool = False):
+    """Y[B, N] = x ld^T lu^T + alpha Q(X_hat) Q(R) (+ bias) on the current stream.
+
+    pdl=True (svdq_linear_ex with SVDQ_LINEAR_PDL): the activation pass starts as a
+    programmatic dependent of the kernel queued before it (the previous linear's
+    GEMM, whose output is x) and reads x only once that kernel has finished. w's
+    buffers and the bias must not be written by work still in flight on the stream.
+    """
     lib = load_library()
     _require_cuda(x)
     x = _rows_ready(x)
@@ -428,9 +438,30 @@ def svdq_linear(w: PreparedWeight, x: torch.Tensor, bias: Optional[torch.Tensor]
     y = out if out is not None else torch.empty((B, w.N), dtype=out_dtype, device=x.device)
     nbytes = linear_workspace_size(w, B)
     ws = (workspace or _default_ws).get(nbytes, x.device)
-    _check(lib.svdq_linear(ctypes.byref(w.desc), _ptr(x), _dt(x), B, x.stride(0), _ptr(bias),
-                           _ptr(act_global_scale), _ptr(y), _dt(y), y.stride(0), _ptr(ws), ws.numel(),
-                           _stream()), "svdq_linear")
+    if pdl:
+        _check(lib.svdq_linear_ex(ctypes.byref(w.desc), _ptr(x), _dt(x), B, x.stride(0), _ptr(bias),
+                                  _ptr(act_global_scale), _ptr(y), _dt(y), y.stride(0), _ptr(ws),
+                                  ws.numel(), SVDQ_LINEAR_PDL, _stream()), "svdq_linear_ex")
+    else:
+        _check(lib.svdq_linear(ctypes.byref(w.desc), _ptr(x), _dt(x), B, x.stride(0), _ptr(bias),
+                               _ptr(act_global_scale), _ptr(y), _dt(y), y.stride(0), _ptr(ws), ws.numel(),
+                               _stream()), "svdq_linear")
+    return y
+
+
+def svdq_linear_chain(weights, x: torch.Tensor, biases=None, out_dtype=torch.bfloat16,
+                      pdl: bool = True, workspace: Optional[LinearWorkspace] = None,
+                      outs=None) -> torch.Tensor:
+    """Consecutive linears y_i = linear(w_i, y_{i-1}) (y_0 = x) on the current stream,
+    every call after the first chained to the one before with PDL (pdl=True). Each
+    intermediate y is in out_dtype (bf16 by default); ``outs`` may hold
+    preallocated outputs, one per linear."""
+    biases = biases if biases is not None else [None] * len(weights)
+    ws = workspace or LinearWorkspace()
+    y = x
+    for i, (w, b) in enumerate(zip(weights, biases)):
+        y = svdq_linear(w, y, bias=b, out_dtype=out_dtype, workspace=ws, pdl=pdl and i > 0,
+                        out=outs[i] if outs is not None else None)
     return y
 
 
@@ -491,7 +522,7 @@ def svdq_selftest_wait_timeout(limit_us: int = 1000) -> int:
 
 __all__ = [
     "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_act_noalloc",
-    "svdq_quantize_residual", "svdq_linear", "svdq_pack_int4",
+    "svdq_quantize_residual", "svdq_linear", "svdq_linear_chain", "svdq_pack_int4",
     "svdq_residual_product_i32", "svdq_residual_linear", "svdq_check_status", "svdq_selftest_wait_timeout",
     "svdq_smooth_scale",
     "PreparedWeight", "LinearWorkspace", "allocate_weight", "weight_from_buffers",

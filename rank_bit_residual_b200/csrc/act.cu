@@ -71,6 +71,7 @@ struct ActArgs {
   int nparts;       // partial maxima written by the stats kernel
   int stages;       // stats kernel: shared-memory stages
   int nacc;         // stats kernel: MMA issuers, each with its own TMEM accumulator
+  int chained;      // stats kernel: launched as a programmatic dependent of the previous kernel
   const void* x;
   const float* scale;
   const float* gs_given;
@@ -189,6 +190,11 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
     fence_mbar_init();
     abort_sh = 0;
   }
+  // chained after another linear: x is that linear's output, complete and
+  // visible once the kernel before this one has finished. Waited for before the
+  // tensor-memory allocation, so a CTA of this kernel that shares an SM with
+  // one of that kernel's never holds columns that kernel is waiting for.
+  if (a.chained) pdl_wait();
   if (rp > 0 && warp == 0) {
     tmem_alloc(&tmem_sh, acc_cols * nacc);
     tmem_relinquish();
@@ -526,8 +532,17 @@ cudaError_t launch_stats(const ActArgs& a, int grid, size_t smem, cudaStream_t s
   cudaError_t err = cudaFuncSetAttribute(act_stats_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  act_stats_kernel<TIn><<<grid, kWork, smem, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kWork);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.chained ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, act_stats_kernel<TIn>, a);
 }
 
 template <typename TIn>
@@ -655,6 +670,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.stages = q.stages;
   // as many MMA issuers (up to 4) as TMEM holds accumulators of rank_pad columns
   a.nacc = a.rank_pad > 0 ? static_cast<int>(std::min<uint32_t>(4u, 512u / tmem_cols_for(a.rank_pad))) : 1;
+  a.chained = p.chained;
   // the codes kernel keeps only the unit's reciprocals in shared memory
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   const size_t smem2 = static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;

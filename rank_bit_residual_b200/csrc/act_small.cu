@@ -45,6 +45,7 @@ constexpr int kZBatch = 20;  // partials one thread loads at once (covers 160 CT
 
 struct SmallArgs {
   int B, M, wc, G, rank_pad, fmt_kind, qmax, has_ld;
+  int chained;        // the stats kernel is a programmatic dependent of the previous kernel
   int64_t ldx;
   const void* x;
   const float* scale;
@@ -94,7 +95,10 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float red[kWarps];
 
-  pdl_trigger();   // the codes kernel launched after this one may start loading x now
+  // the codes kernel launched after this one may start loading x now; when
+  // chained after another linear, x is that linear's output: first the
+  // weight-side loads, then the wait for the previous kernel, then the trigger
+  if (!a.chained) pdl_trigger();
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.x;
@@ -109,13 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
   uint32_t* cm = reinterpret_cast<uint32_t*>(rcp + a.wc);           // kThreads column-max slots
 
   // ------------------------------------------------------------ loads
+  // weight side (ld, scale) first: it does not depend on the previous kernel
   const int vpr = ncols * kEsz / 16;   // 16-byte vectors per chunk row
-  for (int i = tid; i < B * vpr; i += kThreads) {
-    const int r = i / vpr, v = i - r * vpr;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
-        static_cast<const uint8_t*>(a.x) + (static_cast<int64_t>(r) * a.ldx + c0) * kEsz) + v);
-    *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = u;
-  }
   if (a.has_ld) {
     for (int i = tid; i < (bp16 - B) * vpr; i += kThreads) {   // zero rows up to a multiple of 16
       const int r = B + i / vpr, v = i % vpr;
@@ -129,6 +128,17 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
     }
   }
   for (int k = tid; k < ncols; k += kThreads) rcp[k] = __frcp_rn(__ldg(a.scale + c0 + k));
+  if (a.chained) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  // x through L2 (it may be the output of the kernel just waited for)
+  for (int i = tid; i < B * vpr; i += kThreads) {
+    const int r = i / vpr, v = i - r * vpr;
+    const uint4 u = __ldcg(reinterpret_cast<const uint4*>(
+        static_cast<const uint8_t*>(a.x) + (static_cast<int64_t>(r) * a.ldx + c0) * kEsz) + v);
+    *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = u;
+  }
   __syncthreads();
 
   // ------------------------------------------------- column maxima of |x|
@@ -249,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
   const int vpr = ncols * kEsz / 16;
   for (int i = tid; i < B * vpr; i += kThreads) {
     const int r = i / vpr, v = i - r * vpr;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+    const uint4 u = __ldcg(reinterpret_cast<const uint4*>(
         static_cast<const uint8_t*>(a.x) + (static_cast<int64_t>(r) * a.ldx + c0) * kEsz) + v);
     *reinterpret_cast<uint4*>(xs + r * pitch + v * 16) = u;
   }
@@ -431,18 +441,19 @@ cudaError_t launch_pair_of_kernels(K1 k1, K2 k2, const SmallArgs& a, int grid, s
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(k2, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (err != cudaSuccess) return err;
-  k1<<<grid, kThreads, smem1, stream>>>(a);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem2;
+  cfg.dynamicSmemBytes = smem1;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
+  cfg.numAttrs = a.chained ? 1 : 0;   // chained: a dependent of the previous kernel too
+  err = cudaLaunchKernelEx(&cfg, k1, a);
+  if (err != cudaSuccess) return err;
+  cfg.dynamicSmemBytes = smem2;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k2, a);
 }
@@ -485,6 +496,7 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
   a.fmt_kind = fmt.kind;
   a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
   a.has_ld = has_ld ? 1 : 0;
+  a.chained = p.chained;
   a.ldx = ldx;
   a.x = x;
   a.scale = scale;

@@ -338,6 +338,15 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
                         int64_t ldx, const void* bias, const float* act_global_scale, void* y,
                         svdq_dtype y_dtype, int64_t ldy, void* workspace, size_t workspace_bytes,
                         svdq_stream_t stream) {
+  return svdq_linear_ex(w, x, x_dtype, B, ldx, bias, act_global_scale, y, y_dtype, ldy, workspace,
+                        workspace_bytes, 0u, stream);
+}
+
+svdq_status svdq_linear_ex(const svdq_weight* w, const void* x, svdq_dtype x_dtype, int64_t B,
+                           int64_t ldx, const void* bias, const float* act_global_scale, void* y,
+                           svdq_dtype y_dtype, int64_t ldy, void* workspace, size_t workspace_bytes,
+                           uint32_t flags, svdq_stream_t stream) {
+  if (flags & ~SVDQ_LINEAR_PDL) return SVDQ_EINVAL;
   svdq_status s = check_weight(w);
   if (s != SVDQ_OK) return s;
   s = check_act_input(x, x_dtype, B, w->M, ldx);
@@ -351,7 +360,8 @@ svdq_status svdq_linear(const svdq_weight* w, const void* x, svdq_dtype x_dtype,
   LinearCarve c = carve_linear(w, B, workspace, workspace_bytes, x_dtype);
   if (!c.ok) return SVDQ_EWORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const ActPlan p = plan_act(B, w->M, w->rank_pad, x_dtype);
+  ActPlan p = plan_act(B, w->M, w->rank_pad, x_dtype);
+  p.chained = (flags & SVDQ_LINEAR_PDL) ? 1 : 0;
   bool bad = false;
   cudaError_t e = launch_act(p, x, x_dtype, ldx, w->scale, w->fmt, act_global_scale,
                              w->fmt.kind == SVDQ_KIND_NVFP4 ? w->w_scale : nullptr,

@@ -106,6 +106,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  // a chained linear's activation pass queued after this kernel may start its
+  // weight-side setup now (it reads this kernel's output only after griddepcontrol.wait)
+  pdl_trigger();
   const int B = args.B, N = args.N, M = args.M, lr_steps = args.lr_steps;
   unsigned* status = args.status;
   const int warp = threadIdx.x >> 5;

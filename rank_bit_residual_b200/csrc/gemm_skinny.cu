@@ -127,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  // a chained linear's activation pass queued after this kernel may start its
+  // weight-side setup now (it reads this kernel's output only after griddepcontrol.wait)
+  pdl_trigger();
   uint8_t* ring_a = smem;
   uint8_t* ring_b = ring_a + static_cast<size_t>(a.dr) * a.a_slot;
   uint8_t* ring_p = ring_b + static_cast<size_t>(a.dr) * a.b_slot;
@@ -562,6 +565,9 @@ __host__ __device__ constexpr size_t gemv_smem(int rows, int row_bytes, int B, i
 template <bool kPacked, int kOut>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs g) {
   extern __shared__ __align__(16) uint8_t gsm[];
+  // a chained linear's activation pass queued after this kernel may start its
+  // weight-side setup now (it reads this kernel's output only after griddepcontrol.wait)
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * g.rows_per_cta;
   const int rows = min(g.rows_per_cta, g.N - n0);

@@ -58,6 +58,8 @@ struct ActPlan {
   size_t smem;     // dynamic shared memory per CTA
   int small;       // 1: the short-batch kernel (act_small.cu): one column chunk per CTA
   int wc;          // short-batch kernel: columns per chunk (a multiple of 32)
+  int chained;     // 1: the first kernel is a programmatic dependent of the work
+                   // queued before it (reads x only after griddepcontrol.wait)
 };
 // Batches up to this many rows take the short-batch kernel.
 constexpr int64_t kActSmallMaxB = 128;

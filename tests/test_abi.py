@@ -90,3 +90,11 @@ def test_python_binding_rejects_non_int_rank():
             rb.svdq_prepare(W, s, r)
     with pytest.raises(ValueError):      # CPU tensors are refused, never computed on the host
         rb.svdq_prepare(W, s, 1)
+
+
+def test_linear_ex_rejects_unknown_flags(lib):
+    """Checked before anything touches the device."""
+    w = rb.SvdqWeight()
+    st = lib.svdq_linear_ex(ctypes.byref(w), None, 0, 1, 64, None, None, None, 0, 64, None, 0,
+                            ctypes.c_uint32(2), None)
+    assert st == rb.SVDQ_EINVAL
