@@ -9,6 +9,7 @@ import torch
 
 import rank_bit_residual_b200 as rb
 from oracle import codes as ocodes
+from oracle import mxfp4 as omx
 from oracle import nvfp4 as onv
 from oracle import prepared as oprep
 from oracle import svdquant as osq
@@ -20,11 +21,14 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 CASES = [
     ("dit_attn_4096x3072x3072_int4", None),
     ("dit_mlp_4096x3072x12288_nvfp4", None),
+    ("dit_mlp_4096x3072x12288_mxfp4", None),
     ("decode_128x4096x4096_int4", 1),
     ("decode_128x4096x4096_int4", 16),
     ("decode_128x4096x4096_int4", 128),
     ("decode_128x4096x4096_nvfp4", 1),
     ("decode_128x4096x4096_nvfp4", 128),
+    ("decode_128x4096x4096_mxfp4", 1),
+    ("decode_128x4096x4096_mxfp4", 128),
     ("large_8192x12288x3072_int4_r32", None),
     ("large_8192x12288x3072_int4_r128", None),
     ("large_8192x12288x3072_int8_r32", None),
@@ -38,7 +42,7 @@ def _prepare(wl):
     key = (wl.name, wl.fmt, wl.bits, wl.rank)
     if key not in _prepared:
         _prepared.clear()
-        fmt = f"int{wl.bits}" if wl.fmt == "int" else "nvfp4"
+        fmt = f"int{wl.bits}" if wl.fmt == "int" else wl.fmt
         W = to_dev(wl.W, torch.bfloat16)
         w = rb.svdq_prepare(W, to_dev(wl.scale, torch.float32), wl.rank, fmt, seed=0)
         _prepared[key] = w
@@ -64,6 +68,11 @@ def test_fullsize_sampled_parity(name, rows):
         cw = w.codes.view(torch.int8).cpu().numpy().reshape(N, M)
         want = oprep.linear_int(wl.x[sample], ld, L2, q[sample], s_x, cw,
                                 float(w.w_scale[0].item()), wl.bias)
+    elif wl.fmt == "mxfp4":
+        ca, sa = omx.quantize(ocodes.smooth_fp32(wl.x[sample], wl.scale))
+        cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
+        sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 32)
+        want = oprep.linear_mxfp4(wl.x[sample], ld, L2, ca, sa, cw, sfw, wl.bias)
     else:
         ca, sa, gx = onv.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
         cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
