@@ -72,10 +72,12 @@ typedef struct svdq_fmt {
  * svdq_weight_buffer_sizes), fills the pointers, and svdq_prepare fills them.
  * Layouts (all row-major, K = M is the reduction dim):
  *   codes   INT:   int8  [N, M]      residual codes, K-major (row n holds column n of R)
- *           NVFP4: uint8 [N, M/2]    e2m1 nibbles, element 2j in the low nibble of byte j
+ *           fp4:   uint8 [N, M/2]    e2m1 nibbles, element 2j in the low nibble of byte j
  *   sf      NVFP4: uint8, 128x4 layout of the [N, M/16] ue4m3 block scales
+ *           MXFP4: uint8, 128x4 layout of the [N, M/32] E8M0 block scales
  *           (rows padded to 128, scale columns to 4); unused (may be NULL) for INT
- *   w_scale fp32 device scalar: INT s_w = max|R| / qmax; NVFP4 global scale gs_w
+ *   w_scale fp32 device scalar: INT s_w = max|R| / qmax; NVFP4 global scale gs_w;
+ *           MXFP4 1
  *   ld      bf16  [rank_pad, M]      down factor transposed, smoothing folded in:
  *           ld[j, m] = L1[m, j] / scale[m]  (the page's X_hat L1 = x ld^T)
  *   ld32    fp32  [rank_pad, M]      same values as ld, for fp32 activations (may be NULL
@@ -142,7 +144,8 @@ svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq
  * re-orthonormalisation, one-sided Jacobi SVD of the small core), stores the
  * factors in bf16 with 1/scale folded into ld, forms the residual
  * R = ws - diag(scale) ld^T lu^T in fp32 against the stored (rounded) factors,
- * and quantises R per tensor (INT) or per 16-element block (NVFP4).
+ * and quantises R per tensor (INT), per 16-element block (NVFP4) or per
+ * 32-element block with a power-of-two scale (MXFP4).
  *
  * Synchronises `stream` before returning and returns SVDQ_EINVAL if scale held
  * a non-positive or non-finite entry, SVDQ_ETIMEOUT if a device wait ran out.
@@ -158,9 +161,9 @@ svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N
  * ("fake_quantize" grid for INT; NVFP4 block scales for NVFP4).
  *
  *   R        device fp32 [M, N] (ldR >= N)
- *   codes    INT int8 [N, M] / NVFP4 uint8 [N, M/2]   (K-major, as in svdq_weight)
- *   sf       NVFP4 128x4 layout of [N, M/16] (NULL for INT)
- *   w_scale  device fp32 scalar out: s_w (INT) or gs_w (NVFP4)
+ *   codes    INT int8 [N, M] / fp4 uint8 [N, M/2]   (K-major, as in svdq_weight)
+ *   sf       NVFP4 128x4 layout of [N, M/16], MXFP4 of [N, M/32] (NULL for INT)
+ *   w_scale  device fp32 scalar out: s_w (INT), gs_w (NVFP4) or 1 (MXFP4)
  */
 svdq_status svdq_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
                                    svdq_fmt fmt, void* codes, void* sf, float* w_scale,
@@ -186,9 +189,9 @@ svdq_status svdq_quantize_residual_workspace_size(int64_t M, int64_t N, svdq_fmt
  *            gs_x gs_w form. Ignored for INT.
  *   ld       nullable: bf16 [rank_pad, M] (or fp32 for fp32 x) down factor;
  *            NULL (or rank_pad = 0) skips the down-projection
- *   codes    out INT int8 [B, M] / NVFP4 uint8 [B, M/2]
- *   sf       out NVFP4 128x4 layout of [B, M/16]; NULL for INT
- *   act_scale out device fp32 scalar: s_x (INT) or the gs_x used (NVFP4)
+ *   codes    out INT int8 [B, M] / fp4 uint8 [B, M/2]
+ *   sf       out NVFP4 128x4 layout of [B, M/16], MXFP4 of [B, M/32]; NULL for INT
+ *   act_scale out device fp32 scalar: s_x (INT), the gs_x used (NVFP4) or 1 (MXFP4)
  *   down     out bf16 [B, 2*rank_pad]: x ld^T split as hi | lo with
  *            hi = bf16(v), lo = bf16(v - hi) of the fp32 dot product v
  */
@@ -231,7 +234,7 @@ svdq_status svdq_quantize_act_noalloc(const void* x, svdq_dtype x_dtype, int64_t
 /*
  * svdq_linear - the operator ("svdquant_linear" of both pages):
  *   Y = x ld^T lu^T + alpha * (Q(X_hat) . Q(R)) [+ bias]
- * with alpha = s_x * s_w (INT) or 1 / (gs_x * gs_w) (NVFP4). Runs the fused
+ * with alpha = s_x * s_w (INT), 1 / (gs_x * gs_w) (NVFP4) or 1 (MXFP4). Runs the fused
  * activation pass, then one tensor-core GEMM whose epilogue adds the low-rank
  * up-projection and the bias.
  *
@@ -282,8 +285,8 @@ svdq_status svdq_linear_ex(const svdq_weight* w, const void* x, svdq_dtype x_dty
  * up-projection and bias in its epilogue):
  *   Y = alpha * (codes . w->codes^T) + down_hi.lu^T + down_lo.lu^T [+ bias]
  *
- *   act_codes INT int8 [B, M] / NVFP4 uint8 [B, M/2] (from svdq_quantize_act)
- *   act_sf    NVFP4 128x4 scale layout of [B, M/16]; NULL for INT
+ *   act_codes INT int8 [B, M] / fp4 uint8 [B, M/2] (from svdq_quantize_act)
+ *   act_sf    NVFP4 128x4 scale layout of [B, M/16], MXFP4 of [B, M/32]; NULL for INT
  *   act_scale device fp32 scalar from svdq_quantize_act (s_x or gs_x)
  *   down      bf16 [B, 2 * w->rank_pad] from svdq_quantize_act (NVFP4: called with
  *             w_global_scale = w->w_scale); NULL iff rank == 0
