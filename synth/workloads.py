@@ -175,8 +175,8 @@ _SPECS = {
         rank=32, fmt="int", bits=4),
 }
 for _r in (32, 128):
-    for _fmt, _bits in (("int", 4), ("int", 8), ("nvfp4", 4)):
-        _tag = f"{_fmt}{_bits}" if _fmt == "int" else "nvfp4"
+    for _fmt, _bits in (("int", 4), ("int", 8), ("nvfp4", 4), ("mxfp4", 4)):
+        _tag = f"{_fmt}{_bits}" if _fmt == "int" else _fmt
         _SPECS[f"large_8192x12288x3072_{_tag}_r{_r}"] = dict(
             gen=_SPECS["large_8192x12288x3072_int4_r32"]["gen"], rank=_r, fmt=_fmt, bits=_bits)
 
