@@ -122,3 +122,25 @@ def test_linear_workspace_reused_across_shapes():
         assert rb.svdq_check_status() == rb.SVDQ_OK
         assert torch.equal(y_shared, y_fresh), f"call {i} (B={B})"
         assert_y_close(y_shared.cpu().numpy(), w.oracle_y(wl.x), f"call {i} B={B}")
+
+
+@pytest.mark.parametrize("B", [300, 2048])
+@pytest.mark.parametrize("fmt", ["int4", "int8", "nvfp4", "mxfp4"])
+def test_dependent_gemm_launch_equals_separate_calls(B, fmt):
+    """For B > 128, svdq_linear launches the pair GEMM as a dependent of the
+    activation pass (its prologue and first weight loads overlap the codes
+    kernel, its activation loads wait for it): the result must equal the two
+    stages called one after the other, bit for bit, on repeated calls."""
+    M, N, rank = 1536, 768, 32
+    wl = make_case(B, M, N, rank=rank, seed=B + 1, bias=True)
+    w = SyntheticWeight(M, N, rank, fmt, seed=3, scale=wl.scale)
+    x = x_tensor(wl)
+    scale = to_dev(wl.scale, torch.float32)
+    b = to_dev(wl.bias, torch.bfloat16)
+    gsw = w.w.w_scale if fmt == "nvfp4" else None
+    codes, sf, s, down = rb.svdq_quantize_act(x, scale, fmt, ld=w.w.ld, w_global_scale=gsw)
+    y_sep = rb.svdq_residual_linear(w.w, codes, sf, s, down, bias=b, out_dtype=torch.float32)
+    for _ in range(5):
+        y = rb.svdq_linear(w.w, x, bias=b, out_dtype=torch.float32)
+        assert torch.equal(y, y_sep)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
