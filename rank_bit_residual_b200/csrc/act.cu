@@ -352,7 +352,6 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
 template <typename TIn>
 __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
   constexpr int kTileK = kTileBytes / static_cast<int>(sizeof(TIn));
-  pdl_trigger();   // the GEMM launched after this kernel may start its weight loads now
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kWorkWarps];
   float* rcp = reinterpret_cast<float*>(smem);   // the unit's reciprocals

@@ -63,7 +63,7 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
   const int out = raw_i32 ? kOutI32 : (ydt == SVDQ_F32 ? kOutF32 : kOutBF16);
   cudaError_t err = cudaSuccess;
   const bool launched =
-      B > 128 ? launch_gemm_pair(kKind, out, args, act_codes, has_lr ? down2 : nullptr, w, pdl, stream, &err)
+      B > 128 ? launch_gemm_pair(kKind, out, args, act_codes, has_lr ? down2 : nullptr, w, stream, &err)
               : launch_gemm_skinny(kKind, out, args, act_codes, act_sf, has_lr ? down2 : nullptr, w, pdl, stream,
                                    &err);
   if (!launched) *bad_args = true;

@@ -196,7 +196,7 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
 
 // Host: the CTA-pair kernel (gemm_pair.cu); false if a tensor map cannot be encoded.
 bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
-                      const void* down2, const svdq_weight* w, bool pdl, cudaStream_t stream,
+                      const void* down2, const svdq_weight* w, cudaStream_t stream,
                       cudaError_t* err);
 
 }  // namespace svdq

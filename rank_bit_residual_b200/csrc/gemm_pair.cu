@@ -154,69 +154,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // Loads of stage `s` for step j of the tile at (m0, nt): the weight side
-      // (B codes and scales, lu) and the activation side (A codes and scales,
-      // down), with the expected byte count posted before the weight side.
-      auto load_stage = [&](int j, int s, int m0, int nt, bool wside, bool aside) {
-        uint8_t* st = smem + s * kStageBytes;
-        const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
-        const int n0 = nt + static_cast<int>(rank) * kHalf;
-        if (j >= ksteps) {
-          const int l = j - ksteps;
-          if (wside) {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
-            tma_load_2d_pair(st + kABytes, &tm_lu, fb, 64 * l, n0);
-          }
-          if (aside) tma_load_2d_pair(st, &tm_da, fb, 64 * l, m0);
-        } else if constexpr (kF4) {
-          // scale atoms: rows of 256 bytes, two rows per 512-byte atom
-          uint8_t* sfa_s = st + kABytes + kBBytes;
-          uint8_t* sfb_s = sfa_s + kSfaBytes;
-          const int a0 = kSfAtoms * j;
-          if (wside) {
-            if (rank == 0)
-              mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
-            tma_load_2d_pair(st + kABytes, &tm_b, fb, 128 * j, n0);
-            for (int rt = 0; rt < 2; ++rt)
-              tma_load_2d_pair(sfb_s + rt * kSfaBytes, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
-          }
-          if (aside) {
-            tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
-            tma_load_2d_pair(sfa_s, &tm_sfa, fb, 0, 2 * ((m0 / 128) * args.katoms + a0));
-          }
-        } else {
-          // A blocks then B blocks, 128 bytes of K each
-          if (wside) {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kKb * (kABytes + kBBytes));
-            for (int kb = 0; kb < kKb; ++kb)
-              tma_load_2d_pair(st + kKb * kABytes + kb * kBBytes, &tm_b, fb, kStageK * j + 128 * kb, n0);
-          }
-          if (aside)
-            for (int kb = 0; kb < kKb; ++kb)
-              tma_load_2d_pair(st + kb * kABytes, &tm_a, fb, kStageK * j + 128 * kb, m0);
-        }
-      };
-      auto tile_m0 = [&](int t) { return (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf; };
-      auto tile_nt = [&](int t) { return (t / tiles_m) * kTileN; };
-      // Launched as a dependent of the activation pass, the kernel may start
-      // before the codes exist: the first tile's first stages load their
-      // weight side now, the activation side after griddepcontrol.wait (a no-op
-      // when the launch was not a dependent one).
-      const int npre = pair < total ? min(kStages, ksteps) : 0;
-      for (int j = 0; j < npre; ++j) load_stage(j, j, tile_m0(pair), tile_nt(pair), true, false);
-      pdl_wait();
-      for (int j = 0; j < npre; ++j) load_stage(j, j, tile_m0(pair), tile_nt(pair), false, true);
       uint32_t it = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
-        const int m0 = tile_m0(t), nt = tile_nt(t);
+        const int m0 = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf;
+        const int nt = (t / tiles_m) * kTileN;
+        const int n0 = nt + static_cast<int>(rank) * kHalf;
         for (int j = 0; j < steps_per_tile && ok; ++j, ++it) {
-          if (t == pair && j < npre) continue;   // issued above
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           ok = mbar_wait(&empty_bar[s], ph ^ 1, status, &abort_sh);
           if (!ok) break;
-          load_stage(j, s, m0, nt, true, true);
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
+          if (j >= ksteps) {
+            const int l = j - ksteps;
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
+            tma_load_2d_pair(st, &tm_da, fb, 64 * l, m0);
+            tma_load_2d_pair(st + kABytes, &tm_lu, fb, 64 * l, n0);
+          } else if constexpr (kF4) {
+            if (rank == 0)
+              mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
+            tma_load_2d_pair(st, &tm_a, fb, 128 * j, m0);
+            tma_load_2d_pair(st + kABytes, &tm_b, fb, 128 * j, n0);
+            // scale atoms: rows of 256 bytes, two rows per 512-byte atom
+            uint8_t* sfa_s = st + kABytes + kBBytes;
+            uint8_t* sfb_s = sfa_s + kSfaBytes;
+            const int a0 = kSfAtoms * j;
+            tma_load_2d_pair(sfa_s, &tm_sfa, fb, 0, 2 * ((m0 / 128) * args.katoms + a0));
+            for (int rt = 0; rt < 2; ++rt)
+              tma_load_2d_pair(sfb_s + rt * kSfaBytes, &tm_sfb, fb, 0, 2 * ((nt / 128 + rt) * args.katoms + a0));
+          } else {
+            // A blocks then B blocks, 128 bytes of K each
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kKb * (kABytes + kBBytes));
+            for (int kb = 0; kb < kKb; ++kb) {
+              tma_load_2d_pair(st + kb * kABytes, &tm_a, fb, kStageK * j + 128 * kb, m0);
+              tma_load_2d_pair(st + kKb * kABytes + kb * kBBytes, &tm_b, fb, kStageK * j + 128 * kb, n0);
+            }
+          }
         }
       }
       // wait for the MMA's release of the last stages, so no commit arrival
@@ -326,7 +301,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int q = warp & 3;                         // TMEM lane quarter
     const int h = (warp - 2) >> 2;                  // column half of the tile
     const int r_in = q * 32 + lane;
-    pdl_wait();   // s_x (gs_x) comes from the activation pass
     const float alpha = epilogue_alpha<kKind, kOut>(args);
     const bool sep_lr = kKind == kKindInt && kOut != kOutI32 && lr_steps > 0;
     const uint32_t acc_empty_even = mapa_shared(smem_u32(&acc_empty_bar), 0);
@@ -400,28 +374,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   }
 }
 
-// pdl: launched as a programmatic dependent of the kernel before it on the
-// stream (the activation pass), so its prologue and first weight loads
-// overlap that kernel's tail.
 template <int kKind, int kOut>
-cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int grid, bool pdl, cudaStream_t st) {
+cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int grid, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(PairCfg<kKind>::kStages) * PairCfg<kKind>::kStageBytes + 1024;
   cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<kKind, kOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kPairThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kKind, kOut>, maps[0], maps[1], maps[2], maps[3], maps[4],
-                            maps[5], args);
+  gemm_pair_kernel<kKind, kOut><<<grid, kPairThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                    maps[4], maps[5], args);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -429,7 +391,7 @@ cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int g
 // Builds the pair kernel's tensor maps and launches it; returns false (and
 // launches nothing) if a map cannot be encoded.
 bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
-                      const void* down2, const svdq_weight* w, bool pdl, cudaStream_t stream,
+                      const void* down2, const svdq_weight* w, cudaStream_t stream,
                       cudaError_t* err) {
   *err = cudaSuccess;
   const int64_t M = args.M, N = args.N, B = args.B;
@@ -461,15 +423,15 @@ bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_c
   const int64_t tiles = ceil_div(B, 2 * kHalf) * ceil_div(N, kTileN);
   const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, num_sms() / 2));
   if (kind == kKindInt) {
-    if (out == kOutI32) *err = launch_pair_one<kKindInt, kOutI32>(maps, args, grid, pdl, stream);
-    else if (out == kOutF32) *err = launch_pair_one<kKindInt, kOutF32>(maps, args, grid, pdl, stream);
-    else *err = launch_pair_one<kKindInt, kOutBF16>(maps, args, grid, pdl, stream);
+    if (out == kOutI32) *err = launch_pair_one<kKindInt, kOutI32>(maps, args, grid, stream);
+    else if (out == kOutF32) *err = launch_pair_one<kKindInt, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindInt, kOutBF16>(maps, args, grid, stream);
   } else if (kind == kKindMxfp4) {
-    if (out == kOutF32) *err = launch_pair_one<kKindMxfp4, kOutF32>(maps, args, grid, pdl, stream);
-    else *err = launch_pair_one<kKindMxfp4, kOutBF16>(maps, args, grid, pdl, stream);
+    if (out == kOutF32) *err = launch_pair_one<kKindMxfp4, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindMxfp4, kOutBF16>(maps, args, grid, stream);
   } else {
-    if (out == kOutF32) *err = launch_pair_one<kKindNvfp4, kOutF32>(maps, args, grid, pdl, stream);
-    else *err = launch_pair_one<kKindNvfp4, kOutBF16>(maps, args, grid, pdl, stream);
+    if (out == kOutF32) *err = launch_pair_one<kKindNvfp4, kOutF32>(maps, args, grid, stream);
+    else *err = launch_pair_one<kKindNvfp4, kOutBF16>(maps, args, grid, stream);
   }
   return true;
 }

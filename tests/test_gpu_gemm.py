@@ -126,11 +126,10 @@ def test_linear_workspace_reused_across_shapes():
 
 @pytest.mark.parametrize("B", [300, 2048])
 @pytest.mark.parametrize("fmt", ["int4", "int8", "nvfp4", "mxfp4"])
-def test_dependent_gemm_launch_equals_separate_calls(B, fmt):
-    """For B > 128, svdq_linear launches the pair GEMM as a dependent of the
-    activation pass (its prologue and first weight loads overlap the codes
-    kernel, its activation loads wait for it): the result must equal the two
-    stages called one after the other, bit for bit, on repeated calls."""
+def test_large_batch_linear_equals_separate_stages(B, fmt):
+    """For B > 128, svdq_linear (activation pass, then the pair GEMM on the
+    workspace's codes) must equal the two stages called one after the other
+    through their own entry points, bit for bit, on repeated calls."""
     M, N, rank = 1536, 768, 32
     wl = make_case(B, M, N, rank=rank, seed=B + 1, bias=True)
     w = SyntheticWeight(M, N, rank, fmt, seed=3, scale=wl.scale)
