@@ -114,7 +114,7 @@ def main(argv: Optional[Sequence[str]] = None) -> int:
     ap.add_argument("--workload", default="dit_attn_4096x3072x3072_int4")
     ap.add_argument("--rows", type=int, default=None, help="keep only the first rows of x")
     ap.add_argument("--ranks", default="0,1,2,3,4,5,6,16,32")
-    ap.add_argument("--fmt", default=None, help="override the workload's format (int4, int8, nvfp4)")
+    ap.add_argument("--fmt", default=None, help="override the workload's format (int4, int8, nvfp4, mxfp4)")
     ap.add_argument("--alphas", default="0.25,0.5,0.75,0.9",
                     help="migration strengths to compare at the largest rank (empty: skip)")
     args = ap.parse_args(argv)
@@ -126,7 +126,7 @@ def main(argv: Optional[Sequence[str]] = None) -> int:
     x = torch.from_numpy(wl.x).to(dev).to(tdt)
     W = torch.from_numpy(wl.W).to(dev).to(torch.bfloat16 if wl.w_dtype == "bf16" else torch.float32)
     scale = torch.from_numpy(wl.scale).to(dev)
-    fmt = args.fmt or (wl.fmt if wl.fmt == "nvfp4" else f"int{wl.bits}")
+    fmt = args.fmt or (wl.fmt if wl.fmt != "int" else f"int{wl.bits}")
     ranks = [int(r) for r in args.ranks.split(",")]
     res = ablation(x, W, scale, ranks, fmt=fmt)
     res["workload"] = args.workload
