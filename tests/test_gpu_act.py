@@ -178,3 +178,49 @@ def test_mxfp4_down_projection_is_unscaled(B, M, rank):
     want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
     assert g.item() == 1.0
     assert rel_fro(d[:, :rp] + d[:, rp:], want) <= 2e-5
+
+
+def _mx_edge_rows():
+    """32-element blocks at the MXFP4 encoder's boundaries: zero and negative-zero
+    blocks, block maxima exactly at and just below powers of two (the exponent's
+    floor and the clip to 6 2^X), e2m1 ties, huge and tiny exponents, a
+    subnormal block, mixed signs. Every value is bf16-representable."""
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -2.5, -5.0, 4.0] * 3)[:32]
+    blocks = [
+        np.zeros(32),
+        -np.zeros(32),
+        np.r_[4.0, np.linspace(-3.0, 3.0, 31)],
+        np.r_[8.0, -np.linspace(0.0, 7.0, 31)],
+        np.r_[7.96875, np.linspace(-7.0, 7.0, 31)],           # amax just below 8: X = 0, clips to 6
+        ties,
+        np.r_[2.0 ** 120, np.full(31, 2.0 ** 117)],
+        np.r_[-(2.0 ** -120), np.full(31, 2.0 ** -124)],
+        np.full(32, 1.0e-39),                                  # subnormal block
+        np.r_[6.0, -6.0, np.full(30, 0.125)],
+    ]
+    row = np.concatenate(blocks)
+    return to_bf16(np.stack([row, -row, row[::-1].copy(), np.roll(row, 32)]).astype(np.float32))
+
+
+@pytest.mark.parametrize("B", [4, 256])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_mxfp4_encoder_edges(B, dtype):
+    x = np.tile(_mx_edge_rows(), (B // 4, 1))
+    M = x.shape[1]
+    ones = np.ones(M, np.float32)
+    xt = to_dev(x, torch.float32 if dtype == "f32" else torch.bfloat16)
+    codes, sf, g, _ = rb.svdq_quantize_act(xt, to_dev(ones, torch.float32), "mxfp4")
+    c_o, sf_o = omx.quantize(ocodes.smooth_fp32(x, ones))
+    assert g.item() == 1.0
+    assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
+    assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
+
+
+def test_mxfp4_residual_encoder_edges():
+    R = np.ascontiguousarray(_mx_edge_rows().T)          # [M, 4]: the blocks run along M
+    R = np.ascontiguousarray(np.tile(R, (1, 4)))           # N = 16
+    codes, sf, g = rb.svdq_quantize_residual(to_dev(R, torch.float32), "mxfp4")
+    c_o, sf_o = omx.quantize(np.ascontiguousarray(R.T))
+    assert g.item() == 1.0
+    assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
+    assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
