@@ -224,3 +224,37 @@ def test_mxfp4_residual_encoder_edges():
     assert g.item() == 1.0
     assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
     assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
+
+
+def _nv_edge_rows():
+    """16-element blocks at the NVFP4 encoder's boundaries for a given gs = 1:
+    zero and negative-zero blocks, e2m1 ties after the ue4m3 scale, block
+    maxima whose scale amax / 6 lands on, between and below ue4m3 values (the
+    smallest subnormal 2^-9 and under it), the ue4m3 maximum 448 (amax 2688),
+    mixed signs."""
+    blocks = [
+        np.zeros(16),
+        -np.zeros(16),
+        np.r_[6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -2.5, -3.5, -5.0, 4.0, -6.0],
+        np.r_[2688.0, np.linspace(-2000.0, 2000.0, 15)],
+        np.r_[6.0 * 2.0 ** -9, np.full(15, 2.0 ** -10)],
+        np.r_[3.0 * 2.0 ** -9, np.full(15, 2.0 ** -11)],      # amax / 6 below the smallest scale
+        np.r_[6.5, np.linspace(-6.0, 6.0, 15)],                # amax / 6 between two ue4m3 values
+        np.r_[-100.0, np.full(15, 33.0)],
+    ]
+    row = np.concatenate(blocks)
+    return to_bf16(np.stack([row, -row, row[::-1].copy(), np.roll(row, 16)]).astype(np.float32))
+
+
+@pytest.mark.parametrize("B", [4, 256])
+def test_nvfp4_encoder_edges_with_given_global_scale(B):
+    x = np.tile(_nv_edge_rows(), (B // 4, 1))
+    M = x.shape[1]
+    ones = np.ones(M, np.float32)
+    gs = to_dev(np.array([1.0], np.float32), torch.float32)
+    codes, sf, g, _ = rb.svdq_quantize_act(to_dev(x, torch.float32), to_dev(ones, torch.float32), "nvfp4",
+                                           act_global_scale=gs)
+    c_o, sf_o, g_o = onv.quantize(ocodes.smooth_fp32(x, ones), gs=np.float32(1.0))
+    assert np.float32(g.item()) == np.float32(g_o)
+    assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
+    assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
