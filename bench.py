@@ -170,8 +170,9 @@ class ClockSampler:
 
 
 def cpu_oracle_rate(wl, budget_s=12.0, rows=None):
-    """Time the float64 oracle (prepared-operand linear) on the host cores over a
-    bounded sample; returns (TOPS, seconds, cores, sample description)."""
+    """Time the float64 oracle (prepared-operand linear, in the workload's own
+    format) on the host cores over a bounded sample; returns (TOPS, seconds,
+    cores, sample description)."""
     import numpy as np
     from oracle import codes as ocodes
     from oracle import prepared as oprep
@@ -186,21 +187,44 @@ def cpu_oracle_rate(wl, budget_s=12.0, rows=None):
     rows = rows or min(B, 512)
     ld = (rng.standard_normal((M, r)) * 0.01).astype(np.float64)
     L2 = (rng.standard_normal((r, N)) * 0.01).astype(np.float64)
-    cw = rng.integers(-7, 8, (N, M)).astype(np.int8)
     x = wl.x[:rows]
+    if wl.fmt == "int":
+        cw = rng.integers(-7, 8, (N, M)).astype(np.int8)
+
+        def once():
+            q, s_x, _ = ocodes.act_codes_int_fp32(x, wl.scale, wl.bits)
+            oprep.linear_int(x, ld, L2, q, s_x, cw, 0.01)
+        what = "fp32-mode codes + float64 integer product + low-rank"
+    elif wl.fmt == "nvfp4":
+        from oracle import nvfp4 as onv
+        cw = rng.integers(0, 16, (N, M)).astype(np.uint8)
+        sfw = rng.integers(0x20, 0x48, (N, M // 16)).astype(np.uint8)
+
+        def once():
+            ca, sa, gx = onv.quantize(ocodes.smooth_fp32(x, wl.scale))
+            oprep.linear_nvfp4(x, ld, L2, ca, sa, gx, cw, sfw, 448.0)
+        what = "NVFP4 block quantisation + float64 block-scaled product + low-rank"
+    else:
+        from oracle import mxfp4 as omx
+        cw = rng.integers(0, 16, (N, M)).astype(np.uint8)
+        sfw = rng.integers(121, 127, (N, M // 32)).astype(np.uint8)
+
+        def once():
+            ca, sa = omx.quantize(ocodes.smooth_fp32(x, wl.scale))
+            oprep.linear_mxfp4(x, ld, L2, ca, sa, cw, sfw)
+        what = "MXFP4 block quantisation + float64 block-scaled product + low-rank"
     t0 = time.perf_counter()
     ops = 0.0
     reps = 0
     while True:
-        q, s_x, _ = ocodes.act_codes_int_fp32(x, wl.scale, wl.bits)
-        oprep.linear_int(x, ld, L2, q, s_x, cw, 0.01)
+        once()
         ops += workload_ops(rows, M, N, r)
         reps += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    sample = (f"{reps} pass(es) of the oracle's prepared-operand linear (fp32-mode codes + float64 "
-              f"integer product + low-rank) over {rows} of {B} rows of {wl.name}")
+    sample = (f"{reps} pass(es) of the oracle's prepared-operand linear ({what}) over {rows} of {B} rows "
+              f"of {wl.name}")
     return ops / dt / 1e12, dt, cores, sample
 
 
