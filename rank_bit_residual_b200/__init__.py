@@ -6,6 +6,10 @@ libsvdq.so is missing or no GPU is present, the calls raise.
 
     w = svdq_prepare(W, scale, rank, fmt="int4")          # one-time split on the GPU
     y = svdq_linear(w, x, bias=None, out_dtype=torch.bfloat16)
+    y = svdq_linear_chain([w1, w2], x)                     # consecutive layers, PDL-chained
+
+Formats: "int2" .. "int8" (per-tensor grid), "nvfp4" (ue4m3 scales per 16
+elements and an fp32 global scale), "mxfp4" (E8M0 scales per 32 elements).
 
 Conventions follow "SVDQuant Smoothing, Low-rank and Residual Quantization":
 x[B, M] @ W[M, N], positive finite scale[M], rank a Python int in
