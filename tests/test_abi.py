@@ -98,3 +98,23 @@ def test_linear_ex_rejects_unknown_flags(lib):
     st = lib.svdq_linear_ex(ctypes.byref(w), None, 0, 1, 64, None, None, None, 0, 64, None, 0,
                             ctypes.c_uint32(2), None)
     assert st == rb.SVDQ_EINVAL
+
+
+def test_no_cpu_path():
+    """Every operator call takes CUDA tensors only: host tensors raise instead of
+    being computed on the CPU, and a missing library raises on load."""
+    import torch
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rb.svdq_quantize_act(x, torch.ones(64), "mxfp4")
+    with pytest.raises(ValueError):
+        rb.svdq_smooth_scale(x, torch.zeros((64, 32)), 0.5)
+    with pytest.raises(ValueError):
+        rb.svdq_prepare(torch.zeros((64, 32)), torch.ones(64), 4, "nvfp4")
+    saved = rb._lib
+    try:
+        rb._lib = None
+        with pytest.raises(ImportError):
+            rb.load_library("/nonexistent/libsvdq.so")
+    finally:
+        rb._lib = saved
