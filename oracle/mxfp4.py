@@ -18,9 +18,11 @@ configuration, quantises the residual branch and the activations "per_block" as
 * storage as NVFP4: element 2j in the low nibble of byte j; the scales in the
   128x4 layout of oracle.nvfp4 over [rows, K/32].
 
-Division by 2^X is exact in both float64 and fp32 (for X in [-126, 127]), so the
-fp32 evaluation order only enters through the smoothed activation fl32(x * r_k)
-(oracle.codes.smooth_fp32) that the codes are taken of.
+The elements are a / div, with div the per-column smoothing scale for the
+activation (X_hat = x / scale) and 1 for the residual. The block maximum is
+rounded once to fp32, amax_b = fl32(max |a / div|) (the largest IEEE quotient),
+and X is taken of it; every code is the exact round-to-nearest-even of
+a 2^-X / div onto the e2m1 grid (|a| 2^-X and mid * div are exact doubles).
 """
 
 from __future__ import annotations
@@ -49,18 +51,22 @@ def block_exponent(amax) -> np.ndarray:
     return np.where(a > 0, x, -127)
 
 
-def quantize(z):
-    """MXFP4 codes of z[rows, K] (K a multiple of 32): (codes uint8 [rows, K] one
-    nibble per element, scales uint8 [rows, K/32] E8M0 bytes)."""
-    z = np.asarray(z, dtype=np.float64)
-    rows, K = z.shape
+def quantize(a, div=None):
+    """MXFP4 codes of the elements a[rows, K] / div[K] (div None: 1), K a multiple of
+    32: (codes uint8 [rows, K] one nibble per element, scales uint8 [rows, K/32]
+    E8M0 bytes)."""
+    a32 = np.asarray(a, dtype=np.float32)
+    rows, K = a32.shape
     if K % BLOCK:
         raise ValueError("K must be a multiple of 32")
-    zb = z.reshape(rows, K // BLOCK, BLOCK)
-    X = block_exponent(np.max(np.abs(zb), axis=2))
-    scaled = zb * np.ldexp(1.0, -X)[:, :, None]   # exact
-    codes = _nv.e2m1_encode(scaled).reshape(rows, K)
-    return codes, (X + 127).astype(np.uint8)
+    amax_b = _nv._block_amax_fp32(a32, div, BLOCK)
+    X = block_exponent(amax_b)
+    p = np.abs(a32.astype(np.float64)).reshape(rows, K // BLOCK, BLOCK) * \
+        np.ldexp(1.0, -X)[:, :, None]                              # exact
+    c = 1.0 if div is None else np.asarray(div, dtype=np.float32).astype(np.float64).reshape(
+        1, K // BLOCK, BLOCK)
+    codes = _nv.e2m1_encode_ratio(p, c, a32.reshape(rows, K // BLOCK, BLOCK) < 0)
+    return codes.reshape(rows, K), (X + 127).astype(np.uint8)
 
 
 def dequantize(codes, sf) -> np.ndarray:

@@ -24,11 +24,18 @@ reading:
 The recipe (gs and sf above) is parity unpinned by the pages: no page prints
 an NVFP4 example. It is pinned by the format tables and by consistency checks.
 
-Two evaluation orders are provided: ``exact`` (float64 everywhere) and
-``fp32`` (one IEEE fp32 op per step, the order GPU codes are compared in):
-  amax_t = max|z|;  gs = fl32(2688 / amax_t)  (unless given)
+Evaluation order. Every stored scalar carries the one fp32 rounding named
+below (the activation global scale, a block maximum, the block scale value,
+the encode scale); every code is the exact round-to-nearest-even of its real
+value onto the e2m1 grid. The elements are a / div, with div the per-column
+smoothing scale of the activation (X_hat = x / scale) and 1 for the residual:
+  amax_t = fl32(max|a / div|);  gs = fl32(2688 / amax_t)  (unless given)
+  amax_b = fl32(max over the block of |a / div|)
   sfv = fl32(fl32(amax_b / 6) * gs);  sf = ue4m3_rne(sfv)
-  enc = fl32(gs / dec(sf));  code = e2m1_rne(fl32(z * enc))   (0 when sf == 0)
+  enc = fl32(gs / dec(sf));  code = e2m1_rne(a * enc / div)   (0 when sf == 0)
+The e2m1 decision compares |a| enc with mid * div for the grid midpoints mid;
+both products are exact in float64 (24 + 24 and 3 + 24 significant bits), so
+it is exact. ``mode="exact"`` instead keeps every scalar in float64.
 """
 
 from __future__ import annotations
@@ -105,34 +112,67 @@ def global_scale(amax, mode: str = "fp32"):
     return 1.0 if a == 0 else GS_NUMERATOR / a
 
 
-def quantize(z, gs=None, mode: str = "fp32"):
-    """NVFP4 codes of z[rows, K] with 16-element blocks along K.
+def e2m1_encode_ratio(p, c, negative) -> np.ndarray:
+    """e2m1 nibble of the real value +-p / c (p >= 0, c > 0), round to nearest even,
+    saturating at 6, zero stored as +0. Exact when p and mid * c are exact doubles."""
+    p = np.asarray(p, dtype=np.float64)
+    c = np.broadcast_to(np.asarray(c, dtype=np.float64), p.shape)
+    mids = 0.5 * (_E2M1_GRID[:-1] + _E2M1_GRID[1:])          # .25 .75 1.25 1.75 2.5 3.5 5
+    idx = np.zeros(p.shape, dtype=np.int64)
+    for i, mid in enumerate(mids):
+        q = mid * c
+        # above the midpoint between grid points i and i + 1, or on it when i + 1 is even
+        up = (p > q) | ((p == q) & ((i + 1) % 2 == 0))
+        idx = np.where(up, i + 1, idx)
+    sign = (np.asarray(negative) & (idx != 0)).astype(np.uint8) << 3
+    return (sign | idx.astype(np.uint8)).astype(np.uint8)
+
+
+def _block_amax_fp32(a32: np.ndarray, div, block: int) -> np.ndarray:
+    """fl32 of the block maxima of |a / div| (max of the IEEE fp32 quotients)."""
+    rows, K = a32.shape
+    q = np.abs(a32) if div is None else np.abs(a32) / np.asarray(div, dtype=np.float32)[None, :]
+    return np.max(q.astype(np.float32).reshape(rows, K // block, block), axis=2)
+
+
+def quantize(a, gs=None, mode: str = "fp32", div=None):
+    """NVFP4 codes of the elements a[rows, K] / div[K] (div None: 1) with
+    16-element blocks along K.
 
     Returns (codes uint8 [rows, K] one nibble per element, sf uint8 [rows, K/16]
     ue4m3 bytes, gs). K must be a multiple of 16.
     """
-    if mode == "fp32":
-        z = np.asarray(z, dtype=np.float32)
-        ft = np.float32
-    else:
-        z = np.asarray(z, dtype=np.float64)
-        ft = np.float64
-    rows, K = z.shape
+    rows, K = np.shape(a)
     if K % BLOCK:
         raise ValueError("K must be a multiple of 16")
+    if mode != "fp32":
+        z = np.asarray(a, dtype=np.float64)
+        if div is not None:
+            z = z / np.asarray(div, dtype=np.float64)[None, :]
+        if gs is None:
+            gs = global_scale(np.max(np.abs(z)) if z.size else 0.0, "exact")
+        zb = z.reshape(rows, K // BLOCK, BLOCK)
+        sf = ue4m3_encode(np.max(np.abs(zb), axis=2) / 6.0 * gs)
+        d = e4m3_decode(sf)
+        enc = np.where(d > 0, gs / np.where(d > 0, d, 1.0), 0.0)
+        return e2m1_encode(zb * enc[:, :, None]).reshape(rows, K), sf, gs
+    a32 = np.asarray(a, dtype=np.float32)
+    amax_b = _block_amax_fp32(a32, div, BLOCK)
     if gs is None:
-        gs = global_scale(np.max(np.abs(z)) if z.size else 0.0, mode)
-    gs = ft(gs)
-    zb = z.reshape(rows, K // BLOCK, BLOCK)
-    amax_b = np.max(np.abs(zb), axis=2)
-    sfv = ((amax_b / ft(6.0)).astype(ft) * gs).astype(ft)
+        gs = global_scale(np.max(amax_b) if amax_b.size else 0.0, "fp32")
+    gs = np.float32(gs)
+    sfv = ((amax_b / np.float32(6.0)).astype(np.float32) * gs).astype(np.float32)
     sf = ue4m3_encode(sfv.astype(np.float64))
-    d = e4m3_decode(sf).astype(ft)
+    d = e4m3_decode(sf).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        enc = np.where(d > 0, (gs / np.where(d > 0, d, ft(1.0))).astype(ft), ft(0.0)).astype(ft)
-    scaled = (zb * enc[:, :, None]).astype(ft)
-    codes = e2m1_encode(scaled.astype(np.float64)).reshape(rows, K)
-    return codes, sf, gs
+        enc = np.where(d > 0, (gs / np.where(d > 0, d, np.float32(1.0))).astype(np.float32),
+                       np.float32(0.0)).astype(np.float32)
+    p = np.abs(a32.astype(np.float64)).reshape(rows, K // BLOCK, BLOCK) * \
+        enc.astype(np.float64)[:, :, None]
+    c = 1.0 if div is None else np.asarray(div, dtype=np.float32).astype(np.float64).reshape(
+        1, K // BLOCK, BLOCK)
+    codes = e2m1_encode_ratio(p, c, a32.reshape(rows, K // BLOCK, BLOCK) < 0)
+    return codes.reshape(rows, K), sf, gs
 
 
 def dequantize(codes, sf, gs) -> np.ndarray:

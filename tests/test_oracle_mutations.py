@@ -7,6 +7,7 @@ import pytest
 import oracle.svdquant as sq
 import oracle.nvfp4 as nv
 import oracle.prepared as pp
+import oracle.codes as oc
 from tests import test_oracle_svdquant as T1
 from tests import test_oracle_codes as T2
 
@@ -94,6 +95,35 @@ def _e2m1_ties_away(v):
     return (((v < 0) & (idx != 0)).astype(np.uint8) << 3) | idx
 
 
+def _quotient_reciprocal_multiply(a, d1, d2):
+    a32 = np.asarray(a, np.float32)
+    c = ((np.float32(1) / np.asarray(d1, np.float32)).astype(np.float32) *
+         np.float32(np.float32(1) / np.float32(d2))).astype(np.float32)
+    return np.rint((a32 * c).astype(np.float32)).astype(np.float64)
+
+
+def _quotient_two_divisions(a, d1, d2):
+    a32 = np.asarray(a, np.float32)
+    xs = (a32 / np.asarray(d1, np.float32)).astype(np.float32)
+    return np.rint((xs / np.float32(d2)).astype(np.float32)).astype(np.float64)
+
+
+def _quotient_half_away(a, d1, d2):
+    t = np.asarray(a, np.float64) / (np.asarray(d1, np.float64) * np.float64(d2))
+    return np.sign(t) * np.floor(np.abs(t) + 0.5)
+
+
+def _e2m1_ratio_ties_away(p, c, negative):
+    p = np.asarray(p, np.float64)
+    c = np.broadcast_to(np.asarray(c, np.float64), p.shape)
+    mids = 0.5 * (nv._E2M1_GRID[:-1] + nv._E2M1_GRID[1:])
+    idx = np.zeros(p.shape, np.int64)
+    for i, mid in enumerate(mids):
+        idx = np.where(p >= mid * c, i + 1, idx)
+    sign = (np.asarray(negative) & (idx != 0)).astype(np.uint8) << 3
+    return (sign | idx.astype(np.uint8)).astype(np.uint8)
+
+
 def _pack_swapped(codes):
     c = np.asarray(codes, dtype=np.uint8)
     return (c[:, 1::2] & 0xF) | ((c[:, 0::2] & 0xF) << 4)
@@ -121,6 +151,12 @@ MUTATIONS = [
     (sq, "svdquant_linear", _linear_quantized_low_rank, [T1.test_svdquant_linear_hand_case]),
     (nv, "e2m1_encode", _e2m1_ties_away, [T2.test_e2m1_rounding_ties]),
     (nv, "pack_nibbles", _pack_swapped, [T2.test_pack_nibbles_order]),
+    (oc, "_exact_rne_quotient", _quotient_reciprocal_multiply,
+     [T2.test_codes_decided_exactly_where_fp32_orders_differ]),
+    (oc, "_exact_rne_quotient", _quotient_two_divisions,
+     [T2.test_codes_decided_exactly_where_fp32_orders_differ]),
+    (oc, "_exact_rne_quotient", _quotient_half_away, [T2.test_codes_hand_ties]),
+    (nv, "e2m1_encode_ratio", _e2m1_ratio_ties_away, [T2.test_e2m1_ratio_ties_go_to_even]),
     (nv, "sf_offset", _sf_offset_transposed, [T2.test_sf_layout_points_and_bijection]),
     (pp, "int_product", _int_product_transposed, [T1.test_integer_product_matches_brute_force]),
 ]
