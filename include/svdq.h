@@ -216,13 +216,19 @@ svdq_status svdq_quantize_act_workspace_size(int64_t B, int64_t M, svdq_fmt fmt,
  *
  * Scratch lives in one fixed 8 MiB device array inside the library, which
  * every GPU that loads the library holds until the process exits. The first
- * call on a device looks up the array's address on that device; make that
- * call before any stream capture. All calls share the array and it keeps the
- * last call's contents: every scratch word a call reads is written by that call
- * first, so nothing needs clearing, but calls that overlap on the GPU (other
- * streams or other host threads) race on it. Shapes whose scratch does not fit
- * in 8 MiB even with the K split reduced - B * rank_pad of 2^21 or more
- * - return SVDQ_EWORKSPACE and launch nothing.
+ * call on a device looks up the array's address on that device, once per
+ * process (a context torn down and made again, e.g. by cudaDeviceReset, is not
+ * detected); make that call before any stream capture. All calls share the
+ * array and it keeps the last call's contents: every scratch word a call reads
+ * is written by that call first, so nothing needs clearing, but calls that
+ * overlap on the GPU (other streams or other host threads) race on it.
+ * The plan is svdq_quantize_act's, with the K split (column ranges per row
+ * block) halved until the scratch fits: 4 * B * rank_pad * ksplit bytes of
+ * partial down tiles plus the partial maxima, 4 * grid bytes rounded up to 256,
+ * plus 256. At ksplit = 1 that limits B * rank_pad to a little under 2^21 (for
+ * example B = 8192 at rank_pad 128 fits, B = 16384 at rank_pad 128 does not).
+ * Larger shapes return SVDQ_EWORKSPACE and launch nothing. The argument checks
+ * and their status codes are those of svdq_quantize_act.
  */
 svdq_status svdq_quantize_act_noalloc(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
                                       int64_t ldx, const float* scale, svdq_fmt fmt,

@@ -19,18 +19,21 @@
 //                 column maxima of |x| from registers, and runs the unit's
 //                 down-projection x ld^T with warp-level MMAs from padded
 //                 shared-memory tiles; it writes one partial maximum per CTA
-//                 and one partial down tile per unit. Since fl(a r) is monotone
-//                 in a, the tensor maximum of |X_hat| is max_k fl(colmax_k r_k).
+//                 and one partial down tile per unit. Since fl(a / c) is
+//                 monotone in a, the tensor maximum of |X_hat|, rounded to
+//                 fp32, is max_k fl(colmax_k / scale_k) (IEEE quotients).
 //   codes kernel  takes the per-tensor scale from the partial maxima, writes
 //                 the codes from a second read of x (from L2 when x fits
 //                 there) and sums each row block's partial down tiles in split
 //                 order into bf16 hi | lo.
 //
-// fp32 evaluation order (the one the oracle's fp32 code mode repeats): the
-// per-element divisions of the definition are multiplies by correctly rounded
-// reciprocals, r_k = fl(1 / scale_k) once per column and u = fl(1 / s) once
-// per tensor: X_hat = fl(x r_k), INT code = rint(fl(x c_k)) with the per-column
-// constant c_k = fl(r_k u).
+// Rounding: the stored scalars carry one fp32 rounding each (s = fl(m / qmax)
+// with m the fp32 maximum above; the NVFP4 / MXFP4 block maxima and scales),
+// and every code is the exactly rounded value of its real quotient. The codes
+// kernel estimates each quotient with multiplies by the reciprocals
+// r_k = fl(1 / scale_k) and u = fl(1 / s) (INT: rint(fl(x c_k)), c_k =
+// fl(r_k u)) and decides the rare elements next to a rounding boundary again
+// in exact arithmetic (encode.cuh).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -149,7 +152,7 @@ __device__ __forceinline__ uint32_t max_word(uint32_t m, uint32_t w) {
 //                 (i < 4): a warp moves two whole 256-byte row segments;
 //   column maxima warp w scans 32-bit words 4 w .. 4 w + 3 of rows l / 4 + 8 i
 //                 (lane l, i < 16; conflict-free under the swizzle), the eight
-//                 row slices meet by shuffles, and each column's fl(colmax r_k)
+//                 row slices meet by shuffles, and each column's fl(colmax / scale_k)
 //                 is taken once;
 //   down tile     one thread issues the sub-chunk's tcgen05 MMAs (M = 128 rows,
 //                 N = rank_pad, kind::f16 for bf16 x, kind::tf32 for fp32 x)
@@ -274,8 +277,8 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
       if (rp > 0 && c > 0) mbar_wait_warp(&mma_bar[(gc - 1) % stages], ((gc - 1) / stages) & 1, a.status, &abort_sh);
       issue(c + stages - 1);
       {
-        // max_k fl(colmax_k r_k): fl(a r) is monotone in a, so the column maximum
-        // of |x| is scaled once per column
+        // max_k fl(colmax_k / scale_k): fl(a / c) is monotone in a, so the
+        // column maximum of |x| is divided once per column
         uint32_t m = 0u;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -291,12 +294,12 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
             const int e = 2 * wi + rs;
             if (c_lo + c * kSubCols + e < c_hi) {
               const float v = __uint_as_float(rs == 0 ? m << 16 : m & 0xFFFF0000u);
-              run = fmaxf(run, __fmul_rn(v, __frcp_rn(sc[e])));
+              run = fmaxf(run, __fdiv_rn(v, sc[e]));
             }
           }
         } else {
           if (rs == 0 && c_lo + c * kSubCols + wi < c_hi)
-            run = fmaxf(run, __fmul_rn(__uint_as_float(m), __frcp_rn(sc[wi])));
+            run = fmaxf(run, __fdiv_rn(__uint_as_float(m), sc[wi]));
         }
       }
     }
@@ -419,7 +422,8 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
                 float v[8];
                 unpack8<TIn>(uv[i], v);
                 *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r0 + i) * a.M +
-                                          col0 + cl) = int_codes8(v, ck);
+                                          col0 + cl) =
+                    int_codes8(v, ck, a.scale + col0 + cl, s, a.qmax);
               }
             }
           }
@@ -447,15 +451,13 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
             for (int i = 0; i < kR; ++i) {
               const int r = r0 + kHalves * i;
               if (r >= rows) continue;
-              float xs[16];
-              unpack8<TIn>(uv[i][0], *reinterpret_cast<float(*)[8]>(xs));
-              unpack8<TIn>(uv[i][1], *reinterpret_cast<float(*)[8]>(xs + 8));
-              float amax = 0.0f;
+              float xr[16], xs[16];   // the raw elements and their estimates fl(x r_k)
+              unpack8<TIn>(uv[i][0], *reinterpret_cast<float(*)[8]>(xr));
+              unpack8<TIn>(uv[i][1], *reinterpret_cast<float(*)[8]>(xr + 8));
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                xs[j] = __fmul_rn(xs[j], rcp[cl + j]);
-                amax = fmaxf(amax, fabsf(xs[j]));
-              }
+              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xr[j], rcp[cl + j]);
+              const float* sc16 = a.scale + col0 + cl;
+              float amax = block_amax_exact<16>(xr, xs, sc16);
               const int64_t row = m0 + r;
               const int64_t col = col0 + cl;
               uint8_t sfb;
@@ -476,7 +478,7 @@ __global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
               *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
-                  make_uint2(f32x8_to_e2m1(xs), f32x8_to_e2m1(xs + 8));
+                  make_uint2(e2m1x8_exact(xs, xr, enc, sc16), e2m1x8_exact(xs + 8, xr + 8, enc, sc16 + 8));
               if (!mx)
                 a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
               else if ((lane & 1) == 0)

@@ -13,7 +13,7 @@
 // MMAs per CTA.
 //
 //   stats kernel  chunk of x and of ld -> shared memory; column maxima of |x|
-//                 times r_k = fl(1 / scale_k) -> one partial maximum per CTA;
+//                 divided by scale_k (IEEE) -> one partial maximum per CTA;
 //                 partial down-projection of the chunk -> ws_down[g][b][j]
 //   codes kernel  launched as a dependent of the stats kernel: loads its chunk
 //                 of x while that kernel runs, then takes the per-tensor scale
@@ -21,10 +21,11 @@
 //                 sums its share of the (b, j) down outputs over the partials
 //                 in a fixed order
 //
-// fp32 evaluation order of the codes is the one act.cu documents (and the
-// oracle's fp32 code mode repeats): r_k = fl(1 / scale_k), u = fl(1 / s),
-// INT code = rint(fl(x fl(r_k u))); NVFP4 X_hat = fl(x r_k),
-// sf = ue4m3(fl(fl(amax_b / 6) gs)), code = e2m1(fl(X_hat fl(gs / sf))).
+// Rounding as act.cu documents it: one fp32 rounding per stored scalar (s, gs,
+// block maxima, sf = ue4m3(fl(fl(amax_b / 6) gs)), enc = fl(gs / sf)), every
+// code the exactly rounded value of its quotient (x / (scale_k s) for INT,
+// x enc / scale_k or x 2^-X / scale_k onto e2m1), estimated with reciprocals
+// r_k = fl(1 / scale_k) and re-decided exactly next to a boundary.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -109,8 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
   const int pitch = chunk_pitch(a.wc, kEsz);
   uint8_t* xs = smem;                                               // bp16 rows
   uint8_t* lds = xs + static_cast<size_t>(bp16) * pitch;            // rank_pad rows
-  float* rcp = reinterpret_cast<float*>(lds + static_cast<size_t>(a.has_ld ? a.rank_pad : 0) * pitch);
-  uint32_t* cm = reinterpret_cast<uint32_t*>(rcp + a.wc);           // kThreads column-max slots
+  float* scl = reinterpret_cast<float*>(lds + static_cast<size_t>(a.has_ld ? a.rank_pad : 0) * pitch);
+  uint32_t* cm = reinterpret_cast<uint32_t*>(scl + a.wc);           // kThreads column-max slots
 
   // ------------------------------------------------------------ loads
   // weight side (ld, scale) first: it does not depend on the previous kernel
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
       *reinterpret_cast<uint4*>(lds + r * pitch + v * 16) = u;
     }
   }
-  for (int k = tid; k < ncols; k += kThreads) rcp[k] = __frcp_rn(__ldg(a.scale + c0 + k));
+  for (int k = tid; k < ncols; k += kThreads) scl[k] = __ldg(a.scale + c0 + k);
   if (a.chained) {
     pdl_wait();
     pdl_trigger();
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
 
   // ------------------------------------------------- column maxima of |x|
   // thread -> (column, row slice); |x| compared as integers (monotone for
-  // non-negative floats), then fl(colmax r_k)
+  // non-negative floats), then fl(colmax / scale_k)
   {
     auto abs_bits = [&](int r, int col) -> uint32_t {
       if constexpr (kEsz == 2)
@@ -164,13 +165,13 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const Smal
       if (tid < ncols) {
         uint32_t mm = 0u;
         for (int sl = 0; sl < nsl; ++sl) mm = max(mm, cm[sl * ncols + tid]);
-        run = __fmul_rn(__uint_as_float(mm), rcp[tid]);
+        run = __fdiv_rn(__uint_as_float(mm), scl[tid]);
       }
     } else {
       for (int col = tid; col < ncols; col += kThreads) {
         uint32_t m = 0u;
         for (int r = 0; r < B; ++r) m = max(m, abs_bits(r, col));
-        run = fmaxf(run, __fmul_rn(__uint_as_float(m), rcp[col]));
+        run = fmaxf(run, __fdiv_rn(__uint_as_float(m), scl[col]));
       }
     }
 #pragma unroll
@@ -276,12 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
 
   const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
   const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
-  float u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
+  float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
   if (nv || mx) {
     if (nv) gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
     if (g == 0 && tid == 0) *a.act_scale = gs_x;
   } else {
-    const float s = __fdiv_rn(m, static_cast<float>(a.qmax));
+    s = __fdiv_rn(m, static_cast<float>(a.qmax));
     u = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (g == 0 && tid == 0) *a.act_scale = s;
   }
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
 #pragma unroll
       for (int j = 0; j < 8; ++j) ck[j] = __fmul_rn(rcp[c8 + j], u);
       *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(r) * a.M + c0 + c8) =
-          int_codes8(v, ck);
+          int_codes8(v, ck, a.scale + c0 + c8, s, a.qmax);
     }
   } else if (mx) {
     // one 32-element block per item: a scale byte and 16 code bytes
@@ -307,23 +308,21 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
     const int64_t kbp = (a.M / 32 + 3) / 4 * 4;
     for (int i = tid; i < B * per_row; i += kThreads) {
       const int r = i / per_row, c32 = (i - r * per_row) * 32;
-      float v[32];
+      float xr[32], v[32];   // the raw elements and the estimates fl(x r_k)
 #pragma unroll
       for (int h = 0; h < 32 / kPer16; ++h)
-        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c32 + h * kPer16) * kEsz), v + h * kPer16);
-      float amax = 0.0f;
+        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c32 + h * kPer16) * kEsz), xr + h * kPer16);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        v[j] = __fmul_rn(v[j], rcp[c32 + j]);
-        amax = fmaxf(amax, fabsf(v[j]));
-      }
-      const int X = mx_block_exponent(amax);
+      for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(xr[j], rcp[c32 + j]);
+      const float* sc32 = a.scale + c0 + c32;
+      const int X = mx_block_exponent(block_amax_exact<32>(xr, v, sc32));
       const float enc = mx_inv_scale(X);
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], enc);
       const int64_t col = c0 + c32;
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(r) * (a.M / 2) + col / 2) =
-          make_uint4(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8), f32x8_to_e2m1(v + 16), f32x8_to_e2m1(v + 24));
+          make_uint4(e2m1x8_exact(v, xr, enc, sc32), e2m1x8_exact(v + 8, xr + 8, enc, sc32 + 8),
+                     e2m1x8_exact(v + 16, xr + 16, enc, sc32 + 16), e2m1x8_exact(v + 24, xr + 24, enc, sc32 + 24));
       a.sf[sf_swizzle_offset(r, col / 32, kbp)] = static_cast<uint8_t>(X + 127);
     }
   } else {
@@ -332,16 +331,14 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
     const int64_t kbp = (a.M / 16 + 3) / 4 * 4;
     for (int i = tid; i < B * per_row; i += kThreads) {
       const int r = i / per_row, c16 = (i - r * per_row) * 16;
-      float v[16];
+      float xr[16], v[16];   // the raw elements and the estimates fl(x r_k)
 #pragma unroll
       for (int h = 0; h < 16 / kPer16; ++h)
-        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c16 + h * kPer16) * kEsz), v + h * kPer16);
-      float amax = 0.0f;
+        unpack16<TIn>(*reinterpret_cast<const uint4*>(xs + r * pitch + (c16 + h * kPer16) * kEsz), xr + h * kPer16);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        v[j] = __fmul_rn(v[j], rcp[c16 + j]);
-        amax = fmaxf(amax, fabsf(v[j]));
-      }
+      for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(xr[j], rcp[c16 + j]);
+      const float* sc16 = a.scale + c0 + c16;
+      const float amax = block_amax_exact<16>(xr, v, sc16);
       const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
       const float dsf = ue4m3_to_f32(sfb);
       const float enc = dsf > 0.0f ? __fdiv_rn(gs_x, dsf) : 0.0f;
@@ -349,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) act_small_codes_kernel(const Smal
       for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], enc);
       const int64_t col = c0 + c16;
       *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + static_cast<int64_t>(r) * (a.M / 2) + col / 2) =
-          make_uint2(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8));
+          make_uint2(e2m1x8_exact(v, xr, enc, sc16), e2m1x8_exact(v + 8, xr + 8, enc, sc16 + 8));
       a.sf[sf_swizzle_offset(r, col / 16, kbp)] = sfb;
     }
   }

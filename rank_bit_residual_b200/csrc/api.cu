@@ -193,6 +193,22 @@ LinearCarve carve_linear(const svdq_weight* w, int64_t B, void* ws, size_t ws_by
 
 }  // namespace
 
+svdq_status check_quantize_act_args(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx,
+                                    const float* scale, svdq_fmt fmt, const void* ld, int32_t rank_pad,
+                                    const void* codes, const void* sf, const float* act_scale,
+                                    const void* down) {
+  svdq_status s = check_act_input(x, x_dtype, B, M, ldx);
+  if (s != SVDQ_OK) return s;
+  if (check_fmt(fmt) != SVDQ_OK || !scale || rank_pad < 0 || rank_pad % 16 || rank_pad > 256)
+    return SVDQ_EINVAL;
+  if (M % 32 != 0) return SVDQ_EUNSUPPORTED;
+  if (!aligned16(scale)) return SVDQ_EUNSUPPORTED;
+  if (B == 0) return SVDQ_OK;
+  if (!codes || !act_scale || (fmt.kind != SVDQ_KIND_INT && !sf)) return SVDQ_EINVAL;
+  if (ld && rank_pad > 0 && (!down || !aligned16(ld))) return SVDQ_EINVAL;
+  return SVDQ_OK;
+}
+
 }  // namespace svdq
 
 using namespace svdq;
@@ -303,15 +319,9 @@ svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int6
                               const void* ld, int32_t rank_pad,
                               void* codes, void* sf, float* act_scale, void* down,
                               void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
-  svdq_status s = check_act_input(x, x_dtype, B, M, ldx);
-  if (s != SVDQ_OK) return s;
-  if (check_fmt(fmt) != SVDQ_OK || !scale || rank_pad < 0 || rank_pad % 16 || rank_pad > 256)
-    return SVDQ_EINVAL;
-  if (M % 32 != 0) return SVDQ_EUNSUPPORTED;
-  if (!aligned16(scale)) return SVDQ_EUNSUPPORTED;
-  if (B == 0) return SVDQ_OK;
-  if (!codes || !act_scale || (fmt.kind != SVDQ_KIND_INT && !sf)) return SVDQ_EINVAL;
-  if (ld && rank_pad > 0 && (!down || !aligned16(ld))) return SVDQ_EINVAL;
+  const svdq_status s = check_quantize_act_args(x, x_dtype, B, M, ldx, scale, fmt, ld, rank_pad, codes,
+                                                sf, act_scale, down);
+  if (s != SVDQ_OK || B == 0) return s;
   const ActPlan p = plan_act(B, M, rank_pad, x_dtype);
   if (!workspace || workspace_bytes < act_scratch_bytes(p)) return SVDQ_EWORKSPACE;
   bool bad = false;

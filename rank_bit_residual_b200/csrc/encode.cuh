@@ -85,20 +85,163 @@ __device__ __forceinline__ void unpack16(const uint4 u, float* v) {
   }
 }
 
-// INT codes of 8 elements: rint(fl(x c_k)), packed as 8 bytes. Adding
-// 1.5 * 2^23 rounds an fp32 value below 2^22 in magnitude to the nearest
-// integer, ties to even, and leaves that integer in the low bits of the sum,
-// so the low byte of the sum is the two's-complement code. The clamp to
-// [-qmax, qmax] of the definition is omitted: with s = fl(m / qmax) and
-// c_k = fl(fl(1 / scale_k) fl(1 / s)), every |fl(x c_k)| is at most
-// qmax (1 + 6 * 2^-24) < qmax + 1/2, so no code can leave the range.
-__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8]) {
+// ------------------------------------------------------------ exact rounding
+// Every code is the correctly rounded value of a real quotient (the grid of
+// "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula item 3:
+// round half to even of X_hat / s with X_hat = x / scale; the e2m1 encoding of
+// the NVFP4 / MXFP4 blocks). The kernels first form an fp32 estimate of the
+// quotient with a few multiplies by rounded reciprocals; the estimate lies
+// within 2^-21 of the quotient, relatively, so it can only round to the wrong
+// side when the quotient is that close to a rounding boundary. Those rare
+// elements are flagged by cheap tests and decided again with exact arithmetic:
+// a boundary test "a > b * d" is the sign of fma(-b, d, a), computed from the
+// exact product and rounded once, so its sign is exact.
+
+// The exact INT code of a / (scale_k s), given an estimate q_est that is off by
+// at most one: round half to even, clamped to [-qmax, qmax]. scale_k * s is
+// exact in double (24 + 24 significant bits), and fma(-(q + 1/2), D, |a|)
+// has the sign of |a| - (q + 1/2) scale_k s exactly.
+static __device__ __noinline__ int int_code_fix(float a, float scale_k, float s, int q_est, int qmax) {
+  const double D = static_cast<double>(scale_k) * static_cast<double>(s);
+  const double aa = fabs(static_cast<double>(a));
+  int q = abs(q_est);
+  const double up = fma(-(static_cast<double>(q) + 0.5), D, aa);
+  if (up > 0.0 || (up == 0.0 && (q & 1))) {
+    q += 1;
+  } else if (q > 0) {
+    const double dn = fma(-(static_cast<double>(q) - 0.5), D, aa);
+    if (dn < 0.0 || (dn == 0.0 && (q & 1))) q -= 1;
+  }
+  q = min(q, qmax);
+  return a < 0.0f ? -q : q;
+}
+
+// Adding 1.5 * 2^23 rounds an fp32 value below 2^22 in magnitude to the
+// nearest integer, ties to even, and leaves that integer in the low bits of
+// the sum (the low byte is then the two's-complement code); subtracting the
+// constant again gives the rounded value exactly.
+constexpr float kRintMagic = 12582912.0f;
+// An estimate whose distance to its rounded value exceeds this lies near a
+// half-integer: with |t| <= 128 (qmax <= 127) its error is below 2^-15.
+constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
+
+// INT codes of 8 consecutive columns of a row, packed as 8 bytes: the exact
+// round_half_even(x / (scale_k s)), estimated as rint(fl(x c_k)) with the
+// per-column constant c_k = fl(fl(1 / scale_k) fl(1 / s)) and re-decided by
+// int_code_fix where the estimate is near a half-integer. scale8 points at the
+// 8 columns' smoothing scales (read only on that rare path). The estimate
+// never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in magnitude, so the fast
+// path needs no clamp.
+__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8],
+                                            const float* scale8, float s, int qmax) {
   uint32_t f[8];
+  bool near = false;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) f[j] = __float_as_uint(__fadd_rn(__fmul_rn(v[j], ck[j]), 12582912.0f));
+  for (int j = 0; j < 8; ++j) {
+    const float t = __fmul_rn(v[j], ck[j]);
+    const float fs = __fadd_rn(t, kRintMagic);
+    f[j] = __float_as_uint(fs);
+    near |= fabsf(__fsub_rn(t, __fsub_rn(fs, kRintMagic))) > kNearHalf;
+  }
+  if (__builtin_expect(near, 0)) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int q_est = static_cast<int>(f[j] & 0xFFu) - static_cast<int>((f[j] & 0x80u) << 1);
+      f[j] = static_cast<uint32_t>(int_code_fix(v[j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
+    }
+  }
   const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
   const uint32_t hi = __byte_perm(__byte_perm(f[4], f[5], 0x0040), __byte_perm(f[6], f[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
+}
+
+// Residual INT code of one fp32 element: round_half_even(R / s) clamped, with
+// the estimate rint(fl(R u)), u = fl(1 / s), re-decided exactly near a
+// half-integer (fp32 fma: R - (q + 1/2) s is formed exactly and rounded once).
+__device__ __forceinline__ int int_code_residual(float r, float s, float u, int qmax) {
+  const float t = __fmul_rn(r, u);
+  const float rt = __fsub_rn(__fadd_rn(t, kRintMagic), kRintMagic);
+  int q = static_cast<int>(rt);
+  if (__builtin_expect(fabsf(__fsub_rn(t, rt)) > kNearHalf, 0)) {
+    const float ar = fabsf(r);
+    q = abs(q);
+    const float up = __fmaf_rn(-(static_cast<float>(q) + 0.5f), s, ar);
+    if (up > 0.0f || (up == 0.0f && (q & 1))) {
+      q += 1;
+    } else if (q > 0) {
+      const float dn = __fmaf_rn(-(static_cast<float>(q) - 0.5f), s, ar);
+      if (dn < 0.0f || (dn == 0.0f && (q & 1))) q -= 1;
+    }
+    q = r < 0.0f ? -q : q;
+  }
+  return min(max(q, -qmax), qmax);
+}
+
+// fp32 rounding of max_j |x_j| / scale_j over n elements, exactly: est[j] =
+// fl(|x_j| fl(1 / scale_j)) is within 2^-23 of the quotient, relatively, so
+// every element whose estimate is within 2^-21 of the largest estimate is a
+// candidate, and the maximum of their IEEE quotients fl(|x_j| / scale_j)
+// (rounding is monotone) is the rounded maximum.
+template <int N>
+__device__ __forceinline__ float block_amax_exact(const float (&x)[N], const float (&est)[N],
+                                                  const float* scale_n) {
+  float e = 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; ++j) e = fmaxf(e, fabsf(est[j]));
+  const float lim = __fmul_rn(e, 1.0f - 1.0f / 2097152.0f);
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; ++j)
+    if (fabsf(est[j]) >= lim && x[j] != 0.0f) m = fmaxf(m, __fdiv_rn(fabsf(x[j]), __ldg(scale_n + j)));
+  return m;
+}
+
+// Exact e2m1 magnitude index (0..7 for {0, .5, 1, 1.5, 2, 3, 4, 6}) of P / C,
+// P, C >= 0 exact doubles, given an estimate off by at most one: the boundaries
+// are the midpoints {.25, .75, 1.25, 1.75, 2.5, 3.5, 5}, a tie goes to the even
+// index, and values from 5 up saturate at 6.
+static __device__ __noinline__ uint32_t e2m1_index_fix(double P, double C, uint32_t idx) {
+  const double mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+  if (idx < 7) {
+    const double Q = mid[idx] * C;   // exact: mid has at most 3 significant bits
+    if (P > Q || (P == Q && (idx & 1u))) return idx + 1;
+  }
+  if (idx > 0) {
+    const double Q = mid[idx - 1] * C;
+    if (P < Q || (P == Q && (idx & 1u))) return idx - 1;
+  }
+  return idx;
+}
+
+// e2m1 codes of 8 elements: the exact round-to-nearest-even of |a_j| g / c_j
+// onto the e2m1 grid (saturating at 6; +0 for zero), sign of a_j. v holds the
+// fp32 estimates (a fl(1 / c) g, rounded at each step) and a is the raw
+// element; c8 points at the 8 divisors (NULL: every c_j = 1). An element is
+// re-decided exactly when the estimate scaled by 1 -+ 2^-19 encodes to two
+// different codes, i.e. when it lies near a boundary (its error is below
+// 2^-21); |a_j| g is exact in double (24 + 24 bits) and so is mid * c_j.
+__device__ __forceinline__ uint32_t e2m1x8_exact(const float* v, const float* a, float g,
+                                                 const float* c8) {
+  float lo[8], hi[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    lo[j] = __fmul_rn(v[j], 1.0f - 1.0f / 524288.0f);
+    hi[j] = __fmul_rn(v[j], 1.0f + 1.0f / 524288.0f);
+  }
+  uint32_t out = f32x8_to_e2m1(v);
+  const uint32_t wl = f32x8_to_e2m1(lo), wh = f32x8_to_e2m1(hi);
+  if (__builtin_expect(wl != wh || wl != out, 0)) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t idx_est = (out >> (4 * j)) & 7u;
+      const double P = fabs(static_cast<double>(a[j])) * static_cast<double>(g);
+      const double C = c8 != nullptr ? static_cast<double>(__ldg(c8 + j)) : 1.0;
+      const uint32_t idx = e2m1_index_fix(P, C, idx_est);
+      const uint32_t sign = (a[j] < 0.0f && idx != 0u) ? 8u : 0u;
+      out = (out & ~(0xFu << (4 * j))) | ((sign | idx) << (4 * j));
+    }
+  }
+  return out;
 }
 
 }  // namespace svdq

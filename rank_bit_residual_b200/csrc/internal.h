@@ -77,6 +77,13 @@ cudaError_t launch_smooth_scale(const void* x, svdq_dtype xdt, int64_t B, int64_
                                 svdq_dtype wdt, int64_t N, int64_t ldw, float alpha, float* scale, void* workspace,
                                 cudaStream_t st);
 
+// Host checks of svdq_quantize_act's arguments (shared with the allocation-free
+// entry point, so both return the same status for the same arguments).
+svdq_status check_quantize_act_args(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx,
+                                    const float* scale, svdq_fmt fmt, const void* ld, int32_t rank_pad,
+                                    const void* codes, const void* sf, const float* act_scale,
+                                    const void* down);
+
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
                        const float* w_global_scale, const void* ld, void* codes, void* sf,

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -33,19 +34,24 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratch
 
 constexpr int kMaxDev = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDev] = {};
+std::atomic<void*> g_noalloc_ptr[kMaxDev] = {};
 
-// Device address of the array on the current device (nullptr on failure).
+// Device address of the array on the current device (nullptr on failure). It
+// is looked up once per device and process and kept: a context torn down and
+// made again (cudaDeviceReset) would leave a stale address, which this entry
+// point does not detect. The lock is taken only by a device's first lookup.
 void* noalloc_scratch() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
+  p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = p;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
   }
-  return g_noalloc_ptr[dev];
+  return p;
 }
 
 }  // namespace
@@ -59,18 +65,9 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
     svdq_fmt fmt, const float* act_global_scale, const float* w_global_scale, const void* ld,
     int32_t rank_pad, void* codes, void* sf, float* act_scale, void* down,
     svdq_stream_t stream) {
-  if (B < 0 || M <= 0 || (x_dtype != SVDQ_BF16 && x_dtype != SVDQ_F32)) return SVDQ_EINVAL;
-  const bool int_fmt = fmt.kind == SVDQ_KIND_INT && fmt.bits >= 2 && fmt.bits <= 8;
-  const bool f4_fmt = (fmt.kind == SVDQ_KIND_NVFP4 || fmt.kind == SVDQ_KIND_MXFP4) && fmt.bits == 4;
-  if (!int_fmt && !f4_fmt) return SVDQ_EINVAL;
-  if (!scale || rank_pad < 0 || rank_pad % 16 || rank_pad > 256) return SVDQ_EINVAL;
-  if (B == 0) return SVDQ_OK;
-  if (!x || ldx < M || !codes || !act_scale || (f4_fmt && !sf)) return SVDQ_EINVAL;
-  if (ld && rank_pad > 0 && !down) return SVDQ_EINVAL;
-  const int esz = x_dtype == SVDQ_BF16 ? 2 : 4;
-  if (M % 32 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) || (ldx * esz) % 16 ||
-      (reinterpret_cast<uintptr_t>(scale) & 15) || B > (int64_t(1) << 30))
-    return SVDQ_EUNSUPPORTED;
+  const svdq_status st = check_quantize_act_args(x, x_dtype, B, M, ldx, scale, fmt, ld, rank_pad, codes, sf,
+                                                 act_scale, down);
+  if (st != SVDQ_OK || B == 0) return st;
 
   // Same launch plan as svdq_quantize_act, with fewer K splits if that is what
   // it takes to fit the fixed array; beyond that the shape is refused.

@@ -1,15 +1,16 @@
 // quant.cu - quantisation of the residual weight R[M, N] (fp32).
 //
 // INT: the per-tensor grid of "SVDQuant Smoothing, Low-rank and Residual
-// Quantization" (Formula item 3): s_w = max|R| / qmax and
-// codes = clamp(round_half_even(R / s_w), -qmax, qmax), in fp32 with the
-// division taken as a multiply by u = fl(1 / s_w), written K-major as
-// codes[N, M] (row n = column n of R).
+// Quantization" (Formula item 3): s_w = fl(max|R| / qmax) and
+// codes = clamp(round_half_even(R / s_w), -qmax, qmax), the quotient rounded
+// exactly (estimated as fl(R u) with u = fl(1 / s_w), re-decided by an fp32
+// fma next to a half-integer), written K-major as codes[N, M] (row n =
+// column n of R).
 // NVFP4: 16-element blocks along M of each column of R, ue4m3 block scales in
 // the 128x4 layout and an fp32 global scale (the weight_fp4 / weight_sf /
 // alpha storage of "flashinfer.gemm.svdquant_linear"), same recipe as the
 // activation pass: gs = 448*6 / max|R|, sf = ue4m3(fl(amax_b / 6) * gs),
-// code = e2m1(R * fl(gs / sf)).
+// code = the exact e2m1 rounding of R * fl(gs / sf).
 // MXFP4 (the "mxfp4" per-block format of the SVDQuant parameter configuration
 // guide): 32-element blocks along M, E8M0 scales 2^X with X = floor(log2 amax) - 2,
 // codes e2m1(R * 2^-X), no global scale.
@@ -82,10 +83,7 @@ __global__ void __launch_bounds__(256) quant_int_transpose_kernel(
   for (int i = ty; i < 32; i += 8) {
     const int64_t r = m0 + i, c = n0 + tx;
     int q = 0;
-    if (r < M && c < N && s > 0.0f) {
-      q = __float2int_rn(__fmul_rn(R[r * ldR + c], u));
-      q = min(max(q, -qmax), qmax);
-    }
+    if (r < M && c < N && s > 0.0f) q = int_code_residual(R[r * ldR + c], s, u, qmax);
     tile[i][tx] = static_cast<int8_t>(q);
   }
   __syncthreads();
@@ -118,20 +116,20 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
       sf[off] = 0;
       continue;
     }
-    float v[16];
+    float rv[16], v[16];
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      v[j] = R[(b * 16 + j) * ldR + n];
-      amax = fmaxf(amax, fabsf(v[j]));
+      rv[j] = R[(b * 16 + j) * ldR + n];
+      amax = fmaxf(amax, fabsf(rv[j]));
     }
     const uint8_t sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs));
     const float d = ue4m3_to_f32(sfb);
     const float enc = d > 0.0f ? __fdiv_rn(gs, d) : 0.0f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], enc);
+    for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(rv[j], enc);
     *reinterpret_cast<uint2*>(codes + n * (M / 2) + b * 8) =
-        make_uint2(f32x8_to_e2m1(v), f32x8_to_e2m1(v + 8));
+        make_uint2(e2m1x8_exact(v, rv, enc, nullptr), e2m1x8_exact(v + 8, rv + 8, enc, nullptr));
     sf[off] = sfb;
   }
 }

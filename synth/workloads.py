@@ -183,11 +183,25 @@ for _r in (32, 128):
 WORKLOADS = tuple(_SPECS)
 
 
+_LAST_DRAW: dict = {}
+
+
+def _draw(g: dict):
+    """generate(**g), remembering the last draw: the workloads of one sweep share
+    x, W and scale (only rank and format differ); callers must not modify them."""
+    key = tuple(sorted((k, v if not isinstance(v, (list, tuple)) else tuple(v)) for k, v in g.items()))
+    if key not in _LAST_DRAW:
+        _LAST_DRAW.clear()
+        _LAST_DRAW[key] = generate(**g)
+    return _LAST_DRAW[key]
+
+
 def make_workload(name: str, rows: Optional[int] = None) -> Workload:
-    """Build a named workload; ``rows`` keeps only the first rows of x."""
+    """Build a named workload; ``rows`` keeps only the first rows of x. Arrays are
+    shared with the previous call of the same draw (treat them as read-only)."""
     spec = _SPECS[name]
     g = dict(spec["gen"])
-    x, W, scale, bias, idx = generate(**g)
+    x, W, scale, bias, idx = _draw(g)
     wl = Workload(name=name, x=x, x_dtype=g["dtype"], W=W, w_dtype=g["dtype"],
                   scale=scale, rank=spec["rank"], fmt=spec["fmt"], bits=spec["bits"],
                   bias=bias, seed=g["seed"], notes={"outlier_idx": idx})

@@ -29,7 +29,8 @@ def device():
 
 
 def to_dev(a: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
-    t = torch.from_numpy(np.ascontiguousarray(a))
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a if a.flags.writeable else a.copy())
     return t.to(dtype).to(device())
 
 
@@ -114,11 +115,10 @@ class SyntheticWeight:
         ldT = self.ld[: self.rp].T if self.rp else np.zeros((self.M, 0))
         L2 = self.L2[: self.rp] if self.rp else np.zeros((0, self.N))
         if self.fmt.kind == rb.KIND_INT:
-            q, s_x, _ = ocodes.act_codes_int_fp32(x, self.scale, self.fmt.bits)
+            q, s_x, _ = ocodes.act_codes_int(x, self.scale, self.fmt.bits)
             return oprep.linear_int(x, ldT, L2, q, s_x, self.codes, self.s_w, bias)
-        xs = ocodes.smooth_fp32(x, self.scale)
         if self.fmt.kind == rb.KIND_MXFP4:
-            ca, sa = omx.quantize(xs)
+            ca, sa = omx.quantize(x, div=self.scale)
             return oprep.linear_mxfp4(x, ldT, L2, ca, sa, self.codes, self.sf, bias)
-        ca, sa, gx = onv.quantize(xs, gs=gs_x)
+        ca, sa, gx = onv.quantize(x, gs=gs_x, div=self.scale)
         return oprep.linear_nvfp4(x, ldT, L2, ca, sa, gx, self.codes, self.sf, self.s_w, bias)

@@ -23,7 +23,7 @@ SHAPES = [(1, 32), (17, 96), (128, 256), (300, 1024), (129, 3072)]
 def test_int_codes_and_scale(B, M, dtype, bits):
     wl = make_case(B, M, 16, rank=0, seed=B + M + bits, dtype=dtype)
     codes, sf, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), f"int{bits}")
-    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, bits)
+    q, s_o, near = ocodes.act_codes_int(wl.x, wl.scale, bits)
     assert np.float32(s.item()) == s_o, (s.item(), s_o)
     assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype} int{bits}")
     assert sf is None and down is None
@@ -38,8 +38,7 @@ def test_nvfp4_codes_scales_and_layout(B, M, dtype, given_gs):
     gs_t = to_dev(np.array([gs], np.float32), torch.float32) if given_gs else None
     codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "nvfp4",
                                            act_global_scale=gs_t)
-    xs = ocodes.smooth_fp32(wl.x, wl.scale)
-    c_o, sf_o, g_o = onv.quantize(xs, gs=gs)
+    c_o, sf_o, g_o = onv.quantize(wl.x, gs=gs, div=wl.scale)
     assert np.float32(g.item()) == np.float32(g_o)
     got_sf = sf.cpu().numpy()
     want_sf = onv.sf_swizzle(sf_o)
@@ -66,7 +65,7 @@ def test_down_projection(B, M, rank, dtype):
     # bf16 x: exact products, fp32 sums; fp32 x: tf32 operands (10-bit mantissa)
     tol = 2e-5 if dtype == "bf16" else 3e-3
     assert rel_fro(got, want) <= tol, rel_fro(got, want)
-    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+    q, s_o, near = ocodes.act_codes_int(wl.x, wl.scale, 4)
     assert np.float32(s.item()) == s_o
     assert_codes_match(codes.cpu().numpy(), q, near)
 
@@ -88,7 +87,7 @@ LONG = [(1024, 256), (1100, 96), (2048, 3072)]
 def test_long_batch_int_codes_and_scale(B, M, dtype, bits):
     wl = make_case(B, M, 16, rank=0, seed=B + M + bits, dtype=dtype)
     codes, sf, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), f"int{bits}")
-    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, bits)
+    q, s_o, near = ocodes.act_codes_int(wl.x, wl.scale, bits)
     assert np.float32(s.item()) == s_o, (s.item(), s_o)
     assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype} int{bits}")
 
@@ -101,7 +100,7 @@ def test_long_batch_nvfp4_codes_scales_and_layout(B, M, given_gs):
     gs_t = to_dev(np.array([gs], np.float32), torch.float32) if given_gs else None
     codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "nvfp4",
                                            act_global_scale=gs_t)
-    c_o, sf_o, g_o = onv.quantize(ocodes.smooth_fp32(wl.x, wl.scale), gs=gs)
+    c_o, sf_o, g_o = onv.quantize(wl.x, gs=gs, div=wl.scale)
     assert np.float32(g.item()) == np.float32(g_o)
     assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
     assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
@@ -122,7 +121,7 @@ def test_long_batch_down_projection(B, M, rank, dtype):
     want = wl.x.astype(np.float64) @ ld.T.astype(np.float64)
     tol = 2e-5 if dtype == "bf16" else 3e-3
     assert rel_fro(got, want) <= tol, rel_fro(got, want)
-    q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+    q, s_o, near = ocodes.act_codes_int(wl.x, wl.scale, 4)
     assert np.float32(s.item()) == s_o
     assert_codes_match(codes.cpu().numpy(), q, near)
 
@@ -138,7 +137,7 @@ def test_large_batch_units_long_and_short(B, M, dtype):
     ld_t = to_dev(ld, torch.bfloat16 if dtype == "bf16" else torch.float32)
     for _ in range(2):
         codes, _, s, down = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "int4", ld=ld_t)
-        q, s_o, near = ocodes.act_codes_int_fp32(wl.x, wl.scale, 4)
+        q, s_o, near = ocodes.act_codes_int(wl.x, wl.scale, 4)
         assert np.float32(s.item()) == s_o
         assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype}")
         d = down.float().cpu().numpy().astype(np.float64)
@@ -155,7 +154,7 @@ def test_large_batch_units_long_and_short(B, M, dtype):
 def test_mxfp4_codes_scales_and_layout(B, M, dtype):
     wl = make_case(B, M, 16, rank=0, seed=11 * B + M, dtype=dtype)
     codes, sf, g, _ = rb.svdq_quantize_act(x_tensor(wl), to_dev(wl.scale, torch.float32), "mxfp4")
-    c_o, sf_o = omx.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
+    c_o, sf_o = omx.quantize(wl.x, div=wl.scale)
     assert g.item() == 1.0
     got_sf = sf.cpu().numpy()
     want_sf = onv.sf_swizzle(sf_o)
@@ -210,7 +209,7 @@ def test_mxfp4_encoder_edges(B, dtype):
     ones = np.ones(M, np.float32)
     xt = to_dev(x, torch.float32 if dtype == "f32" else torch.bfloat16)
     codes, sf, g, _ = rb.svdq_quantize_act(xt, to_dev(ones, torch.float32), "mxfp4")
-    c_o, sf_o = omx.quantize(ocodes.smooth_fp32(x, ones))
+    c_o, sf_o = omx.quantize(x, div=ones)
     assert g.item() == 1.0
     assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
     assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
@@ -254,7 +253,7 @@ def test_nvfp4_encoder_edges_with_given_global_scale(B):
     gs = to_dev(np.array([1.0], np.float32), torch.float32)
     codes, sf, g, _ = rb.svdq_quantize_act(to_dev(x, torch.float32), to_dev(ones, torch.float32), "nvfp4",
                                            act_global_scale=gs)
-    c_o, sf_o, g_o = onv.quantize(ocodes.smooth_fp32(x, ones), gs=np.float32(1.0))
+    c_o, sf_o, g_o = onv.quantize(x, gs=np.float32(1.0), div=ones)
     assert np.float32(g.item()) == np.float32(g_o)
     assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
     assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)

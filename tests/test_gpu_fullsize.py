@@ -32,7 +32,11 @@ CASES = [
     ("large_8192x12288x3072_int4_r32", None),
     ("large_8192x12288x3072_int4_r128", None),
     ("large_8192x12288x3072_int8_r32", None),
+    ("large_8192x12288x3072_int8_r128", None),
+    ("large_8192x12288x3072_nvfp4_r32", None),
     ("large_8192x12288x3072_nvfp4_r128", None),
+    ("large_8192x12288x3072_mxfp4_r32", None),
+    ("large_8192x12288x3072_mxfp4_r128", None),
 ]
 
 _prepared = {}
@@ -64,17 +68,17 @@ def test_fullsize_sampled_parity(name, rows):
     L2 = w.lu.float().cpu().numpy()[:, :rp].T
     sample = np.random.default_rng(7).choice(B, size=min(B, 64), replace=False)
     if wl.fmt == "int":
-        q, s_x, _ = ocodes.act_codes_int_fp32(wl.x, wl.scale, wl.bits)
+        q, s_x, _ = ocodes.act_codes_int(wl.x, wl.scale, wl.bits)
         cw = w.codes.view(torch.int8).cpu().numpy().reshape(N, M)
         want = oprep.linear_int(wl.x[sample], ld, L2, q[sample], s_x, cw,
                                 float(w.w_scale[0].item()), wl.bias)
     elif wl.fmt == "mxfp4":
-        ca, sa = omx.quantize(ocodes.smooth_fp32(wl.x[sample], wl.scale))
+        ca, sa = omx.quantize(wl.x[sample], div=wl.scale)
         cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
         sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 32)
         want = oprep.linear_mxfp4(wl.x[sample], ld, L2, ca, sa, cw, sfw, wl.bias)
     else:
-        ca, sa, gx = onv.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
+        ca, sa, gx = onv.quantize(wl.x, div=wl.scale)
         cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
         sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 16)
         want = oprep.linear_nvfp4(wl.x[sample], ld, L2, ca[sample], sa[sample], gx, cw, sfw,

@@ -22,6 +22,29 @@ def test_int32_product_is_exact(B, M, N):
     assert np.array_equal(acc.astype(np.int64), want), int((acc != want).sum())
 
 
+@pytest.mark.parametrize("B", [1, 2, 64, 300])
+def test_int32_product_is_exact_at_the_largest_k(B):
+    # bits = 8 at K = 12288 (the large compute-bound shape): codes at +-127 make
+    # |acc| reach 12288 * 127^2 = 198,193,152, the largest sum the INT grid
+    # produces, below 2^31. B = 1, 2 run the GEMV path, 64 the split-K skinny
+    # kernel, 300 the CTA-pair kernel.
+    M, N = 12288, 3072
+    rng = np.random.default_rng(B)
+    w = SyntheticWeight(M, N, 0, "int8", seed=B)
+    cw = rng.integers(-127, 128, (N, M)).astype(np.int8)
+    cw[0], cw[1] = 127, -127
+    cw[2] = np.where(np.arange(M) % 2 == 0, 127, -127)
+    w.w.codes.copy_(torch.from_numpy(cw.view(np.uint8).reshape(-1)).to(w.w.codes.device))
+    a = rng.integers(-127, 128, (B, M)).astype(np.int8)
+    a[0] = 127
+    if B > 1:
+        a[1] = np.where(np.arange(M) % 2 == 0, -127, 127)
+    acc = rb.svdq_residual_product_i32(w.w, to_dev(a, torch.int8)).cpu().numpy()
+    want = a.astype(np.float64) @ cw.astype(np.float64).T    # exact: every sum is below 2^53
+    assert acc[0, 0] == 127 * 127 * M and acc[0, 1] == -127 * 127 * M
+    assert np.array_equal(acc.astype(np.float64), want), int((acc != want).sum())
+
+
 CASES = [
     # B, M, N, rank, fmt, bias
     (16, 256, 128, 16, "int4", False),

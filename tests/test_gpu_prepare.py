@@ -67,7 +67,7 @@ def test_prepare_rank_zero_quantises_smoothed_weight_exactly(fmt):
     w = rb.svdq_prepare(to_dev(wl.W, torch.bfloat16), to_dev(wl.scale, torch.float32), 0, fmt)
     ws32 = (wl.scale[:, None].astype(np.float32) * wl.W.astype(np.float32)).astype(np.float32)
     bits = rb.parse_fmt(fmt).bits
-    q, s, near = ocodes.residual_codes_int_fp32(ws32, bits)
+    q, s, near = ocodes.residual_codes_int(ws32, bits)
     assert np.float32(w.w_scale[0].item()) == s
     got = w.codes.view(torch.int8).cpu().numpy().reshape(96, 256)
     assert_codes_match(got, q, near)
@@ -90,7 +90,7 @@ def test_quantize_residual_bit_exact(M, N, fmt):
         assert np.array_equal(sf.cpu().numpy(), onv.sf_swizzle(sf_o))
         assert np.array_equal(onv.unpack_nibbles(codes.cpu().numpy()), c_o)
     else:
-        q, s, near = ocodes.residual_codes_int_fp32(R, rb.parse_fmt(fmt).bits)
+        q, s, near = ocodes.residual_codes_int(R, rb.parse_fmt(fmt).bits)
         assert np.float32(g.item()) == s
         assert_codes_match(codes.cpu().numpy(), q, near)
 
@@ -112,7 +112,7 @@ def test_prepare_then_linear_tiny_workload():
     ld, lu = _host(w)
     rp = w.rank_pad
     cw = w.codes.view(torch.int8).cpu().numpy().reshape(wl.N, wl.M)
-    q, s_x, _ = ocodes.act_codes_int_fp32(wl.x, wl.scale, wl.bits)
+    q, s_x, _ = ocodes.act_codes_int(wl.x, wl.scale, wl.bits)
     want = oprep.linear_int(wl.x, ld.T, lu[:, :rp].T, q, s_x, cw, float(w.w_scale[0].item()))
     assert_y_close(y, want, "tiny")
     # end to end against the unquantised product: the two-branch error stays small
@@ -141,8 +141,7 @@ def test_prepare_then_linear_nvfp4(M, N, rank, bias):
     cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
     sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 16)
     gs_w = float(w.w_scale[0].item())
-    xs = ocodes.smooth_fp32(wl.x, wl.scale)
-    ca, sa, gx = onv.quantize(xs)
+    ca, sa, gx = onv.quantize(wl.x, div=wl.scale)
     want = oprep.linear_nvfp4(wl.x, ld.T, lu[:, :rp].T, ca, sa, gx, cw, sfw, gs_w,
                               wl.bias if bias else None)
     assert_y_close(y, want, "prepare+nvfp4")
@@ -162,6 +161,6 @@ def test_prepare_then_linear_mxfp4(M, N, rank, B):
     rp = w.rank_pad
     cw = onv.unpack_nibbles(w.codes.cpu().numpy().reshape(N, M // 2))
     sfw = onv.sf_unswizzle(w.sf.cpu().numpy(), N, M // 32)
-    ca, sa = omx.quantize(ocodes.smooth_fp32(wl.x, wl.scale))
+    ca, sa = omx.quantize(wl.x, div=wl.scale)
     want = oprep.linear_mxfp4(wl.x, ld.T, lu[:, :rp].T, ca, sa, cw, sfw, wl.bias)
     assert_y_close(y.cpu().numpy(), want, "prepare+mxfp4")
