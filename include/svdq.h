@@ -333,6 +333,36 @@ svdq_status svdq_smooth_scale(const void* x, svdq_dtype x_dtype, int64_t B, int6
                               const void* W, svdq_dtype w_dtype, int64_t N, int64_t ldw, float alpha,
                               float* scale, void* workspace, size_t workspace_bytes, svdq_stream_t stream);
 
+/*
+ * svdq_fold_scale - the per-channel smoothing scale chosen as the optimal
+ * diagonal fold of the quantized product, upstream of svdq_prepare.
+ * "Contraction-Gauge Preconditioning for Quantized Matrix Multiplication"
+ * (abstract): with independent zero-mean quantization errors of known variance,
+ * the expected squared error of a product of two quantized factors has an exact
+ * expression, the product is unchanged by a gauge A B = (A T)(T^-1 B), and among
+ * positive diagonal gauges (folds) a geometric program gives the globally optimal
+ * shared fold. Read here with A = x (calibration activations), B = W, the fold
+ * t = 1 / scale (the smoothing of "SVDQuant Smoothing, Low-rank and Residual
+ * Quantization", Formula item 1), per-tensor grids of `bits` on both operands and
+ * error variance Delta^2 / 12 per element (Delta = max|operand| / qmax). The
+ * program is solved on the GPU (closed-form channel optima for a given V = the
+ * weight's grid bound, golden-section search over V); channels whose x column or
+ * W row is zero take the geometric mean of the others. Any positive multiple of
+ * the result is the same fold.
+ *
+ *   x        device [B, M] (ldx >= M), bf16 or fp32, B >= 1
+ *   W        device [M, N] (ldw >= N), bf16 or fp32
+ *   bits     2..8, the INT grid both operands are quantised to
+ *   scale    out device fp32 [M]
+ *   workspace  svdq_fold_scale_workspace_size(B, M) bytes, overwritten
+ * Host errors: SVDQ_EINVAL (null pointers, sizes, bits), SVDQ_EWORKSPACE.
+ */
+svdq_status svdq_fold_scale(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx,
+                            const void* W, svdq_dtype w_dtype, int64_t N, int64_t ldw, int32_t bits,
+                            float* scale, void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
+svdq_status svdq_fold_scale_workspace_size(int64_t B, int64_t M, size_t* bytes);
+
 /* Synchronises `stream`, returns and clears the device status word
  * (SVDQ_OK, SVDQ_EINVAL or SVDQ_ETIMEOUT), or SVDQ_ECUDA on a runtime error. */
 svdq_status svdq_check_status(svdq_stream_t stream);

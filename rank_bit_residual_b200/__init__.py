@@ -52,6 +52,9 @@ _SIGS = {
     "svdq_version": (ctypes.c_char_p, []),
     "svdq_smooth_scale": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, c_i32, c_i64, c_i64, ctypes.c_float,
                                   c_vp, c_vp, c_sz, c_vp]),
+    "svdq_fold_scale": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, c_i32, c_i64, c_i64, c_i32,
+                                c_vp, c_vp, c_sz, c_vp]),
+    "svdq_fold_scale_workspace_size": (c_i32, [c_i64, c_i64, ctypes.POINTER(c_sz)]),
     "svdq_status_string": (ctypes.c_char_p, [c_i32]),
     "svdq_weight_buffer_sizes": (c_i32, [c_i64, c_i64, c_i32, SvdqFmt, ctypes.POINTER(c_sz)]),
     "svdq_prepare_workspace_size": (c_i32, [c_i64, c_i64, c_i32, SvdqFmt, c_i32, ctypes.POINTER(c_sz)]),
@@ -514,6 +517,26 @@ def svdq_smooth_scale(x: torch.Tensor, W: torch.Tensor, alpha: float = 0.5) -> t
     return scale
 
 
+def svdq_fold_scale(x: torch.Tensor, W: torch.Tensor, bits: int = 4) -> torch.Tensor:
+    """Per-channel smoothing scale of the optimal diagonal fold of x @ W under per-tensor
+    INT grids of `bits` (the geometric program of svdq_fold_scale; fp32 [M])."""
+    lib = load_library()
+    _require_cuda(x, W)
+    if x.dim() != 2 or W.dim() != 2 or x.shape[1] != W.shape[0]:
+        raise ValueError("x must be [B, M] and W [M, N]")
+    x = _rows_ready(x)
+    W = _rows_ready(W)
+    B, M = x.shape
+    N = W.shape[1]
+    nb = c_sz(0)
+    _check(lib.svdq_fold_scale_workspace_size(B, M, ctypes.byref(nb)), "svdq_fold_scale_workspace_size")
+    scale = torch.empty(M, dtype=torch.float32, device=W.device)
+    ws = torch.empty(nb.value, dtype=torch.uint8, device=W.device)
+    _check(lib.svdq_fold_scale(_ptr(x), _dt(x), B, M, x.stride(0), _ptr(W), _dt(W), N, W.stride(0), int(bits),
+                               _ptr(scale), _ptr(ws), ws.numel(), _stream()), "svdq_fold_scale")
+    return scale
+
+
 def svdq_check_status() -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     return load_library().svdq_check_status(_stream())
@@ -526,7 +549,7 @@ def svdq_selftest_wait_timeout(limit_us: int = 1000) -> int:
 
 __all__ = [
     "svdq_prepare", "svdq_quantize_act", "svdq_quantize_act_into", "svdq_quantize_act_noalloc",
-    "svdq_quantize_residual", "svdq_linear", "svdq_linear_chain", "svdq_pack_int4",
+    "svdq_quantize_residual", "svdq_linear", "svdq_linear_chain", "svdq_pack_int4", "svdq_fold_scale",
     "svdq_residual_product_i32", "svdq_residual_linear", "svdq_check_status", "svdq_selftest_wait_timeout",
     "svdq_smooth_scale",
     "PreparedWeight", "LinearWorkspace", "allocate_weight", "weight_from_buffers",

@@ -17,11 +17,16 @@ same way: select_alpha computes the scale of each candidate strength on the GPU
 (svdq_smooth_scale) from calibration activations, runs the two-branch linear at the
 given rank, and keeps the strength with the smallest output error.
 
-    python -m rank_bit_residual_b200.ablation [--workload NAME] [--rows B] [--ranks 0,1,2,...]
-                                              [--alphas 0.25,0.5,0.75,0.9]
+The diagonal fold of "Contraction-Gauge Preconditioning for Quantized Matrix
+Multiplication" (svdq_fold_scale: the geometric program's optimal shared fold of
+x @ W under per-tensor grids) is a scale of its own; fold_vs_alpha runs the
+two-branch linear with it beside the migration strengths.
 
-prints one JSON object (errors per variant and rank, singular values, timings, and
-the error per migration strength).
+    python -m rank_bit_residual_b200.ablation [--workload NAME] [--rows B] [--ranks 0,1,2,...]
+                                              [--alphas 0.25,0.5,0.75,0.9] [--fold]
+
+prints one JSON object (errors per variant and rank, singular values, timings, the
+error per migration strength, and with --fold the fold's errors).
 """
 
 from __future__ import annotations
@@ -36,7 +41,7 @@ from typing import Dict, Optional, Sequence
 import numpy as np
 import torch
 
-from . import svdq_linear, svdq_prepare, svdq_smooth_scale
+from . import svdq_fold_scale, svdq_linear, svdq_prepare, svdq_smooth_scale
 
 
 def rel_fro(y: torch.Tensor, ref: torch.Tensor) -> float:
@@ -109,6 +114,24 @@ def select_alpha(x_calib: torch.Tensor, W: torch.Tensor, rank: int, fmt: str = "
     return {"errors": table, "alpha": best[0], "error": best[1], "scale": best[2]}
 
 
+def fold_vs_alpha(x_calib: torch.Tensor, W: torch.Tensor, ranks: Sequence[int], fmt: str = "int4",
+                  alphas: Sequence[float] = (0.25, 0.5, 0.75, 0.9), bits: int = 4,
+                  x_eval: Optional[torch.Tensor] = None, seed: int = 0) -> Dict:
+    """Two-branch output errors with the geometric program's fold (svdq_fold_scale of
+    the calibration activations, per-tensor grids of `bits`) and with each migration
+    strength, at each rank; error on x_eval (default x_calib)."""
+    xe = x_calib if x_eval is None else x_eval
+    ref = xe.double() @ W.double()
+    scales = {"fold": svdq_fold_scale(x_calib, W, bits)}
+    for a in alphas:
+        scales[f"alpha={float(a):g}"] = svdq_smooth_scale(x_calib, W, float(a))
+    out = {}
+    for name, sc in scales.items():
+        out[name] = {int(r): rel_fro(svdq_linear(svdq_prepare(W, sc, int(r), fmt, seed=seed), xe,
+                                                 out_dtype=torch.float32), ref) for r in ranks}
+    return out
+
+
 def main(argv: Optional[Sequence[str]] = None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--workload", default="dit_attn_4096x3072x3072_int4")
@@ -117,6 +140,8 @@ def main(argv: Optional[Sequence[str]] = None) -> int:
     ap.add_argument("--fmt", default=None, help="override the workload's format (int4, int8, nvfp4, mxfp4)")
     ap.add_argument("--alphas", default="0.25,0.5,0.75,0.9",
                     help="migration strengths to compare at the largest rank (empty: skip)")
+    ap.add_argument("--fold", action="store_true",
+                    help="also run the geometric program's fold beside the migration strengths")
     args = ap.parse_args(argv)
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     from synth import make_workload
@@ -133,6 +158,10 @@ def main(argv: Optional[Sequence[str]] = None) -> int:
     if args.alphas:
         sel = select_alpha(x, W, max(ranks), fmt, [float(a) for a in args.alphas.split(",")])
         res["alpha_selection"] = {"rank": max(ranks), "errors": sel["errors"], "alpha": sel["alpha"]}
+    if args.fold:
+        alphas = [float(a) for a in args.alphas.split(",")] if args.alphas else []
+        bits = int(fmt[3:]) if fmt.startswith("int") else 4
+        res["fold_vs_alpha"] = fold_vs_alpha(x, W, sorted({0, max(ranks)}), fmt, alphas, bits)
     print(json.dumps(res))
     return 0
 

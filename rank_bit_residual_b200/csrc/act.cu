@@ -1,36 +1,39 @@
 // act.cu - the activation pass of the SVDQuant linear for batches of more
-// than 128 rows: a stats kernel and a codes kernel.
+// than 128 rows: a maximum kernel and a quantise kernel.
 //
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula items 1
 // and 3: X_hat = x / scale is quantised per tensor (INT grid, or NVFP4 blocks
 // for the variant of "flashinfer.gemm.svdquant_linear" step 1, or MXFP4 blocks
 // of 32 with power-of-two scales for the "mxfp4" per-block format of the
-// SVDQuant parameter configuration guide), and the
-// low-rank branch needs X_hat L1 = x ld^T (step 2 of that page) from the same
-// read of x.
+// SVDQuant parameter configuration guide), and the low-rank branch needs
+// X_hat L1 = x ld^T (step 2 of that page) from the same read of x.
 //
-// Work unit = 128 rows x a range of columns; the per-tensor scale needs every
-// unit's maximum before any code is written, and the boundary between the
-// two kernels is that grid-wide barrier (an in-kernel barrier would need its
-// counter zeroed before every launch, a graph node that costs more than the
-// barrier itself).
-//   stats kernel  streams the unit's rows with coalesced 16-byte loads (whole
-//                 row segments: DRAM pages are read front to back), takes the
-//                 column maxima of |x| from registers, and runs the unit's
-//                 down-projection x ld^T with warp-level MMAs from padded
-//                 shared-memory tiles; it writes one partial maximum per CTA
-//                 and one partial down tile per unit. Since fl(a / c) is
-//                 monotone in a, the tensor maximum of |X_hat|, rounded to
-//                 fp32, is max_k fl(colmax_k / scale_k) (IEEE quotients).
-//   codes kernel  takes the per-tensor scale from the partial maxima, writes
-//                 the codes from a second read of x (from L2 when x fits
-//                 there) and sums each row block's partial down tiles in split
-//                 order into bf16 hi | lo.
+// The per-tensor scale needs the maximum of |X_hat| over the whole tensor
+// before any code is written, so x is read twice, by two launches whose
+// boundary is that grid-wide dependency:
+//   max kernel       streams x once at the copy bandwidth (coalesced 16-byte
+//                    loads, eight rows in flight per thread) and takes column
+//                    maxima of |x|; since fl(a / c) is monotone in a, the
+//                    tensor maximum of |X_hat| rounded to fp32 is
+//                    max_k fl(colmax_k / scale_k) (IEEE quotients), one
+//                    partial per CTA. It also clears the row-block counters
+//                    of the quantise kernel. MXFP4, and NVFP4 with a given
+//                    global scale, need no maximum: one block clears the
+//                    counters and x is read once.
+//   quantise kernel  work unit = 128 rows x a range of columns, streamed in
+//                    256-byte row segments through a ring of shared-memory
+//                    stages; one thread issues the segment's tcgen05 MMAs of
+//                    the down-projection (TMEM accumulator per unit) while
+//                    all threads quantise the same segment from shared memory
+//                    and store the codes (and block scales); at the unit's end
+//                    the partial down tile goes to the workspace, and the last
+//                    unit of a row block to finish sums the row block's
+//                    partials in split order into bf16 hi | lo.
 //
 // Rounding: the stored scalars carry one fp32 rounding each (s = fl(m / qmax)
 // with m the fp32 maximum above; the NVFP4 / MXFP4 block maxima and scales),
-// and every code is the exactly rounded value of its real quotient. The codes
-// kernel estimates each quotient with multiplies by the reciprocals
+// and every code is the exactly rounded value of its real quotient. The
+// quantise kernel estimates each quotient with multiplies by the reciprocals
 // r_k = fl(1 / scale_k) and u = fl(1 / s) (INT: rint(fl(x c_k)), c_k =
 // fl(r_k u)) and decides the rare elements next to a rounding boundary again
 // in exact arithmetic (encode.cuh).
@@ -48,33 +51,37 @@ namespace svdq {
 namespace {
 
 constexpr int kWorkWarps = 16;
-constexpr int kWork = 32 * kWorkWarps;      // threads of both kernels
+constexpr int kWork = 32 * kWorkWarps;      // threads of the quantise kernel
 constexpr int kRows = 128;                  // rows per unit
 constexpr int kTileBytes = 128;             // bytes of a row per column tile (64 bf16 / 32 fp32)
-constexpr int kSub = 256;                   // bytes of a row per stats sub-chunk (two tiles)
+constexpr int kSub = 256;                   // bytes of a row per segment (two tiles)
 constexpr int kMaxStages = 6;
-constexpr int kScaleBytes = 512;            // a stage's scale values (at most 128 columns)
+constexpr int kMaxThreads = 256;            // threads of the maximum kernel
+constexpr int kMaxSlab = 2048;              // bytes of a row per maximum-kernel CTA (16 per thread)
+constexpr int kMaxCtasPerSm = 4;
 
-// Bytes of one stats-kernel stage: x and ld as two 128-byte K blocks each, then
-// the scale values; a multiple of 1024 so every block keeps the swizzle atom.
-__host__ __device__ constexpr int stats_stage_bytes(int rank_pad) {
-  return (2 * kRows * kTileBytes + 2 * rank_pad * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
+// Bytes of one quantise-kernel stage: x and ld as two 128-byte K blocks each; a
+// multiple of 1024 so every block keeps the swizzle atom.
+__host__ __device__ constexpr int quant_stage_bytes(int rank_pad) {
+  return (2 * kRows * kTileBytes + 2 * rank_pad * kTileBytes + 1023) / 1024 * 1024;
 }
 
 // TMEM columns for a rank_pad-column fp32 accumulator (a power of two >= 32).
 __host__ __device__ constexpr uint32_t tmem_cols_for(int rank_pad) {
   return rank_pad <= 32 ? 32u : rank_pad <= 64 ? 64u : rank_pad <= 128 ? 128u : 256u;
 }
-constexpr size_t kStatsSmemBudget = 220 * 1024;
+constexpr size_t kQuantSmemBudget = 220 * 1024;
 
 struct ActArgs {
   int B, M;
   int64_t ldx;
   int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
-  int nparts;       // partial maxima written by the stats kernel
-  int stages;       // stats kernel: shared-memory stages
-  int nacc;         // stats kernel: MMA issuers, each with its own TMEM accumulator
-  int chained;      // stats kernel: launched as a programmatic dependent of the previous kernel
+  int nparts;       // partial maxima written by the maximum kernel (0: none needed)
+  int max_rpc;      // maximum kernel: rows per CTA
+  int max_nslabs;   // maximum kernel: column slabs of kMaxSlab bytes
+  int stages;       // quantise kernel: shared-memory stages
+  int nacc;         // quantise kernel: MMA issuers, each with its own TMEM accumulator
+  int chained;      // maximum kernel: launched as a programmatic dependent of the previous kernel
   const void* x;
   const float* scale;
   const float* gs_given;
@@ -82,35 +89,13 @@ struct ActArgs {
   const void* ld;   // [rank_pad][M], x's dtype
   float* ws_down;   // [ksplit][B][rank_pad]
   float* ws_max;    // [nparts]
+  unsigned* ws_cnt; // [nrb] units of a row block done
   void* codes;
   uint8_t* sf;
   __nv_bfloat16* down;
   float* act_scale;
   unsigned* status;   // bounded waits record a timeout here
 };
-
-
-// Eight consecutive elements of x (16 bytes of bf16, or 32 of fp32) from
-// global memory; cl: column within the unit, a multiple of 8.
-template <typename TIn>
-__device__ __forceinline__ void load8(const void* x, int64_t ldx, int64_t row, int64_t col0, int cl,
-                                      uint4 (&u)[2]) {
-  constexpr int kPerChunk = 16 / static_cast<int>(sizeof(TIn));
-  constexpr int kChunks = 8 / kPerChunk;   // 1 (bf16) or 2 (fp32)
-  const uint4* g = reinterpret_cast<const uint4*>(static_cast<const TIn*>(x) + row * ldx + col0 + cl);
-#pragma unroll
-  for (int h = 0; h < kChunks; ++h) u[h] = __ldg(g + h);
-}
-
-template <typename TIn>
-__device__ __forceinline__ void unpack8(const uint4 (&u)[2], float (&v)[8]) {
-  if constexpr (sizeof(TIn) == 2) {
-    unpack16<TIn>(u[0], v);
-  } else {
-    unpack16<TIn>(u[0], v);
-    unpack16<TIn>(u[1], v + 4);
-  }
-}
 
 // Wait until at most stages - 2 groups are pending (stages in [2, kMaxStages]).
 __device__ __forceinline__ void cp_async_wait_ring(int stages) {
@@ -140,27 +125,99 @@ __device__ __forceinline__ uint32_t max_word(uint32_t m, uint32_t w) {
   else
     return max(m, w);
 }
+template <typename TIn>
+__device__ __forceinline__ void abs_max16(uint32_t (&m)[4], const uint4 v) {
+  m[0] = abs_max_word<TIn>(m[0], v.x);
+  m[1] = abs_max_word<TIn>(m[1], v.y);
+  m[2] = abs_max_word<TIn>(m[2], v.z);
+  m[3] = abs_max_word<TIn>(m[3], v.w);
+}
 
-// ------------------------------------------------------------ stats kernel
-// A unit is streamed in sub-chunks of kSub bytes per row through a ring of
-// `stages` shared-memory stages filled by cp.async (stages - 1 sub-chunks in
+// ------------------------------------------------------------ maximum kernel
+// CTA = a slab of kMaxSlab bytes of every row in a range of rows; thread t
+// reads the 16-byte piece t % 128 of rows r0 + t / 128, r0 + t / 128 + 2, ...
+// (a warp reads 512 contiguous bytes of a row), eight loads in flight.
+template <typename TIn>
+__global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
+  constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  constexpr int kPer16 = 16 / kEsz;
+  __shared__ uint32_t xch[kMaxThreads / 2][4];
+  __shared__ float red[kMaxThreads / 32];
+  // chained after another linear: x is that linear's output
+  if (a.chained) pdl_wait();
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0)
+    for (int i = tid; i < a.nrb; i += kMaxThreads) a.ws_cnt[i] = 0u;
+  if (a.nparts == 0) return;
+  const int slab = blockIdx.x % a.max_nslabs, rc = blockIdx.x / a.max_nslabs;
+  const int col = slab * (kMaxSlab / kEsz) + (tid & 127) * kPer16;
+  const int rsl = tid >> 7;
+  const int r0 = rc * a.max_rpc, r1 = min(a.B, r0 + a.max_rpc);
+  uint32_t m[4] = {0u, 0u, 0u, 0u};
+  if (col < a.M && r0 + rsl < r1) {
+    const int64_t step = 2 * a.ldx * kEsz / 16;   // two rows, in 16-byte units (ldx * esz % 16 == 0)
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const TIn*>(a.x) +
+                                                    static_cast<int64_t>(r0 + rsl) * a.ldx + col);
+    int r = r0 + rsl;
+    for (; r + 14 < r1; r += 16) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(p + u * step);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) abs_max16<TIn>(m, v[u]);
+      p += 8 * step;
+    }
+    for (; r < r1; r += 2) {
+      abs_max16<TIn>(m, __ldg(p));
+      p += step;
+    }
+  }
+  if (rsl == 1) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xch[tid & 127][j] = m[j];
+  }
+  __syncthreads();
+  float best = 0.0f;
+  if (rsl == 0 && col < a.M) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m[j] = max_word<TIn>(m[j], xch[tid][j]);
+    float v[kPer16];
+    unpack16<TIn>(make_uint4(m[0], m[1], m[2], m[3]), v);
+#pragma unroll
+    for (int e = 0; e < kPer16; ++e) best = fmaxf(best, __fdiv_rn(v[e], __ldg(a.scale + col + e)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if ((tid & 31) == 0) red[tid >> 5] = best;
+  __syncthreads();
+  if (tid == 0) {
+    float mx = red[0];
+    for (int w = 1; w < kMaxThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+    a.ws_max[blockIdx.x] = mx;
+  }
+}
+
+// ----------------------------------------------------------- quantise kernel
+// A unit is streamed in segments of kSub bytes per row through a ring of
+// `stages` shared-memory stages filled by cp.async (stages - 1 segments in
 // flight while one is consumed). A stage holds the x rows and the ld rows as
 // two 128-byte-wide K blocks each, in the 128-byte-swizzled K-major layout the
 // tensor core reads (16-byte chunk c of row r at chunk c ^ (r & 7) of the
-// row's 128 bytes), then the sub-chunk's scale values.
-//   copies        thread t moves the 16-byte piece t % 16 of rows t / 16 + 32 i
-//                 (i < 4): a warp moves two whole 256-byte row segments;
-//   column maxima warp w scans 32-bit words 4 w .. 4 w + 3 of rows l / 4 + 8 i
-//                 (lane l, i < 16; conflict-free under the swizzle), the eight
-//                 row slices meet by shuffles, and each column's fl(colmax / scale_k)
-//                 is taken once;
-//   down tile     one thread issues the sub-chunk's tcgen05 MMAs (M = 128 rows,
-//                 N = rank_pad, kind::f16 for bf16 x, kind::tf32 for fp32 x)
-//                 into a TMEM accumulator that lives across the unit; their
-//                 commit frees the stage for the copies of a later sub-chunk;
-//                 at the unit's end warps 0-3 drain it (TMEM lane = row).
+// row's 128 bytes).
+//   copies      thread t moves the 16-byte piece t % 16 of rows t / 16 + 32 i
+//               (i < 4): a warp moves two whole 256-byte row segments;
+//   down tile   lane 0 of warps 0 .. nacc - 1 issue the segment's tcgen05 MMAs
+//               (M = 128 rows, N = rank_pad, kind::f16 for bf16 x, kind::tf32
+//               for fp32 x) into TMEM accumulators that live across the unit;
+//               their commit frees the stage for the copies of a later segment;
+//   codes       thread t takes E = 8 (INT) or 16 (fp4) consecutive elements
+//               of a row (element group t % G, G = segment columns / E, rows
+//               t / G + i * 512 / G), reads them from the stage and stores
+//               their codes: a row's codes are written by consecutive threads.
+// The per-column constants of the unit (c_k for INT, r_k for fp4) sit in
+// shared memory after the stages.
 template <typename TIn>
-__global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
+__global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
   constexpr int kSubCols = kSub / kEsz;             // 128 bf16 or 64 fp32 columns
   constexpr int kPer16 = 16 / kEsz;                 // elements per 16-byte piece
@@ -170,21 +227,22 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   __shared__ __align__(8) uint64_t mma_bar[kMaxStages];
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
+  __shared__ int last_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rp = a.rank_pad;                        // 0 without the down factor
   const int stages = a.stages;
-  const int stage_bytes = stats_stage_bytes(rp);
+  const int stage_bytes = quant_stage_bytes(rp);
   const int ld_off = 2 * kRows * kTileBytes;        // the ld blocks follow the x blocks
-  const int sc_off = ld_off + 2 * rp * kTileBytes;  // then the scale values
+  float* colv = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * stage_bytes);
   const int piece = tid & 15, rg = tid >> 4;
-  const int wi = warp * 4 + (lane & 3), rs = lane >> 2;   // column-max word and row slice
   const TIn* x = static_cast<const TIn*>(a.x);
   const TIn* ld = static_cast<const TIn*>(a.ld);
   const uint32_t idesc = kEsz == 2 ? idesc_bf16(kRows, rp > 0 ? rp : 16) : idesc_tf32(kRows, rp > 0 ? rp : 16);
-  float run = 0.0f;
+  const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
+  const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
 
   const int nacc = a.nacc;
   const uint32_t acc_cols = tmem_cols_for(rp);
@@ -193,11 +251,25 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
     fence_mbar_init();
     abort_sh = 0;
   }
-  // chained after another linear: x is that linear's output, complete and
-  // visible once the kernel before this one has finished. Waited for before the
-  // tensor-memory allocation, so a CTA of this kernel that shares an SM with
-  // one of that kernel's never holds columns that kernel is waiting for.
-  if (a.chained) pdl_wait();
+  // the per-tensor scale from the partial maxima (INT; NVFP4 without a given gs)
+  float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
+  {
+    float m = 0.0f;
+    for (int i = tid; i < a.nparts; i += kWork) m = fmaxf(m, __ldcg(a.ws_max + i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = red[0];
+    for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
+    if (nv) {
+      gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
+    } else if (!mx) {
+      s = __fdiv_rn(m, static_cast<float>(a.qmax));
+      u = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    }
+    if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv || mx ? gs_x : s;
+  }
   if (rp > 0 && warp == 0) {
     tmem_alloc(&tmem_sh, acc_cols * nacc);
     tmem_relinquish();
@@ -207,11 +279,19 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   tc_fence_after();
   const uint32_t tmem = tmem_sh;
 
+  // element groups of the codes step
+  const int E = (nv || mx) ? 16 : 8;
+  const int tpr = kSubCols / E;                           // groups per row of a segment
+  const int rpp = kWork / tpr;                            // rows per pass
+  const int grp = tid % tpr, rr0 = tid / tpr;
+  const int64_t kb = a.M / (mx ? 32 : 16);                // fp4 scale blocks per row
+  const int64_t kbp = (kb + 3) / 4 * 4;
+
   // 16-byte chunk c (0..15) of row r of a two-block region with `rows` rows
   auto swz = [](int r, int c, int rows) -> int {
     return (c >> 3) * rows * kTileBytes + r * kTileBytes + (((c & 7) ^ (r & 7)) << 4);
   };
-  uint32_t g = 0;   // sub-chunks begun so far: stage g % stages, barrier phase (g / stages) & 1
+  uint32_t g = 0;   // segments begun so far: stage g % stages, barrier phase (g / stages) & 1
   for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
     const int rb = unit % a.nrb, sp = unit / a.nrb;
     const int m0 = rb * kRows;
@@ -221,7 +301,7 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
     const int c_hi = min(a.M, k_hi * kTileK);
     const int nsub = (c_hi - c_lo + kSubCols - 1) / kSubCols;
 
-    // sub-chunk c -> its stage (one commit group per call, empty past the end)
+    // segment c -> its stage (one commit group per call, empty past the end)
     auto issue = [&](int c) {
       if (c < nsub) {
         uint8_t* st = smem + ((g + c) % stages) * stage_bytes;
@@ -239,25 +319,24 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
           cp_async16(st + ld_off + swz(j, cc, rp),
                      in ? static_cast<const void*>(ld + static_cast<int64_t>(j) * a.M + colj) : a.ld, in ? 16 : 0);
         }
-        if (tid < kSubCols) {   // the sub-chunk's scale values (any 4-byte alignment)
-          const int cc = c_lo + c * kSubCols + tid;
-          const bool in = cc < c_hi;
-          cp_async4(st + sc_off + 4 * tid, in ? a.scale + cc : a.scale, in ? 4 : 0);
-        }
       }
       cp_async_commit();
     };
     for (int c = 0; c < stages - 1; ++c) issue(c);
+    // per-column constants of the unit: c_k = fl(fl(1 / scale_k) u) (INT) or
+    // r_k = fl(1 / scale_k) (fp4); read after the barrier of segment 0
+    for (int j = tid; j < c_hi - c_lo; j += kWork) {
+      const float r = __frcp_rn(__ldg(a.scale + c_lo + j));
+      colv[j] = (nv || mx) ? r : __fmul_rn(r, u);
+    }
     for (int c = 0; c < nsub; ++c) {
       const uint32_t gc = g + c;
       const uint8_t* st = smem + (gc % stages) * stage_bytes;
-      cp_async_wait_ring(stages);   // this thread's copies of sub-chunk c have landed
+      cp_async_wait_ring(stages);   // this thread's copies of segment c have landed
       fence_proxy_async_smem();     // ... and are visible to the tensor core
-      __syncthreads();              // everyone's have; every thread is done with sub-chunk c - 1
+      __syncthreads();              // everyone's have; every thread is done with segment c - 1
       if (abort_sh) break;          // a bounded wait gave up (uniform after the barrier)
       if (rp > 0 && lane == 0 && warp < nacc) {
-        // lane 0 of warps 0 .. nacc - 1 (one per SM sub-partition) each issue a
-        // share of the sub-chunk's MMAs into an accumulator of their own
         tc_fence_after();
         const uint32_t xa = smem_u32(st), la = xa + ld_off;
         const uint32_t acc = tmem + acc_cols * warp;
@@ -272,40 +351,76 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
         }
         mma_commit(&mma_bar[gc % stages]);
       }
-      // refill the stage of sub-chunk c - 1 once its MMAs are done (each warp
+      // refill the stage of segment c - 1 once its MMAs are done (each warp
       // waits for itself, then copies its share)
       if (rp > 0 && c > 0) mbar_wait_warp(&mma_bar[(gc - 1) % stages], ((gc - 1) / stages) & 1, a.status, &abort_sh);
       issue(c + stages - 1);
-      {
-        // max_k fl(colmax_k / scale_k): fl(a / c) is monotone in a, so the
-        // column maximum of |x| is divided once per column
-        uint32_t m = 0u;
+
+      // ---- codes of segment c
+      const int cs = c * kSubCols + grp * E;   // column of this thread's group, within the unit
+      if (c_lo + cs < c_hi) {
+        const int64_t col = c_lo + cs;
+        const uint32_t sbase = smem_u32(st);
+        if (!nv && !mx) {
+          float ck[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          m = abs_max_word<TIn>(m, ld_shared_u32(smem_u32(st + swz(rs + 8 * i, wi >> 2, kRows) + 4 * (wi & 3))));
-        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 4));
-        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 8));
-        m = max_word<TIn>(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        // every lane of the word's group holds its maximum; row slice 0 (and 1
-        // for the second bf16 lane) scales it
-        const float* sc = reinterpret_cast<const float*>(st + sc_off);
-        if constexpr (kEsz == 2) {
-          if (rs < 2) {
-            const int e = 2 * wi + rs;
-            if (c_lo + c * kSubCols + e < c_hi) {
-              const float v = __uint_as_float(rs == 0 ? m << 16 : m & 0xFFFF0000u);
-              run = fmaxf(run, __fdiv_rn(v, sc[e]));
-            }
+          for (int j = 0; j < 8; ++j) ck[j] = colv[cs + j];
+          for (int r = rr0; r < kRows; r += rpp) {
+            const int64_t row = m0 + r;
+            if (row >= a.B) break;
+            float v[8];
+            const int ch = grp * (8 / kPer16);
+#pragma unroll
+            for (int h = 0; h < 8 / kPer16; ++h)
+              unpack16<TIn>(ld_shared_v4(sbase + swz(r, ch + h, kRows)), v + h * kPer16);
+            *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + row * a.M + col) =
+                int_codes8(v, ck, a.scale + col, s, a.qmax);
           }
         } else {
-          if (rs == 0 && c_lo + c * kSubCols + wi < c_hi)
-            run = fmaxf(run, __fdiv_rn(__uint_as_float(m), sc[wi]));
+          float rk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) rk[j] = colv[cs + j];
+          const float* sc16 = a.scale + col;
+          for (int r = rr0; r < kRows; r += rpp) {
+            const int64_t row = m0 + r;
+            if (row >= a.B) break;
+            float xr[16], xs[16];   // the raw elements and their estimates fl(x r_k)
+            const int ch = grp * (16 / kPer16);
+#pragma unroll
+            for (int h = 0; h < 16 / kPer16; ++h)
+              unpack16<TIn>(ld_shared_v4(sbase + swz(r, ch + h, kRows)), xr + h * kPer16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xr[j], rk[j]);
+            float amax = block_amax_exact<16>(xr, xs, sc16);
+            uint8_t sfb;
+            float enc;
+            if (mx) {
+              // threads t and t ^ 1 hold the two halves of one 32-element block
+              // and leave the loop together (same row, same column block)
+              amax = fmaxf(amax, __shfl_xor_sync(3u << (lane & 30), amax, 1));
+              const int X = mx_block_exponent(amax);
+              sfb = static_cast<uint8_t>(X + 127);
+              enc = mx_inv_scale(X);
+            } else {
+              sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
+              const float d = ue4m3_to_f32(sfb);
+              enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
+            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
+                make_uint2(e2m1x8_exact(xs, xr, enc, sc16), e2m1x8_exact(xs + 8, xr + 8, enc, sc16 + 8));
+            if (!mx)
+              a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+            else if ((lane & 1) == 0)
+              a.sf[sf_swizzle_offset(row, col / 32, kbp)] = sfb;
+          }
         }
       }
     }
     // the unit's partial down tile: wait for its last MMAs, then TMEM -> ws_down
-    if (rp > 0 && !abort_sh) {
-      if (warp < 4) {
+    if (rp > 0) {
+      if (warp < 4 && !abort_sh) {
         const uint32_t gl = g + nsub - 1;
         const bool ok = mbar_wait_warp(&mma_bar[gl % stages], (gl / stages) & 1, a.status, &abort_sh);
         tc_fence_after();
@@ -328,22 +443,53 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
           }
         }
         tc_fence_before();
+        __threadfence();   // the partial is visible before the unit is counted
+      }
+      __syncthreads();
+      if (tid == 0) last_sh = atomicAdd(a.ws_cnt + rb, 1u) == static_cast<unsigned>(a.ksplit - 1);
+      __syncthreads();
+      if (last_sh) {
+        // every unit of this row block is done: down = the partials summed in
+        // split order, as bf16 hi | lo
+        __threadfence();
+        const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
+        const int rows = min(kRows, a.B - m0);
+        for (int i = tid; i < rows * rp; i += kWork) {
+          const int row = m0 + i / rp, j = i % rp;
+          float acc = 0.0f;
+          for (int z = 0; z < a.ksplit; ++z)
+            acc += __ldcg(a.ws_down + (static_cast<int64_t>(z) * a.B + row) * rp + j);
+          acc = __fmul_rn(acc, mult);
+          const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
+          a.down[static_cast<int64_t>(row) * 2 * rp + j] = hi;
+          a.down[static_cast<int64_t>(row) * 2 * rp + rp + j] = lo;
+        }
       }
     }
     g += nsub;
-    __syncthreads();   // the drain is done before the next unit's first MMA; stages are free
+    __syncthreads();   // the drain is done and the column constants are free before the next unit
     if (abort_sh) break;
   }
   cp_async_wait<0>();   // no copy is still on its way when the CTA ends
-  // per-CTA maximum -> ws_max[blockIdx.x]
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-  if (lane == 0) red[warp] = run;
-  __syncthreads();
-  if (tid == 0) {
-    float mx = red[0];
-    for (int w = 1; w < kWorkWarps; ++w) mx = fmaxf(mx, red[w]);
-    a.ws_max[blockIdx.x] = mx;
+  // fp4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
+  if (nv || mx) {
+    const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
+    const int64_t pad_cols = kbp - kb;
+    const int64_t n_pad = (rows_p - a.B) * kbp + static_cast<int64_t>(a.B) * pad_cols;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kWork + tid; i < n_pad;
+         i += static_cast<int64_t>(gridDim.x) * kWork) {
+      int64_t row, c;
+      if (i < static_cast<int64_t>(a.B) * pad_cols) {
+        row = i / pad_cols;
+        c = kb + (i - row * pad_cols);
+      } else {
+        const int64_t j = i - static_cast<int64_t>(a.B) * pad_cols;
+        row = a.B + j / kbp;
+        c = j - (j / kbp) * kbp;
+      }
+      a.sf[sf_swizzle_offset(row, c, kbp)] = 0;
+    }
   }
   if (rp > 0 && warp == 0) {
     tc_fence_after();
@@ -351,209 +497,35 @@ __global__ void __launch_bounds__(kWork, 1) act_stats_kernel(const ActArgs a) {
   }
 }
 
-// ------------------------------------------------------------ codes kernel
 template <typename TIn>
-__global__ void __launch_bounds__(kWork, 1) act_codes_kernel(const ActArgs a) {
-  constexpr int kTileK = kTileBytes / static_cast<int>(sizeof(TIn));
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float red[kWorkWarps];
-  float* rcp = reinterpret_cast<float*>(smem);   // the unit's reciprocals
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto unit_range = [&](int unit, int& m0, int& k_lo, int& n) {
-    const int rb = unit % a.nrb, sp = unit / a.nrb;
-    m0 = rb * kRows;
-    k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
-    n = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit) - k_lo;
-  };
-  {
-    float m = 0.0f;
-    for (int i = tid; i < a.nparts; i += kWork) m = fmaxf(m, __ldcg(a.ws_max + i));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __syncthreads();
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    m = red[0];
-    for (int w = 1; w < kWorkWarps; ++w) m = fmaxf(m, red[w]);
-    const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
-    const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
-    float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
-    if (nv) {
-      gs_x = a.gs_given != nullptr ? __ldg(a.gs_given) : (m > 0.0f ? __fdiv_rn(2688.0f, m) : 1.0f);
-    } else if (!mx) {
-      s = __fdiv_rn(m, static_cast<float>(a.qmax));
-      u = s > 0.0f ? __frcp_rn(s) : 0.0f;
-    }
-    if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv || mx ? gs_x : s;
-    const int kb = a.M / (mx ? 32 : 16);   // fp4 scale blocks per row
-    const int64_t kbp = (kb + 3) / 4 * 4;
-
-    for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
-      int m0, k_lo, n;
-      unit_range(unit, m0, k_lo, n);
-      const int sp = unit / a.nrb;
-      const int64_t col0 = static_cast<int64_t>(k_lo) * kTileK;
-      __syncthreads();
-      for (int j = tid; j < n * kTileK; j += kWork) {
-        const int col = k_lo * kTileK + j;
-        rcp[j] = col < a.M ? __frcp_rn(__ldg(a.scale + col)) : 0.0f;
-      }
-      __syncthreads();
-      const int rows = min(kRows, a.B - m0);
-      const int ncols = min(n * kTileK, a.M - k_lo * kTileK);   // a multiple of 32
-      if (!nv && !mx) {
-        // a warp writes 256 consecutive codes of a row (8 per lane, one 256-byte
-        // store) for kR rows, whose loads are all issued first
-        constexpr int kR = sizeof(TIn) == 2 ? 8 : 4;
-        for (int c256 = 0; c256 < ncols; c256 += 256) {
-          const int cl = c256 + 8 * lane;
-          if (cl >= ncols) continue;
-          float ck[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) ck[j] = __fmul_rn(rcp[cl + j], u);
-          for (int r0 = warp * kR; r0 < rows; r0 += kWorkWarps * kR) {
-            uint4 uv[kR][2];
-#pragma unroll
-            for (int i = 0; i < kR; ++i)
-              if (r0 + i < rows) load8<TIn>(a.x, a.ldx, m0 + r0 + i, col0, cl, uv[i]);
-#pragma unroll
-            for (int i = 0; i < kR; ++i) {
-              if (r0 + i < rows) {
-                float v[8];
-                unpack8<TIn>(uv[i], v);
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + static_cast<int64_t>(m0 + r0 + i) * a.M +
-                                          col0 + cl) =
-                    int_codes8(v, ck, a.scale + col0 + cl, s, a.qmax);
-              }
-            }
-          }
-        }
-      } else {
-        // half a warp = 256 consecutive elements of one row (16 elements per
-        // lane: one NVFP4 block, half an MXFP4 block whose other half is the
-        // neighbouring lane's), kR rows per half warp with all loads issued first
-        constexpr int kR = sizeof(TIn) == 2 ? 4 : 2;
-        constexpr int kHalves = 2 * kWorkWarps;
-        const int hw = 2 * warp + (lane >> 4);
-        const int nch = (ncols + 255) / 256;
-        for (int cc = 0; cc < nch; ++cc) {
-          const int cl = cc * 256 + 16 * (lane & 15);
-          if (cl >= ncols) continue;
-          for (int r0 = hw; r0 < rows; r0 += kR * kHalves) {
-            uint4 uv[kR][2][2];
-#pragma unroll
-            for (int i = 0; i < kR; ++i)
-              if (r0 + kHalves * i < rows) {
-                load8<TIn>(a.x, a.ldx, m0 + r0 + kHalves * i, col0, cl, uv[i][0]);
-                load8<TIn>(a.x, a.ldx, m0 + r0 + kHalves * i, col0, cl + 8, uv[i][1]);
-              }
-#pragma unroll
-            for (int i = 0; i < kR; ++i) {
-              const int r = r0 + kHalves * i;
-              if (r >= rows) continue;
-              float xr[16], xs[16];   // the raw elements and their estimates fl(x r_k)
-              unpack8<TIn>(uv[i][0], *reinterpret_cast<float(*)[8]>(xr));
-              unpack8<TIn>(uv[i][1], *reinterpret_cast<float(*)[8]>(xr + 8));
-#pragma unroll
-              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xr[j], rcp[cl + j]);
-              const float* sc16 = a.scale + col0 + cl;
-              float amax = block_amax_exact<16>(xr, xs, sc16);
-              const int64_t row = m0 + r;
-              const int64_t col = col0 + cl;
-              uint8_t sfb;
-              float enc;
-              if (mx) {
-                // lanes 2i and 2i + 1 hold one 32-element block; both take the
-                // same exits above (ncols is a multiple of 32), so the pair is
-                // converged here
-                amax = fmaxf(amax, __shfl_xor_sync(3u << (lane & 30), amax, 1));
-                const int X = mx_block_exponent(amax);
-                sfb = static_cast<uint8_t>(X + 127);
-                enc = mx_inv_scale(X);
-              } else {
-                sfb = f32_to_ue4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), gs_x));
-                const float d = ue4m3_to_f32(sfb);
-                enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
-              }
-#pragma unroll
-              for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
-              *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
-                  make_uint2(e2m1x8_exact(xs, xr, enc, sc16), e2m1x8_exact(xs + 8, xr + 8, enc, sc16 + 8));
-              if (!mx)
-                a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
-              else if ((lane & 1) == 0)
-                a.sf[sf_swizzle_offset(row, col / 32, kbp)] = sfb;
-            }
-          }
-        }
-      }
-      // down = the K-split partials summed in split order, as bf16 hi | lo
-      if (a.has_ld && a.down != nullptr) {
-        const int r_lo = (kRows * sp) / a.ksplit, r_hi = (kRows * (sp + 1)) / a.ksplit;
-        const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
-        const int cnt = (r_hi - r_lo) * a.rank_pad;
-        for (int i = tid; i < cnt; i += kWork) {
-          const int rr = r_lo + i / a.rank_pad, j = i % a.rank_pad;
-          const int row = m0 + rr;
-          if (row >= a.B) continue;
-          float acc = 0.0f;
-          for (int z = 0; z < a.ksplit; ++z)
-            acc += __ldcg(a.ws_down + (static_cast<int64_t>(z) * a.B + row) * a.rank_pad + j);
-          acc = __fmul_rn(acc, mult);
-          const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
-          a.down[static_cast<int64_t>(row) * 2 * a.rank_pad + j] = hi;
-          a.down[static_cast<int64_t>(row) * 2 * a.rank_pad + a.rank_pad + j] = lo;
-        }
-      }
-    }
-    // fp4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
-    if (nv || mx) {
-      const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
-      const int64_t pad_cols = kbp - kb;
-      const int64_t n_pad = (rows_p - a.B) * kbp + static_cast<int64_t>(a.B) * pad_cols;
-      for (int64_t i = static_cast<int64_t>(blockIdx.x) * kWork + tid; i < n_pad;
-           i += static_cast<int64_t>(gridDim.x) * kWork) {
-        int64_t row, c;
-        if (i < static_cast<int64_t>(a.B) * pad_cols) {
-          row = i / pad_cols;
-          c = kb + (i - row * pad_cols);
-        } else {
-          const int64_t j = i - static_cast<int64_t>(a.B) * pad_cols;
-          row = a.B + j / kbp;
-          c = j - (j / kbp) * kbp;
-        }
-        a.sf[sf_swizzle_offset(row, c, kbp)] = 0;
-      }
-    }
-  }
-}
-
-template <typename TIn>
-cudaError_t launch_stats(const ActArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(act_stats_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
+cudaError_t launch_max(const ActArgs& a, int grid, cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kWork);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(kMaxThreads);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.chained ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, act_stats_kernel<TIn>, a);
+  return cudaLaunchKernelEx(&cfg, act_max_kernel<TIn>, a);
 }
 
 template <typename TIn>
-cudaError_t launch_codes(const ActArgs& a, size_t smem, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(act_codes_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+cudaError_t launch_quant(const ActArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(act_quant_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  act_codes_kernel<TIn><<<a.nunits, kWork, smem, stream>>>(a);
+  act_quant_kernel<TIn><<<grid, kWork, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+// Largest column count a unit may have: its per-column constants share the
+// shared memory with two stages at least.
+int max_unit_cols(int rank_pad) {
+  const size_t two = 2 * static_cast<size_t>(quant_stage_bytes(rank_pad)) + 1024;
+  return static_cast<int>((kQuantSmemBudget - two) / sizeof(float)) / 64 * 64;
 }
 
 }  // namespace
@@ -563,17 +535,28 @@ void finish_act_plan(ActPlan& p) {
     finish_act_plan_small(p);
     return;
   }
+  // units of at most max_unit_cols columns (the per-column constants live in
+  // shared memory beside the stages)
+  const int min_split = static_cast<int>(ceil_div(static_cast<int64_t>(p.nsteps) * p.tile_k,
+                                                  max_unit_cols(p.rank_pad)));
+  p.ksplit = std::max(p.ksplit, std::min(p.nsteps, min_split));
   p.nunits = p.nrb * p.ksplit;
-  // stages: as many as fit, no more than the longest unit's sub-chunks + 1
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+  const int unit_cols = steps_max * p.tile_k;
   const int sub_max = (steps_max * kTileBytes + kSub - 1) / kSub;
-  const size_t sb = static_cast<size_t>(stats_stage_bytes(p.rank_pad));
-  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kStatsSmemBudget - 1024) / sb));
+  const size_t sb = static_cast<size_t>(quant_stage_bytes(p.rank_pad));
+  const size_t colv = static_cast<size_t>(unit_cols) * sizeof(float);
+  p.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kQuantSmemBudget - 1024 - colv) / sb));
   p.stages = std::max(2, std::min(p.stages, sub_max + 1));
-  p.smem = sb * p.stages + 1024;   // + alignment of the first stage to 1024 bytes
-  // one CTA per SM (512 threads, most of the shared memory)
+  p.smem = sb * p.stages + colv + 1024;   // + alignment of the first stage to 1024 bytes
+  // one quantise CTA per SM (512 threads, most of the shared memory)
   p.grid = std::min(p.nunits, num_sms());
-  p.nparts = p.grid;
+  // maximum kernel: slabs of kMaxSlab bytes x row ranges, about kMaxCtasPerSm CTAs per SM
+  const int esz = p.bf16 ? 2 : 4;
+  p.max_nslabs = static_cast<int>(ceil_div(p.M * esz, kMaxSlab));
+  const int64_t target = static_cast<int64_t>(kMaxCtasPerSm) * num_sms();
+  p.max_rpc = static_cast<int>(std::max<int64_t>(8, round_up(ceil_div(p.B * p.max_nslabs, target), 2)));
+  p.nparts = static_cast<int>(p.max_nslabs * ceil_div(p.B, p.max_rpc));
 }
 
 ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool allow_small) {
@@ -609,7 +592,9 @@ size_t act_scratch_bytes(const ActPlan& p) {
     return static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * 4, 256)) +
            (p.rank_pad > 0 ? static_cast<size_t>(round_up(static_cast<int64_t>(p.grid) * p.B * p.rank_pad * 4, 256)) : 0) +
            256;
-  size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.grid, 1)) * 4, 256));
+  // partial maxima, row-block counters, partial down tiles
+  size_t b = static_cast<size_t>(round_up(static_cast<int64_t>(std::max(p.nparts, 1)) * 4, 256)) +
+             static_cast<size_t>(round_up(static_cast<int64_t>(p.nrb) * 4, 256));
   if (p.rank_pad > 0)
     b += static_cast<size_t>(round_up(static_cast<int64_t>(p.ksplit) * p.B * p.rank_pad * 4, 256));
   return b + 256;
@@ -633,11 +618,19 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
     *bad_args = true;
     return cudaSuccess;
   }
+  // without the down factor the stages hold x alone (fewer bytes per stage,
+  // the same split: the scratch layout does not change)
+  ActPlan q = p;
+  if (!has_ld) {
+    q.rank_pad = 0;
+    finish_act_plan(q);
+  }
   Carver cv(scratch, ~size_t(0));
-  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.grid, 1)) * 4));
+  float* ws_max = static_cast<float*>(cv.take(static_cast<size_t>(std::max(p.nparts, 1)) * 4));
+  unsigned* ws_cnt = static_cast<unsigned*>(cv.take(static_cast<size_t>(p.nrb) * 4));
   float* ws_down =
-      has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4))
-             : nullptr;
+      has_ld ? static_cast<float*>(cv.take(static_cast<size_t>(p.ksplit) * p.B * p.rank_pad * 4)) : nullptr;
+  const bool need_max = fmt.kind == SVDQ_KIND_INT || (fmt.kind == SVDQ_KIND_NVFP4 && act_global_scale == nullptr);
   ActArgs a{};
   a.B = static_cast<int>(p.B);
   a.M = static_cast<int>(p.M);
@@ -648,7 +641,9 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.nunits = p.nunits;
   a.rank_pad = has_ld ? p.rank_pad : 0;
   a.has_ld = has_ld ? 1 : 0;
-  a.nparts = p.grid;
+  a.nparts = need_max ? p.nparts : 0;
+  a.max_rpc = p.max_rpc;
+  a.max_nslabs = p.max_nslabs;
   a.fmt_kind = fmt.kind;
   a.qmax = fmt.kind == SVDQ_KIND_INT ? (1 << (fmt.bits - 1)) - 1 : 0;
   a.x = x;
@@ -658,28 +653,22 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.ld = has_ld ? ld : nullptr;
   a.ws_down = ws_down;
   a.ws_max = ws_max;
+  a.ws_cnt = ws_cnt;
   a.codes = codes;
   a.sf = static_cast<uint8_t*>(sf);
   a.down = has_ld ? static_cast<__nv_bfloat16*>(down) : nullptr;
   a.act_scale = act_scale;
   a.status = device_status_word();
-  // without the down factor the stages hold x alone (fewer bytes per stage)
-  ActPlan q = p;
-  if (!has_ld) {
-    q.rank_pad = 0;
-    finish_act_plan(q);
-  }
   a.stages = q.stages;
   // as many MMA issuers (up to 4) as TMEM holds accumulators of rank_pad columns
   a.nacc = a.rank_pad > 0 ? static_cast<int>(std::min<uint32_t>(4u, 512u / tmem_cols_for(a.rank_pad))) : 1;
   a.chained = p.chained;
-  // the codes kernel keeps only the unit's reciprocals in shared memory
-  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
-  const size_t smem2 = static_cast<size_t>(steps_max) * p.tile_k * sizeof(float) + 1024;
-  cudaError_t err = xdt == SVDQ_BF16 ? launch_stats<__nv_bfloat16>(a, p.grid, q.smem, stream)
-                                     : launch_stats<float>(a, p.grid, q.smem, stream);
+  const int max_grid = need_max ? p.nparts : 1;
+  cudaError_t err = xdt == SVDQ_BF16 ? launch_max<__nv_bfloat16>(a, max_grid, stream)
+                                     : launch_max<float>(a, max_grid, stream);
   if (err != cudaSuccess) return err;
-  return xdt == SVDQ_BF16 ? launch_codes<__nv_bfloat16>(a, smem2, stream) : launch_codes<float>(a, smem2, stream);
+  return xdt == SVDQ_BF16 ? launch_quant<__nv_bfloat16>(a, p.grid, q.smem, stream)
+                          : launch_quant<float>(a, p.grid, q.smem, stream);
 }
 
 }  // namespace svdq

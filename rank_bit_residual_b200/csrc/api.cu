@@ -447,6 +447,24 @@ svdq_status svdq_smooth_scale(const void* x, svdq_dtype x_dtype, int64_t B, int6
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+svdq_status svdq_fold_scale_workspace_size(int64_t B, int64_t M, size_t* bytes) {
+  if (!bytes || B < 1 || M < 1) return SVDQ_EINVAL;
+  *bytes = fold_scratch_bytes(B, M);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_fold_scale(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M, int64_t ldx, const void* W,
+                            svdq_dtype w_dtype, int64_t N, int64_t ldw, int32_t bits, float* scale,
+                            void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
+  if (!x || !W || !scale || B < 1 || M < 1 || N < 1 || ldx < M || ldw < N || bits < 2 || bits > 8)
+    return SVDQ_EINVAL;
+  if ((x_dtype != SVDQ_BF16 && x_dtype != SVDQ_F32) || (w_dtype != SVDQ_BF16 && w_dtype != SVDQ_F32))
+    return SVDQ_EINVAL;
+  if (!workspace || workspace_bytes < fold_scratch_bytes(B, M)) return SVDQ_EWORKSPACE;
+  return from_cuda(launch_fold_scale(x, x_dtype, B, M, ldx, W, w_dtype, N, ldw, bits, scale, workspace,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
 svdq_status svdq_check_status(svdq_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SVDQ_ECUDA;

@@ -181,18 +181,35 @@ __device__ __forceinline__ int int_code_residual(float r, float s, float u, int 
 // fl(|x_j| fl(1 / scale_j)) is within 2^-23 of the quotient, relatively, so
 // every element whose estimate is within 2^-21 of the largest estimate is a
 // candidate, and the maximum of their IEEE quotients fl(|x_j| / scale_j)
-// (rounding is monotone) is the rounded maximum.
+// (rounding is monotone) is the rounded maximum. Usually the element with the
+// largest estimate is the only candidate: its quotient is taken alone, and
+// the others only when a second candidate exists.
 template <int N>
 __device__ __forceinline__ float block_amax_exact(const float (&x)[N], const float (&est)[N],
                                                   const float* scale_n) {
-  float e = 0.0f;
+  float e = 0.0f, xa = 0.0f;
+  int ja = 0;
 #pragma unroll
-  for (int j = 0; j < N; ++j) e = fmaxf(e, fabsf(est[j]));
+  for (int j = 0; j < N; ++j) {
+    const float a = fabsf(est[j]);
+    if (a > e) {
+      e = a;
+      xa = fabsf(x[j]);
+      ja = j;
+    }
+  }
+  if (e == 0.0f) return 0.0f;
   const float lim = __fmul_rn(e, 1.0f - 1.0f / 2097152.0f);
-  float m = 0.0f;
+  int ncand = 0;
 #pragma unroll
-  for (int j = 0; j < N; ++j)
-    if (fabsf(est[j]) >= lim && x[j] != 0.0f) m = fmaxf(m, __fdiv_rn(fabsf(x[j]), __ldg(scale_n + j)));
+  for (int j = 0; j < N; ++j) ncand += fabsf(est[j]) >= lim ? 1 : 0;
+  float m = __fdiv_rn(xa, __ldg(scale_n + ja));
+  if (__builtin_expect(ncand > 1, 0)) {
+    // unrolled like the loops above, so x and est stay in registers
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if (fabsf(est[j]) >= lim && j != ja) m = fmaxf(m, __fdiv_rn(fabsf(x[j]), __ldg(scale_n + j)));
+  }
   return m;
 }
 

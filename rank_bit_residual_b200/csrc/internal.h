@@ -52,9 +52,11 @@ struct ActPlan {
   int nsteps;      // K tiles
   int ksplit;      // K ranges per row block
   int nunits;      // nrb * ksplit work units
-  int stages;      // large-batch stats kernel: sub-chunk stages in shared memory
-  int grid;        // CTAs of the stats (large batch) or first (short batch) kernel
-  int nparts;      // partial maxima written (one per CTA)
+  int stages;      // large-batch quantise kernel: segment stages in shared memory
+  int grid;        // CTAs of the quantise (large batch) or first (short batch) kernel
+  int nparts;      // partial maxima written (one per CTA of the first kernel)
+  int max_rpc;     // large batch: rows per CTA of the maximum kernel
+  int max_nslabs;  // large batch: 2048-byte column slabs of the maximum kernel
   size_t smem;     // dynamic shared memory per CTA
   int small;       // 1: the short-batch kernel (act_small.cu): one column chunk per CTA
   int wc;          // short-batch kernel: columns per chunk (a multiple of 32)
@@ -83,6 +85,12 @@ svdq_status check_quantize_act_args(const void* x, svdq_dtype x_dtype, int64_t B
                                     const float* scale, svdq_fmt fmt, const void* ld, int32_t rank_pad,
                                     const void* codes, const void* sf, const float* act_scale,
                                     const void* down);
+
+// svdq_fold_scale (fold.cu)
+size_t fold_scratch_bytes(int64_t B, int64_t M);
+cudaError_t launch_fold_scale(const void* x, svdq_dtype xdt, int64_t B, int64_t M, int64_t ldx, const void* w,
+                              svdq_dtype wdt, int64_t N, int64_t ldw, int bits, float* scale, void* workspace,
+                              cudaStream_t st);
 
 cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,

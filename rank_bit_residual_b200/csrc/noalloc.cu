@@ -74,8 +74,10 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
   const int32_t rp = (ld != nullptr) ? rank_pad : 0;
   ActPlan p = plan_act(B, M, rp, x_dtype);
   while (act_scratch_bytes(p) > kNoallocScratchBytes && p.ksplit > 1) {
+    const int before = p.ksplit;
     p.ksplit = std::max(1, p.ksplit / 2);
     finish_act_plan(p);
+    if (!p.small && p.ksplit >= before) break;   // the split cannot shrink further
     // fewer, wider column chunks of the short-batch kernel may outgrow its
     // shared memory: continue with the large-batch plan then
     if (p.small && p.smem > kActSmallSmemMax) p = plan_act(B, M, rp, x_dtype, false);

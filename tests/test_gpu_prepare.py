@@ -41,7 +41,8 @@ def _residual(wl, w):
 
 @pytest.mark.parametrize("M,N,rank,dtype", [(256, 128, 16, "f32"), (64, 512, 40, "bf16"),
                                             (512, 64, 64, "bf16"), (1024, 768, 32, "bf16"),
-                                            (96, 96, 96, "f32"), (3072, 512, 128, "bf16")])
+                                            (96, 96, 96, "f32"), (3072, 512, 128, "bf16"),
+                                            (1024, 768, 200, "bf16")])
 def test_prepare_residual_within_one_percent_of_optimal(M, N, rank, dtype):
     wl = make_case(8, M, N, rank=rank, seed=M + N, dtype=dtype, spikes=(6.0, 4.0, 3.0, 2.0, 1.0))
     W = to_dev(wl.W, torch.bfloat16 if dtype == "bf16" else torch.float32)

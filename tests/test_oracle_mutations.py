@@ -8,6 +8,8 @@ import oracle.svdquant as sq
 import oracle.nvfp4 as nv
 import oracle.prepared as pp
 import oracle.codes as oc
+import oracle.fold as of
+from tests import test_oracle_fold as T6
 from tests import test_oracle_svdquant as T1
 from tests import test_oracle_codes as T2
 
@@ -124,6 +126,21 @@ def _e2m1_ratio_ties_away(p, c, negative):
     return (sign | idx.astype(np.uint8)).astype(np.uint8)
 
 
+def _dither_error_no_cross(A, B, var_a, var_b):
+    A = np.asarray(A, np.float64); B = np.asarray(B, np.float64)
+    va = np.broadcast_to(np.asarray(var_a, np.float64), A.shape)
+    vb = np.broadcast_to(np.asarray(var_b, np.float64), B.shape)
+    return float(np.sum(va @ (B * B)) + np.sum((A * A) @ vb))
+
+
+def _fold_error_delta_not_squared(stats, t, m, n, bits):
+    a, alpha, b, beta = (np.asarray(s_, np.float64) for s_ in stats)
+    q = float(2 ** (bits - 1) - 1)
+    U, V = float(np.max(a * t)), float(np.max(b / t))
+    return (m * U / (12 * q) * float(np.sum(beta / (t * t))) + n * V / (12 * q) * float(np.sum(alpha * t * t)) +
+            len(a) * m * n * U * V / (144 * q * q))
+
+
 def _pack_swapped(codes):
     c = np.asarray(codes, dtype=np.uint8)
     return (c[:, 1::2] & 0xF) | ((c[:, 0::2] & 0xF) << 4)
@@ -157,6 +174,8 @@ MUTATIONS = [
      [T2.test_codes_decided_exactly_where_fp32_orders_differ]),
     (oc, "_exact_rne_quotient", _quotient_half_away, [T2.test_codes_hand_ties]),
     (nv, "e2m1_encode_ratio", _e2m1_ratio_ties_away, [T2.test_e2m1_ratio_ties_go_to_even]),
+    (of, "dither_error", _dither_error_no_cross, [T6.test_dither_identity_matches_monte_carlo]),
+    (of, "fold_error", _fold_error_delta_not_squared, [T6.test_fold_error_is_the_identity_on_the_folded_operands]),
     (nv, "sf_offset", _sf_offset_transposed, [T2.test_sf_layout_points_and_bijection]),
     (pp, "int_product", _int_product_transposed, [T1.test_integer_product_matches_brute_force]),
 ]
