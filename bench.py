@@ -269,6 +269,12 @@ EXTRA_TIMED_MS = 150.0   # device time each extra record's timed region aims for
 SOAK_MS = 400.0          # back-to-back steps just before a sampled timed region
 
 
+def launches_per_step(wl) -> int:
+    """Kernels one svdq_linear call launches: one for one or two rows with INT weights
+    (the single-launch decode kernel), else two for the activation pass and one GEMM."""
+    return 1 if (wl.fmt == "int" and wl.B <= 2) else 3
+
+
 def fmt_name(wl):
     return f"int{wl.bits}" if wl.fmt == "int" else wl.fmt
 
@@ -288,7 +294,7 @@ def run_reference(args, wl_name):
     if rank != 0:
         return 0
     from synth import make_workload
-    wl = make_workload(wl_name)
+    wl = make_workload(wl_name, rows=args.rows)
     per_step = max(0.5, 60.0 / max(args.steps + args.warmup, 1))
     for _ in range(args.warmup):
         cpu_oracle_rate(wl, budget_s=0.0, rows=16)
@@ -609,6 +615,7 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--rows", type=int, default=None, help="keep only the first rows of the workload's x")
     ap.add_argument("--configs", default=None, choices=["all", "none"],
                     help="per-configuration records (default: all for the default workload)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -620,7 +627,7 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args, args.workload)
-    configs = args.configs or ("all" if args.workload == DEFAULT_WORKLOAD else "none")
+    configs = args.configs or ("all" if (args.workload == DEFAULT_WORKLOAD and args.rows is None) else "none")
 
     import numpy as np
     import torch
@@ -640,7 +647,7 @@ def main():
     peaks, peak_src = load_peaks()
 
     # ---------------------------------------------------------------- headline
-    ctx = eng.setup(args.workload, nsets=args.sets)
+    ctx = eng.setup(args.workload, rows=args.rows, nsets=args.sets)
     wl = ctx["wl"]
     B, M, N, r, R = wl.B, wl.M, wl.N, wl.rank, ctx["R"]
     sampler = ClockSampler(local)
@@ -716,7 +723,7 @@ def main():
                 "d2h_bytes_per_step": int(ye.numel() * ye.element_size()), "steps": Ke,
                 "call": "svdq_linear (pinned host x -> device, Y -> pinned host), weights rotating over "
                         f"the {R} sets"},
-        "gpu_launches": 3 * K,   # per step: the activation pass's two kernels and the GEMM
+        "gpu_launches": launches_per_step(wl) * K,
         "clocks": sampler.clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -747,7 +754,7 @@ def main():
                    "kernel_roofline": {k: krf[k] for k in ("kernel", "bound", "duration_us", "achieved",
                                                            "unit", "peak", "frac")},
                    "act_us": mm["act_ms"] * 1e3, "gemm_us": mm["gemm_ms"] * 1e3,
-                   "prepare_ms": c["prepare_ms"], "sets": c["R"]}
+                   "prepare_ms": c["prepare_ms"], "sets": c["R"], "launches_per_step": launches_per_step(cw)}
             eng.step(c, 0)
             torch.cuda.synchronize()
             rec["parity"] = sampled_parity(c, c["sets"][0][6], rows_n=16)

@@ -20,9 +20,10 @@
 //                    of the quantise kernel. MXFP4, and NVFP4 with a given
 //                    global scale, need no maximum: one block clears the
 //                    counters and x is read once.
-//   quantise kernel  work unit = 128 rows x a range of columns, streamed in
-//                    256-byte row segments through a ring of shared-memory
-//                    stages; one thread issues the segment's tcgen05 MMAs of
+//   quantise kernel  work unit = 128 rows x a range of whole 256-byte row
+//                    segments, streamed by TMA (one 16 KB box per 128 bytes of
+//                    the 128 rows) through a ring of shared-memory stages; one
+//                    thread issues the segment's tcgen05 MMAs of
 //                    the down-projection (TMEM accumulator per unit) while
 //                    all threads quantise the same segment from shared memory
 //                    and store the codes (and block scales); at the unit's end
@@ -75,7 +76,8 @@ constexpr size_t kQuantSmemBudget = 220 * 1024;
 struct ActArgs {
   int B, M;
   int64_t ldx;
-  int nsteps, ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
+  int nsteps;       // 256-byte segments of a row (the unit of the K split)
+  int ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
   int nparts;       // partial maxima written by the maximum kernel (0: none needed)
   int max_rpc;      // maximum kernel: rows per CTA
   int max_nslabs;   // maximum kernel: column slabs of kMaxSlab bytes
@@ -96,17 +98,6 @@ struct ActArgs {
   float* act_scale;
   unsigned* status;   // bounded waits record a timeout here
 };
-
-// Wait until at most stages - 2 groups are pending (stages in [2, kMaxStages]).
-__device__ __forceinline__ void cp_async_wait_ring(int stages) {
-  switch (stages) {
-    case 2: cp_async_wait<0>(); break;
-    case 3: cp_async_wait<1>(); break;
-    case 4: cp_async_wait<2>(); break;
-    case 5: cp_async_wait<3>(); break;
-    default: cp_async_wait<4>(); break;
-  }
-}
 
 // Running maximum of |x| over one 32-bit word of a row: two bf16 lanes (the
 // packed 16-bit magnitudes, one SIMD max) or one fp32 (its magnitude bits);
@@ -199,13 +190,14 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
 
 // ----------------------------------------------------------- quantise kernel
 // A unit is streamed in segments of kSub bytes per row through a ring of
-// `stages` shared-memory stages filled by cp.async (stages - 1 segments in
-// flight while one is consumed). A stage holds the x rows and the ld rows as
-// two 128-byte-wide K blocks each, in the 128-byte-swizzled K-major layout the
+// `stages` shared-memory stages filled by TMA (stages - 1 segments in flight
+// while one is consumed). A stage holds the x rows and the ld rows as two
+// 128-byte-wide K blocks each, in the 128-byte-swizzled K-major layout the
 // tensor core reads (16-byte chunk c of row r at chunk c ^ (r & 7) of the
-// row's 128 bytes).
-//   copies      thread t moves the 16-byte piece t % 16 of rows t / 16 + 32 i
-//               (i < 4): a warp moves two whole 256-byte row segments;
+// row's 128 bytes); rows past B and columns past M arrive as zeros.
+//   copies      thread 0 loads the segment's four boxes (x and ld, two K
+//               blocks each) once every thread is done with the stage's
+//               previous segment and its MMAs have completed;
 //   down tile   lane 0 of warps 0 .. nacc - 1 issue the segment's tcgen05 MMAs
 //               (M = 128 rows, N = rank_pad, kind::f16 for bf16 x, kind::tf32
 //               for fp32 x) into TMEM accumulators that live across the unit;
@@ -216,15 +208,19 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
 //               their codes: a row's codes are written by consecutive threads.
 // The per-column constants of the unit (c_k for INT, r_k for fp4) sit in
 // shared memory after the stages.
-template <typename TIn>
-__global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
+template <typename TIn, bool kFp4>
+__global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                             const __grid_constant__ CUtensorMap tm_ld,
+                                                             const ActArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
   constexpr int kSubCols = kSub / kEsz;             // 128 bf16 or 64 fp32 columns
   constexpr int kPer16 = 16 / kEsz;                 // elements per 16-byte piece
   constexpr int kTileK = kTileBytes / kEsz;         // columns per K tile
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ float red[kWorkWarps];
-  __shared__ __align__(8) uint64_t mma_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages];    // the stage's boxes have landed
+  __shared__ __align__(8) uint64_t empty_bar[kMaxStages];   // every warp and every MMA is done with it
+  __shared__ __align__(8) uint64_t unit_bar;                // the unit's MMAs are complete
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
   __shared__ int last_sh;
@@ -237,9 +233,6 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
   const int stage_bytes = quant_stage_bytes(rp);
   const int ld_off = 2 * kRows * kTileBytes;        // the ld blocks follow the x blocks
   float* colv = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * stage_bytes);
-  const int piece = tid & 15, rg = tid >> 4;
-  const TIn* x = static_cast<const TIn*>(a.x);
-  const TIn* ld = static_cast<const TIn*>(a.ld);
   const uint32_t idesc = kEsz == 2 ? idesc_bf16(kRows, rp > 0 ? rp : 16) : idesc_tf32(kRows, rp > 0 ? rp : 16);
   const bool nv = a.fmt_kind == SVDQ_KIND_NVFP4;
   const bool mx = a.fmt_kind == SVDQ_KIND_MXFP4;
@@ -247,9 +240,15 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
   const int nacc = a.nacc;
   const uint32_t acc_cols = tmem_cols_for(rp);
   if (tid == 0) {
-    for (int s = 0; s < kMaxStages; ++s) mbar_init(&mma_bar[s], nacc);
+    for (int s = 0; s < kMaxStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kWorkWarps + (rp > 0 ? nacc : 0));
+    }
+    mbar_init(&unit_bar, nacc);
     fence_mbar_init();
     abort_sh = 0;
+    tma_prefetch_desc(&tm_x);
+    if (rp > 0) tma_prefetch_desc(&tm_ld);
   }
   // the per-tensor scale from the partial maxima (INT; NVFP4 without a given gs)
   float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
@@ -279,11 +278,13 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
   tc_fence_after();
   const uint32_t tmem = tmem_sh;
 
-  // element groups of the codes step
-  const int E = (nv || mx) ? 16 : 8;
-  const int tpr = kSubCols / E;                           // groups per row of a segment
-  const int rpp = kWork / tpr;                            // rows per pass
-  const int grp = tid % tpr, rr0 = tid / tpr;
+  // element groups of the codes step: kE elements of a row per thread, the
+  // threads of a row consecutive, kPasses rows per thread kRpp apart
+  constexpr int kE = kFp4 ? 16 : 8;
+  constexpr int kTpr = kSubCols / kE;                     // groups per row of a segment
+  constexpr int kRpp = kWork / kTpr;                      // rows per pass
+  constexpr int kPasses = kRows / kRpp > 0 ? kRows / kRpp : 1;
+  const int grp = tid % kTpr, rr0 = tid / kTpr;
   const int64_t kb = a.M / (mx ? 32 : 16);                // fp4 scale blocks per row
   const int64_t kbp = (kb + 3) / 4 * 4;
 
@@ -292,50 +293,56 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
     return (c >> 3) * rows * kTileBytes + r * kTileBytes + (((c & 7) ^ (r & 7)) << 4);
   };
   uint32_t g = 0;   // segments begun so far: stage g % stages, barrier phase (g / stages) & 1
+  uint32_t unit_parity = 0;
   for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
     const int rb = unit % a.nrb, sp = unit / a.nrb;
     const int m0 = rb * kRows;
+    // whole segments per unit: no box reaches into another unit's columns
     const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
     const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
-    const int c_lo = k_lo * kTileK;
-    const int c_hi = min(a.M, k_hi * kTileK);
-    const int nsub = (c_hi - c_lo + kSubCols - 1) / kSubCols;
+    const int c_lo = k_lo * kSubCols;
+    const int c_hi = min(a.M, k_hi * kSubCols);
+    const int nsub = k_hi - k_lo;
+    const uint32_t seg_bytes = static_cast<uint32_t>(2 * kRows * kTileBytes + 2 * rp * kTileBytes);
 
-    // segment c -> its stage (one commit group per call, empty past the end)
+    // segment c -> its stage (thread 0; nothing past the unit's end). A stage is
+    // refilled once all 16 warps and the MMAs have released its previous
+    // segment; only thread 0 waits for that, and only when it refills.
     auto issue = [&](int c) {
-      if (c < nsub) {
-        uint8_t* st = smem + ((g + c) % stages) * stage_bytes;
-        const int col = c_lo + c * kSubCols + piece * kPer16;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = rg + 32 * i, row = m0 + r;
-          const bool in = col < c_hi && row < a.B;
-          cp_async16(st + swz(r, piece, kRows),
-                     in ? static_cast<const void*>(x + static_cast<int64_t>(row) * a.ldx + col) : a.x, in ? 16 : 0);
-        }
-        for (int idx = tid; idx < rp * 16; idx += kWork) {
-          const int j = idx >> 4, cc = idx & 15, colj = c_lo + c * kSubCols + cc * kPer16;
-          const bool in = colj < c_hi;
-          cp_async16(st + ld_off + swz(j, cc, rp),
-                     in ? static_cast<const void*>(ld + static_cast<int64_t>(j) * a.M + colj) : a.ld, in ? 16 : 0);
+      if (tid == 0 && c < nsub) {
+        const uint32_t gc = g + c;
+        const uint32_t s_ = gc % stages;
+        if (gc >= static_cast<uint32_t>(stages) &&
+            !mbar_wait(&empty_bar[s_], ((gc / stages) - 1) & 1, a.status, &abort_sh))
+          return;   // a wait ran out: load nothing more
+        uint8_t* st = smem + s_ * stage_bytes;
+        uint64_t* bar = &full_bar[s_];
+        const int col = c_lo + c * kSubCols;
+        mbar_arrive_expect_tx(bar, seg_bytes);
+        tma_load_2d(st, &tm_x, bar, col, m0);
+        tma_load_2d(st + kRows * kTileBytes, &tm_x, bar, col + kTileK, m0);
+        if (rp > 0) {
+          tma_load_2d(st + ld_off, &tm_ld, bar, col, 0);
+          tma_load_2d(st + ld_off + rp * kTileBytes, &tm_ld, bar, col + kTileK, 0);
         }
       }
-      cp_async_commit();
     };
     for (int c = 0; c < stages - 1; ++c) issue(c);
     // per-column constants of the unit: c_k = fl(fl(1 / scale_k) u) (INT) or
-    // r_k = fl(1 / scale_k) (fp4); read after the barrier of segment 0
+    // r_k = fl(1 / scale_k) (fp4)
     for (int j = tid; j < c_hi - c_lo; j += kWork) {
       const float r = __frcp_rn(__ldg(a.scale + c_lo + j));
       colv[j] = (nv || mx) ? r : __fmul_rn(r, u);
     }
+    __syncthreads();   // the column constants are written
     for (int c = 0; c < nsub; ++c) {
       const uint32_t gc = g + c;
-      const uint8_t* st = smem + (gc % stages) * stage_bytes;
-      cp_async_wait_ring(stages);   // this thread's copies of segment c have landed
-      fence_proxy_async_smem();     // ... and are visible to the tensor core
-      __syncthreads();              // everyone's have; every thread is done with segment c - 1
-      if (abort_sh) break;          // a bounded wait gave up (uniform after the barrier)
+      const uint32_t s_ = gc % stages;
+      const uint8_t* st = smem + s_ * stage_bytes;
+      // thread 0 keeps stages - 1 segments in flight
+      issue(c + stages - 1);
+      // segment c has landed (every warp waits for itself)
+      if (!mbar_wait_warp(&full_bar[s_], (gc / stages) & 1, a.status, &abort_sh)) break;
       if (rp > 0 && lane == 0 && warp < nacc) {
         tc_fence_after();
         const uint32_t xa = smem_u32(st), la = xa + ld_off;
@@ -349,54 +356,49 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
           else
             mma_tf32(acc, smem_desc_sw128(xa + off), smem_desc_sw128(la + offl), idesc, (c > 0 || kk > kk0) ? 1u : 0u);
         }
-        mma_commit(&mma_bar[gc % stages]);
+        mma_commit(&empty_bar[s_]);
+        if (c == nsub - 1) mma_commit(&unit_bar);
       }
-      // refill the stage of segment c - 1 once its MMAs are done (each warp
-      // waits for itself, then copies its share)
-      if (rp > 0 && c > 0) mbar_wait_warp(&mma_bar[(gc - 1) % stages], ((gc - 1) / stages) & 1, a.status, &abort_sh);
-      issue(c + stages - 1);
 
-      // ---- codes of segment c
-      const int cs = c * kSubCols + grp * E;   // column of this thread's group, within the unit
-      if (c_lo + cs < c_hi) {
+      // ---- codes of segment c: the passes' loads first, then their arithmetic
+      // (independent chains), then the stores of the rows below B
+      const int cs = c * kSubCols + grp * kE;   // column of this thread's group, within the unit
+      if (rr0 < kRows && c_lo + cs < c_hi) {
         const int64_t col = c_lo + cs;
         const uint32_t sbase = smem_u32(st);
-        if (!nv && !mx) {
-          float ck[8];
+        constexpr int kCh = kE / kPer16;         // 16-byte pieces per group
+        const int ch = grp * kCh;
+        float xv[kPasses][kE];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ck[j] = colv[cs + j];
-          for (int r = rr0; r < kRows; r += rpp) {
-            const int64_t row = m0 + r;
-            if (row >= a.B) break;
-            float v[8];
-            const int ch = grp * (8 / kPer16);
+        for (int p = 0; p < kPasses; ++p)
 #pragma unroll
-            for (int h = 0; h < 8 / kPer16; ++h)
-              unpack16<TIn>(ld_shared_v4(sbase + swz(r, ch + h, kRows)), v + h * kPer16);
-            *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + row * a.M + col) =
-                int_codes8(v, ck, a.scale + col, s, a.qmax);
+          for (int h = 0; h < kCh; ++h)
+            unpack16<TIn>(ld_shared_v4(sbase + swz(rr0 + p * kRpp, ch + h, kRows)), xv[p] + h * kPer16);
+        float cv[kE];
+#pragma unroll
+        for (int j = 0; j < kE; ++j) cv[j] = colv[cs + j];
+        if constexpr (!kFp4) {
+          uint2 q[kPasses];
+#pragma unroll
+          for (int p = 0; p < kPasses; ++p) q[p] = int_codes8(xv[p], cv, a.scale + col, s, a.qmax);
+#pragma unroll
+          for (int p = 0; p < kPasses; ++p) {
+            const int64_t row = m0 + rr0 + p * kRpp;
+            if (row < a.B) *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.codes) + row * a.M + col) = q[p];
           }
         } else {
-          float rk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) rk[j] = colv[cs + j];
           const float* sc16 = a.scale + col;
-          for (int r = rr0; r < kRows; r += rpp) {
-            const int64_t row = m0 + r;
-            if (row >= a.B) break;
-            float xr[16], xs[16];   // the raw elements and their estimates fl(x r_k)
-            const int ch = grp * (16 / kPer16);
 #pragma unroll
-            for (int h = 0; h < 16 / kPer16; ++h)
-              unpack16<TIn>(ld_shared_v4(sbase + swz(r, ch + h, kRows)), xr + h * kPer16);
+          for (int p = 0; p < kPasses; ++p) {
+            float xs[16];   // the estimates fl(x r_k) of the raw elements xv[p]
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xr[j], rk[j]);
-            float amax = block_amax_exact<16>(xr, xs, sc16);
+            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xv[p][j], cv[j]);
+            float amax = block_amax_exact<16>(xv[p], xs, sc16);
             uint8_t sfb;
             float enc;
             if (mx) {
               // threads t and t ^ 1 hold the two halves of one 32-element block
-              // and leave the loop together (same row, same column block)
+              // (same row, same column block, same passes)
               amax = fmaxf(amax, __shfl_xor_sync(3u << (lane & 30), amax, 1));
               const int X = mx_block_exponent(amax);
               sfb = static_cast<uint8_t>(X + 127);
@@ -408,21 +410,26 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
-            *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) =
-                make_uint2(e2m1x8_exact(xs, xr, enc, sc16), e2m1x8_exact(xs + 8, xr + 8, enc, sc16 + 8));
-            if (!mx)
-              a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
-            else if ((lane & 1) == 0)
-              a.sf[sf_swizzle_offset(row, col / 32, kbp)] = sfb;
+            const uint2 q = make_uint2(e2m1x8_exact(xs, xv[p], enc, sc16), e2m1x8_exact(xs + 8, xv[p] + 8, enc, sc16 + 8));
+            const int64_t row = m0 + rr0 + p * kRpp;
+            if (row < a.B) {
+              *reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.codes) + row * (a.M / 2) + col / 2) = q;
+              if (!mx)
+                a.sf[sf_swizzle_offset(row, col / 16, kbp)] = sfb;
+              else if ((lane & 1) == 0)
+                a.sf[sf_swizzle_offset(row, col / 32, kbp)] = sfb;
+            }
           }
         }
       }
+      // this warp is done reading the stage
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s_]);
     }
     // the unit's partial down tile: wait for its last MMAs, then TMEM -> ws_down
     if (rp > 0) {
       if (warp < 4 && !abort_sh) {
-        const uint32_t gl = g + nsub - 1;
-        const bool ok = mbar_wait_warp(&mma_bar[gl % stages], (gl / stages) & 1, a.status, &abort_sh);
+        const bool ok = mbar_wait_warp(&unit_bar, unit_parity, a.status, &abort_sh);
         tc_fence_after();
         const int row = m0 + warp * 32 + lane;
         float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp;
@@ -468,10 +475,12 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const ActArgs a) {
       }
     }
     g += nsub;
+    unit_parity ^= 1u;
     __syncthreads();   // the drain is done and the column constants are free before the next unit
     if (abort_sh) break;
   }
-  cp_async_wait<0>();   // no copy is still on its way when the CTA ends
+  // no copy is still on its way when the CTA ends: the last segments' loads
+  // were all waited for above, unless a wait ran out (then the status records it)
   // fp4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
   if (nv || mx) {
     const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
@@ -512,12 +521,21 @@ cudaError_t launch_max(const ActArgs& a, int grid, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, act_max_kernel<TIn>, a);
 }
 
-template <typename TIn>
+template <typename TIn, bool kFp4>
 cudaError_t launch_quant(const ActArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(act_quant_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  const CUtensorMapDataType dt = kEsz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUtensorMap tx, tl;
+  if (!make_tmap_2d(&tx, a.x, dt, kEsz, a.M, a.B, a.ldx, kTileBytes / kEsz, kRows, true))
+    return cudaErrorInvalidValue;
+  // without the down factor the ld map is never used: a valid stand-in (x) keeps the argument defined
+  if (!make_tmap_2d(&tl, a.rank_pad > 0 ? a.ld : a.x, dt, kEsz, a.M, a.rank_pad > 0 ? a.rank_pad : a.B,
+                    a.rank_pad > 0 ? a.M : a.ldx, kTileBytes / kEsz, a.rank_pad > 0 ? a.rank_pad : kRows, true))
+    return cudaErrorInvalidValue;
+  cudaError_t err = cudaFuncSetAttribute(act_quant_kernel<TIn, kFp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  act_quant_kernel<TIn><<<grid, kWork, smem, stream>>>(a);
+  act_quant_kernel<TIn, kFp4><<<grid, kWork, smem, stream>>>(tx, tl, a);
   return cudaGetLastError();
 }
 
@@ -538,12 +556,12 @@ void finish_act_plan(ActPlan& p) {
   // units of at most max_unit_cols columns (the per-column constants live in
   // shared memory beside the stages)
   const int min_split = static_cast<int>(ceil_div(static_cast<int64_t>(p.nsteps) * p.tile_k,
-                                                  max_unit_cols(p.rank_pad)));
+                                                  max_unit_cols(p.rank_pad)));   // nsteps: segments
   p.ksplit = std::max(p.ksplit, std::min(p.nsteps, min_split));
   p.nunits = p.nrb * p.ksplit;
   const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
   const int unit_cols = steps_max * p.tile_k;
-  const int sub_max = (steps_max * kTileBytes + kSub - 1) / kSub;
+  const int sub_max = steps_max;
   const size_t sb = static_cast<size_t>(quant_stage_bytes(p.rank_pad));
   const size_t colv = static_cast<size_t>(unit_cols) * sizeof(float);
   p.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kQuantSmemBudget - 1024 - colv) / sb));
@@ -577,7 +595,7 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool al
     p.rank_pad = rank_pad;
     p.bf16 = xdt == SVDQ_BF16;
   }
-  p.tile_k = p.bf16 ? 64 : 32;
+  p.tile_k = p.bf16 ? kSub / 2 : kSub / 4;   // columns of a 256-byte segment
   p.nrb = static_cast<int>(ceil_div(B, kRows));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
   // at most one unit per SM: split K until the units cover the SMs
@@ -667,8 +685,11 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   cudaError_t err = xdt == SVDQ_BF16 ? launch_max<__nv_bfloat16>(a, max_grid, stream)
                                      : launch_max<float>(a, max_grid, stream);
   if (err != cudaSuccess) return err;
-  return xdt == SVDQ_BF16 ? launch_quant<__nv_bfloat16>(a, p.grid, q.smem, stream)
-                          : launch_quant<float>(a, p.grid, q.smem, stream);
+  const bool f4 = fmt.kind != SVDQ_KIND_INT;
+  if (xdt == SVDQ_BF16)
+    return f4 ? launch_quant<__nv_bfloat16, true>(a, p.grid, q.smem, stream)
+              : launch_quant<__nv_bfloat16, false>(a, p.grid, q.smem, stream);
+  return f4 ? launch_quant<float, true>(a, p.grid, q.smem, stream) : launch_quant<float, false>(a, p.grid, q.smem, stream);
 }
 
 }  // namespace svdq

@@ -85,6 +85,21 @@ __device__ __forceinline__ void unpack16(const uint4 u, float* v) {
   }
 }
 
+// 16 packed bytes (32 two's-complement nibbles, element 2j in the low nibble
+// of byte j) -> 32 int8 codes in element order.
+__device__ __forceinline__ void widen_int4(const uint4 v, uint32_t (&o)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo = w[i] & 0x0F0F0F0Fu;          // elements 8i + 0, 2, 4, 6
+    uint32_t hi = (w[i] >> 4) & 0x0F0F0F0Fu;   // elements 8i + 1, 3, 5, 7
+    lo |= (lo & 0x08080808u) * 0x1Eu;          // sign-extend each nibble to its byte
+    hi |= (hi & 0x08080808u) * 0x1Eu;
+    o[2 * i] = __byte_perm(lo, hi, 0x5140);
+    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+}
+
 // ------------------------------------------------------------ exact rounding
 // Every code is the correctly rounded value of a real quotient (the grid of
 // "SVDQuant Smoothing, Low-rank and Residual Quantization", Formula item 3:
@@ -135,19 +150,21 @@ constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
 __device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8],
                                             const float* scale8, float s, int qmax) {
   uint32_t f[8];
-  bool near = false;
+  uint32_t near = 0u;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float t = __fmul_rn(v[j], ck[j]);
     const float fs = __fadd_rn(t, kRintMagic);
     f[j] = __float_as_uint(fs);
-    near |= fabsf(__fsub_rn(t, __fsub_rn(fs, kRintMagic))) > kNearHalf;
+    near |= (fabsf(__fsub_rn(t, __fsub_rn(fs, kRintMagic))) > kNearHalf ? 1u : 0u) << j;
   }
-  if (__builtin_expect(near, 0)) {
+  if (__builtin_expect(near != 0u, 0)) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int q_est = static_cast<int>(f[j] & 0xFFu) - static_cast<int>((f[j] & 0x80u) << 1);
-      f[j] = static_cast<uint32_t>(int_code_fix(v[j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
+      if (near & (1u << j)) {
+        const int q_est = static_cast<int>(f[j] & 0xFFu) - static_cast<int>((f[j] & 0x80u) << 1);
+        f[j] = static_cast<uint32_t>(int_code_fix(v[j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
+      }
     }
   }
   const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
@@ -247,9 +264,11 @@ __device__ __forceinline__ uint32_t e2m1x8_exact(const float* v, const float* a,
   }
   uint32_t out = f32x8_to_e2m1(v);
   const uint32_t wl = f32x8_to_e2m1(lo), wh = f32x8_to_e2m1(hi);
-  if (__builtin_expect(wl != wh || wl != out, 0)) {
+  const uint32_t diff = (wl ^ wh) | (wl ^ out);   // nibbles of the elements near a boundary
+  if (__builtin_expect(diff != 0u, 0)) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+      if (((diff >> (4 * j)) & 0xFu) == 0u) continue;
       const uint32_t idx_est = (out >> (4 * j)) & 7u;
       const double P = fabs(static_cast<double>(a[j])) * static_cast<double>(g);
       const double C = c8 != nullptr ? static_cast<double>(__ldg(c8 + j)) : 1.0;

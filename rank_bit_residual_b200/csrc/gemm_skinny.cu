@@ -39,6 +39,7 @@
 
 #include <algorithm>
 
+#include "encode.cuh"
 #include "gemm_common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -81,21 +82,6 @@ struct SkinnyArgs {
   const uint8_t* sfx;   // fp4 activation scales, 128x4 layout
   unsigned* status;
 };
-
-// 16 packed bytes (32 two's-complement nibbles, element 2j in the low nibble
-// of byte j) -> 32 int8 codes in element order.
-__device__ __forceinline__ void widen_int4(const uint4 v, uint32_t (&o)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t lo = w[i] & 0x0F0F0F0Fu;          // elements 8i + 0, 2, 4, 6
-    uint32_t hi = (w[i] >> 4) & 0x0F0F0F0Fu;   // elements 8i + 1, 3, 5, 7
-    lo |= (lo & 0x08080808u) * 0x1Eu;          // sign-extend each nibble to its byte
-    hi |= (hi & 0x08080808u) * 0x1Eu;
-    o[2 * i] = __byte_perm(lo, hi, 0x5140);
-    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);
-  }
-}
 
 // Dequantisation factor of the residual accumulator (s_x s_w for INT,
 // 1 / (gs_x gs_w) for fp4, 1 for MXFP4; unused for the raw int32 product).

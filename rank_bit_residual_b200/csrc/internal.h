@@ -47,9 +47,9 @@ struct ActPlan {
   int64_t B, M;
   int32_t rank_pad;
   bool bf16;       // x is bf16 (else fp32)
-  int tile_k;      // elements per 128-byte K tile (64 bf16 / 32 fp32)
+  int tile_k;      // large batch: columns of a 256-byte row segment (128 bf16 / 64 fp32)
   int nrb;         // row blocks of 128
-  int nsteps;      // K tiles
+  int nsteps;      // large batch: row segments (the unit of the K split)
   int ksplit;      // K ranges per row block
   int nunits;      // nrb * ksplit work units
   int stages;      // large-batch quantise kernel: segment stages in shared memory
@@ -108,6 +108,11 @@ cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const
                             const void* down2, int64_t B, const void* bias, void* y,
                             svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
                             bool* bad_args);
+
+// The whole linear for B <= 2 rows with INT weights in one launch (decode.cu);
+// false (nothing launched) when the shape or the alignment does not allow it.
+bool launch_decode(const svdq_weight* w, const void* x, svdq_dtype xdt, int64_t B, int64_t ldx, const void* bias,
+                   void* y, svdq_dtype ydt, int64_t ldy, bool chained, cudaStream_t st, cudaError_t* err);
 
 // NVFP4 or MXFP4, after w->fmt.kind
 cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,

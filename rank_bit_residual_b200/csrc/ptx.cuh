@@ -395,6 +395,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
+// 32-bit load from the shared memory of a CTA of the cluster (cluster address
+// from mapa_shared).
+__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 // Whole-cluster barrier (all threads of both CTAs); only used right after the
 // mbarriers are initialised, when both CTAs of a cluster are known to run.
 __device__ __forceinline__ void cluster_sync() {

@@ -166,3 +166,32 @@ def test_large_batch_linear_equals_separate_stages(B, fmt):
         y = rb.svdq_linear(w.w, x, bias=b, out_dtype=torch.float32)
         assert torch.equal(y, y_sep)
     assert rb.svdq_check_status() == rb.SVDQ_OK
+
+
+@pytest.mark.parametrize("B", [1, 2])
+@pytest.mark.parametrize("M,N,rank,fmt,packed,bias,xdt", [
+    (4096, 4096, 32, "int4", True, False, "bf16"),
+    (1024, 272, 16, "int4", False, True, "bf16"),
+    (512, 48, 0, "int8", False, False, "f32"),
+    (2048, 1040, 256, "int4", True, True, "f32"),
+    (96, 16, 1, "int2", False, True, "bf16"),
+])
+def test_single_launch_decode_matches_oracle(B, M, N, rank, fmt, packed, bias, xdt):
+    """One or two rows with INT weights run as one kernel (quantisation, down-projection
+    split over a cluster, dp4a dot products and epilogue): Y matches the oracle, and
+    the staged entry points agree within the same tolerance."""
+    wl = make_case(B, M, N, rank=rank, seed=B * 11 + M + N, dtype=xdt, bias=bias)
+    w = SyntheticWeight(M, N, rank, fmt, seed=N + rank + 3, scale=wl.scale, packed=packed)
+    b = to_dev(wl.bias, torch.bfloat16) if bias else None
+    x = x_tensor(wl)
+    y32 = rb.svdq_linear(w.w, x, bias=b, out_dtype=torch.float32)
+    y16 = rb.svdq_linear(w.w, x, bias=b, out_dtype=torch.bfloat16)
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    want = w.oracle_y(wl.x, wl.bias if bias else None)
+    assert_y_close(y32.cpu().numpy(), want, f"decode B={B} {M}x{N} r={rank} {fmt}")
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    scale = to_dev(wl.scale, torch.float32)
+    ld = w.w.ld if xdt == "bf16" else w.w.ld32
+    codes, sf, s, down = rb.svdq_quantize_act(x, scale, fmt, ld=ld if rank else None)
+    y_st = rb.svdq_residual_linear(w.w, codes, sf, s, down, bias=b, out_dtype=torch.float32)
+    assert_y_close(y32.cpu().numpy(), y_st.cpu().numpy().astype(np.float64), "fused vs staged")
