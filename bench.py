@@ -270,9 +270,10 @@ SOAK_MS = 400.0          # back-to-back steps just before a sampled timed region
 
 
 def launches_per_step(wl) -> int:
-    """Kernels one svdq_linear call launches: one for one or two rows with INT weights
-    (the single-launch decode kernel), else two for the activation pass and one GEMM."""
-    return 1 if (wl.fmt == "int" and wl.B <= 2) else 3
+    """Kernels one svdq_linear call launches: one for up to 16 rows with INT weights
+    (the single-launch decode kernel, whose shared memory holds every decode shape
+    benched here), else two for the activation pass and one GEMM."""
+    return 1 if (wl.fmt == "int" and wl.B <= 16) else 3
 
 
 def fmt_name(wl):

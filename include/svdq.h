@@ -222,11 +222,16 @@ svdq_status svdq_quantize_act_workspace_size(int64_t B, int64_t M, svdq_fmt fmt,
  * array and it keeps the last call's contents: every scratch word a call reads
  * is written by that call first, so nothing needs clearing, but calls that
  * overlap on the GPU (other streams or other host threads) race on it.
- * The plan is svdq_quantize_act's, with the K split (column ranges per row
- * block) halved until the scratch fits: 4 * B * rank_pad * ksplit bytes of
- * partial down tiles plus the partial maxima, 4 * grid bytes rounded up to 256,
- * plus 256. At ksplit = 1 that limits B * rank_pad to a little under 2^21 (for
- * example B = 8192 at rank_pad 128 fits, B = 16384 at rank_pad 128 does not).
+ * The plan is svdq_quantize_act's while its scratch fits. Most of the scratch
+ * is partial down tiles, 4 * B * rank_pad * slots bytes, slots being the most
+ * pieces one 128-row block is cut into (for more than 128 rows the plan spreads
+ * all 256-byte row segments evenly over one CTA per SM); the rest is the
+ * partial maxima (4 bytes per CTA of the maximum pass) and one counter per row
+ * block, each rounded up to 256 bytes, plus 256. When that does not fit, the
+ * plan takes equal column ranges per row block (the K split) and halves their
+ * number until it fits. At one range per row block that limits B * rank_pad
+ * to a little under 2^21 (for example B = 8192 at rank_pad 128 fits, B = 16384
+ * at rank_pad 128 does not).
  * Larger shapes return SVDQ_EWORKSPACE and launch nothing. The argument checks
  * and their status codes are those of svdq_quantize_act.
  */

@@ -51,8 +51,7 @@ namespace svdq {
 
 namespace {
 
-constexpr int kWorkWarps = 16;
-constexpr int kWork = 32 * kWorkWarps;      // threads of the quantise kernel
+constexpr int kWork = 512;                  // threads of the quantise kernel (one CTA per SM)
 constexpr int kRows = 128;                  // rows per unit
 constexpr int kTileBytes = 128;             // bytes of a row per column tile (64 bf16 / 32 fp32)
 constexpr int kSub = 256;                   // bytes of a row per segment (two tiles)
@@ -60,6 +59,7 @@ constexpr int kMaxStages = 6;
 constexpr int kMaxThreads = 256;            // threads of the maximum kernel
 constexpr int kMaxSlab = 2048;              // bytes of a row per maximum-kernel CTA (16 per thread)
 constexpr int kMaxCtasPerSm = 4;
+constexpr int kFlatMinSegs = 8;             // segments per SM from which the flat partition pays
 
 // Bytes of one quantise-kernel stage: x and ld as two 128-byte K blocks each; a
 // multiple of 1024 so every block keeps the swizzle atom.
@@ -78,6 +78,7 @@ struct ActArgs {
   int64_t ldx;
   int nsteps;       // 256-byte segments of a row (the unit of the K split)
   int ksplit, nrb, nunits, rank_pad, has_ld, fmt_kind, qmax;
+  int flat;         // 1: flat partition of the segments over the CTAs (else K split units)
   int nparts;       // partial maxima written by the maximum kernel (0: none needed)
   int max_rpc;      // maximum kernel: rows per CTA
   int max_nslabs;   // maximum kernel: column slabs of kMaxSlab bytes
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
                                                              const __grid_constant__ CUtensorMap tm_ld,
                                                              const ActArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));
+  constexpr int kWorkWarps = kWork / 32;
   constexpr int kSubCols = kSub / kEsz;             // 128 bf16 or 64 fp32 columns
   constexpr int kPer16 = 16 / kEsz;                 // elements per 16-byte piece
   constexpr int kTileK = kTileBytes / kEsz;         // columns per K tile
@@ -294,12 +296,41 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
   };
   uint32_t g = 0;   // segments begun so far: stage g % stages, barrier phase (g / stages) & 1
   uint32_t unit_parity = 0;
-  for (int unit = blockIdx.x; unit < a.nunits; unit += gridDim.x) {
-    const int rb = unit % a.nrb, sp = unit / a.nrb;
+  // Pieces of work: a row block and a range of its segments. Flat partition:
+  // CTA i takes segments [W i / G, W (i + 1) / G) of all W = nrb * nsteps
+  // segments in row-block-major order (every SM busy, at most one segment of
+  // imbalance), which cuts a row block into the pieces of consecutive CTAs;
+  // piece p of a row block writes partial slot p. Split partition: unit u =
+  // (row block u % nrb, K range u / nrb of ksplit equal ranges), CTAs striding
+  // over the units.
+  const int64_t W = static_cast<int64_t>(a.nrb) * a.nsteps;
+  const int G = static_cast<int>(gridDim.x);
+  auto cta_of = [&](int64_t f) { return static_cast<int>(((f + 1) * G - 1) / W); };   // CTA holding segment f
+  int64_t f = a.flat ? W * blockIdx.x / G : 0;
+  const int64_t f_end = a.flat ? W * (blockIdx.x + 1) / G : 0;
+  int unit = blockIdx.x;
+  while (true) {
+    int rb, sp, npieces, k_lo, k_hi;
+    if (a.flat) {
+      if (f >= f_end) break;
+      rb = static_cast<int>(f / a.nsteps);
+      k_lo = static_cast<int>(f - static_cast<int64_t>(rb) * a.nsteps);
+      k_hi = static_cast<int>(min(static_cast<int64_t>(a.nsteps), k_lo + (f_end - f)));
+      f += k_hi - k_lo;
+      const int first = cta_of(static_cast<int64_t>(rb) * a.nsteps);
+      sp = static_cast<int>(blockIdx.x) - first;
+      npieces = cta_of(static_cast<int64_t>(rb) * a.nsteps + a.nsteps - 1) - first + 1;
+    } else {
+      if (unit >= a.nunits) break;
+      rb = unit % a.nrb;
+      sp = unit / a.nrb;
+      npieces = a.ksplit;
+      // whole segments per unit: no box reaches into another unit's columns
+      k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
+      k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
+      unit += G;
+    }
     const int m0 = rb * kRows;
-    // whole segments per unit: no box reaches into another unit's columns
-    const int k_lo = static_cast<int>((static_cast<int64_t>(a.nsteps) * sp) / a.ksplit);
-    const int k_hi = static_cast<int>((static_cast<int64_t>(a.nsteps) * (sp + 1)) / a.ksplit);
     const int c_lo = k_lo * kSubCols;
     const int c_hi = min(a.M, k_hi * kSubCols);
     const int nsub = k_hi - k_lo;
@@ -392,7 +423,8 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
           for (int p = 0; p < kPasses; ++p) {
             float xs[16];   // the estimates fl(x r_k) of the raw elements xv[p]
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xv[p][j], cv[j]);
+            for (int j = 0; j < 16; j += 2)
+              upk2(fmul2_rn(pk2(xv[p][j], xv[p][j + 1]), pk2(cv[j], cv[j + 1])), xs[j], xs[j + 1]);
             float amax = block_amax_exact<16>(xv[p], xs, sc16);
             uint8_t sfb;
             float enc;
@@ -409,7 +441,8 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
               enc = d > 0.0f ? __fdiv_rn(gs_x, d) : 0.0f;
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xs[j] = __fmul_rn(xs[j], enc);
+            for (int j = 0; j < 16; j += 2)
+              upk2(fmul2_rn(pk2(xs[j], xs[j + 1]), pk2(enc, enc)), xs[j], xs[j + 1]);
             const uint2 q = make_uint2(e2m1x8_exact(xs, xv[p], enc, sc16), e2m1x8_exact(xs + 8, xv[p] + 8, enc, sc16 + 8));
             const int64_t row = m0 + rr0 + p * kRpp;
             if (row < a.B) {
@@ -453,7 +486,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
         __threadfence();   // the partial is visible before the unit is counted
       }
       __syncthreads();
-      if (tid == 0) last_sh = atomicAdd(a.ws_cnt + rb, 1u) == static_cast<unsigned>(a.ksplit - 1);
+      if (tid == 0) last_sh = atomicAdd(a.ws_cnt + rb, 1u) == static_cast<unsigned>(npieces - 1);
       __syncthreads();
       if (last_sh) {
         // every unit of this row block is done: down = the partials summed in
@@ -464,7 +497,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
         for (int i = tid; i < rows * rp; i += kWork) {
           const int row = m0 + i / rp, j = i % rp;
           float acc = 0.0f;
-          for (int z = 0; z < a.ksplit; ++z)
+          for (int z = 0; z < npieces; ++z)
             acc += __ldcg(a.ws_down + (static_cast<int64_t>(z) * a.B + row) * rp + j);
           acc = __fmul_rn(acc, mult);
           const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
@@ -553,13 +586,31 @@ void finish_act_plan(ActPlan& p) {
     finish_act_plan_small(p);
     return;
   }
-  // units of at most max_unit_cols columns (the per-column constants live in
+  // pieces of at most max_unit_cols columns (the per-column constants live in
   // shared memory beside the stages)
-  const int min_split = static_cast<int>(ceil_div(static_cast<int64_t>(p.nsteps) * p.tile_k,
-                                                  max_unit_cols(p.rank_pad)));   // nsteps: segments
-  p.ksplit = std::max(p.ksplit, std::min(p.nsteps, min_split));
-  p.nunits = p.nrb * p.ksplit;
-  const int steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+  const int seg_cap = std::max(1, max_unit_cols(p.rank_pad) / p.tile_k);
+  int steps_max;
+  if (p.flat) {
+    // every CTA a contiguous run of segments; as many CTAs as asked (the SMs),
+    // more if a run would outgrow the shared memory
+    const int64_t W = static_cast<int64_t>(p.nrb) * p.nsteps;
+    const int64_t G = std::min(W, std::max<int64_t>(std::max(p.qgrid, 1), ceil_div(W, seg_cap)));
+    p.grid = static_cast<int>(G);
+    p.nunits = p.grid;
+    // partial slots per row block: the most pieces a row block is cut into
+    auto cta_of = [&](int64_t f) { return ((f + 1) * G - 1) / W; };
+    int64_t maxp = 1;
+    for (int64_t rb = 0; rb < p.nrb; ++rb)
+      maxp = std::max(maxp, cta_of(rb * p.nsteps + p.nsteps - 1) - cta_of(rb * p.nsteps) + 1);
+    p.ksplit = static_cast<int>(maxp);
+    steps_max = static_cast<int>(std::min<int64_t>(p.nsteps, ceil_div(W, G)));
+  } else {
+    const int min_split = static_cast<int>(ceil_div(p.nsteps, seg_cap));
+    p.ksplit = std::max(p.ksplit, std::min(p.nsteps, min_split));
+    p.nunits = p.nrb * p.ksplit;
+    steps_max = (p.nsteps + p.ksplit - 1) / p.ksplit;
+    p.grid = std::min(p.nunits, num_sms());
+  }
   const int unit_cols = steps_max * p.tile_k;
   const int sub_max = steps_max;
   const size_t sb = static_cast<size_t>(quant_stage_bytes(p.rank_pad));
@@ -567,8 +618,6 @@ void finish_act_plan(ActPlan& p) {
   p.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kQuantSmemBudget - 1024 - colv) / sb));
   p.stages = std::max(2, std::min(p.stages, sub_max + 1));
   p.smem = sb * p.stages + colv + 1024;   // + alignment of the first stage to 1024 bytes
-  // one quantise CTA per SM (512 threads, most of the shared memory)
-  p.grid = std::min(p.nunits, num_sms());
   // maximum kernel: slabs of kMaxSlab bytes x row ranges, about kMaxCtasPerSm CTAs per SM
   const int esz = p.bf16 ? 2 : 4;
   p.max_nslabs = static_cast<int>(ceil_div(p.M * esz, kMaxSlab));
@@ -598,9 +647,19 @@ ActPlan plan_act(int64_t B, int64_t M, int32_t rank_pad, svdq_dtype xdt, bool al
   p.tile_k = p.bf16 ? kSub / 2 : kSub / 4;   // columns of a 256-byte segment
   p.nrb = static_cast<int>(ceil_div(B, kRows));
   p.nsteps = static_cast<int>(ceil_div(M, p.tile_k));
-  // at most one unit per SM: split K until the units cover the SMs
+  // one quantise CTA per SM (most of the shared memory). With many segments per
+  // SM they are spread flat (every SM busy; a CTA's run may be cut into two
+  // pieces, each with its own pipeline start and drain); with few, a piece's
+  // start and drain cost more than the SMs a K split leaves idle
   const int sms = num_sms();
-  p.ksplit = std::max(1, std::min(p.nsteps, sms / std::max(p.nrb, 1)));
+  const int64_t W = static_cast<int64_t>(p.nrb) * p.nsteps;
+  if (W >= static_cast<int64_t>(kFlatMinSegs) * sms) {
+    p.flat = 1;
+    p.qgrid = sms;
+  } else {
+    p.flat = 0;
+    p.ksplit = std::max(1, std::min(p.nsteps, sms / std::max(p.nrb, 1)));
+  }
   finish_act_plan(p);
   return p;
 }
@@ -655,6 +714,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   a.ldx = ldx;
   a.nsteps = p.nsteps;
   a.ksplit = p.ksplit;
+  a.flat = p.flat;
   a.nrb = p.nrb;
   a.nunits = p.nunits;
   a.rank_pad = has_ld ? p.rank_pad : 0;

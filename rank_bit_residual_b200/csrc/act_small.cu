@@ -66,30 +66,6 @@ struct SmallArgs {
 // padding make the 8 rows read by one MMA fragment load hit distinct banks.
 __host__ __device__ constexpr int chunk_pitch(int wc, int esz) { return wc * esz + 16; }
 
-// D[16x8] += A[16x16] B[16x8], bf16 operands, fp32 accumulators.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// D[16x8] += A[16x8] B[8x8], tf32 operands, fp32 accumulators.
-__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ uint32_t to_tf32(uint32_t f) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(__uint_as_float(f)));
-  return r;
-}
-
 template <typename TIn>
 __global__ void __launch_bounds__(kThreads, 1) act_small_stats_kernel(const SmallArgs a) {
   constexpr int kEsz = static_cast<int>(sizeof(TIn));

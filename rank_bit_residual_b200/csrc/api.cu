@@ -370,7 +370,8 @@ svdq_status svdq_linear_ex(const svdq_weight* w, const void* x, svdq_dtype x_dty
   LinearCarve c = carve_linear(w, B, workspace, workspace_bytes, x_dtype);
   if (!c.ok) return SVDQ_EWORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // one or two rows with INT weights: the whole linear in one launch
+  // up to 16 rows with INT weights: the whole linear in one launch (when its
+  // shared memory holds the CTA's weight rows and the codes of x)
   {
     cudaError_t e = cudaSuccess;
     if (launch_decode(w, x, x_dtype, B, ldx, bias, y, y_dtype, ldy, (flags & SVDQ_LINEAR_PDL) != 0, st, &e))

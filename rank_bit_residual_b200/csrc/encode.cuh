@@ -140,28 +140,62 @@ constexpr float kRintMagic = 12582912.0f;
 // half-integer: with |t| <= 128 (qmax <= 127) its error is below 2^-15.
 constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
 
+// Packed pairs of fp32 (sm_100a f32x2 arithmetic): each lane of the pair is
+// rounded to nearest even on its own, exactly as the scalar operation.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fmul2_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fsub2_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // INT codes of 8 consecutive columns of a row, packed as 8 bytes: the exact
 // round_half_even(x / (scale_k s)), estimated as rint(fl(x c_k)) with the
 // per-column constant c_k = fl(fl(1 / scale_k) fl(1 / s)) and re-decided by
 // int_code_fix where the estimate is near a half-integer. scale8 points at the
 // 8 columns' smoothing scales (read only on that rare path). The estimate
 // never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in magnitude, so the fast
-// path needs no clamp.
+// path needs no clamp. The fast path runs on pairs of elements (f32x2); the
+// rare path finds the flagged elements again with the same scalar operations.
 __device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8],
                                             const float* scale8, float s, int qmax) {
   uint32_t f[8];
-  uint32_t near = 0u;
+  bool near = false;
+  const uint64_t mg = pk2(kRintMagic, kRintMagic);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float t = __fmul_rn(v[j], ck[j]);
-    const float fs = __fadd_rn(t, kRintMagic);
-    f[j] = __float_as_uint(fs);
-    near |= (fabsf(__fsub_rn(t, __fsub_rn(fs, kRintMagic))) > kNearHalf ? 1u : 0u) << j;
+  for (int j = 0; j < 8; j += 2) {
+    const uint64_t t = fmul2_rn(pk2(v[j], v[j + 1]), pk2(ck[j], ck[j + 1]));
+    const uint64_t fs = fadd2_rn(t, mg);
+    const uint64_t d = fsub2_rn(t, fsub2_rn(fs, mg));
+    float d0, d1, s0, s1;
+    upk2(d, d0, d1);
+    upk2(fs, s0, s1);
+    f[j] = __float_as_uint(s0);
+    f[j + 1] = __float_as_uint(s1);
+    near = near || fabsf(d0) > kNearHalf || fabsf(d1) > kNearHalf;
   }
-  if (__builtin_expect(near != 0u, 0)) {
+  if (__builtin_expect(near, 0)) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (near & (1u << j)) {
+      const float t = __fmul_rn(v[j], ck[j]);
+      if (fabsf(__fsub_rn(t, __fsub_rn(__fadd_rn(t, kRintMagic), kRintMagic))) > kNearHalf) {
         const int q_est = static_cast<int>(f[j] & 0xFFu) - static_cast<int>((f[j] & 0x80u) << 1);
         f[j] = static_cast<uint32_t>(int_code_fix(v[j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
       }
@@ -257,10 +291,13 @@ static __device__ __noinline__ uint32_t e2m1_index_fix(double P, double C, uint3
 __device__ __forceinline__ uint32_t e2m1x8_exact(const float* v, const float* a, float g,
                                                  const float* c8) {
   float lo[8], hi[8];
+  const uint64_t ml = pk2(1.0f - 1.0f / 524288.0f, 1.0f - 1.0f / 524288.0f);
+  const uint64_t mh = pk2(1.0f + 1.0f / 524288.0f, 1.0f + 1.0f / 524288.0f);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    lo[j] = __fmul_rn(v[j], 1.0f - 1.0f / 524288.0f);
-    hi[j] = __fmul_rn(v[j], 1.0f + 1.0f / 524288.0f);
+  for (int j = 0; j < 8; j += 2) {
+    const uint64_t vv = pk2(v[j], v[j + 1]);
+    upk2(fmul2_rn(vv, ml), lo[j], lo[j + 1]);
+    upk2(fmul2_rn(vv, mh), hi[j], hi[j + 1]);
   }
   uint32_t out = f32x8_to_e2m1(v);
   const uint32_t wl = f32x8_to_e2m1(lo), wh = f32x8_to_e2m1(hi);

@@ -50,7 +50,9 @@ struct ActPlan {
   int tile_k;      // large batch: columns of a 256-byte row segment (128 bf16 / 64 fp32)
   int nrb;         // row blocks of 128
   int nsteps;      // large batch: row segments (the unit of the K split)
-  int ksplit;      // K ranges per row block
+  int ksplit;      // K ranges per row block (flat partition: the most pieces a row block is cut into)
+  int flat;        // large batch: 1 = flat partition of all segments over qgrid CTAs, 0 = ksplit units
+  int qgrid;       // large batch, flat: CTAs asked for (more if a piece would not fit shared memory)
   int nunits;      // nrb * ksplit work units
   int stages;      // large-batch quantise kernel: segment stages in shared memory
   int grid;        // CTAs of the quantise (large batch) or first (short batch) kernel

@@ -70,9 +70,19 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
   if (st != SVDQ_OK || B == 0) return st;
 
   // Same launch plan as svdq_quantize_act, with fewer K splits if that is what
-  // it takes to fit the fixed array; beyond that the shape is refused.
+  // it takes to fit the fixed array; beyond that the shape is refused. The
+  // large-batch flat partition cuts a row block into pieces at CTA boundaries,
+  // one partial slot each; when those slots do not fit, the plan goes over to
+  // K split units, whose count per row block it can then halve.
   const int32_t rp = (ld != nullptr) ? rank_pad : 0;
+  auto to_split = [](ActPlan& q) {
+    if (q.small || !q.flat) return;
+    q.flat = 0;
+    q.ksplit = std::max(1, std::min(q.nsteps, num_sms() / std::max(q.nrb, 1)));
+    finish_act_plan(q);
+  };
   ActPlan p = plan_act(B, M, rp, x_dtype);
+  if (act_scratch_bytes(p) > kNoallocScratchBytes) to_split(p);
   while (act_scratch_bytes(p) > kNoallocScratchBytes && p.ksplit > 1) {
     const int before = p.ksplit;
     p.ksplit = std::max(1, p.ksplit / 2);
@@ -80,7 +90,10 @@ extern "C" svdq_status svdq_quantize_act_noalloc(
     if (!p.small && p.ksplit >= before) break;   // the split cannot shrink further
     // fewer, wider column chunks of the short-batch kernel may outgrow its
     // shared memory: continue with the large-batch plan then
-    if (p.small && p.smem > kActSmallSmemMax) p = plan_act(B, M, rp, x_dtype, false);
+    if (p.small && p.smem > kActSmallSmemMax) {
+      p = plan_act(B, M, rp, x_dtype, false);
+      if (act_scratch_bytes(p) > kNoallocScratchBytes) to_split(p);
+    }
   }
   if (act_scratch_bytes(p) > kNoallocScratchBytes) return SVDQ_EWORKSPACE;
 

@@ -168,18 +168,20 @@ def test_large_batch_linear_equals_separate_stages(B, fmt):
     assert rb.svdq_check_status() == rb.SVDQ_OK
 
 
-@pytest.mark.parametrize("B", [1, 2])
+@pytest.mark.parametrize("B", [1, 2, 3, 8, 16])
 @pytest.mark.parametrize("M,N,rank,fmt,packed,bias,xdt", [
     (4096, 4096, 32, "int4", True, False, "bf16"),
+    (3072, 3072, 128, "int8", False, True, "bf16"),
+    (1056, 2000, 48, "int4", True, False, "f32"),
     (1024, 272, 16, "int4", False, True, "bf16"),
     (512, 48, 0, "int8", False, False, "f32"),
     (2048, 1040, 256, "int4", True, True, "f32"),
     (96, 16, 1, "int2", False, True, "bf16"),
 ])
 def test_single_launch_decode_matches_oracle(B, M, N, rank, fmt, packed, bias, xdt):
-    """One or two rows with INT weights run as one kernel (quantisation, down-projection
-    split over a cluster, dp4a dot products and epilogue): Y matches the oracle, and
-    the staged entry points agree within the same tolerance."""
+    """Up to 16 rows with INT weights run as one kernel (maximum, down-projection and
+    codes split over a cluster, dp4a dot products and epilogue): Y matches the oracle,
+    and the staged entry points agree within the same tolerance."""
     wl = make_case(B, M, N, rank=rank, seed=B * 11 + M + N, dtype=xdt, bias=bias)
     w = SyntheticWeight(M, N, rank, fmt, seed=N + rank + 3, scale=wl.scale, packed=packed)
     b = to_dev(wl.bias, torch.bfloat16) if bias else None
