@@ -247,7 +247,11 @@ svdq_status svdq_quantize_act_noalloc(const void* x, svdq_dtype x_dtype, int64_t
  *   Y = x ld^T lu^T + alpha * (Q(X_hat) . Q(R)) [+ bias]
  * with alpha = s_x * s_w (INT), 1 / (gs_x * gs_w) (NVFP4) or 1 (MXFP4). Runs the fused
  * activation pass, then one tensor-core GEMM whose epilogue adds the low-rank
- * up-projection and the bias.
+ * up-projection and the bias; up to 16 rows with INT weights run as one
+ * kernel. The workspace (svdq_linear_workspace_size) holds the activation
+ * codes, scales and down-projection, the activation pass's scratch, and for
+ * INT with more than 128 rows the partial accumulators of the GEMM tiles it
+ * splits along K (the tiles of a last round that would leave most SMs idle).
  *
  *   w        prepared weight (svdq_prepare)
  *   x        device [B, M] (ldx >= M), bf16 or fp32 (fp32 needs w->ld32)

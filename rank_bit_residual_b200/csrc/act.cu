@@ -93,6 +93,8 @@ struct ActArgs {
   float* ws_down;   // [ksplit][B][rank_pad]
   float* ws_max;    // [nparts]
   unsigned* ws_cnt; // [nrb] units of a row block done
+  unsigned* zero_words;   // cleared by the maximum kernel for the GEMM that follows (nullable)
+  int nzero;
   void* codes;
   uint8_t* sf;
   __nv_bfloat16* down;
@@ -138,8 +140,12 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
   // chained after another linear: x is that linear's output
   if (a.chained) pdl_wait();
   const int tid = threadIdx.x;
-  if (blockIdx.x == 0)
+  // block 0 clears the quantise kernel's row-block counters (and any words the
+  // GEMM after this pass needs zeroed)
+  if (blockIdx.x == 0) {
     for (int i = tid; i < a.nrb; i += kMaxThreads) a.ws_cnt[i] = 0u;
+    for (int i = tid; i < a.nzero; i += kMaxThreads) a.zero_words[i] = 0u;
+  }
   if (a.nparts == 0) return;
   const int slab = blockIdx.x % a.max_nslabs, rc = blockIdx.x / a.max_nslabs;
   const int col = slab * (kMaxSlab / kEsz) + (tid & 127) * kPer16;
@@ -410,8 +416,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
         for (int j = 0; j < kE; ++j) cv[j] = colv[cs + j];
         if constexpr (!kFp4) {
           uint2 q[kPasses];
-#pragma unroll
-          for (int p = 0; p < kPasses; ++p) q[p] = int_codes8(xv[p], cv, a.scale + col, s, a.qmax);
+          int_codes8_rows<kPasses>(xv, cv, a.scale + col, s, a.qmax, q);
 #pragma unroll
           for (int p = 0; p < kPasses; ++p) {
             const int64_t row = m0 + rr0 + p * kRpp;
@@ -681,7 +686,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
                        const float* w_global_scale, const void* ld, void* codes, void* sf,
                        float* act_scale, void* down, void* scratch, cudaStream_t stream,
-                       bool* bad_args) {
+                       bool* bad_args, unsigned* zero_words, int nzero) {
   *bad_args = false;
   if (p.B == 0) return cudaSuccess;
   if (p.small)
@@ -741,6 +746,8 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
   // as many MMA issuers (up to 4) as TMEM holds accumulators of rank_pad columns
   a.nacc = a.rank_pad > 0 ? static_cast<int>(std::min<uint32_t>(4u, 512u / tmem_cols_for(a.rank_pad))) : 1;
   a.chained = p.chained;
+  a.zero_words = zero_words;
+  a.nzero = zero_words != nullptr ? nzero : 0;
   const int max_grid = need_max ? p.nparts : 1;
   cudaError_t err = xdt == SVDQ_BF16 ? launch_max<__nv_bfloat16>(a, max_grid, stream)
                                      : launch_max<float>(a, max_grid, stream);

@@ -172,6 +172,7 @@ struct LinearCarve {
   float* act_scale;
   void* down;
   void* act_scratch;
+  void* split;
   size_t bytes;
   bool ok;
 };
@@ -186,6 +187,9 @@ LinearCarve carve_linear(const svdq_weight* w, int64_t B, void* ws, size_t ws_by
   c.act_scale = static_cast<float*>(cv.take(16));
   c.down = cv.take(static_cast<size_t>(B) * 2 * w->rank_pad * 2);
   c.act_scratch = cv.take(act_scratch_bytes(p));
+  // the pair GEMM's K split of its last round (INT, more than 128 rows)
+  const size_t split = (w->fmt.kind == SVDQ_KIND_INT && B > 128) ? pair_split_bytes(B, w->M, w->N) : 0;
+  c.split = split > 0 ? cv.take(split) : nullptr;
   c.bytes = cv.off;
   c.ok = cv.ok;
   return c;
@@ -380,15 +384,22 @@ svdq_status svdq_linear_ex(const svdq_weight* w, const void* x, svdq_dtype x_dty
   ActPlan p = plan_act(B, w->M, w->rank_pad, x_dtype);
   p.chained = (flags & SVDQ_LINEAR_PDL) ? 1 : 0;
   bool bad = false;
+  // the pair GEMM's split counters are cleared by the activation pass
+  unsigned* zero = c.split != nullptr
+                       ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(c.split) +
+                                                     pair_split_counter_offset(B, w->M, w->N))
+                       : nullptr;
   cudaError_t e = launch_act(p, x, x_dtype, ldx, w->scale, w->fmt, act_global_scale,
                              w->fmt.kind == SVDQ_KIND_NVFP4 ? w->w_scale : nullptr,
                              w->rank > 0 ? ld : nullptr, c.codes, c.sf, c.act_scale,
-                             w->rank > 0 ? c.down : nullptr, c.act_scratch, st, &bad);
+                             w->rank > 0 ? c.down : nullptr, c.act_scratch, st, &bad, zero,
+                             zero != nullptr ? pair_split_counters(B, w->M, w->N) : 0);
   if (bad) return SVDQ_EUNSUPPORTED;
   if (e != cudaSuccess) return SVDQ_ECUDA;
   if (w->fmt.kind == SVDQ_KIND_INT) {
     e = launch_gemm_int(w, static_cast<const int8_t*>(c.codes), c.act_scale,
-                        w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, false, true, st, &bad);
+                        w->rank > 0 ? c.down : nullptr, B, bias, y, y_dtype, ldy, false, true, st, &bad,
+                        c.split);
   } else {
     e = launch_gemm_fp4(w, static_cast<const uint8_t*>(c.codes),
                           static_cast<const uint8_t*>(c.sf), c.act_scale,

@@ -53,7 +53,7 @@ struct DecodeArgs {
   int sstride;       // bytes between rows of the x and ld shares
   int wstride;       // bytes between weight rows
   int astride;       // bytes between rows of the codes
-  int lstride;       // bytes between lu rows
+  int lstride;       // bytes between lu rows (4 rank_pad: one bulk copy)
   int mtiles, ksub;  // 16-row weight tiles; warps splitting K per tile
   int64_t ldx, ldy;
   const void* x;
@@ -197,16 +197,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
       }
     };
     auto issue_w = [&]() {
-      const uint32_t lrow = static_cast<uint32_t>(g.rp) * 4u;
-      if (lane == 0) mbar_arrive_expect_tx(&bar[1], static_cast<uint32_t>(rows) * (g.row_bytes + lrow));
+      const uint32_t ltot = static_cast<uint32_t>(rows) * static_cast<uint32_t>(g.rp) * 4u;
+      if (lane == 0) mbar_arrive_expect_tx(&bar[1], static_cast<uint32_t>(rows * g.row_bytes) + ltot);
       __syncwarp();
-      for (int r = lane; r < rows; r += 32) {
+      for (int r = lane; r < rows; r += 32)
         bulk_load(ws + static_cast<size_t>(r) * g.wstride, g.w + static_cast<int64_t>(n0 + r) * g.row_bytes,
                   static_cast<uint32_t>(g.row_bytes), &bar[1]);
-        if (lrow > 0)
-          bulk_load(lus + static_cast<size_t>(r) * g.lstride,
-                    reinterpret_cast<const uint8_t*>(g.lu) + static_cast<int64_t>(n0 + r) * lrow, lrow, &bar[1]);
-      }
+      if (ltot > 0 && lane == 31)
+        bulk_load(lus, reinterpret_cast<const uint8_t*>(g.lu) + static_cast<int64_t>(n0) * g.rp * 4, ltot, &bar[1]);
     };
     // a chained launch (x is the previous linear's output) starts the weight
     // side before it waits for that kernel; otherwise x goes first (the
@@ -406,8 +404,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   __syncthreads();    // the partial dot products and the down sums
 
   // ---- epilogue: one thread per output, consecutive threads along the batch
-  // (then n), so the lu rows and the partial sums are read without bank conflicts
+  // (then n); each lane starts the up-projection at its own column, so the lu
+  // rows and the down sums are read (nearly) without bank conflicts
   const float alpha = s * __ldg(g.s_w);
+  const int q0 = g.rp > 0 ? lane % g.rp : 0;
   for (int o = tid; o < B * rows; o += kDecThreads) {
     const int r = o / B, b = o - r * B;
     const int mt = r >> 4, rr = r & 15;
@@ -416,7 +416,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     const __nv_bfloat16* lr = reinterpret_cast<const __nv_bfloat16*>(lus + static_cast<size_t>(r) * g.lstride);
     const float* dn = down + b * (g.rp + 1);
     float up = 0.0f;
-    for (int q = 0; q < g.rp; ++q) up = fmaf(dn[q], __bfloat162float(lr[q]), up);
+    for (int i = 0, q = q0; i < g.rp; ++i, q = q + 1 < g.rp ? q + 1 : 0)
+      up = fmaf(dn[q], __bfloat162float(lr[q]), up);
     const int n = n0 + r;
     float yv = alpha * static_cast<float>(isum) + up;
     if (g.bias != nullptr) yv += __bfloat162float(g.bias[n]);
@@ -517,7 +518,7 @@ bool launch_decode(const svdq_weight* w, const void* x, svdq_dtype xdt, int64_t 
   g.sstride = g.kslice * esz + 16;
   g.wstride = g.row_bytes + (packed ? 16 : 32);
   g.astride = static_cast<int>(M) + 32;
-  g.lstride = rp * 4 + 16;
+  g.lstride = rp * 4;
   g.mtiles = static_cast<int>(ceil_div(g.rows_per_cta, 16));
   g.ksub = std::max(1, kDecWarps / g.mtiles);
   const DecodeLayout L = decode_layout(g);

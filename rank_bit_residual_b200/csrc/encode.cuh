@@ -166,44 +166,62 @@ __device__ __forceinline__ uint64_t fsub2_rn(uint64_t a, uint64_t b) {
   return r;
 }
 
-// INT codes of 8 consecutive columns of a row, packed as 8 bytes: the exact
-// round_half_even(x / (scale_k s)), estimated as rint(fl(x c_k)) with the
-// per-column constant c_k = fl(fl(1 / scale_k) fl(1 / s)) and re-decided by
-// int_code_fix where the estimate is near a half-integer. scale8 points at the
-// 8 columns' smoothing scales (read only on that rare path). The estimate
-// never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in magnitude, so the fast
-// path needs no clamp. The fast path runs on pairs of elements (f32x2); the
-// rare path finds the flagged elements again with the same scalar operations.
-__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8],
-                                            const float* scale8, float s, int qmax) {
-  uint32_t f[8];
+// INT codes of 8 consecutive columns in each of kP rows, packed as 8 bytes per
+// row: the exact round_half_even(x / (scale_k s)), estimated as rint(fl(x c_k))
+// with the per-column constant c_k = fl(fl(1 / scale_k) fl(1 / s)) and
+// re-decided by int_code_fix where the estimate is near a half-integer.
+// scale8 points at the 8 columns' smoothing scales (read only on that rare
+// path). The estimate never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in
+// magnitude, so the fast path needs no clamp. The fast path runs on pairs of
+// elements (f32x2) for all rows before the one test for the rare path, so the
+// rows' chains interleave; the rare path finds the flagged elements again with
+// the same scalar operations.
+template <int kP>
+__device__ __forceinline__ void int_codes8_rows(const float (&v)[kP][8], const float (&ck)[8],
+                                                const float* scale8, float s, int qmax, uint2 (&out)[kP]) {
+  uint32_t f[kP][8];
   bool near = false;
   const uint64_t mg = pk2(kRintMagic, kRintMagic);
 #pragma unroll
-  for (int j = 0; j < 8; j += 2) {
-    const uint64_t t = fmul2_rn(pk2(v[j], v[j + 1]), pk2(ck[j], ck[j + 1]));
-    const uint64_t fs = fadd2_rn(t, mg);
-    const uint64_t d = fsub2_rn(t, fsub2_rn(fs, mg));
-    float d0, d1, s0, s1;
-    upk2(d, d0, d1);
-    upk2(fs, s0, s1);
-    f[j] = __float_as_uint(s0);
-    f[j + 1] = __float_as_uint(s1);
-    near = near || fabsf(d0) > kNearHalf || fabsf(d1) > kNearHalf;
-  }
+  for (int p = 0; p < kP; ++p)
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      const uint64_t t = fmul2_rn(pk2(v[p][j], v[p][j + 1]), pk2(ck[j], ck[j + 1]));
+      const uint64_t fs = fadd2_rn(t, mg);
+      const uint64_t d = fsub2_rn(t, fsub2_rn(fs, mg));
+      float d0, d1, s0, s1;
+      upk2(d, d0, d1);
+      upk2(fs, s0, s1);
+      f[p][j] = __float_as_uint(s0);
+      f[p][j + 1] = __float_as_uint(s1);
+      near = near || fabsf(d0) > kNearHalf || fabsf(d1) > kNearHalf;
+    }
   if (__builtin_expect(near, 0)) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float t = __fmul_rn(v[j], ck[j]);
-      if (fabsf(__fsub_rn(t, __fsub_rn(__fadd_rn(t, kRintMagic), kRintMagic))) > kNearHalf) {
-        const int q_est = static_cast<int>(f[j] & 0xFFu) - static_cast<int>((f[j] & 0x80u) << 1);
-        f[j] = static_cast<uint32_t>(int_code_fix(v[j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
+    for (int p = 0; p < kP; ++p)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float t = __fmul_rn(v[p][j], ck[j]);
+        if (fabsf(__fsub_rn(t, __fsub_rn(__fadd_rn(t, kRintMagic), kRintMagic))) > kNearHalf) {
+          const int q_est = static_cast<int>(f[p][j] & 0xFFu) - static_cast<int>((f[p][j] & 0x80u) << 1);
+          f[p][j] = static_cast<uint32_t>(int_code_fix(v[p][j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
+        }
       }
-    }
   }
-  const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(f[4], f[5], 0x0040), __byte_perm(f[6], f[7], 0x0040), 0x5410);
-  return make_uint2(lo, hi);
+#pragma unroll
+  for (int p = 0; p < kP; ++p) {
+    const uint32_t lo = __byte_perm(__byte_perm(f[p][0], f[p][1], 0x0040), __byte_perm(f[p][2], f[p][3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(f[p][4], f[p][5], 0x0040), __byte_perm(f[p][6], f[p][7], 0x0040), 0x5410);
+    out[p] = make_uint2(lo, hi);
+  }
+}
+
+// The same for one row.
+__device__ __forceinline__ uint2 int_codes8(const float (&v)[8], const float (&ck)[8],
+                                            const float* scale8, float s, int qmax) {
+  uint2 out[1];
+  int_codes8_rows<1>(reinterpret_cast<const float(&)[1][8]>(v), ck, scale8, s, qmax, out);
+  return out[0];
 }
 
 // Residual INT code of one fp32 element: round_half_even(R / s) clamped, with

@@ -38,7 +38,7 @@ template <int kKind>
 cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8_t* act_sf,
                         const float* s_x, const void* down2, int64_t B, const void* bias, void* y,
                         svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
-                        bool* bad_args) {
+                        bool* bad_args, void* split_ws) {
   *bad_args = false;
   if (B == 0) return cudaSuccess;
   const int64_t M = w->M, N = w->N;
@@ -63,7 +63,7 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
   const int out = raw_i32 ? kOutI32 : (ydt == SVDQ_F32 ? kOutF32 : kOutBF16);
   cudaError_t err = cudaSuccess;
   const bool launched =
-      B > 128 ? launch_gemm_pair(kKind, out, args, act_codes, has_lr ? down2 : nullptr, w, stream, &err)
+      B > 128 ? launch_gemm_pair(kKind, out, args, act_codes, has_lr ? down2 : nullptr, w, split_ws, stream, &err)
               : launch_gemm_skinny(kKind, out, args, act_codes, act_sf, has_lr ? down2 : nullptr, w, pdl, stream,
                                    &err);
   if (!launched) *bad_args = true;
@@ -75,15 +75,15 @@ cudaError_t launch_gemm(const svdq_weight* w, const void* act_codes, const uint8
 cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
                             const void* down2, int64_t B, const void* bias, void* y,
                             svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
-                            bool* bad_args) {
+                            bool* bad_args, void* split_ws) {
   return launch_gemm<kKindInt>(w, act_codes, nullptr, s_x, down2, B, bias, y, ydt, ldy, raw_i32, pdl,
-                               stream, bad_args);
+                               stream, bad_args, split_ws);
 }
 
 cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,
                             const uint8_t* act_sf, const float* gs_x, const void* down2,
                             int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args) {
+                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args, void* split_ws) {
   if (!act_sf || !w->sf || (reinterpret_cast<uintptr_t>(act_sf) & 15) ||
       (reinterpret_cast<uintptr_t>(w->sf) & 15)) {
     *bad_args = true;
@@ -91,9 +91,9 @@ cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,
   }
   if (w->fmt.kind == SVDQ_KIND_MXFP4)
     return launch_gemm<kKindMxfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false, pdl,
-                                   stream, bad_args);
+                                   stream, bad_args, split_ws);
   return launch_gemm<kKindNvfp4>(w, act_codes, act_sf, gs_x, down2, B, bias, y, ydt, ldy, false, pdl,
-                                 stream, bad_args);
+                                 stream, bad_args, split_ws);
 }
 
 }  // namespace svdq

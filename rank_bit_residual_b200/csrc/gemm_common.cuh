@@ -26,6 +26,11 @@ struct GemmArgs {
   const uint8_t* sfa;             // fp4 activation scales (128x4 layout)
   const uint8_t* sfb;             // fp4 weight scales (128x4 layout)
   int katoms;                     // fp4: 4-scale atoms per row tile, ceil(M / 64) NVFP4, ceil(M / 128) MXFP4
+  // pair kernel: K split of the last round's tiles (nsplit 1: none); the
+  // workspace for the split (partials, then one counter per split tile)
+  int nsplit;
+  uint32_t* split_part;
+  unsigned* split_cnt;
   unsigned* status;
 };
 
@@ -195,8 +200,9 @@ bool launch_gemm_skinny(int kind, int out, const GemmArgs& g, const void* act_co
                         cudaError_t* err);
 
 // Host: the CTA-pair kernel (gemm_pair.cu); false if a tensor map cannot be encoded.
+// split_ws (may be null: no split) holds pair_split_bytes(B, N) bytes.
 bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
-                      const void* down2, const svdq_weight* w, cudaStream_t stream,
+                      const void* down2, const svdq_weight* w, void* split_ws, cudaStream_t stream,
                       cudaError_t* err);
 
 }  // namespace svdq

@@ -81,6 +81,20 @@ struct TwoPass {
   static constexpr bool value = kOut == kOutBF16 || (kKind == kKindInt && kOut == kOutF32);
 };
 
+__device__ __forceinline__ unsigned ld_acquire_gpu_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One round's work of a pair: tile t, residual K steps [j0, j1); role 0 = the
+// whole tile, 1 = owner of a split tile (slice 0: adds the other slices'
+// partials), 2 = a later slice (writes its partial); q = index of the split tile,
+// sl = slice. Only roles 0 and 1 run the low-rank steps and write Y.
+struct PairItem {
+  int t, j0, j1, role, q, sl;
+};
+
 template <int kKind, int kOut>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -122,7 +136,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   constexpr int kKb = PairCfg<kKind>::kKb;
   constexpr int kStageK = kF4 ? 256 : 128 * kKb;   // K elements per stage
   const int ksteps = (M + kStageK - 1) / kStageK;
-  const int steps_per_tile = ksteps + lr_steps;   // residual steps first
+  // Work items of this pair, one per round: the tiles pair, pair + npairs, ...
+  // With a split (nsplit > 1) the tiles of the last, partial round are cut
+  // along K into nsplit slices run by different pairs: slice 0 (the owner)
+  // also runs the low-rank steps and, in its epilogue, adds the other slices'
+  // raw partial accumulators (written to the workspace) in slice order.
+  const int rounds_full = total / npairs, trem = total - rounds_full * npairs;
+  const int nrounds = rounds_full + (trem > 0 ? 1 : 0);
+  const int nsplit = args.nsplit;
+  auto item = [&](int r, PairItem& it) -> bool {
+    it.j0 = 0;
+    it.j1 = ksteps;
+    it.role = 0;
+    it.q = 0;
+    it.sl = 0;
+    if (r < rounds_full) {
+      it.t = pair + r * npairs;
+      return true;
+    }
+    if (r >= nrounds) return false;
+    if (nsplit <= 1) {
+      it.t = rounds_full * npairs + pair;
+      return pair < trem;
+    }
+    if (pair >= trem * nsplit) return false;
+    it.q = pair % trem;
+    it.sl = pair / trem;
+    it.t = rounds_full * npairs + it.q;
+    it.j0 = (ksteps * it.sl) / nsplit;
+    it.j1 = (ksteps * (it.sl + 1)) / nsplit;
+    it.role = it.sl == 0 ? 1 : 2;
+    return true;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -156,19 +201,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
+      PairItem wi;
+      for (int r = 0; ok && item(r, wi); ++r) {
+        const int t = wi.t;
         const int m0 = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf;
         const int nt = (t / tiles_m) * kTileN;
         const int n0 = nt + static_cast<int>(rank) * kHalf;
-        for (int j = 0; j < steps_per_tile && ok; ++j, ++it) {
+        const int nres = wi.j1 - wi.j0;
+        const int nsteps_it = nres + (wi.role != 2 ? lr_steps : 0);
+        for (int jj = 0; jj < nsteps_it && ok; ++jj, ++it) {
+          const int j = wi.j0 + jj;   // residual K step
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           ok = mbar_wait(&empty_bar[s], ph ^ 1, status, &abort_sh);
           if (!ok) break;
           uint8_t* st = smem + s * kStageBytes;
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
-          if (j >= ksteps) {
-            const int l = j - ksteps;
+          if (jj >= nres) {
+            const int l = jj - nres;
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * (kABytes + kBBytes));
             tma_load_2d_pair(st, &tm_da, fb, 64 * l, m0);
             tma_load_2d_pair(st + kABytes, &tm_lu, fb, 64 * l, n0);
@@ -225,12 +275,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
       uint32_t it = 0, lt = 0;
       bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs, ++lt) {
+      PairItem wi;
+      for (int r = 0; ok && item(r, wi); ++r, ++lt) {
         ok = mbar_wait(&acc_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
         if (!ok) break;
         tc_fence_after();
-        for (int j = 0; j < steps_per_tile; ++j, ++it) {
-          if (kKind == kKindInt && j == ksteps) {
+        const int nres = wi.j1 - wi.j0;
+        const bool lr_here = wi.role != 2 && lr_steps > 0;
+        const int nsteps_it = nres + (lr_here ? lr_steps : 0);
+        for (int jj = 0; jj < nsteps_it; ++jj, ++it) {
+          const int j = wi.j0 + jj;   // residual K step
+          if (kKind == kKindInt && jj == nres) {
             // the low-rank columns: the previous tile's stores are done
             ok = mbar_wait(&lr_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
             if (!ok) break;
@@ -243,8 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + s * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
-          if (j >= ksteps) {
-            const int l = j - ksteps;
+          if (jj >= nres) {
+            const int l = jj - nres;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_f16_pair(lr_acc, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_bf,
@@ -262,13 +317,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if constexpr (kKind == kKindNvfp4) {
               for (int kk = 0; kk < na; ++kk)
                 mma_nvf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), id_f4,
-                              (j > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
+                              (jj > 0 || kk > 0) ? 1u : 0u, tmem + kSfaCol + 4 * kk, tmem + kSfbCol + 8 * kk);
             } else {
               // MMA kk: atom kk / 2, scale bytes 2 (kk % 2) and up of each row's four
               const int nm = min(4, kmma - 4 * j);
               for (int kk = 0; kk < nm; ++kk)
                 mma_mxf4_pair(tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), ((kk & 1) ? id_mx1 : id_mx0),
-                              (j > 0 || kk > 0) ? 1u : 0u, sf_taddr(tmem + kSfaCol + 4 * (kk >> 1), kk),
+                              (jj > 0 || kk > 0) ? 1u : 0u, sf_taddr(tmem + kSfaCol + 4 * (kk >> 1), kk),
                               sf_taddr(tmem + kSfbCol + 8 * (kk >> 1), kk));
             }
           } else {
@@ -277,12 +332,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int kk = 0; kk < 4 * kKb; ++kk)
               mma_i8_pair(tmem, smem_desc_sw128(a0 + (kk >> 2) * kABytes + 32 * (kk & 3)),
                           smem_desc_sw128(bb + (kk >> 2) * kBBytes + 32 * (kk & 3)), id_i8,
-                          (j > 0 || kk > 0) ? 1u : 0u);
+                          (jj > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty_bar[s], 0x3);
         }
         if (!ok) break;
-        if (kKind == kKindInt && lr_steps == 0) {
+        if (kKind == kKindInt && !lr_here) {
           // keep the low-rank barrier's phases in step with the tiles
           ok = mbar_wait(&lr_empty_bar, (lt & 1) ^ 1, status, &abort_sh);
           if (!ok) break;
@@ -316,7 +371,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     };
     uint32_t lt = 0;
-    for (int t = pair; t < total; t += npairs, ++lt) {
+    PairItem wi;
+    for (int r = 0; item(r, wi); ++r, ++lt) {
+      const int t = wi.t;
       if (!mbar_wait_warp(&tmem_full_bar, lt & 1, status, &abort_sh)) break;
       tc_fence_after();
       const int row = (t % tiles_m) * 2 * kHalf + static_cast<int>(rank) * kHalf + r_in;
@@ -338,6 +395,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tmem_ld_wait_regs(accs[i]);
         release(acc_empty_even, &acc_empty_bar);
+        if (wi.role != 0) {
+          // split tile: the partial of slice sl, laid out [tile q][slice - 1]
+          // [CTA rank][column half h][16-byte piece][row], so that each warp
+          // access covers 32 consecutive rows' pieces (512 contiguous bytes)
+          const size_t per_slice = static_cast<size_t>(2) * kHalf * kTileN / 4;   // in 16-byte pieces
+          auto part_row = [&](int sl) {
+            return reinterpret_cast<uint4*>(args.split_part) +
+                   (static_cast<size_t>(wi.q) * (nsplit - 1) + (sl - 1)) * per_slice +
+                   (static_cast<size_t>(rank) * 2 + h) * 32 * kHalf + r_in;
+          };
+          if (wi.role == 2) {
+            // a later slice: the raw accumulator to the workspace, then count
+            // this warp's part in; nothing of Y
+            uint4* dst4 = part_row(wi.sl);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                __stcg(dst4 + (8 * i + e) * kHalf, make_uint4(accs[i][4 * e], accs[i][4 * e + 1], accs[i][4 * e + 2],
+                                                    accs[i][4 * e + 3]));
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(args.split_cnt + wi.q, 1u);
+            if (kKind == kKindInt) release(lr_empty_even, &lr_empty_bar);
+            continue;
+          }
+          // the owner: wait (bounded) until every warp of the other slices'
+          // CTAs has written its part, then add the partials in slice order
+          const unsigned target = static_cast<unsigned>(2 * kEpiWarps * (nsplit - 1));
+          int got = 1;
+          if (lane == 0) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (ld_acquire_gpu_u32(args.split_cnt + wi.q) < target) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_status(status, kStatusTimeout);
+                got = 0;
+                break;
+              }
+            }
+          }
+          got = __shfl_sync(0xffffffffu, got, 0);
+          __syncwarp();
+          if (got) {
+            for (int sl = 1; sl < nsplit; ++sl) {
+              const uint4* src4 = part_row(sl);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const uint4 v = __ldcg(src4 + (8 * i + e) * kHalf);
+                  const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    uint32_t& a = accs[i][4 * e + u];
+                    if constexpr (kKind == kKindInt)
+                      a = static_cast<uint32_t>(static_cast<int32_t>(a) + static_cast<int32_t>(pv[u]));
+                    else
+                      a = __float_as_uint(__uint_as_float(a) + __uint_as_float(pv[u]));
+                  }
+                }
+            }
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int c = 4 * h + i;
@@ -374,6 +494,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   }
 }
 
+// The K split of the last round: with P CTA pairs and T tiles, R = T / P full
+// rounds leave T mod P tiles for a last round in which most pairs would idle;
+// each of those tiles is cut into s slices (s (T mod P) <= P), so s (T mod P)
+// pairs share the last round. (A grid of fewer tiles than pairs is one such
+// round.) The split saves (1 - 1/s) of a tile's K steps and costs the owner an
+// exposed epilogue (about 7 K steps' time) and the reading of s - 1 partial
+// tiles (about 2.4 K steps' time each, measured at K = 12288): s maximises the
+// saving net of that cost, and no split is taken when it is not positive.
+int pick_nsplit(int64_t ksteps, int64_t smax) {
+  int best = 1;
+  double best_net = 0.0;
+  for (int64_t s = 2; s <= std::min<int64_t>(smax, 8); ++s) {
+    const double net = (1.0 - 1.0 / static_cast<double>(s)) * static_cast<double>(ksteps) - 7.0 -
+                       2.4 * static_cast<double>(s - 1);
+    if (net > best_net) {
+      best_net = net;
+      best = static_cast<int>(s);
+    }
+  }
+  return best;
+}
+
+struct PairSplit {
+  int pairs, trem, nsplit;
+};
+PairSplit pair_split(int64_t B, int64_t M, int64_t N) {
+  const int64_t tiles = ceil_div(B, 2 * kHalf) * ceil_div(N, kTileN);
+  const int64_t P = std::max(1, num_sms() / 2);
+  const int64_t ksteps = ceil_div(M, 256);
+  PairSplit ps{static_cast<int>(std::min(tiles, P)), 0, 1};
+  const int64_t trem = tiles >= P ? tiles % P : tiles;
+  if (trem == 0) return ps;
+  const int64_t s = pick_nsplit(ksteps, std::min<int64_t>(P / trem, ksteps));
+  if (s < 2) return ps;
+  ps.trem = static_cast<int>(trem);
+  ps.nsplit = static_cast<int>(s);
+  if (tiles < P) ps.pairs = static_cast<int>(trem * s);
+  return ps;
+}
+
 template <int kKind, int kOut>
 cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int grid, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(PairCfg<kKind>::kStages) * PairCfg<kKind>::kStageBytes + 1024;
@@ -390,10 +550,27 @@ cudaError_t launch_pair_one(const CUtensorMap* maps, const GemmArgs& args, int g
 
 // Builds the pair kernel's tensor maps and launches it; returns false (and
 // launches nothing) if a map cannot be encoded.
-bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_codes,
-                      const void* down2, const svdq_weight* w, cudaStream_t stream,
+size_t pair_split_counter_offset(int64_t B, int64_t M, int64_t N) {
+  const PairSplit ps = pair_split(B, M, N);
+  return ps.nsplit < 2 ? 0 : static_cast<size_t>(ps.trem) * (ps.nsplit - 1) * 2 * kHalf * kTileN * 4;
+}
+
+int pair_split_counters(int64_t B, int64_t M, int64_t N) {
+  const PairSplit ps = pair_split(B, M, N);
+  return ps.nsplit < 2 ? 0 : ps.trem;
+}
+
+size_t pair_split_bytes(int64_t B, int64_t M, int64_t N) {
+  const PairSplit ps = pair_split(B, M, N);
+  if (ps.nsplit < 2) return 0;
+  return pair_split_counter_offset(B, M, N) + static_cast<size_t>(round_up(static_cast<int64_t>(ps.trem) * 4, 256));
+}
+
+bool launch_gemm_pair(int kind, int out, const GemmArgs& args_in, const void* act_codes,
+                      const void* down2, const svdq_weight* w, void* split_ws, cudaStream_t stream,
                       cudaError_t* err) {
   *err = cudaSuccess;
+  GemmArgs args = args_in;
   const int64_t M = args.M, N = args.N, B = args.B;
   const int rp = w->rank_pad;
   const int64_t row_bytes = kind != kKindInt ? M / 2 : M;
@@ -420,8 +597,24 @@ bool launch_gemm_pair(int kind, int out, const GemmArgs& args, const void* act_c
     maps[5] = maps[1];
   }
   if (!ok) return false;
-  const int64_t tiles = ceil_div(B, 2 * kHalf) * ceil_div(N, kTileN);
-  const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, num_sms() / 2));
+  // the split needs the workspace and the two-pass epilogue; it is taken for INT
+  // only, whose int32 sums are exact in any order (a split fp4 tile would round
+  // its fp32 sums differently from the same tile unsplit, so the fp32 and bf16
+  // outputs of one call, or the workspace and the staged entry points, could
+  // differ in the last bit)
+  PairSplit ps = pair_split(B, M, N);
+  const bool splittable = kind == kKindInt && (out == kOutBF16 || out == kOutF32);
+  if (split_ws == nullptr || !splittable || (reinterpret_cast<uintptr_t>(split_ws) & 15) != 0) {
+    const int64_t tiles = ceil_div(B, 2 * kHalf) * ceil_div(N, kTileN);
+    ps = PairSplit{static_cast<int>(std::min<int64_t>(tiles, std::max(1, num_sms() / 2))), 0, 1};
+  }
+  args.nsplit = ps.nsplit;
+  if (ps.nsplit > 1) {
+    args.split_part = static_cast<uint32_t*>(split_ws);
+    // the counters must be zero at the launch (the activation pass clears them)
+    args.split_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(split_ws) + pair_split_counter_offset(B, M, N));
+  }
+  const int grid = 2 * ps.pairs;
   if (kind == kKindInt) {
     if (out == kOutI32) *err = launch_pair_one<kKindInt, kOutI32>(maps, args, grid, stream);
     else if (out == kOutF32) *err = launch_pair_one<kKindInt, kOutF32>(maps, args, grid, stream);

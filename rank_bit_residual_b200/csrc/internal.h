@@ -98,7 +98,7 @@ cudaError_t launch_act(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t 
                        const float* scale, svdq_fmt fmt, const float* act_global_scale,
                        const float* w_global_scale, const void* ld, void* codes, void* sf,
                        float* act_scale, void* down, void* scratch, cudaStream_t stream,
-                       bool* bad_args);
+                       bool* bad_args, unsigned* zero_words = nullptr, int nzero = 0);
 cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, int64_t ldx,
                              const float* scale, svdq_fmt fmt, const float* act_global_scale,
                              const float* w_global_scale, const void* ld, void* codes, void* sf,
@@ -106,12 +106,19 @@ cudaError_t launch_act_small(const ActPlan& p, const void* x, svdq_dtype xdt, in
                              bool* bad_args);
 
 // ------------------------------------------------------------ residual GEMM
+// split_ws (may be null) holds pair_split_bytes(B, M, N) bytes: the pair kernel
+// then splits the tiles of its last, partial round along K.
 cudaError_t launch_gemm_int(const svdq_weight* w, const int8_t* act_codes, const float* s_x,
                             const void* down2, int64_t B, const void* bias, void* y,
                             svdq_dtype ydt, int64_t ldy, bool raw_i32, bool pdl, cudaStream_t stream,
-                            bool* bad_args);
+                            bool* bad_args, void* split_ws = nullptr);
+size_t pair_split_bytes(int64_t B, int64_t M, int64_t N);
+// The split's tile counters: pair_split_counters(...) words at that byte offset
+// of the split workspace, which must be zero when the GEMM starts.
+size_t pair_split_counter_offset(int64_t B, int64_t M, int64_t N);
+int pair_split_counters(int64_t B, int64_t M, int64_t N);
 
-// The whole linear for B <= 2 rows with INT weights in one launch (decode.cu);
+// The whole linear for B <= 16 rows with INT weights in one launch (decode.cu);
 // false (nothing launched) when the shape or the alignment does not allow it.
 bool launch_decode(const svdq_weight* w, const void* x, svdq_dtype xdt, int64_t B, int64_t ldx, const void* bias,
                    void* y, svdq_dtype ydt, int64_t ldy, bool chained, cudaStream_t st, cudaError_t* err);
@@ -120,7 +127,8 @@ bool launch_decode(const svdq_weight* w, const void* x, svdq_dtype xdt, int64_t 
 cudaError_t launch_gemm_fp4(const svdq_weight* w, const uint8_t* act_codes,
                             const uint8_t* act_sf, const float* gs_x, const void* down2,
                             int64_t B, const void* bias, void* y, svdq_dtype ydt,
-                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args);
+                            int64_t ldy, bool pdl, cudaStream_t stream, bool* bad_args,
+                            void* split_ws = nullptr);
 
 // -------------------------------------------------------------- quantisers
 size_t residual_scratch_bytes(int64_t M, int64_t N);

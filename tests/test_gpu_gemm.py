@@ -197,3 +197,26 @@ def test_single_launch_decode_matches_oracle(B, M, N, rank, fmt, packed, bias, x
     codes, sf, s, down = rb.svdq_quantize_act(x, scale, fmt, ld=ld if rank else None)
     y_st = rb.svdq_residual_linear(w.w, codes, sf, s, down, bias=b, out_dtype=torch.float32)
     assert_y_close(y32.cpu().numpy(), y_st.cpu().numpy().astype(np.float64), "fused vs staged")
+
+
+@pytest.mark.parametrize("B,N", [(300, 768), (520, 1280)])
+def test_pair_split_tiles_equal_unsplit(B, N):
+    """With a long K and fewer tiles than CTA pairs, svdq_linear cuts the tiles
+    along K over several pairs (slice partials added by the owner, int32) while
+    svdq_residual_linear (no workspace) does not split: the outputs are equal bit
+    for bit, and match the oracle."""
+    M, rank = 12288, 32
+    wl = make_case(B, M, N, rank=rank, seed=B + N, bias=True)
+    w = SyntheticWeight(M, N, rank, "int4", seed=5, scale=wl.scale, packed=True)
+    x = x_tensor(wl)
+    scale = to_dev(wl.scale, torch.float32)
+    b = to_dev(wl.bias, torch.bfloat16)
+    codes, sf, s, down = rb.svdq_quantize_act(x, scale, "int4", ld=w.w.ld)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        y_sep = rb.svdq_residual_linear(w.w, codes, sf, s, down, bias=b, out_dtype=out_dtype)
+        for _ in range(3):
+            y = rb.svdq_linear(w.w, x, bias=b, out_dtype=out_dtype)
+            assert torch.equal(y, y_sep), out_dtype
+    assert rb.svdq_check_status() == rb.SVDQ_OK
+    y32 = rb.svdq_linear(w.w, x, bias=b, out_dtype=torch.float32)
+    assert_y_close(y32.cpu().numpy(), w.oracle_y(wl.x, wl.bias), f"split {B}x{M}x{N}")
