@@ -300,7 +300,12 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
   auto swz = [](int r, int c, int rows) -> int {
     return (c >> 3) * rows * kTileBytes + r * kTileBytes + (((c & 7) ^ (r & 7)) << 4);
   };
-  uint32_t g = 0;   // segments begun so far: stage g % stages, barrier phase (g / stages) & 1
+  // the ring positions, advanced one segment at a time (no divisions): the
+  // producer's (thread 0: next stage to fill and its use parity) and every
+  // thread's (next stage to consume and its parity); a stage's first use is
+  // the only one that does not wait for it to be released
+  uint32_t p_seg = 0, p_stage = 0, p_par = 0;
+  uint32_t c_stage = 0, c_par = 0;
   uint32_t unit_parity = 0;
   // Pieces of work: a row block and a range of its segments. Flat partition:
   // CTA i takes segments [W i / G, W (i + 1) / G) of all W = nrb * nsteps
@@ -347,11 +352,14 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
     // segment; only thread 0 waits for that, and only when it refills.
     auto issue = [&](int c) {
       if (tid == 0 && c < nsub) {
-        const uint32_t gc = g + c;
-        const uint32_t s_ = gc % stages;
-        if (gc >= static_cast<uint32_t>(stages) &&
-            !mbar_wait(&empty_bar[s_], ((gc / stages) - 1) & 1, a.status, &abort_sh))
+        const uint32_t s_ = p_stage;
+        if (p_seg >= static_cast<uint32_t>(stages) && !mbar_wait(&empty_bar[s_], p_par ^ 1u, a.status, &abort_sh))
           return;   // a wait ran out: load nothing more
+        ++p_seg;
+        if (++p_stage == static_cast<uint32_t>(stages)) {
+          p_stage = 0;
+          p_par ^= 1u;
+        }
         uint8_t* st = smem + s_ * stage_bytes;
         uint64_t* bar = &full_bar[s_];
         const int col = c_lo + c * kSubCols;
@@ -373,13 +381,16 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
     }
     __syncthreads();   // the column constants are written
     for (int c = 0; c < nsub; ++c) {
-      const uint32_t gc = g + c;
-      const uint32_t s_ = gc % stages;
+      const uint32_t s_ = c_stage, par = c_par;
+      if (++c_stage == static_cast<uint32_t>(stages)) {
+        c_stage = 0;
+        c_par ^= 1u;
+      }
       const uint8_t* st = smem + s_ * stage_bytes;
       // thread 0 keeps stages - 1 segments in flight
       issue(c + stages - 1);
       // segment c has landed (every warp waits for itself)
-      if (!mbar_wait_warp(&full_bar[s_], (gc / stages) & 1, a.status, &abort_sh)) break;
+      if (!mbar_wait_warp(&full_bar[s_], par, a.status, &abort_sh)) break;
       if (rp > 0 && lane == 0 && warp < nacc) {
         tc_fence_after();
         const uint32_t xa = smem_u32(st), la = xa + ld_off;
@@ -512,7 +523,6 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
         }
       }
     }
-    g += nsub;
     unit_parity ^= 1u;
     __syncthreads();   // the drain is done and the column constants are free before the next unit
     if (abort_sh) break;

@@ -180,7 +180,7 @@ template <int kP>
 __device__ __forceinline__ void int_codes8_rows(const float (&v)[kP][8], const float (&ck)[8],
                                                 const float* scale8, float s, int qmax, uint2 (&out)[kP]) {
   uint32_t f[kP][8];
-  bool near = false;
+  uint32_t near = 0u;   // bitwise (no short-circuit branches)
   const uint64_t mg = pk2(kRintMagic, kRintMagic);
 #pragma unroll
   for (int p = 0; p < kP; ++p)
@@ -194,9 +194,9 @@ __device__ __forceinline__ void int_codes8_rows(const float (&v)[kP][8], const f
       upk2(fs, s0, s1);
       f[p][j] = __float_as_uint(s0);
       f[p][j + 1] = __float_as_uint(s1);
-      near = near || fabsf(d0) > kNearHalf || fabsf(d1) > kNearHalf;
+      near |= static_cast<uint32_t>(fabsf(d0) > kNearHalf) | static_cast<uint32_t>(fabsf(d1) > kNearHalf);
     }
-  if (__builtin_expect(near, 0)) {
+  if (__builtin_expect(near != 0u, 0)) {
 #pragma unroll
     for (int p = 0; p < kP; ++p)
 #pragma unroll
