@@ -139,6 +139,9 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
   __shared__ float red[kMaxThreads / 32];
   // chained after another linear: x is that linear's output
   if (a.chained) pdl_wait();
+  // the quantise kernel may launch now and do its setup (it reads nothing of
+  // this kernel's before its griddepcontrol.wait)
+  pdl_trigger();
   const int tid = threadIdx.x;
   // block 0 clears the quantise kernel's row-block counters (and any words the
   // GEMM after this pass needs zeroed)
@@ -258,6 +261,14 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
     tma_prefetch_desc(&tm_x);
     if (rp > 0) tma_prefetch_desc(&tm_ld);
   }
+  if (rp > 0 && warp == 0) {
+    tmem_alloc(&tmem_sh, acc_cols * nacc);
+    tmem_relinquish();
+  }
+  // launched as a programmatic dependent of the maximum kernel: the setup above
+  // overlaps its tail; everything below (its partial maxima and counters, x,
+  // every output) comes after it has finished
+  pdl_wait();
   // the per-tensor scale from the partial maxima (INT; NVFP4 without a given gs)
   float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
   {
@@ -276,10 +287,6 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
       u = s > 0.0f ? __frcp_rn(s) : 0.0f;
     }
     if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv || mx ? gs_x : s;
-  }
-  if (rp > 0 && warp == 0) {
-    tmem_alloc(&tmem_sh, acc_cols * nacc);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -583,8 +590,17 @@ cudaError_t launch_quant(const ActArgs& a, int grid, size_t smem, cudaStream_t s
   cudaError_t err = cudaFuncSetAttribute(act_quant_kernel<TIn, kFp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  act_quant_kernel<TIn, kFp4><<<grid, kWork, smem, stream>>>(tx, tl, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kWork);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<TIn, kFp4>, tx, tl, a);
 }
 
 // Largest column count a unit may have: its per-column constants share the
