@@ -140,6 +140,16 @@ constexpr float kRintMagic = 12582912.0f;
 // half-integer: with |t| <= 128 (qmax <= 127) its error is below 2^-15.
 constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
 
+// The same limit for the activation codes' estimate x c_k. Its error is below
+// 3 (qmax + 1) 2^-24: c_k carries three roundings relative to 1 / (scale_k s),
+// and |x / (scale_k s)| <= qmax (1 + 2^-23). A distance of at most
+// 1/2 - 8 (qmax + 1) 2^-24 (that error plus the 2^-26 rounding of the distance
+// itself, with room to spare) puts the exact quotient within 1/2 of the same
+// integer. For INT4 the band is 2^-18 wide on each side of a half-integer.
+__device__ __forceinline__ float act_near_limit(int qmax) {
+  return __fmaf_rn(-static_cast<float>(qmax + 1), 1.0f / 2097152.0f, 0.5f);
+}
+
 // Packed pairs of fp32 (sm_100a f32x2 arithmetic): each lane of the pair is
 // rounded to nearest even on its own, exactly as the scalar operation.
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -165,44 +175,54 @@ __device__ __forceinline__ uint64_t fsub2_rn(uint64_t a, uint64_t b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t ffma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 
 // INT codes of 8 consecutive columns in each of kP rows, packed as 8 bytes per
-// row: the exact round_half_even(x / (scale_k s)), estimated as rint(fl(x c_k))
+// row: the exact round_half_even(x / (scale_k s)), estimated as rint(x c_k)
 // with the per-column constant c_k = fl(fl(1 / scale_k) fl(1 / s)) and
 // re-decided by int_code_fix where the estimate is near a half-integer.
-// scale8 points at the 8 columns' smoothing scales (read only on that rare
-// path). The estimate never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in
-// magnitude, so the fast path needs no clamp. The fast path runs on pairs of
-// elements (f32x2) for all rows before the one test for the rare path, so the
-// rows' chains interleave; the rare path finds the flagged elements again with
-// the same scalar operations.
+// The estimate takes one fused rounding, fma(x, c_k, 1.5 * 2^23) (the magic
+// constant's unit spacing makes that rounding the rint of the exact product),
+// and the distance to it is a second fma, x c_k - rint; the largest distance of
+// the group decides whether any element needs the rare path. scale8 points at
+// the 8 columns' smoothing scales (read only on that rare path). The estimate
+// never exceeds qmax (1 + 6 * 2^-24) < qmax + 1/2 in magnitude, so the fast
+// path needs no clamp. The fast path runs on pairs of elements (f32x2) for all
+// rows before the one test, so the rows' chains interleave; the rare path
+// finds the flagged elements again with the same scalar operations.
 template <int kP>
 __device__ __forceinline__ void int_codes8_rows(const float (&v)[kP][8], const float (&ck)[8],
                                                 const float* scale8, float s, int qmax, uint2 (&out)[kP]) {
   uint32_t f[kP][8];
-  uint32_t near = 0u;   // bitwise (no short-circuit branches)
+  float dmax = 0.0f;
   const uint64_t mg = pk2(kRintMagic, kRintMagic);
 #pragma unroll
   for (int p = 0; p < kP; ++p)
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
-      const uint64_t t = fmul2_rn(pk2(v[p][j], v[p][j + 1]), pk2(ck[j], ck[j + 1]));
-      const uint64_t fs = fadd2_rn(t, mg);
-      const uint64_t d = fsub2_rn(t, fsub2_rn(fs, mg));
+      const uint64_t x2 = pk2(v[p][j], v[p][j + 1]);
+      const uint64_t c2 = pk2(ck[j], ck[j + 1]);
+      const uint64_t fs = ffma2_rn(x2, c2, mg);           // 1.5 * 2^23 + rint(x c_k)
+      const uint64_t d = ffma2_rn(x2, c2, fsub2_rn(mg, fs));   // x c_k - rint(x c_k)
       float d0, d1, s0, s1;
       upk2(d, d0, d1);
       upk2(fs, s0, s1);
       f[p][j] = __float_as_uint(s0);
       f[p][j + 1] = __float_as_uint(s1);
-      near |= static_cast<uint32_t>(fabsf(d0) > kNearHalf) | static_cast<uint32_t>(fabsf(d1) > kNearHalf);
+      dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
     }
-  if (__builtin_expect(near != 0u, 0)) {
+  const float lim = act_near_limit(qmax);
+  if (__builtin_expect(dmax > lim, 0)) {
 #pragma unroll
     for (int p = 0; p < kP; ++p)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float t = __fmul_rn(v[p][j], ck[j]);
-        if (fabsf(__fsub_rn(t, __fsub_rn(__fadd_rn(t, kRintMagic), kRintMagic))) > kNearHalf) {
+        const float fs = __fmaf_rn(v[p][j], ck[j], kRintMagic);
+        if (fabsf(__fmaf_rn(v[p][j], ck[j], __fsub_rn(kRintMagic, fs))) > lim) {
           const int q_est = static_cast<int>(f[p][j] & 0xFFu) - static_cast<int>((f[p][j] & 0x80u) << 1);
           f[p][j] = static_cast<uint32_t>(int_code_fix(v[p][j], __ldg(scale8 + j), s, q_est, qmax)) & 0xFFu;
         }
