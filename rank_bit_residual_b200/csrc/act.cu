@@ -58,7 +58,7 @@ constexpr int kSub = 256;                   // bytes of a row per segment (two t
 constexpr int kMaxStages = 6;
 constexpr int kMaxThreads = 256;            // threads of the maximum kernel
 constexpr int kMaxSlab = 2048;              // bytes of a row per maximum-kernel CTA (16 per thread)
-constexpr int kMaxCtasPerSm = 4;
+constexpr int kMaxCtasPerSm = 6;
 constexpr int kFlatMinSegs = 8;             // segments per SM from which the flat partition pays
 
 // Bytes of one quantise-kernel stage: x and ld as two 128-byte K blocks each; a
@@ -127,6 +127,17 @@ __device__ __forceinline__ void abs_max16(uint32_t (&m)[4], const uint4 v) {
   m[3] = abs_max_word<TIn>(m[3], v.w);
 }
 
+// A 16-byte read-only load that allocates no L1 line: the maximum kernel's
+// stream of x is never re-read by the same SM, and without allocation the
+// number of loads in flight is not bounded by the L1's capacity.
+__device__ __forceinline__ uint4 ld_stream_v4(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // ------------------------------------------------------------ maximum kernel
 // CTA = a slab of kMaxSlab bytes of every row in a range of rows; thread t
 // reads the 16-byte piece t % 128 of rows r0 + t / 128, r0 + t / 128 + 2, ...
@@ -163,13 +174,13 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
     for (; r + 14 < r1; r += 16) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(p + u * step);
+      for (int u = 0; u < 8; ++u) v[u] = ld_stream_v4(p + u * step);
 #pragma unroll
       for (int u = 0; u < 8; ++u) abs_max16<TIn>(m, v[u]);
       p += 8 * step;
     }
     for (; r < r1; r += 2) {
-      abs_max16<TIn>(m, __ldg(p));
+      abs_max16<TIn>(m, ld_stream_v4(p));
       p += step;
     }
   }
