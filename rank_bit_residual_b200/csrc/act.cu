@@ -170,18 +170,15 @@ __global__ void __launch_bounds__(kMaxThreads) act_max_kernel(const ActArgs a) {
     const int64_t step = 2 * a.ldx * kEsz / 16;   // two rows, in 16-byte units (ldx * esz % 16 == 0)
     const uint4* p = reinterpret_cast<const uint4*>(static_cast<const TIn*>(a.x) +
                                                     static_cast<int64_t>(r0 + rsl) * a.ldx + col);
-    int r = r0 + rsl;
-    for (; r + 14 < r1; r += 16) {
+    // eight loads issued before any is used, the last batch's past r1 skipped
+    // (a zero word leaves the maximum unchanged)
+    for (int r = r0 + rsl; r < r1; r += 16) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = ld_stream_v4(p + u * step);
+      for (int u = 0; u < 8; ++u) v[u] = r + 2 * u < r1 ? ld_stream_v4(p + u * step) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int u = 0; u < 8; ++u) abs_max16<TIn>(m, v[u]);
       p += 8 * step;
-    }
-    for (; r < r1; r += 2) {
-      abs_max16<TIn>(m, ld_stream_v4(p));
-      p += step;
     }
   }
   if (rsl == 1) {
