@@ -194,6 +194,9 @@ svdq_status svdq_quantize_residual_workspace_size(int64_t M, int64_t N, svdq_fmt
  *   act_scale out device fp32 scalar: s_x (INT), the gs_x used (NVFP4) or 1 (MXFP4)
  *   down     out bf16 [B, 2*rank_pad]: x ld^T split as hi | lo with
  *            hi = bf16(v), lo = bf16(v - hi) of the fp32 dot product v
+ * Host errors: SVDQ_EINVAL for null pointers and sizes, SVDQ_EUNSUPPORTED for
+ * M not a multiple of 32 or a pointer (x, scale, codes, down when written) not
+ * 16-byte aligned, SVDQ_EWORKSPACE for a short workspace.
  */
 svdq_status svdq_quantize_act(const void* x, svdq_dtype x_dtype, int64_t B, int64_t M,
                               int64_t ldx, const float* scale, svdq_fmt fmt,

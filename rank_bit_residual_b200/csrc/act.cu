@@ -490,19 +490,21 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s_]);
     }
-    // the unit's partial down tile: wait for its last MMAs, then TMEM -> ws_down
+    // the unit's partial down tile: wait for its last MMAs, then TMEM -> ws_down;
+    // the 16-column chunks go round the four warps of each TMEM lane quarter
     if (rp > 0) {
-      if (warp < 4 && !abort_sh) {
+      if (!abort_sh) {
+        const int quarter = warp & 3;
         const bool ok = mbar_wait_warp(&unit_bar, unit_parity, a.status, &abort_sh);
         tc_fence_after();
-        const int row = m0 + warp * 32 + lane;
+        const int row = m0 + quarter * 32 + lane;
         float* dst = a.ws_down + (static_cast<int64_t>(sp) * a.B + row) * rp;
-        for (int c0 = 0; c0 < rp; c0 += 16) {
+        for (int c0 = 16 * (warp >> 2); c0 < rp; c0 += 16 * (kWorkWarps / 4)) {
           // the accumulators summed in issuer order
           float sum[16];
           for (int q = 0; q < nacc; ++q) {
             uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc_cols * q + c0, v);
+            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc_cols * q + c0, v);
             tmem_ld_wait_regs(v);
 #pragma unroll
             for (int j = 0; j < 16; ++j) sum[j] = q == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
@@ -521,20 +523,44 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
       __syncthreads();
       if (last_sh) {
         // every unit of this row block is done: down = the partials summed in
-        // split order, as bf16 hi | lo
+        // split order, as bf16 hi | lo; four columns per thread, the loads of
+        // three partials in flight at a time
         __threadfence();
         const float mult = nv ? (a.gs_w != nullptr ? __fmul_rn(gs_x, __ldg(a.gs_w)) : gs_x) : 1.0f;
         const int rows = min(kRows, a.B - m0);
-        for (int i = tid; i < rows * rp; i += kWork) {
-          const int row = m0 + i / rp, j = i % rp;
-          float acc = 0.0f;
-          for (int z = 0; z < npieces; ++z)
-            acc += __ldcg(a.ws_down + (static_cast<int64_t>(z) * a.B + row) * rp + j);
-          acc = __fmul_rn(acc, mult);
-          const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
-          a.down[static_cast<int64_t>(row) * 2 * rp + j] = hi;
-          a.down[static_cast<int64_t>(row) * 2 * rp + rp + j] = lo;
+        const int rp4 = rp / 4;
+        const int64_t zs = static_cast<int64_t>(a.B) * rp4;   // float4s between partial tiles
+        for (int i = tid; i < rows * rp4; i += kWork) {
+          const int row = m0 + i / rp4, j = 4 * (i % rp4);
+          const float4* src = reinterpret_cast<const float4*>(a.ws_down + static_cast<int64_t>(row) * rp + j);
+          float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          auto add = [&](const float4 v) {
+            acc[0] += v.x;
+            acc[1] += v.y;
+            acc[2] += v.z;
+            acc[3] += v.w;
+          };
+          int z = 0;
+          for (; z + 3 <= npieces; z += 3) {
+            const float4 v0 = __ldcg(src + z * zs), v1 = __ldcg(src + (z + 1) * zs), v2 = __ldcg(src + (z + 2) * zs);
+            add(v0);
+            add(v1);
+            add(v2);
+          }
+          for (; z < npieces; ++z) add(__ldcg(src + z * zs));
+          uint32_t hi[2], lo[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float v0 = __fmul_rn(acc[2 * e], mult), v1 = __fmul_rn(acc[2 * e + 1], mult);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(v0, hf.x), __fsub_rn(v1, hf.y));
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l);
+          }
+          __nv_bfloat16* drow = a.down + static_cast<int64_t>(row) * 2 * rp + j;   // 8-byte aligned
+          *reinterpret_cast<uint2*>(drow) = make_uint2(hi[0], hi[1]);
+          *reinterpret_cast<uint2*>(drow + rp) = make_uint2(lo[0], lo[1]);
         }
       }
     }

@@ -210,6 +210,8 @@ svdq_status check_quantize_act_args(const void* x, svdq_dtype x_dtype, int64_t B
   if (B == 0) return SVDQ_OK;
   if (!codes || !act_scale || (fmt.kind != SVDQ_KIND_INT && !sf)) return SVDQ_EINVAL;
   if (ld && rank_pad > 0 && (!down || !aligned16(ld))) return SVDQ_EINVAL;
+  // the codes and the down tile are written in 8- and 16-byte pieces
+  if (!aligned16(codes) || (ld && rank_pad > 0 && !aligned16(down))) return SVDQ_EUNSUPPORTED;
   return SVDQ_OK;
 }
 

@@ -100,6 +100,22 @@ def test_linear_ex_rejects_unknown_flags(lib):
     assert st == rb.SVDQ_EINVAL
 
 
+def test_quantize_act_rejects_unaligned_outputs(lib):
+    """The codes (8-byte stores) and the down tile (8- and 16-byte stores) must be
+    16-byte aligned; checked on the host, before anything touches the device (the
+    pointers here are never dereferenced)."""
+    x, scale, ld, act_scale = 0x10000, 0x20000, 0x30000, 0x40000
+    fmt = rb.parse_fmt("int4")
+
+    def call(codes, down):
+        return lib.svdq_quantize_act(x, rb.SVDQ_BF16, 256, 64, 64, scale, fmt, None, None, ld, 32,
+                                     codes, None, act_scale, down, None, 0, None)
+
+    assert call(0x50008, 0x60000) == rb.SVDQ_EUNSUPPORTED     # codes off by 8 bytes
+    assert call(0x50000, 0x60004) == rb.SVDQ_EUNSUPPORTED     # down off by 4 bytes
+    assert call(0x50000, None) == rb.SVDQ_EINVAL             # ld given without down
+
+
 def test_no_cpu_path():
     """Every operator call takes CUDA tensors only: host tensors raise instead of
     being computed on the CPU, and a missing library raises on load."""

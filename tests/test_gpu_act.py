@@ -92,6 +92,51 @@ def test_long_batch_int_codes_and_scale(B, M, dtype, bits):
     assert_codes_match(codes.cpu().numpy(), q, near, f"B={B} M={M} {dtype} int{bits}")
 
 
+def near_tie_case(B, M, bits, dtype, seed):
+    """x and scale with thousands of quotients x / (scale s) at or next to a
+    half-integer: s = 1 (x[0, 0] = qmax at scale 1 is the maximum), columns 1-16
+    hold exact half-integers at scale 1 (ties to even), and every later column has
+    one element, its largest, tuned through its scale to within 2^-19 of a
+    half-integer (the others of the column stay below it in magnitude)."""
+    rng = np.random.default_rng(seed)
+    qm = ocodes.qmax_of(bits)
+    x = rng.standard_normal((B, M)).astype(np.float32)
+    if dtype == "bf16":
+        x = to_bf16(x)
+    scale = np.ones(M, np.float32)
+    x[:, 0] = 0.0
+    x[0, 0] = qm
+    for k in range(1, 17):
+        col = np.clip(np.round(x[:, k] * 2) / 2, -qm + 0.5, qm - 0.5)
+        x[:, k] = np.where(col == np.floor(col), col + 0.5, col).astype(np.float32)
+    for k in range(17, M):
+        r = int(np.argmax(np.abs(x[:, k])))
+        t = (rng.integers(0, qm) + 0.5 + rng.choice([0.0, 1.0, -1.0]) * rng.uniform(0, 2.0 ** -19)) * np.sign(x[r, k])
+        scale[k] = np.float32(x[r, k] / t)
+    return x, scale
+
+
+@pytest.mark.parametrize("B,M", [(100, 3072), (300, 3072), (1700, 12288)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_int_codes_exact_at_half_integers(B, M, dtype, bits):
+    """Every code equals round_half_even(x / (scale s)) of the exact quotient, also
+    where it lies within an fp32 ulp of a half-integer ("SVDQuant Smoothing,
+    Low-rank and Residual Quantization", Formula and conventions item 3: ties to
+    even): the estimate x c_k must send each such element to the exact decision.
+    B = 100 runs the short-batch pass, 300 the K-split units, 1700 x 12288 the
+    flat partition."""
+    x, scale = near_tie_case(B, M, bits, dtype, seed=B + bits)
+    xt = to_dev(x, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    codes, sf, s, down = rb.svdq_quantize_act(xt, to_dev(scale, torch.float32), f"int{bits}")
+    q, s_o, near = ocodes.act_codes_int(x, scale, bits)
+    assert s_o == np.float32(1.0) and np.float32(s.item()) == s_o, (s.item(), s_o)
+    assert int(near.sum()) >= 16 * B, int(near.sum())   # the case does reach the ties
+    got = codes.cpu().numpy()
+    bad = np.argwhere(got != q)
+    assert bad.size == 0, f"{len(bad)} codes differ from the exact rounding, e.g. {bad[:4].tolist()}"
+
+
 @pytest.mark.parametrize("B,M", LONG)
 @pytest.mark.parametrize("given_gs", [False, True])
 def test_long_batch_nvfp4_codes_scales_and_layout(B, M, given_gs):
