@@ -273,13 +273,20 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
     tmem_alloc(&tmem_sh, acc_cols * nacc);
     tmem_relinquish();
   }
-  // launched as a programmatic dependent of the maximum kernel: the setup above
-  // overlaps its tail; everything below (its partial maxima and counters, x,
-  // every output) comes after it has finished
-  pdl_wait();
-  // the per-tensor scale from the partial maxima (INT; NVFP4 without a given gs)
+  tc_fence_before();
+  __syncthreads();   // barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+
+  // The kernel is launched as a programmatic dependent of the maximum kernel:
+  // the setup above and the first piece's first copies of x and ld (which that
+  // kernel does not write) overlap its tail; its partial maxima and counters,
+  // and every output, are touched only after the wait in take_scale. The
+  // per-tensor scale from the partial maxima (INT; NVFP4 without a given gs).
   float s = 0.0f, u = 0.0f, gs_x = 1.0f;   // MXFP4: no global scale (1)
-  {
+  bool have_scale = false;
+  auto take_scale = [&]() {
+    pdl_wait();
     float m = 0.0f;
     for (int i = tid; i < a.nparts; i += kWork) m = fmaxf(m, __ldcg(a.ws_max + i));
 #pragma unroll
@@ -295,11 +302,8 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
       u = s > 0.0f ? __frcp_rn(s) : 0.0f;
     }
     if (blockIdx.x == 0 && tid == 0) *a.act_scale = nv || mx ? gs_x : s;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_sh;
+    have_scale = true;
+  };
 
   // element groups of the codes step: kE elements of a row per thread, the
   // threads of a row consecutive, kPasses rows per thread kRpp apart
@@ -388,6 +392,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
       }
     };
     for (int c = 0; c < stages - 1; ++c) issue(c);
+    if (!have_scale) take_scale();   // the first piece only (uniform over the CTA)
     // per-column constants of the unit: c_k = fl(fl(1 / scale_k) u) (INT) or
     // r_k = fl(1 / scale_k) (fp4)
     for (int j = tid; j < c_hi - c_lo; j += kWork) {
@@ -570,6 +575,7 @@ __global__ void __launch_bounds__(kWork, 1) act_quant_kernel(const __grid_consta
   }
   // no copy is still on its way when the CTA ends: the last segments' loads
   // were all waited for above, unless a wait ran out (then the status records it)
+  if (!have_scale) take_scale();   // a CTA without pieces still waits (and CTA 0 writes the scale)
   // fp4: zero the scale padding (rows up to a multiple of 128, columns up to 4)
   if (nv || mx) {
     const int64_t rows_p = (static_cast<int64_t>(a.B) + 127) / 128 * 128;
