@@ -149,6 +149,9 @@ svdq_status svdq_prepare_workspace_size(int64_t M, int64_t N, int32_t rank, svdq
  *
  * Synchronises `stream` before returning and returns SVDQ_EINVAL if scale held
  * a non-positive or non-finite entry, SVDQ_ETIMEOUT if a device wait ran out.
+ * Host errors: SVDQ_EINVAL for null pointers and sizes, SVDQ_ERANK, SVDQ_EUNSUPPORTED
+ * for shapes outside the library's limits or an output buffer (codes, codes4, sf,
+ * ld, ld32, lu) or scale not 16-byte aligned, SVDQ_EWORKSPACE for a short workspace.
  */
 svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N, int64_t ldW,
                          const float* scale, int32_t rank, svdq_fmt fmt, uint64_t seed,
@@ -164,6 +167,9 @@ svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N
  *   codes    INT int8 [N, M] / fp4 uint8 [N, M/2]   (K-major, as in svdq_weight)
  *   sf       NVFP4 128x4 layout of [N, M/16], MXFP4 of [N, M/32] (NULL for INT)
  *   w_scale  device fp32 scalar out: s_w (INT), gs_w (NVFP4) or 1 (MXFP4)
+ * Host errors: SVDQ_EINVAL for null pointers and sizes, SVDQ_EUNSUPPORTED for codes
+ * not 16-byte aligned (fp4 codes are stored 8 and 16 bytes at a time),
+ * SVDQ_EWORKSPACE for a short workspace.
  */
 svdq_status svdq_quantize_residual(const float* R, int64_t M, int64_t N, int64_t ldR,
                                    svdq_fmt fmt, void* codes, void* sf, float* w_scale,

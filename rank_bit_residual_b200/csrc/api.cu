@@ -280,6 +280,10 @@ svdq_status svdq_prepare(const void* W, svdq_dtype w_dtype, int64_t M, int64_t N
   if (!out->codes || !out->w_scale || (fmt.kind != SVDQ_KIND_INT && !out->sf) ||
       (rank > 0 && (!out->ld || !out->lu)))
     return SVDQ_EINVAL;
+  // the weight's buffers are written (and later read) in 16-byte pieces
+  if (!aligned16(out->codes) || (out->codes4 && !aligned16(out->codes4)) || (out->sf && !aligned16(out->sf)) ||
+      (out->ld && !aligned16(out->ld)) || (out->ld32 && !aligned16(out->ld32)) || (out->lu && !aligned16(out->lu)))
+    return SVDQ_EUNSUPPORTED;
   if (!workspace || workspace_bytes < prepare_scratch_bytes(M, N, rank, oversample))
     return SVDQ_EWORKSPACE;
   return run_prepare(W, w_dtype, M, N, ldW, scale, rank, fmt, seed, oversample, power_iters,
@@ -303,6 +307,7 @@ svdq_status svdq_quantize_residual(const float* R, int64_t M, int64_t N, int64_t
   if (s != SVDQ_OK) return s;
   if (!R || ldR < N || !codes || !w_scale || (fmt.kind != SVDQ_KIND_INT && !sf))
     return SVDQ_EINVAL;
+  if (!aligned16(codes)) return SVDQ_EUNSUPPORTED;   // fp4 codes go out 8 and 16 bytes at a time
   if (!workspace || workspace_bytes < residual_scratch_bytes(M, N)) return SVDQ_EWORKSPACE;
   return from_cuda(launch_quantize_residual(R, M, N, ldR, fmt, codes, sf, w_scale, workspace,
                                             reinterpret_cast<cudaStream_t>(stream)));

@@ -116,6 +116,28 @@ def test_quantize_act_rejects_unaligned_outputs(lib):
     assert call(0x50000, None) == rb.SVDQ_EINVAL             # ld given without down
 
 
+def test_weight_outputs_must_be_aligned(lib):
+    """svdq_prepare and svdq_quantize_residual write the weight's buffers in 8- and
+    16-byte pieces; a buffer off a 16-byte boundary is refused on the host (the
+    pointers here are never dereferenced)."""
+    W, scale, ws, R = 0x10000, 0x20000, 0x30000, 0x40000
+    fmt = rb.parse_fmt("nvfp4")
+
+    def weight(**off):
+        w = rb.SvdqWeight()
+        for i, f in enumerate(("codes", "sf", "w_scale", "ld", "lu", "ld32")):
+            setattr(w, f, 0x100000 * (i + 1) + off.get(f, 0))
+        return w
+
+    for field in ("codes", "sf", "ld", "lu", "ld32"):
+        w = weight(**{field: 8})
+        st = lib.svdq_prepare(W, rb.SVDQ_BF16, 64, 32, 32, scale, 4, fmt, 0, 0, 0, ws, 1 << 30,
+                              ctypes.byref(w), None)
+        assert st == rb.SVDQ_EUNSUPPORTED, field
+    st = lib.svdq_quantize_residual(R, 64, 32, 32, fmt, 0x50008, 0x60000, 0x70000, ws, 1 << 30, None)
+    assert st == rb.SVDQ_EUNSUPPORTED
+
+
 def test_no_cpu_path():
     """Every operator call takes CUDA tensors only: host tensors raise instead of
     being computed on the CPU, and a missing library raises on load."""
